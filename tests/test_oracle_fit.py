@@ -1,0 +1,147 @@
+"""Pins for the oracle's probes, residual subspace, ridge fit and correction."""
+import numpy as np
+import pytest
+import scipy.linalg
+from sklearn.linear_model import Ridge
+
+import oracle as O
+
+
+def test_ridge_matches_library_ridge():
+    # centred ridge with an unpenalised intercept is exactly sklearn's Ridge
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((64, 20))
+    y = rng.standard_normal((64, 5))
+    for lam in (1e-3, 1e-2, 3.0):
+        w, b = O.ridge_fit(x, y, lam)
+        ref = Ridge(alpha=lam, fit_intercept=True, solver="cholesky").fit(x, y)
+        np.testing.assert_allclose(w, ref.coef_.T, rtol=1e-8, atol=1e-10)
+        np.testing.assert_allclose(b, ref.intercept_, rtol=1e-8, atol=1e-10)
+
+
+def test_ridge_primal_equals_dual_and_limits():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((64, 128))       # more regressors than probes
+    y = rng.standard_normal((64, 7))
+    lam = 1e-2
+    w, b = O.ridge_fit(x, y, lam)
+    xc, yc = x - x.mean(0), y - y.mean(0)
+    wp = np.linalg.solve(xc.T @ xc + lam * np.eye(128), xc.T @ yc)
+    np.testing.assert_allclose(w, wp, rtol=1e-7, atol=1e-9)
+    # lam -> infinity: slope vanishes, intercept is the mean
+    w_inf, b_inf = O.ridge_fit(x, y, 1e12)
+    assert np.abs(w_inf).max() < 1e-9
+    np.testing.assert_allclose(b_inf, y.mean(0), atol=1e-9)
+
+
+def test_ridge_recovers_planted_affine_map():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((64, 10))
+    w0 = rng.standard_normal((10, 3))
+    b0 = rng.standard_normal(3)
+    w, b = O.ridge_fit(x, b0 + x @ w0, 1e-12)
+    np.testing.assert_allclose(w, w0, atol=1e-8)
+    np.testing.assert_allclose(b, b0, atol=1e-8)
+
+
+def test_subspace_eckart_young_and_projector():
+    rng = np.random.default_rng(3)
+    r_p = rng.standard_normal((64, 32)) @ np.diag(np.linspace(3, 0.1, 32))
+    v, sig = O.probe_subspace(r_p, 8)
+    np.testing.assert_allclose(v.T @ v, np.eye(8), atol=1e-12)
+    ev = np.sort(scipy.linalg.eigvalsh(r_p.T @ r_p))[::-1]
+    np.testing.assert_allclose(sig ** 2, ev[:8], rtol=1e-9)
+    resid = r_p - r_p @ v @ v.T
+    np.testing.assert_allclose((resid ** 2).sum(), ev[8:].sum(), rtol=1e-8)
+    w_e, u_e = scipy.linalg.eigh(r_p.T @ r_p)
+    top = u_e[:, np.argsort(-w_e)[:8]]
+    np.testing.assert_allclose(v @ v.T, top @ top.T, atol=1e-9)
+
+
+def test_subspace_rank_deficient_is_zero_columns():
+    rng = np.random.default_rng(4)
+    r_p = np.outer(rng.standard_normal(64), rng.standard_normal(16))   # rank 1
+    v, sig = O.probe_subspace(r_p, 4)
+    assert sig[0] > 0 and np.all(sig[1:] == 0) and np.all(v[:, 1:] == 0)
+    v0, s0 = O.probe_subspace(np.zeros((64, 16)), 4)
+    assert np.all(v0 == 0) and np.all(s0 == 0)
+
+
+def test_correction_exact_for_planted_affine_residual():
+    # if the residual is exactly b + x B with B of rank r inside the probes'
+    # residual span, the corrected output equals the dense one on every row
+    rng = np.random.default_rng(5)
+    n, d, r, p = 400, 12, 3, 64
+    basis = np.linalg.qr(rng.standard_normal((d, r)))[0]
+    b_sub = rng.standard_normal(r)
+    w_sub = rng.standard_normal((d, r))
+    o_sparse = rng.standard_normal((n, d))
+    o_dense = o_sparse + (b_sub + o_sparse @ w_sub) @ basis.T
+    pidx = rng.choice(n, p, replace=False)
+    fit = O.fit_from_probes(pidx, o_dense[pidx], o_sparse[pidx], np.zeros(p), np.zeros(p), r, 1e-12)
+    np.testing.assert_allclose(fit.vr @ fit.vr.T, basis @ basis.T, atol=1e-9)
+    out = O.correct(o_sparse, fit)
+    np.testing.assert_allclose(out, o_dense, atol=1e-7)
+    np.testing.assert_allclose(fit.bmat, fit.w @ fit.vr.T)
+    np.testing.assert_allclose(out[pidx], o_dense[pidx], atol=0)
+
+
+def test_probe_rows_take_exact_dense_output():
+    rng = np.random.default_rng(8)
+    o_s = rng.standard_normal((50, 6))
+    o_d = o_s + rng.standard_normal((50, 6))      # residual not affine: fit is inexact
+    pidx = np.arange(0, 50, 3)
+    fit = O.fit_from_probes(pidx, o_d[pidx], o_s[pidx], np.zeros(17), np.zeros(17), 3, 1e-2)
+    out = O.correct(o_s, fit)
+    np.testing.assert_array_equal(out[pidx], o_d[pidx])
+    rest = np.setdiff1d(np.arange(50), pidx)
+    np.testing.assert_allclose(out[rest], o_s[rest] + fit.b_full + o_s[rest] @ fit.bmat, atol=1e-12)
+
+
+def test_zero_residual_leaves_sparse_output():
+    rng = np.random.default_rng(6)
+    o = rng.standard_normal((100, 8))
+    pidx = np.arange(0, 100, 5)
+    fit = O.fit_from_probes(pidx, o[pidx], o[pidx], np.zeros(20), np.zeros(20), 4, 1e-2)
+    np.testing.assert_array_equal(O.correct(o, fit), o)
+
+
+@pytest.mark.parametrize("sizes,p", [([10, 10, 10, 10], 64), ([100, 3, 0, 50, 7], 64),
+                                     ([2, 1], 64), ([30] * 8, 64), ([9, 9, 9], 10),
+                                     ([5, 1, 5, 1, 5], 7)])
+def test_probe_allocation(sizes, p):
+    sizes = np.array(sizes)
+    alloc = O.probe_allocation(sizes, p)
+    assert alloc.sum() == min(p, sizes.sum())
+    assert np.all(alloc <= sizes) and np.all(alloc >= 0)
+    open_ = alloc < sizes
+    if open_.any():
+        # groups with spare members differ by at most one probe, and no
+        # saturated group holds more than an open group's share + 1
+        assert alloc[open_].max() - alloc[open_].min() <= 1
+        assert np.all(alloc[~open_] <= alloc[open_].max())
+    # the leftover probe of the uneven case goes to the larger group first
+    if list(sizes) == [9, 9, 9]:
+        assert list(alloc) == [4, 3, 3]
+    if list(sizes) == [5, 1, 5, 1, 5]:
+        assert list(alloc) == [2, 1, 2, 1, 1]
+
+
+def test_pick_probes_stratified_and_reproducible():
+    rng = np.random.default_rng(7)
+    lab = rng.integers(0, 8, 1000)
+    perm, off = O.group_permutation(lab, 8)
+    pidx = O.pick_probes(perm, off, 64, seed=5, bh=3)
+    assert len(pidx) == 64 and len(set(pidx)) == 64
+    counts = np.bincount(lab[pidx], minlength=8)
+    assert list(counts) == list(O.probe_allocation(np.diff(off), 64))
+    assert np.array_equal(pidx, O.pick_probes(perm, off, 64, seed=5, bh=3))
+    assert not np.array_equal(pidx, O.pick_probes(perm, off, 64, seed=6, bh=3))
+    # group order, then the stream's draw order inside each group
+    g = O.SplitMix64(O.stream_state(5, 3, O.STREAM_PROBES))
+    alloc = O.probe_allocation(np.diff(off), 64)
+    want = []
+    for a in range(8):
+        mem = perm[off[a]:off[a + 1]]
+        want += [int(mem[i]) for i in O.draw_without_replacement(g, len(mem), int(alloc[a]))]
+    assert list(pidx) == want
