@@ -1,0 +1,487 @@
+// C ABI of the SparsePR library: argument validation, workspace layout and the
+// sequencing of the kernels of each call on the caller's stream.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace spr;
+
+namespace {
+
+thread_local char g_detail[512] = "no error";
+thread_local int g_launches = 0;
+
+sparsepr_status fail(sparsepr_status s, const char* msg) {
+  snprintf(g_detail, sizeof(g_detail), "%s", msg);
+  return s;
+}
+
+sparsepr_status failv(sparsepr_status s, const char* msg, long long v) {
+  snprintf(g_detail, sizeof(g_detail), "%s (got %lld)", msg, v);
+  return s;
+}
+
+sparsepr_status fail_cuda(cudaError_t e, const char* where) {
+  snprintf(g_detail, sizeof(g_detail), "CUDA error in %s: %s", where, cudaGetErrorString(e));
+  return SPARSEPR_ECUDA;
+}
+
+#define SPR_LAUNCH(expr)                                  \
+  do {                                                    \
+    cudaError_t e_ = (expr);                              \
+    ++g_launches;                                         \
+    if (e_ != cudaSuccess) return fail_cuda(e_, #expr);   \
+  } while (0)
+#define SPR_CUDA(expr)                                    \
+  do {                                                    \
+    cudaError_t e_ = (expr);                              \
+    if (e_ != cudaSuccess) return fail_cuda(e_, #expr);   \
+  } while (0)
+
+constexpr size_t kSmemLimit = 227 * 1024;
+
+size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Layout {
+  // header
+  size_t err;
+  // partition
+  size_t sample_idx, metric, eigval, eigvec, proj, Y, cent_k, key_init, C, Z, cent_q, query_init, mass,
+      order, cm, cc, alpha;
+  // attend
+  size_t rlist, rcum, rcnt, tiles, tile_count;
+  // probe
+  size_t probe_grp, part_o, part_ml, o_sparse_p, lse_d, lse_s;
+  size_t total;
+  // forward extras
+  size_t f_perm_q, f_perm_k, f_label_q, f_label_k, f_qoff, f_koff, f_route, f_bmask, f_rho, f_lse, f_probe_idx,
+      f_probe_od, f_bfull, f_vr, f_w;
+  size_t forward_total;
+  int BH, max_tiles, T, S, DTk, DTq;
+};
+
+Layout make_layout(const sparsepr_params& p) {
+  Layout L{};
+  const size_t BH = (size_t)p.B * p.H, N = p.N, d = p.d;
+  const size_t Gk = p.n_kgroups, Gq = p.n_qgroups, re = p.eig_rank, P = p.n_probes, r = p.sub_rank;
+  L.BH = (int)BH;
+  L.max_tiles = ceil_div(p.N, kAttnTileRows) + p.n_qgroups;
+  L.T = ceil_div(p.N, p.block);
+  L.S = probe_splits(p.N);
+  L.DTk = kmeans_dt(p.eig_rank);
+  L.DTq = kmeans_dt(p.n_kgroups);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = al256(o + bytes); return at; };
+  L.err = take(256);
+  L.sample_idx = take(BH * p.n_samples * 4);
+  L.metric = take(BH * d * d * 4);
+  L.eigval = take(BH * re * 4);
+  L.eigvec = take(BH * d * re * 4);
+  L.proj = take(BH * d * re * 4);
+  L.Y = take(BH * N * re * 4);
+  L.cent_k = take(BH * Gk * L.DTk * 4);
+  L.key_init = take(BH * Gk * 4);
+  L.C = take(BH * Gk * d * 4);
+  L.Z = take(BH * N * Gk * 4);
+  L.cent_q = take(BH * Gq * L.DTq * 4);
+  L.query_init = take(BH * Gq * 4);
+  L.mass = take(BH * Gq * Gk * 4);
+  L.order = take(BH * Gq * Gk * 4);
+  L.cm = take(BH * Gq * Gk * 8);
+  L.cc = take(BH * Gq * Gk * 8);
+  L.alpha = take(BH * 8);
+  L.rlist = take(BH * Gq * Gk * 4);
+  L.rcum = take(BH * Gq * (Gk + 1) * 4);
+  L.rcnt = take(BH * Gq * 4);
+  L.tiles = take(BH * L.max_tiles * 8);
+  L.tile_count = take(BH * 4);
+  L.probe_grp = take(BH * P * 4);
+  L.part_o = take(BH * L.S * 64 * 2 * d * 4);
+  L.part_ml = take(BH * L.S * 64 * 4 * 4);
+  L.o_sparse_p = take(BH * P * d * 4);
+  L.lse_d = take(BH * P * 4);
+  L.lse_s = take(BH * P * 4);
+  L.total = o;
+  L.f_perm_q = take(BH * N * 4);
+  L.f_perm_k = take(BH * N * 4);
+  L.f_label_q = take(BH * N * 4);
+  L.f_label_k = take(BH * N * 4);
+  L.f_qoff = take(BH * (Gq + 1) * 4);
+  L.f_koff = take(BH * (Gk + 1) * 4);
+  L.f_route = take(BH * Gq * Gk);
+  L.f_bmask = take(BH * (size_t)L.T * L.T);
+  L.f_rho = take(BH * 4);
+  L.f_lse = take(BH * N * 4);
+  L.f_probe_idx = take(BH * P * 4);
+  L.f_probe_od = take(BH * P * d * 4);
+  L.f_bfull = take(BH * d * 4);
+  L.f_vr = take(BH * d * r * 4);
+  L.f_w = take(BH * d * r * 4);
+  L.forward_total = o;
+  return L;
+}
+
+sparsepr_status check_params(const sparsepr_params* p) {
+  if (!p) return fail(SPARSEPR_EINVAL, "params pointer is NULL");
+  if (p->B < 1 || p->H < 1 || p->N < 1) return fail(SPARSEPR_EINVAL, "B, H and N must be >= 1");
+  if ((long long)p->B * p->H * p->N > (1ll << 30)) return fail(SPARSEPR_EUNSUPPORTED, "B*H*N too large");
+  if (p->d != 64 && p->d != 128) return failv(SPARSEPR_EUNSUPPORTED, "head dim d must be 64 or 128", p->d);
+  if (p->block != 64 && p->block != 128) return failv(SPARSEPR_EINVAL, "block must be 64 or 128", p->block);
+  if (!(p->density > 0.f) || !(p->density <= 1.f)) return fail(SPARSEPR_EINVAL, "density must be in (0, 1]");
+  const int gmax = p->N < 1024 ? p->N : 1024;
+  if (p->n_kgroups < 1 || p->n_kgroups > gmax) return failv(SPARSEPR_EINVAL, "n_kgroups must be in [1, min(N,1024)]", p->n_kgroups);
+  if (p->n_qgroups < 1 || p->n_qgroups > gmax) return failv(SPARSEPR_EINVAL, "n_qgroups must be in [1, min(N,1024)]", p->n_qgroups);
+  if (p->n_samples < 1 || p->n_samples > gmax) return failv(SPARSEPR_EINVAL, "n_samples must be in [1, min(N,1024)]", p->n_samples);
+  const int pmax = p->N < 64 ? p->N : 64;
+  if (p->n_probes < 1 || p->n_probes > pmax) return failv(SPARSEPR_EINVAL, "n_probes must be in [1, min(N,64)]", p->n_probes);
+  if (p->eig_rank < 1 || p->eig_rank > p->d) return failv(SPARSEPR_EINVAL, "eig_rank must be in [1, d]", p->eig_rank);
+  if (p->sub_rank < 1 || p->sub_rank > p->n_probes || p->sub_rank > p->d)
+    return failv(SPARSEPR_EINVAL, "sub_rank must be in [1, min(d, n_probes)]", p->sub_rank);
+  if (p->kmeans_iters < 1 || p->kmeans_iters > 64) return failv(SPARSEPR_EINVAL, "kmeans_iters must be in [1, 64]", p->kmeans_iters);
+  if (!(p->ridge_lambda > 0.f) || !isfinite(p->ridge_lambda)) return fail(SPARSEPR_EINVAL, "ridge_lambda must be > 0");
+  if (!(p->scale >= 0.f) || !isfinite(p->scale)) return fail(SPARSEPR_EINVAL, "scale must be >= 0");
+  if (p->frame_id) return fail(SPARSEPR_EUNSUPPORTED, "frame-causal masking (frame_id) is not built");
+  if (p->density < 1.f &&
+      (double)p->density * (double)p->N * (double)p->N < (double)p->n_probes * (double)p->N)
+    return fail(SPARSEPR_EINVAL, "density is below the probe floor n_probes/N");
+  // kernel limits
+  if (p->n_kgroups > 128) return fail(SPARSEPR_EUNSUPPORTED, "n_kgroups > 128 (query coordinates wider than 128) not built");
+  if ((size_t)p->n_qgroups * kmeans_dt(p->n_kgroups) * 4 > kSmemLimit)
+    return fail(SPARSEPR_EUNSUPPORTED, "query centroid table exceeds shared memory");
+  if ((size_t)p->n_kgroups * kmeans_dt(p->eig_rank) * 4 > kSmemLimit)
+    return fail(SPARSEPR_EUNSUPPORTED, "key centroid table exceeds shared memory");
+  if ((size_t)p->d * p->sub_rank > 64 * 65 || probe_fit_smem(p->d, p->sub_rank) > kSmemLimit)
+    return failv(SPARSEPR_EUNSUPPORTED, "sub_rank too large for the single-CTA fit (d*r)", (long long)p->d * p->sub_rank);
+  if (attn_smem_bytes(p->d, p->n_kgroups) > kSmemLimit || probe_attn_smem(p->d, p->n_kgroups) > kSmemLimit)
+    return fail(SPARSEPR_EUNSUPPORTED, "too many K/V groups for the attention kernels");
+  return SPARSEPR_OK;
+}
+
+sparsepr_status check_ws(const sparsepr_params* p, void* ws, size_t ws_bytes, size_t need) {
+  if (!ws) return fail(SPARSEPR_EINVAL, "workspace is NULL");
+  if (((uintptr_t)ws & 255) != 0) return fail(SPARSEPR_EWORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < need) return failv(SPARSEPR_EWORKSPACE, "workspace too small (bytes needed)", (long long)need);
+  (void)p;
+  return SPARSEPR_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+float eff_scale(const sparsepr_params& p) { return p.scale > 0.f ? p.scale : 1.0f / sqrtf((float)p.d); }
+
+#define SPR_CHECK(expr)                          \
+  do {                                           \
+    sparsepr_status s_ = (expr);                 \
+    if (s_ != SPARSEPR_OK) return s_;            \
+  } while (0)
+#define SPR_NONNULL(ptr)                                                                  \
+  do {                                                                                    \
+    if (!(ptr)) return fail(SPARSEPR_EINVAL, "required pointer " #ptr " is NULL");        \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const void* Q, const void* K, int* perm_q,
+                              int* perm_k, int* label_q, int* label_k, int* qoff, int* koff, unsigned char* route,
+                              unsigned char* bmask, float* rho, const sparsepr_partition_trace* tr, void* ws,
+                              cudaStream_t st) {
+  const int BH = L.BH, N = p.N, d = p.d, Gk = p.n_kgroups, Gq = p.n_qgroups, re = p.eig_rank;
+  int* err = at<int>(ws, L.err);
+  SPR_CUDA(cudaMemsetAsync(err, 0, 4, st));
+  float* metric = at<float>(ws, L.metric);
+  SPR_LAUNCH(launch_sample_metric(Q, BH, N, d, p.n_samples, p.seed, metric, at<int>(ws, L.sample_idx), err, st));
+  SPR_LAUNCH(launch_metric_eigen(metric, BH, d, re, at<float>(ws, L.eigval), at<float>(ws, L.eigvec),
+                                 at<float>(ws, L.proj), st));
+  float* Y = at<float>(ws, L.Y);
+  SPR_LAUNCH(launch_key_coords(K, BH, N, d, re, at<float>(ws, L.proj), Y, st));
+  // key k-means
+  float* cent_k = at<float>(ws, L.cent_k);
+  SPR_LAUNCH(launch_kmeans_seed(Y, BH, N, re, Gk, p.seed, PURPOSE_KEY_KMEANS, cent_k, at<int>(ws, L.key_init),
+                                err, st));
+  for (int t = 0; t < p.kmeans_iters; ++t) {
+    int* trk = (tr && tr->key_label_iters) ? tr->key_label_iters + (size_t)t * BH * N : nullptr;
+    SPR_LAUNCH(launch_kmeans_assign(Y, BH, N, re, Gk, cent_k, label_k, trk, st));
+    SPR_LAUNCH(launch_group_sort(label_k, BH, N, Gk, perm_k, koff, err, st));
+    if (t + 1 < p.kmeans_iters) SPR_LAUNCH(launch_segment_mean_f32(Y, BH, N, re, Gk, perm_k, koff, cent_k, 0, st));
+  }
+  float* C = at<float>(ws, L.C);
+  SPR_LAUNCH(launch_segment_mean_bf16(K, BH, N, d, Gk, perm_k, koff, C, st));
+  float* Z = at<float>(ws, L.Z);
+  SPR_LAUNCH(launch_query_coords(Q, BH, N, d, C, Gk, eff_scale(p), Z, st));
+  // query k-means
+  float* cent_q = at<float>(ws, L.cent_q);
+  SPR_LAUNCH(launch_kmeans_seed(Z, BH, N, Gk, Gq, p.seed, PURPOSE_QUERY_KMEANS, cent_q,
+                                at<int>(ws, L.query_init), err, st));
+  for (int t = 0; t < p.kmeans_iters; ++t) {
+    int* trq = (tr && tr->query_label_iters) ? tr->query_label_iters + (size_t)t * BH * N : nullptr;
+    SPR_LAUNCH(launch_kmeans_assign(Z, BH, N, Gk, Gq, cent_q, label_q, trq, st));
+    SPR_LAUNCH(launch_group_sort(label_q, BH, N, Gq, perm_q, qoff, err, st));
+    if (t + 1 < p.kmeans_iters) SPR_LAUNCH(launch_segment_mean_f32(Z, BH, N, Gk, Gq, perm_q, qoff, cent_q, 0, st));
+  }
+  float* mass = at<float>(ws, L.mass);
+  SPR_LAUNCH(launch_cell_mass(Z, BH, N, Gk, Gq, perm_q, qoff, koff, mass, st));
+  SPR_LAUNCH(launch_route_select(mass, BH, N, Gq, Gk, qoff, koff, p.density, p.n_probes, at<int>(ws, L.order),
+                                 at<double>(ws, L.cm), at<long long>(ws, L.cc), route, rho,
+                                 at<double>(ws, L.alpha), st));
+  if (bmask)
+    SPR_LAUNCH(launch_block_mask(route, BH, N, Gq, Gk, p.block, perm_q, label_q, perm_k, label_k, bmask, st));
+  if (tr) {
+    auto cp = [&](void* dst, size_t off, size_t bytes) -> cudaError_t {
+      return dst ? cudaMemcpyAsync(dst, at<char>(ws, off), bytes, cudaMemcpyDeviceToDevice, st) : cudaSuccess;
+    };
+    const size_t bh = BH;
+    SPR_CUDA(cp(tr->sample_idx, L.sample_idx, bh * p.n_samples * 4));
+    SPR_CUDA(cp(tr->metric, L.metric, bh * d * d * 4));
+    SPR_CUDA(cp(tr->eigval, L.eigval, bh * re * 4));
+    SPR_CUDA(cp(tr->eigvec, L.eigvec, bh * d * re * 4));
+    SPR_CUDA(cp(tr->key_coords, L.Y, bh * N * re * 4));
+    SPR_CUDA(cp(tr->key_init, L.key_init, bh * Gk * 4));
+    SPR_CUDA(cp(tr->key_centroids, L.C, bh * Gk * d * 4));
+    SPR_CUDA(cp(tr->query_coords, L.Z, bh * N * Gk * 4));
+    SPR_CUDA(cp(tr->query_init, L.query_init, bh * Gq * 4));
+    SPR_CUDA(cp(tr->cell_mass, L.mass, bh * Gq * Gk * 4));
+    SPR_CUDA(cp(tr->alpha, L.alpha, bh * 8));
+  }
+  return SPARSEPR_OK;
+}
+
+sparsepr_status run_attend(const sparsepr_params& p, const Layout& L, const void* Q, const void* K, const void* V,
+                           const int* perm_q, const int* perm_k, const int* qoff, const int* koff,
+                           const unsigned char* route, void* O, float* lse, void* ws, cudaStream_t st) {
+  int* rlist = at<int>(ws, L.rlist);
+  int* rcum = at<int>(ws, L.rcum);
+  int* rcnt = at<int>(ws, L.rcnt);
+  int2* tiles = at<int2>(ws, L.tiles);
+  int* tcount = at<int>(ws, L.tile_count);
+  SPR_LAUNCH(launch_worklist(route, qoff, koff, L.BH, p.n_qgroups, p.n_kgroups, kAttnTileRows, L.max_tiles, rlist,
+                             rcum, rcnt, tiles, tcount, st));
+  AttnArgs a{};
+  a.Q = Q; a.K = K; a.V = V;
+  a.BH = L.BH; a.N = p.N; a.D = p.d; a.Gq = p.n_qgroups; a.Gk = p.n_kgroups;
+  a.perm_q = perm_q; a.perm_k = perm_k; a.qoff = qoff; a.koff = koff;
+  a.rlist = rlist; a.rcum = rcum; a.rcnt = rcnt; a.tiles = tiles; a.tile_count = tcount;
+  a.max_tiles = L.max_tiles;
+  a.scale_log2 = eff_scale(p) * 1.4426950408889634f;
+  a.O = O; a.lse = lse; a.err = at<int>(ws, L.err);
+  SPR_LAUNCH(launch_attention(a, false, st));
+  return SPARSEPR_OK;
+}
+
+sparsepr_status run_probe_fit(const sparsepr_params& p, const Layout& L, const void* Q, const void* K,
+                              const void* V, const int* label_k, const int* perm_q, const int* qoff,
+                              const unsigned char* route, int* probe_idx, float* probe_od, float* bfull,
+                              float* Vr, float* W, float* Bmat, const sparsepr_probe_trace* tr, void* ws,
+                              cudaStream_t st) {
+  const int BH = L.BH, N = p.N, d = p.d, P = p.n_probes;
+  int* pgrp = at<int>(ws, L.probe_grp);
+  SPR_LAUNCH(launch_probe_pick(perm_q, qoff, BH, N, p.n_qgroups, P, p.seed, probe_idx, pgrp, at<int>(ws, L.err), st));
+  float* part_o = at<float>(ws, L.part_o);
+  float* part_ml = at<float>(ws, L.part_ml);
+  SPR_LAUNCH(launch_probe_attn(Q, K, V, BH, N, d, p.n_kgroups, p.n_qgroups, P, probe_idx, pgrp, label_k, route,
+                               eff_scale(p) * 1.4426950408889634f, part_o, part_ml, st));
+  float* osp = at<float>(ws, L.o_sparse_p);
+  float* lsd = at<float>(ws, L.lse_d);
+  float* lss = at<float>(ws, L.lse_s);
+  SPR_LAUNCH(launch_probe_combine(part_o, part_ml, BH, N, P, d, probe_od, osp, lsd, lss, st));
+  SPR_LAUNCH(launch_probe_fit(probe_od, osp, BH, d, P, p.sub_rank, (double)p.ridge_lambda, Vr, W, bfull, Bmat,
+                              tr ? tr->sigma : nullptr, tr ? tr->b_sub : nullptr, st));
+  if (tr) {
+    if (tr->probe_o_sparse)
+      SPR_CUDA(cudaMemcpyAsync(tr->probe_o_sparse, osp, (size_t)BH * P * d * 4, cudaMemcpyDeviceToDevice, st));
+    if (tr->probe_lse_dense)
+      SPR_CUDA(cudaMemcpyAsync(tr->probe_lse_dense, lsd, (size_t)BH * P * 4, cudaMemcpyDeviceToDevice, st));
+    if (tr->probe_lse_sparse)
+      SPR_CUDA(cudaMemcpyAsync(tr->probe_lse_sparse, lss, (size_t)BH * P * 4, cudaMemcpyDeviceToDevice, st));
+  }
+  return SPARSEPR_OK;
+}
+
+sparsepr_status run_reconstruct(const sparsepr_params& p, int BH, const void* Os, const int* probe_idx,
+                                const float* probe_od, const float* bfull, const float* Vr, const float* W, void* O,
+                                cudaStream_t st) {
+  SPR_LAUNCH(launch_reconstruct(Os, BH, p.N, p.d, p.sub_rank, W, Vr, bfull, O, st));
+  SPR_LAUNCH(launch_probe_scatter(probe_idx, probe_od, BH, p.N, p.n_probes, p.d, O, st));
+  return SPARSEPR_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+extern "C" {
+
+size_t sparsepr_workspace_bytes(const sparsepr_params* p) {
+  if (check_params(p) != SPARSEPR_OK) return 0;
+  return make_layout(*p).total;
+}
+
+size_t sparsepr_forward_workspace_bytes(const sparsepr_params* p) {
+  if (check_params(p) != SPARSEPR_OK) return 0;
+  return make_layout(*p).forward_total;
+}
+
+sparsepr_status sparsepr_validate(const sparsepr_params* p) { return check_params(p); }
+
+sparsepr_status sparsepr_partition(const sparsepr_params* p, const void* Q, const void* K, int* perm_q, int* perm_k,
+                                   int* label_q, int* label_k, int* qoff, int* koff, unsigned char* route,
+                                   unsigned char* block_mask, float* rho_exec, const sparsepr_partition_trace* trace,
+                                   void* workspace, size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  SPR_CHECK(check_params(p));
+  SPR_NONNULL(Q); SPR_NONNULL(K); SPR_NONNULL(perm_q); SPR_NONNULL(perm_k); SPR_NONNULL(label_q);
+  SPR_NONNULL(label_k); SPR_NONNULL(qoff); SPR_NONNULL(koff); SPR_NONNULL(route); SPR_NONNULL(rho_exec);
+  const Layout L = make_layout(*p);
+  SPR_CHECK(check_ws(p, workspace, ws_bytes, L.total));
+  return run_partition(*p, L, Q, K, perm_q, perm_k, label_q, label_k, qoff, koff, route, block_mask, rho_exec,
+                       trace, workspace, (cudaStream_t)stream);
+}
+
+sparsepr_status sparsepr_attend(const sparsepr_params* p, const void* Q, const void* K, const void* V,
+                                const int* perm_q, const int* perm_k, const int* qoff, const int* koff,
+                                const unsigned char* route, void* O_sparse, float* lse, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  SPR_CHECK(check_params(p));
+  SPR_NONNULL(Q); SPR_NONNULL(K); SPR_NONNULL(V); SPR_NONNULL(perm_q); SPR_NONNULL(perm_k); SPR_NONNULL(qoff);
+  SPR_NONNULL(koff); SPR_NONNULL(route); SPR_NONNULL(O_sparse);
+  const Layout L = make_layout(*p);
+  SPR_CHECK(check_ws(p, workspace, ws_bytes, L.total));
+  return run_attend(*p, L, Q, K, V, perm_q, perm_k, qoff, koff, route, O_sparse, lse, workspace,
+                    (cudaStream_t)stream);
+}
+
+sparsepr_status sparsepr_probe_fit(const sparsepr_params* p, const void* Q, const void* K, const void* V,
+                                   const int* label_k, const int* perm_q, const int* qoff, const unsigned char* route,
+                                   int* probe_idx, float* probe_o_dense, float* b_full, float* Vr, float* W,
+                                   float* Bmat, const sparsepr_probe_trace* trace, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+  g_launches = 0;
+  SPR_CHECK(check_params(p));
+  SPR_NONNULL(Q); SPR_NONNULL(K); SPR_NONNULL(V); SPR_NONNULL(label_k); SPR_NONNULL(perm_q); SPR_NONNULL(qoff);
+  SPR_NONNULL(route); SPR_NONNULL(probe_idx); SPR_NONNULL(probe_o_dense); SPR_NONNULL(b_full); SPR_NONNULL(Vr);
+  SPR_NONNULL(W);
+  const Layout L = make_layout(*p);
+  SPR_CHECK(check_ws(p, workspace, ws_bytes, L.total));
+  return run_probe_fit(*p, L, Q, K, V, label_k, perm_q, qoff, route, probe_idx, probe_o_dense, b_full, Vr, W, Bmat,
+                       trace, workspace, (cudaStream_t)stream);
+}
+
+sparsepr_status sparsepr_reconstruct(const sparsepr_params* p, const void* O_sparse, const int* probe_idx,
+                                     const float* probe_o_dense, const float* b_full, const float* Vr,
+                                     const float* W, void* O, void* stream) {
+  g_launches = 0;
+  SPR_CHECK(check_params(p));
+  SPR_NONNULL(O_sparse); SPR_NONNULL(probe_idx); SPR_NONNULL(probe_o_dense); SPR_NONNULL(b_full); SPR_NONNULL(Vr);
+  SPR_NONNULL(W); SPR_NONNULL(O);
+  return run_reconstruct(*p, p->B * p->H, O_sparse, probe_idx, probe_o_dense, b_full, Vr, W, O,
+                         (cudaStream_t)stream);
+}
+
+sparsepr_status sparsepr_forward(const sparsepr_params* p, const void* Q, const void* K, const void* V, void* O,
+                                 float* rho_exec, void* workspace, size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  SPR_CHECK(check_params(p));
+  SPR_NONNULL(Q); SPR_NONNULL(K); SPR_NONNULL(V); SPR_NONNULL(O);
+  const Layout L = make_layout(*p);
+  SPR_CHECK(check_ws(p, workspace, ws_bytes, L.forward_total));
+  cudaStream_t st = (cudaStream_t)stream;
+  void* ws = workspace;
+  int* perm_q = at<int>(ws, L.f_perm_q);
+  int* perm_k = at<int>(ws, L.f_perm_k);
+  int* label_q = at<int>(ws, L.f_label_q);
+  int* label_k = at<int>(ws, L.f_label_k);
+  int* qoff = at<int>(ws, L.f_qoff);
+  int* koff = at<int>(ws, L.f_koff);
+  unsigned char* route = at<unsigned char>(ws, L.f_route);
+  float* rho = rho_exec ? rho_exec : at<float>(ws, L.f_rho);
+  SPR_CHECK(run_partition(*p, L, Q, K, perm_q, perm_k, label_q, label_k, qoff, koff, route, nullptr, rho, nullptr,
+                          ws, st));
+  SPR_CHECK(run_attend(*p, L, Q, K, V, perm_q, perm_k, qoff, koff, route, O, at<float>(ws, L.f_lse), ws, st));
+  int* pidx = at<int>(ws, L.f_probe_idx);
+  float* pod = at<float>(ws, L.f_probe_od);
+  float* bfull = at<float>(ws, L.f_bfull);
+  float* vr = at<float>(ws, L.f_vr);
+  float* w = at<float>(ws, L.f_w);
+  SPR_CHECK(run_probe_fit(*p, L, Q, K, V, label_k, perm_q, qoff, route, pidx, pod, bfull, vr, w, nullptr, nullptr,
+                          ws, st));
+  SPR_CHECK(run_reconstruct(*p, L.BH, O, pidx, pod, bfull, vr, w, O, st));
+  return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_forward_host(const sparsepr_params* p, const void* Q_host, const void* K_host,
+                                      const void* V_host, void* O_host, void* qkv_dev, void* o_dev, void* workspace,
+                                      size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  SPR_CHECK(check_params(p));
+  SPR_NONNULL(Q_host); SPR_NONNULL(K_host); SPR_NONNULL(V_host); SPR_NONNULL(O_host); SPR_NONNULL(qkv_dev);
+  SPR_NONNULL(o_dev);
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t bytes = (size_t)p->B * p->H * p->N * p->d * 2;
+  char* q = static_cast<char*>(qkv_dev);
+  SPR_CUDA(cudaMemcpyAsync(q, Q_host, bytes, cudaMemcpyHostToDevice, st));
+  SPR_CUDA(cudaMemcpyAsync(q + bytes, K_host, bytes, cudaMemcpyHostToDevice, st));
+  SPR_CUDA(cudaMemcpyAsync(q + 2 * bytes, V_host, bytes, cudaMemcpyHostToDevice, st));
+  SPR_CHECK(sparsepr_forward(p, q, q + bytes, q + 2 * bytes, o_dev, nullptr, workspace, ws_bytes, stream));
+  SPR_CUDA(cudaMemcpyAsync(O_host, o_dev, bytes, cudaMemcpyDeviceToHost, st));
+  return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_dense_attention(const sparsepr_params* p, const void* Q, const void* K, const void* V,
+                                         void* O, float* lse, void* workspace, size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  SPR_CHECK(check_params(p));
+  SPR_NONNULL(Q); SPR_NONNULL(K); SPR_NONNULL(V); SPR_NONNULL(O);
+  int* err = nullptr;
+  if (workspace) {
+    if (((uintptr_t)workspace & 255) != 0 || ws_bytes < 256)
+      return fail(SPARSEPR_EWORKSPACE, "workspace must be 256-byte aligned and >= 256 bytes");
+    err = static_cast<int*>(workspace);
+  }
+  AttnArgs a{};
+  a.Q = Q; a.K = K; a.V = V;
+  a.BH = p->B * p->H; a.N = p->N; a.D = p->d;
+  a.scale_log2 = eff_scale(*p) * 1.4426950408889634f;
+  a.O = O; a.lse = lse; a.err = err;
+  SPR_LAUNCH(launch_attention(a, true, (cudaStream_t)stream));
+  return SPARSEPR_OK;
+}
+
+int sparsepr_workspace_error(const sparsepr_params* p, void* workspace, void* stream) {
+  if (check_params(p) != SPARSEPR_OK || !workspace) return -1;
+  int h = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&h, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return -1;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return -1;
+  return h;
+}
+
+sparsepr_status sparsepr_workspace_clear_error(const sparsepr_params* p, void* workspace, void* stream) {
+  SPR_CHECK(check_params(p));
+  SPR_NONNULL(workspace);
+  cudaStream_t st = (cudaStream_t)stream;
+  SPR_CUDA(cudaMemsetAsync(workspace, 0, 4, st));
+  SPR_CUDA(cudaStreamSynchronize(st));
+  return SPARSEPR_OK;
+}
+
+const char* sparsepr_status_string(sparsepr_status s) {
+  switch (s) {
+    case SPARSEPR_OK: return "ok";
+    case SPARSEPR_EINVAL: return "invalid argument";
+    case SPARSEPR_EUNSUPPORTED: return "unsupported configuration";
+    case SPARSEPR_EWORKSPACE: return "workspace too small or misaligned";
+    case SPARSEPR_ECUDA: return "CUDA error";
+    case SPARSEPR_EDEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+const char* sparsepr_last_error(void) { return g_detail; }
+
+int sparsepr_last_launch_count(void) { return g_launches; }
+
+}  // extern "C"

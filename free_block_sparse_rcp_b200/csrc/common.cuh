@@ -1,0 +1,131 @@
+// Shared device helpers of the SparsePR CUDA library (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sparsepr.h"
+
+namespace spr {
+
+// ---------------------------------------------------------------------------
+// Device error codes written to the workspace error word (first writer wins).
+// ---------------------------------------------------------------------------
+enum DeviceError : int {
+  DERR_NONE = 0,
+  DERR_INDEX = 1,        // an index read from an input array was out of range
+  DERR_WAIT_TIMEOUT = 2, // a bounded wait on an mbarrier ran out
+  DERR_DRAW = 3,         // random draw map overflow
+  DERR_NONFINITE = 4     // non-finite value where the algorithm forbids one
+};
+
+__device__ __forceinline__ void set_error(int* err, int code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+// ---------------------------------------------------------------------------
+// SplitMix64 (Steele, Lea & Flood 2014): state += 0x9E3779B97F4A7C15, output =
+// mix(state) with the two xor-shift-multiply rounds and a final xor-shift.
+// Streams: state0 = mix(seed + 0xD1B54A32D192ED03 * (8*bh + purpose + 1)).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t sm64_mix(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+struct SplitMix64 {
+  uint64_t s;
+  __device__ explicit SplitMix64(uint64_t state) : s(state) {}
+  __device__ __forceinline__ uint64_t next() {
+    s += 0x9E3779B97F4A7C15ull;
+    return sm64_mix(s);
+  }
+};
+
+enum Purpose : int { PURPOSE_QUERY_SAMPLE = 0, PURPOSE_KEY_KMEANS = 1, PURPOSE_QUERY_KMEANS = 2,
+                     PURPOSE_PROBES = 3 };
+
+__device__ __forceinline__ uint64_t stream_state(uint64_t seed, int bh, int purpose) {
+  return sm64_mix(seed + 0xD1B54A32D192ED03ull * (uint64_t)(8ll * bh + purpose + 1));
+}
+
+// Partial Fisher-Yates over the virtual array [0, n) with the swapped slots kept in
+// a small open-addressing map (slot -> value) in shared memory.  One thread runs it.
+struct SlotMap {
+  int* key;
+  int* val;
+  int cap;  // power of two
+  __device__ void clear_all(int tid, int nthreads) {
+    for (int i = tid; i < cap; i += nthreads) key[i] = -1;
+  }
+  __device__ __forceinline__ int find(int pos) const {
+    uint32_t h = ((uint32_t)pos * 2654435761u) & (cap - 1);
+    while (key[h] != -1 && key[h] != pos) h = (h + 1) & (cap - 1);
+    return (int)h;
+  }
+  __device__ __forceinline__ int get(int pos) const {
+    int h = find(pos);
+    return key[h] == pos ? val[h] : pos;
+  }
+  __device__ __forceinline__ void put(int pos, int v) {
+    int h = find(pos);
+    key[h] = pos;
+    val[h] = v;
+  }
+};
+
+// Draw m distinct values of [0, n) (m <= cap/2); out[i] = i-th drawn value.
+// The map must be cleared.  Returns false on overflow.
+__device__ inline bool draw_without_replacement(SplitMix64& g, int n, int m, SlotMap& map,
+                                                int* out) {
+  if (2 * m > map.cap) return false;
+  for (int i = 0; i < m; ++i) {
+    int j = i + (int)(g.next() % (uint64_t)(n - i));
+    int vi = map.get(i);
+    int vj = map.get(j);
+    map.put(i, vj);
+    map.put(j, vi);
+    out[i] = vj;
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// 2^x with the hardware approximation (ex2.approx, max error ~2 ulp).
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace spr

@@ -1,0 +1,87 @@
+// Internal launcher declarations of the SparsePR CUDA library.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace spr {
+
+// partition.cu
+cudaError_t launch_sample_metric(const void* Q, int BH, int N, int D, int Ms, uint64_t seed, float* metric,
+                                 int* sample_idx, int* err, cudaStream_t st);
+cudaError_t launch_metric_eigen(const float* metric, int BH, int D, int R, float* eigval, float* eigvec,
+                                float* proj, cudaStream_t st);
+cudaError_t launch_key_coords(const void* K, int BH, int N, int D, int R, const float* proj, float* Y,
+                              cudaStream_t st);
+int kmeans_dt(int Dc);
+cudaError_t launch_kmeans_seed(const float* X, int BH, int N, int Dc, int G, uint64_t seed, int purpose,
+                               float* cent, int* init_out, int* err, cudaStream_t st);
+cudaError_t launch_kmeans_assign(const float* X, int BH, int N, int Dc, int G, const float* cent, int* labels,
+                                 int* trace, cudaStream_t st);
+cudaError_t launch_group_sort(const int* labels, int BH, int N, int G, int* perm, int* offsets, int* err,
+                              cudaStream_t st);
+cudaError_t launch_segment_mean_f32(const float* X, int BH, int N, int Dc, int G, const int* perm,
+                                    const int* offsets, float* cent, int zero_empty, cudaStream_t st);
+cudaError_t launch_segment_mean_bf16(const void* X, int BH, int N, int D, int G, const int* perm,
+                                     const int* offsets, float* cent, cudaStream_t st);
+cudaError_t launch_query_coords(const void* Q, int BH, int N, int D, const float* C, int G, float scale,
+                                float* Z, cudaStream_t st);
+cudaError_t launch_cell_mass(const float* Z, int BH, int N, int Gk, int Gq, const int* perm_q, const int* qoff,
+                             const int* koff, float* mass, cudaStream_t st);
+cudaError_t launch_route_select(const float* mass, int BH, int N, int Gq, int Gk, const int* qoff,
+                                const int* koff, float density, int P, int* order, double* cm,
+                                long long* cc, unsigned char* route, float* rho_exec, double* alpha,
+                                cudaStream_t st);
+cudaError_t launch_block_mask(const unsigned char* route, int BH, int N, int Gq, int Gk, int blk,
+                              const int* perm_q, const int* label_q, const int* perm_k, const int* label_k,
+                              unsigned char* bmask, cudaStream_t st);
+
+// probe.cu
+cudaError_t launch_worklist(const unsigned char* route, const int* qoff, const int* koff, int BH, int Gq, int Gk,
+                           int tile_rows, int max_tiles, int* rlist, int* rcum, int* rcnt, int2* tiles,
+                           int* tile_count, cudaStream_t st);
+cudaError_t launch_probe_pick(const int* perm_q, const int* qoff, int BH, int N, int Gq, int P, uint64_t seed,
+                              int* probe_idx, int* probe_grp, int* err, cudaStream_t st);
+int probe_splits(int N);
+size_t probe_attn_smem(int D, int Gk);
+size_t probe_fit_smem(int D, int Rk);
+cudaError_t launch_probe_attn(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk, int Gq,
+                              int P, const int* probe_idx, const int* probe_grp, const int* label_k,
+                              const unsigned char* route, float scale_log2, float* part_o, float* part_ml,
+                              cudaStream_t st);
+cudaError_t launch_probe_combine(const float* part_o, const float* part_ml, int BH, int N, int P, int D,
+                                 float* o_dense, float* o_sparse, float* lse_d, float* lse_s, cudaStream_t st);
+cudaError_t launch_probe_fit(const float* o_dense, const float* o_sparse, int BH, int D, int P, int Rk,
+                             double lam, float* Vr, float* W, float* bfull, float* Bmat, float* sigma,
+                             float* bsub, cudaStream_t st);
+cudaError_t launch_reconstruct(const void* Os, int BH, int N, int D, int Rk, const float* W, const float* Vr,
+                               const float* bfull, void* O, cudaStream_t st);
+cudaError_t launch_probe_scatter(const int* probe_idx, const float* o_dense, int BH, int N, int P, int D, void* O,
+                                 cudaStream_t st);
+
+// attention
+struct AttnArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  int BH, N, D, Gq, Gk;
+  const int* perm_q;
+  const int* perm_k;
+  const int* qoff;
+  const int* koff;
+  const int* rlist;
+  const int* rcum;
+  const int* rcnt;
+  const int2* tiles;
+  const int* tile_count;
+  int max_tiles;
+  float scale_log2;
+  void* O;
+  float* lse;
+  int* err;
+};
+size_t attn_smem_bytes(int D, int Gk);
+cudaError_t launch_attention(const AttnArgs& a, bool dense, cudaStream_t st);
+constexpr int kAttnTileRows = 128;
+
+}  // namespace spr

@@ -1,0 +1,670 @@
+// Response-coupled partition kernels (gist.science technical summary, section 2.A;
+// huashangw.com article, method walkthrough and sparse-execution section).
+//
+//   sample + metric   M_K = Q_s^T Q_s / M_s over M_s sampled query rows
+//   eigen             leading r_e eigenpairs of M_K (single-CTA Jacobi)
+//   key coordinates   y = Lambda^{1/2} U^T k
+//   k-means           Lloyd: direct-form squared distances in fp32, ties to the
+//                     lowest cluster, fp64 member sums, empty clusters keep
+//                     their centroid
+//   group sort        stable counting sort by label -> permutation + offsets
+//   centroids         mean raw key of every K/V group
+//   query coordinates z = s C q (logits against the K/V group centroids)
+//   cell mass         mean over group a of softmax_g(z_q[g] + ln n_g)
+//   route             shared alpha by bisection under the pair budget
+//   block mask        tile-level view of the route on the permuted layout
+#include "common.cuh"
+#include "jacobi.cuh"
+#include "kernels.h"
+
+namespace spr {
+
+// ---------------------------------------------------------------------------
+// Sampled queries and M_K.  grid = BH, block = 256.
+// ---------------------------------------------------------------------------
+constexpr int kMapCap = 4096;
+
+template <int D>
+__global__ void __launch_bounds__(256) k_sample_metric(const __nv_bfloat16* __restrict__ Q, int N,
+                                                      int Ms, uint64_t seed, float* __restrict__ metric,
+                                                      int* __restrict__ sample_idx, int* err) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  int* mkey = reinterpret_cast<int*>(smem);
+  int* mval = mkey + kMapCap;
+  int* sidx = mval + kMapCap;                                   // [Ms]
+  float* qs = reinterpret_cast<float*>(sidx + ((Ms + 3) & ~3)); // [64][D]
+  const int bh = blockIdx.x, tid = threadIdx.x;
+  SlotMap map{mkey, mval, kMapCap};
+  map.clear_all(tid, blockDim.x);
+  __syncthreads();
+  if (tid == 0) {
+    SplitMix64 g(stream_state(seed, bh, PURPOSE_QUERY_SAMPLE));
+    if (!draw_without_replacement(g, N, Ms, map, sidx)) set_error(err, DERR_DRAW);
+  }
+  __syncthreads();
+  for (int i = tid; i < Ms; i += blockDim.x) sample_idx[(size_t)bh * Ms + i] = sidx[i];
+  constexpr int PER = D * D / 256;
+  float acc[PER];
+#pragma unroll
+  for (int j = 0; j < PER; ++j) acc[j] = 0.f;
+  const __nv_bfloat16* Qh = Q + (size_t)bh * N * D;
+  for (int s0 = 0; s0 < Ms; s0 += 64) {
+    const int ns = min(64, Ms - s0);
+    for (int e = tid; e < ns * D; e += blockDim.x) {
+      int s = e / D, c = e - s * D;
+      qs[s * D + c] = bf2f(Qh[(size_t)sidx[s0 + s] * D + c]);
+    }
+    __syncthreads();
+    for (int s = 0; s < ns; ++s) {
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        int e = tid + 256 * j;
+        int r = e / D, c = e - r * D;
+        acc[j] = fmaf(qs[s * D + r], qs[s * D + c], acc[j]);
+      }
+    }
+    __syncthreads();
+  }
+  const float inv = 1.0f / (float)Ms;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) metric[(size_t)bh * D * D + tid + 256 * j] = acc[j] * inv;
+}
+
+// ---------------------------------------------------------------------------
+// Leading eigenpairs of M_K.  grid = BH, block = 512.
+// Writes eigval [BH, R] (clamped >= 0), eigvec [BH, D, R] and the projector
+// P = U_R Lambda_R^{1/2} [BH, D, R] used for the key coordinates.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(512) k_metric_eigen(const float* __restrict__ metric, int R,
+                                                     float* __restrict__ eigval, float* __restrict__ eigvec,
+                                                     float* __restrict__ proj) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  constexpr int LD = D + 1;
+  float* A = reinterpret_cast<float*>(smem);
+  float* V = A + D * LD;
+  float* cs = V + D * LD;
+  float* red = cs + D;
+  int* pr = reinterpret_cast<int*>(red + 64);
+  int* rank = pr + D;
+  const int bh = blockIdx.x;
+  for (int i = threadIdx.x; i < D * D; i += blockDim.x) {
+    int r = i / D, c = i - r * D;
+    A[r * LD + c] = metric[(size_t)bh * D * D + i];
+  }
+  __syncthreads();
+  jacobi_eigen<float>(A, V, D, LD, cs, pr, red, 30, 2e-7f);
+  eigen_ranks<float>(A, D, LD, rank);
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    int k = rank[i];
+    if (k < R) {
+      float lam = fmaxf(A[i * LD + i], 0.f);
+      eigval[(size_t)bh * R + k] = lam;
+      float sl = sqrtf(lam);
+      for (int c = 0; c < D; ++c) {
+        float u = V[c * LD + i];
+        eigvec[((size_t)bh * D + c) * R + k] = u;
+        proj[((size_t)bh * D + c) * R + k] = u * sl;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Key coordinates y = P^T k.  grid = (ceil(N/64), BH), block = 256.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) k_key_coords(const __nv_bfloat16* __restrict__ K, int N, int R,
+                                                   const float* __restrict__ proj, float* __restrict__ Y) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* ps = reinterpret_cast<float*>(smem);  // [D][R]
+  float* ks = ps + D * R;                      // [64][D+1]
+  const int bh = blockIdx.y, n0 = blockIdx.x * 64, tid = threadIdx.x;
+  for (int i = tid; i < D * R; i += blockDim.x) ps[i] = proj[(size_t)bh * D * R + i];
+  const int nr = min(64, N - n0);
+  const __nv_bfloat16* Kh = K + ((size_t)bh * N + n0) * D;
+  for (int e = tid; e < nr * D; e += blockDim.x) {
+    int r = e / D, c = e - r * D;
+    ks[r * (D + 1) + c] = bf2f(Kh[e]);
+  }
+  __syncthreads();
+  for (int e = tid; e < nr * R; e += blockDim.x) {
+    int r = e / R, j = e - r * R;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < D; ++c) acc = fmaf(ks[r * (D + 1) + c], ps[c * R + j], acc);
+    Y[((size_t)bh * N + n0 + r) * R + j] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// k-means seeds: G distinct rows of X drawn with the purpose's stream; centroid j
+// starts at the j-th drawn row.  grid = BH, block = 256.  Centroids are stored
+// with row stride DT (zero padded past Dc).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_kmeans_seed(const float* __restrict__ X, int N, int Dc, int DT,
+                                                    int G, uint64_t seed, int purpose,
+                                                    float* __restrict__ cent, int* __restrict__ init_out,
+                                                    int* err) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  int* mkey = reinterpret_cast<int*>(smem);
+  int* mval = mkey + kMapCap;
+  int* sidx = mval + kMapCap;
+  const int bh = blockIdx.x, tid = threadIdx.x;
+  SlotMap map{mkey, mval, kMapCap};
+  map.clear_all(tid, blockDim.x);
+  __syncthreads();
+  if (tid == 0) {
+    SplitMix64 g(stream_state(seed, bh, purpose));
+    if (!draw_without_replacement(g, N, G, map, sidx)) set_error(err, DERR_DRAW);
+  }
+  __syncthreads();
+  for (int e = tid; e < G * DT; e += blockDim.x) {
+    int g = e / DT, c = e - g * DT;
+    cent[(size_t)bh * G * DT + e] = c < Dc ? X[((size_t)bh * N + sidx[g]) * Dc + c] : 0.f;
+  }
+  if (init_out)
+    for (int g = tid; g < G; g += blockDim.x) init_out[(size_t)bh * G + g] = sidx[g];
+}
+
+// ---------------------------------------------------------------------------
+// k-means assignment: label = argmin_g sum_c (x_c - mu_gc)^2 (sequential fp32 fma
+// over c), strict '<' so ties keep the lowest g.  grid = (ceil(N/128), BH),
+// block = 128, dynamic smem = G * DT floats.
+// ---------------------------------------------------------------------------
+template <int DT>
+__global__ void __launch_bounds__(128) k_kmeans_assign(const float* __restrict__ X, int N, int Dc, int G,
+                                                      const float* __restrict__ cent, int* __restrict__ labels,
+                                                      int* __restrict__ trace) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* mu = reinterpret_cast<float*>(smem);
+  const int bh = blockIdx.y, tid = threadIdx.x;
+  const float4* c4 = reinterpret_cast<const float4*>(cent + (size_t)bh * G * DT);
+  float4* m4 = reinterpret_cast<float4*>(mu);
+  for (int i = tid; i < G * DT / 4; i += blockDim.x) m4[i] = c4[i];
+  __syncthreads();
+  const int i = blockIdx.x * 128 + tid;
+  if (i >= N) return;
+  float x[DT];
+  const float* xr = X + ((size_t)bh * N + i) * Dc;
+#pragma unroll
+  for (int c = 0; c < DT; ++c) x[c] = c < Dc ? xr[c] : 0.f;
+  float best = __int_as_float(0x7f800000);
+  int lab = 0;
+  for (int g = 0; g < G; ++g) {
+    const float4* mg = m4 + g * (DT / 4);
+    float dist = 0.f;
+#pragma unroll
+    for (int c4i = 0; c4i < DT / 4; ++c4i) {
+      float4 m = mg[c4i];
+      float t;
+      t = x[4 * c4i + 0] - m.x; dist = fmaf(t, t, dist);
+      t = x[4 * c4i + 1] - m.y; dist = fmaf(t, t, dist);
+      t = x[4 * c4i + 2] - m.z; dist = fmaf(t, t, dist);
+      t = x[4 * c4i + 3] - m.w; dist = fmaf(t, t, dist);
+    }
+    if (dist < best) { best = dist; lab = g; }
+  }
+  labels[(size_t)bh * N + i] = lab;
+  if (trace) trace[(size_t)bh * N + i] = lab;
+}
+
+// ---------------------------------------------------------------------------
+// Stable counting sort by label.  grid = BH, block = 1024, dynamic smem =
+// (33 * G) ints.  perm[pos] = original index; offsets[g] = first position.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) k_group_sort(const int* __restrict__ labels, int N, int G,
+                                                    int* __restrict__ perm, int* __restrict__ offsets,
+                                                    int* err) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  int* base = reinterpret_cast<int*>(smem);  // [G]
+  int* wcnt = base + G;                       // [32][G]
+  const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int* lab = labels + (size_t)bh * N;
+  for (int g = tid; g < G; g += blockDim.x) base[g] = 0;
+  __syncthreads();
+  for (int i = tid; i < N; i += blockDim.x) {
+    int l = lab[i];
+    if (l < 0 || l >= G) { set_error(err, DERR_INDEX); continue; }
+    atomicAdd(&base[l], 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int g = 0; g < G; ++g) {
+      int c = base[g];
+      base[g] = run;
+      offsets[(size_t)bh * (G + 1) + g] = run;
+      run += c;
+    }
+    offsets[(size_t)bh * (G + 1) + G] = run;
+  }
+  __syncthreads();
+  for (int t0 = 0; t0 < N; t0 += blockDim.x) {
+    for (int e = tid; e < 32 * G; e += blockDim.x) wcnt[e] = 0;
+    __syncthreads();
+    const int i = t0 + tid;
+    int l = (i < N) ? lab[i] : -1;
+    if (l >= G) l = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, l);
+    const int rank = __popc(peers & ((1u << lane) - 1));
+    if (l >= 0 && lane == __ffs(peers) - 1) wcnt[warp * G + l] = __popc(peers);
+    __syncthreads();
+    if (l >= 0) {
+      int pre = 0;
+      for (int w = 0; w < warp; ++w) pre += wcnt[w * G + l];
+      perm[(size_t)bh * N + base[l] + pre + rank] = i;
+    }
+    __syncthreads();
+    for (int g = tid; g < G; g += blockDim.x) {
+      int s = 0;
+      for (int w = 0; w < 32; ++w) s += wcnt[w * G + g];
+      base[g] += s;
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Segment means: cent[g][c] = mean over permuted positions of group g of X[perm][c]
+// (fp64 sums in ascending original order); empty groups keep their value unless
+// zero_empty, in which case they become 0.  grid = (G, BH), block = 128.
+// ---------------------------------------------------------------------------
+template <typename TIn>
+__global__ void __launch_bounds__(128) k_segment_mean(const TIn* __restrict__ X, int N, int Dc, int DT, int G,
+                                                     const int* __restrict__ perm,
+                                                     const int* __restrict__ offsets, float* __restrict__ cent,
+                                                     int zero_empty) {
+  const int g = blockIdx.x, bh = blockIdx.y;
+  const int s0 = offsets[(size_t)bh * (G + 1) + g], s1 = offsets[(size_t)bh * (G + 1) + g + 1];
+  const int* pm = perm + (size_t)bh * N;
+  const TIn* Xh = X + (size_t)bh * N * Dc;
+  float* out = cent + ((size_t)bh * G + g) * DT;
+  for (int c = threadIdx.x; c < DT; c += blockDim.x) {
+    if (c >= Dc) { out[c] = 0.f; continue; }
+    if (s1 == s0) { if (zero_empty) out[c] = 0.f; continue; }
+    double acc = 0.0;
+    for (int s = s0; s < s1; ++s) acc += (double)to_f32(Xh[(size_t)pm[s] * Dc + c]);
+    out[c] = (float)(acc / (double)(s1 - s0));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Query coordinates z = s Q C^T (fp32).  grid = (ceil(N/64), ceil(G/64), BH),
+// block = 256, each thread a 4 x 4 output patch.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) k_query_coords(const __nv_bfloat16* __restrict__ Q, int N,
+                                                     const float* __restrict__ C, int G, float scale,
+                                                     float* __restrict__ Z) {
+  __shared__ __align__(16) float qs[16][64 + 4];
+  __shared__ __align__(16) float csm[16][64 + 4];
+  const int bh = blockIdx.z, n0 = blockIdx.x * 64, g0 = blockIdx.y * 64, tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  float acc[4][4] = {};
+  const __nv_bfloat16* Qh = Q + (size_t)bh * N * D;
+  const float* Ch = C + (size_t)bh * G * D;
+  for (int k0 = 0; k0 < D; k0 += 16) {
+    for (int e = tid; e < 64 * 16; e += 256) {
+      int r = e >> 4, k = e & 15;
+      qs[k][r] = (n0 + r < N) ? bf2f(Qh[(size_t)(n0 + r) * D + k0 + k]) : 0.f;
+      csm[k][r] = (g0 + r < G) ? Ch[(size_t)(g0 + r) * D + k0 + k] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      float4 a = *reinterpret_cast<const float4*>(&qs[k][ty * 4]);
+      float4 b = *reinterpret_cast<const float4*>(&csm[k][tx * 4]);
+      float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int n = n0 + ty * 4 + i;
+    if (n >= N) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int g = g0 + tx * 4 + j;
+      if (g < G) Z[((size_t)bh * N + n) * G + g] = scale * acc[i][j];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Cell mass p(a, g) = mean over queries of group a of softmax_g(z_q[g] + ln n_g)
+// (empty K/V groups excluded).  grid = (Gq, BH), block = 256; each warp owns
+// every 8th member and accumulates its own row of partial sums (deterministic).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_cell_mass(const float* __restrict__ Z, int N, int Gk, int Gq,
+                                                  const int* __restrict__ perm_q, const int* __restrict__ qoff,
+                                                  const int* __restrict__ koff, float* __restrict__ mass) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* lnn = reinterpret_cast<float*>(smem);  // [Gk]
+  float* part = lnn + Gk;                       // [8][Gk]
+  const int a = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float NEG_INF = __int_as_float(0xff800000);
+  for (int g = tid; g < Gk; g += blockDim.x) {
+    int n = koff[(size_t)bh * (Gk + 1) + g + 1] - koff[(size_t)bh * (Gk + 1) + g];
+    lnn[g] = n > 0 ? logf((float)n) : NEG_INF;
+  }
+  for (int e = tid; e < 8 * Gk; e += blockDim.x) part[e] = 0.f;
+  __syncthreads();
+  const int s0 = qoff[(size_t)bh * (Gq + 1) + a], s1 = qoff[(size_t)bh * (Gq + 1) + a + 1];
+  const int* pm = perm_q + (size_t)bh * N;
+  for (int s = s0 + warp; s < s1; s += 8) {
+    const float* zr = Z + ((size_t)bh * N + pm[s]) * Gk;
+    float mx = NEG_INF;
+    for (int g = lane; g < Gk; g += 32) mx = fmaxf(mx, lnn[g] == NEG_INF ? NEG_INF : zr[g] + lnn[g]);
+    mx = warp_max(mx);
+    float sum = 0.f;
+    for (int g = lane; g < Gk; g += 32) sum += lnn[g] == NEG_INF ? 0.f : expf(zr[g] + lnn[g] - mx);
+    sum = warp_sum(sum);
+    const float inv = 1.0f / sum;
+    for (int g = lane; g < Gk; g += 32)
+      part[warp * Gk + g] += lnn[g] == NEG_INF ? 0.f : expf(zr[g] + lnn[g] - mx) * inv;
+  }
+  __syncthreads();
+  const int na = s1 - s0;
+  for (int g = tid; g < Gk; g += blockDim.x) {
+    float t = 0.f;
+    for (int w = 0; w < 8; ++w) t += part[w * Gk + g];
+    mass[((size_t)bh * Gq + a) * Gk + g] = na > 0 ? t / (float)na : 0.f;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Route selection (one CTA per head, block = 1024).
+// Per query group a: non-empty K/V groups sorted by mass descending (ties -> lower
+// g), sequential fp64 cumulative mass and int64 cumulative cost n_a * n_g.  The
+// shared alpha is the largest value in [0, 1] whose total cost fits
+// budget = density * N^2 - P * N (60 bisection steps in fp64); each group keeps
+// the shortest prefix reaching alpha (at least one cell).  density >= 1 routes all
+// non-empty cells.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int prefix_len(const double* cm, int L, double alpha) {
+  int lo = 0, hi = L;
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (cm[mid] >= alpha) hi = mid; else lo = mid + 1;
+  }
+  int n = lo < L ? lo + 1 : L;
+  return n < 1 ? 1 : n;
+}
+
+__device__ long long block_sum_ll(long long v, long long* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  long long t = 0;
+  for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) t += red[w];
+  __syncthreads();
+  return t;
+}
+
+__global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__ mass, int N, int Gq, int Gk,
+                                                      const int* __restrict__ qoff, const int* __restrict__ koff,
+                                                      float density, int P, int* __restrict__ order,
+                                                      double* __restrict__ cm, long long* __restrict__ cc,
+                                                      unsigned char* __restrict__ route,
+                                                      float* __restrict__ rho_exec, double* __restrict__ alpha_out) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  long long* red = reinterpret_cast<long long*>(smem);     // [32]
+  int* nk = reinterpret_cast<int*>(red + 32);              // [Gk]
+  int* nq = nk + Gk;                                       // [Gq]
+  int* ne = nq + Gq;                                       // [1]: number of non-empty K/V groups
+  const int bh = blockIdx.x, tid = threadIdx.x;
+  const float* mh = mass + (size_t)bh * Gq * Gk;
+  int* oh = order + (size_t)bh * Gq * Gk;
+  double* cmh = cm + (size_t)bh * Gq * Gk;
+  long long* cch = cc + (size_t)bh * Gq * Gk;
+  unsigned char* rh = route + (size_t)bh * Gq * Gk;
+  for (int g = tid; g < Gk; g += blockDim.x) nk[g] = koff[(size_t)bh * (Gk + 1) + g + 1] - koff[(size_t)bh * (Gk + 1) + g];
+  for (int a = tid; a < Gq; a += blockDim.x) nq[a] = qoff[(size_t)bh * (Gq + 1) + a + 1] - qoff[(size_t)bh * (Gq + 1) + a];
+  __syncthreads();
+  if (tid == 0) {
+    int c = 0;
+    for (int g = 0; g < Gk; ++g) c += nk[g] > 0;
+    ne[0] = c;
+  }
+  __syncthreads();
+  const int L = ne[0];
+  // ranks inside each row
+  for (int e = tid; e < Gq * Gk; e += blockDim.x) {
+    int a = e / Gk, g = e - a * Gk;
+    if (nq[a] == 0 || nk[g] == 0) continue;
+    const float m = mh[e];
+    int r = 0;
+    for (int h = 0; h < Gk; ++h) {
+      if (nk[h] == 0) continue;
+      float mh2 = mh[a * Gk + h];
+      r += (mh2 > m) || (mh2 == m && h < g);
+    }
+    oh[a * Gk + r] = g;
+  }
+  __syncthreads();
+  for (int a = tid; a < Gq; a += blockDim.x) {
+    if (nq[a] == 0) continue;
+    double s = 0.0;
+    long long c = 0;
+    for (int r = 0; r < L; ++r) {
+      int g = oh[a * Gk + r];
+      s += (double)mh[a * Gk + g];
+      c += (long long)nq[a] * (long long)nk[g];
+      cmh[a * Gk + r] = s;
+      cch[a * Gk + r] = c;
+    }
+  }
+  __syncthreads();
+  const double visible = (double)N * (double)N;
+  const double probe_pairs = (double)P * (double)N;
+  const double budget = (double)density * visible - probe_pairs;
+  double alpha;
+  const bool all = density >= 1.0f;
+  if (all) {
+    alpha = 1.0;
+  } else {
+    auto cost_at = [&](double al) -> long long {
+      long long t = 0;
+      for (int a = tid; a < Gq; a += blockDim.x)
+        if (nq[a] > 0) t += cch[a * Gk + prefix_len(cmh + a * Gk, L, al) - 1];
+      return block_sum_ll(t, red);
+    };
+    double lo = 0.0, hi = 1.0;
+    if ((double)cost_at(lo) <= budget) {
+      for (int it = 0; it < 60; ++it) {
+        double mid = 0.5 * (lo + hi);
+        if ((double)cost_at(mid) <= budget) lo = mid; else hi = mid;
+      }
+    }
+    alpha = lo;
+  }
+  for (int e = tid; e < Gq * Gk; e += blockDim.x) rh[e] = 0;
+  __syncthreads();
+  long long routed = 0;
+  for (int a = tid; a < Gq; a += blockDim.x) {
+    if (nq[a] == 0) continue;
+    int len = all ? L : prefix_len(cmh + a * Gk, L, alpha);
+    for (int r = 0; r < len; ++r) rh[a * Gk + oh[a * Gk + r]] = 1;
+    routed += cch[a * Gk + len - 1];
+  }
+  routed = block_sum_ll(routed, red);
+  if (tid == 0) {
+    rho_exec[bh] = (float)(((double)routed + probe_pairs) / visible);
+    if (alpha_out) alpha_out[bh] = alpha;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tile mask of the permuted layout.  grid = (T, BH), block = 256.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_block_mask(const unsigned char* __restrict__ route, int N, int Gq,
+                                                   int Gk, int blk, const int* __restrict__ perm_q,
+                                                   const int* __restrict__ label_q,
+                                                   const int* __restrict__ perm_k,
+                                                   const int* __restrict__ label_k,
+                                                   unsigned char* __restrict__ bmask) {
+  const int i = blockIdx.x, bh = blockIdx.y, T = (N + blk - 1) / blk;
+  const int* pq = perm_q + (size_t)bh * N;
+  const int* pk = perm_k + (size_t)bh * N;
+  const int* lq = label_q + (size_t)bh * N;
+  const int* lk = label_k + (size_t)bh * N;
+  const int a0 = lq[pq[i * blk]], a1 = lq[pq[min(N, (i + 1) * blk) - 1]];
+  const unsigned char* rh = route + (size_t)bh * Gq * Gk;
+  for (int j = threadIdx.x; j < T; j += blockDim.x) {
+    const int g0 = lk[pk[j * blk]], g1 = lk[pk[min(N, (j + 1) * blk) - 1]];
+    unsigned char v = 0;
+    for (int a = a0; a <= a1 && !v; ++a)
+      for (int g = g0; g <= g1; ++g)
+        if (rh[a * Gk + g]) { v = 1; break; }
+    bmask[((size_t)bh * T + i) * T + j] = v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers
+// ---------------------------------------------------------------------------
+static size_t sample_smem(int Ms, int D) {
+  return (size_t)(2 * kMapCap + ((Ms + 3) & ~3)) * 4 + (size_t)64 * D * 4;
+}
+
+cudaError_t launch_sample_metric(const void* Q, int BH, int N, int D, int Ms, uint64_t seed, float* metric,
+                                 int* sample_idx, int* err, cudaStream_t st) {
+  size_t sm = sample_smem(Ms, D);
+  if (D == 64) {
+    cudaFuncSetAttribute(k_sample_metric<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_sample_metric<64><<<BH, 256, sm, st>>>((const __nv_bfloat16*)Q, N, Ms, seed, metric, sample_idx, err);
+  } else {
+    cudaFuncSetAttribute(k_sample_metric<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_sample_metric<128><<<BH, 256, sm, st>>>((const __nv_bfloat16*)Q, N, Ms, seed, metric, sample_idx, err);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_metric_eigen(const float* metric, int BH, int D, int R, float* eigval, float* eigvec,
+                                float* proj, cudaStream_t st) {
+  size_t sm = (size_t)(2 * D * (D + 1) + D + 64) * 4 + (size_t)(2 * D) * 4;
+  if (D == 64) {
+    cudaFuncSetAttribute(k_metric_eigen<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_metric_eigen<64><<<BH, 512, sm, st>>>(metric, R, eigval, eigvec, proj);
+  } else {
+    cudaFuncSetAttribute(k_metric_eigen<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_metric_eigen<128><<<BH, 512, sm, st>>>(metric, R, eigval, eigvec, proj);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_key_coords(const void* K, int BH, int N, int D, int R, const float* proj, float* Y,
+                              cudaStream_t st) {
+  size_t sm = (size_t)(D * R + 64 * (D + 1)) * 4;
+  dim3 grid(ceil_div(N, 64), BH);
+  if (D == 64) {
+    cudaFuncSetAttribute(k_key_coords<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_key_coords<64><<<grid, 256, sm, st>>>((const __nv_bfloat16*)K, N, R, proj, Y);
+  } else {
+    cudaFuncSetAttribute(k_key_coords<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_key_coords<128><<<grid, 256, sm, st>>>((const __nv_bfloat16*)K, N, R, proj, Y);
+  }
+  return cudaGetLastError();
+}
+
+int kmeans_dt(int Dc) {
+  int dt = 8;
+  while (dt < Dc) dt *= 2;
+  return dt;
+}
+
+cudaError_t launch_kmeans_seed(const float* X, int BH, int N, int Dc, int G, uint64_t seed, int purpose,
+                               float* cent, int* init_out, int* err, cudaStream_t st) {
+  size_t sm = (size_t)(2 * kMapCap + G) * 4;
+  cudaFuncSetAttribute(k_kmeans_seed, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  k_kmeans_seed<<<BH, 256, sm, st>>>(X, N, Dc, kmeans_dt(Dc), G, seed, purpose, cent, init_out, err);
+  return cudaGetLastError();
+}
+
+template <int DT>
+static cudaError_t assign_dt(const float* X, int BH, int N, int Dc, int G, const float* cent, int* labels,
+                             int* trace, cudaStream_t st) {
+  size_t sm = (size_t)G * DT * 4;
+  cudaFuncSetAttribute(k_kmeans_assign<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  k_kmeans_assign<DT><<<dim3(ceil_div(N, 128), BH), 128, sm, st>>>(X, N, Dc, G, cent, labels, trace);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kmeans_assign(const float* X, int BH, int N, int Dc, int G, const float* cent, int* labels,
+                                 int* trace, cudaStream_t st) {
+  switch (kmeans_dt(Dc)) {
+    case 8: return assign_dt<8>(X, BH, N, Dc, G, cent, labels, trace, st);
+    case 16: return assign_dt<16>(X, BH, N, Dc, G, cent, labels, trace, st);
+    case 32: return assign_dt<32>(X, BH, N, Dc, G, cent, labels, trace, st);
+    case 64: return assign_dt<64>(X, BH, N, Dc, G, cent, labels, trace, st);
+    case 128: return assign_dt<128>(X, BH, N, Dc, G, cent, labels, trace, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_group_sort(const int* labels, int BH, int N, int G, int* perm, int* offsets, int* err,
+                              cudaStream_t st) {
+  size_t sm = (size_t)33 * G * 4;
+  cudaFuncSetAttribute(k_group_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  k_group_sort<<<BH, 1024, sm, st>>>(labels, N, G, perm, offsets, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_segment_mean_f32(const float* X, int BH, int N, int Dc, int G, const int* perm,
+                                    const int* offsets, float* cent, int zero_empty, cudaStream_t st) {
+  k_segment_mean<float><<<dim3(G, BH), 128, 0, st>>>(X, N, Dc, kmeans_dt(Dc), G, perm, offsets, cent,
+                                                    zero_empty);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_segment_mean_bf16(const void* X, int BH, int N, int D, int G, const int* perm,
+                                     const int* offsets, float* cent, cudaStream_t st) {
+  k_segment_mean<__nv_bfloat16><<<dim3(G, BH), 128, 0, st>>>((const __nv_bfloat16*)X, N, D, D, G, perm,
+                                                            offsets, cent, 1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_query_coords(const void* Q, int BH, int N, int D, const float* C, int G, float scale,
+                                float* Z, cudaStream_t st) {
+  dim3 grid(ceil_div(N, 64), ceil_div(G, 64), BH);
+  if (D == 64)
+    k_query_coords<64><<<grid, 256, 0, st>>>((const __nv_bfloat16*)Q, N, C, G, scale, Z);
+  else
+    k_query_coords<128><<<grid, 256, 0, st>>>((const __nv_bfloat16*)Q, N, C, G, scale, Z);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cell_mass(const float* Z, int BH, int N, int Gk, int Gq, const int* perm_q, const int* qoff,
+                             const int* koff, float* mass, cudaStream_t st) {
+  size_t sm = (size_t)9 * Gk * 4;
+  cudaFuncSetAttribute(k_cell_mass, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  k_cell_mass<<<dim3(Gq, BH), 256, sm, st>>>(Z, N, Gk, Gq, perm_q, qoff, koff, mass);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_select(const float* mass, int BH, int N, int Gq, int Gk, const int* qoff,
+                                const int* koff, float density, int P, int* order, double* cm,
+                                long long* cc, unsigned char* route, float* rho_exec, double* alpha,
+                                cudaStream_t st) {
+  size_t sm = 32 * 8 + (size_t)(Gk + Gq + 4) * 4;
+  k_route_select<<<BH, 1024, sm, st>>>(mass, N, Gq, Gk, qoff, koff, density, P, order, cm, cc, route,
+                                       rho_exec, alpha);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_block_mask(const unsigned char* route, int BH, int N, int Gq, int Gk, int blk,
+                              const int* perm_q, const int* label_q, const int* perm_k, const int* label_k,
+                              unsigned char* bmask, cudaStream_t st) {
+  const int T = ceil_div(N, blk);
+  k_block_mask<<<dim3(T, BH), 256, 0, st>>>(route, N, Gq, Gk, blk, perm_q, label_q, perm_k, label_k, bmask);
+  return cudaGetLastError();
+}
+
+}  // namespace spr

@@ -1,0 +1,632 @@
+// Exact probe rows, residual subspace, ridge fit and correction (gist.science
+// technical summary, section 2.B; huashangw.com article, method walkthrough:
+// 64 probe rows per head drawn evenly from every query group, ridge regression,
+// correction inside the leading singular directions of the probe residuals).
+#include "common.cuh"
+#include "jacobi.cuh"
+#include "kernels.h"
+
+namespace spr {
+
+// ---------------------------------------------------------------------------
+// Probe rows.  Allocation by water-filling over the query groups (every group with
+// spare members gets floor(remaining / #open) per round; a share of 0 sends the
+// leftovers one each to open groups by decreasing size, ties to the lower index);
+// inside group a, alloc_a members drawn without replacement with the probe stream,
+// groups in ascending order.  grid = BH, block = 256.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_probe_pick(const int* __restrict__ perm_q, const int* __restrict__ qoff,
+                                                   int N, int Gq, int P, uint64_t seed,
+                                                   int* __restrict__ probe_idx, int* __restrict__ probe_grp,
+                                                   int* err) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  int* size = reinterpret_cast<int*>(smem);  // [Gq]
+  int* alloc = size + Gq;                     // [Gq]
+  int* order = alloc + Gq;                    // [Gq] open groups by decreasing size
+  int* draw = order + Gq;                     // [P]
+  int* mkey = draw + 64;                      // [256]
+  int* mval = mkey + 256;                     // [256]
+  int* red = mval + 256;                      // [8]
+  const int bh = blockIdx.x, tid = threadIdx.x;
+  const int* qo = qoff + (size_t)bh * (Gq + 1);
+  for (int a = tid; a < Gq; a += blockDim.x) { size[a] = qo[a + 1] - qo[a]; alloc[a] = 0; }
+  __syncthreads();
+  for (int a = tid; a < Gq; a += blockDim.x) {
+    int r = 0;
+    for (int b = 0; b < Gq; ++b) r += (size[b] > size[a]) || (size[b] == size[a] && b < a);
+    order[r] = a;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int remaining = P;
+    while (remaining > 0) {
+      int open = 0;
+      for (int a = 0; a < Gq; ++a) open += alloc[a] < size[a];
+      if (open == 0) break;
+      int share = remaining / open;
+      if (share == 0) {
+        for (int r = 0; r < Gq && remaining > 0; ++r) {
+          int a = order[r];
+          if (alloc[a] < size[a]) { alloc[a] += 1; --remaining; }
+        }
+        break;
+      }
+      for (int a = 0; a < Gq; ++a) {
+        if (alloc[a] >= size[a]) continue;
+        int add = min(share, size[a] - alloc[a]);
+        alloc[a] += add;
+        remaining -= add;
+      }
+    }
+    SplitMix64 g(stream_state(seed, bh, PURPOSE_PROBES));
+    SlotMap map{mkey, mval, 256};
+    int outp = 0;
+    for (int a = 0; a < Gq; ++a) {
+      const int m = alloc[a];
+      if (m == 0) continue;
+      for (int i = 0; i < 256; ++i) mkey[i] = -1;
+      if (!draw_without_replacement(g, size[a], m, map, draw)) { set_error(err, DERR_DRAW); break; }
+      for (int i = 0; i < m; ++i) {
+        probe_idx[(size_t)bh * P + outp] = perm_q[(size_t)bh * N + qo[a] + draw[i]];
+        probe_grp[(size_t)bh * P + outp] = a;
+        ++outp;
+      }
+    }
+    for (; outp < P; ++outp) { probe_idx[(size_t)bh * P + outp] = -1; probe_grp[(size_t)bh * P + outp] = -1; }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Dense and routed attention of the probe rows over one key split (fp32).
+// grid = (S, BH), block = 256.  Rows >= P are padding.  Writes per split and row
+// the base-2 running max, sum and unnormalised output of both accumulators.
+// ---------------------------------------------------------------------------
+constexpr int PR = 64;  // probe rows handled per CTA
+constexpr int KC = 32;  // keys per chunk
+
+template <int D>
+__global__ void __launch_bounds__(256) k_probe_attn(const __nv_bfloat16* __restrict__ Q,
+                                                   const __nv_bfloat16* __restrict__ K,
+                                                   const __nv_bfloat16* __restrict__ V, int N, int Gk, int Gq,
+                                                   int P, const int* __restrict__ probe_idx,
+                                                   const int* __restrict__ probe_grp,
+                                                   const int* __restrict__ label_k,
+                                                   const unsigned char* __restrict__ route, int keys_per_split,
+                                                   float scale_log2, float* __restrict__ part_o,
+                                                   float* __restrict__ part_ml) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* qs = reinterpret_cast<float*>(smem);      // [PR][D]
+  float* ks = qs + PR * D;                          // [D][KC]
+  float* vs = ks + D * KC;                          // [KC][D]
+  float* pd = vs + KC * D;                          // [PR][KC+1]
+  float* ps = pd + PR * (KC + 1);                   // [PR][KC+1]
+  float* st = ps + PR * (KC + 1);                   // [PR][8]: m_d l_d a_d m_s l_s a_s
+  int* klab = reinterpret_cast<int*>(st + PR * 8);  // [KC]
+  unsigned char* rt = reinterpret_cast<unsigned char*>(klab + KC);  // [PR][Gk]
+  const int split = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t head = (size_t)bh * N;
+  for (int e = tid; e < PR * D; e += 256) {
+    int r = e / D, c = e - r * D;
+    int row = r < P ? probe_idx[(size_t)bh * P + r] : -1;
+    qs[e] = row >= 0 ? bf2f(Q[(head + row) * D + c]) : 0.f;
+  }
+  for (int e = tid; e < PR * Gk; e += 256) {
+    int r = e / Gk, g = e - r * Gk;
+    int a = r < P ? probe_grp[(size_t)bh * P + r] : -1;
+    rt[e] = a >= 0 ? route[((size_t)bh * Gq + a) * Gk + g] : 0;
+  }
+  for (int r = tid; r < PR; r += 256) {
+    st[r * 8 + 0] = -INFINITY; st[r * 8 + 1] = 0.f;
+    st[r * 8 + 3] = -INFINITY; st[r * 8 + 4] = 0.f;
+  }
+  const int orow = tid >> 2;       // output row owned in the PV stage
+  const int ocol = tid & 3;        // columns ocol + 4 m
+  float od[D / 4], os[D / 4];
+#pragma unroll
+  for (int m = 0; m < D / 4; ++m) od[m] = os[m] = 0.f;
+  const int k0 = split * keys_per_split, k1 = min(N, k0 + keys_per_split);
+  __syncthreads();
+  for (int kc = k0; kc < k1; kc += KC) {
+    const int nk = min(KC, k1 - kc);
+    for (int e = tid; e < KC * D; e += 256) {
+      int j = e / D, c = e - j * D;
+      bool ok = j < nk;
+      ks[c * KC + j] = ok ? bf2f(K[(head + kc + j) * D + c]) : 0.f;
+      vs[j * D + c] = ok ? bf2f(V[(head + kc + j) * D + c]) : 0.f;
+    }
+    if (tid < KC) klab[tid] = tid < nk ? label_k[head + kc + tid] : -1;
+    __syncthreads();
+    // scores: warp w owns rows w + 8 i, lane = key
+    for (int i = 0; i < PR / 8; ++i) {
+      const int r = warp + 8 * i;
+      float sc = 0.f;
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) sc = fmaf(qs[r * D + c], ks[c * KC + lane], sc);
+      const bool valid = lane < nk;
+      const int lb = klab[lane];
+      const bool routed = valid && lb >= 0 && lb < Gk && rt[r * Gk + lb];
+      const float sd = valid ? sc * scale_log2 : -INFINITY;
+      const float ss = routed ? sc * scale_log2 : -INFINITY;
+      // dense
+      float mo = st[r * 8 + 0];
+      float mn = fmaxf(mo, warp_max(sd));
+      float p = valid ? ex2f(sd - mn) : 0.f;
+      float al = (mo == -INFINITY) ? 0.f : ex2f(mo - mn);
+      float sum = warp_sum(p);
+      pd[r * (KC + 1) + lane] = p;
+      // routed
+      float mos = st[r * 8 + 3];
+      float mns = fmaxf(mos, warp_max(ss));
+      float q = (routed && mns != -INFINITY) ? ex2f(ss - mns) : 0.f;
+      float als = (mos == -INFINITY) ? 0.f : ex2f(mos - mns);
+      float sums = warp_sum(q);
+      ps[r * (KC + 1) + lane] = q;
+      __syncwarp();
+      if (lane == 0) {
+        st[r * 8 + 0] = mn; st[r * 8 + 1] = st[r * 8 + 1] * al + sum; st[r * 8 + 2] = al;
+        st[r * 8 + 3] = mns; st[r * 8 + 4] = st[r * 8 + 4] * als + sums; st[r * 8 + 5] = als;
+      }
+    }
+    __syncthreads();
+    {
+      const float ad = st[orow * 8 + 2], as_ = st[orow * 8 + 5];
+#pragma unroll
+      for (int m = 0; m < D / 4; ++m) { od[m] *= ad; os[m] *= as_; }
+      for (int j = 0; j < nk; ++j) {
+        const float a1 = pd[orow * (KC + 1) + j], a2 = ps[orow * (KC + 1) + j];
+#pragma unroll
+        for (int m = 0; m < D / 4; ++m) {
+          const float v = vs[j * D + ocol + 4 * m];
+          od[m] = fmaf(a1, v, od[m]);
+          os[m] = fmaf(a2, v, os[m]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const size_t base = ((size_t)bh * gridDim.x + split) * PR;
+#pragma unroll
+  for (int m = 0; m < D / 4; ++m) {
+    part_o[((base + orow) * 2 + 0) * D + ocol + 4 * m] = od[m];
+    part_o[((base + orow) * 2 + 1) * D + ocol + 4 * m] = os[m];
+  }
+  if (ocol == 0) {
+    part_ml[(base + orow) * 4 + 0] = st[orow * 8 + 0];
+    part_ml[(base + orow) * 4 + 1] = st[orow * 8 + 1];
+    part_ml[(base + orow) * 4 + 2] = st[orow * 8 + 3];
+    part_ml[(base + orow) * 4 + 3] = st[orow * 8 + 4];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Merge the key splits.  grid = BH, block = 256.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_probe_combine(const float* __restrict__ part_o,
+                                                      const float* __restrict__ part_ml, int S, int P, int D,
+                                                      float* __restrict__ o_dense, float* __restrict__ o_sparse,
+                                                      float* __restrict__ lse_d, float* __restrict__ lse_s) {
+  const int bh = blockIdx.x;
+  const float LN2 = 0.69314718055994531f;
+  for (int e = threadIdx.x; e < P * D; e += blockDim.x) {
+    const int r = e / D, c = e - r * D;
+    for (int acc = 0; acc < 2; ++acc) {
+      float M = -INFINITY;
+      for (int s = 0; s < S; ++s) M = fmaxf(M, part_ml[(((size_t)bh * S + s) * PR + r) * 4 + 2 * acc]);
+      float L = 0.f, Ov = 0.f;
+      if (M != -INFINITY) {
+        for (int s = 0; s < S; ++s) {
+          const size_t rr = ((size_t)bh * S + s) * PR + r;
+          const float ms = part_ml[rr * 4 + 2 * acc];
+          if (ms == -INFINITY) continue;
+          const float w = ex2f(ms - M);
+          L += part_ml[rr * 4 + 2 * acc + 1] * w;
+          Ov += part_o[(rr * 2 + acc) * D + c] * w;
+        }
+      }
+      const float val = L > 0.f ? Ov / L : 0.f;
+      (acc == 0 ? o_dense : o_sparse)[((size_t)bh * P + r) * D + c] = val;
+      if (c == 0) {
+        float* dst = acc == 0 ? lse_d : lse_s;
+        if (dst) dst[(size_t)bh * P + r] = L > 0.f ? (M + log2f(L)) * LN2 : -INFINITY;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Residual subspace + ridge fit, one CTA per head (fp64 arithmetic).
+//   R = O_dense - O_sparse (P x D); Gram R R^T -> Jacobi -> u_i, sigma_i;
+//   v_i = R^T u_i normalised and re-orthogonalised (zero when sigma_i <= 1e-6 sigma_0);
+//   Y = R V_r; centred dual ridge  W = Xc^T (Xc Xc^T + lam I)^-1 Yc, b = ybar - xbar W.
+// grid = BH, block = 256.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_dense,
+                                                  const float* __restrict__ o_sparse, int P, int Rk,
+                                                  double lam, float* __restrict__ Vr_out,
+                                                  float* __restrict__ W_out, float* __restrict__ bfull_out,
+                                                  float* __restrict__ Bmat, float* __restrict__ sigma_out,
+                                                  float* __restrict__ bsub_out) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  constexpr int LDP = PR + 1;
+  double* G = reinterpret_cast<double*>(smem);   // [PR][LDP]  Gram, later Cholesky
+  double* U = G + PR * LDP;                       // [PR][LDP]  Jacobi vectors
+  double* Vr = U + PR * LDP;                      // [D][Rk]
+  double* Y = Vr + D * Rk;                        // [PR][Rk] -> solution
+  double* xbar = Y + PR * Rk;                     // [D]
+  double* ybar = xbar + D;                        // [64]
+  double* bsub = ybar + 64;                       // [64]
+  double* cs = bsub + 64;                         // [PR]
+  double* red = cs + PR;                          // [64]
+  float* Rm = reinterpret_cast<float*>(red + 64); // [PR][D]
+  float* Xm = Rm + PR * D;                        // [PR][D]
+  int* pr = reinterpret_cast<int*>(Xm + PR * D);  // [PR]
+  int* rank = pr + PR;                            // [PR]
+  int* ridx = rank + PR;                          // [64] eigen index of subspace column j
+  const int bh = blockIdx.x, tid = threadIdx.x;
+  const int n = (P + 1) & ~1;  // Jacobi needs an even size; a padded zero row is harmless
+  for (int e = tid; e < PR * D; e += 256) {
+    const int r = e / D;
+    float od = 0.f, os = 0.f;
+    if (r < P) {
+      od = o_dense[(size_t)bh * P * D + e];
+      os = o_sparse[(size_t)bh * P * D + e];
+    }
+    Rm[e] = od - os;
+    Xm[e] = os;
+  }
+  __syncthreads();
+  for (int e = tid; e < n * n; e += 256) {
+    const int i = e / n, j = e - i * n;
+    double s = 0.0;
+    for (int c = 0; c < D; ++c) s += (double)Rm[i * D + c] * (double)Rm[j * D + c];
+    G[i * LDP + j] = s;
+  }
+  __syncthreads();
+  jacobi_eigen<double>(G, U, n, LDP, cs, pr, red, 40, 1e-14);
+  eigen_ranks<double>(G, n, LDP, rank);
+  for (int i = tid; i < n; i += 256)
+    if (rank[i] < Rk) ridx[rank[i]] = i;
+  __syncthreads();
+  // subspace basis
+  double lam0 = 0.0;
+  for (int i = 0; i < n; ++i) lam0 = fmax(lam0, G[i * LDP + i]);
+  const double smax = sqrt(fmax(lam0, 0.0));
+  for (int j = 0; j < Rk; ++j) {
+    const int i = ridx[j];
+    const double sj = sqrt(fmax(G[i * LDP + i], 0.0));
+    const bool keep = smax > 0.0 && sj > 1e-6 * smax;
+    for (int c = tid; c < D; c += 256) {
+      double v = 0.0;
+      if (keep)
+        for (int p = 0; p < n; ++p) v += (double)Rm[p * D + c] * U[p * LDP + i];
+      Vr[c * Rk + j] = v;
+    }
+    if (tid == 0 && sigma_out) sigma_out[(size_t)bh * Rk + j] = keep ? (float)sj : 0.f;
+    __syncthreads();
+    // Gram-Schmidt against earlier columns (twice), then normalise
+    for (int pass = 0; pass < 2 && keep; ++pass) {
+      for (int k = 0; k < j; ++k) {
+        double dot = 0.0;
+        for (int c = tid; c < D; c += 256) dot += Vr[c * Rk + j] * Vr[c * Rk + k];
+        dot = warp_sum_d(dot);
+        if ((tid & 31) == 0) red[tid >> 5] = dot;
+        __syncthreads();
+        dot = 0.0;
+        for (int w = 0; w < 8; ++w) dot += red[w];
+        __syncthreads();
+        for (int c = tid; c < D; c += 256) Vr[c * Rk + j] -= dot * Vr[c * Rk + k];
+        __syncthreads();
+      }
+    }
+    if (keep) {
+      double nn = 0.0;
+      for (int c = tid; c < D; c += 256) nn += Vr[c * Rk + j] * Vr[c * Rk + j];
+      nn = warp_sum_d(nn);
+      if ((tid & 31) == 0) red[tid >> 5] = nn;
+      __syncthreads();
+      nn = 0.0;
+      for (int w = 0; w < 8; ++w) nn += red[w];
+      __syncthreads();
+      const double inv = nn > 0.0 ? 1.0 / sqrt(nn) : 0.0;
+      for (int c = tid; c < D; c += 256) Vr[c * Rk + j] *= inv;
+    }
+    __syncthreads();
+  }
+  // Y = R Vr, means
+  for (int e = tid; e < P * Rk; e += 256) {
+    const int p = e / Rk, j = e - p * Rk;
+    double s = 0.0;
+    for (int c = 0; c < D; ++c) s += (double)Rm[p * D + c] * Vr[c * Rk + j];
+    Y[p * Rk + j] = s;
+  }
+  for (int c = tid; c < D; c += 256) {
+    double s = 0.0;
+    for (int p = 0; p < P; ++p) s += (double)Xm[p * D + c];
+    xbar[c] = s / P;
+  }
+  __syncthreads();
+  for (int j = tid; j < Rk; j += 256) {
+    double s = 0.0;
+    for (int p = 0; p < P; ++p) s += Y[p * Rk + j];
+    ybar[j] = s / P;
+  }
+  __syncthreads();
+  for (int e = tid; e < P * Rk; e += 256) {
+    const int p = e / Rk, j = e - p * Rk;
+    Y[p * Rk + j] -= ybar[j];
+  }
+  // A = Xc Xc^T + lam I  (into G)
+  for (int e = tid; e < P * P; e += 256) {
+    const int i = e / P, j = e - i * P;
+    double s = 0.0;
+    for (int c = 0; c < D; ++c) s += ((double)Xm[i * D + c] - xbar[c]) * ((double)Xm[j * D + c] - xbar[c]);
+    G[i * LDP + j] = s + (i == j ? lam : 0.0);
+  }
+  __syncthreads();
+  // Cholesky A = L L^T (lower triangle of G)
+  for (int k = 0; k < P; ++k) {
+    if (tid == 0) G[k * LDP + k] = sqrt(G[k * LDP + k]);
+    __syncthreads();
+    const double dkk = G[k * LDP + k];
+    for (int i = k + 1 + tid; i < P; i += 256) G[i * LDP + k] /= dkk;
+    __syncthreads();
+    for (int e = tid; e < (P - k - 1) * (P - k - 1); e += 256) {
+      const int i = k + 1 + e / (P - k - 1), j = k + 1 + e % (P - k - 1);
+      if (j <= i) G[i * LDP + j] -= G[i * LDP + k] * G[j * LDP + k];
+    }
+    __syncthreads();
+  }
+  // solve L L^T Z = Yc, one right-hand side per thread
+  for (int j = tid; j < Rk; j += 256) {
+    for (int i = 0; i < P; ++i) {
+      double s = Y[i * Rk + j];
+      for (int k = 0; k < i; ++k) s -= G[i * LDP + k] * Y[k * Rk + j];
+      Y[i * Rk + j] = s / G[i * LDP + i];
+    }
+    for (int i = P - 1; i >= 0; --i) {
+      double s = Y[i * Rk + j];
+      for (int k = i + 1; k < P; ++k) s -= G[k * LDP + i] * Y[k * Rk + j];
+      Y[i * Rk + j] = s / G[i * LDP + i];
+    }
+  }
+  __syncthreads();
+  // W = Xc^T Z (D x Rk) kept in the Jacobi-vector region, b = ybar - xbar W
+  double* Wd = U;
+  for (int e = tid; e < D * Rk; e += 256) {
+    const int c = e / Rk, j = e - c * Rk;
+    double s = 0.0;
+    for (int p = 0; p < P; ++p) s += ((double)Xm[p * D + c] - xbar[c]) * Y[p * Rk + j];
+    Wd[e] = s;
+    W_out[(size_t)bh * D * Rk + e] = (float)s;
+    Vr_out[(size_t)bh * D * Rk + e] = (float)Vr[c * Rk + j];
+  }
+  __syncthreads();
+  for (int j = tid; j < Rk; j += 256) {
+    double s = 0.0;
+    for (int c = 0; c < D; ++c) s += xbar[c] * Wd[c * Rk + j];
+    bsub[j] = ybar[j] - s;
+    if (bsub_out) bsub_out[(size_t)bh * Rk + j] = (float)bsub[j];
+  }
+  __syncthreads();
+  for (int c = tid; c < D; c += 256) {
+    double s = 0.0;
+    for (int j = 0; j < Rk; ++j) s += Vr[c * Rk + j] * bsub[j];
+    bfull_out[(size_t)bh * D + c] = (float)s;
+  }
+  if (Bmat) {
+    for (int e = tid; e < D * D; e += 256) {
+      const int r = e / D, c = e - r * D;
+      double s = 0.0;
+      for (int j = 0; j < Rk; ++j) s += Wd[r * Rk + j] * Vr[c * Rk + j];
+      Bmat[(size_t)bh * D * D + e] = (float)s;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Correction O = x + b_full + (x W) V_r^T for every row (probe rows are then
+// overwritten by k_probe_scatter).  grid = (ceil(N/64), BH), block = 256.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) k_reconstruct(const __nv_bfloat16* __restrict__ Os, int N, int Rk,
+                                                    const float* __restrict__ W, const float* __restrict__ Vr,
+                                                    const float* __restrict__ bfull, __nv_bfloat16* __restrict__ O) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* xs = reinterpret_cast<float*>(smem);  // [64][D+1]
+  float* ws = xs + 64 * (D + 1);               // [D][Rk]
+  float* vt = ws + D * Rk;                     // [Rk][D]  (V_r transposed)
+  float* ts = vt + Rk * D;                     // [64][Rk+1]
+  float* bf = ts + 64 * (Rk + 1);              // [D]
+  const int bh = blockIdx.y, n0 = blockIdx.x * 64, tid = threadIdx.x;
+  const int nr = min(64, N - n0);
+  for (int e = tid; e < D * Rk; e += 256) {
+    ws[e] = W[(size_t)bh * D * Rk + e];
+    const int c = e / Rk, j = e - c * Rk;
+    vt[j * D + c] = Vr[(size_t)bh * D * Rk + e];
+  }
+  for (int c = tid; c < D; c += 256) bf[c] = bfull[(size_t)bh * D + c];
+  const __nv_bfloat16* src = Os + ((size_t)bh * N + n0) * D;
+  for (int e = tid; e < nr * D; e += 256) {
+    const int r = e / D, c = e - r * D;
+    xs[r * (D + 1) + c] = bf2f(src[e]);
+  }
+  __syncthreads();
+  for (int e = tid; e < nr * Rk; e += 256) {
+    const int r = e / Rk, j = e - r * Rk;
+    float t = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < D; ++c) t = fmaf(xs[r * (D + 1) + c], ws[c * Rk + j], t);
+    ts[r * (Rk + 1) + j] = t;
+  }
+  __syncthreads();
+  __nv_bfloat16* dst = O + ((size_t)bh * N + n0) * D;
+  for (int e = tid; e < nr * D; e += 256) {
+    const int r = e / D, c = e - r * D;
+    float o = xs[r * (D + 1) + c] + bf[c];
+    for (int j = 0; j < Rk; ++j) o = fmaf(ts[r * (Rk + 1) + j], vt[j * D + c], o);
+    dst[e] = __float2bfloat16(o);
+  }
+}
+
+__global__ void k_probe_scatter(const int* __restrict__ probe_idx, const float* __restrict__ o_dense, int N, int P,
+                                int D, __nv_bfloat16* __restrict__ O) {
+  const int bh = blockIdx.x;
+  for (int e = threadIdx.x; e < P * D; e += blockDim.x) {
+    const int p = e / D, c = e - p * D;
+    const int row = probe_idx[(size_t)bh * P + p];
+    if (row >= 0 && row < N) O[((size_t)bh * N + row) * D + c] = __float2bfloat16(o_dense[(size_t)bh * P * D + e]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Route lists and q-tile work list.  grid = BH, block = 256 (one warp per group).
+//   rlist[a][i] = i-th routed non-empty K/V group of query group a (ascending g)
+//   rcum[a][i]  = key rows before it, rcum[a][cnt] = total routed rows
+//   tiles       = (a, t) for every 128-row tile of every non-empty query group
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_worklist(const unsigned char* __restrict__ route,
+                                                 const int* __restrict__ qoff, const int* __restrict__ koff,
+                                                 int Gq, int Gk, int tile_rows, int max_tiles,
+                                                 int* __restrict__ rlist, int* __restrict__ rcum,
+                                                 int* __restrict__ rcnt, int2* __restrict__ tiles,
+                                                 int* __restrict__ tile_count) {
+  const int bh = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int* ko = koff + (size_t)bh * (Gk + 1);
+  for (int a = warp; a < Gq; a += 8) {
+    const unsigned char* rr = route + ((size_t)bh * Gq + a) * Gk;
+    int* rl = rlist + ((size_t)bh * Gq + a) * Gk;
+    int* rc = rcum + ((size_t)bh * Gq + a) * (Gk + 1);
+    int cnt = 0, cum = 0;
+    for (int g0 = 0; g0 < Gk; g0 += 32) {
+      const int g = g0 + lane;
+      const int sz = g < Gk ? ko[g + 1] - ko[g] : 0;
+      const bool on = g < Gk && rr[g] && sz > 0;
+      const unsigned m = __ballot_sync(0xffffffffu, on);
+      // exclusive prefix of sizes over the lanes that are on
+      int v = on ? sz : 0, incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      if (on) {
+        const int pos = cnt + __popc(m & ((1u << lane) - 1));
+        rl[pos] = g;
+        rc[pos] = cum + incl - v;
+      }
+      cnt += __popc(m);
+      cum += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      rc[cnt] = cum;
+      rcnt[(size_t)bh * Gq + a] = cnt;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int* qo = qoff + (size_t)bh * (Gq + 1);
+    int t = 0;
+    for (int a = 0; a < Gq; ++a) {
+      const int nt = (qo[a + 1] - qo[a] + tile_rows - 1) / tile_rows;
+      for (int k = 0; k < nt && t < max_tiles; ++k) tiles[(size_t)bh * max_tiles + t++] = make_int2(a, k);
+    }
+    tile_count[bh] = t;
+  }
+}
+
+// ---------------------------------------------------------------------------
+cudaError_t launch_worklist(const unsigned char* route, const int* qoff, const int* koff, int BH, int Gq, int Gk,
+                           int tile_rows, int max_tiles, int* rlist, int* rcum, int* rcnt, int2* tiles,
+                           int* tile_count, cudaStream_t st) {
+  k_worklist<<<BH, 256, 0, st>>>(route, qoff, koff, Gq, Gk, tile_rows, max_tiles, rlist, rcum, rcnt, tiles,
+                                 tile_count);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_probe_pick(const int* perm_q, const int* qoff, int BH, int N, int Gq, int P, uint64_t seed,
+                              int* probe_idx, int* probe_grp, int* err, cudaStream_t st) {
+  size_t sm = (size_t)(3 * Gq + 64 + 512 + 8) * 4;
+  cudaFuncSetAttribute(k_probe_pick, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  k_probe_pick<<<BH, 256, sm, st>>>(perm_q, qoff, N, Gq, P, seed, probe_idx, probe_grp, err);
+  return cudaGetLastError();
+}
+
+int probe_splits(int N) {
+  int s = (N + 2047) / 2048;
+  return s < 1 ? 1 : (s > 64 ? 64 : s);
+}
+
+size_t probe_attn_smem(int D, int Gk) {
+  return (size_t)(PR * D + D * KC + KC * D + 2 * PR * (KC + 1) + PR * 8 + KC) * 4 + (size_t)PR * Gk;
+}
+
+cudaError_t launch_probe_attn(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk, int Gq,
+                              int P, const int* probe_idx, const int* probe_grp, const int* label_k,
+                              const unsigned char* route, float scale_log2, float* part_o, float* part_ml,
+                              cudaStream_t st) {
+  const int S = probe_splits(N);
+  int kps = (N + S - 1) / S;
+  kps = (kps + KC - 1) / KC * KC;
+  const size_t sm = probe_attn_smem(D, Gk);
+  dim3 grid(S, BH);
+  if (D == 64) {
+    cudaFuncSetAttribute(k_probe_attn<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_probe_attn<64><<<grid, 256, sm, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
+                                            (const __nv_bfloat16*)V, N, Gk, Gq, P, probe_idx, probe_grp,
+                                            label_k, route, kps, scale_log2, part_o, part_ml);
+  } else {
+    cudaFuncSetAttribute(k_probe_attn<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_probe_attn<128><<<grid, 256, sm, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
+                                             (const __nv_bfloat16*)V, N, Gk, Gq, P, probe_idx, probe_grp,
+                                             label_k, route, kps, scale_log2, part_o, part_ml);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_probe_combine(const float* part_o, const float* part_ml, int BH, int N, int P, int D,
+                                 float* o_dense, float* o_sparse, float* lse_d, float* lse_s, cudaStream_t st) {
+  k_probe_combine<<<BH, 256, 0, st>>>(part_o, part_ml, probe_splits(N), P, D, o_dense, o_sparse, lse_d, lse_s);
+  return cudaGetLastError();
+}
+
+size_t probe_fit_smem(int D, int Rk) {
+  return (size_t)(2 * PR * (PR + 1) + D * Rk + PR * Rk + D + 64 + 64 + PR + 64) * 8 + (size_t)2 * PR * D * 4 +
+         (size_t)(2 * PR + 64) * 4;
+}
+
+cudaError_t launch_probe_fit(const float* o_dense, const float* o_sparse, int BH, int D, int P, int Rk,
+                             double lam, float* Vr, float* W, float* bfull, float* Bmat, float* sigma,
+                             float* bsub, cudaStream_t st) {
+  const size_t sm = probe_fit_smem(D, Rk);
+  if (D == 64) {
+    cudaFuncSetAttribute(k_probe_fit<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_probe_fit<64><<<BH, 256, sm, st>>>(o_dense, o_sparse, P, Rk, lam, Vr, W, bfull, Bmat, sigma, bsub);
+  } else {
+    cudaFuncSetAttribute(k_probe_fit<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_probe_fit<128><<<BH, 256, sm, st>>>(o_dense, o_sparse, P, Rk, lam, Vr, W, bfull, Bmat, sigma, bsub);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reconstruct(const void* Os, int BH, int N, int D, int Rk, const float* W, const float* Vr,
+                               const float* bfull, void* O, cudaStream_t st) {
+  const size_t sm = (size_t)(64 * (D + 1) + 2 * D * Rk + 64 * (Rk + 1) + D) * 4;
+  dim3 grid(ceil_div(N, 64), BH);
+  if (D == 64) {
+    cudaFuncSetAttribute(k_reconstruct<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_reconstruct<64><<<grid, 256, sm, st>>>((const __nv_bfloat16*)Os, N, Rk, W, Vr, bfull, (__nv_bfloat16*)O);
+  } else {
+    cudaFuncSetAttribute(k_reconstruct<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_reconstruct<128><<<grid, 256, sm, st>>>((const __nv_bfloat16*)Os, N, Rk, W, Vr, bfull, (__nv_bfloat16*)O);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_probe_scatter(const int* probe_idx, const float* o_dense, int BH, int N, int P, int D, void* O,
+                                 cudaStream_t st) {
+  k_probe_scatter<<<BH, 256, 0, st>>>(probe_idx, o_dense, N, P, D, (__nv_bfloat16*)O);
+  return cudaGetLastError();
+}
+
+}  // namespace spr

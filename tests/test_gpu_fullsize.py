@@ -1,0 +1,53 @@
+"""Parity at the full 32,760-token, 40-head, d=128 workload in the configuration the
+benchmark times: every integer output of two heads bit-exact (labels with the
+near-tie exemption, teacher-forced per Lloyd step), attention and reconstruction
+on 512 sampled rows per head, probes and fit in full; property checks on all heads."""
+import numpy as np
+import pytest
+
+from synth import generate, workload
+
+from helpers import params_dict
+from test_gpu_parity import _np, _run, stage_checks
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def wan_run(gpu):
+    w = workload("wan")
+    pd = params_dict(w)
+    qb, kb, vb = generate(w, seed=0)
+    p, out = _run(pd, qb, kb, vb, gpu)
+    return w, pd, (qb, kb, vb), out
+
+
+def test_fullsize_sampled_heads(wan_run):
+    w, pd, (qb, kb, vb), out = wan_run
+    stage_checks(pd, qb, kb, vb, out, [0, w.H - 1], rows=512)
+
+
+def test_fullsize_properties_all_heads(wan_run):
+    w, pd, _, out = wan_run
+    N, Gq, Gk = w.N, w.n_qgroups, w.n_kgroups
+    rho = _np(out["rho_exec"])
+    assert np.all(rho <= w.density + 1e-6) and np.all(rho > 0.5 * w.density)
+    for bh in range(w.B * w.H):
+        pq = _np(out["perm_q"][bh])
+        pk = _np(out["perm_k"][bh])
+        lq = _np(out["label_q"][bh])
+        lk = _np(out["label_k"][bh])
+        qo = _np(out["qoff"][bh])
+        ko = _np(out["koff"][bh])
+        assert np.array_equal(np.sort(pq), np.arange(N)) and np.array_equal(np.sort(pk), np.arange(N))
+        assert np.all(np.diff(lq[pq]) >= 0) and np.all(np.diff(lk[pk]) >= 0)
+        assert qo[-1] == N and ko[-1] == N
+        route = _np(out["route"][bh])
+        nq = np.diff(qo)
+        assert np.all((route.sum(axis=1) > 0) == (nq > 0))
+        cost = (np.outer(nq, np.diff(ko)) * route).sum()
+        assert abs((cost + w.n_probes * N) / N ** 2 - rho[bh]) < 1e-6
+        pidx = _np(out["probe_idx"][bh])
+        assert len(set(pidx.tolist())) == w.n_probes
+    o = out["o"].float()
+    assert bool(o.isfinite().all())
