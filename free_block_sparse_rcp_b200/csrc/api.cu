@@ -43,6 +43,7 @@ sparsepr_status fail_cuda(cudaError_t e, const char* where) {
 
 constexpr size_t kSmemLimit = 227 * 1024;
 
+
 size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct Layout {
@@ -155,7 +156,7 @@ sparsepr_status check_params(const sparsepr_params* p) {
     return fail(SPARSEPR_EUNSUPPORTED, "key centroid table exceeds shared memory");
   if ((size_t)p->d * p->sub_rank > 64 * 65 || probe_fit_smem(p->d, p->sub_rank) > kSmemLimit)
     return failv(SPARSEPR_EUNSUPPORTED, "sub_rank too large for the single-CTA fit (d*r)", (long long)p->d * p->sub_rank);
-  if (attn_smem_bytes(p->d, p->n_kgroups) > kSmemLimit || probe_attn_smem(p->d, p->n_kgroups) > kSmemLimit)
+  if (attn_tc_smem_bytes(p->d, p->n_kgroups) > kSmemLimit || probe_attn_smem(p->d, p->n_kgroups) > kSmemLimit)
     return fail(SPARSEPR_EUNSUPPORTED, "too many K/V groups for the attention kernels");
   return SPARSEPR_OK;
 }
@@ -268,7 +269,7 @@ sparsepr_status run_attend(const sparsepr_params& p, const Layout& L, const void
   a.max_tiles = L.max_tiles;
   a.scale_log2 = eff_scale(p) * 1.4426950408889634f;
   a.O = O; a.lse = lse; a.err = at<int>(ws, L.err);
-  SPR_LAUNCH(launch_attention(a, false, st));
+  SPR_LAUNCH(launch_attention_tc(a, false, st));
   return SPARSEPR_OK;
 }
 
@@ -446,7 +447,7 @@ sparsepr_status sparsepr_dense_attention(const sparsepr_params* p, const void* Q
   a.BH = p->B * p->H; a.N = p->N; a.D = p->d;
   a.scale_log2 = eff_scale(*p) * 1.4426950408889634f;
   a.O = O; a.lse = lse; a.err = err;
-  SPR_LAUNCH(launch_attention(a, true, (cudaStream_t)stream));
+  SPR_LAUNCH(launch_attention_tc(a, true, (cudaStream_t)stream));
   return SPARSEPR_OK;
 }
 

@@ -80,8 +80,8 @@ struct AttnArgs {
   float* lse;
   int* err;
 };
-size_t attn_smem_bytes(int D, int Gk);
-cudaError_t launch_attention(const AttnArgs& a, bool dense, cudaStream_t st);
+size_t attn_tc_smem_bytes(int D, int Gk);
+cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, cudaStream_t st);
 constexpr int kAttnTileRows = 128;
 
 }  // namespace spr
