@@ -16,7 +16,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsparsepr.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m free_block_sparse_rcp_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python free_block_sparse_rcp_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
 _vp = ctypes.c_void_p
@@ -78,6 +78,8 @@ _sig = {
                                        ctypes.c_size_t, _vp]),
     "sparsepr_probe_fit": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                           _vp, ctypes.POINTER(ProbeTrace), _vp, ctypes.c_size_t, _vp]),
+    "sparsepr_probe_fit_noalloc": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                                  _vp, _vp, _vp]),
     "sparsepr_reconstruct": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "sparsepr_forward": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "sparsepr_forward_host": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
@@ -176,6 +178,14 @@ def sparsepr_probe_fit(p, Q, K, V, label_k, perm_q, qoff, route, probe_idx, prob
                                    _ptr(qoff), _ptr(route), _ptr(probe_idx), _ptr(probe_o_dense),
                                    _ptr(b_full), _ptr(Vr), _ptr(W), _ptr(Bmat), _trace(ProbeTrace, trace),
                                    _ptr(ws), ws.numel(), _stream(Q)), "sparsepr_probe_fit")
+
+
+def sparsepr_probe_fit_noalloc(p, Q, K, V, label_k, perm_q, qoff, route, probe_idx, probe_o_dense, b_full,
+                               Vr, W, Bmat):
+    _check(_lib.sparsepr_probe_fit_noalloc(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(label_k),
+                                           _ptr(perm_q), _ptr(qoff), _ptr(route), _ptr(probe_idx),
+                                           _ptr(probe_o_dense), _ptr(b_full), _ptr(Vr), _ptr(W), _ptr(Bmat),
+                                           _stream(Q)), "sparsepr_probe_fit_noalloc")
 
 
 def sparsepr_reconstruct(p, O_sparse, probe_idx, probe_o_dense, b_full, Vr, W, O):

@@ -312,6 +312,11 @@ sparsepr_status run_reconstruct(const sparsepr_params& p, int BH, const void* Os
 
 }  // namespace
 
+namespace spr {
+void set_last_error(const char* msg) { snprintf(g_detail, sizeof(g_detail), "%s", msg); }
+void set_launch_count(int n) { g_launches = n; }
+}  // namespace spr
+
 // ===========================================================================
 extern "C" {
 

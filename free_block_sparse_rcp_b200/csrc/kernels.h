@@ -49,6 +49,13 @@ cudaError_t launch_probe_attn(const void* Q, const void* K, const void* V, int B
                               int P, const int* probe_idx, const int* probe_grp, const int* label_k,
                               const unsigned char* route, float scale_log2, float* part_o, float* part_ml,
                               cudaStream_t st);
+cudaError_t launch_probe_attn_splits(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk,
+                                     int Gq, int P, const int* probe_idx, const int* probe_grp, const int* label_k,
+                                     const unsigned char* route, float scale_log2, int S, float* part_o,
+                                     float* part_ml, cudaStream_t st);
+cudaError_t launch_probe_combine_splits(const float* part_o, const float* part_ml, int BH, int S, int P, int D,
+                                        float* o_dense, float* o_sparse, float* lse_d, float* lse_s,
+                                        cudaStream_t st);
 cudaError_t launch_probe_combine(const float* part_o, const float* part_ml, int BH, int N, int P, int D,
                                  float* o_dense, float* o_sparse, float* lse_d, float* lse_s, cudaStream_t st);
 cudaError_t launch_probe_fit(const float* o_dense, const float* o_sparse, int BH, int D, int P, int Rk,
@@ -83,5 +90,10 @@ struct AttnArgs {
 size_t attn_tc_smem_bytes(int D, int Gk);
 cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, cudaStream_t st);
 constexpr int kAttnTileRows = 128;
+constexpr int kProbeRowsPerCta = 64;  // probe rows per CTA of k_probe_attn (its PR)
+
+// api.cu: per-thread error detail and launch count of the last call
+void set_last_error(const char* msg);
+void set_launch_count(int n);
 
 }  // namespace spr

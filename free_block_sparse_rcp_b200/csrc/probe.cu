@@ -584,6 +584,37 @@ cudaError_t launch_probe_attn(const void* Q, const void* K, const void* V, int B
   return cudaGetLastError();
 }
 
+// Split-count-explicit variants (the key-split count S is chosen by the caller instead
+// of probe_splits(N)); used by the entry point whose scratch has a fixed size.
+cudaError_t launch_probe_attn_splits(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk,
+                                     int Gq, int P, const int* probe_idx, const int* probe_grp, const int* label_k,
+                                     const unsigned char* route, float scale_log2, int S, float* part_o,
+                                     float* part_ml, cudaStream_t st) {
+  int kps = (N + S - 1) / S;
+  kps = (kps + KC - 1) / KC * KC;
+  const size_t sm = probe_attn_smem(D, Gk);
+  dim3 grid(S, BH);
+  if (D == 64) {
+    cudaFuncSetAttribute(k_probe_attn<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_probe_attn<64><<<grid, 256, sm, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
+                                            (const __nv_bfloat16*)V, N, Gk, Gq, P, probe_idx, probe_grp,
+                                            label_k, route, kps, scale_log2, part_o, part_ml);
+  } else {
+    cudaFuncSetAttribute(k_probe_attn<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_probe_attn<128><<<grid, 256, sm, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
+                                             (const __nv_bfloat16*)V, N, Gk, Gq, P, probe_idx, probe_grp,
+                                             label_k, route, kps, scale_log2, part_o, part_ml);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_probe_combine_splits(const float* part_o, const float* part_ml, int BH, int S, int P, int D,
+                                        float* o_dense, float* o_sparse, float* lse_d, float* lse_s,
+                                        cudaStream_t st) {
+  k_probe_combine<<<BH, 256, 0, st>>>(part_o, part_ml, S, P, D, o_dense, o_sparse, lse_d, lse_s);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_probe_combine(const float* part_o, const float* part_ml, int BH, int N, int P, int D,
                                  float* o_dense, float* o_sparse, float* lse_d, float* lse_s, cudaStream_t st) {
   k_probe_combine<<<BH, 256, 0, st>>>(part_o, part_ml, probe_splits(N), P, D, o_dense, o_sparse, lse_d, lse_s);

@@ -164,6 +164,29 @@ SPARSEPR_API sparsepr_status sparsepr_probe_fit(const sparsepr_params* p, const 
                                    const sparsepr_probe_trace* trace,
                                    void* workspace, size_t ws_bytes, void* stream);
 
+/* sparsepr_probe_fit without a workspace: allocates nothing and uses no caller scratch.
+ * The paper has no counterpart; this variant exists for callers that cannot call
+ * cudaMalloc (runtimes that fix their device memory plan at start-up and forbid later
+ * allocation, or host code where an allocation, which can synchronize the device, is not
+ * allowed).  Arguments and outputs are those of sparsepr_probe_fit minus the trace and the
+ * workspace; results agree with it up to floating-point summation order.
+ * Scratch: a 16 MiB device array owned by the library, present on every GPU that loads
+ * it until the process exits.  The key-split count shrinks to fit it; a problem whose
+ * per-call buffers (about B*H*n_probes*(8*d + 16) bytes plus one split) exceed it returns
+ * SPARSEPR_EUNSUPPORTED before any work is enqueued.  The first call on a device looks up
+ * the array's device address (cudaGetSymbolAddress, with that device current); make that
+ * first call before any stream capture.  All calls share the one array and it keeps the
+ * previous call's contents (every byte is rewritten before it is read): calls that overlap
+ * on the GPU, on other streams or from other host threads, race and must be serialized by
+ * the caller.  Device-side index checks of this variant are not reported.               */
+SPARSEPR_API sparsepr_status sparsepr_probe_fit_noalloc(const sparsepr_params* p, const void* Q,
+                                                        const void* K, const void* V,
+                                                        const int* label_k, const int* perm_q,
+                                                        const int* qoff, const unsigned char* route,
+                                                        int* probe_idx, float* probe_o_dense,
+                                                        float* b_full, float* Vr, float* W,
+                                                        float* Bmat, void* stream);
+
 /* Correction of every unprobed row and restoration of the probe rows (gist.science 2.B):
  *   O(q) = x + b_full + (x W) V_r^T   with x = O_sparse(q), for q not a probe;
  *   O(q) = probe_o_dense              for probe rows.
