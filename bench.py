@@ -142,7 +142,7 @@ def run_cuda(args):
     import free_block_sparse_rcp_b200 as spr
     from synth import generate, workload
 
-    w = workload(WORKLOAD)
+    w = workload(WORKLOAD, H=args.heads) if args.heads else workload(WORKLOAD)
     pd = dict(B=w.B, H=w.H, N=w.N, d=w.d, block=w.block, density=w.density, n_kgroups=w.n_kgroups,
               n_qgroups=w.n_qgroups, n_samples=w.n_samples, n_probes=w.n_probes, eig_rank=w.eig_rank,
               sub_rank=w.sub_rank, kmeans_iters=w.kmeans_iters, ridge_lambda=w.ridge_lambda, seed=0)
@@ -297,7 +297,7 @@ def run_cuda(args):
         "gpu_launches": launches[0],
         "clocks": clk.summary(),
     }
-    if rank == 0 and ws == 1:
+    if rank == 0 and ws == 1 and not args.heads:
         line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
     if ws > 1:
         import torch.distributed as dist
@@ -403,6 +403,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=30.0)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (small cases for ncu captures; default: the workload's 40)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

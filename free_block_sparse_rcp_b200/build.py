@@ -1,6 +1,6 @@
 """Build libsparsepr.so (sm_100a) in-tree with nvcc.
 
-    python -m free_block_sparse_rcp_b200.build [--verbose]
+    python free_block_sparse_rcp_b200/build.py [--verbose] [--force] [--ptxas]
 
 Every .cu file under csrc/ is compiled with -gencode arch=compute_100a,code=sm_100a
 and linked into free_block_sparse_rcp_b200/libsparsepr.so.  Rebuilds only when a
