@@ -50,8 +50,8 @@ struct Layout {
   // header
   size_t err;
   // partition
-  size_t sample_idx, metric, eigval, eigvec, proj, Y, cent_k, key_init, C, Z, cent_q, query_init, mass,
-      order, cm, cc, alpha;
+  size_t sample_idx, metric, eigval, eigvec, proj, m_k, nu_k, key_init, C, Z, m_q, nu_q, query_init, bias, wnorm,
+      w_hi, w_lo, flag_count, flag_rows, mass, order, cm, cc, alpha;
   // attend
   size_t rlist, rcum, rcnt, tiles, tile_count;
   // probe
@@ -82,13 +82,21 @@ Layout make_layout(const sparsepr_params& p) {
   L.eigval = take(BH * re * 4);
   L.eigvec = take(BH * d * re * 4);
   L.proj = take(BH * d * re * 4);
-  L.Y = take(BH * N * re * 4);
-  L.cent_k = take(BH * Gk * L.DTk * 4);
+  const size_t GPmax = (size_t)kmeans_gp(p.n_kgroups > p.n_qgroups ? p.n_kgroups : p.n_qgroups);
+  L.m_k = take(BH * Gk * d * 4);
+  L.nu_k = take(BH * Gk * L.DTk * 4);
   L.key_init = take(BH * Gk * 4);
   L.C = take(BH * Gk * d * 4);
   L.Z = take(BH * N * Gk * 4);
-  L.cent_q = take(BH * Gq * L.DTq * 4);
+  L.m_q = take(BH * Gq * d * 4);
+  L.nu_q = take(BH * Gq * L.DTq * 4);
   L.query_init = take(BH * Gq * 4);
+  L.bias = take(BH * GPmax * 4);
+  L.wnorm = take(BH * GPmax * 4);
+  L.w_hi = take(BH * GPmax * d * 2);
+  L.w_lo = take(BH * GPmax * d * 2);
+  L.flag_count = take(BH * 4);
+  L.flag_rows = take(BH * N * 4);
   L.mass = take(BH * Gq * Gk * 4);
   L.order = take(BH * Gq * Gk * 4);
   L.cm = take(BH * Gq * Gk * 8);
@@ -150,10 +158,7 @@ sparsepr_status check_params(const sparsepr_params* p) {
     return fail(SPARSEPR_EINVAL, "density is below the probe floor n_probes/N");
   // kernel limits
   if (p->n_kgroups > 128) return fail(SPARSEPR_EUNSUPPORTED, "n_kgroups > 128 (query coordinates wider than 128) not built");
-  if ((size_t)p->n_qgroups * kmeans_dt(p->n_kgroups) * 4 > kSmemLimit)
-    return fail(SPARSEPR_EUNSUPPORTED, "query centroid table exceeds shared memory");
-  if ((size_t)p->n_kgroups * kmeans_dt(p->eig_rank) * 4 > kSmemLimit)
-    return fail(SPARSEPR_EUNSUPPORTED, "key centroid table exceeds shared memory");
+  if (p->n_qgroups > 128) return fail(SPARSEPR_EUNSUPPORTED, "n_qgroups > 128 not built");
   if ((size_t)p->d * p->sub_rank > 64 * 65 || probe_fit_smem(p->d, p->sub_rank) > kSmemLimit)
     return failv(SPARSEPR_EUNSUPPORTED, "sub_rank too large for the single-CTA fit (d*r)", (long long)p->d * p->sub_rank);
   if (attn_tc_smem_bytes(p->d, p->n_kgroups) > kSmemLimit || probe_attn_smem(p->d, p->n_kgroups) > kSmemLimit)
@@ -192,38 +197,52 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
                               unsigned char* bmask, float* rho, const sparsepr_partition_trace* tr, void* ws,
                               cudaStream_t st) {
   const int BH = L.BH, N = p.N, d = p.d, Gk = p.n_kgroups, Gq = p.n_qgroups, re = p.eig_rank;
+  const float scale = eff_scale(p);
   int* err = at<int>(ws, L.err);
   SPR_CUDA(cudaMemsetAsync(err, 0, 4, st));
   float* metric = at<float>(ws, L.metric);
+  float* proj = at<float>(ws, L.proj);
   SPR_LAUNCH(launch_sample_metric(Q, BH, N, d, p.n_samples, p.seed, metric, at<int>(ws, L.sample_idx), err, st));
-  SPR_LAUNCH(launch_metric_eigen(metric, BH, d, re, at<float>(ws, L.eigval), at<float>(ws, L.eigvec),
-                                 at<float>(ws, L.proj), st));
-  float* Y = at<float>(ws, L.Y);
-  SPR_LAUNCH(launch_key_coords(K, BH, N, d, re, at<float>(ws, L.proj), Y, st));
-  // key k-means
-  float* cent_k = at<float>(ws, L.cent_k);
-  SPR_LAUNCH(launch_kmeans_seed(Y, BH, N, re, Gk, p.seed, PURPOSE_KEY_KMEANS, cent_k, at<int>(ws, L.key_init),
-                                err, st));
-  for (int t = 0; t < p.kmeans_iters; ++t) {
-    int* trk = (tr && tr->key_label_iters) ? tr->key_label_iters + (size_t)t * BH * N : nullptr;
-    SPR_LAUNCH(launch_kmeans_assign(Y, BH, N, re, Gk, cent_k, label_k, trk, st));
-    SPR_LAUNCH(launch_group_sort(label_k, BH, N, Gk, perm_k, koff, err, st));
-    if (t + 1 < p.kmeans_iters) SPR_LAUNCH(launch_segment_mean_f32(Y, BH, N, re, Gk, perm_k, koff, cent_k, 0, st));
-  }
+  SPR_LAUNCH(launch_metric_eigen(metric, BH, d, re, at<float>(ws, L.eigval), at<float>(ws, L.eigvec), proj, st));
+  if (tr && tr->key_coords) SPR_LAUNCH(launch_key_coords(K, BH, N, d, re, proj, tr->key_coords, st));
+  float* bias = at<float>(ws, L.bias);
+  float* wnorm = at<float>(ws, L.wnorm);
+  void* w_hi = at<char>(ws, L.w_hi);
+  void* w_lo = at<char>(ws, L.w_lo);
+  int* fcount = at<int>(ws, L.flag_count);
+  int* frows = at<int>(ws, L.flag_rows);
+  // One Lloyd k-means of the rows X (bf16, d) on coordinates A x; A(j, c) = a_scale * A[j*sj + c*sc].
+  auto kmeans = [&](const void* X, int G, int purpose, const float* A, size_t a_head, int sj, int sc, float a_scale,
+                    int D, int DT, float* m, float* nu, int* init, int* labels, int* perm, int* off,
+                    int* trace_iters) -> sparsepr_status {
+    SPR_LAUNCH(launch_seed_rows(X, BH, N, d, G, p.seed, purpose, m, init, err, st));
+    for (int t = 0; t < p.kmeans_iters; ++t) {
+      int* trc = trace_iters ? trace_iters + (size_t)t * BH * N : nullptr;
+      SPR_LAUNCH(launch_centroid_weights(m, BH, G, d, A, a_head, sj, sc, a_scale, D, DT, nu, bias, wnorm, w_hi,
+                                         w_lo, st));
+      SPR_CUDA(cudaMemsetAsync(fcount, 0, (size_t)BH * 4, st));
+      SPR_LAUNCH(launch_assign_tc(X, BH, N, d, G, w_hi, w_lo, bias, wnorm, labels, trc, fcount, frows, err, st));
+      SPR_LAUNCH(launch_assign_recheck(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, fcount, frows, labels,
+                                       trc, st));
+      SPR_LAUNCH(launch_group_sort(labels, BH, N, G, perm, off, err, st));
+      if (t + 1 < p.kmeans_iters) SPR_LAUNCH(launch_segment_mean_rows(X, BH, N, d, G, perm, off, m, st));
+    }
+    return SPARSEPR_OK;
+  };
+  // keys on y = Lambda^{1/2} U^T k: A(j, c) = proj[c][j]
+  SPR_CHECK(kmeans(K, Gk, PURPOSE_KEY_KMEANS, proj, (size_t)d * re, 1, re, 1.0f, re, L.DTk, at<float>(ws, L.m_k),
+                   at<float>(ws, L.nu_k), at<int>(ws, L.key_init), label_k, perm_k, koff,
+                   tr ? tr->key_label_iters : nullptr));
+  // K/V group centroids: mean raw key (empty group -> 0)
   float* C = at<float>(ws, L.C);
-  SPR_LAUNCH(launch_segment_mean_bf16(K, BH, N, d, Gk, perm_k, koff, C, st));
+  SPR_CUDA(cudaMemsetAsync(C, 0, (size_t)BH * Gk * d * 4, st));
+  SPR_LAUNCH(launch_segment_mean_rows(K, BH, N, d, Gk, perm_k, koff, C, st));
   float* Z = at<float>(ws, L.Z);
-  SPR_LAUNCH(launch_query_coords(Q, BH, N, d, C, Gk, eff_scale(p), Z, st));
-  // query k-means
-  float* cent_q = at<float>(ws, L.cent_q);
-  SPR_LAUNCH(launch_kmeans_seed(Z, BH, N, Gk, Gq, p.seed, PURPOSE_QUERY_KMEANS, cent_q,
-                                at<int>(ws, L.query_init), err, st));
-  for (int t = 0; t < p.kmeans_iters; ++t) {
-    int* trq = (tr && tr->query_label_iters) ? tr->query_label_iters + (size_t)t * BH * N : nullptr;
-    SPR_LAUNCH(launch_kmeans_assign(Z, BH, N, Gk, Gq, cent_q, label_q, trq, st));
-    SPR_LAUNCH(launch_group_sort(label_q, BH, N, Gq, perm_q, qoff, err, st));
-    if (t + 1 < p.kmeans_iters) SPR_LAUNCH(launch_segment_mean_f32(Z, BH, N, Gk, Gq, perm_q, qoff, cent_q, 0, st));
-  }
+  SPR_LAUNCH(launch_query_coords(Q, BH, N, d, C, Gk, scale, Z, st));
+  // queries on z = s C q: A(j, c) = s * C[j][c]
+  SPR_CHECK(kmeans(Q, Gq, PURPOSE_QUERY_KMEANS, C, (size_t)Gk * d, d, 1, scale, Gk, L.DTq, at<float>(ws, L.m_q),
+                   at<float>(ws, L.nu_q), at<int>(ws, L.query_init), label_q, perm_q, qoff,
+                   tr ? tr->query_label_iters : nullptr));
   float* mass = at<float>(ws, L.mass);
   SPR_LAUNCH(launch_cell_mass(Z, BH, N, Gk, Gq, perm_q, qoff, koff, mass, st));
   SPR_LAUNCH(launch_route_select(mass, BH, N, Gq, Gk, qoff, koff, p.density, p.n_probes, at<int>(ws, L.order),
@@ -240,7 +259,6 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
     SPR_CUDA(cp(tr->metric, L.metric, bh * d * d * 4));
     SPR_CUDA(cp(tr->eigval, L.eigval, bh * re * 4));
     SPR_CUDA(cp(tr->eigvec, L.eigvec, bh * d * re * 4));
-    SPR_CUDA(cp(tr->key_coords, L.Y, bh * N * re * 4));
     SPR_CUDA(cp(tr->key_init, L.key_init, bh * Gk * 4));
     SPR_CUDA(cp(tr->key_centroids, L.C, bh * Gk * d * 4));
     SPR_CUDA(cp(tr->query_coords, L.Z, bh * N * Gk * 4));

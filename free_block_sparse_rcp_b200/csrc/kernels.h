@@ -14,16 +14,8 @@ cudaError_t launch_metric_eigen(const float* metric, int BH, int D, int R, float
 cudaError_t launch_key_coords(const void* K, int BH, int N, int D, int R, const float* proj, float* Y,
                               cudaStream_t st);
 int kmeans_dt(int Dc);
-cudaError_t launch_kmeans_seed(const float* X, int BH, int N, int Dc, int G, uint64_t seed, int purpose,
-                               float* cent, int* init_out, int* err, cudaStream_t st);
-cudaError_t launch_kmeans_assign(const float* X, int BH, int N, int Dc, int G, const float* cent, int* labels,
-                                 int* trace, cudaStream_t st);
 cudaError_t launch_group_sort(const int* labels, int BH, int N, int G, int* perm, int* offsets, int* err,
                               cudaStream_t st);
-cudaError_t launch_segment_mean_f32(const float* X, int BH, int N, int Dc, int G, const int* perm,
-                                    const int* offsets, float* cent, int zero_empty, cudaStream_t st);
-cudaError_t launch_segment_mean_bf16(const void* X, int BH, int N, int D, int G, const int* perm,
-                                     const int* offsets, float* cent, cudaStream_t st);
 cudaError_t launch_query_coords(const void* Q, int BH, int N, int D, const float* C, int G, float scale,
                                 float* Z, cudaStream_t st);
 cudaError_t launch_cell_mass(const float* Z, int BH, int N, int Gk, int Gq, const int* perm_q, const int* qoff,
@@ -35,6 +27,22 @@ cudaError_t launch_route_select(const float* mass, int BH, int N, int Gq, int Gk
 cudaError_t launch_block_mask(const unsigned char* route, int BH, int N, int Gq, int Gk, int blk,
                               const int* perm_q, const int* label_q, const int* perm_k, const int* label_k,
                               unsigned char* bmask, cudaStream_t st);
+
+// kmeans_tc.cu
+int kmeans_gp(int G);
+cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_t seed, int purpose, float* m,
+                             int* init_out, int* err, cudaStream_t st);
+cudaError_t launch_centroid_weights(const float* m, int BH, int G, int d, const float* A, size_t a_head, int sj,
+                                    int sc, float a_scale, int D, int DT, float* nu, float* bias, float* wnorm,
+                                    void* w_hi, void* w_lo, cudaStream_t st);
+cudaError_t launch_assign_tc(const void* X, int BH, int N, int d, int G, const void* w_hi, const void* w_lo,
+                             const float* bias, const float* wnorm, int* labels, int* trace, int* flag_count,
+                             int* flag_rows, int* err, cudaStream_t st);
+cudaError_t launch_assign_recheck(const void* X, int BH, int N, int d, const float* A, size_t a_head, int sj, int sc,
+                                  float a_scale, int D, const float* nu, int G, const int* flag_count,
+                                  const int* flag_rows, int* labels, int* trace, cudaStream_t st);
+cudaError_t launch_segment_mean_rows(const void* X, int BH, int N, int d, int G, const int* perm, const int* offsets,
+                                     float* m, cudaStream_t st);
 
 // probe.cu
 cudaError_t launch_worklist(const unsigned char* route, const int* qoff, const int* koff, int BH, int Gq, int Gk,

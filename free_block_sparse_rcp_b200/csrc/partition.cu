@@ -4,9 +4,7 @@
 //   sample + metric   M_K = Q_s^T Q_s / M_s over M_s sampled query rows
 //   eigen             leading r_e eigenpairs of M_K (single-CTA Jacobi)
 //   key coordinates   y = Lambda^{1/2} U^T k
-//   k-means           Lloyd: direct-form squared distances in fp32, ties to the
-//                     lowest cluster, fp64 member sums, empty clusters keep
-//                     their centroid
+//   (k-means itself: kmeans_tc.cu)
 //   group sort        stable counting sort by label -> permutation + offsets
 //   centroids         mean raw key of every K/V group
 //   query coordinates z = s C q (logits against the K/V group centroids)
@@ -71,12 +69,12 @@ __global__ void __launch_bounds__(256) k_sample_metric(const __nv_bfloat16* __re
 }
 
 // ---------------------------------------------------------------------------
-// Leading eigenpairs of M_K.  grid = BH, block = 512.
+// Leading eigenpairs of M_K.  grid = BH, block = 1024.
 // Writes eigval [BH, R] (clamped >= 0), eigvec [BH, D, R] and the projector
 // P = U_R Lambda_R^{1/2} [BH, D, R] used for the key coordinates.
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(512) k_metric_eigen(const float* __restrict__ metric, int R,
+__global__ void __launch_bounds__(1024) k_metric_eigen(const float* __restrict__ metric, int R,
                                                      float* __restrict__ eigval, float* __restrict__ eigvec,
                                                      float* __restrict__ proj) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -93,8 +91,8 @@ __global__ void __launch_bounds__(512) k_metric_eigen(const float* __restrict__ 
     A[r * LD + c] = metric[(size_t)bh * D * D + i];
   }
   __syncthreads();
-  jacobi_eigen<float>(A, V, D, LD, cs, pr, red, 30, 2e-7f);
-  eigen_ranks<float>(A, D, LD, rank);
+  jacobi_eigen<float, D>(A, V, cs, pr, red, 15, 4e-6f);
+  eigen_ranks<float, D>(A, rank);
   for (int i = threadIdx.x; i < D; i += blockDim.x) {
     int k = rank[i];
     if (k < R) {
@@ -135,78 +133,6 @@ __global__ void __launch_bounds__(256) k_key_coords(const __nv_bfloat16* __restr
     for (int c = 0; c < D; ++c) acc = fmaf(ks[r * (D + 1) + c], ps[c * R + j], acc);
     Y[((size_t)bh * N + n0 + r) * R + j] = acc;
   }
-}
-
-// ---------------------------------------------------------------------------
-// k-means seeds: G distinct rows of X drawn with the purpose's stream; centroid j
-// starts at the j-th drawn row.  grid = BH, block = 256.  Centroids are stored
-// with row stride DT (zero padded past Dc).
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_kmeans_seed(const float* __restrict__ X, int N, int Dc, int DT,
-                                                    int G, uint64_t seed, int purpose,
-                                                    float* __restrict__ cent, int* __restrict__ init_out,
-                                                    int* err) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  int* mkey = reinterpret_cast<int*>(smem);
-  int* mval = mkey + kMapCap;
-  int* sidx = mval + kMapCap;
-  const int bh = blockIdx.x, tid = threadIdx.x;
-  SlotMap map{mkey, mval, kMapCap};
-  map.clear_all(tid, blockDim.x);
-  __syncthreads();
-  if (tid == 0) {
-    SplitMix64 g(stream_state(seed, bh, purpose));
-    if (!draw_without_replacement(g, N, G, map, sidx)) set_error(err, DERR_DRAW);
-  }
-  __syncthreads();
-  for (int e = tid; e < G * DT; e += blockDim.x) {
-    int g = e / DT, c = e - g * DT;
-    cent[(size_t)bh * G * DT + e] = c < Dc ? X[((size_t)bh * N + sidx[g]) * Dc + c] : 0.f;
-  }
-  if (init_out)
-    for (int g = tid; g < G; g += blockDim.x) init_out[(size_t)bh * G + g] = sidx[g];
-}
-
-// ---------------------------------------------------------------------------
-// k-means assignment: label = argmin_g sum_c (x_c - mu_gc)^2 (sequential fp32 fma
-// over c), strict '<' so ties keep the lowest g.  grid = (ceil(N/128), BH),
-// block = 128, dynamic smem = G * DT floats.
-// ---------------------------------------------------------------------------
-template <int DT>
-__global__ void __launch_bounds__(128) k_kmeans_assign(const float* __restrict__ X, int N, int Dc, int G,
-                                                      const float* __restrict__ cent, int* __restrict__ labels,
-                                                      int* __restrict__ trace) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  float* mu = reinterpret_cast<float*>(smem);
-  const int bh = blockIdx.y, tid = threadIdx.x;
-  const float4* c4 = reinterpret_cast<const float4*>(cent + (size_t)bh * G * DT);
-  float4* m4 = reinterpret_cast<float4*>(mu);
-  for (int i = tid; i < G * DT / 4; i += blockDim.x) m4[i] = c4[i];
-  __syncthreads();
-  const int i = blockIdx.x * 128 + tid;
-  if (i >= N) return;
-  float x[DT];
-  const float* xr = X + ((size_t)bh * N + i) * Dc;
-#pragma unroll
-  for (int c = 0; c < DT; ++c) x[c] = c < Dc ? xr[c] : 0.f;
-  float best = __int_as_float(0x7f800000);
-  int lab = 0;
-  for (int g = 0; g < G; ++g) {
-    const float4* mg = m4 + g * (DT / 4);
-    float dist = 0.f;
-#pragma unroll
-    for (int c4i = 0; c4i < DT / 4; ++c4i) {
-      float4 m = mg[c4i];
-      float t;
-      t = x[4 * c4i + 0] - m.x; dist = fmaf(t, t, dist);
-      t = x[4 * c4i + 1] - m.y; dist = fmaf(t, t, dist);
-      t = x[4 * c4i + 2] - m.z; dist = fmaf(t, t, dist);
-      t = x[4 * c4i + 3] - m.w; dist = fmaf(t, t, dist);
-    }
-    if (dist < best) { best = dist; lab = g; }
-  }
-  labels[(size_t)bh * N + i] = lab;
-  if (trace) trace[(size_t)bh * N + i] = lab;
 }
 
 // ---------------------------------------------------------------------------
@@ -262,30 +188,6 @@ __global__ void __launch_bounds__(1024) k_group_sort(const int* __restrict__ lab
       base[g] += s;
     }
     __syncthreads();
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Segment means: cent[g][c] = mean over permuted positions of group g of X[perm][c]
-// (fp64 sums in ascending original order); empty groups keep their value unless
-// zero_empty, in which case they become 0.  grid = (G, BH), block = 128.
-// ---------------------------------------------------------------------------
-template <typename TIn>
-__global__ void __launch_bounds__(128) k_segment_mean(const TIn* __restrict__ X, int N, int Dc, int DT, int G,
-                                                     const int* __restrict__ perm,
-                                                     const int* __restrict__ offsets, float* __restrict__ cent,
-                                                     int zero_empty) {
-  const int g = blockIdx.x, bh = blockIdx.y;
-  const int s0 = offsets[(size_t)bh * (G + 1) + g], s1 = offsets[(size_t)bh * (G + 1) + g + 1];
-  const int* pm = perm + (size_t)bh * N;
-  const TIn* Xh = X + (size_t)bh * N * Dc;
-  float* out = cent + ((size_t)bh * G + g) * DT;
-  for (int c = threadIdx.x; c < DT; c += blockDim.x) {
-    if (c >= Dc) { out[c] = 0.f; continue; }
-    if (s1 == s0) { if (zero_empty) out[c] = 0.f; continue; }
-    double acc = 0.0;
-    for (int s = s0; s < s1; ++s) acc += (double)to_f32(Xh[(size_t)pm[s] * Dc + c]);
-    out[c] = (float)(acc / (double)(s1 - s0));
   }
 }
 
@@ -552,10 +454,10 @@ cudaError_t launch_metric_eigen(const float* metric, int BH, int D, int R, float
   size_t sm = (size_t)(2 * D * (D + 1) + D + 64) * 4 + (size_t)(2 * D) * 4;
   if (D == 64) {
     cudaFuncSetAttribute(k_metric_eigen<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_metric_eigen<64><<<BH, 512, sm, st>>>(metric, R, eigval, eigvec, proj);
+    k_metric_eigen<64><<<BH, 1024, sm, st>>>(metric, R, eigval, eigvec, proj);
   } else {
     cudaFuncSetAttribute(k_metric_eigen<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_metric_eigen<128><<<BH, 512, sm, st>>>(metric, R, eigval, eigvec, proj);
+    k_metric_eigen<128><<<BH, 1024, sm, st>>>(metric, R, eigval, eigvec, proj);
   }
   return cudaGetLastError();
 }
@@ -580,54 +482,11 @@ int kmeans_dt(int Dc) {
   return dt;
 }
 
-cudaError_t launch_kmeans_seed(const float* X, int BH, int N, int Dc, int G, uint64_t seed, int purpose,
-                               float* cent, int* init_out, int* err, cudaStream_t st) {
-  size_t sm = (size_t)(2 * kMapCap + G) * 4;
-  cudaFuncSetAttribute(k_kmeans_seed, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  k_kmeans_seed<<<BH, 256, sm, st>>>(X, N, Dc, kmeans_dt(Dc), G, seed, purpose, cent, init_out, err);
-  return cudaGetLastError();
-}
-
-template <int DT>
-static cudaError_t assign_dt(const float* X, int BH, int N, int Dc, int G, const float* cent, int* labels,
-                             int* trace, cudaStream_t st) {
-  size_t sm = (size_t)G * DT * 4;
-  cudaFuncSetAttribute(k_kmeans_assign<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  k_kmeans_assign<DT><<<dim3(ceil_div(N, 128), BH), 128, sm, st>>>(X, N, Dc, G, cent, labels, trace);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_kmeans_assign(const float* X, int BH, int N, int Dc, int G, const float* cent, int* labels,
-                                 int* trace, cudaStream_t st) {
-  switch (kmeans_dt(Dc)) {
-    case 8: return assign_dt<8>(X, BH, N, Dc, G, cent, labels, trace, st);
-    case 16: return assign_dt<16>(X, BH, N, Dc, G, cent, labels, trace, st);
-    case 32: return assign_dt<32>(X, BH, N, Dc, G, cent, labels, trace, st);
-    case 64: return assign_dt<64>(X, BH, N, Dc, G, cent, labels, trace, st);
-    case 128: return assign_dt<128>(X, BH, N, Dc, G, cent, labels, trace, st);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
 cudaError_t launch_group_sort(const int* labels, int BH, int N, int G, int* perm, int* offsets, int* err,
                               cudaStream_t st) {
   size_t sm = (size_t)33 * G * 4;
   cudaFuncSetAttribute(k_group_sort, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   k_group_sort<<<BH, 1024, sm, st>>>(labels, N, G, perm, offsets, err);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_segment_mean_f32(const float* X, int BH, int N, int Dc, int G, const int* perm,
-                                    const int* offsets, float* cent, int zero_empty, cudaStream_t st) {
-  k_segment_mean<float><<<dim3(G, BH), 128, 0, st>>>(X, N, Dc, kmeans_dt(Dc), G, perm, offsets, cent,
-                                                    zero_empty);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_segment_mean_bf16(const void* X, int BH, int N, int D, int G, const int* perm,
-                                     const int* offsets, float* cent, cudaStream_t st) {
-  k_segment_mean<__nv_bfloat16><<<dim3(G, BH), 128, 0, st>>>((const __nv_bfloat16*)X, N, D, D, G, perm,
-                                                            offsets, cent, 1);
   return cudaGetLastError();
 }
 

@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_d
   int* rank = pr + PR;                            // [PR]
   int* ridx = rank + PR;                          // [64] eigen index of subspace column j
   const int bh = blockIdx.x, tid = threadIdx.x;
-  const int n = (P + 1) & ~1;  // Jacobi needs an even size; a padded zero row is harmless
+  // the Gram is padded to PR x PR with zero rows (P <= PR): padding adds zero eigenvalues only
   for (int e = tid; e < PR * D; e += 256) {
     const int r = e / D;
     float od = 0.f, os = 0.f;
@@ -276,21 +276,21 @@ __global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_d
     Xm[e] = os;
   }
   __syncthreads();
-  for (int e = tid; e < n * n; e += 256) {
-    const int i = e / n, j = e - i * n;
+  for (int e = tid; e < PR * PR; e += 256) {
+    const int i = e / PR, j = e - i * PR;
     double s = 0.0;
     for (int c = 0; c < D; ++c) s += (double)Rm[i * D + c] * (double)Rm[j * D + c];
     G[i * LDP + j] = s;
   }
   __syncthreads();
-  jacobi_eigen<double>(G, U, n, LDP, cs, pr, red, 40, 1e-14);
-  eigen_ranks<double>(G, n, LDP, rank);
-  for (int i = tid; i < n; i += 256)
+  jacobi_eigen<double, PR>(G, U, cs, pr, red, 40, 1e-13);
+  eigen_ranks<double, PR>(G, rank);
+  for (int i = tid; i < PR; i += 256)
     if (rank[i] < Rk) ridx[rank[i]] = i;
   __syncthreads();
   // subspace basis
   double lam0 = 0.0;
-  for (int i = 0; i < n; ++i) lam0 = fmax(lam0, G[i * LDP + i]);
+  for (int i = 0; i < PR; ++i) lam0 = fmax(lam0, G[i * LDP + i]);
   const double smax = sqrt(fmax(lam0, 0.0));
   for (int j = 0; j < Rk; ++j) {
     const int i = ridx[j];
@@ -299,7 +299,7 @@ __global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_d
     for (int c = tid; c < D; c += 256) {
       double v = 0.0;
       if (keep)
-        for (int p = 0; p < n; ++p) v += (double)Rm[p * D + c] * U[p * LDP + i];
+        for (int p = 0; p < PR; ++p) v += (double)Rm[p * D + c] * U[p * LDP + i];
       Vr[c * Rk + j] = v;
     }
     if (tid == 0 && sigma_out) sigma_out[(size_t)bh * Rk + j] = keep ? (float)sj : 0.f;
