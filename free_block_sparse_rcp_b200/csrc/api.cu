@@ -50,7 +50,7 @@ struct Layout {
   // header
   size_t err;
   // partition
-  size_t sample_idx, metric, eigval, eigvec, proj, m_k, nu_k, key_init, C, Z, m_q, nu_q, query_init, bias, wnorm,
+  size_t sample_idx, metric, eigval, eigvec, proj, m_k, nu_k, key_init, C, m_q, nu_q, query_init, bias, wnorm,
       w_hi, w_lo, flag_count, flag_rows, mass, order, cm, cc, alpha;
   // attend
   size_t rlist, rcum, rcnt, tiles, tile_count;
@@ -87,14 +87,13 @@ Layout make_layout(const sparsepr_params& p) {
   L.nu_k = take(BH * Gk * L.DTk * 4);
   L.key_init = take(BH * Gk * 4);
   L.C = take(BH * Gk * d * 4);
-  L.Z = take(BH * N * Gk * 4);
   L.m_q = take(BH * Gq * d * 4);
   L.nu_q = take(BH * Gq * L.DTq * 4);
   L.query_init = take(BH * Gq * 4);
   L.bias = take(BH * GPmax * 4);
   L.wnorm = take(BH * GPmax * 4);
   L.w_hi = take(BH * GPmax * d * 2);
-  L.w_lo = take(BH * GPmax * d * 2);
+  L.w_lo = take(BH * GPmax * d * 2 * 2);   // also holds the third part of C for the cell mass
   L.flag_count = take(BH * 4);
   L.flag_rows = take(BH * N * 4);
   L.mass = take(BH * Gq * Gk * 4);
@@ -159,9 +158,15 @@ sparsepr_status check_params(const sparsepr_params* p) {
   // kernel limits
   if (p->n_kgroups > 128) return fail(SPARSEPR_EUNSUPPORTED, "n_kgroups > 128 (query coordinates wider than 128) not built");
   if (p->n_qgroups > 128) return fail(SPARSEPR_EUNSUPPORTED, "n_qgroups > 128 not built");
+  if (recheck_smem(p->d, p->n_kgroups, kmeans_dt(p->n_kgroups), p->n_qgroups) > kSmemLimit ||
+      recheck_smem(p->d, p->eig_rank, kmeans_dt(p->eig_rank), p->n_kgroups) > kSmemLimit ||
+      centroid_weights_smem(p->d, p->n_kgroups) > kSmemLimit)
+    return fail(SPARSEPR_EUNSUPPORTED, "too many groups for the k-means kernels");
+  if (cell_mass_tc_smem(p->d, kmeans_gp(p->n_kgroups)) > kSmemLimit)
+    return fail(SPARSEPR_EUNSUPPORTED, "too many K/V groups for the cell-mass kernel");
   if ((size_t)p->d * p->sub_rank > 64 * 65 || probe_fit_smem(p->d, p->sub_rank) > kSmemLimit)
     return failv(SPARSEPR_EUNSUPPORTED, "sub_rank too large for the single-CTA fit (d*r)", (long long)p->d * p->sub_rank);
-  if (attn_tc_smem_bytes(p->d, p->n_kgroups) > kSmemLimit || probe_attn_smem(p->d, p->n_kgroups) > kSmemLimit)
+  if (attn_tc_smem_bytes(p->d, p->n_kgroups) > kSmemLimit || probe_tc_smem_bytes(p->d, p->n_kgroups) > kSmemLimit)
     return fail(SPARSEPR_EUNSUPPORTED, "too many K/V groups for the attention kernels");
   return SPARSEPR_OK;
 }
@@ -237,14 +242,16 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
   float* C = at<float>(ws, L.C);
   SPR_CUDA(cudaMemsetAsync(C, 0, (size_t)BH * Gk * d * 4, st));
   SPR_LAUNCH(launch_segment_mean_rows(K, BH, N, d, Gk, perm_k, koff, C, st));
-  float* Z = at<float>(ws, L.Z);
-  SPR_LAUNCH(launch_query_coords(Q, BH, N, d, C, Gk, scale, Z, st));
+  if (tr && tr->query_coords) SPR_LAUNCH(launch_query_coords(Q, BH, N, d, C, Gk, scale, tr->query_coords, st));
   // queries on z = s C q: A(j, c) = s * C[j][c]
   SPR_CHECK(kmeans(Q, Gq, PURPOSE_QUERY_KMEANS, C, (size_t)Gk * d, d, 1, scale, Gk, L.DTq, at<float>(ws, L.m_q),
                    at<float>(ws, L.nu_q), at<int>(ws, L.query_init), label_q, perm_q, qoff,
                    tr ? tr->query_label_iters : nullptr));
   float* mass = at<float>(ws, L.mass);
-  SPR_LAUNCH(launch_cell_mass(Z, BH, N, Gk, Gq, perm_q, qoff, koff, mass, st));
+  // the weight buffers are free again: they hold the three bf16 parts of C
+  const size_t cpart = (size_t)BH * kmeans_gp(Gk) * d * 2;
+  SPR_LAUNCH(launch_cell_mass_tc(Q, BH, N, d, Gq, Gk, perm_q, qoff, koff, C, scale, w_hi, w_lo,
+                                 at<char>(ws, L.w_lo) + cpart, mass, err, st));
   SPR_LAUNCH(launch_route_select(mass, BH, N, Gq, Gk, qoff, koff, p.density, p.n_probes, at<int>(ws, L.order),
                                  at<double>(ws, L.cm), at<long long>(ws, L.cc), route, rho,
                                  at<double>(ws, L.alpha), st));
@@ -261,7 +268,6 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
     SPR_CUDA(cp(tr->eigvec, L.eigvec, bh * d * re * 4));
     SPR_CUDA(cp(tr->key_init, L.key_init, bh * Gk * 4));
     SPR_CUDA(cp(tr->key_centroids, L.C, bh * Gk * d * 4));
-    SPR_CUDA(cp(tr->query_coords, L.Z, bh * N * Gk * 4));
     SPR_CUDA(cp(tr->query_init, L.query_init, bh * Gq * 4));
     SPR_CUDA(cp(tr->cell_mass, L.mass, bh * Gq * Gk * 4));
     SPR_CUDA(cp(tr->alpha, L.alpha, bh * 8));
@@ -302,7 +308,7 @@ sparsepr_status run_probe_fit(const sparsepr_params& p, const Layout& L, const v
   float* part_o = at<float>(ws, L.part_o);
   float* part_ml = at<float>(ws, L.part_ml);
   SPR_LAUNCH(launch_probe_attn(Q, K, V, BH, N, d, p.n_kgroups, p.n_qgroups, P, probe_idx, pgrp, label_k, route,
-                               eff_scale(p) * 1.4426950408889634f, part_o, part_ml, st));
+                               eff_scale(p) * 1.4426950408889634f, part_o, part_ml, at<int>(ws, L.err), st));
   float* osp = at<float>(ws, L.o_sparse_p);
   float* lsd = at<float>(ws, L.lse_d);
   float* lss = at<float>(ws, L.lse_s);

@@ -12,7 +12,8 @@
 //              128-row chunk, by index through perm_q / perm_k, into 128B-swizzled
 //              shared-memory tiles (the permuted layout is never materialised)
 // Per chunk j:  S_j = Q K_j^T  -> TMEM (two buffers, so S_{j+1} overlaps softmax_j)
-//               P_j = exp2(S_j * s*log2e - m) in bf16 -> shared memory
+//               P_j = exp2(S_j * s*log2e - m) in bf16 -> shared memory (two buffers, so
+//                     softmax_{j+1} overlaps PV_j)
 //               O  += P_j V_j   (TMEM accumulator, rescaled in place only when a row's
 //                                 running max grows by more than 2^8)
 // Every mbarrier wait is bounded (2 s); a timeout raises an abort flag that ends every
@@ -35,7 +36,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct Bars {
-  uint64_t q, full[2], empty[2], s_full[2], s_free[2], p_full, o_done, mma_done;
+  uint64_t q, full[2], empty[2], s_full[2], s_free[2], p_full[2], p_empty[2], o_done, mma_done;
 };
 
 template <int D>
@@ -44,9 +45,10 @@ struct Layout {
   static constexpr uint32_t oQ = 0;
   static constexpr uint32_t oK = oQ + kTile;
   static constexpr uint32_t oV = oK + 2 * kTile;
-  static constexpr uint32_t oP = oV + 2 * kTile;
-  static constexpr uint32_t oBar = oP + 128 * 128 * 2;
-  static constexpr uint32_t oInt = oBar + 256;
+  static constexpr uint32_t kP = 128 * 128 * 2;
+  static constexpr uint32_t oP = oV + 2 * kTile;          // two P buffers
+  static constexpr uint32_t oBar = oP + 2 * kP;
+  static constexpr uint32_t oInt = oBar + 128;
 };
 
 template <int D, bool DENSE>
@@ -58,11 +60,15 @@ __global__ void __launch_bounds__(NT, 1)
               const int2* __restrict__ tiles, const int* __restrict__ tile_count, int max_tiles, float scale_log2,
               __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int* err) {
   using L = Layout<D>;
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  // 1024-byte aligned base for the swizzled tiles
-  const uint32_t raw = su32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  unsigned char* smem = smem_raw + (base - raw);
+  // The 128B-swizzled tiles need a 1024-byte aligned base; dynamic shared memory starts
+  // at the CTA's shared window, which is aligned, and the layout leaves no room for a
+  // realignment pad, so a misaligned base is reported and the tile skipped.
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const uint32_t base = su32(smem);
+  if (base & 1023u) {
+    if (threadIdx.x == 0) set_error(err, DERR_INDEX);
+    return;
+  }
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.y;
@@ -71,8 +77,7 @@ __global__ void __launch_bounds__(NT, 1)
   Bars* bars = reinterpret_cast<Bars*>(smem + L::oBar);
   int* ints = reinterpret_cast<int*>(smem + L::oInt);
   int* sQrow = ints;                  // [128]
-  int* sKrow = sQrow + 128;           // [2][128]
-  int* sMisc = sKrow + 256;           // [0] tmem base, [1] abort, [2] total, [3] cnt, [4] slot ok
+  int* sMisc = sQrow + 128;           // [0] tmem base, [1] abort, [2] total, [3] cnt, [4] slot ok
   int* sList = sMisc + 8;             // [Gk]
   int* sKoffL = sList + Gk;           // [Gk]
   int* sCum = sKoffL + Gk;            // [Gk + 1]
@@ -119,8 +124,9 @@ __global__ void __launch_bounds__(NT, 1)
       mbar_init(su32(&bars->empty[s]), 1);
       mbar_init(su32(&bars->s_full[s]), 1);
       mbar_init(su32(&bars->s_free[s]), NSOFT);
+      mbar_init(su32(&bars->p_full[s]), NSOFT);
+      mbar_init(su32(&bars->p_empty[s]), 1);
     }
-    mbar_init(su32(&bars->p_full), NSOFT);
     mbar_init(su32(&bars->o_done), 1);
     mbar_init(su32(&bars->mma_done), 1);
     fence_barrier_init();
@@ -161,31 +167,32 @@ __global__ void __launch_bounds__(NT, 1)
       const int s = j & 1;
       // one thread waits for the slot; the named barrier below publishes the outcome
       if (p == 0) *prod_ok = (j < 2 || wait(bars->empty[s], ((j >> 1) - 1) & 1)) ? 1 : 0;
-      // key row of slot p of chunk j
+      // key row of slot p of chunk j (this warp's 32 rows: 32 * pw + lane)
+      int myrow = -1;
       {
         const int pos = j * BN + p;
-        int row = -1;
         if (pos < total) {
           if (DENSE) {
-            row = pos;
+            myrow = pos;
           } else {
             int lo = 0, hi = cnt - 1;
             while (lo < hi) {
               const int mid = (lo + hi + 1) >> 1;
               if (sCum[mid] <= pos) lo = mid; else hi = mid - 1;
             }
-            row = perm_k[head + sKoffL[lo] + (pos - sCum[lo])];
-            if (row < 0 || row >= N) { set_error(err, DERR_INDEX); row = -1; }
+            myrow = perm_k[head + sKoffL[lo] + (pos - sCum[lo])];
+            if (myrow < 0 || myrow >= N) { set_error(err, DERR_INDEX); myrow = -1; }
           }
         }
-        sKrow[s * 128 + p] = row;
       }
       named_sync(1, NPROD);
       if (!*prod_ok) break;
       const uint32_t dk = sK + s * L::kTile, dv = sV + s * L::kTile;
+#pragma unroll
       for (int i = 0; i < 32 / RPI; ++i) {
-        const int r = pw * 32 + i * RPI + pl / CPR, c = pl % CPR;
-        const int row = sKrow[s * 128 + r];
+        const int rl = i * RPI + pl / CPR, c = pl % CPR;   // row within this warp's 32
+        const int row = __shfl_sync(0xffffffffu, myrow, rl);
+        const int r = pw * 32 + rl;
         const size_t off = (head + (row < 0 ? 0 : row)) * D + c * 8;
         const uint32_t o = tile_off(r, c, 128);
         cp_async16(dk + o, K + off, row >= 0);
@@ -201,16 +208,18 @@ __global__ void __launch_bounds__(NT, 1)
       constexpr uint32_t IDO = idesc_bf16(128, D, true);
       bool ok = nchunks == 0 || wait(bars->q, 0);
       auto issue_pv = [&](int i) -> bool {
-        if (!wait(bars->p_full, i & 1)) return false;
+        if (!wait(bars->p_full[i & 1], (i >> 1) & 1)) return false;
         tc_fence_after();
         const uint32_t vb = sV + (i & 1) * L::kTile;
+        const uint32_t pb = sP + (i & 1) * L::kP;
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k) {
-          const uint64_t ad = sdesc(sP + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
+          const uint64_t ad = sdesc(pb + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
           const uint64_t bd = sdesc(vb + k * 2048, 16384, 1024);
           tc_mma(tO, ad, bd, IDO, (i > 0 || k > 0) ? 1u : 0u);
         }
         tc_commit(su32(&bars->empty[i & 1]));
+        tc_commit(su32(&bars->p_empty[i & 1]));
         tc_commit(su32(&bars->o_done));
         return true;
       };
@@ -273,25 +282,27 @@ __global__ void __launch_bounds__(NT, 1)
         pk[c >> 1] = pack_bf16(p0, p1);
       }
       l = l * alpha + rs;
-      if (j >= 1) {
-        ok = wait(bars->o_done, (j - 1) & 1);
-        ok = __all_sync(0xffffffffu, ok);
+      if (warp_need && j >= 1) {
+        // O row *= alpha (in TMEM, warp-uniform) once PV_{j-1} has finished with it
+        ok = __all_sync(0xffffffffu, wait(bars->o_done, (j - 1) & 1));
         if (!ok) break;
         tc_fence_after();
-        if (warp_need) {
-          // O row *= alpha (in TMEM), warp-uniform
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tc_ld32(tO + lane_off + c * 32, o);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tc_ld32(tO + lane_off + c * 32, o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tc_st32(tO + lane_off + c * 32, o);
-          }
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tc_st32(tO + lane_off + c * 32, o);
         }
       }
+      if (j >= 2) {
+        // P buffer b was last read by PV_{j-2}
+        ok = __all_sync(0xffffffffu, wait(bars->p_empty[b], ((j >> 1) - 1) & 1));
+        if (!ok) break;
+      }
       // P row t -> shared memory ([2 halves][128 rows][64] bf16, 128B-swizzled)
-      unsigned char* prow = smem + L::oP;
+      unsigned char* prow = smem + L::oP + b * L::kP;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
@@ -299,7 +310,7 @@ __global__ void __launch_bounds__(NT, 1)
       }
       fence_proxy_async();
       tc_fence_before();
-      mbar_arrive(su32(&bars->p_full));
+      mbar_arrive(su32(&bars->p_full[b]));
     }
     // epilogue
     const int row = sQrow[t];
@@ -343,7 +354,7 @@ __global__ void __launch_bounds__(NT, 1)
 
 size_t attn_tc_smem_bytes(int D, int Gk) {
   const size_t tiles = (D == 64) ? tc::Layout<64>::oInt : tc::Layout<128>::oInt;
-  size_t s = 1024 + tiles + (size_t)(128 + 256 + 8 + 3 * Gk + 1) * 4;
+  size_t s = tiles + (size_t)(128 + 8 + 3 * Gk + 1) * 4;
   // at most one CTA per SM: the kernel allocates all 512 TMEM columns
   return s < 120 * 1024 ? 120 * 1024 : s;
 }

@@ -5,8 +5,8 @@
 // first (A <- J^T A) then columns (A <- A J, V <- V J); each rotation zeroes its
 // (p, q) entry (Golub & Van Loan, symmetric Schur decomposition).  A sweep is n-1
 // rounds.  Sweeps stop when the off-diagonal Frobenius norm is at most tol times the
-// diagonal one (for fp32 the floor is about sqrt(n) u, so tol = 4e-6 at n = 128), or
-// after max_sweeps.
+// diagonal one (for fp32 the rounding floor of that ratio is near sqrt(n) u ~ 1e-6 at
+// n = 128, so fp32 callers use tol = 2e-5), or after max_sweeps.
 #pragma once
 #include "common.cuh"
 

@@ -18,8 +18,6 @@ cudaError_t launch_group_sort(const int* labels, int BH, int N, int G, int* perm
                               cudaStream_t st);
 cudaError_t launch_query_coords(const void* Q, int BH, int N, int D, const float* C, int G, float scale,
                                 float* Z, cudaStream_t st);
-cudaError_t launch_cell_mass(const float* Z, int BH, int N, int Gk, int Gq, const int* perm_q, const int* qoff,
-                             const int* koff, float* mass, cudaStream_t st);
 cudaError_t launch_route_select(const float* mass, int BH, int N, int Gq, int Gk, const int* qoff,
                                 const int* koff, float density, int P, int* order, double* cm,
                                 long long* cc, unsigned char* route, float* rho_exec, double* alpha,
@@ -30,6 +28,8 @@ cudaError_t launch_block_mask(const unsigned char* route, int BH, int N, int Gq,
 
 // kmeans_tc.cu
 int kmeans_gp(int G);
+size_t centroid_weights_smem(int d, int D);
+size_t recheck_smem(int d, int D, int DT, int G);
 cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_t seed, int purpose, float* m,
                              int* init_out, int* err, cudaStream_t st);
 cudaError_t launch_centroid_weights(const float* m, int BH, int G, int d, const float* A, size_t a_head, int sj,
@@ -43,6 +43,10 @@ cudaError_t launch_assign_recheck(const void* X, int BH, int N, int d, const flo
                                   const int* flag_rows, int* labels, int* trace, cudaStream_t st);
 cudaError_t launch_segment_mean_rows(const void* X, int BH, int N, int d, int G, const int* perm, const int* offsets,
                                      float* m, cudaStream_t st);
+size_t cell_mass_tc_smem(int D, int GP);
+cudaError_t launch_cell_mass_tc(const void* Q, int BH, int N, int d, int Gq, int Gk, const int* perm_q, const int* qoff,
+                                const int* koff, const float* C, float scale, void* c1, void* c2, void* c3,
+                                float* mass, int* err, cudaStream_t st);
 
 // probe.cu
 cudaError_t launch_worklist(const unsigned char* route, const int* qoff, const int* koff, int BH, int Gq, int Gk,
@@ -51,11 +55,14 @@ cudaError_t launch_worklist(const unsigned char* route, const int* qoff, const i
 cudaError_t launch_probe_pick(const int* perm_q, const int* qoff, int BH, int N, int Gq, int P, uint64_t seed,
                               int* probe_idx, int* probe_grp, int* err, cudaStream_t st);
 int probe_splits(int N);
-size_t probe_attn_smem(int D, int Gk);
+size_t probe_tc_smem_bytes(int D, int Gk);
+cudaError_t launch_probe_tc(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk, int Gq, int P,
+                            const int* probe_idx, const int* probe_grp, const int* label_k, const unsigned char* route,
+                            float scale_log2, int S, float* part_o, float* part_ml, int* err, cudaStream_t st);
 size_t probe_fit_smem(int D, int Rk);
 cudaError_t launch_probe_attn(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk, int Gq,
                               int P, const int* probe_idx, const int* probe_grp, const int* label_k,
-                              const unsigned char* route, float scale_log2, float* part_o, float* part_ml,
+                              const unsigned char* route, float scale_log2, float* part_o, float* part_ml, int* err,
                               cudaStream_t st);
 cudaError_t launch_probe_attn_splits(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk,
                                      int Gq, int P, const int* probe_idx, const int* probe_grp, const int* label_k,

@@ -51,11 +51,15 @@ __global__ void __launch_bounds__(256) k_seed_rows(const __nv_bfloat16* __restri
 }
 
 // ---------------------------------------------------------------------------
-// Centroid weights.  A(j, c) = a_scale * A[j * sj + c * sc] (D x d).
+// Centroid weights.  A(j, c) = a_scale * A[j * sj + c * sc] (D x d) is staged once per
+// CTA in shared memory as sA[j][c] with row stride d + 1 (conflict-free both ways).
 //   nu = A m (fp32, sequential over c), bias = ||nu||^2 (sequential over j),
 //   w = A^T nu -> w_hi = bf16(w), w_lo = bf16(w - w_hi); wnorm = ||w||.
-// Rows g in [G, GP) are padding: w = 0, bias = +inf.  grid = (GP, BH), block = 128.
+// Rows g in [G, GP) are padding: w = 0, bias = +inf.
+// grid = (ceil(GP / WG_PER_CTA), BH), block = 128.
 // ---------------------------------------------------------------------------
+constexpr int WG_PER_CTA = 16;
+
 __global__ void __launch_bounds__(128) k_centroid_weights(const float* __restrict__ m, int G, int GP, int d,
                                                          const float* __restrict__ A, size_t a_head, int sj,
                                                          int sc, float a_scale, int D, int DT,
@@ -63,48 +67,59 @@ __global__ void __launch_bounds__(128) k_centroid_weights(const float* __restric
                                                          float* __restrict__ wnorm,
                                                          __nv_bfloat16* __restrict__ w_hi,
                                                          __nv_bfloat16* __restrict__ w_lo) {
-  __shared__ float sm_m[128];
-  __shared__ float sm_nu[128];
-  __shared__ float sm_w[128];
-  const int g = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
-  const size_t wrow = ((size_t)bh * GP + g) * d;
-  if (g >= G) {
-    for (int c = tid; c < d; c += 128) {
-      w_hi[wrow + c] = __float2bfloat16(0.f);
-      w_lo[wrow + c] = __float2bfloat16(0.f);
-    }
-    if (tid == 0) {
-      bias[(size_t)bh * GP + g] = __int_as_float(0x7f800000);
-      wnorm[(size_t)bh * GP + g] = 0.f;
-    }
-    return;
-  }
+  extern __shared__ __align__(16) float sw[];
+  float* sA = sw;                        // [D][d + 1]
+  float* sm_m = sA + D * (d + 1);        // [d]
+  float* sm_nu = sm_m + d;               // [128]
+  float* sm_w = sm_nu + 128;             // [d]
+  const int bh = blockIdx.y, tid = threadIdx.x;
   const float* Ah = A + a_head * bh;
-  for (int c = tid; c < d; c += 128) sm_m[c] = m[((size_t)bh * G + g) * d + c];
-  __syncthreads();
-  for (int j = tid; j < D; j += 128) {
-    float acc = 0.f;
-    for (int c = 0; c < d; ++c) acc = fmaf(Ah[(size_t)j * sj + (size_t)c * sc], sm_m[c], acc);
-    sm_nu[j] = a_scale * acc;
+  for (int e = tid; e < D * d; e += 128) {
+    const int j = e / d, c = e - j * d;
+    sA[j * (d + 1) + c] = Ah[(size_t)j * sj + (size_t)c * sc];
   }
   __syncthreads();
-  for (int j = tid; j < DT; j += 128) nu[((size_t)bh * G + g) * DT + j] = j < D ? sm_nu[j] : 0.f;
-  for (int c = tid; c < d; c += 128) {
-    float acc = 0.f;
-    for (int j = 0; j < D; ++j) acc = fmaf(Ah[(size_t)j * sj + (size_t)c * sc], sm_nu[j], acc);
-    const float w = a_scale * acc;
-    sm_w[c] = w;
-    const __nv_bfloat16 hi = __float2bfloat16(w);
-    w_hi[wrow + c] = hi;
-    w_lo[wrow + c] = __float2bfloat16(w - __bfloat162float(hi));
-  }
-  __syncthreads();
-  if (tid == 0) {
-    float b = 0.f, n2 = 0.f;
-    for (int j = 0; j < D; ++j) b = fmaf(sm_nu[j], sm_nu[j], b);
-    for (int c = 0; c < d; ++c) n2 = fmaf(sm_w[c], sm_w[c], n2);
-    bias[(size_t)bh * GP + g] = b;
-    wnorm[(size_t)bh * GP + g] = sqrtf(n2);
+  const int g0 = blockIdx.x * WG_PER_CTA, g1 = min(GP, g0 + WG_PER_CTA);
+  for (int g = g0; g < g1; ++g) {
+    const size_t wrow = ((size_t)bh * GP + g) * d;
+    if (g >= G) {
+      for (int c = tid; c < d; c += 128) {
+        w_hi[wrow + c] = __float2bfloat16(0.f);
+        w_lo[wrow + c] = __float2bfloat16(0.f);
+      }
+      if (tid == 0) {
+        bias[(size_t)bh * GP + g] = __int_as_float(0x7f800000);
+        wnorm[(size_t)bh * GP + g] = 0.f;
+      }
+      continue;
+    }
+    for (int c = tid; c < d; c += 128) sm_m[c] = m[((size_t)bh * G + g) * d + c];
+    __syncthreads();
+    for (int j = tid; j < D; j += 128) {
+      float acc = 0.f;
+      for (int c = 0; c < d; ++c) acc = fmaf(sA[j * (d + 1) + c], sm_m[c], acc);
+      sm_nu[j] = a_scale * acc;
+    }
+    __syncthreads();
+    for (int j = tid; j < DT; j += 128) nu[((size_t)bh * G + g) * DT + j] = j < D ? sm_nu[j] : 0.f;
+    for (int c = tid; c < d; c += 128) {
+      float acc = 0.f;
+      for (int j = 0; j < D; ++j) acc = fmaf(sA[j * (d + 1) + c], sm_nu[j], acc);
+      const float w = a_scale * acc;
+      sm_w[c] = w;
+      const __nv_bfloat16 hi = __float2bfloat16(w);
+      w_hi[wrow + c] = hi;
+      w_lo[wrow + c] = __float2bfloat16(w - __bfloat162float(hi));
+    }
+    __syncthreads();
+    if (tid == 0) {
+      float b = 0.f, n2 = 0.f;
+      for (int j = 0; j < D; ++j) b = fmaf(sm_nu[j], sm_nu[j], b);
+      for (int c = 0; c < d; ++c) n2 = fmaf(sm_w[c], sm_w[c], n2);
+      bias[(size_t)bh * GP + g] = b;
+      wnorm[(size_t)bh * GP + g] = sqrtf(n2);
+    }
+    __syncthreads();
   }
 }
 
@@ -252,42 +267,60 @@ __global__ void __launch_bounds__(128) k_assign_tc(const __nv_bfloat16* __restri
 // ---------------------------------------------------------------------------
 // Exact re-assignment of the uncertified rows: y = A x (fp32, sequential over c),
 // dist_g = sum_c (y_c - nu_gc)^2 (sequential fp32 fma over c), argmin with ties to the
-// lowest g.  One warp per row.  grid = (64, BH), block = 256.
+// lowest g.  A and the centroids are staged in shared memory (padded rows); one warp per
+// row.  grid = (RC_PER_HEAD, BH), block = 512.
 // ---------------------------------------------------------------------------
+constexpr int RC_PER_HEAD = 8;
+
 template <int DT>
-__global__ void __launch_bounds__(256) k_assign_recheck(const __nv_bfloat16* __restrict__ X, int N, int d,
+__global__ void __launch_bounds__(512) k_assign_recheck(const __nv_bfloat16* __restrict__ X, int N, int d,
                                                        const float* __restrict__ A, size_t a_head, int sj, int sc,
                                                        float a_scale, int D, const float* __restrict__ nu, int G,
                                                        const int* __restrict__ flag_count,
                                                        const int* __restrict__ flag_rows, int* __restrict__ labels,
                                                        int* __restrict__ trace) {
-  __shared__ float sx[8][128];
-  __shared__ float sy[8][DT];
+  extern __shared__ __align__(16) float sr[];
   const int bh = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const size_t head = (size_t)bh * N;
   const int cnt = flag_count[bh];
+  if ((int)blockIdx.x * 16 >= cnt) return;
+  float* sA = sr;                       // [D][d + 1]
+  float* sNu = sA + D * (d + 1);        // [G][DT + 1]
+  float* sx = sNu + G * (DT + 1);       // [16][d]
+  float* sy = sx + 16 * d;              // [16][DT]
+  const size_t head = (size_t)bh * N;
   const float* Ah = A + a_head * bh;
   const float* nuh = nu + (size_t)bh * G * DT;
-  for (int i = blockIdx.x * 8 + warp; i < cnt; i += gridDim.x * 8) {
+  for (int e = threadIdx.x; e < D * d; e += 512) {
+    const int j = e / d, c = e - j * d;
+    sA[j * (d + 1) + c] = Ah[(size_t)j * sj + (size_t)c * sc];
+  }
+  for (int e = threadIdx.x; e < G * DT; e += 512) {
+    const int g = e / DT, c = e - g * DT;
+    sNu[g * (DT + 1) + c] = nuh[e];
+  }
+  __syncthreads();
+  float* wx = sx + warp * d;
+  float* wy = sy + warp * DT;
+  for (int i = blockIdx.x * 16 + warp; i < cnt; i += gridDim.x * 16) {
     const int row = flag_rows[head + i];
-    for (int c = lane; c < d; c += 32) sx[warp][c] = bf2f(X[(head + row) * d + c]);
+    for (int c = lane; c < d; c += 32) wx[c] = bf2f(X[(head + row) * d + c]);
     __syncwarp();
     for (int j = lane; j < DT; j += 32) {
       float acc = 0.f;
       if (j < D) {
-        for (int c = 0; c < d; ++c) acc = fmaf(sx[warp][c], Ah[(size_t)j * sj + (size_t)c * sc], acc);
+        for (int c = 0; c < d; ++c) acc = fmaf(wx[c], sA[j * (d + 1) + c], acc);
         acc *= a_scale;
       }
-      sy[warp][j] = acc;
+      wy[j] = acc;
     }
     __syncwarp();
     float best = __int_as_float(0x7f800000);
     int bi = 0x7fffffff;
     for (int g = lane; g < G; g += 32) {
-      const float* mu = nuh + (size_t)g * DT;
+      const float* mu = sNu + g * (DT + 1);
       float dist = 0.f;
       for (int c = 0; c < DT; ++c) {
-        const float t = sy[warp][c] - mu[c];
+        const float t = wy[c] - mu[c];
         dist = fmaf(t, t, dist);
       }
       if (dist < best) { best = dist; bi = g; }
@@ -351,6 +384,159 @@ __global__ void __launch_bounds__(256) k_segment_mean_rows(const __nv_bfloat16* 
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Cell mass on the tensor cores.  p(a, g) = mean over the queries q of group a of
+// softmax_g(z_q[g] + ln n_g) over non-empty K/V groups, z_q = s q . c_g.
+// c_g is split into three bf16 parts (c = c1 + c2 + c3 to ~2^-24), so the products with
+// the exact bf16 q are exact and z carries only fp32 accumulation error.
+// One CTA = one head x a run of query groups; every group's permuted rows are gathered
+// through perm_q in 128-row tiles; column sums run over rows in fixed order, so the
+// result is deterministic.  grid = (CTAS_PER_HEAD, BH), block = 128.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) k_split3(const float* __restrict__ C, int G, int GP, int d,
+                                               __nv_bfloat16* __restrict__ c1, __nv_bfloat16* __restrict__ c2,
+                                               __nv_bfloat16* __restrict__ c3) {
+  const int g = blockIdx.x, bh = blockIdx.y;
+  for (int c = threadIdx.x; c < d; c += 128) {
+    const float x = g < G ? C[((size_t)bh * G + g) * d + c] : 0.f;
+    const __nv_bfloat16 a = __float2bfloat16(x);
+    const float r1 = x - __bfloat162float(a);
+    const __nv_bfloat16 b = __float2bfloat16(r1);
+    const __nv_bfloat16 e = __float2bfloat16(r1 - __bfloat162float(b));
+    const size_t o = ((size_t)bh * GP + g) * d + c;
+    c1[o] = a;
+    c2[o] = b;
+    c3[o] = e;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) k_cell_mass_tc(const __nv_bfloat16* __restrict__ Q, int N, int Gq, int Gk,
+                                                     int GP, const int* __restrict__ perm_q,
+                                                     const int* __restrict__ qoff, const int* __restrict__ koff,
+                                                     const __nv_bfloat16* __restrict__ c1,
+                                                     const __nv_bfloat16* __restrict__ c2,
+                                                     const __nv_bfloat16* __restrict__ c3, float scale,
+                                                     float* __restrict__ mass, int* err) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = su32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* smem = smem_raw + (base - raw);
+  constexpr uint32_t kX = 128u * D * 2u;
+  const uint32_t kC = (uint32_t)GP * D * 2u;
+  const uint32_t sX = base, sC1 = base + kX, sC2 = sC1 + kC, sC3 = sC2 + kC;
+  float* pst = reinterpret_cast<float*>(smem + kX + 3 * kC);   // [128][GP + 1]
+  float* lnn = pst + 128 * (GP + 1);                           // [GP]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(lnn + GP);
+  int* sMisc = reinterpret_cast<int*>(bar + 1);                 // [0] tmem, [1] abort
+  int* sRow = sMisc + 4;                                        // [128]
+  volatile int* abort_flag = sMisc + 1;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int bh = blockIdx.y;
+  const size_t head = (size_t)bh * N;
+  constexpr int CPR = D / 8;
+  const float NEG_INF = __int_as_float(0xff800000);
+
+  for (int e = tid; e < GP * CPR; e += 128) {
+    const int r = e / CPR, c = e - r * CPR;
+    const size_t off = ((size_t)bh * GP + r) * D + c * 8;
+    const uint32_t o = tile_off(r, c, GP);
+    cp_async16(sC1 + o, c1 + off, true);
+    cp_async16(sC2 + o, c2 + off, true);
+    cp_async16(sC3 + o, c3 + off, true);
+  }
+  for (int g = tid; g < GP; g += 128) {
+    const int n = g < Gk ? koff[(size_t)bh * (Gk + 1) + g + 1] - koff[(size_t)bh * (Gk + 1) + g] : 0;
+    lnn[g] = n > 0 ? logf((float)n) : NEG_INF;
+  }
+  if (tid == 0) {
+    sMisc[1] = 0;
+    mbar_init(su32(bar), 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tc_alloc(su32(&sMisc[0]), 128);
+    tc_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = (uint32_t)sMisc[0];
+  const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(GP >> 3) << 17) | (8u << 24);
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int* qo = qoff + (size_t)bh * (Gq + 1);
+  const int per = (Gq + gridDim.x - 1) / gridDim.x;
+  const int a0 = blockIdx.x * per, a1 = min(Gq, a0 + per);
+  int phase = 0;
+  bool ok = true;
+  for (int a = a0; a < a1 && ok; ++a) {
+    const int s0 = qo[a], s1 = qo[a + 1];
+    float colsum = 0.f;   // thread tid owns column tid
+    for (int t0 = s0; t0 < s1; t0 += 128) {
+      const int nr = min(128, s1 - t0);
+      sRow[tid] = tid < nr ? perm_q[head + t0 + tid] : -1;
+      __syncthreads();
+      for (int e = tid; e < 128 * CPR; e += 128) {
+        const int r = e / CPR, c = e - r * CPR;
+        const int row = sRow[r];
+        cp_async16(sX + tile_off(r, c, 128), Q + (head + (row < 0 ? 0 : row)) * D + c * 8, row >= 0);
+      }
+      cp_async_wait_all();
+      fence_proxy_async();
+      __syncthreads();
+      if (tid == 0) {
+        tc_fence_after();
+        int n = 0;
+        for (uint32_t cb : {sC1, sC2, sC3}) {
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
+            const uint32_t oc = (k >> 2) * (GP * 128) + (k & 3) * 32;
+            tc_mma(tmem, sdesc(sX + ox, 16, 1024), sdesc(cb + oc, 16, 1024), idesc, n++ > 0 ? 1u : 0u);
+          }
+        }
+        tc_commit(su32(bar));
+      }
+      ok = __syncthreads_and(bounded_wait(su32(bar), phase & 1, abort_flag, err) ? 1 : 0) != 0;
+      ++phase;
+      if (!ok) break;
+      tc_fence_after();
+      // row softmax over the non-empty groups
+      float mx = NEG_INF;
+      for (int c0 = 0; c0 < GP; c0 += 32) {
+        uint32_t r[32];
+        tc_ld32(tmem + lane_off + c0, r);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float l = lnn[c0 + e] == NEG_INF ? NEG_INF : scale * __uint_as_float(r[e]) + lnn[c0 + e];
+          pst[tid * (GP + 1) + c0 + e] = l;
+          mx = fmaxf(mx, l);
+        }
+      }
+      float sum = 0.f;
+      for (int g = 0; g < GP; ++g) {
+        const float l = pst[tid * (GP + 1) + g];
+        const float e = l == NEG_INF ? 0.f : expf(l - mx);
+        pst[tid * (GP + 1) + g] = e;
+        sum += e;
+      }
+      const float inv = (tid < nr && sum > 0.f) ? 1.f / sum : 0.f;
+      for (int g = 0; g < GP; ++g) pst[tid * (GP + 1) + g] *= inv;
+      tc_fence_before();
+      __syncthreads();
+      if (tid < Gk)
+        for (int r = 0; r < nr; ++r) colsum += pst[r * (GP + 1) + tid];
+      __syncthreads();
+    }
+    if (tid < Gk) mass[((size_t)bh * Gq + a) * Gk + tid] = s1 > s0 ? colsum / (float)(s1 - s0) : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tc_dealloc(tmem, 128);
+}
+
 }  // namespace km
 
 // ---------------------------------------------------------------------------
@@ -370,12 +556,16 @@ cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_
   return cudaGetLastError();
 }
 
+size_t centroid_weights_smem(int d, int D) { return ((size_t)D * (d + 1) + 2 * d + 128) * 4; }
+
 cudaError_t launch_centroid_weights(const float* m, int BH, int G, int d, const float* A, size_t a_head, int sj,
                                     int sc, float a_scale, int D, int DT, float* nu, float* bias, float* wnorm,
                                     void* w_hi, void* w_lo, cudaStream_t st) {
   const int GP = kmeans_gp(G);
-  km::k_centroid_weights<<<dim3(GP, BH), 128, 0, st>>>(m, G, GP, d, A, a_head, sj, sc, a_scale, D, DT, nu, bias,
-                                                        wnorm, (__nv_bfloat16*)w_hi, (__nv_bfloat16*)w_lo);
+  const size_t sm = centroid_weights_smem(d, D);
+  cudaFuncSetAttribute(km::k_centroid_weights, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  km::k_centroid_weights<<<dim3(ceil_div(GP, km::WG_PER_CTA), BH), 128, sm, st>>>(
+      m, G, GP, d, A, a_head, sj, sc, a_scale, D, DT, nu, bias, wnorm, (__nv_bfloat16*)w_hi, (__nv_bfloat16*)w_lo);
   return cudaGetLastError();
 }
 
@@ -399,12 +589,19 @@ cudaError_t launch_assign_tc(const void* X, int BH, int N, int d, int G, const v
   return cudaGetLastError();
 }
 
+size_t recheck_smem(int d, int D, int DT, int G) {
+  return ((size_t)D * (d + 1) + (size_t)G * (DT + 1) + 16 * (size_t)d + 16 * (size_t)DT) * 4;
+}
+
 template <int DT>
 static cudaError_t recheck_dt(const void* X, int BH, int N, int d, const float* A, size_t a_head, int sj, int sc,
                               float a_scale, int D, const float* nu, int G, const int* flag_count,
                               const int* flag_rows, int* labels, int* trace, cudaStream_t st) {
-  km::k_assign_recheck<DT><<<dim3(64, BH), 256, 0, st>>>((const __nv_bfloat16*)X, N, d, A, a_head, sj, sc, a_scale,
-                                                         D, nu, G, flag_count, flag_rows, labels, trace);
+  const size_t sm = recheck_smem(d, D, DT, G);
+  cudaFuncSetAttribute(km::k_assign_recheck<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  km::k_assign_recheck<DT><<<dim3(km::RC_PER_HEAD, BH), 512, sm, st>>>((const __nv_bfloat16*)X, N, d, A, a_head, sj,
+                                                                      sc, a_scale, D, nu, G, flag_count, flag_rows,
+                                                                      labels, trace);
   return cudaGetLastError();
 }
 
@@ -427,6 +624,37 @@ cudaError_t launch_segment_mean_rows(const void* X, int BH, int N, int d, int G,
     km::k_segment_mean_rows<64><<<dim3(G, BH), 256, 0, st>>>((const __nv_bfloat16*)X, N, G, perm, offsets, m);
   else
     km::k_segment_mean_rows<128><<<dim3(G, BH), 256, 0, st>>>((const __nv_bfloat16*)X, N, G, perm, offsets, m);
+  return cudaGetLastError();
+}
+
+size_t cell_mass_tc_smem(int D, int GP) {
+  return 1024 + (size_t)128 * D * 2 + 3 * (size_t)GP * D * 2 + (size_t)128 * (GP + 1) * 4 + (size_t)GP * 4 + 8 +
+         (4 + 128) * 4;
+}
+
+constexpr int kCellMassCtasPerHead = 8;
+
+cudaError_t launch_cell_mass_tc(const void* Q, int BH, int N, int d, int Gq, int Gk, const int* perm_q, const int* qoff,
+                                const int* koff, const float* C, float scale, void* c1, void* c2, void* c3,
+                                float* mass, int* err, cudaStream_t st) {
+  const int GP = kmeans_gp(Gk);
+  km::k_split3<<<dim3(GP, BH), 128, 0, st>>>(C, Gk, GP, d, (__nv_bfloat16*)c1, (__nv_bfloat16*)c2,
+                                            (__nv_bfloat16*)c3);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t sm = cell_mass_tc_smem(d, GP);
+  dim3 grid(kCellMassCtasPerHead, BH);
+  if (d == 64) {
+    cudaFuncSetAttribute(km::k_cell_mass_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    km::k_cell_mass_tc<64><<<grid, 128, sm, st>>>((const __nv_bfloat16*)Q, N, Gq, Gk, GP, perm_q, qoff, koff,
+                                                  (const __nv_bfloat16*)c1, (const __nv_bfloat16*)c2,
+                                                  (const __nv_bfloat16*)c3, scale, mass, err);
+  } else {
+    cudaFuncSetAttribute(km::k_cell_mass_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    km::k_cell_mass_tc<128><<<grid, 128, sm, st>>>((const __nv_bfloat16*)Q, N, Gq, Gk, GP, perm_q, qoff, koff,
+                                                   (const __nv_bfloat16*)c1, (const __nv_bfloat16*)c2,
+                                                   (const __nv_bfloat16*)c3, scale, mass, err);
+  }
   return cudaGetLastError();
 }
 

@@ -3,12 +3,11 @@
 //
 //   sample + metric   M_K = Q_s^T Q_s / M_s over M_s sampled query rows
 //   eigen             leading r_e eigenpairs of M_K (single-CTA Jacobi)
-//   key coordinates   y = Lambda^{1/2} U^T k
+//   key coordinates   y = Lambda^{1/2} U^T k (materialised for traces only)
 //   (k-means itself: kmeans_tc.cu)
 //   group sort        stable counting sort by label -> permutation + offsets
 //   centroids         mean raw key of every K/V group
-//   query coordinates z = s C q (logits against the K/V group centroids)
-//   cell mass         mean over group a of softmax_g(z_q[g] + ln n_g)
+//   query coordinates z = s C q (materialised for traces only)
 //   route             shared alpha by bisection under the pair budget
 //   block mask        tile-level view of the route on the permuted layout
 #include "common.cuh"
@@ -91,7 +90,7 @@ __global__ void __launch_bounds__(1024) k_metric_eigen(const float* __restrict__
     A[r * LD + c] = metric[(size_t)bh * D * D + i];
   }
   __syncthreads();
-  jacobi_eigen<float, D>(A, V, cs, pr, red, 15, 4e-6f);
+  jacobi_eigen<float, D>(A, V, cs, pr, red, 10, 2e-5f);
   eigen_ranks<float, D>(A, rank);
   for (int i = threadIdx.x; i < D; i += blockDim.x) {
     int k = rank[i];
@@ -234,48 +233,6 @@ __global__ void __launch_bounds__(256) k_query_coords(const __nv_bfloat16* __res
       int g = g0 + tx * 4 + j;
       if (g < G) Z[((size_t)bh * N + n) * G + g] = scale * acc[i][j];
     }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Cell mass p(a, g) = mean over queries of group a of softmax_g(z_q[g] + ln n_g)
-// (empty K/V groups excluded).  grid = (Gq, BH), block = 256; each warp owns
-// every 8th member and accumulates its own row of partial sums (deterministic).
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_cell_mass(const float* __restrict__ Z, int N, int Gk, int Gq,
-                                                  const int* __restrict__ perm_q, const int* __restrict__ qoff,
-                                                  const int* __restrict__ koff, float* __restrict__ mass) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  float* lnn = reinterpret_cast<float*>(smem);  // [Gk]
-  float* part = lnn + Gk;                       // [8][Gk]
-  const int a = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const float NEG_INF = __int_as_float(0xff800000);
-  for (int g = tid; g < Gk; g += blockDim.x) {
-    int n = koff[(size_t)bh * (Gk + 1) + g + 1] - koff[(size_t)bh * (Gk + 1) + g];
-    lnn[g] = n > 0 ? logf((float)n) : NEG_INF;
-  }
-  for (int e = tid; e < 8 * Gk; e += blockDim.x) part[e] = 0.f;
-  __syncthreads();
-  const int s0 = qoff[(size_t)bh * (Gq + 1) + a], s1 = qoff[(size_t)bh * (Gq + 1) + a + 1];
-  const int* pm = perm_q + (size_t)bh * N;
-  for (int s = s0 + warp; s < s1; s += 8) {
-    const float* zr = Z + ((size_t)bh * N + pm[s]) * Gk;
-    float mx = NEG_INF;
-    for (int g = lane; g < Gk; g += 32) mx = fmaxf(mx, lnn[g] == NEG_INF ? NEG_INF : zr[g] + lnn[g]);
-    mx = warp_max(mx);
-    float sum = 0.f;
-    for (int g = lane; g < Gk; g += 32) sum += lnn[g] == NEG_INF ? 0.f : expf(zr[g] + lnn[g] - mx);
-    sum = warp_sum(sum);
-    const float inv = 1.0f / sum;
-    for (int g = lane; g < Gk; g += 32)
-      part[warp * Gk + g] += lnn[g] == NEG_INF ? 0.f : expf(zr[g] + lnn[g] - mx) * inv;
-  }
-  __syncthreads();
-  const int na = s1 - s0;
-  for (int g = tid; g < Gk; g += blockDim.x) {
-    float t = 0.f;
-    for (int w = 0; w < 8; ++w) t += part[w * Gk + g];
-    mass[((size_t)bh * Gq + a) * Gk + g] = na > 0 ? t / (float)na : 0.f;
   }
 }
 
@@ -497,14 +454,6 @@ cudaError_t launch_query_coords(const void* Q, int BH, int N, int D, const float
     k_query_coords<64><<<grid, 256, 0, st>>>((const __nv_bfloat16*)Q, N, C, G, scale, Z);
   else
     k_query_coords<128><<<grid, 256, 0, st>>>((const __nv_bfloat16*)Q, N, C, G, scale, Z);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_cell_mass(const float* Z, int BH, int N, int Gk, int Gq, const int* perm_q, const int* qoff,
-                             const int* koff, float* mass, cudaStream_t st) {
-  size_t sm = (size_t)9 * Gk * 4;
-  cudaFuncSetAttribute(k_cell_mass, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  k_cell_mass<<<dim3(Gq, BH), 256, sm, st>>>(Z, N, Gk, Gq, perm_q, qoff, koff, mass);
   return cudaGetLastError();
 }
 

@@ -5,6 +5,7 @@
 #include "common.cuh"
 #include "jacobi.cuh"
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace spr {
 
@@ -76,127 +77,7 @@ __global__ void __launch_bounds__(256) k_probe_pick(const int* __restrict__ perm
   }
 }
 
-// ---------------------------------------------------------------------------
-// Dense and routed attention of the probe rows over one key split (fp32).
-// grid = (S, BH), block = 256.  Rows >= P are padding.  Writes per split and row
-// the base-2 running max, sum and unnormalised output of both accumulators.
-// ---------------------------------------------------------------------------
-constexpr int PR = 64;  // probe rows handled per CTA
-constexpr int KC = 32;  // keys per chunk
-
-template <int D>
-__global__ void __launch_bounds__(256) k_probe_attn(const __nv_bfloat16* __restrict__ Q,
-                                                   const __nv_bfloat16* __restrict__ K,
-                                                   const __nv_bfloat16* __restrict__ V, int N, int Gk, int Gq,
-                                                   int P, const int* __restrict__ probe_idx,
-                                                   const int* __restrict__ probe_grp,
-                                                   const int* __restrict__ label_k,
-                                                   const unsigned char* __restrict__ route, int keys_per_split,
-                                                   float scale_log2, float* __restrict__ part_o,
-                                                   float* __restrict__ part_ml) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  float* qs = reinterpret_cast<float*>(smem);      // [PR][D]
-  float* ks = qs + PR * D;                          // [D][KC]
-  float* vs = ks + D * KC;                          // [KC][D]
-  float* pd = vs + KC * D;                          // [PR][KC+1]
-  float* ps = pd + PR * (KC + 1);                   // [PR][KC+1]
-  float* st = ps + PR * (KC + 1);                   // [PR][8]: m_d l_d a_d m_s l_s a_s
-  int* klab = reinterpret_cast<int*>(st + PR * 8);  // [KC]
-  unsigned char* rt = reinterpret_cast<unsigned char*>(klab + KC);  // [PR][Gk]
-  const int split = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const size_t head = (size_t)bh * N;
-  for (int e = tid; e < PR * D; e += 256) {
-    int r = e / D, c = e - r * D;
-    int row = r < P ? probe_idx[(size_t)bh * P + r] : -1;
-    qs[e] = row >= 0 ? bf2f(Q[(head + row) * D + c]) : 0.f;
-  }
-  for (int e = tid; e < PR * Gk; e += 256) {
-    int r = e / Gk, g = e - r * Gk;
-    int a = r < P ? probe_grp[(size_t)bh * P + r] : -1;
-    rt[e] = a >= 0 ? route[((size_t)bh * Gq + a) * Gk + g] : 0;
-  }
-  for (int r = tid; r < PR; r += 256) {
-    st[r * 8 + 0] = -INFINITY; st[r * 8 + 1] = 0.f;
-    st[r * 8 + 3] = -INFINITY; st[r * 8 + 4] = 0.f;
-  }
-  const int orow = tid >> 2;       // output row owned in the PV stage
-  const int ocol = tid & 3;        // columns ocol + 4 m
-  float od[D / 4], os[D / 4];
-#pragma unroll
-  for (int m = 0; m < D / 4; ++m) od[m] = os[m] = 0.f;
-  const int k0 = split * keys_per_split, k1 = min(N, k0 + keys_per_split);
-  __syncthreads();
-  for (int kc = k0; kc < k1; kc += KC) {
-    const int nk = min(KC, k1 - kc);
-    for (int e = tid; e < KC * D; e += 256) {
-      int j = e / D, c = e - j * D;
-      bool ok = j < nk;
-      ks[c * KC + j] = ok ? bf2f(K[(head + kc + j) * D + c]) : 0.f;
-      vs[j * D + c] = ok ? bf2f(V[(head + kc + j) * D + c]) : 0.f;
-    }
-    if (tid < KC) klab[tid] = tid < nk ? label_k[head + kc + tid] : -1;
-    __syncthreads();
-    // scores: warp w owns rows w + 8 i, lane = key
-    for (int i = 0; i < PR / 8; ++i) {
-      const int r = warp + 8 * i;
-      float sc = 0.f;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) sc = fmaf(qs[r * D + c], ks[c * KC + lane], sc);
-      const bool valid = lane < nk;
-      const int lb = klab[lane];
-      const bool routed = valid && lb >= 0 && lb < Gk && rt[r * Gk + lb];
-      const float sd = valid ? sc * scale_log2 : -INFINITY;
-      const float ss = routed ? sc * scale_log2 : -INFINITY;
-      // dense
-      float mo = st[r * 8 + 0];
-      float mn = fmaxf(mo, warp_max(sd));
-      float p = valid ? ex2f(sd - mn) : 0.f;
-      float al = (mo == -INFINITY) ? 0.f : ex2f(mo - mn);
-      float sum = warp_sum(p);
-      pd[r * (KC + 1) + lane] = p;
-      // routed
-      float mos = st[r * 8 + 3];
-      float mns = fmaxf(mos, warp_max(ss));
-      float q = (routed && mns != -INFINITY) ? ex2f(ss - mns) : 0.f;
-      float als = (mos == -INFINITY) ? 0.f : ex2f(mos - mns);
-      float sums = warp_sum(q);
-      ps[r * (KC + 1) + lane] = q;
-      __syncwarp();
-      if (lane == 0) {
-        st[r * 8 + 0] = mn; st[r * 8 + 1] = st[r * 8 + 1] * al + sum; st[r * 8 + 2] = al;
-        st[r * 8 + 3] = mns; st[r * 8 + 4] = st[r * 8 + 4] * als + sums; st[r * 8 + 5] = als;
-      }
-    }
-    __syncthreads();
-    {
-      const float ad = st[orow * 8 + 2], as_ = st[orow * 8 + 5];
-#pragma unroll
-      for (int m = 0; m < D / 4; ++m) { od[m] *= ad; os[m] *= as_; }
-      for (int j = 0; j < nk; ++j) {
-        const float a1 = pd[orow * (KC + 1) + j], a2 = ps[orow * (KC + 1) + j];
-#pragma unroll
-        for (int m = 0; m < D / 4; ++m) {
-          const float v = vs[j * D + ocol + 4 * m];
-          od[m] = fmaf(a1, v, od[m]);
-          os[m] = fmaf(a2, v, os[m]);
-        }
-      }
-    }
-    __syncthreads();
-  }
-  const size_t base = ((size_t)bh * gridDim.x + split) * PR;
-#pragma unroll
-  for (int m = 0; m < D / 4; ++m) {
-    part_o[((base + orow) * 2 + 0) * D + ocol + 4 * m] = od[m];
-    part_o[((base + orow) * 2 + 1) * D + ocol + 4 * m] = os[m];
-  }
-  if (ocol == 0) {
-    part_ml[(base + orow) * 4 + 0] = st[orow * 8 + 0];
-    part_ml[(base + orow) * 4 + 1] = st[orow * 8 + 1];
-    part_ml[(base + orow) * 4 + 2] = st[orow * 8 + 3];
-    part_ml[(base + orow) * 4 + 3] = st[orow * 8 + 4];
-  }
-}
+constexpr int PR = 64;  // probe rows per split in the partial buffers
 
 // ---------------------------------------------------------------------------
 // Merge the key splits.  grid = BH, block = 256.
@@ -288,51 +169,34 @@ __global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_d
   for (int i = tid; i < PR; i += 256)
     if (rank[i] < Rk) ridx[rank[i]] = i;
   __syncthreads();
-  // subspace basis
+  // subspace basis: v_j = R^T u_i / ||R^T u_i|| for the j-th largest eigenvalue i of R R^T
+  // (in fp64 these are orthogonal to ~1e-10 whenever sigma_i > 1e-6 sigma_max; smaller
+  // singular values give zero columns)
   double lam0 = 0.0;
   for (int i = 0; i < PR; ++i) lam0 = fmax(lam0, G[i * LDP + i]);
   const double smax = sqrt(fmax(lam0, 0.0));
-  for (int j = 0; j < Rk; ++j) {
+  for (int e = tid; e < D * Rk; e += 256) {
+    const int c = e / Rk, j = e - c * Rk;
+    const int i = ridx[j];
+    const double sj = sqrt(fmax(G[i * LDP + i], 0.0));
+    double v = 0.0;
+    if (smax > 0.0 && sj > 1e-6 * smax)
+      for (int p = 0; p < PR; ++p) v += (double)Rm[p * D + c] * U[p * LDP + i];
+    Vr[c * Rk + j] = v;
+  }
+  __syncthreads();
+  for (int j = tid; j < Rk; j += 256) {
     const int i = ridx[j];
     const double sj = sqrt(fmax(G[i * LDP + i], 0.0));
     const bool keep = smax > 0.0 && sj > 1e-6 * smax;
-    for (int c = tid; c < D; c += 256) {
-      double v = 0.0;
-      if (keep)
-        for (int p = 0; p < PR; ++p) v += (double)Rm[p * D + c] * U[p * LDP + i];
-      Vr[c * Rk + j] = v;
-    }
-    if (tid == 0 && sigma_out) sigma_out[(size_t)bh * Rk + j] = keep ? (float)sj : 0.f;
-    __syncthreads();
-    // Gram-Schmidt against earlier columns (twice), then normalise
-    for (int pass = 0; pass < 2 && keep; ++pass) {
-      for (int k = 0; k < j; ++k) {
-        double dot = 0.0;
-        for (int c = tid; c < D; c += 256) dot += Vr[c * Rk + j] * Vr[c * Rk + k];
-        dot = warp_sum_d(dot);
-        if ((tid & 31) == 0) red[tid >> 5] = dot;
-        __syncthreads();
-        dot = 0.0;
-        for (int w = 0; w < 8; ++w) dot += red[w];
-        __syncthreads();
-        for (int c = tid; c < D; c += 256) Vr[c * Rk + j] -= dot * Vr[c * Rk + k];
-        __syncthreads();
-      }
-    }
-    if (keep) {
-      double nn = 0.0;
-      for (int c = tid; c < D; c += 256) nn += Vr[c * Rk + j] * Vr[c * Rk + j];
-      nn = warp_sum_d(nn);
-      if ((tid & 31) == 0) red[tid >> 5] = nn;
-      __syncthreads();
-      nn = 0.0;
-      for (int w = 0; w < 8; ++w) nn += red[w];
-      __syncthreads();
-      const double inv = nn > 0.0 ? 1.0 / sqrt(nn) : 0.0;
-      for (int c = tid; c < D; c += 256) Vr[c * Rk + j] *= inv;
-    }
-    __syncthreads();
+    if (sigma_out) sigma_out[(size_t)bh * Rk + j] = keep ? (float)sj : 0.f;
+    double nn = 0.0;
+    for (int c = 0; c < D; ++c) nn += Vr[c * Rk + j] * Vr[c * Rk + j];
+    cs[j] = nn > 0.0 ? 1.0 / sqrt(nn) : 0.0;
   }
+  __syncthreads();
+  for (int e = tid; e < D * Rk; e += 256) Vr[e] *= cs[e % Rk];
+  __syncthreads();
   // Y = R Vr, means
   for (int e = tid; e < P * Rk; e += 256) {
     const int p = e / Rk, j = e - p * Rk;
@@ -425,48 +289,145 @@ __global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_d
 }
 
 // ---------------------------------------------------------------------------
-// Correction O = x + b_full + (x W) V_r^T for every row (probe rows are then
-// overwritten by k_probe_scatter).  grid = (ceil(N/64), BH), block = 256.
+// Correction on the tensor cores: O = x + b_full + x B with B = W V_r^T (d x d).
+// Each CTA forms B^T[n][k] = sum_j V_r[n][j] W[k][j] once (fp32), splits it into bf16
+// hi + lo (K-major tile), then for every 128-row tile of O_sparse computes x B with two
+// tcgen05 MMAs (exact bf16 products, fp32 accumulation) and writes x + b + x B in bf16.
+// Rows are read into shared memory before any is written, so O may alias O_sparse.
+// grid = (RC_CTAS, BH), block = 128.
 // ---------------------------------------------------------------------------
+constexpr int RC_CTAS = 16;
+
 template <int D>
-__global__ void __launch_bounds__(256) k_reconstruct(const __nv_bfloat16* __restrict__ Os, int N, int Rk,
-                                                    const float* __restrict__ W, const float* __restrict__ Vr,
-                                                    const float* __restrict__ bfull, __nv_bfloat16* __restrict__ O) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  float* xs = reinterpret_cast<float*>(smem);  // [64][D+1]
-  float* ws = xs + 64 * (D + 1);               // [D][Rk]
-  float* vt = ws + D * Rk;                     // [Rk][D]  (V_r transposed)
-  float* ts = vt + Rk * D;                     // [64][Rk+1]
-  float* bf = ts + 64 * (Rk + 1);              // [D]
-  const int bh = blockIdx.y, n0 = blockIdx.x * 64, tid = threadIdx.x;
-  const int nr = min(64, N - n0);
-  for (int e = tid; e < D * Rk; e += 256) {
-    ws[e] = W[(size_t)bh * D * Rk + e];
-    const int c = e / Rk, j = e - c * Rk;
-    vt[j * D + c] = Vr[(size_t)bh * D * Rk + e];
+__global__ void __launch_bounds__(128) k_reconstruct_tc(const __nv_bfloat16* __restrict__ Os, int N, int Rk,
+                                                       const float* __restrict__ W, const float* __restrict__ Vr,
+                                                       const float* __restrict__ bfull,
+                                                       __nv_bfloat16* __restrict__ O, int* err) {
+  using namespace spr::tc;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw = su32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* smem = smem_raw + (base - raw);
+  constexpr uint32_t kT = (uint32_t)128 * D * 2;   // X tile (128 rows)
+  constexpr uint32_t kB = (uint32_t)D * D * 2;     // B^T tile (D rows)
+  const uint32_t sX = base, sBh = base + kT, sBl = sBh + kB;
+  float* sb = reinterpret_cast<float*>(smem + kT + 2 * kB);   // [D]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sb + D);
+  int* sMisc = reinterpret_cast<int*>(bar + 1);
+  volatile int* abort_flag = sMisc + 1;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int bh = blockIdx.y;
+  const size_t head = (size_t)bh * N;
+  constexpr int CPR = D / 8;
+  const float* Wh = W + (size_t)bh * D * Rk;
+  const float* Vh = Vr + (size_t)bh * D * Rk;
+  // stage V_r [n][j] and W^T [j][k] in the (still unused) X-tile region when they fit
+  const bool staged = (size_t)2 * D * Rk * 4 <= kT;
+  float* sV = reinterpret_cast<float*>(smem);
+  float* sWt = sV + D * Rk;
+  if (staged) {
+    for (int e = tid; e < D * Rk; e += 128) {
+      sV[e] = Vh[e];
+      const int k = e / Rk, j = e - k * Rk;
+      sWt[j * D + k] = Wh[e];
+    }
+    __syncthreads();
   }
-  for (int c = tid; c < D; c += 256) bf[c] = bfull[(size_t)bh * D + c];
-  const __nv_bfloat16* src = Os + ((size_t)bh * N + n0) * D;
-  for (int e = tid; e < nr * D; e += 256) {
-    const int r = e / D, c = e - r * D;
-    xs[r * (D + 1) + c] = bf2f(src[e]);
+  // B^T rows n, columns k, stored as a K-major 128B-swizzled tile of D rows
+  for (int e = tid; e < D * D; e += 128) {
+    const int n = e / D, k = e - n * D;
+    float acc = 0.f;
+    if (staged)
+      for (int j = 0; j < Rk; ++j) acc = fmaf(sV[n * Rk + j], sWt[j * D + k], acc);
+    else
+      for (int j = 0; j < Rk; ++j) acc = fmaf(Vh[n * Rk + j], Wh[k * Rk + j], acc);
+    const __nv_bfloat16 hi = __float2bfloat16(acc);
+    const __nv_bfloat16 lo = __float2bfloat16(acc - __bfloat162float(hi));
+    const uint32_t off = tile_off(n, k >> 3, D) + (k & 7) * 2;
+    *reinterpret_cast<__nv_bfloat16*>(smem + kT + off) = hi;
+    *reinterpret_cast<__nv_bfloat16*>(smem + kT + kB + off) = lo;
   }
+  for (int c = tid; c < D; c += 128) sb[c] = bfull[(size_t)bh * D + c];
   __syncthreads();
-  for (int e = tid; e < nr * Rk; e += 256) {
-    const int r = e / Rk, j = e - r * Rk;
-    float t = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < D; ++c) t = fmaf(xs[r * (D + 1) + c], ws[c * Rk + j], t);
-    ts[r * (Rk + 1) + j] = t;
+  if (tid == 0) {
+    sMisc[1] = 0;
+    mbar_init(su32(bar), 1);
+    fence_barrier_init();
   }
+  if (warp == 0) {
+    tc_alloc(su32(&sMisc[0]), 128);
+    tc_relinquish();
+  }
+  fence_proxy_async();
+  tc_fence_before();
   __syncthreads();
-  __nv_bfloat16* dst = O + ((size_t)bh * N + n0) * D;
-  for (int e = tid; e < nr * D; e += 256) {
-    const int r = e / D, c = e - r * D;
-    float o = xs[r * (D + 1) + c] + bf[c];
-    for (int j = 0; j < Rk; ++j) o = fmaf(ts[r * (Rk + 1) + j], vt[j * D + c], o);
-    dst[e] = __float2bfloat16(o);
+  tc_fence_after();
+  const uint32_t tmem = (uint32_t)sMisc[0];
+  constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(D >> 3) << 17) | (8u << 24);
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int ntiles = (N + 127) / 128;
+  int phase = 0;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int n0 = tile * 128;
+    for (int e = tid; e < 128 * CPR; e += 128) {
+      const int r = e / CPR, c = e - r * CPR;
+      const bool ok = n0 + r < N;
+      cp_async16(sX + tile_off(r, c, 128), Os + (head + (ok ? n0 + r : 0)) * D + c * 8, ok);
+    }
+    cp_async_wait_all();
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
+        const uint32_t ob = (k >> 2) * (D * 128) + (k & 3) * 32;
+        tc_mma(tmem, sdesc(sX + ox, 16, 1024), sdesc(sBh + ob, 16, 1024), idesc, k > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < D / 16; ++k) {
+        const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
+        const uint32_t ob = (k >> 2) * (D * 128) + (k & 3) * 32;
+        tc_mma(tmem, sdesc(sX + ox, 16, 1024), sdesc(sBl + ob, 16, 1024), idesc, 1u);
+      }
+      tc_commit(su32(bar));
+    }
+    const bool ok = __syncthreads_and(bounded_wait(su32(bar), phase & 1, abort_flag, err) ? 1 : 0) != 0;
+    ++phase;
+    if (!ok) break;
+    tc_fence_after();
+    const int row = n0 + tid;
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t acc[32];
+      tc_ld32(tmem + lane_off + c0, acc);
+      uint32_t w[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 xv = *reinterpret_cast<const uint4*>(smem + tile_off(tid, (c0 >> 3) + q, 128));
+        const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 x = __bfloat1622float2(x2[e]);
+          const int c = c0 + q * 8 + 2 * e;
+          w[q * 4 + e] = pack_bf16(x.x + sb[c] + __uint_as_float(acc[q * 8 + 2 * e]),
+                                   x.y + sb[c + 1] + __uint_as_float(acc[q * 8 + 2 * e + 1]));
+        }
+      }
+      if (row < N) {
+        uint4* dst = reinterpret_cast<uint4*>(O + (head + row) * D + c0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tc_dealloc(tmem, 128);
 }
 
 __global__ void k_probe_scatter(const int* __restrict__ probe_idx, const float* __restrict__ o_dense, int N, int P,
@@ -557,31 +518,12 @@ int probe_splits(int N) {
   return s < 1 ? 1 : (s > 64 ? 64 : s);
 }
 
-size_t probe_attn_smem(int D, int Gk) {
-  return (size_t)(PR * D + D * KC + KC * D + 2 * PR * (KC + 1) + PR * 8 + KC) * 4 + (size_t)PR * Gk;
-}
-
 cudaError_t launch_probe_attn(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk, int Gq,
                               int P, const int* probe_idx, const int* probe_grp, const int* label_k,
-                              const unsigned char* route, float scale_log2, float* part_o, float* part_ml,
+                              const unsigned char* route, float scale_log2, float* part_o, float* part_ml, int* err,
                               cudaStream_t st) {
-  const int S = probe_splits(N);
-  int kps = (N + S - 1) / S;
-  kps = (kps + KC - 1) / KC * KC;
-  const size_t sm = probe_attn_smem(D, Gk);
-  dim3 grid(S, BH);
-  if (D == 64) {
-    cudaFuncSetAttribute(k_probe_attn<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_probe_attn<64><<<grid, 256, sm, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
-                                            (const __nv_bfloat16*)V, N, Gk, Gq, P, probe_idx, probe_grp,
-                                            label_k, route, kps, scale_log2, part_o, part_ml);
-  } else {
-    cudaFuncSetAttribute(k_probe_attn<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_probe_attn<128><<<grid, 256, sm, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
-                                             (const __nv_bfloat16*)V, N, Gk, Gq, P, probe_idx, probe_grp,
-                                             label_k, route, kps, scale_log2, part_o, part_ml);
-  }
-  return cudaGetLastError();
+  return launch_probe_tc(Q, K, V, BH, N, D, Gk, Gq, P, probe_idx, probe_grp, label_k, route, scale_log2,
+                         probe_splits(N), part_o, part_ml, err, st);
 }
 
 // Split-count-explicit variants (the key-split count S is chosen by the caller instead
@@ -590,22 +532,8 @@ cudaError_t launch_probe_attn_splits(const void* Q, const void* K, const void* V
                                      int Gq, int P, const int* probe_idx, const int* probe_grp, const int* label_k,
                                      const unsigned char* route, float scale_log2, int S, float* part_o,
                                      float* part_ml, cudaStream_t st) {
-  int kps = (N + S - 1) / S;
-  kps = (kps + KC - 1) / KC * KC;
-  const size_t sm = probe_attn_smem(D, Gk);
-  dim3 grid(S, BH);
-  if (D == 64) {
-    cudaFuncSetAttribute(k_probe_attn<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_probe_attn<64><<<grid, 256, sm, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
-                                            (const __nv_bfloat16*)V, N, Gk, Gq, P, probe_idx, probe_grp,
-                                            label_k, route, kps, scale_log2, part_o, part_ml);
-  } else {
-    cudaFuncSetAttribute(k_probe_attn<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_probe_attn<128><<<grid, 256, sm, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
-                                             (const __nv_bfloat16*)V, N, Gk, Gq, P, probe_idx, probe_grp,
-                                             label_k, route, kps, scale_log2, part_o, part_ml);
-  }
-  return cudaGetLastError();
+  return launch_probe_tc(Q, K, V, BH, N, D, Gk, Gq, P, probe_idx, probe_grp, label_k, route, scale_log2, S, part_o,
+                         part_ml, nullptr, st);
 }
 
 cudaError_t launch_probe_combine_splits(const float* part_o, const float* part_ml, int BH, int S, int P, int D,
@@ -642,14 +570,16 @@ cudaError_t launch_probe_fit(const float* o_dense, const float* o_sparse, int BH
 
 cudaError_t launch_reconstruct(const void* Os, int BH, int N, int D, int Rk, const float* W, const float* Vr,
                                const float* bfull, void* O, cudaStream_t st) {
-  const size_t sm = (size_t)(64 * (D + 1) + 2 * D * Rk + 64 * (Rk + 1) + D) * 4;
-  dim3 grid(ceil_div(N, 64), BH);
+  const size_t sm = 1024 + (size_t)128 * D * 2 + 2 * (size_t)D * D * 2 + (size_t)D * 4 + 8 + 16;
+  dim3 grid(RC_CTAS, BH);
   if (D == 64) {
-    cudaFuncSetAttribute(k_reconstruct<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_reconstruct<64><<<grid, 256, sm, st>>>((const __nv_bfloat16*)Os, N, Rk, W, Vr, bfull, (__nv_bfloat16*)O);
+    cudaFuncSetAttribute(k_reconstruct_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_reconstruct_tc<64><<<grid, 128, sm, st>>>((const __nv_bfloat16*)Os, N, Rk, W, Vr, bfull, (__nv_bfloat16*)O,
+                                                nullptr);
   } else {
-    cudaFuncSetAttribute(k_reconstruct<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_reconstruct<128><<<grid, 256, sm, st>>>((const __nv_bfloat16*)Os, N, Rk, W, Vr, bfull, (__nv_bfloat16*)O);
+    cudaFuncSetAttribute(k_reconstruct_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    k_reconstruct_tc<128><<<grid, 128, sm, st>>>((const __nv_bfloat16*)Os, N, Rk, W, Vr, bfull, (__nv_bfloat16*)O,
+                                                 nullptr);
   }
   return cudaGetLastError();
 }
