@@ -66,10 +66,15 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            # the timed region starts once the sampler is producing lines
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 5.0:
+                time.sleep(0.01)
+            self.lines.clear()
         except Exception:
             self.proc = None
         return self
@@ -214,10 +219,10 @@ def run_cuda(args):
     nq = torch.diff(part["qoff"].long(), dim=1)
     nk = torch.diff(part["koff"].long(), dim=1)
     routed_pairs = int((nq[:, :, None] * nk[:, None, :] * part["route"].long()).sum().item())
-    # MMA-issued pairs: q-tiles of 128 rows x routed key rows padded to 64-row chunks
+    # MMA-issued pairs: q-tiles of 128 rows x routed key rows padded to 128-key chunks
     ntile = (nq + 127) // 128
     rk = (nk[:, None, :] * part["route"].long()).sum(-1)
-    issued_pairs = int((ntile * 128 * ((rk + 63) // 64) * 64).sum().item())
+    issued_pairs = int((ntile * 128 * ((rk + 127) // 128) * 128).sum().item())
     attn_flops = 4.0 * d * routed_pairs
     attn_ms = stage_ms[1]
     pk = _peaks()
@@ -399,7 +404,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=30.0)

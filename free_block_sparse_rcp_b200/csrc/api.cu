@@ -50,7 +50,7 @@ struct Layout {
   // header
   size_t err;
   // partition
-  size_t sample_idx, metric, eigval, eigvec, proj, m_k, nu_k, key_init, C, m_q, nu_q, query_init, bias, wnorm,
+  size_t sample_idx, metric, eigval, eigvec, proj, eig_lu, m_k, nu_k, key_init, C, m_q, nu_q, query_init, bias, wnorm,
       w_hi, w_lo, flag_count, flag_rows, mass, order, cm, cc, alpha;
   // attend
   size_t rlist, rcum, rcnt, tiles, tile_count;
@@ -82,6 +82,7 @@ Layout make_layout(const sparsepr_params& p) {
   L.eigval = take(BH * re * 4);
   L.eigvec = take(BH * d * re * 4);
   L.proj = take(BH * d * re * 4);
+  L.eig_lu = take(BH * 3 * d * re * 8);
   const size_t GPmax = (size_t)kmeans_gp(p.n_kgroups > p.n_qgroups ? p.n_kgroups : p.n_qgroups);
   L.m_k = take(BH * Gk * d * 4);
   L.nu_k = take(BH * Gk * L.DTk * 4);
@@ -146,6 +147,8 @@ sparsepr_status check_params(const sparsepr_params* p) {
   const int pmax = p->N < 64 ? p->N : 64;
   if (p->n_probes < 1 || p->n_probes > pmax) return failv(SPARSEPR_EINVAL, "n_probes must be in [1, min(N,64)]", p->n_probes);
   if (p->eig_rank < 1 || p->eig_rank > p->d) return failv(SPARSEPR_EINVAL, "eig_rank must be in [1, d]", p->eig_rank);
+  if (p->eig_rank > 64 || metric_eigen_smem(p->d, p->eig_rank) > kSmemLimit)
+    return failv(SPARSEPR_EUNSUPPORTED, "eig_rank > 64 not built (single-CTA eigensolver)", p->eig_rank);
   if (p->sub_rank < 1 || p->sub_rank > p->n_probes || p->sub_rank > p->d)
     return failv(SPARSEPR_EINVAL, "sub_rank must be in [1, min(d, n_probes)]", p->sub_rank);
   if (p->kmeans_iters < 1 || p->kmeans_iters > 64) return failv(SPARSEPR_EINVAL, "kmeans_iters must be in [1, 64]", p->kmeans_iters);
@@ -208,7 +211,8 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
   float* metric = at<float>(ws, L.metric);
   float* proj = at<float>(ws, L.proj);
   SPR_LAUNCH(launch_sample_metric(Q, BH, N, d, p.n_samples, p.seed, metric, at<int>(ws, L.sample_idx), err, st));
-  SPR_LAUNCH(launch_metric_eigen(metric, BH, d, re, at<float>(ws, L.eigval), at<float>(ws, L.eigvec), proj, st));
+  SPR_LAUNCH(launch_metric_eigen(metric, BH, d, re, at<float>(ws, L.eigval), at<float>(ws, L.eigvec), proj,
+                                 at<double>(ws, L.eig_lu), st));
   if (tr && tr->key_coords) SPR_LAUNCH(launch_key_coords(K, BH, N, d, re, proj, tr->key_coords, st));
   float* bias = at<float>(ws, L.bias);
   float* wnorm = at<float>(ws, L.wnorm);

@@ -11,7 +11,7 @@
 //   route             shared alpha by bisection under the pair budget
 //   block mask        tile-level view of the route on the permuted layout
 #include "common.cuh"
-#include "jacobi.cuh"
+#include "symeig.cuh"
 #include "kernels.h"
 
 namespace spr {
@@ -68,42 +68,35 @@ __global__ void __launch_bounds__(256) k_sample_metric(const __nv_bfloat16* __re
 }
 
 // ---------------------------------------------------------------------------
-// Leading eigenpairs of M_K.  grid = BH, block = 1024.
-// Writes eigval [BH, R] (clamped >= 0), eigvec [BH, D, R] and the projector
-// P = U_R Lambda_R^{1/2} [BH, D, R] used for the key coordinates.
+// Leading eigenpairs of M_K (fp64, Householder + multisection + inverse iteration).
+// grid = BH, block = 1024.  Writes eigval [BH, R] (clamped >= 0), eigvec [BH, D, R] and
+// the projector P = U_R Lambda_R^{1/2} [BH, D, R].  lu: BH * 3 * D * R doubles of scratch.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(1024) k_metric_eigen(const float* __restrict__ metric, int R,
                                                      float* __restrict__ eigval, float* __restrict__ eigvec,
-                                                     float* __restrict__ proj) {
+                                                     float* __restrict__ proj, double* __restrict__ lu) {
   extern __shared__ __align__(16) unsigned char smem[];
   constexpr int LD = D + 1;
-  float* A = reinterpret_cast<float*>(smem);
-  float* V = A + D * LD;
-  float* cs = V + D * LD;
-  float* red = cs + D;
-  int* pr = reinterpret_cast<int*>(red + 64);
-  int* rank = pr + D;
+  const int ldz = R + 1;
+  double* A = reinterpret_cast<double*>(smem);  // [D][D+1]
+  double* Z = A + D * LD;                       // [D][R+1]
+  double* lam = Z + D * ldz;                    // [64]
+  double* sc = lam + 64;                        // SymEigScratch<D>
   const int bh = blockIdx.x;
   for (int i = threadIdx.x; i < D * D; i += blockDim.x) {
-    int r = i / D, c = i - r * D;
-    A[r * LD + c] = metric[(size_t)bh * D * D + i];
+    const int r = i / D, c = i - r * D;
+    A[r * LD + c] = (double)metric[(size_t)bh * D * D + i];
   }
   __syncthreads();
-  jacobi_eigen<float, D>(A, V, cs, pr, red, 10, 2e-5f);
-  eigen_ranks<float, D>(A, rank);
-  for (int i = threadIdx.x; i < D; i += blockDim.x) {
-    int k = rank[i];
-    if (k < R) {
-      float lam = fmaxf(A[i * LD + i], 0.f);
-      eigval[(size_t)bh * R + k] = lam;
-      float sl = sqrtf(lam);
-      for (int c = 0; c < D; ++c) {
-        float u = V[c * LD + i];
-        eigvec[((size_t)bh * D + c) * R + k] = u;
-        proj[((size_t)bh * D + c) * R + k] = u * sl;
-      }
-    }
+  sym_top_eigen<D>(A, R, Z, ldz, lam, sc, lu + (size_t)bh * 3 * D * R);
+  for (int e = threadIdx.x; e < D * R; e += blockDim.x) {
+    const int c = e / R, k = e - c * R;
+    const double l = fmax(lam[k], 0.0);
+    const double u = Z[c * ldz + k];
+    if (c == 0) eigval[(size_t)bh * R + k] = (float)l;
+    eigvec[(size_t)bh * D * R + e] = (float)u;
+    proj[(size_t)bh * D * R + e] = (float)(u * sqrt(l));
   }
 }
 
@@ -406,15 +399,20 @@ cudaError_t launch_sample_metric(const void* Q, int BH, int N, int D, int Ms, ui
   return cudaGetLastError();
 }
 
+size_t metric_eigen_smem(int D, int R) {
+  const size_t sc = D == 64 ? SymEigScratch<64>::kDoubles : SymEigScratch<128>::kDoubles;
+  return ((size_t)D * (D + 1) + (size_t)D * (R + 1) + 64 + sc) * 8;
+}
+
 cudaError_t launch_metric_eigen(const float* metric, int BH, int D, int R, float* eigval, float* eigvec,
-                                float* proj, cudaStream_t st) {
-  size_t sm = (size_t)(2 * D * (D + 1) + D + 64) * 4 + (size_t)(2 * D) * 4;
+                                float* proj, double* lu, cudaStream_t st) {
+  const size_t sm = metric_eigen_smem(D, R);
   if (D == 64) {
     cudaFuncSetAttribute(k_metric_eigen<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_metric_eigen<64><<<BH, 1024, sm, st>>>(metric, R, eigval, eigvec, proj);
+    k_metric_eigen<64><<<BH, 1024, sm, st>>>(metric, R, eigval, eigvec, proj, lu);
   } else {
     cudaFuncSetAttribute(k_metric_eigen<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_metric_eigen<128><<<BH, 1024, sm, st>>>(metric, R, eigval, eigvec, proj);
+    k_metric_eigen<128><<<BH, 1024, sm, st>>>(metric, R, eigval, eigvec, proj, lu);
   }
   return cudaGetLastError();
 }

@@ -3,7 +3,7 @@
 // 64 probe rows per head drawn evenly from every query group, ridge regression,
 // correction inside the leading singular directions of the probe residuals).
 #include "common.cuh"
-#include "jacobi.cuh"
+#include "symeig.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
 
@@ -27,7 +27,6 @@ __global__ void __launch_bounds__(256) k_probe_pick(const int* __restrict__ perm
   int* draw = order + Gq;                     // [P]
   int* mkey = draw + 64;                      // [256]
   int* mval = mkey + 256;                     // [256]
-  int* red = mval + 256;                      // [8]
   const int bh = blockIdx.x, tid = threadIdx.x;
   const int* qo = qoff + (size_t)bh * (Gq + 1);
   for (int a = tid; a < Gq; a += blockDim.x) { size[a] = qo[a + 1] - qo[a]; alloc[a] = 0; }
@@ -116,13 +115,28 @@ __global__ void __launch_bounds__(256) k_probe_combine(const float* __restrict__
 
 // ---------------------------------------------------------------------------
 // Residual subspace + ridge fit, one CTA per head (fp64 arithmetic).
-//   R = O_dense - O_sparse (P x D); Gram R R^T -> Jacobi -> u_i, sigma_i;
-//   v_i = R^T u_i normalised and re-orthogonalised (zero when sigma_i <= 1e-6 sigma_0);
-//   Y = R V_r; centred dual ridge  W = Xc^T (Xc Xc^T + lam I)^-1 Yc, b = ybar - xbar W.
-// grid = BH, block = 256.
+//   R = O_dense - O_sparse (P x D); top eigenpairs u_i, sigma_i^2 of the Gram R R^T
+//   (Householder + multisection + inverse iteration); v_i = R^T u_i normalised (zero when
+//   sigma_i <= 1e-6 sigma_0); Y = R V_r; centred dual ridge
+//   W = Xc^T (Xc Xc^T + lam I)^-1 Yc, b = ybar - xbar W.
+// grid = BH, block = FIT_THREADS.
 // ---------------------------------------------------------------------------
+constexpr int FIT_THREADS = 1024;
+
 template <int D>
-__global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_dense,
+struct FitLayout {
+  // doubles: G [PR][PR+1] (Gram -> Cholesky -> W), Z [PR][Rk+1], lam [64], eigen scratch,
+  // X = max(3 PR Rk (solver scratch), D Rk + PR Rk (V_r, Y)), xbar [D], ybar, bsub, cs [64 each];
+  // then floats Rm, Xm [PR][D]
+  static size_t doubles(int Rk) {
+    const size_t x = (size_t)3 * PR * Rk > (size_t)(D + PR) * Rk ? (size_t)3 * PR * Rk : (size_t)(D + PR) * Rk;
+    return (size_t)PR * (PR + 1) + (size_t)PR * (Rk + 1) + 64 + SymEigScratch<PR>::kDoubles + x + D + 3 * 64;
+  }
+  static size_t bytes(int Rk) { return doubles(Rk) * 8 + (size_t)2 * PR * D * 4; }
+};
+
+template <int D>
+__global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restrict__ o_dense,
                                                   const float* __restrict__ o_sparse, int P, int Rk,
                                                   double lam, float* __restrict__ Vr_out,
                                                   float* __restrict__ W_out, float* __restrict__ bfull_out,
@@ -130,23 +144,24 @@ __global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_d
                                                   float* __restrict__ bsub_out) {
   extern __shared__ __align__(16) unsigned char smem[];
   constexpr int LDP = PR + 1;
-  double* G = reinterpret_cast<double*>(smem);   // [PR][LDP]  Gram, later Cholesky
-  double* U = G + PR * LDP;                       // [PR][LDP]  Jacobi vectors
-  double* Vr = U + PR * LDP;                      // [D][Rk]
-  double* Y = Vr + D * Rk;                        // [PR][Rk] -> solution
-  double* xbar = Y + PR * Rk;                     // [D]
-  double* ybar = xbar + D;                        // [64]
-  double* bsub = ybar + 64;                       // [64]
-  double* cs = bsub + 64;                         // [PR]
-  double* red = cs + PR;                          // [64]
-  float* Rm = reinterpret_cast<float*>(red + 64); // [PR][D]
-  float* Xm = Rm + PR * D;                        // [PR][D]
-  int* pr = reinterpret_cast<int*>(Xm + PR * D);  // [PR]
-  int* rank = pr + PR;                            // [PR]
-  int* ridx = rank + PR;                          // [64] eigen index of subspace column j
-  const int bh = blockIdx.x, tid = threadIdx.x;
+  const int ldz = Rk + 1;
+  const size_t xsz = (size_t)3 * PR * Rk > (size_t)(D + PR) * Rk ? (size_t)3 * PR * Rk : (size_t)(D + PR) * Rk;
+  double* G = reinterpret_cast<double*>(smem);    // [PR][LDP]  Gram, later Cholesky, later W
+  double* Z = G + PR * LDP;                        // [PR][Rk+1] eigenvectors of R R^T
+  double* ev = Z + PR * ldz;                       // [64] eigenvalues, descending
+  double* esc = ev + 64;                           // eigen scratch
+  double* X = esc + SymEigScratch<PR>::kDoubles;   // solver scratch, then V_r and Y
+  double* Vr = X;                                  // [D][Rk]
+  double* Y = Vr + D * Rk;                         // [PR][Rk] -> solution
+  double* xbar = X + xsz;                          // [D]
+  double* ybar = xbar + D;                         // [64]
+  double* bsub = ybar + 64;                        // [64]
+  double* cs = bsub + 64;                          // [64]
+  float* Rm = reinterpret_cast<float*>(cs + 64);   // [PR][D]
+  float* Xm = Rm + PR * D;                         // [PR][D]
+  const int bh = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
   // the Gram is padded to PR x PR with zero rows (P <= PR): padding adds zero eigenvalues only
-  for (int e = tid; e < PR * D; e += 256) {
+  for (int e = tid; e < PR * D; e += nt) {
     const int r = e / D;
     float od = 0.f, os = 0.f;
     if (r < P) {
@@ -157,37 +172,31 @@ __global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_d
     Xm[e] = os;
   }
   __syncthreads();
-  for (int e = tid; e < PR * PR; e += 256) {
+  for (int e = tid; e < PR * PR; e += nt) {
     const int i = e / PR, j = e - i * PR;
+    if (j > i) continue;
     double s = 0.0;
     for (int c = 0; c < D; ++c) s += (double)Rm[i * D + c] * (double)Rm[j * D + c];
     G[i * LDP + j] = s;
+    G[j * LDP + i] = s;
   }
   __syncthreads();
-  jacobi_eigen<double, PR>(G, U, cs, pr, red, 40, 1e-13);
-  eigen_ranks<double, PR>(G, rank);
-  for (int i = tid; i < PR; i += 256)
-    if (rank[i] < Rk) ridx[rank[i]] = i;
-  __syncthreads();
-  // subspace basis: v_j = R^T u_i / ||R^T u_i|| for the j-th largest eigenvalue i of R R^T
-  // (in fp64 these are orthogonal to ~1e-10 whenever sigma_i > 1e-6 sigma_max; smaller
+  sym_top_eigen<PR>(G, Rk, Z, ldz, ev, esc, X);
+  // subspace basis: v_j = R^T u_j / ||R^T u_j|| for the j-th largest eigenvalue of R R^T
+  // (in fp64 these are orthogonal to ~1e-10 whenever sigma_j > 1e-6 sigma_max; smaller
   // singular values give zero columns)
-  double lam0 = 0.0;
-  for (int i = 0; i < PR; ++i) lam0 = fmax(lam0, G[i * LDP + i]);
-  const double smax = sqrt(fmax(lam0, 0.0));
-  for (int e = tid; e < D * Rk; e += 256) {
+  const double smax = sqrt(fmax(ev[0], 0.0));
+  for (int e = tid; e < D * Rk; e += nt) {
     const int c = e / Rk, j = e - c * Rk;
-    const int i = ridx[j];
-    const double sj = sqrt(fmax(G[i * LDP + i], 0.0));
+    const double sj = sqrt(fmax(ev[j], 0.0));
     double v = 0.0;
     if (smax > 0.0 && sj > 1e-6 * smax)
-      for (int p = 0; p < PR; ++p) v += (double)Rm[p * D + c] * U[p * LDP + i];
+      for (int p = 0; p < PR; ++p) v += (double)Rm[p * D + c] * Z[p * ldz + j];
     Vr[c * Rk + j] = v;
   }
   __syncthreads();
-  for (int j = tid; j < Rk; j += 256) {
-    const int i = ridx[j];
-    const double sj = sqrt(fmax(G[i * LDP + i], 0.0));
+  for (int j = tid; j < Rk; j += nt) {
+    const double sj = sqrt(fmax(ev[j], 0.0));
     const bool keep = smax > 0.0 && sj > 1e-6 * smax;
     if (sigma_out) sigma_out[(size_t)bh * Rk + j] = keep ? (float)sj : 0.f;
     double nn = 0.0;
@@ -195,33 +204,33 @@ __global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_d
     cs[j] = nn > 0.0 ? 1.0 / sqrt(nn) : 0.0;
   }
   __syncthreads();
-  for (int e = tid; e < D * Rk; e += 256) Vr[e] *= cs[e % Rk];
+  for (int e = tid; e < D * Rk; e += nt) Vr[e] *= cs[e % Rk];
   __syncthreads();
   // Y = R Vr, means
-  for (int e = tid; e < P * Rk; e += 256) {
+  for (int e = tid; e < P * Rk; e += nt) {
     const int p = e / Rk, j = e - p * Rk;
     double s = 0.0;
     for (int c = 0; c < D; ++c) s += (double)Rm[p * D + c] * Vr[c * Rk + j];
     Y[p * Rk + j] = s;
   }
-  for (int c = tid; c < D; c += 256) {
+  for (int c = tid; c < D; c += nt) {
     double s = 0.0;
     for (int p = 0; p < P; ++p) s += (double)Xm[p * D + c];
     xbar[c] = s / P;
   }
   __syncthreads();
-  for (int j = tid; j < Rk; j += 256) {
+  for (int j = tid; j < Rk; j += nt) {
     double s = 0.0;
     for (int p = 0; p < P; ++p) s += Y[p * Rk + j];
     ybar[j] = s / P;
   }
   __syncthreads();
-  for (int e = tid; e < P * Rk; e += 256) {
+  for (int e = tid; e < P * Rk; e += nt) {
     const int p = e / Rk, j = e - p * Rk;
     Y[p * Rk + j] -= ybar[j];
   }
   // A = Xc Xc^T + lam I  (into G)
-  for (int e = tid; e < P * P; e += 256) {
+  for (int e = tid; e < P * P; e += nt) {
     const int i = e / P, j = e - i * P;
     double s = 0.0;
     for (int c = 0; c < D; ++c) s += ((double)Xm[i * D + c] - xbar[c]) * ((double)Xm[j * D + c] - xbar[c]);
@@ -233,16 +242,16 @@ __global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_d
     if (tid == 0) G[k * LDP + k] = sqrt(G[k * LDP + k]);
     __syncthreads();
     const double dkk = G[k * LDP + k];
-    for (int i = k + 1 + tid; i < P; i += 256) G[i * LDP + k] /= dkk;
+    for (int i = k + 1 + tid; i < P; i += nt) G[i * LDP + k] /= dkk;
     __syncthreads();
-    for (int e = tid; e < (P - k - 1) * (P - k - 1); e += 256) {
+    for (int e = tid; e < (P - k - 1) * (P - k - 1); e += nt) {
       const int i = k + 1 + e / (P - k - 1), j = k + 1 + e % (P - k - 1);
       if (j <= i) G[i * LDP + j] -= G[i * LDP + k] * G[j * LDP + k];
     }
     __syncthreads();
   }
   // solve L L^T Z = Yc, one right-hand side per thread
-  for (int j = tid; j < Rk; j += 256) {
+  for (int j = tid; j < Rk; j += nt) {
     for (int i = 0; i < P; ++i) {
       double s = Y[i * Rk + j];
       for (int k = 0; k < i; ++k) s -= G[i * LDP + k] * Y[k * Rk + j];
@@ -255,9 +264,9 @@ __global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_d
     }
   }
   __syncthreads();
-  // W = Xc^T Z (D x Rk) kept in the Jacobi-vector region, b = ybar - xbar W
-  double* Wd = U;
-  for (int e = tid; e < D * Rk; e += 256) {
+  // W = Xc^T Z (D x Rk, D * Rk <= PR * (PR + 1)) kept in the Cholesky region, b = ybar - xbar W
+  double* Wd = G;
+  for (int e = tid; e < D * Rk; e += nt) {
     const int c = e / Rk, j = e - c * Rk;
     double s = 0.0;
     for (int p = 0; p < P; ++p) s += ((double)Xm[p * D + c] - xbar[c]) * Y[p * Rk + j];
@@ -266,20 +275,20 @@ __global__ void __launch_bounds__(256) k_probe_fit(const float* __restrict__ o_d
     Vr_out[(size_t)bh * D * Rk + e] = (float)Vr[c * Rk + j];
   }
   __syncthreads();
-  for (int j = tid; j < Rk; j += 256) {
+  for (int j = tid; j < Rk; j += nt) {
     double s = 0.0;
     for (int c = 0; c < D; ++c) s += xbar[c] * Wd[c * Rk + j];
     bsub[j] = ybar[j] - s;
     if (bsub_out) bsub_out[(size_t)bh * Rk + j] = (float)bsub[j];
   }
   __syncthreads();
-  for (int c = tid; c < D; c += 256) {
+  for (int c = tid; c < D; c += nt) {
     double s = 0.0;
     for (int j = 0; j < Rk; ++j) s += Vr[c * Rk + j] * bsub[j];
     bfull_out[(size_t)bh * D + c] = (float)s;
   }
   if (Bmat) {
-    for (int e = tid; e < D * D; e += 256) {
+    for (int e = tid; e < D * D; e += nt) {
       const int r = e / D, c = e - r * D;
       double s = 0.0;
       for (int j = 0; j < Rk; ++j) s += Wd[r * Rk + j] * Vr[c * Rk + j];
@@ -549,10 +558,7 @@ cudaError_t launch_probe_combine(const float* part_o, const float* part_ml, int 
   return cudaGetLastError();
 }
 
-size_t probe_fit_smem(int D, int Rk) {
-  return (size_t)(2 * PR * (PR + 1) + D * Rk + PR * Rk + D + 64 + 64 + PR + 64) * 8 + (size_t)2 * PR * D * 4 +
-         (size_t)(2 * PR + 64) * 4;
-}
+size_t probe_fit_smem(int D, int Rk) { return D == 64 ? FitLayout<64>::bytes(Rk) : FitLayout<128>::bytes(Rk); }
 
 cudaError_t launch_probe_fit(const float* o_dense, const float* o_sparse, int BH, int D, int P, int Rk,
                              double lam, float* Vr, float* W, float* bfull, float* Bmat, float* sigma,
@@ -560,10 +566,10 @@ cudaError_t launch_probe_fit(const float* o_dense, const float* o_sparse, int BH
   const size_t sm = probe_fit_smem(D, Rk);
   if (D == 64) {
     cudaFuncSetAttribute(k_probe_fit<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_probe_fit<64><<<BH, 256, sm, st>>>(o_dense, o_sparse, P, Rk, lam, Vr, W, bfull, Bmat, sigma, bsub);
+    k_probe_fit<64><<<BH, FIT_THREADS, sm, st>>>(o_dense, o_sparse, P, Rk, lam, Vr, W, bfull, Bmat, sigma, bsub);
   } else {
     cudaFuncSetAttribute(k_probe_fit<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_probe_fit<128><<<BH, 256, sm, st>>>(o_dense, o_sparse, P, Rk, lam, Vr, W, bfull, Bmat, sigma, bsub);
+    k_probe_fit<128><<<BH, FIT_THREADS, sm, st>>>(o_dense, o_sparse, P, Rk, lam, Vr, W, bfull, Bmat, sigma, bsub);
   }
   return cudaGetLastError();
 }

@@ -64,11 +64,12 @@ def stage_checks(pd, qb, kb, vb, out, heads, rows=None, check_kmeans=True):
         lam_gpu = _np(tr["eigval"][bh]).astype(np.float64)
         u_gpu = _np(tr["eigvec"][bh]).astype(np.float64)
         lam_ref, _ = O.top_eigenpairs(mk_gpu, pd["eig_rank"])
-        # fp32 Jacobi: eigenvalue error O(n u ||A||) with u = 2^-24, n = d <= 128
-        assert np.abs(lam_gpu - lam_ref).max() <= 1e-4 * lam_ref[0]
-        assert np.abs(u_gpu.T @ u_gpu - np.eye(pd["eig_rank"])).max() <= 1e-4
+        # the solver runs in fp64 on the fp32 metric; its outputs are rounded to fp32, so the
+        # errors are O(sqrt(d) 2^-24) relative to ||M_K|| = lam_ref[0]
+        assert np.abs(lam_gpu - lam_ref).max() <= 1e-5 * lam_ref[0]
+        assert np.abs(u_gpu.T @ u_gpu - np.eye(pd["eig_rank"])).max() <= 1e-5
         resid = mk_gpu @ u_gpu - u_gpu * lam_gpu
-        assert np.abs(resid).max() <= 2e-4 * lam_ref[0]
+        assert np.abs(resid).max() <= 2e-5 * lam_ref[0]
         # --- a4: key coordinates from the device eigenpairs
         y_gpu = _np(tr["key_coords"][bh]).astype(np.float64)
         y_ref = O.key_coords(k, lam_gpu, u_gpu)
