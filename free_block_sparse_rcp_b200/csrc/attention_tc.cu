@@ -1,23 +1,32 @@
 // Route-walking flash attention on the 5th-generation tensor cores (tcgen05 + TMEM).
 //
-// Computes, for one q-tile of up to 128 permuted query rows of one query group,
+// Computes, for the permuted query rows of one query group,
 //   O(q) = sum_{k routed} softmax(s q.k) v_k,   LSE(q) = ln sum_{k routed} exp(s q.k)
 // (gist.science technical summary, section 2.C: attention over the routed cells of the
 // group-contiguous layout), and writes O and LSE back to the original token positions.
 //
-// Roles of the 288 threads of a CTA:
-//   warps 0-3  softmax + epilogue: thread t owns query row t = TMEM lane t
-//   warp  4    TMEM allocation; lane 0 issues every tcgen05.mma
-//   warps 5-8  gather: cp.async of the q rows and of the routed key/value rows of each
-//              128-row chunk, by index through perm_q / perm_k, into 128B-swizzled
-//              shared-memory tiles (the permuted layout is never materialised)
-// Per chunk j:  S_j = Q K_j^T  -> TMEM (two buffers, so S_{j+1} overlaps softmax_j)
-//               P_j = exp2(S_j * s*log2e - m) in bf16 -> shared memory (two buffers, so
-//                     softmax_{j+1} overlaps PV_j)
-//               O  += P_j V_j   (TMEM accumulator, rescaled in place only when a row's
-//                                 running max grows by more than 2^8)
-// Every mbarrier wait is bounded (2 s); a timeout raises an abort flag that ends every
-// role, records DERR_WAIT_TIMEOUT in the workspace and still frees the TMEM.
+// One CTA takes a unit of up to 256 permuted query rows of one query group: two q-tiles
+// of 128 rows that share one stream of routed key/value chunks, so every K/V chunk that
+// reaches shared memory feeds two tiles and the tensor pipe always has one tile's MMAs to
+// run while the other tile's softmax works.
+//
+// Roles of the 416 threads:
+//   warps 0-3   softmax + epilogue of tile 0: thread r owns query row r = TMEM lane r
+//   warps 4-7   softmax + epilogue of tile 1
+//   warps 8-11  gather: cp.async of the q rows and of the routed key/value rows of each
+//               128-row chunk, by index through perm_q / perm_k, into 128B-swizzled
+//               shared-memory tiles (the permuted layout is never materialised)
+//   warp  12    TMEM allocation; lane 0 issues every tcgen05.mma
+// TMEM (512 columns): tile t holds S_t at columns 256t .. 256t+127 and O_t at 256t+128 ..
+// The softmax writes P_t = exp2(S_t * s log2e - m) as packed bf16 pairs over the first 64
+// columns of S_t, and PV reads it straight from TMEM (A operand in tensor memory).
+// Per chunk j the MMA issue order is  PV_0,j  S_0,j+1  PV_1,j  S_1,j+1: S_t,j+1 reuses the
+// columns of P_t,j only after PV_t,j (tcgen05 MMAs of one thread execute in issue order),
+// and when S_t,j+1 is complete so is PV_t,j, so the softmax may rescale O_t in place.
+// Rescaling is lazy: only when a row's running max grows by more than 2^8.
+// K is staged in a 3-deep ring, V in a 2-deep ring.  Every mbarrier wait is bounded (2 s);
+// a timeout raises an abort flag that ends every role, records DERR_WAIT_TIMEOUT in the
+// workspace and still frees the TMEM.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -26,30 +35,32 @@ namespace spr {
 namespace tc {
 
 constexpr int BM = 128;       // q rows per tile
+constexpr int TPC = 2;        // tiles per CTA
 constexpr int BN = 128;       // key rows per chunk
-constexpr int NSOFT = 128;    // softmax threads (warps 0-3)
-constexpr int MMA_WARP = 4;
-constexpr int PROD0 = 160;    // first producer thread (warp 5)
+constexpr int KST = 3;        // K ring depth
+constexpr int VST = 2;        // V ring depth
+constexpr int NSOFT = 128;    // softmax threads per tile
+constexpr int PROD0 = 256;    // first gather thread (warp 8)
 constexpr int NPROD = 128;
-constexpr int NT = 288;
+constexpr int MMA_WARP = 12;
+constexpr int NT = 416;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct Bars {
-  uint64_t q, full[2], empty[2], s_full[2], s_free[2], p_full[2], p_empty[2], o_done, mma_done;
+  uint64_t q, kfull[KST], kempty[KST], vfull[VST], vempty[VST], s_full[TPC], p_full[TPC], o_done[TPC], mma_done;
 };
 
 template <int D>
 struct Layout {
   static constexpr uint32_t kTile = (uint32_t)D * 128 * 2;  // Q / K / V tile bytes
-  static constexpr uint32_t oQ = 0;
-  static constexpr uint32_t oK = oQ + kTile;
-  static constexpr uint32_t oV = oK + 2 * kTile;
-  static constexpr uint32_t kP = 128 * 128 * 2;
-  static constexpr uint32_t oP = oV + 2 * kTile;          // two P buffers
-  static constexpr uint32_t oBar = oP + 2 * kP;
-  static constexpr uint32_t oInt = oBar + 128;
+  static constexpr uint32_t oQ = 0;                          // TPC q tiles
+  static constexpr uint32_t oK = oQ + TPC * kTile;
+  static constexpr uint32_t oV = oK + KST * kTile;
+  static constexpr uint32_t oBar = oV + VST * kTile;
+  static constexpr uint32_t oInt = oBar + 256;
 };
+static_assert(sizeof(Bars) <= 256, "barrier block");
 
 template <int D, bool DENSE>
 __global__ void __launch_bounds__(NT, 1)
@@ -62,7 +73,7 @@ __global__ void __launch_bounds__(NT, 1)
   using L = Layout<D>;
   // The 128B-swizzled tiles need a 1024-byte aligned base; dynamic shared memory starts
   // at the CTA's shared window, which is aligned, and the layout leaves no room for a
-  // realignment pad, so a misaligned base is reported and the tile skipped.
+  // realignment pad, so a misaligned base is reported and the unit skipped.
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t base = su32(smem);
   if (base & 1023u) {
@@ -76,8 +87,8 @@ __global__ void __launch_bounds__(NT, 1)
 
   Bars* bars = reinterpret_cast<Bars*>(smem + L::oBar);
   int* ints = reinterpret_cast<int*>(smem + L::oInt);
-  int* sQrow = ints;                  // [128]
-  int* sMisc = sQrow + 128;           // [0] tmem base, [1] abort, [2] total, [3] cnt, [4] slot ok
+  int* sQrow = ints;                  // [TPC * BM]
+  int* sMisc = sQrow + TPC * BM;      // [0] tmem base, [1] abort, [2] total, [3] cnt, [4] slot ok
   int* sList = sMisc + 8;             // [Gk]
   int* sKoffL = sList + Gk;           // [Gk]
   int* sCum = sKoffL + Gk;            // [Gk + 1]
@@ -86,16 +97,16 @@ __global__ void __launch_bounds__(NT, 1)
   // ---------------- setup (all threads) ----------------
   int q0, qn;
   if (DENSE) {
-    q0 = blockIdx.x * BM;
+    q0 = blockIdx.x * (TPC * BM);
     if (q0 >= N) return;
-    qn = min(BM, N - q0);
+    qn = min(TPC * BM, N - q0);
   } else {
     if ((int)blockIdx.x >= tile_count[bh]) return;
     const int2 tl = tiles[(size_t)bh * max_tiles + blockIdx.x];
     const int a = tl.x;
     const int* qo = qoff + (size_t)bh * (Gq + 1);
-    q0 = qo[a] + tl.y * BM;
-    qn = min(BM, qo[a + 1] - q0);
+    q0 = qo[a] + tl.y * (TPC * BM);
+    qn = min(TPC * BM, qo[a + 1] - q0);
     const int cnt = rcnt[(size_t)bh * Gq + a];
     const int* rl = rlist + ((size_t)bh * Gq + a) * Gk;
     const int* rc = rcum + ((size_t)bh * Gq + a) * (Gk + 1);
@@ -108,7 +119,7 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0) { sMisc[2] = rc[cnt]; sMisc[3] = cnt; }
   }
   if (DENSE && tid == 0) { sMisc[2] = N; sMisc[3] = 0; }
-  if (tid < BM) {
+  if (tid < TPC * BM) {
     int row = -1;
     if (tid < qn) {
       row = DENSE ? q0 + tid : perm_q[head + q0 + tid];
@@ -116,18 +127,23 @@ __global__ void __launch_bounds__(NT, 1)
     }
     sQrow[tid] = row;
   }
+  const int ntile = qn > BM ? 2 : 1;
   if (tid == 0) {
     sMisc[1] = 0;
     mbar_init(su32(&bars->q), NPROD);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(su32(&bars->full[s]), NPROD);
-      mbar_init(su32(&bars->empty[s]), 1);
-      mbar_init(su32(&bars->s_full[s]), 1);
-      mbar_init(su32(&bars->s_free[s]), NSOFT);
-      mbar_init(su32(&bars->p_full[s]), NSOFT);
-      mbar_init(su32(&bars->p_empty[s]), 1);
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(su32(&bars->kfull[s]), NPROD);
+      mbar_init(su32(&bars->kempty[s]), 1);
     }
-    mbar_init(su32(&bars->o_done), 1);
+    for (int s = 0; s < VST; ++s) {
+      mbar_init(su32(&bars->vfull[s]), NPROD);
+      mbar_init(su32(&bars->vempty[s]), 1);
+    }
+    for (int t = 0; t < TPC; ++t) {
+      mbar_init(su32(&bars->s_full[t]), 1);
+      mbar_init(su32(&bars->p_full[t]), NSOFT);
+      mbar_init(su32(&bars->o_done[t]), 1);
+    }
     mbar_init(su32(&bars->mma_done), 1);
     fence_barrier_init();
   }
@@ -142,31 +158,29 @@ __global__ void __launch_bounds__(NT, 1)
   const int total = sMisc[2];
   const int cnt = sMisc[3];
   const int nchunks = (total + BN - 1) / BN;
-  const uint32_t sQ = base + L::oQ, sK = base + L::oK, sV = base + L::oV, sP = base + L::oP;
-  const uint32_t tS0 = tmem, tO = tmem + 256;   // S buffers at columns 0 / 128, O at 256
+  const uint32_t sQ = base + L::oQ, sK = base + L::oK, sV = base + L::oV;
 
   auto wait = [&](uint64_t& bar, uint32_t parity) -> bool {
     return bounded_wait(su32(&bar), parity, abort_flag, err);
   };
 
-  if (tid >= PROD0) {
+  if (tid >= PROD0 && tid < PROD0 + NPROD) {
     // ---------------- gather warps ----------------
     const int p = tid - PROD0;          // 0..127
     const int pl = p & 31, pw = p >> 5;
     constexpr int CPR = D / 8;          // 16-byte chunks per row
     constexpr int RPI = 32 / CPR;       // rows per warp instruction
-    // q rows
-    for (int i = 0; i < 32 / RPI; ++i) {
-      const int r = pw * 32 + i * RPI + pl / CPR, c = pl % CPR;
+    // q rows of both tiles (rows of an absent tile are zero-filled)
+    for (int i = 0; i < TPC * BM * CPR / NPROD; ++i) {
+      const int e = i * NPROD + p;
+      const int r = e / CPR, c = e % CPR;
       const int row = sQrow[r];
-      cp_async16(sQ + tile_off(r, c, 128), Q + (head + (row < 0 ? 0 : row)) * D + c * 8, row >= 0);
+      cp_async16(sQ + (r / BM) * L::kTile + tile_off(r % BM, c, 128),
+                 Q + (head + (row < 0 ? 0 : row)) * D + c * 8, row >= 0);
     }
     cp_async_arrive_noinc(su32(&bars->q));
     volatile int* prod_ok = sMisc + 4;
     for (int j = 0; j < nchunks; ++j) {
-      const int s = j & 1;
-      // one thread waits for the slot; the named barrier below publishes the outcome
-      if (p == 0) *prod_ok = (j < 2 || wait(bars->empty[s], ((j >> 1) - 1) & 1)) ? 1 : 0;
       // key row of slot p of chunk j (this warp's 32 rows: 32 * pw + lane)
       int myrow = -1;
       {
@@ -185,20 +199,37 @@ __global__ void __launch_bounds__(NT, 1)
           }
         }
       }
+      // K_j -> ring slot j % KST (one thread waits; the named barrier publishes the outcome)
+      const int ks = j % KST, vs = j % VST;
+      if (p == 0) *prod_ok = (j < KST || wait(bars->kempty[ks], ((j / KST) - 1) & 1)) ? 1 : 0;
       named_sync(1, NPROD);
       if (!*prod_ok) break;
-      const uint32_t dk = sK + s * L::kTile, dv = sV + s * L::kTile;
+      {
+        const uint32_t dk = sK + ks * L::kTile;
 #pragma unroll
-      for (int i = 0; i < 32 / RPI; ++i) {
-        const int rl = i * RPI + pl / CPR, c = pl % CPR;   // row within this warp's 32
-        const int row = __shfl_sync(0xffffffffu, myrow, rl);
-        const int r = pw * 32 + rl;
-        const size_t off = (head + (row < 0 ? 0 : row)) * D + c * 8;
-        const uint32_t o = tile_off(r, c, 128);
-        cp_async16(dk + o, K + off, row >= 0);
-        cp_async16(dv + o, V + off, row >= 0);
+        for (int i = 0; i < 32 / RPI; ++i) {
+          const int rl = i * RPI + pl / CPR, c = pl % CPR;   // row within this warp's 32
+          const int row = __shfl_sync(0xffffffffu, myrow, rl);
+          cp_async16(dk + tile_off(pw * 32 + rl, c, 128), K + (head + (row < 0 ? 0 : row)) * D + c * 8, row >= 0);
+        }
       }
-      cp_async_arrive_noinc(su32(&bars->full[s]));
+      cp_async_arrive_noinc(su32(&bars->kfull[ks]));
+      // V_j -> ring slot j % VST
+      named_sync(1, NPROD);   // every thread has read *prod_ok before it is rewritten
+      if (p == 0) *prod_ok = (j < VST || wait(bars->vempty[vs], ((j / VST) - 1) & 1)) ? 1 : 0;
+      named_sync(1, NPROD);
+      if (!*prod_ok) break;
+      {
+        const uint32_t dv = sV + vs * L::kTile;
+#pragma unroll
+        for (int i = 0; i < 32 / RPI; ++i) {
+          const int rl = i * RPI + pl / CPR, c = pl % CPR;
+          const int row = __shfl_sync(0xffffffffu, myrow, rl);
+          cp_async16(dv + tile_off(pw * 32 + rl, c, 128), V + (head + (row < 0 ? 0 : row)) * D + c * 8, row >= 0);
+        }
+      }
+      cp_async_arrive_noinc(su32(&bars->vfull[vs]));
+      named_sync(1, NPROD);   // *prod_ok is rewritten at the top of the next chunk
     }
     cp_async_wait_all();
   } else if (warp == MMA_WARP) {
@@ -207,141 +238,141 @@ __global__ void __launch_bounds__(NT, 1)
       constexpr uint32_t IDS = idesc_bf16(128, BN, false);
       constexpr uint32_t IDO = idesc_bf16(128, D, true);
       bool ok = nchunks == 0 || wait(bars->q, 0);
-      auto issue_pv = [&](int i) -> bool {
-        if (!wait(bars->p_full[i & 1], (i >> 1) & 1)) return false;
-        tc_fence_after();
-        const uint32_t vb = sV + (i & 1) * L::kTile;
-        const uint32_t pb = sP + (i & 1) * L::kP;
-#pragma unroll
-        for (int k = 0; k < BN / 16; ++k) {
-          const uint64_t ad = sdesc(pb + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc(vb + k * 2048, 16384, 1024);
-          tc_mma(tO, ad, bd, IDO, (i > 0 || k > 0) ? 1u : 0u);
+      // S_t,j = Q_t K_j^T into the S columns of tile t; the last tile releases K_j
+      auto issue_s = [&](int t, int j) -> bool {
+        const int ks = j % KST;
+        if (t == 0) {
+          if (!wait(bars->kfull[ks], (j / KST) & 1)) return false;
+          tc_fence_after();
         }
-        tc_commit(su32(&bars->empty[i & 1]));
-        tc_commit(su32(&bars->p_empty[i & 1]));
-        tc_commit(su32(&bars->o_done));
-        return true;
-      };
-      for (int j = 0; ok && j < nchunks; ++j) {
-        const int s = j & 1;
-        if (!wait(bars->full[s], (j >> 1) & 1)) { ok = false; break; }
-        if (j >= 2 && !wait(bars->s_free[s], ((j >> 1) - 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kb = sK + s * L::kTile;
+        const uint32_t kb = sK + ks * L::kTile, qb = sQ + t * L::kTile;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-          tc_mma(tS0 + s * 128, sdesc(sQ + off, 16, 1024), sdesc(kb + off, 16, 1024), IDS, k > 0 ? 1u : 0u);
+          tc_mma(tmem + 256 * t, sdesc(qb + off, 16, 1024), sdesc(kb + off, 16, 1024), IDS, k > 0 ? 1u : 0u);
         }
-        tc_commit(su32(&bars->s_full[s]));
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        tc_commit(su32(&bars->s_full[t]));
+        if (t == ntile - 1) tc_commit(su32(&bars->kempty[ks]));
+        return true;
+      };
+      // O_t += P_t,j V_j with P_t,j read from TMEM; the last tile releases V_j
+      auto issue_pv = [&](int t, int j) -> bool {
+        const int vs = j % VST;
+        if (!wait(bars->p_full[t], j & 1)) return false;
+        if (t == 0 && !wait(bars->vfull[vs], (j / VST) & 1)) return false;
+        tc_fence_after();
+        const uint32_t vb = sV + vs * L::kTile;
+#pragma unroll
+        for (int k = 0; k < BN / 16; ++k)
+          tc_mma_ts(tmem + 256 * t + 128, tmem + 256 * t + k * 8, sdesc(vb + k * 2048, 16384, 1024), IDO,
+                    (j > 0 || k > 0) ? 1u : 0u);
+        if (t == ntile - 1) tc_commit(su32(&bars->vempty[vs]));
+        return true;
+      };
+      for (int t = 0; ok && t < ntile && nchunks > 0; ++t) ok = issue_s(t, 0);
+      for (int j = 0; ok && j < nchunks; ++j) {
+        for (int t = 0; ok && t < ntile; ++t) {
+          ok = issue_pv(t, j);
+          if (ok && j + 1 < nchunks) ok = issue_s(t, j + 1);
+        }
       }
-      if (ok && nchunks > 0) issue_pv(nchunks - 1);
+      for (int t = 0; t < ntile; ++t) tc_commit(su32(&bars->o_done[t]));
       // drain: every MMA issued above completes before the TMEM is released
       tc_commit(su32(&bars->mma_done));
       wait(bars->mma_done, 0);
     }
-  } else {
-    // ---------------- softmax + epilogue (thread t = row t) ----------------
-    const int t = tid;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  } else if (warp < 4 * TPC) {
+    // ---------------- softmax + epilogue (tile t, thread r = row r) ----------------
+    const int t = warp >> 2;
+    const int r = tid & (BM - 1);
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + 256 * t + lane_off, tO = tS + 128;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    uint32_t sreg[128];
-    for (int j = 0; j < nchunks; ++j) {
-      const int b = j & 1;
-      ok = wait(bars->s_full[b], (j >> 1) & 1);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      tc_ld128(tS0 + lane_off + b * 128, sreg);
-      tc_fence_before();
-      mbar_arrive(su32(&bars->s_free[b]));
-      const int valid = total - j * BN;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c)
-        if (c < valid) mx = fmaxf(mx, __uint_as_float(sreg[c]));
-      const float m_new = fmaxf(m_used, mx * scale_log2);
-      const bool need = (m_new > m_used + kRescaleThreshold) || (m_used == -INFINITY && m_new != -INFINITY);
-      const bool warp_need = __any_sync(0xffffffffu, need);
-      float alpha = 1.f;
-      if (warp_need && m_new > m_used) {
-        alpha = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_new);
-        m_used = m_new;
-      }
-      const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-      float rs = 0.f;
-      uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = c < valid ? ex2(__uint_as_float(sreg[c]) * scale_log2 - mu) : 0.f;
-        const float p1 = c + 1 < valid ? ex2(__uint_as_float(sreg[c + 1]) * scale_log2 - mu) : 0.f;
-        rs += p0 + p1;
-        pk[c >> 1] = pack_bf16(p0, p1);
-      }
-      l = l * alpha + rs;
-      if (warp_need && j >= 1) {
-        // O row *= alpha (in TMEM, warp-uniform) once PV_{j-1} has finished with it
-        ok = __all_sync(0xffffffffu, wait(bars->o_done, (j - 1) & 1));
+    if (t < ntile) {
+      uint32_t sreg[64];
+      uint32_t pk[32];
+      for (int j = 0; j < nchunks; ++j) {
+        ok = __all_sync(0xffffffffu, wait(bars->s_full[t], j & 1));
         if (!ok) break;
         tc_fence_after();
+        const int valid = total - j * BN;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          tc_ld64(tS + 64 * h, sreg);
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (64 * h + c < valid) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sreg[c]));
+          mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+        }
+        const float m_new = fmaxf(m_used, mx * scale_log2);
+        const bool need = (m_new > m_used + kRescaleThreshold) || (m_used == -INFINITY && m_new != -INFINITY);
+        const bool warp_need = __any_sync(0xffffffffu, need);
+        float alpha = 1.f;
+        if (warp_need && m_new > m_used) {
+          alpha = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_new);
+          m_used = m_new;
+        }
+        if (warp_need && j >= 1) {
+          // O row *= alpha in TMEM: PV_t,j-1 completed before S_t,j did
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tc_ld32(tO + c * 32, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tc_st32(tO + c * 32, o);
+          }
+        }
+        const float mu = (m_used == -INFINITY) ? 0.f : m_used;
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          // keys 64h .. 64h+63 -> packed P in columns 32h .. 32h+31 (their S was read above)
+          tc_ld64(tS + 64 * h, sreg);
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const float p0 = 64 * h + c < valid ? ex2(__uint_as_float(sreg[c]) * scale_log2 - mu) : 0.f;
+            const float p1 = 64 * h + c + 1 < valid ? ex2(__uint_as_float(sreg[c + 1]) * scale_log2 - mu) : 0.f;
+            rs[(c >> 1) & 3] += p0 + p1;
+            pk[c >> 1] = pack_bf16(p0, p1);
+          }
+          tc_st32(tS + 32 * h, pk);
+        }
+        l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+        tc_fence_before();
+        mbar_arrive(su32(&bars->p_full[t]));
+      }
+      // epilogue
+      const int row = sQrow[t * BM + r];
+      if (ok && nchunks > 0) ok = __all_sync(0xffffffffu, wait(bars->o_done[t], 0));
+      if (ok) {
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16* orow = O + (head + (row < 0 ? 0 : row)) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tc_ld32(tO + lane_off + c * 32, o);
+          if (nchunks > 0) {
+            tc_ld32(tO + c * 32, o);
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tc_st32(tO + lane_off + c * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+          if (row >= 0) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
         }
+        if (row >= 0 && lse) lse[head + row] = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
       }
-      if (j >= 2) {
-        // P buffer b was last read by PV_{j-2}
-        ok = __all_sync(0xffffffffu, wait(bars->p_empty[b], ((j >> 1) - 1) & 1));
-        if (!ok) break;
-      }
-      // P row t -> shared memory ([2 halves][128 rows][64] bf16, 128B-swizzled)
-      unsigned char* prow = smem + L::oP + b * L::kP;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(prow + tile_off(t, c, 128)) = v;
-      }
-      fence_proxy_async();
-      tc_fence_before();
-      mbar_arrive(su32(&bars->p_full[b]));
-    }
-    // epilogue
-    const int row = sQrow[t];
-    if (ok && nchunks > 0) {
-      ok = wait(bars->o_done, (nchunks - 1) & 1);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = O + (head + (row < 0 ? 0 : row)) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (nchunks > 0) {
-          tc_ld32(tO + lane_off + c * 32, o);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-        if (row >= 0) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-        }
-      }
-      if (row >= 0 && lse) lse[head + row] = l > 0.f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
   tc_fence_before();
@@ -354,7 +385,7 @@ __global__ void __launch_bounds__(NT, 1)
 
 size_t attn_tc_smem_bytes(int D, int Gk) {
   const size_t tiles = (D == 64) ? tc::Layout<64>::oInt : tc::Layout<128>::oInt;
-  size_t s = tiles + (size_t)(128 + 8 + 3 * Gk + 1) * 4;
+  size_t s = tiles + (size_t)(tc::TPC * tc::BM + 8 + 3 * Gk + 1) * 4;
   // at most one CTA per SM: the kernel allocates all 512 TMEM columns
   return s < 120 * 1024 ? 120 * 1024 : s;
 }
@@ -365,7 +396,7 @@ static cudaError_t launch_tc_t(const AttnArgs& a, cudaStream_t st) {
   auto kern = tc::k_attn_tc<D, DENSE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
-  dim3 grid(DENSE ? ceil_div(a.N, tc::BM) : a.max_tiles, a.BH);
+  dim3 grid(DENSE ? ceil_div(a.N, tc::TPC * tc::BM) : a.max_tiles, a.BH);
   kern<<<grid, tc::NT, sm, st>>>((const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K, (const __nv_bfloat16*)a.V,
                                  a.N, a.Gq, a.Gk, a.perm_q, a.perm_k, a.qoff, a.koff, a.rlist, a.rcum, a.rcnt,
                                  a.tiles, a.tile_count, a.max_tiles, a.scale_log2, (__nv_bfloat16*)a.O, a.lse,

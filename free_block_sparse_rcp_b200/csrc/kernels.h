@@ -105,7 +105,7 @@ struct AttnArgs {
 };
 size_t attn_tc_smem_bytes(int D, int Gk);
 cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, cudaStream_t st);
-constexpr int kAttnTileRows = 128;
+constexpr int kAttnTileRows = 256;   // query rows per attention work unit (two 128-row tiles)
 constexpr int kProbeRowsPerCta = 64;  // probe rows per CTA of k_probe_attn (its PR)
 
 // api.cu: per-thread error detail and launch count of the last call
