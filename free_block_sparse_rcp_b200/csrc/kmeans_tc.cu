@@ -411,130 +411,244 @@ __global__ void __launch_bounds__(128) k_split3(const float* __restrict__ C, int
   }
 }
 
+// Roles of the 192 threads of the persistent cell-mass kernel: warps 0-3 take the softmax
+// of tile row r = TMEM lane r and the column sums, warp 4 allocates TMEM and its lane 0
+// issues the MMAs, warp 5 gathers the tile's query rows through perm_q (cp.async) into a
+// two-deep ring.  CTA b takes the (head, query group) items [b per, (b+1) per) in order;
+// the K/V centroid parts of a head are reloaded when the head changes.
+namespace cmk {
+constexpr int NT = 192;
+constexpr int MMA_WARP = 4;
+constexpr int LOAD_WARP = 5;
+struct Bars {
+  uint64_t xfull[2], xempty[2], tfull[2], tempty[2];
+};
+}  // namespace cmk
+
+// Sum over the 32 lanes of each of the 32 columns in v[]: afterwards lane l holds, in v[0],
+// the sum of column l (butterfly reduce-scatter; fixed order, so deterministic).
+__device__ __forceinline__ float lane_column_sum32(float* v, int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool upper = (lane & w) != 0;
+#pragma unroll
+    for (int k = 0; k < w; ++k) {
+      const float send = upper ? v[k] : v[k + w];
+      const float keep = upper ? v[k + w] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+  return v[0];
+}
+
 template <int D>
-__global__ void __launch_bounds__(128) k_cell_mass_tc(const __nv_bfloat16* __restrict__ Q, int N, int Gq, int Gk,
-                                                     int GP, const int* __restrict__ perm_q,
-                                                     const int* __restrict__ qoff, const int* __restrict__ koff,
-                                                     const __nv_bfloat16* __restrict__ c1,
-                                                     const __nv_bfloat16* __restrict__ c2,
-                                                     const __nv_bfloat16* __restrict__ c3, float scale,
-                                                     float* __restrict__ mass, int* err) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  const uint32_t raw = su32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  unsigned char* smem = smem_raw + (base - raw);
+__global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16* __restrict__ Q, int N, int Gq,
+                                                            int Gk, int GP, int nitems,
+                                                            const int* __restrict__ perm_q,
+                                                            const int* __restrict__ qoff,
+                                                            const int* __restrict__ koff,
+                                                            const __nv_bfloat16* __restrict__ c1,
+                                                            const __nv_bfloat16* __restrict__ c2,
+                                                            const __nv_bfloat16* __restrict__ c3, float scale_log2,
+                                                            float* __restrict__ mass, int* err) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const uint32_t base = su32(smem);
+  if (base & 1023u) {
+    if (threadIdx.x == 0) set_error(err, DERR_INDEX);
+    return;
+  }
+  const int per = (nitems + gridDim.x - 1) / gridDim.x;
+  const int i0 = blockIdx.x * per, i1 = min(nitems, i0 + per);
+  if (i0 >= i1) return;
   constexpr uint32_t kX = 128u * D * 2u;
-  const uint32_t kC = (uint32_t)GP * D * 2u;
-  const uint32_t sX = base, sC1 = base + kX, sC2 = sC1 + kC, sC3 = sC2 + kC;
-  float* pst = reinterpret_cast<float*>(smem + kX + 3 * kC);   // [128][GP + 1]
-  float* lnn = pst + 128 * (GP + 1);                           // [GP]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(lnn + GP);
-  int* sMisc = reinterpret_cast<int*>(bar + 1);                 // [0] tmem, [1] abort
-  int* sRow = sMisc + 4;                                        // [128]
-  volatile int* abort_flag = sMisc + 1;
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int bh = blockIdx.y;
-  const size_t head = (size_t)bh * N;
   constexpr int CPR = D / 8;
+  const uint32_t kC = (uint32_t)GP * D * 2u;
+  const uint32_t sX = base, sC = base + 2 * kX;
+  float* part = reinterpret_cast<float*>(smem + 2 * kX + 3 * kC);   // [4][GP]
+  float* colacc = part + 4 * GP;                                     // [GP]
+  float* lnn = colacc + GP;                                          // [GP] log2 n_g or -inf
+  cmk::Bars* bars = reinterpret_cast<cmk::Bars*>(lnn + GP);
+  int* sMisc = reinterpret_cast<int*>(bars + 1);                     // [0] tmem, [1] abort
+  volatile int* abort_flag = sMisc + 1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float NEG_INF = __int_as_float(0xff800000);
 
-  for (int e = tid; e < GP * CPR; e += 128) {
-    const int r = e / CPR, c = e - r * CPR;
-    const size_t off = ((size_t)bh * GP + r) * D + c * 8;
-    const uint32_t o = tile_off(r, c, GP);
-    cp_async16(sC1 + o, c1 + off, true);
-    cp_async16(sC2 + o, c2 + off, true);
-    cp_async16(sC3 + o, c3 + off, true);
-  }
-  for (int g = tid; g < GP; g += 128) {
-    const int n = g < Gk ? koff[(size_t)bh * (Gk + 1) + g + 1] - koff[(size_t)bh * (Gk + 1) + g] : 0;
-    lnn[g] = n > 0 ? logf((float)n) : NEG_INF;
-  }
   if (tid == 0) {
     sMisc[1] = 0;
-    mbar_init(su32(bar), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(su32(&bars->xfull[b]), 32);
+      mbar_init(su32(&bars->xempty[b]), 1);
+      mbar_init(su32(&bars->tfull[b]), 1);
+      mbar_init(su32(&bars->tempty[b]), 128);
+    }
     fence_barrier_init();
   }
-  if (warp == 0) {
-    tc_alloc(su32(&sMisc[0]), 128);
+  if (warp == cmk::MMA_WARP) {
+    tc_alloc(su32(&sMisc[0]), 256);
     tc_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = (uint32_t)sMisc[0];
-  const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(GP >> 3) << 17) | (8u << 24);
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const int* qo = qoff + (size_t)bh * (Gq + 1);
-  const int per = (Gq + gridDim.x - 1) / gridDim.x;
-  const int a0 = blockIdx.x * per, a1 = min(Gq, a0 + per);
-  int phase = 0;
+  const uint32_t idesc = idesc_bf16(128, GP, false);
+  auto wait = [&](uint64_t& bar, uint32_t parity) -> bool {
+    return bounded_wait(su32(&bar), parity, abort_flag, err);
+  };
+
+  int tile = 0;   // running tile counter of this role (identical across roles)
   bool ok = true;
-  for (int a = a0; a < a1 && ok; ++a) {
-    const int s0 = qo[a], s1 = qo[a + 1];
-    float colsum = 0.f;   // thread tid owns column tid
-    for (int t0 = s0; t0 < s1; t0 += 128) {
-      const int nr = min(128, s1 - t0);
-      sRow[tid] = tid < nr ? perm_q[head + t0 + tid] : -1;
-      __syncthreads();
-      for (int e = tid; e < 128 * CPR; e += 128) {
-        const int r = e / CPR, c = e - r * CPR;
-        const int row = sRow[r];
-        cp_async16(sX + tile_off(r, c, 128), Q + (head + (row < 0 ? 0 : row)) * D + c * 8, row >= 0);
+  for (int seg0 = i0; seg0 < i1 && ok;) {
+    const int bh = seg0 / Gq;
+    const int seg1 = min(i1, (bh + 1) * Gq);
+    const size_t head = (size_t)bh * N;
+    const int* qo = qoff + (size_t)bh * (Gq + 1);
+    // ---- this head's centroid parts and log2 group sizes (every role is idle here)
+    __syncthreads();
+    for (int e = tid; e < GP * CPR; e += cmk::NT) {
+      const int r = e / CPR, c = e - r * CPR;
+      const size_t off = ((size_t)bh * GP + r) * D + c * 8;
+      const uint32_t o = tile_off(r, c, GP);
+      cp_async16(sC + o, c1 + off, true);
+      cp_async16(sC + kC + o, c2 + off, true);
+      cp_async16(sC + 2 * kC + o, c3 + off, true);
+    }
+    for (int g = tid; g < GP; g += cmk::NT) {
+      const int n = g < Gk ? koff[(size_t)bh * (Gk + 1) + g + 1] - koff[(size_t)bh * (Gk + 1) + g] : 0;
+      lnn[g] = n > 0 ? log2f((float)n) : NEG_INF;
+      colacc[g] = 0.f;
+    }
+    cp_async_wait_all();
+    fence_proxy_async();
+    __syncthreads();
+    const int a0 = seg0 - bh * Gq, a1 = seg1 - bh * Gq;
+
+    if (warp == cmk::LOAD_WARP) {
+      // ---------------- gather ----------------
+      for (int a = a0; a < a1 && ok; ++a) {
+        for (int t0 = qo[a]; t0 < qo[a + 1]; t0 += 128, ++tile) {
+          const int b = tile & 1, nr = min(128, qo[a + 1] - t0);
+          if (tile >= 2) ok = __all_sync(0xffffffffu, wait(bars->xempty[b], ((tile >> 1) - 1) & 1));
+          if (!ok) break;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int r = 32 * k + lane;
+            int myrow = -1;
+            if (r < nr) {
+              myrow = perm_q[head + t0 + r];
+              if (myrow < 0 || myrow >= N) { set_error(err, DERR_INDEX); myrow = -1; }
+            }
+#pragma unroll
+            for (int it = 0; it < CPR; ++it) {
+              const int e = it * 32 + lane, rr = e / CPR, c = e % CPR;
+              const int row = __shfl_sync(0xffffffffu, myrow, rr);
+              cp_async16(sX + b * kX + tile_off(32 * k + rr, c, 128), Q + (head + (row < 0 ? 0 : row)) * D + c * 8,
+                         row >= 0);
+            }
+          }
+          cp_async_arrive_noinc(su32(&bars->xfull[b]));
+        }
       }
       cp_async_wait_all();
-      fence_proxy_async();
-      __syncthreads();
-      if (tid == 0) {
-        tc_fence_after();
-        int n = 0;
-        for (uint32_t cb : {sC1, sC2, sC3}) {
+    } else if (warp == cmk::MMA_WARP) {
+      // ---------------- MMA ----------------
+      if (lane == 0) {
+        for (int a = a0; a < a1 && ok; ++a) {
+          for (int t0 = qo[a]; t0 < qo[a + 1]; t0 += 128, ++tile) {
+            const int b = tile & 1;
+            ok = wait(bars->xfull[b], (tile >> 1) & 1) && (tile < 2 || wait(bars->tempty[b], ((tile >> 1) - 1) & 1));
+            if (!ok) break;
+            tc_fence_after();
+            int n = 0;
+            for (int part3 = 0; part3 < 3; ++part3) {
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
-            const uint32_t oc = (k >> 2) * (GP * 128) + (k & 3) * 32;
-            tc_mma(tmem, sdesc(sX + ox, 16, 1024), sdesc(cb + oc, 16, 1024), idesc, n++ > 0 ? 1u : 0u);
+              for (int k = 0; k < D / 16; ++k) {
+                const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
+                const uint32_t oc = (k >> 2) * (GP * 128) + (k & 3) * 32;
+                tc_mma(tmem + 128 * b, sdesc(sX + b * kX + ox, 16, 1024), sdesc(sC + part3 * kC + oc, 16, 1024),
+                       idesc, n++ > 0 ? 1u : 0u);
+              }
+            }
+            tc_commit(su32(&bars->tfull[b]));
+            tc_commit(su32(&bars->xempty[b]));
           }
         }
-        tc_commit(su32(bar));
       }
-      ok = __syncthreads_and(bounded_wait(su32(bar), phase & 1, abort_flag, err) ? 1 : 0) != 0;
-      ++phase;
-      if (!ok) break;
-      tc_fence_after();
-      // row softmax over the non-empty groups
-      float mx = NEG_INF;
-      for (int c0 = 0; c0 < GP; c0 += 32) {
-        uint32_t r[32];
-        tc_ld32(tmem + lane_off + c0, r);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+    } else if (warp < 4) {
+      // ---------------- softmax + column sums ----------------
+      const int r = tid;   // tile row = TMEM lane
+      const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+      for (int a = a0; a < a1 && ok; ++a) {
+        const int n_a = qo[a + 1] - qo[a];
+        if (n_a == 0) {
+          if (r < Gk) mass[((size_t)bh * Gq + a) * Gk + r] = 0.f;
+          continue;
+        }
+        for (int t0 = qo[a]; t0 < qo[a + 1]; t0 += 128, ++tile) {
+          const int b = tile & 1, nr = min(128, qo[a + 1] - t0);
+          ok = __all_sync(0xffffffffu, wait(bars->tfull[b], (tile >> 1) & 1));
+          if (!ok) break;
+          tc_fence_after();
+          float v[128];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float l = lnn[c0 + e] == NEG_INF ? NEG_INF : scale * __uint_as_float(r[e]) + lnn[c0 + e];
-          pst[tid * (GP + 1) + c0 + e] = l;
-          mx = fmaxf(mx, l);
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            if (c0 < GP) {
+              uint32_t u[32];
+              tc_ld32(tmem + 128 * b + lane_off + c0, u);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[c0 + e] = __uint_as_float(u[e]);
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(su32(&bars->tempty[b]));
+          float mx = NEG_INF;
+#pragma unroll
+          for (int g = 0; g < 128; ++g) {
+            if (g < GP) {
+              const float ln = lnn[g];
+              v[g] = ln == NEG_INF ? NEG_INF : fmaf(v[g], scale_log2, ln);
+              mx = fmaxf(mx, v[g]);
+            }
+          }
+          float sum = 0.f;
+#pragma unroll
+          for (int g = 0; g < 128; ++g) {
+            if (g < GP) {
+              v[g] = v[g] == NEG_INF ? 0.f : ex2(v[g] - mx);
+              sum += v[g];
+            }
+          }
+          const float inv = (r < nr && sum > 0.f) ? 1.f / sum : 0.f;
+#pragma unroll
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            if (c0 < GP) {
+              float w[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) w[e] = v[c0 + e] * inv;
+              part[warp * GP + c0 + lane] = lane_column_sum32(w, lane);
+            }
+          }
+          named_sync(1, 128);
+          if (r < GP) {
+            colacc[r] += (part[r] + part[GP + r]) + (part[2 * GP + r] + part[3 * GP + r]);
+            if (t0 + 128 >= qo[a + 1]) {
+              if (r < Gk) mass[((size_t)bh * Gq + a) * Gk + r] = colacc[r] / (float)n_a;
+              colacc[r] = 0.f;
+            }
+          }
+          named_sync(1, 128);
         }
       }
-      float sum = 0.f;
-      for (int g = 0; g < GP; ++g) {
-        const float l = pst[tid * (GP + 1) + g];
-        const float e = l == NEG_INF ? 0.f : expf(l - mx);
-        pst[tid * (GP + 1) + g] = e;
-        sum += e;
-      }
-      const float inv = (tid < nr && sum > 0.f) ? 1.f / sum : 0.f;
-      for (int g = 0; g < GP; ++g) pst[tid * (GP + 1) + g] *= inv;
-      tc_fence_before();
-      __syncthreads();
-      if (tid < Gk)
-        for (int r = 0; r < nr; ++r) colsum += pst[r * (GP + 1) + tid];
-      __syncthreads();
     }
-    if (tid < Gk) mass[((size_t)bh * Gq + a) * Gk + tid] = s1 > s0 ? colsum / (float)(s1 - s0) : 0.f;
+    ok = __syncthreads_and(ok ? 1 : 0) != 0;
+    seg0 = seg1;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tc_dealloc(tmem, 128);
+  if (warp == cmk::MMA_WARP) tc_dealloc(tmem, 256);
 }
 
 }  // namespace km
@@ -628,11 +742,19 @@ cudaError_t launch_segment_mean_rows(const void* X, int BH, int N, int d, int G,
 }
 
 size_t cell_mass_tc_smem(int D, int GP) {
-  return 1024 + (size_t)128 * D * 2 + 3 * (size_t)GP * D * 2 + (size_t)128 * (GP + 1) * 4 + (size_t)GP * 4 + 8 +
-         (4 + 128) * 4;
+  return (size_t)2 * 128 * D * 2 + 3 * (size_t)GP * D * 2 + (size_t)6 * GP * 4 + sizeof(km::cmk::Bars) + 16;
 }
 
-constexpr int kCellMassCtasPerHead = 8;
+static int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        n <= 0)
+      n = 148;
+  }
+  return n;
+}
 
 cudaError_t launch_cell_mass_tc(const void* Q, int BH, int N, int d, int Gq, int Gk, const int* perm_q, const int* qoff,
                                 const int* koff, const float* C, float scale, void* c1, void* c2, void* c3,
@@ -643,17 +765,20 @@ cudaError_t launch_cell_mass_tc(const void* Q, int BH, int N, int d, int Gq, int
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t sm = cell_mass_tc_smem(d, GP);
-  dim3 grid(kCellMassCtasPerHead, BH);
+  const int nitems = BH * Gq;
+  const int grid = nitems < sm_count() ? nitems : sm_count();
+  const float scale_log2 = scale * 1.4426950408889634f;
   if (d == 64) {
     cudaFuncSetAttribute(km::k_cell_mass_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    km::k_cell_mass_tc<64><<<grid, 128, sm, st>>>((const __nv_bfloat16*)Q, N, Gq, Gk, GP, perm_q, qoff, koff,
-                                                  (const __nv_bfloat16*)c1, (const __nv_bfloat16*)c2,
-                                                  (const __nv_bfloat16*)c3, scale, mass, err);
+    km::k_cell_mass_tc<64><<<grid, km::cmk::NT, sm, st>>>((const __nv_bfloat16*)Q, N, Gq, Gk, GP, nitems, perm_q, qoff,
+                                                         koff, (const __nv_bfloat16*)c1, (const __nv_bfloat16*)c2,
+                                                         (const __nv_bfloat16*)c3, scale_log2, mass, err);
   } else {
     cudaFuncSetAttribute(km::k_cell_mass_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    km::k_cell_mass_tc<128><<<grid, 128, sm, st>>>((const __nv_bfloat16*)Q, N, Gq, Gk, GP, perm_q, qoff, koff,
-                                                   (const __nv_bfloat16*)c1, (const __nv_bfloat16*)c2,
-                                                   (const __nv_bfloat16*)c3, scale, mass, err);
+    km::k_cell_mass_tc<128><<<grid, km::cmk::NT, sm, st>>>((const __nv_bfloat16*)Q, N, Gq, Gk, GP, nitems, perm_q,
+                                                          qoff, koff, (const __nv_bfloat16*)c1,
+                                                          (const __nv_bfloat16*)c2, (const __nv_bfloat16*)c3,
+                                                          scale_log2, mass, err);
   }
   return cudaGetLastError();
 }
