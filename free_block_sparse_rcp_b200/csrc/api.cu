@@ -51,7 +51,7 @@ struct Layout {
   size_t err;
   // partition
   size_t sample_idx, metric, eigval, eigvec, proj, eig_lu, m_k, nu_k, key_init, C, m_q, nu_q, query_init, bias, wnorm,
-      w_hi, w_lo, flag_count, flag_rows, mass, order, cm, cc, alpha;
+      w_hi, w_lo, flag_count, flag_rows, corr_count, corr, psum, pcnt, mass, order, cm, cc, alpha;
   // attend
   size_t rlist, rcum, rcnt, tiles, tile_count;
   // probe
@@ -97,6 +97,13 @@ Layout make_layout(const sparsepr_params& p) {
   L.w_lo = take(BH * GPmax * d * 2 * 2);   // also holds the third part of C for the cell mass
   L.flag_count = take(BH * 4);
   L.flag_rows = take(BH * N * 4);
+  L.corr_count = take(BH * 4);
+  L.corr = take(BH * N * 16);
+  {
+    const KmPlan kp = kmeans_plan((int)BH, p.N);
+    L.psum = take((size_t)kp.grid * kp.maxh * GPmax * d * 4);
+    L.pcnt = take((size_t)kp.grid * kp.maxh * GPmax * 4);
+  }
   L.mass = take(BH * Gq * Gk * 4);
   L.order = take(BH * Gq * Gk * 4);
   L.cm = take(BH * Gq * Gk * 8);
@@ -163,7 +170,8 @@ sparsepr_status check_params(const sparsepr_params* p) {
   if (p->n_qgroups > 128) return fail(SPARSEPR_EUNSUPPORTED, "n_qgroups > 128 not built");
   if (recheck_smem(p->d, p->n_kgroups, kmeans_dt(p->n_kgroups), p->n_qgroups) > kSmemLimit ||
       recheck_smem(p->d, p->eig_rank, kmeans_dt(p->eig_rank), p->n_kgroups) > kSmemLimit ||
-      centroid_weights_smem(p->d, p->n_kgroups) > kSmemLimit)
+      centroid_weights_smem(p->d, p->n_kgroups) > kSmemLimit ||
+      assign_acc_smem(p->d, kmeans_gp(p->n_kgroups > p->n_qgroups ? p->n_kgroups : p->n_qgroups)) > kSmemLimit)
     return fail(SPARSEPR_EUNSUPPORTED, "too many groups for the k-means kernels");
   if (cell_mass_tc_smem(p->d, kmeans_gp(p->n_kgroups)) > kSmemLimit)
     return fail(SPARSEPR_EUNSUPPORTED, "too many K/V groups for the cell-mass kernel");
@@ -220,37 +228,45 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
   void* w_lo = at<char>(ws, L.w_lo);
   int* fcount = at<int>(ws, L.flag_count);
   int* frows = at<int>(ws, L.flag_rows);
+  int* ccount = at<int>(ws, L.corr_count);
+  void* corr = at<char>(ws, L.corr);
+  float* psum = at<float>(ws, L.psum);
+  int* pcnt = at<int>(ws, L.pcnt);
   // One Lloyd k-means of the rows X (bf16, d) on coordinates A x; A(j, c) = a_scale * A[j*sj + c*sc].
+  // Each pass assigns every row and leaves the per-group sums of its rows for the next
+  // centroid update; means_out (if set) receives the means of the final groups.
   auto kmeans = [&](const void* X, int G, int purpose, const float* A, size_t a_head, int sj, int sc, float a_scale,
                     int D, int DT, float* m, float* nu, int* init, int* labels, int* perm, int* off,
-                    int* trace_iters) -> sparsepr_status {
+                    int* trace_iters, float* means_out) -> sparsepr_status {
     SPR_LAUNCH(launch_seed_rows(X, BH, N, d, G, p.seed, purpose, m, init, err, st));
     for (int t = 0; t < p.kmeans_iters; ++t) {
       int* trc = trace_iters ? trace_iters + (size_t)t * BH * N : nullptr;
-      SPR_LAUNCH(launch_centroid_weights(m, BH, G, d, A, a_head, sj, sc, a_scale, D, DT, nu, bias, wnorm, w_hi,
-                                         w_lo, st));
+      SPR_LAUNCH(launch_centroid_weights(m, BH, G, d, A, a_head, sj, sc, a_scale, D, DT, t == 0 ? 0 : 1, psum, pcnt,
+                                         ccount, corr, X, N, nu, bias, wnorm, w_hi, w_lo, err, st));
       SPR_CUDA(cudaMemsetAsync(fcount, 0, (size_t)BH * 4, st));
-      SPR_LAUNCH(launch_assign_tc(X, BH, N, d, G, w_hi, w_lo, bias, wnorm, labels, trc, fcount, frows, err, st));
+      SPR_CUDA(cudaMemsetAsync(ccount, 0, (size_t)BH * 4, st));
+      SPR_LAUNCH(launch_assign_acc(X, BH, N, d, G, w_hi, w_lo, bias, wnorm, labels, trc, fcount, frows, psum, pcnt,
+                                   err, st));
       SPR_LAUNCH(launch_assign_recheck(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, fcount, frows, labels,
-                                       trc, st));
-      SPR_LAUNCH(launch_group_sort(labels, BH, N, G, perm, off, err, st));
-      if (t + 1 < p.kmeans_iters) SPR_LAUNCH(launch_segment_mean_rows(X, BH, N, d, G, perm, off, m, st));
+                                       trc, ccount, corr, st));
     }
+    SPR_LAUNCH(launch_group_sort(labels, BH, N, G, perm, off, err, st));
+    if (means_out)
+      SPR_LAUNCH(launch_centroid_weights(means_out, BH, G, d, A, a_head, sj, sc, a_scale, D, DT, 2, psum, pcnt, ccount,
+                                         corr, X, N, nullptr, nullptr, nullptr, nullptr, nullptr, err, st));
     return SPARSEPR_OK;
   };
-  // keys on y = Lambda^{1/2} U^T k: A(j, c) = proj[c][j]
+  // keys on y = Lambda^{1/2} U^T k: A(j, c) = proj[c][j]; K/V group centroids = mean raw key
+  // of the final groups (empty group -> 0)
+  float* C = at<float>(ws, L.C);
   SPR_CHECK(kmeans(K, Gk, PURPOSE_KEY_KMEANS, proj, (size_t)d * re, 1, re, 1.0f, re, L.DTk, at<float>(ws, L.m_k),
                    at<float>(ws, L.nu_k), at<int>(ws, L.key_init), label_k, perm_k, koff,
-                   tr ? tr->key_label_iters : nullptr));
-  // K/V group centroids: mean raw key (empty group -> 0)
-  float* C = at<float>(ws, L.C);
-  SPR_CUDA(cudaMemsetAsync(C, 0, (size_t)BH * Gk * d * 4, st));
-  SPR_LAUNCH(launch_segment_mean_rows(K, BH, N, d, Gk, perm_k, koff, C, st));
+                   tr ? tr->key_label_iters : nullptr, C));
   if (tr && tr->query_coords) SPR_LAUNCH(launch_query_coords(Q, BH, N, d, C, Gk, scale, tr->query_coords, st));
   // queries on z = s C q: A(j, c) = s * C[j][c]
   SPR_CHECK(kmeans(Q, Gq, PURPOSE_QUERY_KMEANS, C, (size_t)Gk * d, d, 1, scale, Gk, L.DTq, at<float>(ws, L.m_q),
                    at<float>(ws, L.nu_q), at<int>(ws, L.query_init), label_q, perm_q, qoff,
-                   tr ? tr->query_label_iters : nullptr));
+                   tr ? tr->query_label_iters : nullptr, nullptr));
   float* mass = at<float>(ws, L.mass);
   // the weight buffers are free again: they hold the three bf16 parts of C
   const size_t cpart = (size_t)BH * kmeans_gp(Gk) * d * 2;

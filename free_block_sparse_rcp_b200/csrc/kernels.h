@@ -33,17 +33,25 @@ size_t centroid_weights_smem(int d, int D);
 size_t recheck_smem(int d, int D, int DT, int G);
 cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_t seed, int purpose, float* m,
                              int* init_out, int* err, cudaStream_t st);
-cudaError_t launch_centroid_weights(const float* m, int BH, int G, int d, const float* A, size_t a_head, int sj,
-                                    int sc, float a_scale, int D, int DT, float* nu, float* bias, float* wnorm,
-                                    void* w_hi, void* w_lo, cudaStream_t st);
-cudaError_t launch_assign_tc(const void* X, int BH, int N, int d, int G, const void* w_hi, const void* w_lo,
-                             const float* bias, const float* wnorm, int* labels, int* trace, int* flag_count,
-                             int* flag_rows, int* err, cudaStream_t st);
+// Persistent k-means assignment: CTA b takes the global 128-row tiles [b per, (b+1) per)
+// and leaves one partial-sum slot per head it touches (maxh slots per CTA).
+constexpr int kKmeansCtas = 148;
+struct KmPlan {
+  int grid, per, T, maxh, total;
+};
+KmPlan kmeans_plan(int BH, int N);
+size_t assign_acc_smem(int D, int GP);
+cudaError_t launch_centroid_weights(float* m, int BH, int G, int d, const float* A, size_t a_head, int sj, int sc,
+                                    float a_scale, int D, int DT, int mode, const float* psum, const int* pcnt,
+                                    const int* corr_count, const void* corr, const void* X, int N, float* nu,
+                                    float* bias, float* wnorm, void* w_hi, void* w_lo, int* err, cudaStream_t st);
+cudaError_t launch_assign_acc(const void* X, int BH, int N, int d, int G, const void* w_hi, const void* w_lo,
+                              const float* bias, const float* wnorm, int* labels, int* trace, int* flag_count,
+                              int* flag_rows, float* psum, int* pcnt, int* err, cudaStream_t st);
 cudaError_t launch_assign_recheck(const void* X, int BH, int N, int d, const float* A, size_t a_head, int sj, int sc,
                                   float a_scale, int D, const float* nu, int G, const int* flag_count,
-                                  const int* flag_rows, int* labels, int* trace, cudaStream_t st);
-cudaError_t launch_segment_mean_rows(const void* X, int BH, int N, int d, int G, const int* perm, const int* offsets,
-                                     float* m, cudaStream_t st);
+                                  const int* flag_rows, int* labels, int* trace, int* corr_count, void* corr,
+                                  cudaStream_t st);
 size_t cell_mass_tc_smem(int D, int GP);
 cudaError_t launch_cell_mass_tc(const void* Q, int BH, int N, int d, int Gq, int Gk, const int* perm_q, const int* qoff,
                                 const int* koff, const float* C, float scale, void* c1, void* c2, void* c3,

@@ -29,8 +29,8 @@ constexpr int kMapCap = 4096;
 __global__ void __launch_bounds__(256) k_seed_rows(const __nv_bfloat16* __restrict__ X, int N, int d, int G,
                                                   uint64_t seed, int purpose, float* __restrict__ m,
                                                   int* __restrict__ init_out, int* err) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  int* mkey = reinterpret_cast<int*>(smem);
+  extern __shared__ __align__(16) unsigned char smem_seed[];
+  int* mkey = reinterpret_cast<int*>(smem_seed);
   int* mval = mkey + kMapCap;
   int* sidx = mval + kMapCap;
   const int bh = blockIdx.x, tid = threadIdx.x;
@@ -53,221 +53,448 @@ __global__ void __launch_bounds__(256) k_seed_rows(const __nv_bfloat16* __restri
 // ---------------------------------------------------------------------------
 // Centroid weights.  A(j, c) = a_scale * A[j * sj + c * sc] (D x d) is staged once per
 // CTA in shared memory as sA[j][c] with row stride d + 1 (conflict-free both ways).
-//   nu = A m (fp32, sequential over c), bias = ||nu||^2 (sequential over j),
+// mode 0: m holds the centroids (the seeds).
+// mode 1: m_g = (sum of the rows assigned to g) / (their count): the partial sums the
+//         previous assignment pass left per (CTA, head) slot, added in ascending CTA order
+//         in fp64, then the label corrections of the exact re-check applied in ascending
+//         row order (a row moves from its provisional group to its final one); an empty
+//         group keeps its centroid.  m is updated in place.
+// mode 2: as mode 1 but an empty group gets 0, the means are written to m and no weights
+//         are formed (the K/V group centroids after the last pass).
+// Weights, one warp per centroid: nu = A m (fp32, sequential over c), bias = ||nu||^2,
 //   w = A^T nu -> w_hi = bf16(w), w_lo = bf16(w - w_hi); wnorm = ||w||.
 // Rows g in [G, GP) are padding: w = 0, bias = +inf.
-// grid = (ceil(GP / WG_PER_CTA), BH), block = 128.
+// grid = (ceil(GP / WG_PER_CTA), BH), block = 256.
 // ---------------------------------------------------------------------------
 constexpr int WG_PER_CTA = 16;
+constexpr int CW_THREADS = 256;
 
-__global__ void __launch_bounds__(128) k_centroid_weights(const float* __restrict__ m, int G, int GP, int d,
-                                                         const float* __restrict__ A, size_t a_head, int sj,
-                                                         int sc, float a_scale, int D, int DT,
-                                                         float* __restrict__ nu, float* __restrict__ bias,
-                                                         float* __restrict__ wnorm,
-                                                         __nv_bfloat16* __restrict__ w_hi,
-                                                         __nv_bfloat16* __restrict__ w_lo) {
+struct KmPartials {
+  const float* psum;          // [grid][maxh][GP][d]
+  const int* pcnt;            // [grid][maxh][GP]
+  const int* corr_count;      // [BH]
+  const int4* corr;           // [BH][N] (row, provisional label, final label, -)
+  const __nv_bfloat16* X;     // rows
+  int N, T, per, maxh, grid;
+};
+
+__global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restrict__ m, int G, int GP, int d,
+                                                                const float* __restrict__ A, size_t a_head, int sj,
+                                                                int sc, float a_scale, int D, int DT, int mode,
+                                                                KmPartials pp, float* __restrict__ nu,
+                                                                float* __restrict__ bias, float* __restrict__ wnorm,
+                                                                __nv_bfloat16* __restrict__ w_hi,
+                                                                __nv_bfloat16* __restrict__ w_lo, int* err) {
   extern __shared__ __align__(16) float sw[];
-  float* sA = sw;                        // [D][d + 1]
-  float* sm_m = sA + D * (d + 1);        // [d]
-  float* sm_nu = sm_m + d;               // [128]
-  float* sm_w = sm_nu + 128;             // [d]
-  const int bh = blockIdx.y, tid = threadIdx.x;
+  double* acc = reinterpret_cast<double*>(sw);               // [WG_PER_CTA][d]
+  int* cnt = reinterpret_cast<int*>(acc + WG_PER_CTA * d);   // [WG_PER_CTA]
+  float* sA = reinterpret_cast<float*>(cnt + WG_PER_CTA);    // [D][d + 1]
+  float* sm_m = sA + D * (d + 1);                            // [8][d]
+  float* sm_nu = sm_m + 8 * d;                               // [8][128]
+  const int bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g0 = blockIdx.x * WG_PER_CTA, g1 = min(GP, g0 + WG_PER_CTA);
+  if (mode != 0) {
+    // ---- means from the partial sums of the previous pass
+    for (int e = tid; e < WG_PER_CTA * d; e += CW_THREADS) acc[e] = 0.0;
+    if (tid < WG_PER_CTA) cnt[tid] = 0;
+    __syncthreads();
+    const int h0 = bh * pp.T, h1 = h0 + pp.T;
+    const int b_lo = h0 / pp.per, b_hi = min(pp.grid - 1, (h1 - 1) / pp.per);
+    for (int b = b_lo; b <= b_hi; ++b) {
+      const int slot = b * pp.maxh + (bh - (b * pp.per) / pp.T);
+      for (int e = tid; e < (g1 - g0) * d; e += CW_THREADS) {
+        const int gi = e / d, c = e - gi * d;
+        acc[gi * d + c] += (double)pp.psum[((size_t)slot * GP + g0 + gi) * d + c];
+      }
+      if (tid < g1 - g0) cnt[tid] += pp.pcnt[(size_t)slot * GP + g0 + tid];
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // corrections in ascending row order (the list itself is in arbitrary order)
+      const int nc = min(pp.corr_count[bh], pp.N);
+      const int4* cl = pp.corr + (size_t)bh * pp.N;
+      int last = -1;
+      while (true) {
+        int best = 0x7fffffff, bi = -1;
+        for (int i = lane; i < nc; i += 32) {
+          const int r = cl[i].x;
+          if (r > last && r < best) { best = r; bi = i; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const int ob = __shfl_xor_sync(0xffffffffu, best, o);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+          if (ob < best) { best = ob; bi = oi; }
+        }
+        if (bi < 0) break;
+        last = best;
+        const int4 cr = cl[bi];
+        if (cr.x < 0 || cr.x >= pp.N) { if (lane == 0) set_error(err, DERR_INDEX); break; }
+        const bool from = cr.y >= g0 && cr.y < g1, to = cr.z >= g0 && cr.z < g1;
+        if (from || to) {
+          const __nv_bfloat16* xr = pp.X + ((size_t)bh * pp.N + cr.x) * d;
+          for (int c = lane; c < d; c += 32) {
+            const double x = (double)bf2f(xr[c]);
+            if (from) acc[(cr.y - g0) * d + c] -= x;
+            if (to) acc[(cr.z - g0) * d + c] += x;
+          }
+          if (lane == 0) {
+            if (from) cnt[cr.y - g0] -= 1;
+            if (to) cnt[cr.z - g0] += 1;
+          }
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    for (int e = tid; e < (g1 - g0) * d; e += CW_THREADS) {
+      const int gi = e / d, c = e - gi * d, g = g0 + gi;
+      if (g >= G) continue;
+      const int n = cnt[gi];
+      if (n > 0) m[((size_t)bh * G + g) * d + c] = (float)(acc[e] / (double)n);
+      else if (mode == 2) m[((size_t)bh * G + g) * d + c] = 0.f;
+    }
+    __syncthreads();
+    if (mode == 2) return;
+  }
   const float* Ah = A + a_head * bh;
-  for (int e = tid; e < D * d; e += 128) {
+  for (int e = tid; e < D * d; e += CW_THREADS) {
     const int j = e / d, c = e - j * d;
     sA[j * (d + 1) + c] = Ah[(size_t)j * sj + (size_t)c * sc];
   }
   __syncthreads();
-  const int g0 = blockIdx.x * WG_PER_CTA, g1 = min(GP, g0 + WG_PER_CTA);
-  for (int g = g0; g < g1; ++g) {
+  float* wm = sm_m + warp * d;
+  float* wnu = sm_nu + warp * 128;
+  for (int g = g0 + warp; g < g1; g += CW_THREADS / 32) {
     const size_t wrow = ((size_t)bh * GP + g) * d;
     if (g >= G) {
-      for (int c = tid; c < d; c += 128) {
+      for (int c = lane; c < d; c += 32) {
         w_hi[wrow + c] = __float2bfloat16(0.f);
         w_lo[wrow + c] = __float2bfloat16(0.f);
       }
-      if (tid == 0) {
+      if (lane == 0) {
         bias[(size_t)bh * GP + g] = __int_as_float(0x7f800000);
         wnorm[(size_t)bh * GP + g] = 0.f;
       }
       continue;
     }
-    for (int c = tid; c < d; c += 128) sm_m[c] = m[((size_t)bh * G + g) * d + c];
-    __syncthreads();
-    for (int j = tid; j < D; j += 128) {
-      float acc = 0.f;
-      for (int c = 0; c < d; ++c) acc = fmaf(sA[j * (d + 1) + c], sm_m[c], acc);
-      sm_nu[j] = a_scale * acc;
+    for (int c = lane; c < d; c += 32) wm[c] = m[((size_t)bh * G + g) * d + c];
+    __syncwarp();
+    float b2 = 0.f;
+    for (int j = lane; j < D; j += 32) {
+      float a = 0.f;
+      for (int c = 0; c < d; ++c) a = fmaf(sA[j * (d + 1) + c], wm[c], a);
+      a *= a_scale;
+      wnu[j] = a;
+      b2 = fmaf(a, a, b2);
     }
-    __syncthreads();
-    for (int j = tid; j < DT; j += 128) nu[((size_t)bh * G + g) * DT + j] = j < D ? sm_nu[j] : 0.f;
-    for (int c = tid; c < d; c += 128) {
-      float acc = 0.f;
-      for (int j = 0; j < D; ++j) acc = fmaf(sA[j * (d + 1) + c], sm_nu[j], acc);
-      const float w = a_scale * acc;
-      sm_w[c] = w;
+    __syncwarp();
+    for (int j = lane; j < DT; j += 32) nu[((size_t)bh * G + g) * DT + j] = j < D ? wnu[j] : 0.f;
+    float n2 = 0.f;
+    for (int c = lane; c < d; c += 32) {
+      float a = 0.f;
+      for (int j = 0; j < D; ++j) a = fmaf(sA[j * (d + 1) + c], wnu[j], a);
+      const float w = a_scale * a;
+      n2 = fmaf(w, w, n2);
       const __nv_bfloat16 hi = __float2bfloat16(w);
       w_hi[wrow + c] = hi;
       w_lo[wrow + c] = __float2bfloat16(w - __bfloat162float(hi));
     }
-    __syncthreads();
-    if (tid == 0) {
-      float b = 0.f, n2 = 0.f;
-      for (int j = 0; j < D; ++j) b = fmaf(sm_nu[j], sm_nu[j], b);
-      for (int c = 0; c < d; ++c) n2 = fmaf(sm_w[c], sm_w[c], n2);
-      bias[(size_t)bh * GP + g] = b;
+    b2 = warp_sum(b2);
+    n2 = warp_sum(n2);
+    if (lane == 0) {
+      bias[(size_t)bh * GP + g] = b2;
       wnorm[(size_t)bh * GP + g] = sqrtf(n2);
     }
-    __syncthreads();
+    __syncwarp();
   }
 }
 
 // ---------------------------------------------------------------------------
-// Tensor-core assignment.  One CTA = TPC consecutive 128-row tiles of one head.
-// 128 threads: every thread owns one row in the epilogue (TMEM lane = row); thread 0
-// issues the MMAs; warp 0 owns the TMEM allocation (128 columns).
+// Tensor-core assignment fused with the centroid sums of the next update.
+// Persistent: CTA b takes the global 128-row tiles [b per, (b+1) per) (tile i = row tile
+// i mod T of head i / T) and runs them through a pipeline:
+//   warp 5      loads the X tile (contiguous rows, cp.async) into a two-deep ring
+//   warp 4      (lane 0) scores S = X [w_hi w_lo]^T into a double-buffered TMEM tile, then,
+//               once the labels are known, adds onehot(labels)^T X into a TMEM sum
+//               (M = 128 groups x N = d; A and B both MN-major, read straight from the
+//               one-hot tile and the X tile)
+//   warps 0-3   row r: argmin of bias_g - 2 s_g -> label and one-hot row; a row whose
+//               runner-up is within twice the error bound also goes on the list of the
+//               exact re-check, which corrects its label (and, through the correction
+//               list, the sums) if the exact argmin differs.
+// When the CTA leaves a head (or ends) the sums and the per-group counts go to the
+// partial slot (CTA, head - first head of the CTA).
 // ---------------------------------------------------------------------------
-constexpr int TPC = 4;
+namespace kma {
+constexpr int NT = 192;
+constexpr int MMA_WARP = 4;
+constexpr int LOAD_WARP = 5;
+constexpr int XS = 3;   // X ring depth
+struct Bars {
+  uint64_t xfull[XS], xempty[XS], tfull[2], tempty[2], ohfull[2], ohempty[2], sumdone;
+};
+}  // namespace kma
 
 template <int D>
-__global__ void __launch_bounds__(128) k_assign_tc(const __nv_bfloat16* __restrict__ X, int N, int GP,
-                                                  const __nv_bfloat16* __restrict__ w_hi,
-                                                  const __nv_bfloat16* __restrict__ w_lo,
-                                                  const float* __restrict__ bias, const float* __restrict__ wnorm,
-                                                  int* __restrict__ labels, int* __restrict__ trace,
-                                                  int* __restrict__ flag_count, int* __restrict__ flag_rows,
-                                                  int* err) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  const uint32_t raw = su32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  unsigned char* smem = smem_raw + (base - raw);
-  constexpr uint32_t kX = 128u * D * 2u;          // X tile bytes
-  const uint32_t kW = (uint32_t)GP * D * 2u;      // one W tile
-  const uint32_t sX = base, sWh = base + kX, sWl = sWh + kW;
-  float* sBias = reinterpret_cast<float*>(smem + kX + 2 * kW);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sBias + 128);
-  int* sMisc = reinterpret_cast<int*>(bar + 1);  // [0] tmem, [1] abort, [2] wmax bits
-  volatile int* abort_flag = sMisc + 1;
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int bh = blockIdx.y;
-  const size_t head = (size_t)bh * N;
+__global__ void __launch_bounds__(kma::NT, 1)
+    k_assign_acc(const __nv_bfloat16* __restrict__ X, int N, int GP, int T, int total, int per, int maxh,
+                 const __nv_bfloat16* __restrict__ w_hi, const __nv_bfloat16* __restrict__ w_lo,
+                 const float* __restrict__ bias, const float* __restrict__ wnorm, int* __restrict__ labels,
+                 int* __restrict__ trace, int* __restrict__ flag_count, int* __restrict__ flag_rows,
+                 float* __restrict__ psum, int* __restrict__ pcnt, int* err) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const uint32_t base = su32(smem);
+  if (base & 1023u) {
+    if (threadIdx.x == 0) set_error(err, DERR_INDEX);
+    return;
+  }
+  const int t0 = blockIdx.x * per, t1 = min(total, t0 + per);
+  if (t0 >= t1) return;
   constexpr int CPR = D / 8;
+  constexpr uint32_t kX = 128u * D * 2u;      // X tile
+  constexpr uint32_t kOH = 128u * 128u * 2u;  // one-hot tile [2 halves][128 rows][64 groups]
+  const uint32_t kW = (uint32_t)GP * D * 2u;
+  constexpr int XS = kma::XS;
+  const uint32_t sX = base, sOH = base + XS * kX, sWh = sOH + 2 * kOH, sWl = sWh + kW;
+  float* sBias = reinterpret_cast<float*>(smem + XS * kX + 2 * kOH + 2 * kW);   // [GP]
+  int* sCnt = reinterpret_cast<int*>(sBias + GP);                              // [GP]
+  kma::Bars* bars = reinterpret_cast<kma::Bars*>(sCnt + GP);
+  int* sMisc = reinterpret_cast<int*>(bars + 1);   // [0] tmem, [1] abort, [2] max ||w|| bits
+  volatile int* abort_flag = sMisc + 1;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  // weights, bias, max ||w||
-  for (int e = tid; e < GP * CPR; e += 128) {
-    const int r = e / CPR, c = e - r * CPR;
-    const size_t off = ((size_t)bh * GP + r) * D + c * 8;
-    cp_async16(sWh + tile_off(r, c, GP), w_hi + off, true);
-    cp_async16(sWl + tile_off(r, c, GP), w_lo + off, true);
-  }
-  float wmax = 0.f;
-  for (int g = tid; g < GP; g += 128) {
-    sBias[g] = bias[(size_t)bh * GP + g];
-    wmax = fmaxf(wmax, wnorm[(size_t)bh * GP + g]);
-  }
-  wmax = warp_max(wmax);
   if (tid == 0) {
     sMisc[1] = 0;
-    sMisc[2] = 0;
-    mbar_init(su32(bar), 1);
+    for (int b = 0; b < XS; ++b) {
+      mbar_init(su32(&bars->xfull[b]), 32);
+      mbar_init(su32(&bars->xempty[b]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(su32(&bars->tfull[b]), 1);
+      mbar_init(su32(&bars->tempty[b]), 128);
+      mbar_init(su32(&bars->ohfull[b]), 128);
+      mbar_init(su32(&bars->ohempty[b]), 1);
+    }
+    mbar_init(su32(&bars->sumdone), 1);
     fence_barrier_init();
   }
-  __syncthreads();
-  if ((tid & 31) == 0) atomicMax(&sMisc[2], __float_as_int(wmax));  // non-negative floats order as ints
-  if (warp == 0) {
-    tc_alloc(su32(&sMisc[0]), 128);
+  if (warp == kma::MMA_WARP) {
+    tc_alloc(su32(&sMisc[0]), 512);
     tc_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = (uint32_t)sMisc[0];
-  wmax = __int_as_float(sMisc[2]);
-  const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(GP >> 3) << 17) | (8u << 24);
+  const uint32_t tSum = tmem + 256;
+  const uint32_t IDS = idesc_bf16(128, GP, false);
+  constexpr uint32_t IDA = idesc_bf16_mn(128, D, true, true);
   // error bound of one score: 2 |x.w_hi + x.w_lo - x.w| <= 2 (2^-18 + 2 D 2^-24) ||x|| ||w||
   const float kc = 2.f * (3.814697265625e-06f + 2.f * D * 5.9604644775390625e-08f);
+  auto wait = [&](uint64_t& bar, uint32_t parity) -> bool {
+    return bounded_wait(su32(&bar), parity, abort_flag, err);
+  };
 
-  for (int it = 0; it < TPC; ++it) {
-    const int n0 = (blockIdx.x * TPC + it) * 128;
-    if (n0 >= N) break;
-    for (int e = tid; e < 128 * CPR; e += 128) {
+  int it = 0, sg = 0;   // running tile / segment counters (identical across roles)
+  bool ok = true;
+  for (int s0 = t0; s0 < t1 && ok;) {
+    const int bh = s0 / T;
+    const int s1 = min(t1, (bh + 1) * T);
+    const int slot = blockIdx.x * maxh + (bh - t0 / T);
+    const size_t head = (size_t)bh * N;
+    // ---- this head's weights (every role is idle here)
+    __syncthreads();
+    for (int e = tid; e < GP * CPR; e += kma::NT) {
       const int r = e / CPR, c = e - r * CPR;
-      const bool ok = n0 + r < N;
-      cp_async16(sX + tile_off(r, c, 128), X + (head + (ok ? n0 + r : 0)) * D + c * 8, ok);
+      const size_t off = ((size_t)bh * GP + r) * D + c * 8;
+      cp_async16(sWh + tile_off(r, c, GP), w_hi + off, true);
+      cp_async16(sWl + tile_off(r, c, GP), w_lo + off, true);
     }
+    float wm = 0.f;
+    for (int g = tid; g < GP; g += kma::NT) {
+      sBias[g] = bias[(size_t)bh * GP + g];
+      sCnt[g] = 0;
+      wm = fmaxf(wm, wnorm[(size_t)bh * GP + g]);
+    }
+    wm = warp_max(wm);
+    if (tid == 0) sMisc[2] = 0;
     cp_async_wait_all();
     fence_proxy_async();
     __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
-        const uint32_t ow = (k >> 2) * (GP * 128) + (k & 3) * 32;
-        tc_mma(tmem, sdesc(sX + ox, 16, 1024), sdesc(sWh + ow, 16, 1024), idesc, k > 0 ? 1u : 0u);
-      }
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
-        const uint32_t ow = (k >> 2) * (GP * 128) + (k & 3) * 32;
-        tc_mma(tmem, sdesc(sX + ox, 16, 1024), sdesc(sWl + ow, 16, 1024), idesc, 1u);
-      }
-      tc_commit(su32(bar));
-    }
-    // ||x|| of this thread's row (from the swizzled tile)
-    float xx = 0.f;
-#pragma unroll
-    for (int c = 0; c < CPR; ++c) {
-      const uint4 v = *reinterpret_cast<const uint4*>(smem + tile_off(tid, c, 128));
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h2[e]);
-        xx = fmaf(f.x, f.x, fmaf(f.y, f.y, xx));
-      }
-    }
-    // CTA-uniform outcome, so every thread takes the same barriers afterwards
-    const bool ok = __syncthreads_and(bounded_wait(su32(bar), it & 1, abort_flag, err) ? 1 : 0) != 0;
-    if (!ok) break;
-    tc_fence_after();
-    float best = __int_as_float(0x7f800000), second = best;
-    int bi = 0;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    for (int c0 = 0; c0 < GP; c0 += 32) {
-      uint32_t r[32];
-      tc_ld32(tmem + lane_off + c0, r);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float v = sBias[c0 + e] - 2.f * __uint_as_float(r[e]);
-        if (v < best) { second = best; best = v; bi = c0 + e; }
-        else if (v < second) second = v;
-      }
-    }
-    const int row = n0 + tid;
-    if (row < N) {
-      const float bound = kc * sqrtf(xx) * wmax + 1e-6f * (fabsf(best) + fabsf(second));
-      if (second - best > 2.f * bound) {
-        labels[head + row] = bi;
-        if (trace) trace[head + row] = bi;
-      } else {
-        const int slot = atomicAdd(&flag_count[bh], 1);
-        flag_rows[head + slot] = row;
-      }
-    }
-    tc_fence_before();
+    if (lane == 0) atomicMax(&sMisc[2], __float_as_int(wm));   // non-negative floats order as ints
     __syncthreads();
+    const float wmax = __int_as_float(sMisc[2]);
+
+    if (warp == kma::LOAD_WARP) {
+      // ---------------- loads ----------------
+      for (int i = s0; i < s1 && ok; ++i, ++it) {
+        const int xb = it % XS, n0 = (i - bh * T) * 128;
+        if (it >= XS) ok = __all_sync(0xffffffffu, wait(bars->xempty[xb], ((it / XS) - 1) & 1));
+        if (!ok) break;
+#pragma unroll 4
+        for (int q = 0; q < 128 * CPR / 32; ++q) {
+          const int e = q * 32 + lane, r = e / CPR, c = e % CPR;
+          const bool in = n0 + r < N;
+          cp_async16(sX + xb * kX + tile_off(r, c, 128), X + (head + (in ? n0 + r : 0)) * D + c * 8, in);
+        }
+        cp_async_arrive_noinc(su32(&bars->xfull[xb]));
+      }
+      cp_async_wait_all();
+    } else if (warp == kma::MMA_WARP) {
+      // ---------------- MMA ----------------
+      if (lane == 0) {
+        const int first = it;
+        auto sums = [&](int j) -> bool {
+          const int bj = j & 1, xj = j % XS;
+          if (!wait(bars->ohfull[bj], (j >> 1) & 1)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            tc_mma(tSum, sdesc(sOH + bj * kOH + k * 2048, 16384, 1024), sdesc(sX + xj * kX + k * 2048, 16384, 1024),
+                   IDA, (j > first || k > 0) ? 1u : 0u);
+          tc_commit(su32(&bars->xempty[xj]));
+          tc_commit(su32(&bars->ohempty[bj]));
+          return true;
+        };
+        for (int i = s0; i < s1 && ok; ++i, ++it) {
+          const int b = it & 1, xb = it % XS;
+          ok = wait(bars->xfull[xb], (it / XS) & 1) && (it < 2 || wait(bars->tempty[b], ((it >> 1) - 1) & 1));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
+            const uint32_t ow = (k >> 2) * (GP * 128) + (k & 3) * 32;
+            tc_mma(tmem + 128 * b, sdesc(sX + xb * kX + ox, 16, 1024), sdesc(sWh + ow, 16, 1024), IDS, k > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
+            const uint32_t ow = (k >> 2) * (GP * 128) + (k & 3) * 32;
+            tc_mma(tmem + 128 * b, sdesc(sX + xb * kX + ox, 16, 1024), sdesc(sWl + ow, 16, 1024), IDS, 1u);
+          }
+          tc_commit(su32(&bars->tfull[b]));
+          if (it > first) ok = sums(it - 1);
+        }
+        if (ok && it > first) ok = sums(it - 1);
+        tc_commit(su32(&bars->sumdone));
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      it = __shfl_sync(0xffffffffu, it, 0);
+    } else if (warp < 4) {
+      // ---------------- labels, one-hot rows, flags ----------------
+      const int r = tid;
+      const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+      for (int i = s0; i < s1 && ok; ++i, ++it) {
+        const int b = it & 1, xb = it % XS, row = (i - bh * T) * 128 + r;
+        ok = __all_sync(0xffffffffu, wait(bars->tfull[b], (it >> 1) & 1));
+        if (!ok) break;
+        tc_fence_after();
+        // argmin and runner-up of bias_g - 2 s_g over four interleaved column sets, merged
+        // at the end (ties keep the lowest index)
+        float bst[4], snd[4];
+        int bix[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) { bst[q] = __int_as_float(0x7f800000); snd[q] = bst[q]; bix[q] = 0; }
+        for (int c0 = 0; c0 < GP; c0 += 32) {
+          uint32_t v[32];
+          tc_ld32(tmem + 128 * b + lane_off + c0, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int q = e & 3;
+            const float sc = fmaf(-2.f, __uint_as_float(v[e]), sBias[c0 + e]);
+            snd[q] = fminf(snd[q], fmaxf(bst[q], sc));
+            bix[q] = sc < bst[q] ? c0 + e : bix[q];
+            bst[q] = fminf(bst[q], sc);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(su32(&bars->tempty[b]));
+        float best = bst[0], second = snd[0];
+        int bi = bix[0];
+#pragma unroll
+        for (int q = 1; q < 4; ++q) {
+          const bool take = bst[q] < best || (bst[q] == best && bix[q] < bi);
+          second = take ? fminf(best, snd[q]) : fminf(second, bst[q]);
+          if (take) { best = bst[q]; bi = bix[q]; }
+        }
+        // ||x|| of this row from the swizzled tile
+        float xx = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPR; ++c) {
+          const uint4 u = *reinterpret_cast<const uint4*>(smem + xb * kX + tile_off(r, c, 128));
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h2[e]);
+            xx = fmaf(f.x, f.x, fmaf(f.y, f.y, xx));
+          }
+        }
+        const bool in = row < N;
+        if (in) {
+          const float bound = kc * sqrtf(xx) * wmax + 1e-6f * (fabsf(best) + fabsf(second));
+          labels[head + row] = bi;
+          atomicAdd(&sCnt[bi], 1);
+          if (second - best > 2.f * bound) {
+            if (trace) trace[head + row] = bi;
+          } else {
+            const int fs = atomicAdd(&flag_count[bh], 1);
+            flag_rows[head + fs] = row;
+          }
+        }
+        // one-hot row r of this tile (zero for rows past N)
+        if (it >= 2) ok = __all_sync(0xffffffffu, wait(bars->ohempty[b], ((it >> 1) - 1) & 1));
+        if (!ok) break;
+        unsigned char* oh = smem + XS * kX + b * kOH;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          uint4 u = make_uint4(0u, 0u, 0u, 0u);
+          if (in && (bi >> 3) == c) {
+            const uint32_t one = 0x3F80u << (16 * (bi & 1));   // bf16 1.0 in the low or high half
+            const int wd = (bi & 7) >> 1;
+            if (wd == 0) u.x = one; else if (wd == 1) u.y = one; else if (wd == 2) u.z = one; else u.w = one;
+          }
+          *reinterpret_cast<uint4*>(oh + tile_off(r, c, 128)) = u;
+        }
+        fence_proxy_async();
+        mbar_arrive(su32(&bars->ohfull[b]));
+      }
+      // ---- sums and counts of this head -> partial slot
+      if (ok) ok = __all_sync(0xffffffffu, wait(bars->sumdone, sg & 1));
+      named_sync(1, 128);
+      if (ok) {
+        tc_fence_after();
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t v[32];
+          tc_ld32(tSum + lane_off + c0, v);
+          if (r < GP) {
+            float* dst = psum + ((size_t)slot * GP + r) * D + c0;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
+                                                                __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+          }
+        }
+        if (r < GP) pcnt[(size_t)slot * GP + r] = sCnt[r];
+        tc_fence_before();
+      }
+    }
+    ++sg;
+    ok = __syncthreads_and(ok ? 1 : 0) != 0;
+    s0 = s1;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tc_dealloc(tmem, 128);
+  if (warp == kma::MMA_WARP) tc_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------------------
 // Exact re-assignment of the uncertified rows: y = A x (fp32, sequential over c),
 // dist_g = sum_c (y_c - nu_gc)^2 (sequential fp32 fma over c), argmin with ties to the
-// lowest g.  A and the centroids are staged in shared memory (padded rows); one warp per
+// lowest g.  A row whose exact label differs from its provisional one is appended to the
+// correction list (row, provisional, final) used by the next centroid update.  A and the centroids are staged in shared memory (padded rows); one warp per
 // row.  grid = (RC_PER_HEAD, BH), block = 512.
 // ---------------------------------------------------------------------------
 constexpr int RC_PER_HEAD = 8;
@@ -278,7 +505,8 @@ __global__ void __launch_bounds__(512) k_assign_recheck(const __nv_bfloat16* __r
                                                        float a_scale, int D, const float* __restrict__ nu, int G,
                                                        const int* __restrict__ flag_count,
                                                        const int* __restrict__ flag_rows, int* __restrict__ labels,
-                                                       int* __restrict__ trace) {
+                                                       int* __restrict__ trace, int* __restrict__ corr_count,
+                                                       int4* __restrict__ corr) {
   extern __shared__ __align__(16) float sr[];
   const int bh = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int cnt = flag_count[bh];
@@ -332,58 +560,18 @@ __global__ void __launch_bounds__(512) k_assign_recheck(const __nv_bfloat16* __r
       if (ob < best || (ob == best && oi < bi)) { best = ob; bi = oi; }
     }
     if (lane == 0) {
+      const int prov = labels[head + row];
+      if (prov != bi) {
+        // the row entered the pass's sums under its provisional label
+        const int slot = atomicAdd(&corr_count[bh], 1);
+        if (slot < N) corr[head + slot] = make_int4(row, prov, bi, 0);
+      }
       labels[head + row] = bi;
       if (trace) trace[head + row] = bi;
     }
     __syncwarp();
   }
 }
-
-// ---------------------------------------------------------------------------
-// Segment means of raw rows: m[g] = mean over permuted positions of group g of X[perm]
-// (fp64 sums; warp w sums members w, w+8, ...; warps combined in order).  Empty groups
-// keep m.  grid = (G, BH), block = 256.
-// ---------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(256) k_segment_mean_rows(const __nv_bfloat16* __restrict__ X, int N, int G,
-                                                          const int* __restrict__ perm,
-                                                          const int* __restrict__ offsets, float* __restrict__ m) {
-  constexpr int PL = D / 32;  // columns per lane
-  __shared__ double part[8][D];
-  const int g = blockIdx.x, bh = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int s0 = offsets[(size_t)bh * (G + 1) + g], s1 = offsets[(size_t)bh * (G + 1) + g + 1];
-  if (s1 == s0) return;
-  const int* pm = perm + (size_t)bh * N;
-  const __nv_bfloat16* Xh = X + (size_t)bh * N * D;
-  double acc[PL];
-#pragma unroll
-  for (int e = 0; e < PL; ++e) acc[e] = 0.0;
-  for (int s = s0 + warp; s < s1; s += 8) {
-    const __nv_bfloat16* row = Xh + (size_t)pm[s] * D + lane * PL;
-    if constexpr (PL == 4) {
-      const uint2 v = *reinterpret_cast<const uint2*>(row);
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-      const float2 a = __bfloat1622float2(h2[0]), b = __bfloat1622float2(h2[1]);
-      acc[0] += a.x;
-      acc[1] += a.y;
-      acc[2] += b.x;
-      acc[3] += b.y;
-    } else {
-      const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(row));
-      acc[0] += a.x;
-      acc[1] += a.y;
-    }
-  }
-#pragma unroll
-  for (int e = 0; e < PL; ++e) part[warp][lane * PL + e] = acc[e];
-  __syncthreads();
-  for (int c = threadIdx.x; c < D; c += 256) {
-    double t = 0.0;
-    for (int w = 0; w < 8; ++w) t += part[w][c];
-    m[((size_t)bh * G + g) * D + c] = (float)(t / (double)(s1 - s0));
-  }
-}
-
 
 // ---------------------------------------------------------------------------
 // Cell mass on the tensor cores.  p(a, g) = mean over the queries q of group a of
@@ -658,8 +846,19 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
 // ---------------------------------------------------------------------------
 int kmeans_gp(int G) { return (G + 31) / 32 * 32; }
 
-size_t assign_tc_smem(int D, int GP) {
-  return 1024 + (size_t)128 * D * 2 + 2 * (size_t)GP * D * 2 + 128 * 4 + 8 + 16;
+size_t assign_acc_smem(int D, int GP) {
+  return (size_t)km::kma::XS * 128 * D * 2 + (size_t)2 * 128 * 128 * 2 + 2 * (size_t)GP * D * 2 + (size_t)GP * 8 +
+         sizeof(km::kma::Bars) + 16;
+}
+
+KmPlan kmeans_plan(int BH, int N) {
+  KmPlan pl{};
+  pl.T = ceil_div(N, 128);
+  pl.total = BH * pl.T;
+  pl.grid = pl.total < kKmeansCtas ? pl.total : kKmeansCtas;
+  pl.per = ceil_div(pl.total, pl.grid);
+  pl.maxh = pl.per / pl.T + 2;
+  return pl;
 }
 
 cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_t seed, int purpose, float* m,
@@ -670,35 +869,42 @@ cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_
   return cudaGetLastError();
 }
 
-size_t centroid_weights_smem(int d, int D) { return ((size_t)D * (d + 1) + 2 * d + 128) * 4; }
+size_t centroid_weights_smem(int d, int D) {
+  return (size_t)km::WG_PER_CTA * d * 8 + km::WG_PER_CTA * 4 + ((size_t)D * (d + 1) + 8 * d + 8 * 128) * 4;
+}
 
-cudaError_t launch_centroid_weights(const float* m, int BH, int G, int d, const float* A, size_t a_head, int sj,
-                                    int sc, float a_scale, int D, int DT, float* nu, float* bias, float* wnorm,
-                                    void* w_hi, void* w_lo, cudaStream_t st) {
+cudaError_t launch_centroid_weights(float* m, int BH, int G, int d, const float* A, size_t a_head, int sj, int sc,
+                                    float a_scale, int D, int DT, int mode, const float* psum, const int* pcnt,
+                                    const int* corr_count, const void* corr, const void* X, int N, float* nu,
+                                    float* bias, float* wnorm, void* w_hi, void* w_lo, int* err, cudaStream_t st) {
   const int GP = kmeans_gp(G);
   const size_t sm = centroid_weights_smem(d, D);
+  const KmPlan pl = kmeans_plan(BH, N);
+  km::KmPartials pp{psum, pcnt, corr_count, (const int4*)corr, (const __nv_bfloat16*)X, N, pl.T, pl.per, pl.maxh,
+                    pl.grid};
   cudaFuncSetAttribute(km::k_centroid_weights, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  km::k_centroid_weights<<<dim3(ceil_div(GP, km::WG_PER_CTA), BH), 128, sm, st>>>(
-      m, G, GP, d, A, a_head, sj, sc, a_scale, D, DT, nu, bias, wnorm, (__nv_bfloat16*)w_hi, (__nv_bfloat16*)w_lo);
+  km::k_centroid_weights<<<dim3(ceil_div(GP, km::WG_PER_CTA), BH), km::CW_THREADS, sm, st>>>(
+      m, G, GP, d, A, a_head, sj, sc, a_scale, D, DT, mode, pp, nu, bias, wnorm, (__nv_bfloat16*)w_hi,
+      (__nv_bfloat16*)w_lo, err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_assign_tc(const void* X, int BH, int N, int d, int G, const void* w_hi, const void* w_lo,
-                             const float* bias, const float* wnorm, int* labels, int* trace, int* flag_count,
-                             int* flag_rows, int* err, cudaStream_t st) {
+cudaError_t launch_assign_acc(const void* X, int BH, int N, int d, int G, const void* w_hi, const void* w_lo,
+                              const float* bias, const float* wnorm, int* labels, int* trace, int* flag_count,
+                              int* flag_rows, float* psum, int* pcnt, int* err, cudaStream_t st) {
   const int GP = kmeans_gp(G);
-  const size_t sm = assign_tc_smem(d, GP);
-  dim3 grid(ceil_div(N, 128 * km::TPC), BH);
+  const size_t sm = assign_acc_smem(d, GP);
+  const KmPlan pl = kmeans_plan(BH, N);
   if (d == 64) {
-    cudaFuncSetAttribute(km::k_assign_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    km::k_assign_tc<64><<<grid, 128, sm, st>>>((const __nv_bfloat16*)X, N, GP, (const __nv_bfloat16*)w_hi,
-                                               (const __nv_bfloat16*)w_lo, bias, wnorm, labels, trace, flag_count,
-                                               flag_rows, err);
+    cudaFuncSetAttribute(km::k_assign_acc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    km::k_assign_acc<64><<<pl.grid, km::kma::NT, sm, st>>>(
+        (const __nv_bfloat16*)X, N, GP, pl.T, pl.total, pl.per, pl.maxh, (const __nv_bfloat16*)w_hi,
+        (const __nv_bfloat16*)w_lo, bias, wnorm, labels, trace, flag_count, flag_rows, psum, pcnt, err);
   } else {
-    cudaFuncSetAttribute(km::k_assign_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    km::k_assign_tc<128><<<grid, 128, sm, st>>>((const __nv_bfloat16*)X, N, GP, (const __nv_bfloat16*)w_hi,
-                                                (const __nv_bfloat16*)w_lo, bias, wnorm, labels, trace, flag_count,
-                                                flag_rows, err);
+    cudaFuncSetAttribute(km::k_assign_acc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    km::k_assign_acc<128><<<pl.grid, km::kma::NT, sm, st>>>(
+        (const __nv_bfloat16*)X, N, GP, pl.T, pl.total, pl.per, pl.maxh, (const __nv_bfloat16*)w_hi,
+        (const __nv_bfloat16*)w_lo, bias, wnorm, labels, trace, flag_count, flag_rows, psum, pcnt, err);
   }
   return cudaGetLastError();
 }
@@ -710,35 +916,28 @@ size_t recheck_smem(int d, int D, int DT, int G) {
 template <int DT>
 static cudaError_t recheck_dt(const void* X, int BH, int N, int d, const float* A, size_t a_head, int sj, int sc,
                               float a_scale, int D, const float* nu, int G, const int* flag_count,
-                              const int* flag_rows, int* labels, int* trace, cudaStream_t st) {
+                              const int* flag_rows, int* labels, int* trace, int* corr_count, void* corr,
+                              cudaStream_t st) {
   const size_t sm = recheck_smem(d, D, DT, G);
   cudaFuncSetAttribute(km::k_assign_recheck<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   km::k_assign_recheck<DT><<<dim3(km::RC_PER_HEAD, BH), 512, sm, st>>>((const __nv_bfloat16*)X, N, d, A, a_head, sj,
                                                                       sc, a_scale, D, nu, G, flag_count, flag_rows,
-                                                                      labels, trace);
+                                                                      labels, trace, corr_count, (int4*)corr);
   return cudaGetLastError();
 }
 
 cudaError_t launch_assign_recheck(const void* X, int BH, int N, int d, const float* A, size_t a_head, int sj, int sc,
                                   float a_scale, int D, const float* nu, int G, const int* flag_count,
-                                  const int* flag_rows, int* labels, int* trace, cudaStream_t st) {
+                                  const int* flag_rows, int* labels, int* trace, int* corr_count, void* corr,
+                                  cudaStream_t st) {
   switch (kmeans_dt(D)) {
-    case 8: return recheck_dt<8>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, st);
-    case 16: return recheck_dt<16>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, st);
-    case 32: return recheck_dt<32>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, st);
-    case 64: return recheck_dt<64>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, st);
-    case 128: return recheck_dt<128>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, st);
+    case 8: return recheck_dt<8>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, corr_count, corr, st);
+    case 16: return recheck_dt<16>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, corr_count, corr, st);
+    case 32: return recheck_dt<32>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, corr_count, corr, st);
+    case 64: return recheck_dt<64>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, corr_count, corr, st);
+    case 128: return recheck_dt<128>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, corr_count, corr, st);
     default: return cudaErrorInvalidValue;
   }
-}
-
-cudaError_t launch_segment_mean_rows(const void* X, int BH, int N, int d, int G, const int* perm, const int* offsets,
-                                     float* m, cudaStream_t st) {
-  if (d == 64)
-    km::k_segment_mean_rows<64><<<dim3(G, BH), 256, 0, st>>>((const __nv_bfloat16*)X, N, G, perm, offsets, m);
-  else
-    km::k_segment_mean_rows<128><<<dim3(G, BH), 256, 0, st>>>((const __nv_bfloat16*)X, N, G, perm, offsets, m);
-  return cudaGetLastError();
 }
 
 size_t cell_mass_tc_smem(int D, int GP) {

@@ -148,6 +148,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
          ((uint32_t)(M >> 4) << 24);
 }
 
+// Same with the operand majors chosen: A MN-major sets bit 15, B MN-major bit 16.
+__host__ __device__ constexpr uint32_t idesc_bf16_mn(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // Byte offset of 16-byte chunk `c` (of the row's D/8 chunks) of row `r` in a tile stored
 // as [D/64 halves][rows][64] with 128-byte rows swizzled by (r & 7).
 __device__ __forceinline__ uint32_t tile_off(int r, int c, int rows) {
