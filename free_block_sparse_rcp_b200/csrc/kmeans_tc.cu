@@ -214,25 +214,32 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
 // Tensor-core assignment fused with the centroid sums of the next update.
 // Persistent: CTA b takes the global 128-row tiles [b per, (b+1) per) (tile i = row tile
 // i mod T of head i / T) and runs them through a pipeline:
-//   warp 5      loads the X tile (contiguous rows, cp.async) into a two-deep ring
-//   warp 4      (lane 0) scores S = X [w_hi w_lo]^T into a double-buffered TMEM tile, then,
+//   warp 9      loads the X tile (contiguous rows, cp.async) into a three-deep ring
+//   warp 8      (lane 0) scores S = X [w_hi w_lo]^T into a double-buffered TMEM tile, then,
 //               once the labels are known, adds onehot(labels)^T X into a TMEM sum
 //               (M = 128 groups x N = d; A and B both MN-major, read straight from the
 //               one-hot tile and the X tile)
-//   warps 0-3   row r: argmin of bias_g - 2 s_g -> label and one-hot row; a row whose
-//               runner-up is within twice the error bound also goes on the list of the
-//               exact re-check, which corrects its label (and, through the correction
-//               list, the sums) if the exact argmin differs.
+//   warps 0-7   row r = TMEM lane r, columns split in two halves (warps w and w + 4):
+//               argmin of bias_g - 2 s_g per half, merged through shared memory; the
+//               label goes into the sums through a one-hot row; a row whose runner-up is
+//               within twice the error bound also goes on the list of the exact re-check,
+//               which corrects its label (and, through the correction list, the sums) if
+//               the exact argmin differs.
 // When the CTA leaves a head (or ends) the sums and the per-group counts go to the
 // partial slot (CTA, head - first head of the CTA).
 // ---------------------------------------------------------------------------
 namespace kma {
-constexpr int NT = 192;
-constexpr int MMA_WARP = 4;
-constexpr int LOAD_WARP = 5;
+constexpr int NT = 320;
+constexpr int NEPI = 256;
+constexpr int MMA_WARP = 8;
+constexpr int LOAD_WARP = 9;
 constexpr int XS = 3;   // X ring depth
 struct Bars {
-  uint64_t xfull[XS], xempty[XS], tfull[2], tempty[2], ohfull[2], ohempty[2], sumdone;
+  uint64_t xfull[XS], xempty[XS], tfull[2], tempty[2], ohfull, ohempty, sumdone, xready[2], epidone;
+};
+struct Half {
+  float best, second, xx;
+  int bi;
 };
 }  // namespace kma
 
@@ -256,9 +263,10 @@ __global__ void __launch_bounds__(kma::NT, 1)
   constexpr uint32_t kOH = 128u * 128u * 2u;  // one-hot tile [2 halves][128 rows][64 groups]
   const uint32_t kW = (uint32_t)GP * D * 2u;
   constexpr int XS = kma::XS;
-  const uint32_t sX = base, sOH = base + XS * kX, sWh = sOH + 2 * kOH, sWl = sWh + kW;
-  float* sBias = reinterpret_cast<float*>(smem + XS * kX + 2 * kOH + 2 * kW);   // [GP]
-  int* sCnt = reinterpret_cast<int*>(sBias + GP);                              // [GP]
+  const uint32_t sX = base, sOH = base + XS * kX, sWh = sOH + kOH, sWl = sWh + kW;
+  kma::Half* xchg = reinterpret_cast<kma::Half*>(smem + XS * kX + kOH + 2 * kW);   // [2 tiles][2 halves][128]
+  float* sBias = reinterpret_cast<float*>(xchg + 2 * 2 * 128);                      // [GP]
+  int* sCnt = reinterpret_cast<int*>(sBias + GP);                                    // [GP]
   kma::Bars* bars = reinterpret_cast<kma::Bars*>(sCnt + GP);
   int* sMisc = reinterpret_cast<int*>(bars + 1);   // [0] tmem, [1] abort, [2] max ||w|| bits
   volatile int* abort_flag = sMisc + 1;
@@ -272,11 +280,14 @@ __global__ void __launch_bounds__(kma::NT, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(su32(&bars->tfull[b]), 1);
-      mbar_init(su32(&bars->tempty[b]), 128);
-      mbar_init(su32(&bars->ohfull[b]), 128);
-      mbar_init(su32(&bars->ohempty[b]), 1);
+      mbar_init(su32(&bars->tempty[b]), kma::NEPI);
     }
+    mbar_init(su32(&bars->ohfull), kma::NEPI);
+    mbar_init(su32(&bars->ohempty), 1);
     mbar_init(su32(&bars->sumdone), 1);
+    mbar_init(su32(&bars->xready[0]), kma::NEPI);
+    mbar_init(su32(&bars->xready[1]), kma::NEPI);
+    mbar_init(su32(&bars->epidone), kma::NEPI);
     fence_barrier_init();
   }
   if (warp == kma::MMA_WARP) {
@@ -346,15 +357,15 @@ __global__ void __launch_bounds__(kma::NT, 1)
       if (lane == 0) {
         const int first = it;
         auto sums = [&](int j) -> bool {
-          const int bj = j & 1, xj = j % XS;
-          if (!wait(bars->ohfull[bj], (j >> 1) & 1)) return false;
+          const int xj = j % XS;
+          if (!wait(bars->ohfull, j & 1)) return false;
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            tc_mma(tSum, sdesc(sOH + bj * kOH + k * 2048, 16384, 1024), sdesc(sX + xj * kX + k * 2048, 16384, 1024),
-                   IDA, (j > first || k > 0) ? 1u : 0u);
+            tc_mma(tSum, sdesc(sOH + k * 2048, 16384, 1024), sdesc(sX + xj * kX + k * 2048, 16384, 1024), IDA,
+                   (j > first || k > 0) ? 1u : 0u);
           tc_commit(su32(&bars->xempty[xj]));
-          tc_commit(su32(&bars->ohempty[bj]));
+          tc_commit(su32(&bars->ohempty));
           return true;
         };
         for (int i = s0; i < s1 && ok; ++i, ++it) {
@@ -382,48 +393,52 @@ __global__ void __launch_bounds__(kma::NT, 1)
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       it = __shfl_sync(0xffffffffu, it, 0);
-    } else if (warp < 4) {
-      // ---------------- labels, one-hot rows, flags ----------------
-      const int r = tid;
-      const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    } else {
+      // ---------------- labels, one-hot rows, flags (warps 0-7) ----------------
+      const int hf = warp >> 2;                 // column half
+      const int r = (warp & 3) * 32 + lane;     // row = TMEM lane
+      const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       for (int i = s0; i < s1 && ok; ++i, ++it) {
         const int b = it & 1, xb = it % XS, row = (i - bh * T) * 128 + r;
         ok = __all_sync(0xffffffffu, wait(bars->tfull[b], (it >> 1) & 1));
         if (!ok) break;
         tc_fence_after();
-        // argmin and runner-up of bias_g - 2 s_g over four interleaved column sets, merged
-        // at the end (ties keep the lowest index)
+        // argmin and runner-up of bias_g - 2 s_g over this half, in four interleaved sets
         float bst[4], snd[4];
         int bix[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) { bst[q] = __int_as_float(0x7f800000); snd[q] = bst[q]; bix[q] = 0; }
-        for (int c0 = 0; c0 < GP; c0 += 32) {
-          uint32_t v[32];
-          tc_ld32(tmem + 128 * b + lane_off + c0, v);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int q = e & 3;
-            const float sc = fmaf(-2.f, __uint_as_float(v[e]), sBias[c0 + e]);
-            snd[q] = fminf(snd[q], fmaxf(bst[q], sc));
-            bix[q] = sc < bst[q] ? c0 + e : bix[q];
-            bst[q] = fminf(bst[q], sc);
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          const int cb = hf * 64 + c0;
+          if (cb < GP) {
+            uint32_t v[32];
+            tc_ld32(tmem + 128 * b + lane_off + cb, v);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int q = e & 3;
+              const float sc = fmaf(-2.f, __uint_as_float(v[e]), sBias[cb + e]);
+              snd[q] = fminf(snd[q], fmaxf(bst[q], sc));
+              bix[q] = sc < bst[q] ? cb + e : bix[q];
+              bst[q] = fminf(bst[q], sc);
+            }
           }
         }
         tc_fence_before();
         mbar_arrive(su32(&bars->tempty[b]));
-        float best = bst[0], second = snd[0];
-        int bi = bix[0];
+        kma::Half h;
+        h.best = bst[0]; h.second = snd[0]; h.bi = bix[0];
 #pragma unroll
         for (int q = 1; q < 4; ++q) {
-          const bool take = bst[q] < best || (bst[q] == best && bix[q] < bi);
-          second = take ? fminf(best, snd[q]) : fminf(second, bst[q]);
-          if (take) { best = bst[q]; bi = bix[q]; }
+          const bool take = bst[q] < h.best || (bst[q] == h.best && bix[q] < h.bi);
+          h.second = take ? fminf(h.best, snd[q]) : fminf(h.second, bst[q]);
+          if (take) { h.best = bst[q]; h.bi = bix[q]; }
         }
-        // ||x|| of this row from the swizzled tile
+        // ||x||^2 of this half of the row, from the swizzled tile
         float xx = 0.f;
 #pragma unroll
-        for (int c = 0; c < CPR; ++c) {
-          const uint4 u = *reinterpret_cast<const uint4*>(smem + xb * kX + tile_off(r, c, 128));
+        for (int c = 0; c < CPR / 2; ++c) {
+          const uint4 u = *reinterpret_cast<const uint4*>(smem + xb * kX + tile_off(r, hf * (CPR / 2) + c, 128));
           const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -431,9 +446,21 @@ __global__ void __launch_bounds__(kma::NT, 1)
             xx = fmaf(f.x, f.x, fmaf(f.y, f.y, xx));
           }
         }
+        h.xx = xx;
+        xchg[(b * 2 + hf) * 128 + r] = h;
+        // both halves of every row are in (an mbarrier, so an abort cannot strand a warp)
+        mbar_arrive(su32(&bars->xready[b]));
+        ok = __all_sync(0xffffffffu, wait(bars->xready[b], (it >> 1) & 1));
+        if (!ok) break;
+        const kma::Half h0 = xchg[(b * 2 + 0) * 128 + r], h1 = xchg[(b * 2 + 1) * 128 + r];
+        // merge: half 0 holds the lower columns, so it wins ties
+        const bool take1 = h1.best < h0.best;
+        const float best = take1 ? h1.best : h0.best;
+        const float second = take1 ? fminf(h0.best, h1.second) : fminf(h0.second, h1.best);
+        const int bi = take1 ? h1.bi : h0.bi;
         const bool in = row < N;
-        if (in) {
-          const float bound = kc * sqrtf(xx) * wmax + 1e-6f * (fabsf(best) + fabsf(second));
+        if (in && hf == 0) {
+          const float bound = kc * sqrtf(h0.xx + h1.xx) * wmax + 1e-6f * (fabsf(best) + fabsf(second));
           labels[head + row] = bi;
           atomicAdd(&sCnt[bi], 1);
           if (second - best > 2.f * bound) {
@@ -443,40 +470,44 @@ __global__ void __launch_bounds__(kma::NT, 1)
             flag_rows[head + fs] = row;
           }
         }
-        // one-hot row r of this tile (zero for rows past N)
-        if (it >= 2) ok = __all_sync(0xffffffffu, wait(bars->ohempty[b], ((it >> 1) - 1) & 1));
+        // one-hot row r of this tile, this half's 8 chunks (zero for rows past N)
+        if (it >= 1) ok = __all_sync(0xffffffffu, wait(bars->ohempty, (it - 1) & 1));
         if (!ok) break;
-        unsigned char* oh = smem + XS * kX + b * kOH;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int cc = 0; cc < 8; ++cc) {
+          const int c = hf * 8 + cc;
           uint4 u = make_uint4(0u, 0u, 0u, 0u);
           if (in && (bi >> 3) == c) {
             const uint32_t one = 0x3F80u << (16 * (bi & 1));   // bf16 1.0 in the low or high half
             const int wd = (bi & 7) >> 1;
             if (wd == 0) u.x = one; else if (wd == 1) u.y = one; else if (wd == 2) u.z = one; else u.w = one;
           }
-          *reinterpret_cast<uint4*>(oh + tile_off(r, c, 128)) = u;
+          *reinterpret_cast<uint4*>(smem + XS * kX + tile_off(r, c, 128)) = u;
         }
         fence_proxy_async();
-        mbar_arrive(su32(&bars->ohfull[b]));
+        mbar_arrive(su32(&bars->ohfull));
       }
-      // ---- sums and counts of this head -> partial slot
+      // ---- sums and counts of this head -> partial slot (each half writes half the columns)
       if (ok) ok = __all_sync(0xffffffffu, wait(bars->sumdone, sg & 1));
-      named_sync(1, 128);
+      // every row's count is in sCnt
+      mbar_arrive(su32(&bars->epidone));
+      if (ok) ok = __all_sync(0xffffffffu, wait(bars->epidone, sg & 1));
       if (ok) {
         tc_fence_after();
-        for (int c0 = 0; c0 < D; c0 += 32) {
+#pragma unroll
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
+          const int cb = hf * (D / 2) + c0;
           uint32_t v[32];
-          tc_ld32(tSum + lane_off + c0, v);
+          tc_ld32(tSum + lane_off + cb, v);
           if (r < GP) {
-            float* dst = psum + ((size_t)slot * GP + r) * D + c0;
+            float* dst = psum + ((size_t)slot * GP + r) * D + cb;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
               *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
                                                                 __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
           }
         }
-        if (r < GP) pcnt[(size_t)slot * GP + r] = sCnt[r];
+        if (r < GP && hf == 0) pcnt[(size_t)slot * GP + r] = sCnt[r];
         tc_fence_before();
       }
     }
@@ -609,7 +640,7 @@ constexpr int NT = 192;
 constexpr int MMA_WARP = 4;
 constexpr int LOAD_WARP = 5;
 struct Bars {
-  uint64_t xfull[2], xempty[2], tfull[2], tempty[2];
+  uint64_t xfull[2], xempty[2], tfull[2], tempty[2], pready[2];
 };
 }  // namespace cmk
 
@@ -652,8 +683,8 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
   constexpr int CPR = D / 8;
   const uint32_t kC = (uint32_t)GP * D * 2u;
   const uint32_t sX = base, sC = base + 2 * kX;
-  float* part = reinterpret_cast<float*>(smem + 2 * kX + 3 * kC);   // [4][GP]
-  float* colacc = part + 4 * GP;                                     // [GP]
+  float* part = reinterpret_cast<float*>(smem + 2 * kX + 3 * kC);   // [2 tiles][4][GP]
+  float* colacc = part + 8 * GP;                                     // [GP]
   float* lnn = colacc + GP;                                          // [GP] log2 n_g or -inf
   cmk::Bars* bars = reinterpret_cast<cmk::Bars*>(lnn + GP);
   int* sMisc = reinterpret_cast<int*>(bars + 1);                     // [0] tmem, [1] abort
@@ -668,6 +699,7 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
       mbar_init(su32(&bars->xempty[b]), 1);
       mbar_init(su32(&bars->tfull[b]), 1);
       mbar_init(su32(&bars->tempty[b]), 128);
+      mbar_init(su32(&bars->pready[b]), 128);
     }
     fence_barrier_init();
   }
@@ -815,18 +847,22 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
               float w[32];
 #pragma unroll
               for (int e = 0; e < 32; ++e) w[e] = v[c0 + e] * inv;
-              part[warp * GP + c0 + lane] = lane_column_sum32(w, lane);
+              part[(b * 4 + warp) * GP + c0 + lane] = lane_column_sum32(w, lane);
             }
           }
-          named_sync(1, 128);
+          // every warp's column partials are in (double-buffered by tile, so one handshake
+          // per tile; an mbarrier, so an abort cannot strand a warp)
+          mbar_arrive(su32(&bars->pready[b]));
+          ok = __all_sync(0xffffffffu, wait(bars->pready[b], (tile >> 1) & 1));
+          if (!ok) break;
           if (r < GP) {
-            colacc[r] += (part[r] + part[GP + r]) + (part[2 * GP + r] + part[3 * GP + r]);
+            const float* pb = part + b * 4 * GP;
+            colacc[r] += (pb[r] + pb[GP + r]) + (pb[2 * GP + r] + pb[3 * GP + r]);
             if (t0 + 128 >= qo[a + 1]) {
               if (r < Gk) mass[((size_t)bh * Gq + a) * Gk + r] = colacc[r] / (float)n_a;
               colacc[r] = 0.f;
             }
           }
-          named_sync(1, 128);
         }
       }
     }
@@ -847,8 +883,8 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
 int kmeans_gp(int G) { return (G + 31) / 32 * 32; }
 
 size_t assign_acc_smem(int D, int GP) {
-  return (size_t)km::kma::XS * 128 * D * 2 + (size_t)2 * 128 * 128 * 2 + 2 * (size_t)GP * D * 2 + (size_t)GP * 8 +
-         sizeof(km::kma::Bars) + 16;
+  return (size_t)km::kma::XS * 128 * D * 2 + (size_t)128 * 128 * 2 + 2 * (size_t)GP * D * 2 +
+         4 * 128 * sizeof(km::kma::Half) + (size_t)GP * 8 + sizeof(km::kma::Bars) + 16;
 }
 
 KmPlan kmeans_plan(int BH, int N) {
@@ -941,7 +977,7 @@ cudaError_t launch_assign_recheck(const void* X, int BH, int N, int d, const flo
 }
 
 size_t cell_mass_tc_smem(int D, int GP) {
-  return (size_t)2 * 128 * D * 2 + 3 * (size_t)GP * D * 2 + (size_t)6 * GP * 4 + sizeof(km::cmk::Bars) + 16;
+  return (size_t)2 * 128 * D * 2 + 3 * (size_t)GP * D * 2 + (size_t)10 * GP * 4 + sizeof(km::cmk::Bars) + 16;
 }
 
 static int sm_count() {
