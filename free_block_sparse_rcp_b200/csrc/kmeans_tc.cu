@@ -214,13 +214,13 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
 // Tensor-core assignment fused with the centroid sums of the next update.
 // Persistent: CTA b takes the global 128-row tiles [b per, (b+1) per) (tile i = row tile
 // i mod T of head i / T) and runs them through a pipeline:
-//   warp 9      loads the X tile (contiguous rows, cp.async) into a three-deep ring
-//   warp 8      (lane 0) scores S = X [w_hi w_lo]^T into a double-buffered TMEM tile, then,
+//   warp 17     loads the X tile (contiguous rows, cp.async) into a three-deep ring
+//   warp 16     (lane 0) scores S = X [w_hi w_lo]^T into a double-buffered TMEM tile, then,
 //               once the labels are known, adds onehot(labels)^T X into a TMEM sum
 //               (M = 128 groups x N = d; A and B both MN-major, read straight from the
 //               one-hot tile and the X tile)
-//   warps 0-7   row r = TMEM lane r, columns split in two halves (warps w and w + 4):
-//               argmin of bias_g - 2 s_g per half, merged through shared memory; the
+//   warps 0-15  row r = TMEM lane r, columns split in four quarters (warps w, w + 4, w + 8,
+//               w + 12): argmin of bias_g - 2 s_g per quarter, merged through shared memory; the
 //               label goes into the sums through a one-hot row; a row whose runner-up is
 //               within twice the error bound also goes on the list of the exact re-check,
 //               which corrects its label (and, through the correction list, the sums) if
@@ -229,10 +229,11 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
 // partial slot (CTA, head - first head of the CTA).
 // ---------------------------------------------------------------------------
 namespace kma {
-constexpr int NT = 320;
-constexpr int NEPI = 256;
-constexpr int MMA_WARP = 8;
-constexpr int LOAD_WARP = 9;
+constexpr int NT = 576;
+constexpr int NEPI = 512;
+constexpr int NQ = 4;   // column quarters
+constexpr int MMA_WARP = 16;
+constexpr int LOAD_WARP = 17;
 constexpr int XS = 3;   // X ring depth
 struct Bars {
   uint64_t xfull[XS], xempty[XS], tfull[2], tempty[2], ohfull, ohempty, sumdone, xready[2], epidone;
@@ -264,8 +265,8 @@ __global__ void __launch_bounds__(kma::NT, 1)
   const uint32_t kW = (uint32_t)GP * D * 2u;
   constexpr int XS = kma::XS;
   const uint32_t sX = base, sOH = base + XS * kX, sWh = sOH + kOH, sWl = sWh + kW;
-  kma::Half* xchg = reinterpret_cast<kma::Half*>(smem + XS * kX + kOH + 2 * kW);   // [2 tiles][2 halves][128]
-  float* sBias = reinterpret_cast<float*>(xchg + 2 * 2 * 128);                      // [GP]
+  kma::Half* xchg = reinterpret_cast<kma::Half*>(smem + XS * kX + kOH + 2 * kW);   // [2 tiles][NQ][128]
+  float* sBias = reinterpret_cast<float*>(xchg + 2 * kma::NQ * 128);                // [GP]
   int* sCnt = reinterpret_cast<int*>(sBias + GP);                                    // [GP]
   kma::Bars* bars = reinterpret_cast<kma::Bars*>(sCnt + GP);
   int* sMisc = reinterpret_cast<int*>(bars + 1);   // [0] tmem, [1] abort, [2] max ||w|| bits
@@ -394,8 +395,8 @@ __global__ void __launch_bounds__(kma::NT, 1)
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       it = __shfl_sync(0xffffffffu, it, 0);
     } else {
-      // ---------------- labels, one-hot rows, flags (warps 0-7) ----------------
-      const int hf = warp >> 2;                 // column half
+      // ---------------- labels, one-hot rows, flags (warps 0-15) ----------------
+      const int hf = warp >> 2;                 // column quarter
       const int r = (warp & 3) * 32 + lane;     // row = TMEM lane
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       for (int i = s0; i < s1 && ok; ++i, ++it) {
@@ -403,14 +404,13 @@ __global__ void __launch_bounds__(kma::NT, 1)
         ok = __all_sync(0xffffffffu, wait(bars->tfull[b], (it >> 1) & 1));
         if (!ok) break;
         tc_fence_after();
-        // argmin and runner-up of bias_g - 2 s_g over this half, in four interleaved sets
+        // argmin and runner-up of bias_g - 2 s_g over this quarter, in four interleaved sets
         float bst[4], snd[4];
         int bix[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) { bst[q] = __int_as_float(0x7f800000); snd[q] = bst[q]; bix[q] = 0; }
-#pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          const int cb = hf * 64 + c0;
+        {
+          const int cb = hf * 32;
           if (cb < GP) {
             uint32_t v[32];
             tc_ld32(tmem + 128 * b + lane_off + cb, v);
@@ -434,11 +434,11 @@ __global__ void __launch_bounds__(kma::NT, 1)
           h.second = take ? fminf(h.best, snd[q]) : fminf(h.second, bst[q]);
           if (take) { h.best = bst[q]; h.bi = bix[q]; }
         }
-        // ||x||^2 of this half of the row, from the swizzled tile
+        // ||x||^2 of this quarter of the row, from the swizzled tile
         float xx = 0.f;
 #pragma unroll
-        for (int c = 0; c < CPR / 2; ++c) {
-          const uint4 u = *reinterpret_cast<const uint4*>(smem + xb * kX + tile_off(r, hf * (CPR / 2) + c, 128));
+        for (int c = 0; c < CPR / kma::NQ; ++c) {
+          const uint4 u = *reinterpret_cast<const uint4*>(smem + xb * kX + tile_off(r, hf * (CPR / kma::NQ) + c, 128));
           const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -447,20 +447,27 @@ __global__ void __launch_bounds__(kma::NT, 1)
           }
         }
         h.xx = xx;
-        xchg[(b * 2 + hf) * 128 + r] = h;
-        // both halves of every row are in (an mbarrier, so an abort cannot strand a warp)
+        xchg[(b * kma::NQ + hf) * 128 + r] = h;
+        // every quarter of every row is in (an mbarrier, so an abort cannot strand a warp)
         mbar_arrive(su32(&bars->xready[b]));
         ok = __all_sync(0xffffffffu, wait(bars->xready[b], (it >> 1) & 1));
         if (!ok) break;
-        const kma::Half h0 = xchg[(b * 2 + 0) * 128 + r], h1 = xchg[(b * 2 + 1) * 128 + r];
-        // merge: half 0 holds the lower columns, so it wins ties
-        const bool take1 = h1.best < h0.best;
-        const float best = take1 ? h1.best : h0.best;
-        const float second = take1 ? fminf(h0.best, h1.second) : fminf(h0.second, h1.best);
-        const int bi = take1 ? h1.bi : h0.bi;
+        // merge in column order, so a lower quarter wins ties
+        kma::Half m = xchg[(b * kma::NQ + 0) * 128 + r];
+        float xsum = m.xx;
+#pragma unroll
+        for (int q = 1; q < kma::NQ; ++q) {
+          const kma::Half o = xchg[(b * kma::NQ + q) * 128 + r];
+          xsum += o.xx;
+          const bool take = o.best < m.best;
+          m.second = take ? fminf(m.best, o.second) : fminf(m.second, o.best);
+          if (take) { m.best = o.best; m.bi = o.bi; }
+        }
+        const float best = m.best, second = m.second;
+        const int bi = m.bi;
         const bool in = row < N;
         if (in && hf == 0) {
-          const float bound = kc * sqrtf(h0.xx + h1.xx) * wmax + 1e-6f * (fabsf(best) + fabsf(second));
+          const float bound = kc * sqrtf(xsum) * wmax + 1e-6f * (fabsf(best) + fabsf(second));
           labels[head + row] = bi;
           atomicAdd(&sCnt[bi], 1);
           if (second - best > 2.f * bound) {
@@ -470,12 +477,12 @@ __global__ void __launch_bounds__(kma::NT, 1)
             flag_rows[head + fs] = row;
           }
         }
-        // one-hot row r of this tile, this half's 8 chunks (zero for rows past N)
+        // one-hot row r of this tile, this quarter's 4 chunks (zero for rows past N)
         if (it >= 1) ok = __all_sync(0xffffffffu, wait(bars->ohempty, (it - 1) & 1));
         if (!ok) break;
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          const int c = hf * 8 + cc;
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = hf * 4 + cc;
           uint4 u = make_uint4(0u, 0u, 0u, 0u);
           if (in && (bi >> 3) == c) {
             const uint32_t one = 0x3F80u << (16 * (bi & 1));   // bf16 1.0 in the low or high half
@@ -487,16 +494,14 @@ __global__ void __launch_bounds__(kma::NT, 1)
         fence_proxy_async();
         mbar_arrive(su32(&bars->ohfull));
       }
-      // ---- sums and counts of this head -> partial slot (each half writes half the columns)
+      // ---- sums and counts of this head -> partial slot (each quarter writes 32 columns)
       if (ok) ok = __all_sync(0xffffffffu, wait(bars->sumdone, sg & 1));
       // every row's count is in sCnt
       mbar_arrive(su32(&bars->epidone));
       if (ok) ok = __all_sync(0xffffffffu, wait(bars->epidone, sg & 1));
       if (ok) {
         tc_fence_after();
-#pragma unroll
-        for (int c0 = 0; c0 < D / 2; c0 += 32) {
-          const int cb = hf * (D / 2) + c0;
+        for (int cb = hf * 32; cb < D; cb += 32 * kma::NQ) {
           uint32_t v[32];
           tc_ld32(tSum + lane_off + cb, v);
           if (r < GP) {
@@ -630,17 +635,20 @@ __global__ void __launch_bounds__(128) k_split3(const float* __restrict__ C, int
   }
 }
 
-// Roles of the 192 threads of the persistent cell-mass kernel: warps 0-3 take the softmax
-// of tile row r = TMEM lane r and the column sums, warp 4 allocates TMEM and its lane 0
-// issues the MMAs, warp 5 gathers the tile's query rows through perm_q (cp.async) into a
-// two-deep ring.  CTA b takes the (head, query group) items [b per, (b+1) per) in order;
+// Roles of the 576 threads of the persistent cell-mass kernel: warps 0-15 take the softmax
+// of tile row r = TMEM lane r, split over four column quarters (warps w, w+4, w+8, w+12):
+// each quarter exponentiates against its own running max, the quarters exchange (max, sum)
+// once, scale, and reduce their columns over the warp's 32 rows with a fixed butterfly;
+// warp 16 allocates TMEM and its lane 0 issues the MMAs, warp 17 gathers the tile's query
+// rows through perm_q (cp.async) into a two-deep ring.  CTA b takes the (head, query group) items [b per, (b+1) per) in order;
 // the K/V centroid parts of a head are reloaded when the head changes.
 namespace cmk {
-constexpr int NT = 192;
-constexpr int MMA_WARP = 4;
-constexpr int LOAD_WARP = 5;
+constexpr int NT = 576;
+constexpr int NSM = 512;   // softmax threads
+constexpr int MMA_WARP = 16;
+constexpr int LOAD_WARP = 17;
 struct Bars {
-  uint64_t xfull[2], xempty[2], tfull[2], tempty[2], pready[2];
+  uint64_t xfull[2], xempty[2], tfull[2], tempty[2], mready[2], pready[2];
 };
 }  // namespace cmk
 
@@ -683,8 +691,9 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
   constexpr int CPR = D / 8;
   const uint32_t kC = (uint32_t)GP * D * 2u;
   const uint32_t sX = base, sC = base + 2 * kX;
-  float* part = reinterpret_cast<float*>(smem + 2 * kX + 3 * kC);   // [2 tiles][4][GP]
-  float* colacc = part + 8 * GP;                                     // [GP]
+  float* part = reinterpret_cast<float*>(smem + 2 * kX + 3 * kC);   // [2 tiles][16 warps][32]
+  float2* msx = reinterpret_cast<float2*>(part + 2 * 16 * 32);       // [2 tiles][4 quarters][128]
+  float* colacc = reinterpret_cast<float*>(msx + 2 * 4 * 128);       // [GP]
   float* lnn = colacc + GP;                                          // [GP] log2 n_g or -inf
   cmk::Bars* bars = reinterpret_cast<cmk::Bars*>(lnn + GP);
   int* sMisc = reinterpret_cast<int*>(bars + 1);                     // [0] tmem, [1] abort
@@ -698,8 +707,9 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
       mbar_init(su32(&bars->xfull[b]), 32);
       mbar_init(su32(&bars->xempty[b]), 1);
       mbar_init(su32(&bars->tfull[b]), 1);
-      mbar_init(su32(&bars->tempty[b]), 128);
-      mbar_init(su32(&bars->pready[b]), 128);
+      mbar_init(su32(&bars->tempty[b]), cmk::NSM);
+      mbar_init(su32(&bars->mready[b]), cmk::NSM);
+      mbar_init(su32(&bars->pready[b]), cmk::NSM);
     }
     fence_barrier_init();
   }
@@ -796,14 +806,16 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       tile = __shfl_sync(0xffffffffu, tile, 0);
-    } else if (warp < 4) {
-      // ---------------- softmax + column sums ----------------
-      const int r = tid;   // tile row = TMEM lane
-      const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    } else if (warp < 16) {
+      // ---------------- softmax + column sums (warp = quarter * 4 + row group) ----------------
+      const int qt = warp >> 2, rg = warp & 3;
+      const int r = rg * 32 + lane;   // tile row = TMEM lane
+      const int cb = qt * 32;         // this quarter's columns
+      const uint32_t lane_off = (uint32_t)(rg * 32) << 16;
       for (int a = a0; a < a1 && ok; ++a) {
         const int n_a = qo[a + 1] - qo[a];
         if (n_a == 0) {
-          if (r < Gk) mass[((size_t)bh * Gq + a) * Gk + r] = 0.f;
+          if (qt == 0 && r < Gk) mass[((size_t)bh * Gq + a) * Gk + r] = 0.f;
           continue;
         }
         for (int t0 = qo[a]; t0 < qo[a + 1]; t0 += 128, ++tile) {
@@ -811,53 +823,56 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
           ok = __all_sync(0xffffffffu, wait(bars->tfull[b], (tile >> 1) & 1));
           if (!ok) break;
           tc_fence_after();
-          float v[128];
+          float v[32];
+          if (cb < GP) {
+            uint32_t u[32];
+            tc_ld32(tmem + 128 * b + lane_off + cb, u);
 #pragma unroll
-          for (int c0 = 0; c0 < 128; c0 += 32) {
-            if (c0 < GP) {
-              uint32_t u[32];
-              tc_ld32(tmem + 128 * b + lane_off + c0, u);
-#pragma unroll
-              for (int e = 0; e < 32; ++e) v[c0 + e] = __uint_as_float(u[e]);
-            }
+            for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(u[e]);
           }
           tc_fence_before();
           mbar_arrive(su32(&bars->tempty[b]));
-          float mx = NEG_INF;
+          // this quarter: logits in log2 units, local max and local sum
+          float mq = NEG_INF;
+          if (cb < GP) {
 #pragma unroll
-          for (int g = 0; g < 128; ++g) {
-            if (g < GP) {
-              const float ln = lnn[g];
-              v[g] = ln == NEG_INF ? NEG_INF : fmaf(v[g], scale_log2, ln);
-              mx = fmaxf(mx, v[g]);
+            for (int e = 0; e < 32; ++e) {
+              const float ln = lnn[cb + e];
+              v[e] = ln == NEG_INF ? NEG_INF : fmaf(v[e], scale_log2, ln);
+              mq = fmaxf(mq, v[e]);
             }
           }
-          float sum = 0.f;
+          float sq = 0.f;
 #pragma unroll
-          for (int g = 0; g < 128; ++g) {
-            if (g < GP) {
-              v[g] = v[g] == NEG_INF ? 0.f : ex2(v[g] - mx);
-              sum += v[g];
-            }
+          for (int e = 0; e < 32; ++e) {
+            v[e] = (cb < GP && v[e] != NEG_INF) ? ex2(v[e] - mq) : 0.f;
+            sq += v[e];
           }
-          const float inv = (r < nr && sum > 0.f) ? 1.f / sum : 0.f;
+          msx[(b * 4 + qt) * 128 + r] = make_float2(mq, sq);
+          mbar_arrive(su32(&bars->mready[b]));
+          ok = __all_sync(0xffffffffu, wait(bars->mready[b], (tile >> 1) & 1));
+          if (!ok) break;
+          // row max and sum over the quarters (fixed order), then this quarter's scale
+          float M = NEG_INF;
 #pragma unroll
-          for (int c0 = 0; c0 < 128; c0 += 32) {
-            if (c0 < GP) {
-              float w[32];
+          for (int q = 0; q < 4; ++q) M = fmaxf(M, msx[(b * 4 + q) * 128 + r].x);
+          float S = 0.f;
 #pragma unroll
-              for (int e = 0; e < 32; ++e) w[e] = v[c0 + e] * inv;
-              part[(b * 4 + warp) * GP + c0 + lane] = lane_column_sum32(w, lane);
-            }
+          for (int q = 0; q < 4; ++q) {
+            const float2 ms = msx[(b * 4 + q) * 128 + r];
+            S += ms.x == NEG_INF ? 0.f : ms.y * ex2(ms.x - M);
           }
-          // every warp's column partials are in (double-buffered by tile, so one handshake
-          // per tile; an mbarrier, so an abort cannot strand a warp)
+          const float f = (r < nr && S > 0.f && mq != NEG_INF) ? ex2(mq - M) / S : 0.f;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] *= f;
+          part[(b * 16 + warp) * 32 + lane] = lane_column_sum32(v, lane);
           mbar_arrive(su32(&bars->pready[b]));
           ok = __all_sync(0xffffffffu, wait(bars->pready[b], (tile >> 1) & 1));
           if (!ok) break;
-          if (r < GP) {
-            const float* pb = part + b * 4 * GP;
-            colacc[r] += (pb[r] + pb[GP + r]) + (pb[2 * GP + r] + pb[3 * GP + r]);
+          if (qt == 0 && r < GP) {
+            // column r: the four row groups of its quarter, in order
+            const float* pb = part + (b * 16 + (r >> 5) * 4) * 32 + (r & 31);
+            colacc[r] += (pb[0] + pb[32]) + (pb[64] + pb[96]);
             if (t0 + 128 >= qo[a + 1]) {
               if (r < Gk) mass[((size_t)bh * Gq + a) * Gk + r] = colacc[r] / (float)n_a;
               colacc[r] = 0.f;
@@ -884,7 +899,7 @@ int kmeans_gp(int G) { return (G + 31) / 32 * 32; }
 
 size_t assign_acc_smem(int D, int GP) {
   return (size_t)km::kma::XS * 128 * D * 2 + (size_t)128 * 128 * 2 + 2 * (size_t)GP * D * 2 +
-         4 * 128 * sizeof(km::kma::Half) + (size_t)GP * 8 + sizeof(km::kma::Bars) + 16;
+         2 * km::kma::NQ * 128 * sizeof(km::kma::Half) + (size_t)GP * 8 + sizeof(km::kma::Bars) + 16;
 }
 
 KmPlan kmeans_plan(int BH, int N) {
@@ -977,7 +992,8 @@ cudaError_t launch_assign_recheck(const void* X, int BH, int N, int d, const flo
 }
 
 size_t cell_mass_tc_smem(int D, int GP) {
-  return (size_t)2 * 128 * D * 2 + 3 * (size_t)GP * D * 2 + (size_t)10 * GP * 4 + sizeof(km::cmk::Bars) + 16;
+  return (size_t)2 * 128 * D * 2 + 3 * (size_t)GP * D * 2 + (size_t)2 * 16 * 32 * 4 + (size_t)2 * 4 * 128 * 8 +
+         (size_t)2 * GP * 4 + sizeof(km::cmk::Bars) + 16;
 }
 
 static int sm_count() {
