@@ -27,6 +27,13 @@ cudaError_t launch_block_mask(const unsigned char* route, int BH, int N, int Gq,
                               const int* perm_q, const int* label_q, const int* perm_k, const int* label_k,
                               unsigned char* bmask, cudaStream_t st);
 
+// tma_host.cu: 128-byte tensor map (CUtensorMap) of a row-major bf16 matrix for boxes of
+// box_rows x 64 columns with 128B swizzle; rows past the end read as zeros.
+cudaError_t make_tmap_bf16_rows(void* tmap, const void* base, unsigned long long rows, int cols, int box_rows);
+struct alignas(64) TmapBlob {
+  unsigned long long w[16];
+};
+
 // kmeans_tc.cu
 int kmeans_gp(int G);
 size_t centroid_weights_smem(int d, int D);

@@ -11,6 +11,8 @@
 // rigorous error bound of the split-bf16 products and fp32 accumulation; otherwise the
 // row is re-assigned by the exact fp32 direct form sum_c (y_c - nu_gc)^2 (ties -> lowest
 // g), which is the semantics the coordinates-based definition has.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -214,7 +216,8 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
 // Tensor-core assignment fused with the centroid sums of the next update.
 // Persistent: CTA b takes the global 128-row tiles [b per, (b+1) per) (tile i = row tile
 // i mod T of head i / T) and runs them through a pipeline:
-//   warp 17     loads the X tile (contiguous rows, cp.async) into a three-deep ring
+//   warp 17     (lane 0) loads the X tile (contiguous rows, two TMA boxes of 128 rows x 64
+//               columns, 128B-swizzled) into a three-deep ring
 //   warp 16     (lane 0) scores S = X [w_hi w_lo]^T into a double-buffered TMEM tile, then,
 //               once the labels are known, adds onehot(labels)^T X into a TMEM sum
 //               (M = 128 groups x N = d; A and B both MN-major, read straight from the
@@ -246,7 +249,7 @@ struct Half {
 
 template <int D>
 __global__ void __launch_bounds__(kma::NT, 1)
-    k_assign_acc(const __nv_bfloat16* __restrict__ X, int N, int GP, int T, int total, int per, int maxh,
+    k_assign_acc(const __grid_constant__ CUtensorMap tmx, int N, int GP, int T, int total, int per, int maxh,
                  const __nv_bfloat16* __restrict__ w_hi, const __nv_bfloat16* __restrict__ w_lo,
                  const float* __restrict__ bias, const float* __restrict__ wnorm, int* __restrict__ labels,
                  int* __restrict__ trace, int* __restrict__ flag_count, int* __restrict__ flag_rows,
@@ -276,7 +279,7 @@ __global__ void __launch_bounds__(kma::NT, 1)
   if (tid == 0) {
     sMisc[1] = 0;
     for (int b = 0; b < XS; ++b) {
-      mbar_init(su32(&bars->xfull[b]), 32);
+      mbar_init(su32(&bars->xfull[b]), 1);
       mbar_init(su32(&bars->xempty[b]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -339,20 +342,21 @@ __global__ void __launch_bounds__(kma::NT, 1)
     const float wmax = __int_as_float(sMisc[2]);
 
     if (warp == kma::LOAD_WARP) {
-      // ---------------- loads ----------------
-      for (int i = s0; i < s1 && ok; ++i, ++it) {
-        const int xb = it % XS, n0 = (i - bh * T) * 128;
-        if (it >= XS) ok = __all_sync(0xffffffffu, wait(bars->xempty[xb], ((it / XS) - 1) & 1));
-        if (!ok) break;
-#pragma unroll 4
-        for (int q = 0; q < 128 * CPR / 32; ++q) {
-          const int e = q * 32 + lane, r = e / CPR, c = e % CPR;
-          const bool in = n0 + r < N;
-          cp_async16(sX + xb * kX + tile_off(r, c, 128), X + (head + (in ? n0 + r : 0)) * D + c * 8, in);
+      // ---------------- loads (rows past this head's N belong to the next head or read as
+      // zeros; their labels and one-hot rows are never used) ----------------
+      if (lane == 0) {
+        for (int i = s0; i < s1 && ok; ++i, ++it) {
+          const int xb = it % XS, n0 = (i - bh * T) * 128;
+          if (it >= XS) ok = wait(bars->xempty[xb], ((it / XS) - 1) & 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(su32(&bars->xfull[xb]), kX);
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_2d(sX + xb * kX + h * 16384, &tmx, 64 * h, (int)(head + n0), su32(&bars->xfull[xb]));
         }
-        cp_async_arrive_noinc(su32(&bars->xfull[xb]));
       }
-      cp_async_wait_all();
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      it = __shfl_sync(0xffffffffu, it, 0);
     } else if (warp == kma::MMA_WARP) {
       // ---------------- MMA ----------------
       if (lane == 0) {
@@ -401,7 +405,8 @@ __global__ void __launch_bounds__(kma::NT, 1)
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       for (int i = s0; i < s1 && ok; ++i, ++it) {
         const int b = it & 1, xb = it % XS, row = (i - bh * T) * 128 + r;
-        ok = __all_sync(0xffffffffu, wait(bars->tfull[b], (it >> 1) & 1));
+        // scores ready; the X tile (read below for ||x||) completed before them
+        ok = __all_sync(0xffffffffu, wait(bars->tfull[b], (it >> 1) & 1) && wait(bars->xfull[xb], (it / XS) & 1));
         if (!ok) break;
         tc_fence_after();
         // argmin and runner-up of bias_g - 2 s_g over this quarter, in four interleaved sets
@@ -946,16 +951,19 @@ cudaError_t launch_assign_acc(const void* X, int BH, int N, int d, int G, const 
   const int GP = kmeans_gp(G);
   const size_t sm = assign_acc_smem(d, GP);
   const KmPlan pl = kmeans_plan(BH, N);
+  CUtensorMap tmx;
+  cudaError_t e = make_tmap_bf16_rows(&tmx, X, (unsigned long long)BH * N, d, 128);
+  if (e != cudaSuccess) return e;
   if (d == 64) {
     cudaFuncSetAttribute(km::k_assign_acc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     km::k_assign_acc<64><<<pl.grid, km::kma::NT, sm, st>>>(
-        (const __nv_bfloat16*)X, N, GP, pl.T, pl.total, pl.per, pl.maxh, (const __nv_bfloat16*)w_hi,
-        (const __nv_bfloat16*)w_lo, bias, wnorm, labels, trace, flag_count, flag_rows, psum, pcnt, err);
+        tmx, N, GP, pl.T, pl.total, pl.per, pl.maxh, (const __nv_bfloat16*)w_hi, (const __nv_bfloat16*)w_lo, bias,
+        wnorm, labels, trace, flag_count, flag_rows, psum, pcnt, err);
   } else {
     cudaFuncSetAttribute(km::k_assign_acc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     km::k_assign_acc<128><<<pl.grid, km::kma::NT, sm, st>>>(
-        (const __nv_bfloat16*)X, N, GP, pl.T, pl.total, pl.per, pl.maxh, (const __nv_bfloat16*)w_hi,
-        (const __nv_bfloat16*)w_lo, bias, wnorm, labels, trace, flag_count, flag_rows, psum, pcnt, err);
+        tmx, N, GP, pl.T, pl.total, pl.per, pl.maxh, (const __nv_bfloat16*)w_hi, (const __nv_bfloat16*)w_lo, bias,
+        wnorm, labels, trace, flag_count, flag_rows, psum, pcnt, err);
   }
   return cudaGetLastError();
 }

@@ -1,19 +1,24 @@
 // Exact probe rows on the tensor cores (gist.science technical summary, section 2.B:
 // probe rows evaluated exactly, R = O_dense - O_sparse).
 //
-// One CTA = the (up to 64) probe rows of one head against one contiguous key split.
-// For every 64-key chunk the tensor cores compute S = Q K^T once; the softmax warps
-// turn it into two probability tiles -- over all keys (dense) and over the keys whose
-// K/V group is routed for the probe row's query group (sparse) -- and the tensor cores
-// accumulate both O_dense += P_dense V and O_sparse += P_sparse V in TMEM.  The
-// probabilities are kept to ~2^-17 by splitting them into bf16 hi + lo tiles (two MMAs
-// each), so the probe outputs carry fp32-level error, not bf16's.  Each split
-// writes base-2 running maxima, sums and unnormalised outputs in fp32; the existing
-// combine kernel merges the splits.
+// One CTA = the (up to 64) probe rows of one head against one contiguous key split.  The
+// 128-row MMA tile holds every probe row twice: rows 0-63 take the softmax over all keys
+// (dense), rows 64-127 the softmax over the keys whose K/V group is routed for the probe
+// row's query group (sparse).  So for every 128-key chunk one S = Q K^T gives both, one
+// set of PV MMAs accumulates both O_dense (rows 0-63) and O_sparse (rows 64-127) in TMEM,
+// and each of the four softmax warps (one per TMEM sub-partition) has real rows.  The
+// probabilities are kept to ~2^-17 by splitting them into bf16 hi + lo, both written to
+// TMEM and both used as the A operand of the PV MMAs, so the probe outputs carry
+// fp32-level error, not bf16's.  Each split writes base-2 running maxima, sums and
+// unnormalised outputs in fp32; the combine kernel merges the splits.
 //
-// Roles (256 threads): warps 0-3 softmax (thread t = probe row t, TMEM lane t), warp 4
-// TMEM allocation + MMA issue (lane 0), warps 5-7 cp.async loads (probe rows gathered
-// through probe_idx; key/value rows and their labels contiguous).  All waits bounded.
+// Roles (192 threads): warps 0-3 softmax (thread r = tile row r = TMEM lane r), warp 4
+// TMEM allocation + MMA issue (lane 0), warp 5 loads: the probe rows (cp.async, gathered
+// through probe_idx), the K and V chunks (TMA, two-deep ring) and the chunk's key labels.
+// TMEM: S at columns 0 / 128 (two buffers), P hi at 256, P lo at 320, O at 384.
+// All waits bounded.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -23,55 +28,52 @@ namespace ptc {
 
 using namespace spr::tc;
 
-constexpr int BM = 128;   // rows of the MMA tile (probe rows + zero padding)
-constexpr int BN = 64;    // keys per chunk
+constexpr int BM = 128;    // tile rows: probe rows (dense) then probe rows again (sparse)
+constexpr int PROWS = 64;  // probe rows per split (matches the combine's layout)
+constexpr int BN = 128;    // keys per chunk
 constexpr int NSOFT = 128;
 constexpr int MMA_WARP = 4;
-constexpr int PROD0 = 160;
-constexpr int NPROD = 96;
-constexpr int NT = 256;
-constexpr int PROWS = 64;  // probe rows stored per split (matches the combine's layout)
+constexpr int LOAD_WARP = 5;
+constexpr int NT = 192;
 constexpr float kRescaleThreshold = 8.0f;
 
 struct Bars {
-  uint64_t q, full[2], empty[2], s_full[2], s_free[2], p_full, o_done, mma_done;
+  uint64_t q, full[2], empty[2], s_full[2], s_free[2], p_full, p_empty, o_done, mma_done;
 };
 
 template <int D>
 struct Layout {
   static constexpr uint32_t kQ = (uint32_t)BM * D * 2;    // Q tile
   static constexpr uint32_t kKV = (uint32_t)BN * D * 2;   // one K or V chunk
-  static constexpr uint32_t kP = (uint32_t)BM * BN * 2;   // one P tile
   static constexpr uint32_t oQ = 0;
   static constexpr uint32_t oK = oQ + kQ;
   static constexpr uint32_t oV = oK + 2 * kKV;
-  static constexpr uint32_t oPd = oV + 2 * kKV;            // P_dense hi, then lo at + kP
-  static constexpr uint32_t oPs = oPd + 2 * kP;            // P_sparse hi, then lo at + kP
-  static constexpr uint32_t oLab = oPs + 2 * kP;           // int [2][BN]
+  static constexpr uint32_t oLab = oV + 2 * kKV;           // int [2][BN]
   static constexpr uint32_t oBar = oLab + 2 * BN * 4;
   static constexpr uint32_t oInt = oBar + 256;
 };
 
 template <int D>
 __global__ void __launch_bounds__(NT, 1)
-    k_probe_tc(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
-               const __nv_bfloat16* __restrict__ V, int N, int Gk, int Gq, int P, const int* __restrict__ probe_idx,
-               const int* __restrict__ probe_grp, const int* __restrict__ label_k,
+    k_probe_tc(const __nv_bfloat16* __restrict__ Q, const __grid_constant__ CUtensorMap tmk,
+               const __grid_constant__ CUtensorMap tmv, int N, int Gk, int Gq, int P,
+               const int* __restrict__ probe_idx, const int* __restrict__ probe_grp, const int* __restrict__ label_k,
                const unsigned char* __restrict__ route, int keys_per_split, float scale_log2,
                float* __restrict__ part_o, float* __restrict__ part_ml, int* err) {
   using L = Layout<D>;
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  const uint32_t raw = su32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  unsigned char* smem = smem_raw + (base - raw);
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const uint32_t base = su32(smem);
+  if (base & 1023u) {
+    if (threadIdx.x == 0) set_error(err, DERR_INDEX);
+    return;
+  }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x, bh = blockIdx.y;
   const size_t head = (size_t)bh * N;
   Bars* bars = reinterpret_cast<Bars*>(smem + L::oBar);
   int* sLab = reinterpret_cast<int*>(smem + L::oLab);
-  int* sMisc = reinterpret_cast<int*>(smem + L::oInt);   // [0] tmem, [1] abort, [2] slot ok
-  int* sQrow = sMisc + 8;                                  // [BM]
-  unsigned char* sRoute = reinterpret_cast<unsigned char*>(sQrow + BM);  // [BM][Gk]
+  int* sMisc = reinterpret_cast<int*>(smem + L::oInt);   // [0] tmem, [1] abort
+  int* sQrow = sMisc + 8;                                  // [PROWS]
   volatile int* abort_flag = sMisc + 1;
 
   const int k0 = split * keys_per_split;
@@ -79,29 +81,25 @@ __global__ void __launch_bounds__(NT, 1)
   const int nchunks = k1 > k0 ? (k1 - k0 + BN - 1) / BN : 0;
 
   // ---------------- setup ----------------
-  for (int r = tid; r < BM; r += NT) {
+  for (int r = tid; r < PROWS; r += NT) {
     int row = -1;
     if (r < P) {
       row = probe_idx[(size_t)bh * P + r];
-      if (row < 0 || row >= N) row = -1;
+      if (row < 0 || row >= N) { set_error(err, DERR_INDEX); row = -1; }
     }
     sQrow[r] = row;
   }
-  for (int e = tid; e < BM * Gk; e += NT) {
-    const int r = e / Gk, g = e - r * Gk;
-    const int a = r < P ? probe_grp[(size_t)bh * P + r] : -1;
-    sRoute[e] = (a >= 0 && a < Gq) ? route[((size_t)bh * Gq + a) * Gk + g] : 0;
-  }
   if (tid == 0) {
     sMisc[1] = 0;
-    mbar_init(su32(&bars->q), NPROD);
+    mbar_init(su32(&bars->q), 32);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(su32(&bars->full[s]), NPROD);
+      mbar_init(su32(&bars->full[s]), 33);   // 32 label arrivals + the TMA transaction arrival
       mbar_init(su32(&bars->empty[s]), 1);
       mbar_init(su32(&bars->s_full[s]), 1);
       mbar_init(su32(&bars->s_free[s]), NSOFT);
     }
     mbar_init(su32(&bars->p_full), NSOFT);
+    mbar_init(su32(&bars->p_empty), 1);
     mbar_init(su32(&bars->o_done), 1);
     mbar_init(su32(&bars->mma_done), 1);
     fence_barrier_init();
@@ -114,40 +112,38 @@ __global__ void __launch_bounds__(NT, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = (uint32_t)sMisc[0];
-  const uint32_t sQ = base + L::oQ, sK = base + L::oK, sV = base + L::oV, sPd = base + L::oPd, sPs = base + L::oPs;
-  const uint32_t tS0 = tmem, tOd = tmem + 128, tOs = tmem + 128 + D;   // S buffers at 0 / 64
+  const uint32_t sQ = base + L::oQ, sK = base + L::oK, sV = base + L::oV;
+  const uint32_t tP = tmem + 256, tO = tmem + 384;
   auto wait = [&](uint64_t& bar, uint32_t parity) -> bool {
     return bounded_wait(su32(&bar), parity, abort_flag, err);
   };
 
-  if (tid >= PROD0) {
+  if (warp == LOAD_WARP) {
     // ---------------- loads ----------------
-    const int p = tid - PROD0;
     constexpr int CPR = D / 8;
-    for (int e = p; e < BM * CPR; e += NPROD) {
+    // probe rows, twice (tile rows r and r + 64)
+    for (int e = lane; e < BM * CPR; e += 32) {
       const int r = e / CPR, c = e - r * CPR;
-      const int row = sQrow[r];
+      const int row = sQrow[r & (PROWS - 1)];
       cp_async16(sQ + tile_off(r, c, BM), Q + (head + (row < 0 ? 0 : row)) * D + c * 8, row >= 0);
     }
     cp_async_arrive_noinc(su32(&bars->q));
-    volatile int* prod_ok = sMisc + 2;
-    for (int j = 0; j < nchunks; ++j) {
+    bool ok = true;
+    for (int j = 0; j < nchunks && ok; ++j) {
       const int s = j & 1;
-      if (p == 0) *prod_ok = (j < 2 || wait(bars->empty[s], ((j >> 1) - 1) & 1)) ? 1 : 0;
-      named_sync(1, NPROD);
-      if (!*prod_ok) break;
+      if (j >= 2) ok = __all_sync(0xffffffffu, wait(bars->empty[s], ((j >> 1) - 1) & 1));
+      if (!ok) break;
       const int c0 = k0 + j * BN;
-      const uint32_t dk = sK + s * L::kKV, dv = sV + s * L::kKV;
-      // 64 rows x CPR chunks for K and for V: 2 * 64 * CPR / 128 per thread
-      for (int e = p; e < BN * CPR; e += NPROD) {
-        const int r = e / CPR, c = e - r * CPR;
-        const bool ok = c0 + r < k1;
-        const size_t off = (head + (ok ? c0 + r : 0)) * D + c * 8;
-        const uint32_t o = tile_off(r, c, BN);
-        cp_async16(dk + o, K + off, ok);
-        cp_async16(dv + o, V + off, ok);
+      if (lane == 0) {
+        // K and V rows c0 .. c0+127 of this head (rows past k1 are masked in the softmax)
+        mbar_arrive_expect_tx(su32(&bars->full[s]), 2 * L::kKV);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_2d(sK + s * L::kKV + h * BN * 128, &tmk, 64 * h, (int)(head + c0), su32(&bars->full[s]));
+          tma_load_2d(sV + s * L::kKV + h * BN * 128, &tmv, 64 * h, (int)(head + c0), su32(&bars->full[s]));
+        }
       }
-      for (int r = p; r < BN; r += NPROD) {  // 4-byte labels (label rows are only 4-byte aligned)
+      for (int r = lane; r < BN; r += 32) {  // 4-byte labels (label rows are only 4-byte aligned)
         const bool v = c0 + r < k1;
         asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(su32(sLab + s * BN + r)),
                      "l"(label_k + head + (v ? c0 + r : 0)), "r"(v ? 4 : 0)
@@ -169,14 +165,11 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k) {
           const uint64_t bd = sdesc(vb + k * 2048, (uint32_t)BN * 128, 1024);
-          const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
-          tc_mma(tOd, sdesc(sPd + k * 32, 16, 1024), bd, IDO, acc);
-          tc_mma(tOd, sdesc(sPd + L::kP + k * 32, 16, 1024), bd, IDO, 1u);
-          tc_mma(tOs, sdesc(sPs + k * 32, 16, 1024), bd, IDO, acc);
-          tc_mma(tOs, sdesc(sPs + L::kP + k * 32, 16, 1024), bd, IDO, 1u);
+          tc_mma_ts(tO, tP + k * 8, bd, IDO, (i > 0 || k > 0) ? 1u : 0u);
+          tc_mma_ts(tO, tP + 64 + k * 8, bd, IDO, 1u);
         }
         tc_commit(su32(&bars->empty[i & 1]));
-        tc_commit(su32(&bars->o_done));
+        tc_commit(su32(&bars->p_empty));
         return true;
       };
       for (int j = 0; ok && j < nchunks; ++j) {
@@ -189,150 +182,143 @@ __global__ void __launch_bounds__(NT, 1)
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t oq = (k >> 2) * (BM * 128) + (k & 3) * 32;
           const uint32_t ok2 = (k >> 2) * (BN * 128) + (k & 3) * 32;
-          tc_mma(tS0 + s * BN, sdesc(sQ + oq, 16, 1024), sdesc(kb + ok2, 16, 1024), IDS, k > 0 ? 1u : 0u);
+          tc_mma(tmem + s * BN, sdesc(sQ + oq, 16, 1024), sdesc(kb + ok2, 16, 1024), IDS, k > 0 ? 1u : 0u);
         }
         tc_commit(su32(&bars->s_full[s]));
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok && nchunks > 0) issue_pv(nchunks - 1);
+      tc_commit(su32(&bars->o_done));
       tc_commit(su32(&bars->mma_done));
       wait(bars->mma_done, 0);
     }
   } else {
-    // ---------------- softmax (thread t = row t) ----------------
-    const int t = tid;
+    // ---------------- softmax (thread r = tile row r) ----------------
+    const int r = tid;
+    const bool sparse = r >= PROWS;
+    const int prow = r & (PROWS - 1);
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const unsigned char* rrow = sRoute + t * Gk;
-    float md = -INFINITY, ld = 0.f, ms = -INFINITY, ls = 0.f;
+    // routed K/V groups of this probe row's query group, as bits (sparse rows only)
+    uint32_t rm[4] = {0u, 0u, 0u, 0u};
+    if (sparse && prow < P) {
+      const int a = probe_grp[(size_t)bh * P + prow];
+      if (a >= 0 && a < Gq) {
+        const unsigned char* rr = route + ((size_t)bh * Gq + a) * Gk;
+        for (int g = 0; g < Gk; ++g)
+          if (rr[g]) rm[g >> 5] |= 1u << (g & 31);
+      }
+    }
+    float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nchunks; ++j) {
       const int b = j & 1;
-      ok = __all_sync(0xffffffffu, wait(bars->s_full[b], (j >> 1) & 1));
+      // S ready; the chunk's labels (read below) landed before it
+      ok = __all_sync(0xffffffffu, wait(bars->s_full[b], (j >> 1) & 1) && wait(bars->full[b], (j >> 1) & 1));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[64];
-      tc_ld32(tS0 + lane_off + b * BN, sr);
-      tc_ld32(tS0 + lane_off + b * BN + 32, sr + 32);
-      tc_fence_before();
-      mbar_arrive(su32(&bars->s_free[b]));
       const int valid = k1 - (k0 + j * BN);
       const int* lab = sLab + b * BN;
-      uint64_t rmask = 0;  // bit c: key c is routed for this row
-      float mxd = -INFINITY, mxs = -INFINITY;
+      // keys this row may use in the chunk, as 4 x 32 bits
+      uint32_t km[4];
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        if (c < valid) {
-          const float x = __uint_as_float(sr[c]);
-          mxd = fmaxf(mxd, x);
-          const int g = lab[c];
-          if (g >= 0 && g < Gk && rrow[g]) {
-            rmask |= 1ull << c;
-            mxs = fmaxf(mxs, x);
+      for (int w = 0; w < 4; ++w) {
+        uint32_t bits = 0u;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = 32 * w + e;
+          bool use = c < valid;
+          if (sparse) {
+            const int g = lab[c];
+            const uint32_t word = g < 32 ? rm[0] : g < 64 ? rm[1] : g < 96 ? rm[2] : rm[3];
+            use = use && g >= 0 && g < Gk && ((word >> (g & 31)) & 1u);
           }
+          bits |= (use ? 1u : 0u) << e;
         }
+        km[w] = bits;
       }
-      const float mnd = fmaxf(md, mxd * scale_log2);
-      const float mns = fmaxf(ms, mxs * scale_log2);
-      const bool need = (mnd > md + kRescaleThreshold) || (mns > ms + kRescaleThreshold) ||
-                        (md == -INFINITY && mnd != -INFINITY) || (ms == -INFINITY && mns != -INFINITY);
-      const bool warp_need = __any_sync(0xffffffffu, need);
-      float ad = 1.f, as = 1.f;
-      if (warp_need) {
-        if (mnd > md) { ad = (md == -INFINITY) ? 0.f : ex2(md - mnd); md = mnd; }
-        if (mns > ms) { as = (ms == -INFINITY) ? 0.f : ex2(ms - mns); ms = mns; }
-      }
-      const float mud = md == -INFINITY ? 0.f : md, mus = ms == -INFINITY ? 0.f : ms;
-      uint32_t pd[BN / 2], ps[BN / 2], pdl[BN / 2], psl[BN / 2];
-      float sd = 0.f, ss = 0.f;
+      uint32_t sreg[64];
+      float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < BN; c += 2) {
-        float e0 = 0.f, e1 = 0.f, f0 = 0.f, f1 = 0.f;
-        if (c < valid) {
-          const float x = __uint_as_float(sr[c]) * scale_log2;
-          e0 = ex2(x - mud);
-          if ((rmask >> c) & 1) f0 = ex2(x - mus);
-        }
-        if (c + 1 < valid) {
-          const float x = __uint_as_float(sr[c + 1]) * scale_log2;
-          e1 = ex2(x - mud);
-          if ((rmask >> (c + 1)) & 1) f1 = ex2(x - mus);
-        }
-        sd += e0 + e1;
-        ss += f0 + f1;
-        pd[c >> 1] = pack_bf16(e0, e1);
-        ps[c >> 1] = pack_bf16(f0, f1);
-        const __nv_bfloat162 hd = *reinterpret_cast<const __nv_bfloat162*>(&pd[c >> 1]);
-        const __nv_bfloat162 hs = *reinterpret_cast<const __nv_bfloat162*>(&ps[c >> 1]);
-        pdl[c >> 1] = pack_bf16(e0 - __low2float(hd), e1 - __high2float(hd));
-        psl[c >> 1] = pack_bf16(f0 - __low2float(hs), f1 - __high2float(hs));
+      for (int h = 0; h < 2; ++h) {
+        tc_ld64(tmem + b * BN + lane_off + 64 * h, sreg);
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if ((km[2 * h + (c >> 5)] >> (c & 31)) & 1u) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sreg[c]));
+        mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
       }
-      ld = ld * ad + sd;
-      ls = ls * as + ss;
+      const float mn = fmaxf(m, mx * scale_log2);
+      const bool need = (mn > m + kRescaleThreshold) || (m == -INFINITY && mn != -INFINITY);
+      const bool warp_need = __any_sync(0xffffffffu, need);
+      float alpha = 1.f;
+      if (warp_need && mn > m) {
+        alpha = (m == -INFINITY) ? 0.f : ex2(m - mn);
+        m = mn;
+      }
+      // P (single buffer) and O are free once PV of the previous chunk has completed
       if (j >= 1) {
-        ok = __all_sync(0xffffffffu, wait(bars->o_done, (j - 1) & 1));
+        ok = __all_sync(0xffffffffu, wait(bars->p_empty, (j - 1) & 1));
         if (!ok) break;
         tc_fence_after();
         if (warp_need) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tc_ld32(tOd + lane_off + c * 32, o);
+            tc_ld32(tO + lane_off + c * 32, o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * ad);
-            tc_st32(tOd + lane_off + c * 32, o);
-            tc_ld32(tOs + lane_off + c * 32, o);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * as);
-            tc_st32(tOs + lane_off + c * 32, o);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tc_st32(tO + lane_off + c * 32, o);
           }
         }
       }
+      const float mu = (m == -INFINITY) ? 0.f : m;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < BN / 8; ++c) {
-        const uint32_t o = tile_off(t, c, BM);
-        *reinterpret_cast<uint4*>(smem + L::oPd + o) = make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
-        *reinterpret_cast<uint4*>(smem + L::oPd + L::kP + o) =
-            make_uint4(pdl[4 * c], pdl[4 * c + 1], pdl[4 * c + 2], pdl[4 * c + 3]);
-        *reinterpret_cast<uint4*>(smem + L::oPs + o) = make_uint4(ps[4 * c], ps[4 * c + 1], ps[4 * c + 2], ps[4 * c + 3]);
-        *reinterpret_cast<uint4*>(smem + L::oPs + L::kP + o) =
-            make_uint4(psl[4 * c], psl[4 * c + 1], psl[4 * c + 2], psl[4 * c + 3]);
+      for (int h = 0; h < 2; ++h) {
+        tc_ld64(tmem + b * BN + lane_off + 64 * h, sreg);
+        uint32_t phi[32], plo[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const uint32_t kw = km[2 * h + (c >> 5)];
+          const float p0 = ((kw >> (c & 31)) & 1u) ? ex2(__uint_as_float(sreg[c]) * scale_log2 - mu) : 0.f;
+          const float p1 = ((kw >> ((c + 1) & 31)) & 1u) ? ex2(__uint_as_float(sreg[c + 1]) * scale_log2 - mu) : 0.f;
+          rs[(c >> 1) & 3] += p0 + p1;
+          const uint32_t hi = pack_bf16(p0, p1);
+          const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hi);
+          phi[c >> 1] = hi;
+          plo[c >> 1] = pack_bf16(p0 - __low2float(h2), p1 - __high2float(h2));
+        }
+        tc_st32(tP + lane_off + 32 * h, phi);
+        tc_st32(tP + lane_off + 64 + 32 * h, plo);
       }
-      fence_proxy_async();
       tc_fence_before();
+      mbar_arrive(su32(&bars->s_free[b]));
+      l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
       mbar_arrive(su32(&bars->p_full));
     }
-    if (ok && nchunks > 0) ok = __all_sync(0xffffffffu, wait(bars->o_done, (nchunks - 1) & 1));
+    if (ok && nchunks > 0) ok = __all_sync(0xffffffffu, wait(bars->o_done, 0));
     if (ok) {
       tc_fence_after();
-      const size_t rowbase = ((size_t)bh * gridDim.x + split) * PROWS + t;
+      const size_t rowbase = ((size_t)bh * gridDim.x + split) * PROWS + prow;
+      const int acc = sparse ? 1 : 0;
+      float* dst = part_o + (rowbase * 2 + acc) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t od[32], os[32];
+        uint32_t o[32];
         if (nchunks > 0) {
-          tc_ld32(tOd + lane_off + c * 32, od);
-          tc_ld32(tOs + lane_off + c * 32, os);
+          tc_ld32(tO + lane_off + c * 32, o);
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) od[e] = os[e] = 0u;
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
         }
-        if (t < PROWS) {
-          float4* dd = reinterpret_cast<float4*>(part_o + (rowbase * 2 + 0) * D + c * 32);
-          float4* dsp = reinterpret_cast<float4*>(part_o + (rowbase * 2 + 1) * D + c * 32);
+        float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            dd[e] = make_float4(__uint_as_float(od[4 * e]), __uint_as_float(od[4 * e + 1]),
-                                __uint_as_float(od[4 * e + 2]), __uint_as_float(od[4 * e + 3]));
-            dsp[e] = make_float4(__uint_as_float(os[4 * e]), __uint_as_float(os[4 * e + 1]),
-                                 __uint_as_float(os[4 * e + 2]), __uint_as_float(os[4 * e + 3]));
-          }
-        }
+        for (int e = 0; e < 8; ++e)
+          d4[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]), __uint_as_float(o[4 * e + 2]),
+                              __uint_as_float(o[4 * e + 3]));
       }
-      if (t < PROWS) {
-        part_ml[rowbase * 4 + 0] = md;
-        part_ml[rowbase * 4 + 1] = ld;
-        part_ml[rowbase * 4 + 2] = ms;
-        part_ml[rowbase * 4 + 3] = ls;
-      }
+      part_ml[rowbase * 4 + 2 * acc + 0] = m;
+      part_ml[rowbase * 4 + 2 * acc + 1] = l;
     }
   }
   tc_fence_before();
@@ -344,8 +330,9 @@ __global__ void __launch_bounds__(NT, 1)
 }  // namespace ptc
 
 size_t probe_tc_smem_bytes(int D, int Gk) {
+  (void)Gk;
   const size_t tiles = D == 64 ? ptc::Layout<64>::oInt : ptc::Layout<128>::oInt;
-  const size_t s = 1024 + tiles + (8 + ptc::BM) * 4 + (size_t)ptc::BM * Gk;
+  const size_t s = tiles + (8 + ptc::PROWS) * 4;
   return s < 120 * 1024 ? 120 * 1024 : s;  // one CTA per SM: it allocates all 512 TMEM columns
 }
 
@@ -355,17 +342,19 @@ cudaError_t launch_probe_tc(const void* Q, const void* K, const void* V, int BH,
   int kps = (N + S - 1) / S;
   kps = (kps + ptc::BN - 1) / ptc::BN * ptc::BN;
   const size_t sm = probe_tc_smem_bytes(D, Gk);
+  CUtensorMap tmk, tmv;
+  cudaError_t e = make_tmap_bf16_rows(&tmk, K, (unsigned long long)BH * N, D, ptc::BN);
+  if (e == cudaSuccess) e = make_tmap_bf16_rows(&tmv, V, (unsigned long long)BH * N, D, ptc::BN);
+  if (e != cudaSuccess) return e;
   dim3 grid(S, BH);
   if (D == 64) {
     cudaFuncSetAttribute(ptc::k_probe_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    ptc::k_probe_tc<64><<<grid, ptc::NT, sm, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
-                                                   (const __nv_bfloat16*)V, N, Gk, Gq, P, probe_idx, probe_grp,
-                                                   label_k, route, kps, scale_log2, part_o, part_ml, err);
+    ptc::k_probe_tc<64><<<grid, ptc::NT, sm, st>>>((const __nv_bfloat16*)Q, tmk, tmv, N, Gk, Gq, P, probe_idx,
+                                                   probe_grp, label_k, route, kps, scale_log2, part_o, part_ml, err);
   } else {
     cudaFuncSetAttribute(ptc::k_probe_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    ptc::k_probe_tc<128><<<grid, ptc::NT, sm, st>>>((const __nv_bfloat16*)Q, (const __nv_bfloat16*)K,
-                                                    (const __nv_bfloat16*)V, N, Gk, Gq, P, probe_idx, probe_grp,
-                                                    label_k, route, kps, scale_log2, part_o, part_ml, err);
+    ptc::k_probe_tc<128><<<grid, ptc::NT, sm, st>>>((const __nv_bfloat16*)Q, tmk, tmv, N, Gk, Gq, P, probe_idx,
+                                                    probe_grp, label_k, route, kps, scale_log2, part_o, part_ml, err);
   }
   return cudaGetLastError();
 }
