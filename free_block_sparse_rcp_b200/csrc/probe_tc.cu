@@ -12,9 +12,12 @@
 // fp32-level error, not bf16's.  Each split writes base-2 running maxima, sums and
 // unnormalised outputs in fp32; the combine kernel merges the splits.
 //
-// Roles (192 threads): warps 0-3 softmax (thread r = tile row r = TMEM lane r), warp 4
-// TMEM allocation + MMA issue (lane 0), warp 5 loads: the probe rows (cp.async, gathered
-// through probe_idx), the K and V chunks (TMA, two-deep ring) and the chunk's key labels.
+// Roles (576 threads): warps 0-15 softmax, warp = quarter * 4 + row group: thread = tile row
+// (row group * 32 + lane = TMEM lane) x 32-key quarter of the chunk; the four quarters of a
+// row exchange their maxima once per chunk (mbarrier) and keep separate partial sums,
+// added at the end.  Warp 16: TMEM allocation + MMA issue (lane 0).  Warp 17: loads -- the
+// probe rows (cp.async, gathered through probe_idx), the K and V chunks (TMA, two-deep
+// ring) and the chunk's key labels.
 // TMEM: S at columns 0 / 128 (two buffers), P hi at 256, P lo at 320, O at 384.
 // All waits bounded.
 #include <cuda.h>
@@ -31,14 +34,14 @@ using namespace spr::tc;
 constexpr int BM = 128;    // tile rows: probe rows (dense) then probe rows again (sparse)
 constexpr int PROWS = 64;  // probe rows per split (matches the combine's layout)
 constexpr int BN = 128;    // keys per chunk
-constexpr int NSOFT = 128;
-constexpr int MMA_WARP = 4;
-constexpr int LOAD_WARP = 5;
-constexpr int NT = 192;
+constexpr int NSOFT = 512;   // softmax threads
+constexpr int MMA_WARP = 16;
+constexpr int LOAD_WARP = 17;
+constexpr int NT = 576;
 constexpr float kRescaleThreshold = 8.0f;
 
 struct Bars {
-  uint64_t q, full[2], empty[2], s_full[2], s_free[2], p_full, p_empty, o_done, mma_done;
+  uint64_t q, full[2], empty[2], s_full[2], s_free[2], p_full, p_empty, o_done, mma_done, mready[2], ldone;
 };
 
 template <int D>
@@ -49,7 +52,8 @@ struct Layout {
   static constexpr uint32_t oK = oQ + kQ;
   static constexpr uint32_t oV = oK + 2 * kKV;
   static constexpr uint32_t oLab = oV + 2 * kKV;           // int [2][BN]
-  static constexpr uint32_t oBar = oLab + 2 * BN * 4;
+  static constexpr uint32_t oXm = oLab + 2 * BN * 4;       // float [2][4][BM] quarter maxima, [4][BM] sums
+  static constexpr uint32_t oBar = oXm + 3 * 4 * BM * 4;
   static constexpr uint32_t oInt = oBar + 256;
 };
 
@@ -102,6 +106,9 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(su32(&bars->p_empty), 1);
     mbar_init(su32(&bars->o_done), 1);
     mbar_init(su32(&bars->mma_done), 1);
+    mbar_init(su32(&bars->mready[0]), NSOFT);
+    mbar_init(su32(&bars->mready[1]), NSOFT);
+    mbar_init(su32(&bars->ldone), NSOFT);
     fence_barrier_init();
   }
   if (warp == MMA_WARP) {
@@ -192,12 +199,14 @@ __global__ void __launch_bounds__(NT, 1)
       tc_commit(su32(&bars->mma_done));
       wait(bars->mma_done, 0);
     }
-  } else {
-    // ---------------- softmax (thread r = tile row r) ----------------
-    const int r = tid;
+  } else if (warp < 16) {
+    // ---------------- softmax (row r, keys of quarter qt) ----------------
+    const int qt = warp >> 2, rg = warp & 3;
+    const int r = rg * 32 + lane;
     const bool sparse = r >= PROWS;
     const int prow = r & (PROWS - 1);
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(rg * 32) << 16;
+    float* xm = reinterpret_cast<float*>(smem + L::oXm);   // [2][4][BM]
     // routed K/V groups of this probe row's query group, as bits (sparse rows only)
     uint32_t rm[4] = {0u, 0u, 0u, 0u};
     if (sparse && prow < P) {
@@ -217,36 +226,37 @@ __global__ void __launch_bounds__(NT, 1)
       if (!ok) break;
       tc_fence_after();
       const int valid = k1 - (k0 + j * BN);
-      const int* lab = sLab + b * BN;
-      // keys this row may use in the chunk, as 4 x 32 bits
-      uint32_t km[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        uint32_t bits = 0u;
+      // keys of this quarter the row may use
+      uint32_t km = 0u;
+      {
+        const int* lab = sLab + b * BN + qt * 32;
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const int c = 32 * w + e;
-          bool use = c < valid;
+          bool use = qt * 32 + e < valid;
           if (sparse) {
-            const int g = lab[c];
+            const int g = lab[e];
             const uint32_t word = g < 32 ? rm[0] : g < 64 ? rm[1] : g < 96 ? rm[2] : rm[3];
             use = use && g >= 0 && g < Gk && ((word >> (g & 31)) & 1u);
           }
-          bits |= (use ? 1u : 0u) << e;
+          km |= (use ? 1u : 0u) << e;
         }
-        km[w] = bits;
       }
-      uint32_t sreg[64];
-      float mx = -INFINITY;
+      uint32_t sreg[32];
+      tc_ld32(tmem + b * BN + lane_off + qt * 32, sreg);
+      tc_fence_before();
+      mbar_arrive(su32(&bars->s_free[b]));
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        tc_ld64(tmem + b * BN + lane_off + 64 * h, sreg);
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      for (int e = 0; e < 32; ++e)
+        if ((km >> e) & 1u) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(sreg[e]));
+      xm[(b * 4 + qt) * BM + r] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      mbar_arrive(su32(&bars->mready[b]));
+      ok = __all_sync(0xffffffffu, wait(bars->mready[b], (j >> 1) & 1));
+      if (!ok) break;
+      float mx = xm[(b * 4 + 0) * BM + r];
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if ((km[2 * h + (c >> 5)] >> (c & 31)) & 1u) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sreg[c]));
-        mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
-      }
+      for (int q = 1; q < 4; ++q) mx = fmaxf(mx, xm[(b * 4 + q) * BM + r]);
+      // every quarter of the row takes the same decision from the same values
       const float mn = fmaxf(m, mx * scale_log2);
       const bool need = (mn > m + kRescaleThreshold) || (m == -INFINITY && mn != -INFINITY);
       const bool warp_need = __any_sync(0xffffffffu, need);
@@ -261,64 +271,81 @@ __global__ void __launch_bounds__(NT, 1)
         if (!ok) break;
         tc_fence_after();
         if (warp_need) {
+          // this quarter rescales D/4 columns of the row's O
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tc_ld32(tO + lane_off + c * 32, o);
+          for (int c0 = 0; c0 < D / 4; c0 += 16) {
+            uint32_t o[16];
+            const uint32_t ta = tO + lane_off + qt * (D / 4) + c0;
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+                "tcgen05.wait::ld.sync.aligned;\n"
+                : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]), "=r"(o[7]),
+                  "=r"(o[8]), "=r"(o[9]), "=r"(o[10]), "=r"(o[11]), "=r"(o[12]), "=r"(o[13]), "=r"(o[14]), "=r"(o[15])
+                : "r"(ta)
+                : "memory");
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tc_st32(tO + lane_off + c * 32, o);
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tc_st16(ta, o);
           }
         }
       }
       const float mu = (m == -INFINITY) ? 0.f : m;
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t phi[16], plo[16];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        tc_ld64(tmem + b * BN + lane_off + 64 * h, sreg);
-        uint32_t phi[32], plo[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const uint32_t kw = km[2 * h + (c >> 5)];
-          const float p0 = ((kw >> (c & 31)) & 1u) ? ex2(__uint_as_float(sreg[c]) * scale_log2 - mu) : 0.f;
-          const float p1 = ((kw >> ((c + 1) & 31)) & 1u) ? ex2(__uint_as_float(sreg[c + 1]) * scale_log2 - mu) : 0.f;
-          rs[(c >> 1) & 3] += p0 + p1;
-          const uint32_t hi = pack_bf16(p0, p1);
-          const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hi);
-          phi[c >> 1] = hi;
-          plo[c >> 1] = pack_bf16(p0 - __low2float(h2), p1 - __high2float(h2));
-        }
-        tc_st32(tP + lane_off + 32 * h, phi);
-        tc_st32(tP + lane_off + 64 + 32 * h, plo);
+      for (int e = 0; e < 32; e += 2) {
+        const float p0 = ((km >> e) & 1u) ? ex2(__uint_as_float(sreg[e]) * scale_log2 - mu) : 0.f;
+        const float p1 = ((km >> (e + 1)) & 1u) ? ex2(__uint_as_float(sreg[e + 1]) * scale_log2 - mu) : 0.f;
+        rs[(e >> 1) & 3] += p0 + p1;
+        const uint32_t hi = pack_bf16(p0, p1);
+        const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hi);
+        phi[e >> 1] = hi;
+        plo[e >> 1] = pack_bf16(p0 - __low2float(h2), p1 - __high2float(h2));
       }
+      // keys 32 qt .. 32 qt + 31 -> packed columns 16 qt .. 16 qt + 15 of P hi / P lo
+      tc_st16(tP + lane_off + 16 * qt, phi);
+      tc_st16(tP + lane_off + 64 + 16 * qt, plo);
       tc_fence_before();
-      mbar_arrive(su32(&bars->s_free[b]));
       l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
       mbar_arrive(su32(&bars->p_full));
     }
+    // ---- this split's outputs: O quarter columns, and (quarter 0) max and the row sum
+    float* xl = xm + 2 * 4 * BM;   // [4][BM] partial sums (the maxima buffers may still be read)
+    xl[qt * BM + r] = l;
     if (ok && nchunks > 0) ok = __all_sync(0xffffffffu, wait(bars->o_done, 0));
+    mbar_arrive(su32(&bars->ldone));
+    if (ok) ok = __all_sync(0xffffffffu, wait(bars->ldone, 0));
     if (ok) {
       tc_fence_after();
       const size_t rowbase = ((size_t)bh * gridDim.x + split) * PROWS + prow;
       const int acc = sparse ? 1 : 0;
-      float* dst = part_o + (rowbase * 2 + acc) * D;
+      float* dst = part_o + (rowbase * 2 + acc) * D + qt * (D / 4);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
+      for (int c0 = 0; c0 < D / 4; c0 += 16) {
+        uint32_t o[16];
         if (nchunks > 0) {
-          tc_ld32(tO + lane_off + c * 32, o);
+          const uint32_t ta = tO + lane_off + qt * (D / 4) + c0;
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+              "tcgen05.wait::ld.sync.aligned;\n"
+              : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]), "=r"(o[4]), "=r"(o[5]), "=r"(o[6]), "=r"(o[7]),
+                "=r"(o[8]), "=r"(o[9]), "=r"(o[10]), "=r"(o[11]), "=r"(o[12]), "=r"(o[13]), "=r"(o[14]), "=r"(o[15])
+              : "r"(ta)
+              : "memory");
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
+          for (int e = 0; e < 16; ++e) o[e] = 0u;
         }
-        float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+        float4* d4 = reinterpret_cast<float4*>(dst + c0);
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
+        for (int e = 0; e < 4; ++e)
           d4[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]), __uint_as_float(o[4 * e + 2]),
                               __uint_as_float(o[4 * e + 3]));
       }
-      part_ml[rowbase * 4 + 2 * acc + 0] = m;
-      part_ml[rowbase * 4 + 2 * acc + 1] = l;
+      if (qt == 0) {
+        part_ml[rowbase * 4 + 2 * acc + 0] = m;
+        part_ml[rowbase * 4 + 2 * acc + 1] = (xl[r] + xl[BM + r]) + (xl[2 * BM + r] + xl[3 * BM + r]);
+      }
     }
   }
   tc_fence_before();
