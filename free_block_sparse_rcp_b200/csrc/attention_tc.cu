@@ -23,7 +23,9 @@
 // Per chunk j the MMA issue order is  PV_0,j  S_0,j+1  PV_1,j  S_1,j+1: S_t,j+1 reuses the
 // columns of P_t,j only after PV_t,j (tcgen05 MMAs of one thread execute in issue order),
 // and when S_t,j+1 is complete so is PV_t,j, so the softmax may rescale O_t in place.
-// Rescaling is lazy: only when a row's running max grows by more than 2^8.
+// The softmax makes one speculative pass per chunk against the running max (exponentials
+// and the chunk max together, packed fp32x2 arithmetic) and keeps it unless some row's max
+// grew by more than 2^8; then the chunk is redone against the new max and O is rescaled.
 // K is staged in a 3-deep ring, V in a 2-deep ring.  Every mbarrier wait is bounded (2 s);
 // a timeout raises an abort flag that ends every role, records DERR_WAIT_TIMEOUT in the
 // workspace and still frees the TMEM.
@@ -291,57 +293,98 @@ __global__ void __launch_bounds__(NT, 1)
     bool ok = true;
     if (t < ntile) {
       uint32_t sreg[64];
-      uint32_t pk[32];
+      uint32_t pk[64];
+      const uint64_t sc2 = f2pack(scale_log2, scale_log2);
       for (int j = 0; j < nchunks; ++j) {
         ok = __all_sync(0xffffffffu, wait(bars->s_full[t], j & 1));
         if (!ok) break;
         tc_fence_after();
         const int valid = total - j * BN;
+        const bool full = valid >= BN;
+        // Speculative single pass against the running max: P = exp2(S s log2e - m) and the
+        // chunk's max together; kept only if no row's max grew by more than the threshold.
+        bool need = true;
         float mx = -INFINITY;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          tc_ld64(tS + 64 * h, sreg);
+        uint64_t rs2 = 0ull;
+        const bool spec = __all_sync(0xffffffffu, m_used != -INFINITY);
+        if (spec) {
+          const uint64_t nmu2 = f2pack(-m_used, -m_used);
           float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (64 * h + c < valid) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sreg[c]));
-          mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+          for (int q = 0; q < 4; ++q) {
+            tc_ld32(tS + 32 * q, sreg);
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              float s0 = __uint_as_float(sreg[c]), s1 = __uint_as_float(sreg[c + 1]);
+              if (!full) {
+                if (32 * q + c >= valid) s0 = -INFINITY;
+                if (32 * q + c + 1 >= valid) s1 = -INFINITY;
+              }
+              m4[(c >> 1) & 3] = fmaxf(m4[(c >> 1) & 3], fmaxf(s0, s1));
+              float x0, x1;
+              f2unpack(ffma2(f2pack(s0, s1), sc2, nmu2), x0, x1);
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              rs2 = fadd2(rs2, f2pack(p0, p1));
+              pk[16 * q + (c >> 1)] = pack_bf16(p0, p1);
+            }
+          }
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          need = mx * scale_log2 > m_used + kRescaleThreshold;
         }
-        const float m_new = fmaxf(m_used, mx * scale_log2);
-        const bool need = (m_new > m_used + kRescaleThreshold) || (m_used == -INFINITY && m_new != -INFINITY);
         const bool warp_need = __any_sync(0xffffffffu, need);
         float alpha = 1.f;
-        if (warp_need && m_new > m_used) {
-          alpha = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_new);
-          m_used = m_new;
-        }
-        if (warp_need && j >= 1) {
-          // O row *= alpha in TMEM: PV_t,j-1 completed before S_t,j did
+        if (!warp_need) {
+          // keys 64h .. 64h+63 -> packed P in columns 32h .. 32h+31 (all S of the chunk read)
+          tc_st32(tS, pk);
+          tc_st32(tS + 32, pk + 32);
+          float r0, r1;
+          f2unpack(rs2, r0, r1);
+          l += r0 + r1;
+        } else {
+          // slow path: the chunk's max (if not known yet), rescale O, then P against it
+          if (!spec) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tc_ld32(tO + c * 32, o);
+            for (int h = 0; h < 2; ++h) {
+              tc_ld64(tS + 64 * h, sreg);
+              float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tc_st32(tO + c * 32, o);
+              for (int c = 0; c < 64; ++c)
+                if (64 * h + c < valid) m4[c & 3] = fmaxf(m4[c & 3], __uint_as_float(sreg[c]));
+              mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+            }
           }
-        }
-        const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          // keys 64h .. 64h+63 -> packed P in columns 32h .. 32h+31 (their S was read above)
-          tc_ld64(tS + 64 * h, sreg);
-#pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            const float p0 = 64 * h + c < valid ? ex2(__uint_as_float(sreg[c]) * scale_log2 - mu) : 0.f;
-            const float p1 = 64 * h + c + 1 < valid ? ex2(__uint_as_float(sreg[c + 1]) * scale_log2 - mu) : 0.f;
-            rs[(c >> 1) & 3] += p0 + p1;
-            pk[c >> 1] = pack_bf16(p0, p1);
+          const float m_new = fmaxf(m_used, mx * scale_log2);
+          if (m_new > m_used) {
+            alpha = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_new);
+            m_used = m_new;
           }
-          tc_st32(tS + 32 * h, pk);
+          if (j >= 1) {
+            // O row *= alpha in TMEM: PV_t,j-1 completed before S_t,j did
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              tc_ld32(tO + c * 32, o);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tc_st32(tO + c * 32, o);
+            }
+          }
+          const float mu = (m_used == -INFINITY) ? 0.f : m_used;
+          float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            tc_ld64(tS + 64 * h, sreg);
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+              const float p0 = 64 * h + c < valid ? ex2(__uint_as_float(sreg[c]) * scale_log2 - mu) : 0.f;
+              const float p1 = 64 * h + c + 1 < valid ? ex2(__uint_as_float(sreg[c + 1]) * scale_log2 - mu) : 0.f;
+              rs[(c >> 1) & 3] += p0 + p1;
+              pk[c >> 1] = pack_bf16(p0, p1);
+            }
+            tc_st32(tS + 32 * h, pk);
+          }
+          l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
         }
-        l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
         tc_fence_before();
         mbar_arrive(su32(&bars->p_full[t]));
       }
