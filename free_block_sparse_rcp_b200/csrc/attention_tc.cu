@@ -10,13 +10,16 @@
 // reaches shared memory feeds two tiles and the tensor pipe always has one tile's MMAs to
 // run while the other tile's softmax works.
 //
-// Roles of the 416 threads:
+// Roles of the threads:
 //   warps 0-3   softmax + epilogue of tile 0: thread r owns query row r = TMEM lane r
 //   warps 4-7   softmax + epilogue of tile 1
-//   warps 8-11  gather: cp.async of the q rows and of the routed key/value rows of each
-//               128-row chunk, by index through perm_q / perm_k, into 128B-swizzled
-//               shared-memory tiles (the permuted layout is never materialised)
-//   warp  12    TMEM allocation; lane 0 issues every tcgen05.mma
+//   routed:  warps 8-11 gather by cp.async the q rows and the routed key/value rows of each
+//            128-row chunk, by index through perm_q / perm_k, into 128B-swizzled shared-
+//            memory tiles (the permuted layout is never materialised); warp 12 allocates
+//            TMEM and its lane 0 issues every tcgen05.mma  (416 threads)
+//   dense:   warp 8 loads 128-row boxes by TMA; warp 9 issues the MMAs  (320 threads)
+// (TMA's four-row gather was measured far slower than the cp.async gather for the routed
+// rows, so only the dense variant uses TMA.)
 // TMEM (512 columns): tile t holds S_t at columns 256t .. 256t+127 and O_t at 256t+128 ..
 // The softmax writes P_t = exp2(S_t * s log2e - m) as packed bf16 pairs over the first 64
 // columns of S_t, and PV reads it straight from TMEM (A operand in tensor memory).
@@ -29,6 +32,8 @@
 // K is staged in a 3-deep ring, V in a 2-deep ring.  Every mbarrier wait is bounded (2 s);
 // a timeout raises an abort flag that ends every role, records DERR_WAIT_TIMEOUT in the
 // workspace and still frees the TMEM.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -42,10 +47,16 @@ constexpr int BN = 128;       // key rows per chunk
 constexpr int KST = 3;        // K ring depth
 constexpr int VST = 2;        // V ring depth
 constexpr int NSOFT = 128;    // softmax threads per tile
-constexpr int PROD0 = 256;    // first gather thread (warp 8)
-constexpr int NPROD = 128;
-constexpr int MMA_WARP = 12;
-constexpr int NT = 416;
+// dense: one TMA warp (8) + MMA warp (9); routed: four cp.async gather warps (8-11) + MMA
+// warp (12)
+constexpr int PROD_WARP = 8;
+constexpr int NPROD_G = 128;   // gather threads of the routed variant
+template <bool DENSE>
+struct Roles {
+  static constexpr int MMA_WARP = DENSE ? 9 : 12;
+  static constexpr int NT = DENSE ? 320 : 416;
+  static constexpr uint32_t kLoadArrivals = DENSE ? 1 : NPROD_G;   // arrivals per q / K / V stage
+};
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -65,14 +76,18 @@ struct Layout {
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
 template <int D, bool DENSE>
-__global__ void __launch_bounds__(NT, 1)
-    k_attn_tc(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
-              const __nv_bfloat16* __restrict__ V, int N, int Gq, int Gk, const int* __restrict__ perm_q,
+__global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
+    k_attn_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+              const __grid_constant__ CUtensorMap tmv, const __nv_bfloat16* __restrict__ Q,
+              const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V, int N, int Gq, int Gk,
+              const int* __restrict__ perm_q,
               const int* __restrict__ perm_k, const int* __restrict__ qoff, const int* __restrict__ koff,
               const int* __restrict__ rlist, const int* __restrict__ rcum, const int* __restrict__ rcnt,
               const int2* __restrict__ tiles, const int* __restrict__ tile_count, int max_tiles, float scale_log2,
               __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int* err) {
   using L = Layout<D>;
+  constexpr int NT = Roles<DENSE>::NT;
+  constexpr int MMA_WARP = Roles<DENSE>::MMA_WARP;
   // The 128B-swizzled tiles need a 1024-byte aligned base; dynamic shared memory starts
   // at the CTA's shared window, which is aligned, and the layout leaves no room for a
   // realignment pad, so a misaligned base is reported and the unit skipped.
@@ -132,13 +147,13 @@ __global__ void __launch_bounds__(NT, 1)
   const int ntile = qn > BM ? 2 : 1;
   if (tid == 0) {
     sMisc[1] = 0;
-    mbar_init(su32(&bars->q), NPROD);
+    mbar_init(su32(&bars->q), Roles<DENSE>::kLoadArrivals);
     for (int s = 0; s < KST; ++s) {
-      mbar_init(su32(&bars->kfull[s]), NPROD);
+      mbar_init(su32(&bars->kfull[s]), Roles<DENSE>::kLoadArrivals);
       mbar_init(su32(&bars->kempty[s]), 1);
     }
     for (int s = 0; s < VST; ++s) {
-      mbar_init(su32(&bars->vfull[s]), NPROD);
+      mbar_init(su32(&bars->vfull[s]), Roles<DENSE>::kLoadArrivals);
       mbar_init(su32(&bars->vempty[s]), 1);
     }
     for (int t = 0; t < TPC; ++t) {
@@ -166,15 +181,45 @@ __global__ void __launch_bounds__(NT, 1)
     return bounded_wait(su32(&bar), parity, abort_flag, err);
   };
 
-  if (tid >= PROD0 && tid < PROD0 + NPROD) {
+  if (DENSE && warp == PROD_WARP) {
+    // ---------------- TMA loads (one warp) ----------------
+    bool ok = true;
+    // q rows of both tiles (rows of an absent tile or past the group read row 0: never stored)
+    if (lane == 0) mbar_arrive_expect_tx(su32(&bars->q), TPC * L::kTile);
+    __syncwarp();
+    if (lane < TPC * (D / 64)) {
+      const int t = lane / (D / 64), h = lane % (D / 64);
+      tma_load_2d(sQ + t * L::kTile + h * 16384, &tmq, 64 * h, (int)(head + q0 + BM * t), su32(&bars->q));
+    }
+    for (int j = 0; j < nchunks && ok; ++j) {
+      const int ks = j % KST, vs = j % VST;
+      // K_j, V_j: rows j BN .. j BN + 127 of the head (rows past N are masked in the softmax)
+      if (lane == 0) {
+        ok = j < KST || wait(bars->kempty[ks], ((j / KST) - 1) & 1);
+        if (ok) mbar_arrive_expect_tx(su32(&bars->kfull[ks]), L::kTile);
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      if (lane < D / 64)
+        tma_load_2d(sK + ks * L::kTile + lane * 16384, &tmk, 64 * lane, (int)(head + j * BN), su32(&bars->kfull[ks]));
+      if (lane == 0) {
+        ok = j < VST || wait(bars->vempty[vs], ((j / VST) - 1) & 1);
+        if (ok) mbar_arrive_expect_tx(su32(&bars->vfull[vs]), L::kTile);
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      if (lane < D / 64)
+        tma_load_2d(sV + vs * L::kTile + lane * 16384, &tmv, 64 * lane, (int)(head + j * BN), su32(&bars->vfull[vs]));
+    }
+  } else if (!DENSE && warp >= PROD_WARP && warp < PROD_WARP + 4) {
     // ---------------- gather warps ----------------
-    const int p = tid - PROD0;          // 0..127
+    const int p = tid - PROD_WARP * 32;   // 0..127
     const int pl = p & 31, pw = p >> 5;
     constexpr int CPR = D / 8;          // 16-byte chunks per row
     constexpr int RPI = 32 / CPR;       // rows per warp instruction
     // q rows of both tiles (rows of an absent tile are zero-filled)
-    for (int i = 0; i < TPC * BM * CPR / NPROD; ++i) {
-      const int e = i * NPROD + p;
+    for (int i = 0; i < TPC * BM * CPR / NPROD_G; ++i) {
+      const int e = i * NPROD_G + p;
       const int r = e / CPR, c = e % CPR;
       const int row = sQrow[r];
       cp_async16(sQ + (r / BM) * L::kTile + tile_off(r % BM, c, 128),
@@ -204,7 +249,7 @@ __global__ void __launch_bounds__(NT, 1)
       // K_j -> ring slot j % KST (one thread waits; the named barrier publishes the outcome)
       const int ks = j % KST, vs = j % VST;
       if (p == 0) *prod_ok = (j < KST || wait(bars->kempty[ks], ((j / KST) - 1) & 1)) ? 1 : 0;
-      named_sync(1, NPROD);
+      named_sync(1, NPROD_G);
       if (!*prod_ok) break;
       {
         const uint32_t dk = sK + ks * L::kTile;
@@ -217,9 +262,9 @@ __global__ void __launch_bounds__(NT, 1)
       }
       cp_async_arrive_noinc(su32(&bars->kfull[ks]));
       // V_j -> ring slot j % VST
-      named_sync(1, NPROD);   // every thread has read *prod_ok before it is rewritten
+      named_sync(1, NPROD_G);   // every thread has read *prod_ok before it is rewritten
       if (p == 0) *prod_ok = (j < VST || wait(bars->vempty[vs], ((j / VST) - 1) & 1)) ? 1 : 0;
-      named_sync(1, NPROD);
+      named_sync(1, NPROD_G);
       if (!*prod_ok) break;
       {
         const uint32_t dv = sV + vs * L::kTile;
@@ -231,7 +276,7 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
       cp_async_arrive_noinc(su32(&bars->vfull[vs]));
-      named_sync(1, NPROD);   // *prod_ok is rewritten at the top of the next chunk
+      named_sync(1, NPROD_G);   // *prod_ok is rewritten at the top of the next chunk
     }
     cp_async_wait_all();
   } else if (warp == MMA_WARP) {
@@ -439,11 +484,19 @@ static cudaError_t launch_tc_t(const AttnArgs& a, cudaStream_t st) {
   auto kern = tc::k_attn_tc<D, DENSE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
+  // tensor maps of 128-row boxes (used by the dense variant only)
+  CUtensorMap tq{}, tk{}, tv{};
+  if (DENSE) {
+    const unsigned long long rows = (unsigned long long)a.BH * a.N;
+    if ((e = make_tmap_bf16_rows(&tq, a.Q, rows, D, tc::BM)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16_rows(&tk, a.K, rows, D, tc::BM)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16_rows(&tv, a.V, rows, D, tc::BM)) != cudaSuccess) return e;
+  }
   dim3 grid(DENSE ? ceil_div(a.N, tc::TPC * tc::BM) : a.max_tiles, a.BH);
-  kern<<<grid, tc::NT, sm, st>>>((const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K, (const __nv_bfloat16*)a.V,
-                                 a.N, a.Gq, a.Gk, a.perm_q, a.perm_k, a.qoff, a.koff, a.rlist, a.rcum, a.rcnt,
-                                 a.tiles, a.tile_count, a.max_tiles, a.scale_log2, (__nv_bfloat16*)a.O, a.lse,
-                                 a.err);
+  kern<<<grid, tc::Roles<DENSE>::NT, sm, st>>>(tq, tk, tv, (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K,
+                                               (const __nv_bfloat16*)a.V, a.N, a.Gq, a.Gk, a.perm_q, a.perm_k, a.qoff,
+                                               a.koff, a.rlist, a.rcum, a.rcnt, a.tiles, a.tile_count, a.max_tiles,
+                                               a.scale_log2, (__nv_bfloat16*)a.O, a.lse, a.err);
   return cudaGetLastError();
 }
 

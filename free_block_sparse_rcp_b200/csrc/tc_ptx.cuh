@@ -49,6 +49,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+// TMA gather of four rows (tile::gather4; the tensor map's box is one row high): 64 columns
+// starting at column x of rows y0..y3 land as four consecutive 128-byte rows at dst.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int x, int y0, int y1, int y2, int y3,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4, %5, %6}], [%7];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
+      : "memory");
+}
 __device__ __forceinline__ uint64_t gtimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
@@ -145,21 +155,6 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
-}
-// 2^x on the FMA pipe, for values that are rounded to bf16 afterwards: x = j + f with j the
-// nearest integer (magic-number rounding: adding 1.5 * 2^23 leaves j in the low mantissa
-// bits) and |f| <= 1/2; 2^f by a degree-3 polynomial fitted here for least maximum relative
-// error on [-1/2, 1/2] (7.5e-5, against bf16's 3.9e-3 rounding); 2^j by adding j to the
-// exponent field.  x is clamped to [-125, 125].
-__device__ __forceinline__ float ex2_fma(float x) {
-  x = fminf(fmaxf(x, -125.f), 125.f);
-  const float t = x + 12582912.f;
-  const float j = t - 12582912.f;
-  const float f = x - j;
-  float p = fmaf(f, 0.05517132f, 0.24261054f);
-  p = fmaf(f, p, 0.69326099f);
-  p = fmaf(f, p, 0.99992811f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 // Packed fp32 pair arithmetic (one instruction for two lanes of work on sm_100a).
 __device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
