@@ -173,6 +173,8 @@ sparsepr_status check_params(const sparsepr_params* p) {
       centroid_weights_smem(p->d, p->n_kgroups) > kSmemLimit ||
       assign_acc_smem(p->d, kmeans_gp(p->n_kgroups > p->n_qgroups ? p->n_kgroups : p->n_qgroups)) > kSmemLimit)
     return fail(SPARSEPR_EUNSUPPORTED, "too many groups for the k-means kernels");
+  if (route_select_smem(p->n_qgroups, p->n_kgroups) > kSmemLimit)
+    return fail(SPARSEPR_EUNSUPPORTED, "too many groups for the route selection kernel");
   if (cell_mass_tc_smem(p->d, kmeans_gp(p->n_kgroups)) > kSmemLimit)
     return fail(SPARSEPR_EUNSUPPORTED, "too many K/V groups for the cell-mass kernel");
   if ((size_t)p->d * p->sub_rank > 64 * 65 || probe_fit_smem(p->d, p->sub_rank) > kSmemLimit)

@@ -19,6 +19,7 @@ cudaError_t launch_group_sort(const int* labels, int BH, int N, int G, int* perm
                               cudaStream_t st);
 cudaError_t launch_query_coords(const void* Q, int BH, int N, int D, const float* C, int G, float scale,
                                 float* Z, cudaStream_t st);
+size_t route_select_smem(int Gq, int Gk);
 cudaError_t launch_route_select(const float* mass, int BH, int N, int Gq, int Gk, const int* qoff,
                                 const int* koff, float density, int P, int* order, double* cm,
                                 long long* cc, unsigned char* route, float* rho_exec, double* alpha,

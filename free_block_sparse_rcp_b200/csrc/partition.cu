@@ -260,79 +260,133 @@ __device__ long long block_sum_ll(long long v, long long* red) {
   return t;
 }
 
+// The 60 fp64 bisection steps on alpha are reproduced exactly: the first 50 run as 10
+// rounds of 32-way multisection (the points lo + i (hi - lo) / 32 are dyadic with at most
+// 50 bits, so exact, and the cost is monotone in alpha, so the round lands on the bracket
+// five bisection steps would reach); the last 10 run as plain bisection, with the same
+// rounding of mid = (lo + hi) / 2.  Per-row cumulative masses and K/V sizes live in shared
+// memory (the cumulative mass is summed sequentially in rank order, as the definition
+// reads); one warp evaluates one candidate alpha over all query groups.
+// grid = BH, block = 1024, dynamic smem = route_select_smem(Gq, Gk).
 __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__ mass, int N, int Gq, int Gk,
                                                       const int* __restrict__ qoff, const int* __restrict__ koff,
                                                       float density, int P, int* __restrict__ order,
-                                                      double* __restrict__ cm, long long* __restrict__ cc,
                                                       unsigned char* __restrict__ route,
                                                       float* __restrict__ rho_exec, double* __restrict__ alpha_out) {
   extern __shared__ __align__(16) unsigned char smem[];
-  long long* red = reinterpret_cast<long long*>(smem);     // [32]
-  int* nk = reinterpret_cast<int*>(red + 32);              // [Gk]
-  int* nq = nk + Gk;                                       // [Gq]
-  int* ne = nq + Gq;                                       // [1]: number of non-empty K/V groups
-  const int bh = blockIdx.x, tid = threadIdx.x;
+  double* cmh = reinterpret_cast<double*>(smem);               // [Gq][Gk] cumulative mass in rank order
+  int* pnk = reinterpret_cast<int*>(cmh + (size_t)Gq * Gk);     // [Gq][Gk] cumulative K/V sizes
+  int* nk = pnk + (size_t)Gq * Gk;                              // [Gk]
+  int* nq = nk + Gk;                                            // [Gq]
+  int* misc = nq + Gq;                                          // [0] L, [1..32] round flags
+  long long* red = reinterpret_cast<long long*>(                // [32], 8-byte aligned
+      (reinterpret_cast<uintptr_t>(misc + 40) + 7) & ~(uintptr_t)7);
+  const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* mh = mass + (size_t)bh * Gq * Gk;
   int* oh = order + (size_t)bh * Gq * Gk;
-  double* cmh = cm + (size_t)bh * Gq * Gk;
-  long long* cch = cc + (size_t)bh * Gq * Gk;
   unsigned char* rh = route + (size_t)bh * Gq * Gk;
   for (int g = tid; g < Gk; g += blockDim.x) nk[g] = koff[(size_t)bh * (Gk + 1) + g + 1] - koff[(size_t)bh * (Gk + 1) + g];
   for (int a = tid; a < Gq; a += blockDim.x) nq[a] = qoff[(size_t)bh * (Gq + 1) + a + 1] - qoff[(size_t)bh * (Gq + 1) + a];
   __syncthreads();
-  if (tid == 0) {
+  if (warp == 0) {
     int c = 0;
-    for (int g = 0; g < Gk; ++g) c += nk[g] > 0;
-    ne[0] = c;
+    for (int g = lane; g < Gk; g += 32) c += nk[g] > 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (lane == 0) misc[0] = c;
   }
+  // per row, one warp: ranks (mass descending, ties to the lower group) into the warp's
+  // scratch, then lane 0 takes the cumulative mass (fp64, rank order) and K/V sizes
+  float* wm = reinterpret_cast<float*>(red + 32) + warp * 2 * Gk;   // [Gk] masses in rank order
+  int* wg = reinterpret_cast<int*>(wm + Gk);                        // [Gk] groups in rank order
   __syncthreads();
-  const int L = ne[0];
-  // ranks inside each row
-  for (int e = tid; e < Gq * Gk; e += blockDim.x) {
-    int a = e / Gk, g = e - a * Gk;
-    if (nq[a] == 0 || nk[g] == 0) continue;
-    const float m = mh[e];
-    int r = 0;
-    for (int h = 0; h < Gk; ++h) {
-      if (nk[h] == 0) continue;
-      float mh2 = mh[a * Gk + h];
-      r += (mh2 > m) || (mh2 == m && h < g);
-    }
-    oh[a * Gk + r] = g;
-  }
-  __syncthreads();
-  for (int a = tid; a < Gq; a += blockDim.x) {
+  const int L = misc[0];
+  for (int a = warp; a < Gq; a += blockDim.x / 32) {
     if (nq[a] == 0) continue;
-    double s = 0.0;
-    long long c = 0;
-    for (int r = 0; r < L; ++r) {
-      int g = oh[a * Gk + r];
-      s += (double)mh[a * Gk + g];
-      c += (long long)nq[a] * (long long)nk[g];
-      cmh[a * Gk + r] = s;
-      cch[a * Gk + r] = c;
+    for (int g0 = 0; g0 < Gk; g0 += 32) {
+      const int g = g0 + lane;
+      const bool on = g < Gk && nk[g] > 0;
+      const float m = on ? mh[a * Gk + g] : 0.f;
+      int r = 0;
+      for (int h0 = 0; h0 < Gk; h0 += 32) {
+        const int h = h0 + lane;
+        const bool hv = h < Gk && nk[h] > 0;
+        const float mo = hv ? mh[a * Gk + h] : -INFINITY;
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) {
+          const float m2 = __shfl_sync(0xffffffffu, mo, k);
+          const bool v2 = __shfl_sync(0xffffffffu, hv, k);
+          r += v2 && ((m2 > m) || (m2 == m && h0 + k < g));
+        }
+      }
+      if (on) {
+        oh[a * Gk + r] = g;
+        wm[r] = m;
+        wg[r] = g;
+      }
     }
+    __syncwarp();
+    if (lane == 0) {
+      double sm = 0.0;
+      int c = 0;
+      for (int r = 0; r < L; ++r) {
+        sm += (double)wm[r];
+        c += nk[wg[r]];
+        cmh[(size_t)a * Gk + r] = sm;
+        pnk[(size_t)a * Gk + r] = c;
+      }
+    }
+    __syncwarp();
   }
   __syncthreads();
   const double visible = (double)N * (double)N;
   const double probe_pairs = (double)P * (double)N;
   const double budget = (double)density * visible - probe_pairs;
+  // cost of alpha over the rows a = lane, lane + 32, ... (warp-wide sum)
+  auto warp_cost = [&](double al) -> long long {
+    long long t = 0;
+    for (int a = lane; a < Gq; a += 32)
+      if (nq[a] > 0) t += (long long)nq[a] * (long long)pnk[(size_t)a * Gk + prefix_len(cmh + (size_t)a * Gk, L, al) - 1];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    return t;
+  };
   double alpha;
   const bool all = density >= 1.0f;
   if (all) {
     alpha = 1.0;
   } else {
-    auto cost_at = [&](double al) -> long long {
-      long long t = 0;
-      for (int a = tid; a < Gq; a += blockDim.x)
-        if (nq[a] > 0) t += cch[a * Gk + prefix_len(cmh + a * Gk, L, al) - 1];
-      return block_sum_ll(t, red);
-    };
     double lo = 0.0, hi = 1.0;
-    if ((double)cost_at(lo) <= budget) {
-      for (int it = 0; it < 60; ++it) {
-        double mid = 0.5 * (lo + hi);
-        if ((double)cost_at(mid) <= budget) lo = mid; else hi = mid;
+    if (warp == 0) {
+      const long long c0 = warp_cost(lo);
+      if (lane == 0) misc[1] = (double)c0 <= budget ? 1 : 0;
+    }
+    __syncthreads();
+    if (misc[1]) {
+      for (int round = 0; round < 10; ++round) {
+        const double w = (hi - lo) * (1.0 / 32.0);
+        if (warp >= 1) {
+          const long long c = warp_cost(lo + warp * w);
+          if (lane == 0) misc[1 + warp] = (double)c <= budget ? 1 : 0;
+        }
+        __syncthreads();
+        int k = 0;
+        for (int i = 1; i < 32; ++i) k += misc[1 + i];
+        __syncthreads();
+        // monotone cost: the points that fit are exactly i = 1 .. k
+        const double nlo = lo + k * w;
+        hi = k < 31 ? lo + (k + 1) * w : hi;
+        lo = nlo;
+      }
+      for (int it = 50; it < 60; ++it) {
+        const double mid = 0.5 * (lo + hi);
+        if (warp == 0) {
+          const long long c = warp_cost(mid);
+          if (lane == 0) misc[1] = (double)c <= budget ? 1 : 0;
+        }
+        __syncthreads();
+        if (misc[1]) lo = mid; else hi = mid;
+        __syncthreads();
       }
     }
     alpha = lo;
@@ -342,9 +396,9 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
   long long routed = 0;
   for (int a = tid; a < Gq; a += blockDim.x) {
     if (nq[a] == 0) continue;
-    int len = all ? L : prefix_len(cmh + a * Gk, L, alpha);
+    const int len = all ? L : prefix_len(cmh + (size_t)a * Gk, L, alpha);
     for (int r = 0; r < len; ++r) rh[a * Gk + oh[a * Gk + r]] = 1;
-    routed += cch[a * Gk + len - 1];
+    routed += (long long)nq[a] * (long long)pnk[(size_t)a * Gk + len - 1];
   }
   routed = block_sum_ll(routed, red);
   if (tid == 0) {
@@ -455,13 +509,20 @@ cudaError_t launch_query_coords(const void* Q, int BH, int N, int D, const float
   return cudaGetLastError();
 }
 
+size_t route_select_smem(int Gq, int Gk) {
+  return (size_t)Gq * Gk * 8 + (size_t)Gq * Gk * 4 + (size_t)(Gk + Gq + 40) * 4 + 8 + 32 * 8 +
+         (size_t)32 * 2 * Gk * 4;
+}
+
 cudaError_t launch_route_select(const float* mass, int BH, int N, int Gq, int Gk, const int* qoff,
                                 const int* koff, float density, int P, int* order, double* cm,
                                 long long* cc, unsigned char* route, float* rho_exec, double* alpha,
                                 cudaStream_t st) {
-  size_t sm = 32 * 8 + (size_t)(Gk + Gq + 4) * 4;
-  k_route_select<<<BH, 1024, sm, st>>>(mass, N, Gq, Gk, qoff, koff, density, P, order, cm, cc, route,
-                                       rho_exec, alpha);
+  (void)cm;
+  (void)cc;
+  const size_t sm = route_select_smem(Gq, Gk);
+  cudaFuncSetAttribute(k_route_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  k_route_select<<<BH, 1024, sm, st>>>(mass, N, Gq, Gk, qoff, koff, density, P, order, route, rho_exec, alpha);
   return cudaGetLastError();
 }
 

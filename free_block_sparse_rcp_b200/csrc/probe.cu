@@ -2,6 +2,8 @@
 // technical summary, section 2.B; huashangw.com article, method walkthrough:
 // 64 probe rows per head drawn evenly from every query group, ridge regression,
 // correction inside the leading singular directions of the probe residuals).
+#include <cuda.h>
+
 #include "common.cuh"
 #include "symeig.cuh"
 #include "kernels.h"
@@ -79,36 +81,40 @@ __global__ void __launch_bounds__(256) k_probe_pick(const int* __restrict__ perm
 constexpr int PR = 64;  // probe rows per split in the partial buffers
 
 // ---------------------------------------------------------------------------
-// Merge the key splits.  grid = BH, block = 256.
+// Merge the key splits: for each probe row and accumulator (dense / routed), the split
+// maxima M_s, sums L_s and unnormalised outputs O_s combine as
+//   M = max_s M_s, L = sum_s L_s 2^(M_s - M), O = sum_s O_s 2^(M_s - M) / L   (s ascending).
+// grid = (P, BH), block = D (one output column per thread).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_probe_combine(const float* __restrict__ part_o,
+__global__ void __launch_bounds__(128) k_probe_combine(const float* __restrict__ part_o,
                                                       const float* __restrict__ part_ml, int S, int P, int D,
                                                       float* __restrict__ o_dense, float* __restrict__ o_sparse,
                                                       float* __restrict__ lse_d, float* __restrict__ lse_s) {
-  const int bh = blockIdx.x;
+  __shared__ float sml[64 * 4];   // [S][M_dense, L_dense, M_sparse, L_sparse]
+  const int r = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
   const float LN2 = 0.69314718055994531f;
-  for (int e = threadIdx.x; e < P * D; e += blockDim.x) {
-    const int r = e / D, c = e - r * D;
-    for (int acc = 0; acc < 2; ++acc) {
-      float M = -INFINITY;
-      for (int s = 0; s < S; ++s) M = fmaxf(M, part_ml[(((size_t)bh * S + s) * PR + r) * 4 + 2 * acc]);
-      float L = 0.f, Ov = 0.f;
-      if (M != -INFINITY) {
-        for (int s = 0; s < S; ++s) {
-          const size_t rr = ((size_t)bh * S + s) * PR + r;
-          const float ms = part_ml[rr * 4 + 2 * acc];
-          if (ms == -INFINITY) continue;
-          const float w = ex2f(ms - M);
-          L += part_ml[rr * 4 + 2 * acc + 1] * w;
-          Ov += part_o[(rr * 2 + acc) * D + c] * w;
-        }
+  for (int e = threadIdx.x; e < S * 4; e += blockDim.x) {
+    const int sidx = e >> 2, k = e & 3;
+    sml[e] = part_ml[(((size_t)bh * S + sidx) * PR + r) * 4 + k];
+  }
+  __syncthreads();
+  for (int acc = 0; acc < 2; ++acc) {
+    float M = -INFINITY;
+    for (int sidx = 0; sidx < S; ++sidx) M = fmaxf(M, sml[sidx * 4 + 2 * acc]);
+    float L = 0.f, Ov = 0.f;
+    if (M != -INFINITY) {
+      for (int sidx = 0; sidx < S; ++sidx) {
+        const float ms = sml[sidx * 4 + 2 * acc];
+        if (ms == -INFINITY) continue;
+        const float w = ex2f(ms - M);
+        L += sml[sidx * 4 + 2 * acc + 1] * w;
+        if (c < D) Ov += part_o[((((size_t)bh * S + sidx) * PR + r) * 2 + acc) * D + c] * w;
       }
-      const float val = L > 0.f ? Ov / L : 0.f;
-      (acc == 0 ? o_dense : o_sparse)[((size_t)bh * P + r) * D + c] = val;
-      if (c == 0) {
-        float* dst = acc == 0 ? lse_d : lse_s;
-        if (dst) dst[(size_t)bh * P + r] = L > 0.f ? (M + log2f(L)) * LN2 : -INFINITY;
-      }
+    }
+    if (c < D) (acc == 0 ? o_dense : o_sparse)[((size_t)bh * P + r) * D + c] = L > 0.f ? Ov / L : 0.f;
+    if (c == 0) {
+      float* dst = acc == 0 ? lse_d : lse_s;
+      if (dst) dst[(size_t)bh * P + r] = L > 0.f ? (M + log2f(L)) * LN2 : -INFINITY;
     }
   }
 }
@@ -299,144 +305,202 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
 
 // ---------------------------------------------------------------------------
 // Correction on the tensor cores: O = x + b_full + x B with B = W V_r^T (d x d).
-// Each CTA forms B^T[n][k] = sum_j V_r[n][j] W[k][j] once (fp32), splits it into bf16
-// hi + lo (K-major tile), then for every 128-row tile of O_sparse computes x B with two
-// tcgen05 MMAs (exact bf16 products, fp32 accumulation) and writes x + b + x B in bf16.
-// Rows are read into shared memory before any is written, so O may alias O_sparse.
-// grid = (RC_CTAS, BH), block = 128.
+// Persistent: CTA c takes the global 128-row tiles [c per, (c+1) per) (tile i = row tile
+// i mod T of head i / T).  When the CTA enters a head it forms B^T[n][k] = sum_j V_r[n][j]
+// W[k][j] (fp32) and splits it into bf16 hi + lo (K-major tile).  Then a pipeline:
+//   warp 17     (lane 0) loads the O_sparse tile (two TMA boxes of 128 rows x 64 columns)
+//               into a three-deep ring
+//   warp 16     (lane 0) issues x B_hi + x B_lo (exact bf16 products, fp32 accumulation)
+//               into a double-buffered TMEM tile
+//   warps 0-15  row r = TMEM lane r, column quarter q: x + b + xB -> bf16 -> O
+// Every row of a tile is loaded before the tile's outputs are written, so O may alias
+// O_sparse.
 // ---------------------------------------------------------------------------
-constexpr int RC_CTAS = 16;
+namespace rct {
+constexpr int NT = 576;
+constexpr int NEPI = 512;
+constexpr int MMA_WARP = 16;
+constexpr int LOAD_WARP = 17;
+constexpr int XS = 3;
+constexpr int kCtas = 148;
+struct Bars {
+  uint64_t xfull[XS], xempty[XS], tfull[2], tempty[2];
+};
+}  // namespace rct
 
 template <int D>
-__global__ void __launch_bounds__(128) k_reconstruct_tc(const __nv_bfloat16* __restrict__ Os, int N, int Rk,
-                                                       const float* __restrict__ W, const float* __restrict__ Vr,
-                                                       const float* __restrict__ bfull,
-                                                       __nv_bfloat16* __restrict__ O, int* err) {
+__global__ void __launch_bounds__(rct::NT, 1)
+    k_reconstruct_tc(const __grid_constant__ CUtensorMap tmx, int N, int T, int total, int per, int Rk,
+                     const float* __restrict__ W, const float* __restrict__ Vr, const float* __restrict__ bfull,
+                     __nv_bfloat16* __restrict__ O, int* err) {
   using namespace spr::tc;
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  const uint32_t raw = su32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  unsigned char* smem = smem_raw + (base - raw);
+  extern __shared__ __align__(1024) unsigned char smem_rc[];
+  const uint32_t base = su32(smem_rc);
+  if (base & 1023u) {
+    if (threadIdx.x == 0) set_error(err, DERR_INDEX);
+    return;
+  }
+  const int t0 = blockIdx.x * per, t1 = min(total, t0 + per);
+  if (t0 >= t1) return;
+  constexpr int XS = rct::XS;
   constexpr uint32_t kT = (uint32_t)128 * D * 2;   // X tile (128 rows)
   constexpr uint32_t kB = (uint32_t)D * D * 2;     // B^T tile (D rows)
-  const uint32_t sX = base, sBh = base + kT, sBl = sBh + kB;
-  float* sb = reinterpret_cast<float*>(smem + kT + 2 * kB);   // [D]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sb + D);
-  int* sMisc = reinterpret_cast<int*>(bar + 1);
+  const uint32_t sX = base, sBh = base + XS * kT, sBl = sBh + kB;
+  float* sb = reinterpret_cast<float*>(smem_rc + XS * kT + 2 * kB);   // [D]
+  rct::Bars* bars = reinterpret_cast<rct::Bars*>(sb + D);
+  int* sMisc = reinterpret_cast<int*>(bars + 1);   // [0] tmem, [1] abort
   volatile int* abort_flag = sMisc + 1;
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int bh = blockIdx.y;
-  const size_t head = (size_t)bh * N;
-  constexpr int CPR = D / 8;
-  const float* Wh = W + (size_t)bh * D * Rk;
-  const float* Vh = Vr + (size_t)bh * D * Rk;
-  // stage V_r [n][j] and W^T [j][k] in the (still unused) X-tile region when they fit
-  const bool staged = (size_t)2 * D * Rk * 4 <= kT;
-  float* sV = reinterpret_cast<float*>(smem);
-  float* sWt = sV + D * Rk;
-  if (staged) {
-    for (int e = tid; e < D * Rk; e += 128) {
-      sV[e] = Vh[e];
-      const int k = e / Rk, j = e - k * Rk;
-      sWt[j * D + k] = Wh[e];
-    }
-    __syncthreads();
-  }
-  // B^T rows n, columns k, stored as a K-major 128B-swizzled tile of D rows
-  for (int e = tid; e < D * D; e += 128) {
-    const int n = e / D, k = e - n * D;
-    float acc = 0.f;
-    if (staged)
-      for (int j = 0; j < Rk; ++j) acc = fmaf(sV[n * Rk + j], sWt[j * D + k], acc);
-    else
-      for (int j = 0; j < Rk; ++j) acc = fmaf(Vh[n * Rk + j], Wh[k * Rk + j], acc);
-    const __nv_bfloat16 hi = __float2bfloat16(acc);
-    const __nv_bfloat16 lo = __float2bfloat16(acc - __bfloat162float(hi));
-    const uint32_t off = tile_off(n, k >> 3, D) + (k & 7) * 2;
-    *reinterpret_cast<__nv_bfloat16*>(smem + kT + off) = hi;
-    *reinterpret_cast<__nv_bfloat16*>(smem + kT + kB + off) = lo;
-  }
-  for (int c = tid; c < D; c += 128) sb[c] = bfull[(size_t)bh * D + c];
-  __syncthreads();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
     sMisc[1] = 0;
-    mbar_init(su32(bar), 1);
+    for (int b = 0; b < XS; ++b) {
+      mbar_init(su32(&bars->xfull[b]), 1);
+      mbar_init(su32(&bars->xempty[b]), rct::NEPI);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(su32(&bars->tfull[b]), 1);
+      mbar_init(su32(&bars->tempty[b]), rct::NEPI);
+    }
     fence_barrier_init();
   }
-  if (warp == 0) {
-    tc_alloc(su32(&sMisc[0]), 128);
+  if (warp == rct::MMA_WARP) {
+    tc_alloc(su32(&sMisc[0]), 256);
     tc_relinquish();
   }
-  fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = (uint32_t)sMisc[0];
   constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(D >> 3) << 17) | (8u << 24);
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  const int ntiles = (N + 127) / 128;
-  int phase = 0;
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int n0 = tile * 128;
-    for (int e = tid; e < 128 * CPR; e += 128) {
-      const int r = e / CPR, c = e - r * CPR;
-      const bool ok = n0 + r < N;
-      cp_async16(sX + tile_off(r, c, 128), Os + (head + (ok ? n0 + r : 0)) * D + c * 8, ok);
+  auto wait = [&](uint64_t& bar, uint32_t parity) -> bool {
+    return bounded_wait(su32(&bar), parity, abort_flag, err);
+  };
+  int it = 0;
+  bool ok = true;
+  for (int s0 = t0; s0 < t1 && ok;) {
+    const int bh = s0 / T;
+    const int s1 = min(t1, (bh + 1) * T);
+    const size_t head = (size_t)bh * N;
+    // ---- B^T of this head (every role is idle here)
+    __syncthreads();
+    {
+      // V_r [n][j] and W^T [j][k] staged in the (idle) X ring: D * Rk <= 64 * 65 floats each
+      const float* Wh = W + (size_t)bh * D * Rk;
+      const float* Vh = Vr + (size_t)bh * D * Rk;
+      float* sV = reinterpret_cast<float*>(smem_rc);
+      float* sWt = sV + D * Rk;
+      for (int e = tid; e < D * Rk; e += rct::NT) {
+        sV[e] = Vh[e];
+        const int k = e / Rk, j = e - k * Rk;
+        sWt[j * D + k] = Wh[e];
+      }
+      __syncthreads();
+      for (int e = tid; e < D * D; e += rct::NT) {
+        const int n = e / D, k = e - n * D;
+        float acc = 0.f;
+        for (int j = 0; j < Rk; ++j) acc = fmaf(sV[n * Rk + j], sWt[j * D + k], acc);
+        const __nv_bfloat16 hi = __float2bfloat16(acc);
+        const __nv_bfloat16 lo = __float2bfloat16(acc - __bfloat162float(hi));
+        const uint32_t off = tile_off(n, k >> 3, D) + (k & 7) * 2;
+        *reinterpret_cast<__nv_bfloat16*>(smem_rc + XS * kT + off) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(smem_rc + XS * kT + kB + off) = lo;
+      }
+      for (int c = tid; c < D; c += rct::NT) sb[c] = bfull[(size_t)bh * D + c];
     }
-    cp_async_wait_all();
     fence_proxy_async();
     __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
+    if (warp == rct::LOAD_WARP) {
+      if (lane == 0) {
+        for (int i = s0; i < s1 && ok; ++i, ++it) {
+          const int xb = it % XS, n0 = (i - bh * T) * 128;
+          if (it >= XS) ok = wait(bars->xempty[xb], ((it / XS) - 1) & 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(su32(&bars->xfull[xb]), kT);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
-        const uint32_t ob = (k >> 2) * (D * 128) + (k & 3) * 32;
-        tc_mma(tmem, sdesc(sX + ox, 16, 1024), sdesc(sBh + ob, 16, 1024), idesc, k > 0 ? 1u : 0u);
-      }
-#pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
-        const uint32_t ob = (k >> 2) * (D * 128) + (k & 3) * 32;
-        tc_mma(tmem, sdesc(sX + ox, 16, 1024), sdesc(sBl + ob, 16, 1024), idesc, 1u);
-      }
-      tc_commit(su32(bar));
-    }
-    const bool ok = __syncthreads_and(bounded_wait(su32(bar), phase & 1, abort_flag, err) ? 1 : 0) != 0;
-    ++phase;
-    if (!ok) break;
-    tc_fence_after();
-    const int row = n0 + tid;
-#pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t acc[32];
-      tc_ld32(tmem + lane_off + c0, acc);
-      uint32_t w[16];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(smem + tile_off(tid, (c0 >> 3) + q, 128));
-        const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 x = __bfloat1622float2(x2[e]);
-          const int c = c0 + q * 8 + 2 * e;
-          w[q * 4 + e] = pack_bf16(x.x + sb[c] + __uint_as_float(acc[q * 8 + 2 * e]),
-                                   x.y + sb[c + 1] + __uint_as_float(acc[q * 8 + 2 * e + 1]));
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_2d(sX + xb * kT + h * 16384, &tmx, 64 * h, (int)(head + n0), su32(&bars->xfull[xb]));
         }
       }
-      if (row < N) {
-        uint4* dst = reinterpret_cast<uint4*>(O + (head + row) * D + c0);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      it = __shfl_sync(0xffffffffu, it, 0);
+    } else if (warp == rct::MMA_WARP) {
+      if (lane == 0) {
+        for (int i = s0; i < s1 && ok; ++i, ++it) {
+          const int b = it & 1, xb = it % XS;
+          ok = wait(bars->xfull[xb], (it / XS) & 1) && (it < 2 || wait(bars->tempty[b], ((it >> 1) - 1) & 1));
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
+            const uint32_t ob = (k >> 2) * (D * 128) + (k & 3) * 32;
+            tc_mma(tmem + 128 * b, sdesc(sX + xb * kT + ox, 16, 1024), sdesc(sBh + ob, 16, 1024), idesc,
+                   k > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
+            const uint32_t ob = (k >> 2) * (D * 128) + (k & 3) * 32;
+            tc_mma(tmem + 128 * b, sdesc(sX + xb * kT + ox, 16, 1024), sdesc(sBl + ob, 16, 1024), idesc, 1u);
+          }
+          tc_commit(su32(&bars->tfull[b]));
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      it = __shfl_sync(0xffffffffu, it, 0);
+    } else {
+      const int qt = warp >> 2, r = (warp & 3) * 32 + lane;
+      const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+      constexpr int CQ = D / 4;   // columns of this quarter
+      for (int i = s0; i < s1 && ok; ++i, ++it) {
+        const int b = it & 1, xb = it % XS, row = (i - bh * T) * 128 + r;
+        // xB ready; the X tile (read below) completed before it
+        ok = __all_sync(0xffffffffu, wait(bars->tfull[b], (it >> 1) & 1) && wait(bars->xfull[xb], (it / XS) & 1));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c0 = 0; c0 < CQ; c0 += 16) {
+          const int cb = qt * CQ + c0;
+          uint32_t acc[16];
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+              "tcgen05.wait::ld.sync.aligned;\n"
+              : "=r"(acc[0]), "=r"(acc[1]), "=r"(acc[2]), "=r"(acc[3]), "=r"(acc[4]), "=r"(acc[5]), "=r"(acc[6]),
+                "=r"(acc[7]), "=r"(acc[8]), "=r"(acc[9]), "=r"(acc[10]), "=r"(acc[11]), "=r"(acc[12]),
+                "=r"(acc[13]), "=r"(acc[14]), "=r"(acc[15])
+              : "r"(tmem + 128 * b + lane_off + cb)
+              : "memory");
+          uint32_t w[8];
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const uint4 xv = *reinterpret_cast<const uint4*>(smem_rc + xb * kT + tile_off(r, (cb >> 3) + q, 128));
+            const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 x = __bfloat1622float2(x2[e]);
+              const int c = cb + q * 8 + 2 * e;
+              w[q * 4 + e] = pack_bf16(x.x + sb[c] + __uint_as_float(acc[q * 8 + 2 * e]),
+                                       x.y + sb[c + 1] + __uint_as_float(acc[q * 8 + 2 * e + 1]));
+            }
+          }
+          if (row < N) {
+            uint4* dst = reinterpret_cast<uint4*>(O + (head + row) * D + cb);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(su32(&bars->tempty[b]));
+        mbar_arrive(su32(&bars->xempty[xb]));
       }
     }
-    tc_fence_before();
-    __syncthreads();
+    ok = __syncthreads_and(ok ? 1 : 0) != 0;
+    s0 = s1;
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tc_dealloc(tmem, 128);
+  if (warp == rct::MMA_WARP) tc_dealloc(tmem, 256);
 }
 
 __global__ void k_probe_scatter(const int* __restrict__ probe_idx, const float* __restrict__ o_dense, int N, int P,
@@ -548,13 +612,15 @@ cudaError_t launch_probe_attn_splits(const void* Q, const void* K, const void* V
 cudaError_t launch_probe_combine_splits(const float* part_o, const float* part_ml, int BH, int S, int P, int D,
                                         float* o_dense, float* o_sparse, float* lse_d, float* lse_s,
                                         cudaStream_t st) {
-  k_probe_combine<<<BH, 256, 0, st>>>(part_o, part_ml, S, P, D, o_dense, o_sparse, lse_d, lse_s);
+  if (S > 64) return cudaErrorInvalidValue;
+  k_probe_combine<<<dim3(P, BH), 128, 0, st>>>(part_o, part_ml, S, P, D, o_dense, o_sparse, lse_d, lse_s);
   return cudaGetLastError();
 }
 
 cudaError_t launch_probe_combine(const float* part_o, const float* part_ml, int BH, int N, int P, int D,
                                  float* o_dense, float* o_sparse, float* lse_d, float* lse_s, cudaStream_t st) {
-  k_probe_combine<<<BH, 256, 0, st>>>(part_o, part_ml, probe_splits(N), P, D, o_dense, o_sparse, lse_d, lse_s);
+  k_probe_combine<<<dim3(P, BH), 128, 0, st>>>(part_o, part_ml, probe_splits(N), P, D, o_dense, o_sparse, lse_d,
+                                               lse_s);
   return cudaGetLastError();
 }
 
@@ -576,16 +642,21 @@ cudaError_t launch_probe_fit(const float* o_dense, const float* o_sparse, int BH
 
 cudaError_t launch_reconstruct(const void* Os, int BH, int N, int D, int Rk, const float* W, const float* Vr,
                                const float* bfull, void* O, cudaStream_t st) {
-  const size_t sm = 1024 + (size_t)128 * D * 2 + 2 * (size_t)D * D * 2 + (size_t)D * 4 + 8 + 16;
-  dim3 grid(RC_CTAS, BH);
+  const size_t sm = (size_t)rct::XS * 128 * D * 2 + 2 * (size_t)D * D * 2 + (size_t)D * 4 + sizeof(rct::Bars) + 16;
+  const int T = ceil_div(N, 128), total = BH * T;
+  const int grid = total < rct::kCtas ? total : rct::kCtas;
+  const int per = ceil_div(total, grid);
+  CUtensorMap tmx;
+  cudaError_t e = make_tmap_bf16_rows(&tmx, Os, (unsigned long long)BH * N, D, 128);
+  if (e != cudaSuccess) return e;
   if (D == 64) {
     cudaFuncSetAttribute(k_reconstruct_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_reconstruct_tc<64><<<grid, 128, sm, st>>>((const __nv_bfloat16*)Os, N, Rk, W, Vr, bfull, (__nv_bfloat16*)O,
-                                                nullptr);
+    k_reconstruct_tc<64><<<grid, rct::NT, sm, st>>>(tmx, N, T, total, per, Rk, W, Vr, bfull, (__nv_bfloat16*)O,
+                                                    nullptr);
   } else {
     cudaFuncSetAttribute(k_reconstruct_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_reconstruct_tc<128><<<grid, 128, sm, st>>>((const __nv_bfloat16*)Os, N, Rk, W, Vr, bfull, (__nv_bfloat16*)O,
-                                                 nullptr);
+    k_reconstruct_tc<128><<<grid, rct::NT, sm, st>>>(tmx, N, T, total, per, Rk, W, Vr, bfull, (__nv_bfloat16*)O,
+                                                     nullptr);
   }
   return cudaGetLastError();
 }
