@@ -295,34 +295,65 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
     for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
     if (lane == 0) misc[0] = c;
   }
-  // per row, one warp: ranks (mass descending, ties to the lower group) into the warp's
-  // scratch, then lane 0 takes the cumulative mass (fp64, rank order) and K/V sizes
+  // per row, one warp: bitonic sort of the row's groups (mass descending, ties to the lower
+  // group; empty groups last) into the warp's scratch, then lane 0 takes the cumulative mass
+  // (fp64, rank order, sequential) and cumulative K/V sizes
   float* wm = reinterpret_cast<float*>(red + 32) + warp * 2 * Gk;   // [Gk] masses in rank order
-  int* wg = reinterpret_cast<int*>(wm + Gk);                        // [Gk] groups in rank order
+  int* wn = reinterpret_cast<int*>(wm + Gk);                        // [Gk] their K/V sizes
   __syncthreads();
   const int L = misc[0];
+  int GS = 32;
+  while (GS < Gk) GS <<= 1;                   // sort width (power of two, <= 128 * 4 / 4)
+  const int per_lane = GS / 32;               // 1, 2 or 4 elements per lane
   for (int a = warp; a < Gq; a += blockDim.x / 32) {
     if (nq[a] == 0) continue;
-    for (int g0 = 0; g0 < Gk; g0 += 32) {
-      const int g = g0 + lane;
-      const bool on = g < Gk && nk[g] > 0;
-      const float m = on ? mh[a * Gk + g] : 0.f;
-      int r = 0;
-      for (int h0 = 0; h0 < Gk; h0 += 32) {
-        const int h = h0 + lane;
-        const bool hv = h < Gk && nk[h] > 0;
-        const float mo = hv ? mh[a * Gk + h] : -INFINITY;
-#pragma unroll 8
-        for (int k = 0; k < 32; ++k) {
-          const float m2 = __shfl_sync(0xffffffffu, mo, k);
-          const bool v2 = __shfl_sync(0xffffffffu, hv, k);
-          r += v2 && ((m2 > m) || (m2 == m && h0 + k < g));
+    float km[4];
+    int ki[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int g = lane * per_lane + q;
+      const bool on = q < per_lane && g < Gk && nk[g] > 0;
+      km[q] = on ? mh[a * Gk + g] : -INFINITY;
+      ki[q] = q < per_lane ? g : 0x7fffffff;
+    }
+    // element e = per_lane * lane + q; "x before y" <=> x.m > y.m || (x.m == y.m && x.i < y.i)
+    for (int k = 2; k <= GS; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        if (j >= per_lane) {
+          const int lx = j / per_lane;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (q >= per_lane) continue;
+            const float om = __shfl_xor_sync(0xffffffffu, km[q], lx);
+            const int oi = __shfl_xor_sync(0xffffffffu, ki[q], lx);
+            const int e = lane * per_lane + q;
+            const bool first = ((e & k) == 0) == ((e & j) == 0);   // keep the earlier of the pair
+            const bool mine_before = km[q] > om || (km[q] == om && ki[q] < oi);
+            if (first != mine_before) { km[q] = om; ki[q] = oi; }
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int q2 = q ^ j;
+            if (q >= per_lane || q2 < q) continue;
+            const int e = lane * per_lane + q;
+            const bool asc = (e & k) == 0;
+            const bool q_before = km[q] > km[q2] || (km[q] == km[q2] && ki[q] < ki[q2]);
+            if (asc != q_before) {
+              const float tm = km[q]; km[q] = km[q2]; km[q2] = tm;
+              const int ti = ki[q]; ki[q] = ki[q2]; ki[q2] = ti;
+            }
+          }
         }
       }
-      if (on) {
-        oh[a * Gk + r] = g;
-        wm[r] = m;
-        wg[r] = g;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int r = lane * per_lane + q;
+      if (q < per_lane && r < L) {
+        oh[a * Gk + r] = ki[q];
+        wm[r] = km[q];
+        wn[r] = nk[ki[q]];
       }
     }
     __syncwarp();
@@ -331,7 +362,7 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
       int c = 0;
       for (int r = 0; r < L; ++r) {
         sm += (double)wm[r];
-        c += nk[wg[r]];
+        c += wn[r];
         cmh[(size_t)a * Gk + r] = sm;
         pnk[(size_t)a * Gk + r] = c;
       }

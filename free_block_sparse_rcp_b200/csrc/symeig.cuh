@@ -6,9 +6,10 @@
 //      diagonal onto its first entry; the trailing block is updated as A -= v w^T + w v^T
 //      with p = beta A v, w = p - (beta/2)(v^T p) v.  The reflector v_k is kept in column k
 //      below the diagonal.
-//   2. Eigenvalues of T by multisection on the Sturm count (the number of negative pivots of
-//      the LDL^T factorisation of T - x I): each warp brackets one eigenvalue and its 32
-//      lanes test 32 interior points per step, so the bracket shrinks 33-fold a step.
+//   2. Eigenvalues of T bracketed by multisection on the Sturm count (the number of negative
+//      pivots of the LDL^T factorisation of T - x I), evaluated in fp32: each warp brackets one
+//      eigenvalue and its 32 lanes test 32 interior points per step, so the bracket shrinks
+//      33-fold a step, down to fp32 resolution (the shift of step 3).
 //   3. Eigenvectors of T by inverse iteration: two solves with (T - mu I), tridiagonal LU with
 //      partial pivoting, tiny pivots replaced by eps ||T||.  Eigenvalues closer than 1e-3 ||T||
 //      form a cluster: their shifts are separated and their vectors re-orthogonalised by
@@ -30,15 +31,17 @@ __device__ __forceinline__ double warp_sum_f64(double v) {
   return v;
 }
 
-// number of eigenvalues of the tridiagonal (d, e2 = e^2) not above x
-__device__ __forceinline__ int sturm_count(const double* d, const double* e2, int n, double x, double pivmin) {
-  double q = d[0] - x;
-  if (fabs(q) < pivmin) q = -pivmin;
-  int c = q <= 0.0;
+// number of eigenvalues of the tridiagonal (d, e2 = e^2, fp32 copies) not above x, in fp32:
+// it only brackets the eigenvalue for the inverse iteration, whose Rayleigh quotient gives
+// the fp64 value, so an fp32 bracket (and fast division) is enough
+__device__ __forceinline__ int sturm_count_f32(const float* d, const float* e2, int n, float x, float pivmin) {
+  float q = d[0] - x;
+  if (fabsf(q) < pivmin) q = -pivmin;
+  int c = q <= 0.f;
   for (int i = 1; i < n; ++i) {
-    q = (d[i] - x) - e2[i - 1] / q;
-    if (fabs(q) < pivmin) q = -pivmin;
-    c += q <= 0.0;
+    q = (d[i] - x) - __fdividef(e2[i - 1], q);
+    if (fabsf(q) < pivmin) q = -pivmin;
+    c += q <= 0.f;
   }
   return c;
 }
@@ -87,7 +90,7 @@ __device__ __forceinline__ double start_entry(int i, int j) {
 // Shared scratch (doubles) needed besides A and Z.
 template <int N>
 struct SymEigScratch {
-  static constexpr int kDoubles = 6 * N + 3 * 64 + 8;
+  static constexpr int kDoubles = 7 * N + 3 * 64 + 8;
 };
 
 // A: N x N symmetric, row stride N + 1, overwritten (reflectors below the diagonal).
@@ -105,7 +108,9 @@ __device__ inline void sym_top_eigen(double* A, int R, double* Z, int ldz, doubl
   double* beta = e2 + N;     // [N]
   double* v = beta + N;      // [N]
   double* p = v + N;         // [N]
-  double* shift = p + N;     // [64]
+  float* d32 = reinterpret_cast<float*>(p + N);   // [N]
+  float* e232 = d32 + N;                          // [N]
+  double* shift = p + 2 * N; // [64]
   int* cstart = reinterpret_cast<int*>(shift + 64);  // [64]
   double* misc = shift + 64 + 64;                    // [64 + 8]: gl, gu, tnorm, pivmin
 
@@ -197,26 +202,30 @@ __device__ inline void sym_top_eigen(double* A, int R, double* Z, int ldz, doubl
       hi = fmax(hi, __shfl_xor_sync(0xffffffffu, hi, o));
       me2 = fmax(me2, __shfl_xor_sync(0xffffffffu, me2, o));
     }
+    for (int i = lane; i < N; i += 32) {
+      d32[i] = (float)d[i];
+      e232[i] = i + 1 < N ? (float)e2[i] : 0.f;
+    }
     if (lane == 0) {
       const double tn = fmax(fabs(lo), fabs(hi));
-      const double pivmin = DBL_MIN * fmax(1.0, me2);
-      const double pad = 2.0 * DBL_EPSILON * tn * N + 4.0 * pivmin;
+      const double pad = 4e-6 * tn + 1e-30;   // covers the fp32 rounding of the counts
       misc[0] = lo - pad;
       misc[1] = hi + pad;
       misc[2] = tn;
-      misc[3] = pivmin;
+      misc[3] = fmax((double)FLT_MIN * fmax(1.0, me2), 1e-30 * tn);
     }
   }
   __syncthreads();
-  const double tnorm = misc[2], pivmin = misc[3];
+  const double tnorm = misc[2];
+  const float pivmin32 = (float)misc[3];
   // ---- 2. eigenvalues (j-th largest = ascending index N-1-j)
   for (int j = warp; j < R; j += nw) {
     const int t = N - 1 - j;
     double a = misc[0], b = misc[1];
-    for (int it = 0; it < 14; ++it) {
-      if (b - a <= 2.0 * DBL_EPSILON * fmax(fabs(a), fabs(b)) + 1e-14 * tnorm + 4.0 * pivmin) break;
+    for (int it = 0; it < 8; ++it) {
+      if (b - a <= 2e-7 * fmax(fabs(a), fabs(b)) + 1e-7 * tnorm + 1e-30) break;
       const double x = a + (b - a) * (double)(lane + 1) * (1.0 / 33.0);
-      const unsigned below = __ballot_sync(0xffffffffu, sturm_count(d, e2, N, x, pivmin) <= t);
+      const unsigned below = __ballot_sync(0xffffffffu, sturm_count_f32(d32, e232, N, (float)x, pivmin32) <= t);
       const int lo = below ? 31 - __clz(below) : -1;
       const double xlo = __shfl_sync(0xffffffffu, x, lo < 0 ? 0 : lo);
       const double xhi = __shfl_sync(0xffffffffu, x, lo < 31 ? lo + 1 : 31);
