@@ -139,6 +139,34 @@ def attention(q, k, v, scale, mask=None, chunk=1024):
 
 
 # ---------------------------------------------------------------------------
+# Frame-causal masking (the world-model rollout workload: queries in frame f see the
+# keys of frames <= f, intersected with the route).  The pages' sources describe the
+# per-call path without causality; READING: causality enters only where pairs are
+# counted or attended -- the masks, the cell mass (visible keys only), the cell cost
+# and the budget (visible pairs) -- and the grouping itself is unchanged.
+# ---------------------------------------------------------------------------
+def causal_mask(frames, rows=None) -> np.ndarray:
+    """bool [len(rows), N]: key k is visible to query q iff frame(k) <= frame(q)."""
+    f = np.asarray(frames)
+    fq = f if rows is None else f[np.asarray(rows)]
+    return f[None, :] <= fq[:, None]
+
+
+def visible_counts(labels, frames, n_groups: int, n_frames: int) -> np.ndarray:
+    """int64 [n_groups, n_frames]: tokens of group g in frames <= f (cumulative in f)."""
+    c = np.zeros((n_groups, n_frames), np.int64)
+    np.add.at(c, (np.asarray(labels), np.asarray(frames)), 1)
+    return np.cumsum(c, axis=1)
+
+
+def frame_histogram(labels, frames, n_groups: int, n_frames: int) -> np.ndarray:
+    """int64 [n_groups, n_frames]: tokens of group a in frame f."""
+    c = np.zeros((n_groups, n_frames), np.int64)
+    np.add.at(c, (np.asarray(labels), np.asarray(frames)), 1)
+    return c
+
+
+# ---------------------------------------------------------------------------
 # Response-coupled partitioning  [gist 2.A], [hs method], [abstract]
 # ---------------------------------------------------------------------------
 def sample_queries(n: int, m_s: int, seed: int, bh: int) -> np.ndarray:
@@ -262,16 +290,21 @@ def group_permutation(labels, n_groups: int):
 # ---------------------------------------------------------------------------
 # Route  [hs exec] budget by product of group sizes; [hs method] Fig. 2 alpha
 # ---------------------------------------------------------------------------
-def cell_mass(z, label_q, n_k, n_qgroups: int) -> np.ndarray:
+def cell_mass(z, label_q, n_k, n_qgroups: int, frames=None, vis_k=None) -> np.ndarray:
     """Estimated attention mass of query group a on K/V group g.
 
     READING: a query's mass on group g is estimated from its centroid logit,
     sum_{k in g} exp(s q.k) ~ n_g exp(z_q[g]), normalised over groups:
     p_q(g) = softmax_g(z_q[g] + ln n_g) (empty groups excluded); the cell mass
-    p(a, g) is the mean of p_q(g) over the queries of group a (0 for empty a)."""
+    p(a, g) is the mean of p_q(g) over the queries of group a (0 for empty a).
+    Frame-causal (frames = frame per token, vis_k = visible_counts of the keys):
+    n_g is the number of keys of g the query can see, vis_k[g, frame(q)]."""
     z = np.asarray(z, np.float64)
-    n_k = np.asarray(n_k)
-    logit = np.where(n_k[None, :] > 0, z + np.log(np.maximum(n_k, 1))[None, :], -np.inf)
+    if frames is None:
+        n_vis = np.broadcast_to(np.asarray(n_k)[None, :], z.shape)
+    else:
+        n_vis = np.asarray(vis_k)[:, np.asarray(frames)].T       # [N, Gk]
+    logit = np.where(n_vis > 0, z + np.log(np.maximum(n_vis, 1)), -np.inf)
     mx = logit.max(axis=1, keepdims=True)
     p = np.exp(logit - mx)
     p /= p.sum(axis=1, keepdims=True)
@@ -283,9 +316,13 @@ def cell_mass(z, label_q, n_k, n_qgroups: int) -> np.ndarray:
     return out
 
 
-def cell_cost(n_q, n_k) -> np.ndarray:
-    """Executed token pairs of cell (a, g): n_a * n_g (non-causal)  [hs exec]."""
-    return np.outer(np.asarray(n_q, np.int64), np.asarray(n_k, np.int64))
+def cell_cost(n_q, n_k, hist_q=None, vis_k=None) -> np.ndarray:
+    """Executed token pairs of cell (a, g): n_a * n_g  [hs exec].  Frame-causal
+    (hist_q = frame_histogram of the queries, vis_k = visible_counts of the keys):
+    the visible pairs sum_f hist_q[a, f] * vis_k[g, f]."""
+    if hist_q is None:
+        return np.outer(np.asarray(n_q, np.int64), np.asarray(n_k, np.int64))
+    return np.asarray(hist_q, np.int64) @ np.asarray(vis_k, np.int64).T
 
 
 @dataclass
@@ -333,7 +370,7 @@ def _route_cost(rows, alpha):
 
 
 def route_select(mass, n_q, n_k, density: float, n_probes: int, n_tokens: int,
-                 bisect_steps: int = 60) -> RouteResult:
+                 bisect_steps: int = 60, cost=None, visible=None) -> RouteResult:
     """Pick the (query group, K/V group) cells to execute.
 
     READING (parity unpinned as a rule -- the pages fix only its ingredients):
@@ -343,13 +380,16 @@ def route_select(mass, n_q, n_k, density: float, n_probes: int, n_tokens: int,
     group sizes (hs exec); the probe rows' exact pairs are charged first
     (gist 2.C: rho_exec includes the probe rows); alpha is the largest value in
     [0, 1] whose cost fits the budget, found by bisection in fp64.  density >= 1
-    routes every non-empty cell."""
+    routes every non-empty cell.  Frame-causal: cost = the visible pairs per cell and
+    visible = all visible pairs; READING: the probe rows are charged their expected
+    visible keys, n_probes * visible / n_tokens (= n_probes * n_tokens without
+    causality), since they are drawn after the route."""
     mass = np.asarray(mass, np.float64)
     n_q = np.asarray(n_q, np.int64)
     n_k = np.asarray(n_k, np.int64)
-    cost = cell_cost(n_q, n_k)
-    visible = float(n_tokens) * float(n_tokens)
-    probe_pairs = float(n_probes) * float(n_tokens)
+    cost = cell_cost(n_q, n_k) if cost is None else np.asarray(cost, np.int64)
+    visible = float(n_tokens) * float(n_tokens) if visible is None else float(visible)
+    probe_pairs = float(n_probes) * visible / float(n_tokens)
     budget = density * visible - probe_pairs
     rows = _route_prefix(mass, cost, n_q, n_k)
     route = np.zeros(mass.shape, np.uint8)
@@ -400,16 +440,20 @@ def block_mask(route, label_q, perm_q, label_k, perm_k, block: int) -> np.ndarra
 # ---------------------------------------------------------------------------
 # Sparse attention over the route  [gist 2.C]
 # ---------------------------------------------------------------------------
-def pair_mask(route, label_q, label_k, rows=None) -> np.ndarray:
-    """Token-pair mask: query q may see key k iff route[label_q[q], label_k[k]]."""
+def pair_mask(route, label_q, label_k, rows=None, frames=None) -> np.ndarray:
+    """Token-pair mask: query q may see key k iff route[label_q[q], label_k[k]]
+    (and, frame-causal, frame(k) <= frame(q))."""
     lq = np.asarray(label_q) if rows is None else np.asarray(label_q)[rows]
-    return np.asarray(route, bool)[lq][:, np.asarray(label_k)]
+    m = np.asarray(route, bool)[lq][:, np.asarray(label_k)]
+    if frames is not None:
+        m &= causal_mask(frames, rows)
+    return m
 
 
-def sparse_attention(q, k, v, scale, route, label_q, label_k, rows=None):
+def sparse_attention(q, k, v, scale, route, label_q, label_k, rows=None, frames=None):
     """O_sparse and LSE for rows (all rows by default), original token order."""
     rows = np.arange(len(q)) if rows is None else np.asarray(rows)
-    m = pair_mask(route, label_q, label_k, rows)
+    m = pair_mask(route, label_q, label_k, rows, frames)
     return attention(np.asarray(q)[rows], k, v, scale, mask=m)
 
 
@@ -596,7 +640,7 @@ class HeadPartition:
 
 
 def partition_head(q, k, p: Params, bh: int, key_coords_override=None,
-                   query_coords_override=None, mass_override=None) -> HeadPartition:
+                   query_coords_override=None, mass_override=None, frames=None) -> HeadPartition:
     """Response-coupled partition of one head: Q -> K grouping, then K -> Q grouping,
     a single asymmetric pass (gist 2.A; hs method), followed by the route.
 
@@ -619,8 +663,18 @@ def partition_head(q, k, p: Params, bh: int, key_coords_override=None,
     n_q = np.bincount(label_q, minlength=p.n_qgroups).astype(np.int64)
     perm_q, qoff = group_permutation(label_q, p.n_qgroups)
     perm_k, koff = group_permutation(label_k, p.n_kgroups)
-    mass = cell_mass(z, label_q, n_k, p.n_qgroups) if mass_override is None else np.asarray(mass_override, np.float64)
-    rr = route_select(mass, n_q, n_k, p.density, p.n_probes, n)
+    if frames is None:
+        mass = cell_mass(z, label_q, n_k, p.n_qgroups) if mass_override is None else np.asarray(mass_override, np.float64)
+        rr = route_select(mass, n_q, n_k, p.density, p.n_probes, n)
+    else:
+        nf = int(np.max(frames)) + 1
+        vis_k = visible_counts(label_k, frames, p.n_kgroups, nf)
+        hist_q = frame_histogram(label_q, frames, p.n_qgroups, nf)
+        mass = (cell_mass(z, label_q, n_k, p.n_qgroups, frames, vis_k) if mass_override is None
+                else np.asarray(mass_override, np.float64))
+        cost = cell_cost(n_q, n_k, hist_q, vis_k)
+        visible = float(hist_q.sum(axis=0) @ vis_k.sum(axis=0))
+        rr = route_select(mass, n_q, n_k, p.density, p.n_probes, n, cost=cost, visible=visible)
     bm = block_mask(rr.route, label_q, perm_q, label_k, perm_k, p.block)
     return HeadPartition(sample_idx=idx, metric=m_k, eigval=lam, eigvec=u, key_coords=y,
                          key_init=kinit, label_k=label_k, key_label_history=hist_k,
@@ -631,14 +685,14 @@ def partition_head(q, k, p: Params, bh: int, key_coords_override=None,
 
 
 def probe_fit_head(q, k, v, part_label_q, part_label_k, route, perm_q, q_offsets,
-                   p: Params, bh: int) -> ProbeFit:
+                   p: Params, bh: int, frames=None) -> ProbeFit:
     """Exact probe rows (dense and routed attention), residual, subspace, ridge."""
     q = np.asarray(q, np.float64)
     d = q.shape[1]
     s = p.eff_scale(d)
     pidx = pick_probes(perm_q, q_offsets, p.n_probes, p.seed, bh)
-    o_d, l_d = attention(q[pidx], k, v, s)
-    o_s, l_s = sparse_attention(q, k, v, s, route, part_label_q, part_label_k, rows=pidx)
+    o_d, l_d = attention(q[pidx], k, v, s, mask=None if frames is None else causal_mask(frames, pidx))
+    o_s, l_s = sparse_attention(q, k, v, s, route, part_label_q, part_label_k, rows=pidx, frames=frames)
     return fit_from_probes(pidx, o_d, o_s, l_d, l_s, p.sub_rank, p.ridge_lambda)
 
 
@@ -651,18 +705,18 @@ class HeadResult:
     o: np.ndarray
 
 
-def sparsepr_head(q, k, v, p: Params, bh: int) -> HeadResult:
+def sparsepr_head(q, k, v, p: Params, bh: int, frames=None) -> HeadResult:
     """The whole per-call path for one head (huashangw sparse-execution section's
     stage list: grouping, route, permutation, sparse attention, exact probes,
     residual fit, correction, output restoration)."""
     q = np.asarray(q, np.float64)
     d = q.shape[1]
     s = p.eff_scale(d)
-    part = partition_head(q, k, p, bh)
+    part = partition_head(q, k, p, bh, frames=frames)
     route = part.route.route
-    o_s, l_s = sparse_attention(q, k, v, s, route, part.label_q, part.label_k)
+    o_s, l_s = sparse_attention(q, k, v, s, route, part.label_q, part.label_k, frames=frames)
     fit = probe_fit_head(q, k, v, part.label_q, part.label_k, route, part.perm_q,
-                         part.q_offsets, p, bh)
+                         part.q_offsets, p, bh, frames=frames)
     o = correct(o_s, fit)
     return HeadResult(part=part, o_sparse=o_s, lse_sparse=l_s, fit=fit, o=o)
 

@@ -88,6 +88,9 @@ WORKLOADS = {
                   calibrated=True, drift=0.1),
     "world": _make("world", 4, 16, (16, 32, 32), 128, 128, 256, 128, 0.25,
                    calibrated=True, frame_causal=True),
+    # the 1024-token case with the frame-causal mask (4 frames of 256 tokens)
+    "tiny_causal": _make("tiny_causal", 1, 2, (4, 16, 16), 64, 16, 16, 64, 0.25, groups=8,
+                         n_samples=64, sub_rank=16, kmeans_iters=8, frame_causal=True),
 }
 
 
