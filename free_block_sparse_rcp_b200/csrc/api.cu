@@ -51,9 +51,11 @@ struct Layout {
   size_t err;
   // partition
   size_t sample_idx, metric, eigval, eigvec, proj, eig_lu, m_k, nu_k, key_init, C, m_q, nu_q, query_init, bias, wnorm,
-      w_hi, w_lo, flag_count, flag_rows, corr_count, corr, psum, pcnt, mass, order, cm, cc, alpha;
+      w_hi, w_lo, flag_count, flag_rows, corr_count, corr, psum, pcnt, mass, order, alpha;
   // attend
   size_t rlist, rcum, rcnt, tiles, tile_count;
+  // frame-causal tables (zero-sized without frame ids): partition / attend / probe regions
+  size_t c_fend, c_visk, c_qcum, a_visk, a_klist, a_tlim, p_fend;
   // probe
   size_t probe_grp, part_o, part_ml, o_sparse_p, lse_d, lse_s;
   size_t total;
@@ -61,7 +63,7 @@ struct Layout {
   size_t f_perm_q, f_perm_k, f_label_q, f_label_k, f_qoff, f_koff, f_route, f_bmask, f_rho, f_lse, f_probe_idx,
       f_probe_od, f_bfull, f_vr, f_w;
   size_t forward_total;
-  int BH, max_tiles, T, S, DTk, DTq;
+  int BH, max_tiles, T, S, DTk, DTq, F;
 };
 
 Layout make_layout(const sparsepr_params& p) {
@@ -106,14 +108,23 @@ Layout make_layout(const sparsepr_params& p) {
   }
   L.mass = take(BH * Gq * Gk * 4);
   L.order = take(BH * Gq * Gk * 4);
-  L.cm = take(BH * Gq * Gk * 8);
-  L.cc = take(BH * Gq * Gk * 8);
   L.alpha = take(BH * 8);
   L.rlist = take(BH * Gq * Gk * 4);
   L.rcum = take(BH * Gq * (Gk + 1) * 4);
   L.rcnt = take(BH * Gq * 4);
   L.tiles = take(BH * L.max_tiles * 8);
   L.tile_count = take(BH * 4);
+  L.F = p.frame_id ? p.n_frames : 0;
+  {
+    const size_t F = (size_t)L.F;
+    L.c_fend = take(F * 4);
+    L.c_visk = take(BH * Gk * F * 4);
+    L.c_qcum = take(BH * Gq * F * 4);
+    L.a_visk = take(BH * Gk * F * 4);
+    L.a_klist = take(F ? BH * Gq * N * 4 : 0);
+    L.a_tlim = take(BH * Gq * F * 4);
+    L.p_fend = take(F * 4);
+  }
   L.probe_grp = take(BH * P * 4);
   L.part_o = take(BH * L.S * 64 * 2 * d * 4);
   L.part_ml = take(BH * L.S * 64 * 4 * 4);
@@ -161,7 +172,13 @@ sparsepr_status check_params(const sparsepr_params* p) {
   if (p->kmeans_iters < 1 || p->kmeans_iters > 64) return failv(SPARSEPR_EINVAL, "kmeans_iters must be in [1, 64]", p->kmeans_iters);
   if (!(p->ridge_lambda > 0.f) || !isfinite(p->ridge_lambda)) return fail(SPARSEPR_EINVAL, "ridge_lambda must be > 0");
   if (!(p->scale >= 0.f) || !isfinite(p->scale)) return fail(SPARSEPR_EINVAL, "scale must be >= 0");
-  if (p->frame_id) return fail(SPARSEPR_EUNSUPPORTED, "frame-causal masking (frame_id) is not built");
+  if (p->frame_id) {
+    if (p->n_frames < 1 || p->n_frames > kMaxFrames)
+      return failv(SPARSEPR_EINVAL, "n_frames must be in [1, 64] with frame_id", p->n_frames);
+    if (p->N > 65535) return failv(SPARSEPR_EUNSUPPORTED, "frame-causal calls need N <= 65535", p->N);
+    if (causal_stream_smem(p->n_kgroups, p->n_frames) > kSmemLimit)
+      return fail(SPARSEPR_EUNSUPPORTED, "too many K/V groups x frames for the causal key stream");
+  }
   if (p->density < 1.f &&
       (double)p->density * (double)p->N * (double)p->N < (double)p->n_probes * (double)p->N)
     return fail(SPARSEPR_EINVAL, "density is below the probe floor n_probes/N");
@@ -175,7 +192,7 @@ sparsepr_status check_params(const sparsepr_params* p) {
     return fail(SPARSEPR_EUNSUPPORTED, "too many groups for the k-means kernels");
   if (route_select_smem(p->n_qgroups, p->n_kgroups) > kSmemLimit)
     return fail(SPARSEPR_EUNSUPPORTED, "too many groups for the route selection kernel");
-  if (cell_mass_tc_smem(p->d, kmeans_gp(p->n_kgroups)) > kSmemLimit)
+  if (cell_mass_tc_smem(p->d, kmeans_gp(p->n_kgroups), p->frame_id ? p->n_frames : 0) > kSmemLimit)
     return fail(SPARSEPR_EUNSUPPORTED, "too many K/V groups for the cell-mass kernel");
   if ((size_t)p->d * p->sub_rank > 64 * 65 || probe_fit_smem(p->d, p->sub_rank) > kSmemLimit)
     return failv(SPARSEPR_EUNSUPPORTED, "sub_rank too large for the single-CTA fit (d*r)", (long long)p->d * p->sub_rank);
@@ -270,13 +287,24 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
                    at<float>(ws, L.nu_q), at<int>(ws, L.query_init), label_q, perm_q, qoff,
                    tr ? tr->query_label_iters : nullptr, nullptr));
   float* mass = at<float>(ws, L.mass);
+  // frame-causal: visible keys per (K/V group, frame), query frame histograms, frame ends
+  Causal cz{};
+  if (p.frame_id) {
+    cz.frame_id = p.frame_id;
+    cz.F = L.F;
+    cz.fend = at<int>(ws, L.c_fend);
+    cz.visk = at<int>(ws, L.c_visk);
+    cz.qcum = at<int>(ws, L.c_qcum);
+    SPR_LAUNCH(launch_frame_ends(p.frame_id, N, L.F, at<int>(ws, L.c_fend), err, st));
+    SPR_LAUNCH(launch_group_frame_cum(perm_k, koff, p.frame_id, BH, N, Gk, L.F, at<int>(ws, L.c_visk), err, st));
+    SPR_LAUNCH(launch_group_frame_cum(perm_q, qoff, p.frame_id, BH, N, Gq, L.F, at<int>(ws, L.c_qcum), err, st));
+  }
   // the weight buffers are free again: they hold the three bf16 parts of C
   const size_t cpart = (size_t)BH * kmeans_gp(Gk) * d * 2;
   SPR_LAUNCH(launch_cell_mass_tc(Q, BH, N, d, Gq, Gk, perm_q, qoff, koff, C, scale, w_hi, w_lo,
-                                 at<char>(ws, L.w_lo) + cpart, mass, err, st));
-  SPR_LAUNCH(launch_route_select(mass, BH, N, Gq, Gk, qoff, koff, p.density, p.n_probes, at<int>(ws, L.order),
-                                 at<double>(ws, L.cm), at<long long>(ws, L.cc), route, rho,
-                                 at<double>(ws, L.alpha), st));
+                                 at<char>(ws, L.w_lo) + cpart, cz, mass, err, st));
+  SPR_LAUNCH(launch_route_select(mass, BH, N, Gq, Gk, qoff, koff, p.density, p.n_probes, cz, at<int>(ws, L.order),
+                                 route, rho, at<double>(ws, L.alpha), st));
   if (bmask)
     SPR_LAUNCH(launch_block_mask(route, BH, N, Gq, Gk, p.block, perm_q, label_q, perm_k, label_k, bmask, st));
   if (tr) {
@@ -315,6 +343,17 @@ sparsepr_status run_attend(const sparsepr_params& p, const Layout& L, const void
   a.max_tiles = L.max_tiles;
   a.scale_log2 = eff_scale(p) * 1.4426950408889634f;
   a.O = O; a.lse = lse; a.err = at<int>(ws, L.err);
+  if (p.frame_id) {
+    // each query group's routed keys in frame-major order, and its prefix per frame
+    int* visk = at<int>(ws, L.a_visk);
+    SPR_LAUNCH(launch_group_frame_cum(perm_k, koff, p.frame_id, L.BH, p.N, p.n_kgroups, L.F, visk, a.err, st));
+    SPR_LAUNCH(launch_causal_stream(rlist, rcnt, koff, perm_k, visk, L.BH, p.N, p.n_qgroups, p.n_kgroups, L.F,
+                                    at<int>(ws, L.a_klist), at<int>(ws, L.a_tlim), a.err, st));
+    a.cz.frame_id = p.frame_id;
+    a.cz.F = L.F;
+    a.cz.klist = at<int>(ws, L.a_klist);
+    a.cz.tlim = at<int>(ws, L.a_tlim);
+  }
   SPR_LAUNCH(launch_attention_tc(a, false, st));
   return SPARSEPR_OK;
 }
@@ -329,8 +368,15 @@ sparsepr_status run_probe_fit(const sparsepr_params& p, const Layout& L, const v
   SPR_LAUNCH(launch_probe_pick(perm_q, qoff, BH, N, p.n_qgroups, P, p.seed, probe_idx, pgrp, at<int>(ws, L.err), st));
   float* part_o = at<float>(ws, L.part_o);
   float* part_ml = at<float>(ws, L.part_ml);
+  Causal cz{};
+  if (p.frame_id) {
+    cz.frame_id = p.frame_id;
+    cz.F = L.F;
+    cz.fend = at<int>(ws, L.p_fend);
+    SPR_LAUNCH(launch_frame_ends(p.frame_id, N, L.F, at<int>(ws, L.p_fend), at<int>(ws, L.err), st));
+  }
   SPR_LAUNCH(launch_probe_attn(Q, K, V, BH, N, d, p.n_kgroups, p.n_qgroups, P, probe_idx, pgrp, label_k, route,
-                               eff_scale(p) * 1.4426950408889634f, part_o, part_ml, at<int>(ws, L.err), st));
+                               eff_scale(p) * 1.4426950408889634f, cz, part_o, part_ml, at<int>(ws, L.err), st));
   float* osp = at<float>(ws, L.o_sparse_p);
   float* lsd = at<float>(ws, L.lse_d);
   float* lss = at<float>(ws, L.lse_s);
@@ -488,9 +534,10 @@ sparsepr_status sparsepr_dense_attention(const sparsepr_params* p, const void* Q
   SPR_CHECK(check_params(p));
   SPR_NONNULL(Q); SPR_NONNULL(K); SPR_NONNULL(V); SPR_NONNULL(O);
   int* err = nullptr;
-  if (workspace) {
-    if (((uintptr_t)workspace & 255) != 0 || ws_bytes < 256)
-      return fail(SPARSEPR_EWORKSPACE, "workspace must be 256-byte aligned and >= 256 bytes");
+  const size_t need = p->frame_id ? 512 : 256;   // error word, then the frame ends
+  if (workspace || p->frame_id) {
+    if (!workspace || ((uintptr_t)workspace & 255) != 0 || ws_bytes < need)
+      return failv(SPARSEPR_EWORKSPACE, "workspace must be 256-byte aligned and hold (bytes)", (long long)need);
     err = static_cast<int*>(workspace);
   }
   AttnArgs a{};
@@ -498,6 +545,13 @@ sparsepr_status sparsepr_dense_attention(const sparsepr_params* p, const void* Q
   a.BH = p->B * p->H; a.N = p->N; a.D = p->d;
   a.scale_log2 = eff_scale(*p) * 1.4426950408889634f;
   a.O = O; a.lse = lse; a.err = err;
+  if (p->frame_id) {
+    int* fend = at<int>(workspace, 256);
+    SPR_LAUNCH(launch_frame_ends(p->frame_id, p->N, p->n_frames, fend, err, (cudaStream_t)stream));
+    a.cz.frame_id = p->frame_id;
+    a.cz.F = p->n_frames;
+    a.cz.fend = fend;
+  }
   SPR_LAUNCH(launch_attention_tc(a, true, (cudaStream_t)stream));
   return SPARSEPR_OK;
 }

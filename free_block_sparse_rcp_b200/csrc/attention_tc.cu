@@ -29,6 +29,12 @@
 // The softmax makes one speculative pass per chunk against the running max (exponentials
 // and the chunk max together, packed fp32x2 arithmetic) and keeps it unless some row's max
 // grew by more than 2^8; then the chunk is redone against the new max and O is rescaled.
+// Frame-causal variant (CAUSAL): a query of frame f sees only keys of frames <= f.  The
+// key stream is then ordered so that the keys a frame-f row may use are a prefix of it:
+// dense, the token order itself (frame ids are nondecreasing), prefix fend[f]; routed, the
+// query group's causal stream (its routed K/V groups' keys frame by frame), prefix
+// tlim[a][f].  A unit streams the prefix of its last row's frame; every row masks the
+// columns past its own prefix, which only the few chunks straddling a row's limit need.
 // K is staged in a 3-deep ring, V in a 2-deep ring.  Every mbarrier wait is bounded (2 s);
 // a timeout raises an abort flag that ends every role, records DERR_WAIT_TIMEOUT in the
 // workspace and still frees the TMEM.
@@ -75,7 +81,7 @@ struct Layout {
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
-template <int D, bool DENSE>
+template <int D, bool DENSE, bool CAUSAL>
 __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
               const __grid_constant__ CUtensorMap tmv, const __nv_bfloat16* __restrict__ Q,
@@ -84,7 +90,9 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
               const int* __restrict__ perm_k, const int* __restrict__ qoff, const int* __restrict__ koff,
               const int* __restrict__ rlist, const int* __restrict__ rcum, const int* __restrict__ rcnt,
               const int2* __restrict__ tiles, const int* __restrict__ tile_count, int max_tiles, float scale_log2,
-              __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int* err) {
+              const int* __restrict__ frame_id, const int* __restrict__ fend, const int* __restrict__ klist,
+              const int* __restrict__ tlim, int F, __nv_bfloat16* __restrict__ O, float* __restrict__ lse,
+              int* err) {
   using L = Layout<D>;
   constexpr int NT = Roles<DENSE>::NT;
   constexpr int MMA_WARP = Roles<DENSE>::MMA_WARP;
@@ -112,7 +120,7 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
   volatile int* abort_flag = sMisc + 1;
 
   // ---------------- setup (all threads) ----------------
-  int q0, qn;
+  int q0, qn, a = 0;
   if (DENSE) {
     q0 = blockIdx.x * (TPC * BM);
     if (q0 >= N) return;
@@ -120,22 +128,37 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
   } else {
     if ((int)blockIdx.x >= tile_count[bh]) return;
     const int2 tl = tiles[(size_t)bh * max_tiles + blockIdx.x];
-    const int a = tl.x;
+    a = tl.x;
     const int* qo = qoff + (size_t)bh * (Gq + 1);
     q0 = qo[a] + tl.y * (TPC * BM);
     qn = min(TPC * BM, qo[a + 1] - q0);
-    const int cnt = rcnt[(size_t)bh * Gq + a];
-    const int* rl = rlist + ((size_t)bh * Gq + a) * Gk;
-    const int* rc = rcum + ((size_t)bh * Gq + a) * (Gk + 1);
-    const int* ko = koff + (size_t)bh * (Gk + 1);
-    for (int i = tid; i < cnt; i += NT) {
-      sList[i] = rl[i];
-      sKoffL[i] = ko[rl[i]];
+    if (!CAUSAL) {
+      const int cnt = rcnt[(size_t)bh * Gq + a];
+      const int* rl = rlist + ((size_t)bh * Gq + a) * Gk;
+      const int* rc = rcum + ((size_t)bh * Gq + a) * (Gk + 1);
+      const int* ko = koff + (size_t)bh * (Gk + 1);
+      for (int i = tid; i < cnt; i += NT) {
+        sList[i] = rl[i];
+        sKoffL[i] = ko[rl[i]];
+      }
+      for (int i = tid; i <= cnt; i += NT) sCum[i] = rc[i];
+      if (tid == 0) { sMisc[2] = rc[cnt]; sMisc[3] = cnt; }
     }
-    for (int i = tid; i <= cnt; i += NT) sCum[i] = rc[i];
-    if (tid == 0) { sMisc[2] = rc[cnt]; sMisc[3] = cnt; }
   }
-  if (DENSE && tid == 0) { sMisc[2] = N; sMisc[3] = 0; }
+  // per-frame key prefix of the stream: fend (dense) or this query group's tlim (routed)
+  const int* frame_lim = CAUSAL ? (DENSE ? fend : tlim + ((size_t)bh * Gq + a) * F) : nullptr;
+  auto frame_of = [&](int row) -> int {
+    int f = (row >= 0 && row < N) ? frame_id[row] : F - 1;
+    return f < 0 ? 0 : (f >= F ? F - 1 : f);
+  };
+  if (CAUSAL && tid == 0) {
+    // the unit streams the prefix of its last (latest-frame) row
+    int tot = 0;
+    if (qn > 0) tot = frame_lim[frame_of(DENSE ? q0 + qn - 1 : perm_q[head + q0 + qn - 1])];
+    sMisc[2] = tot < 0 ? 0 : (tot > N ? N : tot);
+    sMisc[3] = 0;
+  }
+  if (DENSE && !CAUSAL && tid == 0) { sMisc[2] = N; sMisc[3] = 0; }
   if (tid < TPC * BM) {
     int row = -1;
     if (tid < qn) {
@@ -235,6 +258,9 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
         if (pos < total) {
           if (DENSE) {
             myrow = pos;
+          } else if (CAUSAL) {
+            myrow = klist[((size_t)bh * Gq + a) * N + pos];
+            if (myrow < 0 || myrow >= N) { set_error(err, DERR_INDEX); myrow = -1; }
           } else {
             int lo = 0, hi = cnt - 1;
             while (lo < hi) {
@@ -336,6 +362,12 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
     const uint32_t tS = tmem + 256 * t + lane_off, tO = tS + 128;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
+    // keys this row may use: the stream prefix of its frame (frame-causal), else all
+    int lim = total;
+    if (CAUSAL) {
+      const int row = sQrow[t * BM + r];
+      if (row >= 0) lim = min(total, frame_lim[frame_of(row)]);
+    }
     if (t < ntile) {
       uint32_t sreg[64];
       uint32_t pk[64];
@@ -344,8 +376,8 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
         ok = __all_sync(0xffffffffu, wait(bars->s_full[t], j & 1));
         if (!ok) break;
         tc_fence_after();
-        const int valid = total - j * BN;
-        const bool full = valid >= BN;
+        const int valid = lim - j * BN;
+        const bool full = CAUSAL ? __all_sync(0xffffffffu, valid >= BN) : valid >= BN;
         // Speculative single pass against the running max: P = exp2(S s log2e - m) and the
         // chunk's max together; kept only if no row's max grew by more than the threshold.
         bool need = true;
@@ -478,10 +510,10 @@ size_t attn_tc_smem_bytes(int D, int Gk) {
   return s < 120 * 1024 ? 120 * 1024 : s;
 }
 
-template <int D, bool DENSE>
+template <int D, bool DENSE, bool CAUSAL>
 static cudaError_t launch_tc_t(const AttnArgs& a, cudaStream_t st) {
   const size_t sm = attn_tc_smem_bytes(D, DENSE ? 0 : a.Gk);
-  auto kern = tc::k_attn_tc<D, DENSE>;
+  auto kern = tc::k_attn_tc<D, DENSE, CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   // tensor maps of 128-row boxes (used by the dense variant only)
@@ -496,13 +528,19 @@ static cudaError_t launch_tc_t(const AttnArgs& a, cudaStream_t st) {
   kern<<<grid, tc::Roles<DENSE>::NT, sm, st>>>(tq, tk, tv, (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K,
                                                (const __nv_bfloat16*)a.V, a.N, a.Gq, a.Gk, a.perm_q, a.perm_k, a.qoff,
                                                a.koff, a.rlist, a.rcum, a.rcnt, a.tiles, a.tile_count, a.max_tiles,
-                                               a.scale_log2, (__nv_bfloat16*)a.O, a.lse, a.err);
+                                               a.scale_log2, a.cz.frame_id, a.cz.fend, a.cz.klist, a.cz.tlim, a.cz.F,
+                                               (__nv_bfloat16*)a.O, a.lse, a.err);
   return cudaGetLastError();
 }
 
+template <int D>
+static cudaError_t launch_tc_d(const AttnArgs& a, bool dense, cudaStream_t st) {
+  if (a.cz.on()) return dense ? launch_tc_t<D, true, true>(a, st) : launch_tc_t<D, false, true>(a, st);
+  return dense ? launch_tc_t<D, true, false>(a, st) : launch_tc_t<D, false, false>(a, st);
+}
+
 cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, cudaStream_t st) {
-  if (a.D == 64) return dense ? launch_tc_t<64, true>(a, st) : launch_tc_t<64, false>(a, st);
-  return dense ? launch_tc_t<128, true>(a, st) : launch_tc_t<128, false>(a, st);
+  return a.D == 64 ? launch_tc_d<64>(a, dense, st) : launch_tc_d<128>(a, dense, st);
 }
 
 }  // namespace spr

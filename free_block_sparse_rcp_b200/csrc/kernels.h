@@ -6,6 +6,18 @@
 
 namespace spr {
 
+// Frame-causal inputs of the kernels below (all NULL / 0 without frame ids).
+struct Causal {
+  const int* frame_id = nullptr;   // [N]
+  const int* fend = nullptr;       // [F] tokens with frame <= f
+  const int* visk = nullptr;       // [BH][Gk][F] keys of group g with frame <= f
+  const int* qcum = nullptr;       // [BH][Gq][F] queries of group a with frame <= f
+  const int* klist = nullptr;      // [BH][Gq][N] causal key stream of each query group
+  const int* tlim = nullptr;       // [BH][Gq][F] its length through frame f
+  int F = 0;
+  bool on() const { return frame_id != nullptr; }
+};
+
 // partition.cu
 cudaError_t launch_sample_metric(const void* Q, int BH, int N, int D, int Ms, uint64_t seed, float* metric,
                                  int* sample_idx, int* err, cudaStream_t st);
@@ -21,13 +33,21 @@ cudaError_t launch_query_coords(const void* Q, int BH, int N, int D, const float
                                 float* Z, cudaStream_t st);
 size_t route_select_smem(int Gq, int Gk);
 cudaError_t launch_route_select(const float* mass, int BH, int N, int Gq, int Gk, const int* qoff,
-                                const int* koff, float density, int P, int* order, double* cm,
-                                long long* cc, unsigned char* route, float* rho_exec, double* alpha,
-                                cudaStream_t st);
+                                const int* koff, float density, int P, const Causal& cz, int* order,
+                                unsigned char* route, float* rho_exec, double* alpha, cudaStream_t st);
 cudaError_t launch_block_mask(const unsigned char* route, int BH, int N, int Gq, int Gk, int blk,
                               const int* perm_q, const int* label_q, const int* perm_k, const int* label_k,
                               unsigned char* bmask, cudaStream_t st);
 
+// frames.cu: tables of the frame-causal mask (frame ids nondecreasing in token order)
+constexpr int kMaxFrames = 64;
+cudaError_t launch_frame_ends(const int* frame_id, int N, int F, int* fend, int* err, cudaStream_t st);
+cudaError_t launch_group_frame_cum(const int* perm, const int* off, const int* frame_id, int BH, int N, int G, int F,
+                                   int* cum, int* err, cudaStream_t st);
+size_t causal_stream_smem(int Gk, int F);
+cudaError_t launch_causal_stream(const int* rlist, const int* rcnt, const int* koff, const int* perm_k,
+                                 const int* visk, int BH, int N, int Gq, int Gk, int F, int* klist, int* tlim,
+                                 int* err, cudaStream_t st);
 // tma_host.cu: 128-byte tensor map (CUtensorMap) of a row-major bf16 matrix for boxes of
 // box_rows x 64 columns with 128B swizzle; rows past the end read as zeros.
 cudaError_t make_tmap_bf16_rows(void* tmap, const void* base, unsigned long long rows, int cols, int box_rows);
@@ -60,10 +80,10 @@ cudaError_t launch_assign_recheck(const void* X, int BH, int N, int d, const flo
                                   float a_scale, int D, const float* nu, int G, const int* flag_count,
                                   const int* flag_rows, int* labels, int* trace, int* corr_count, void* corr,
                                   cudaStream_t st);
-size_t cell_mass_tc_smem(int D, int GP);
+size_t cell_mass_tc_smem(int D, int GP, int F);
 cudaError_t launch_cell_mass_tc(const void* Q, int BH, int N, int d, int Gq, int Gk, const int* perm_q, const int* qoff,
                                 const int* koff, const float* C, float scale, void* c1, void* c2, void* c3,
-                                float* mass, int* err, cudaStream_t st);
+                                const Causal& cz, float* mass, int* err, cudaStream_t st);
 
 // probe.cu
 cudaError_t launch_worklist(const unsigned char* route, const int* qoff, const int* koff, int BH, int Gq, int Gk,
@@ -75,12 +95,13 @@ int probe_splits(int N);
 size_t probe_tc_smem_bytes(int D, int Gk);
 cudaError_t launch_probe_tc(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk, int Gq, int P,
                             const int* probe_idx, const int* probe_grp, const int* label_k, const unsigned char* route,
-                            float scale_log2, int S, float* part_o, float* part_ml, int* err, cudaStream_t st);
+                            float scale_log2, int S, const Causal& cz, float* part_o, float* part_ml, int* err,
+                            cudaStream_t st);
 size_t probe_fit_smem(int D, int Rk);
 cudaError_t launch_probe_attn(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk, int Gq,
                               int P, const int* probe_idx, const int* probe_grp, const int* label_k,
-                              const unsigned char* route, float scale_log2, float* part_o, float* part_ml, int* err,
-                              cudaStream_t st);
+                              const unsigned char* route, float scale_log2, const Causal& cz, float* part_o,
+                              float* part_ml, int* err, cudaStream_t st);
 cudaError_t launch_probe_attn_splits(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk,
                                      int Gq, int P, const int* probe_idx, const int* probe_grp, const int* label_k,
                                      const unsigned char* route, float scale_log2, int S, float* part_o,
@@ -115,6 +136,7 @@ struct AttnArgs {
   const int* tile_count;
   int max_tiles;
   float scale_log2;
+  Causal cz;
   void* O;
   float* lse;
   int* err;

@@ -682,6 +682,8 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
                                                             const __nv_bfloat16* __restrict__ c1,
                                                             const __nv_bfloat16* __restrict__ c2,
                                                             const __nv_bfloat16* __restrict__ c3, float scale_log2,
+                                                            const int* __restrict__ frame_id,
+                                                            const int* __restrict__ visk, int F,
                                                             float* __restrict__ mass, int* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t base = su32(smem);
@@ -702,6 +704,9 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
   float* lnn = colacc + GP;                                          // [GP] log2 n_g or -inf
   cmk::Bars* bars = reinterpret_cast<cmk::Bars*>(lnn + GP);
   int* sMisc = reinterpret_cast<int*>(bars + 1);                     // [0] tmem, [1] abort
+  // frame-causal: [F][GP + 1] log2 of the keys of g a frame-f query sees, or -inf
+  float* lnf = reinterpret_cast<float*>(sMisc + 4);
+  const bool causal = frame_id != nullptr;
   volatile int* abort_flag = sMisc + 1;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float NEG_INF = __int_as_float(0xff800000);
@@ -752,6 +757,13 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
       const int n = g < Gk ? koff[(size_t)bh * (Gk + 1) + g + 1] - koff[(size_t)bh * (Gk + 1) + g] : 0;
       lnn[g] = n > 0 ? log2f((float)n) : NEG_INF;
       colacc[g] = 0.f;
+    }
+    if (causal) {
+      for (int e = tid; e < F * GP; e += cmk::NT) {
+        const int f = e / GP, g = e - f * GP;
+        const int n = g < Gk ? visk[((size_t)bh * Gk + g) * F + f] : 0;
+        lnf[f * (GP + 1) + g] = n > 0 ? log2f((float)n) : NEG_INF;
+      }
     }
     cp_async_wait_all();
     fence_proxy_async();
@@ -837,12 +849,20 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
           }
           tc_fence_before();
           mbar_arrive(su32(&bars->tempty[b]));
+          // log2 group sizes this row sees (frame-causal: the keys of frames <= its frame)
+          const float* lnrow = lnn;
+          if (causal && r < nr) {
+            const int row = perm_q[head + t0 + r];
+            int f = (row >= 0 && row < N) ? frame_id[row] : 0;
+            f = f < 0 ? 0 : (f >= F ? F - 1 : f);
+            lnrow = lnf + f * (GP + 1);
+          }
           // this quarter: logits in log2 units, local max and local sum
           float mq = NEG_INF;
           if (cb < GP) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const float ln = lnn[cb + e];
+              const float ln = lnrow[cb + e];
               v[e] = ln == NEG_INF ? NEG_INF : fmaf(v[e], scale_log2, ln);
               mq = fmaxf(mq, v[e]);
             }
@@ -999,9 +1019,9 @@ cudaError_t launch_assign_recheck(const void* X, int BH, int N, int d, const flo
   }
 }
 
-size_t cell_mass_tc_smem(int D, int GP) {
+size_t cell_mass_tc_smem(int D, int GP, int F) {
   return (size_t)2 * 128 * D * 2 + 3 * (size_t)GP * D * 2 + (size_t)2 * 16 * 32 * 4 + (size_t)2 * 4 * 128 * 8 +
-         (size_t)2 * GP * 4 + sizeof(km::cmk::Bars) + 16;
+         (size_t)2 * GP * 4 + sizeof(km::cmk::Bars) + 16 + (size_t)F * (GP + 1) * 4;
 }
 
 static int sm_count() {
@@ -1017,13 +1037,14 @@ static int sm_count() {
 
 cudaError_t launch_cell_mass_tc(const void* Q, int BH, int N, int d, int Gq, int Gk, const int* perm_q, const int* qoff,
                                 const int* koff, const float* C, float scale, void* c1, void* c2, void* c3,
-                                float* mass, int* err, cudaStream_t st) {
+                                const Causal& cz, float* mass, int* err, cudaStream_t st) {
   const int GP = kmeans_gp(Gk);
   km::k_split3<<<dim3(GP, BH), 128, 0, st>>>(C, Gk, GP, d, (__nv_bfloat16*)c1, (__nv_bfloat16*)c2,
                                             (__nv_bfloat16*)c3);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t sm = cell_mass_tc_smem(d, GP);
+  const int F = cz.on() ? cz.F : 0;
+  const size_t sm = cell_mass_tc_smem(d, GP, F);
   const int nitems = BH * Gq;
   const int grid = nitems < sm_count() ? nitems : sm_count();
   const float scale_log2 = scale * 1.4426950408889634f;
@@ -1031,13 +1052,14 @@ cudaError_t launch_cell_mass_tc(const void* Q, int BH, int N, int d, int Gq, int
     cudaFuncSetAttribute(km::k_cell_mass_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     km::k_cell_mass_tc<64><<<grid, km::cmk::NT, sm, st>>>((const __nv_bfloat16*)Q, N, Gq, Gk, GP, nitems, perm_q, qoff,
                                                          koff, (const __nv_bfloat16*)c1, (const __nv_bfloat16*)c2,
-                                                         (const __nv_bfloat16*)c3, scale_log2, mass, err);
+                                                         (const __nv_bfloat16*)c3, scale_log2, cz.frame_id, cz.visk,
+                                                         F, mass, err);
   } else {
     cudaFuncSetAttribute(km::k_cell_mass_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     km::k_cell_mass_tc<128><<<grid, km::cmk::NT, sm, st>>>((const __nv_bfloat16*)Q, N, Gq, Gk, GP, nitems, perm_q,
                                                           qoff, koff, (const __nv_bfloat16*)c1,
                                                           (const __nv_bfloat16*)c2, (const __nv_bfloat16*)c3,
-                                                          scale_log2, mass, err);
+                                                          scale_log2, cz.frame_id, cz.visk, F, mass, err);
   }
   return cudaGetLastError();
 }

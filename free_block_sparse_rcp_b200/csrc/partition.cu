@@ -268,15 +268,24 @@ __device__ long long block_sum_ll(long long v, long long* red) {
 // memory (the cumulative mass is summed sequentially in rank order, as the definition
 // reads); one warp evaluates one candidate alpha over all query groups.
 // grid = BH, block = 1024, dynamic smem = route_select_smem(Gq, Gk).
+//
+// Frame-causal (qcum != NULL): the cost of cell (a, g) is its visible pairs,
+// sum_f hist_q[a][f] * visk[g][f] with hist_q the per-frame query counts of group a, and the
+// budget is density * V - P * V / N with V = sum_f (tokens of frame f) * (tokens of frames
+// <= f).  Per-row cumulative costs are then at most n_a * N < 2^32 (N <= 65535).
 __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__ mass, int N, int Gq, int Gk,
                                                       const int* __restrict__ qoff, const int* __restrict__ koff,
-                                                      float density, int P, int* __restrict__ order,
+                                                      float density, int P, const int* __restrict__ qcum,
+                                                      const int* __restrict__ visk, const int* __restrict__ fend,
+                                                      int F, int* __restrict__ order,
                                                       unsigned char* __restrict__ route,
                                                       float* __restrict__ rho_exec, double* __restrict__ alpha_out) {
   extern __shared__ __align__(16) unsigned char smem[];
+  const bool causal = qcum != nullptr;
   double* cmh = reinterpret_cast<double*>(smem);               // [Gq][Gk] cumulative mass in rank order
-  int* pnk = reinterpret_cast<int*>(cmh + (size_t)Gq * Gk);     // [Gq][Gk] cumulative K/V sizes
-  int* nk = pnk + (size_t)Gq * Gk;                              // [Gk]
+  // [Gq][Gk] cumulative K/V sizes (causal: cumulative cell costs)
+  unsigned* pnk = reinterpret_cast<unsigned*>(cmh + (size_t)Gq * Gk);
+  int* nk = reinterpret_cast<int*>(pnk + (size_t)Gq * Gk);      // [Gk]
   int* nq = nk + Gk;                                            // [Gq]
   int* misc = nq + Gq;                                          // [0] L, [1..32] round flags
   long long* red = reinterpret_cast<long long*>(                // [32], 8-byte aligned
@@ -299,7 +308,9 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
   // group; empty groups last) into the warp's scratch, then lane 0 takes the cumulative mass
   // (fp64, rank order, sequential) and cumulative K/V sizes
   float* wm = reinterpret_cast<float*>(red + 32) + warp * 2 * Gk;   // [Gk] masses in rank order
-  int* wn = reinterpret_cast<int*>(wm + Gk);                        // [Gk] their K/V sizes
+  unsigned* wn = reinterpret_cast<unsigned*>(wm + Gk);              // [Gk] their K/V sizes / cell costs
+  const int* qc_h = causal ? qcum + (size_t)blockIdx.x * Gq * F : nullptr;
+  const int* vk_h = causal ? visk + (size_t)blockIdx.x * Gk * F : nullptr;
   __syncthreads();
   const int L = misc[0];
   int GS = 32;
@@ -353,13 +364,22 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
       if (q < per_lane && r < L) {
         oh[a * Gk + r] = ki[q];
         wm[r] = km[q];
-        wn[r] = nk[ki[q]];
+        if (causal) {
+          // visible pairs of cell (a, g): sum_f (queries of a in frame f) (keys of g in frames <= f)
+          const int* qa = qc_h + (size_t)a * F;
+          const int* vg = vk_h + (size_t)ki[q] * F;
+          unsigned c = 0u;
+          for (int f = 0; f < F; ++f) c += (unsigned)(qa[f] - (f > 0 ? qa[f - 1] : 0)) * (unsigned)vg[f];
+          wn[r] = c;
+        } else {
+          wn[r] = (unsigned)nk[ki[q]];
+        }
       }
     }
     __syncwarp();
     if (lane == 0) {
       double sm = 0.0;
-      int c = 0;
+      unsigned c = 0u;
       for (int r = 0; r < L; ++r) {
         sm += (double)wm[r];
         c += wn[r];
@@ -370,14 +390,24 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
     __syncwarp();
   }
   __syncthreads();
-  const double visible = (double)N * (double)N;
-  const double probe_pairs = (double)P * (double)N;
+  double visible = (double)N * (double)N;
+  if (causal) {
+    long long v = 0;
+    for (int f = 0; f < F; ++f) v += (long long)(fend[f] - (f > 0 ? fend[f - 1] : 0)) * (long long)fend[f];
+    visible = (double)v;
+  }
+  const double probe_pairs = causal ? (double)P * visible / (double)N : (double)P * (double)N;
   const double budget = (double)density * visible - probe_pairs;
+  // routed pairs of row a when its prefix holds len cells
+  auto row_cost = [&](int a, int len) -> long long {
+    const long long c = (long long)pnk[(size_t)a * Gk + len - 1];
+    return causal ? c : (long long)nq[a] * c;
+  };
   // cost of alpha over the rows a = lane, lane + 32, ... (warp-wide sum)
   auto warp_cost = [&](double al) -> long long {
     long long t = 0;
     for (int a = lane; a < Gq; a += 32)
-      if (nq[a] > 0) t += (long long)nq[a] * (long long)pnk[(size_t)a * Gk + prefix_len(cmh + (size_t)a * Gk, L, al) - 1];
+      if (nq[a] > 0) t += row_cost(a, prefix_len(cmh + (size_t)a * Gk, L, al));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
     return t;
@@ -429,7 +459,7 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
     if (nq[a] == 0) continue;
     const int len = all ? L : prefix_len(cmh + (size_t)a * Gk, L, alpha);
     for (int r = 0; r < len; ++r) rh[a * Gk + oh[a * Gk + r]] = 1;
-    routed += (long long)nq[a] * (long long)pnk[(size_t)a * Gk + len - 1];
+    routed += row_cost(a, len);
   }
   routed = block_sum_ll(routed, red);
   if (tid == 0) {
@@ -546,14 +576,12 @@ size_t route_select_smem(int Gq, int Gk) {
 }
 
 cudaError_t launch_route_select(const float* mass, int BH, int N, int Gq, int Gk, const int* qoff,
-                                const int* koff, float density, int P, int* order, double* cm,
-                                long long* cc, unsigned char* route, float* rho_exec, double* alpha,
-                                cudaStream_t st) {
-  (void)cm;
-  (void)cc;
+                                const int* koff, float density, int P, const Causal& cz, int* order,
+                                unsigned char* route, float* rho_exec, double* alpha, cudaStream_t st) {
   const size_t sm = route_select_smem(Gq, Gk);
   cudaFuncSetAttribute(k_route_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  k_route_select<<<BH, 1024, sm, st>>>(mass, N, Gq, Gk, qoff, koff, density, P, order, route, rho_exec, alpha);
+  k_route_select<<<BH, 1024, sm, st>>>(mass, N, Gq, Gk, qoff, koff, density, P, cz.on() ? cz.qcum : nullptr,
+                                       cz.visk, cz.fend, cz.F, order, route, rho_exec, alpha);
   return cudaGetLastError();
 }
 

@@ -593,10 +593,10 @@ int probe_splits(int N) {
 
 cudaError_t launch_probe_attn(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk, int Gq,
                               int P, const int* probe_idx, const int* probe_grp, const int* label_k,
-                              const unsigned char* route, float scale_log2, float* part_o, float* part_ml, int* err,
-                              cudaStream_t st) {
+                              const unsigned char* route, float scale_log2, const Causal& cz, float* part_o,
+                              float* part_ml, int* err, cudaStream_t st) {
   return launch_probe_tc(Q, K, V, BH, N, D, Gk, Gq, P, probe_idx, probe_grp, label_k, route, scale_log2,
-                         probe_splits(N), part_o, part_ml, err, st);
+                         probe_splits(N), cz, part_o, part_ml, err, st);
 }
 
 // Split-count-explicit variants (the key-split count S is chosen by the caller instead
@@ -605,8 +605,8 @@ cudaError_t launch_probe_attn_splits(const void* Q, const void* K, const void* V
                                      int Gq, int P, const int* probe_idx, const int* probe_grp, const int* label_k,
                                      const unsigned char* route, float scale_log2, int S, float* part_o,
                                      float* part_ml, cudaStream_t st) {
-  return launch_probe_tc(Q, K, V, BH, N, D, Gk, Gq, P, probe_idx, probe_grp, label_k, route, scale_log2, S, part_o,
-                         part_ml, nullptr, st);
+  return launch_probe_tc(Q, K, V, BH, N, D, Gk, Gq, P, probe_idx, probe_grp, label_k, route, scale_log2, S, Causal{},
+                         part_o, part_ml, nullptr, st);
 }
 
 cudaError_t launch_probe_combine_splits(const float* part_o, const float* part_ml, int BH, int S, int P, int D,

@@ -77,6 +77,10 @@ extern "C" sparsepr_status sparsepr_probe_fit_noalloc(const sparsepr_params* p, 
                                                       float* Bmat, void* stream) {
   const sparsepr_status st0 = sparsepr_validate(p);
   if (st0 != SPARSEPR_OK) return st0;
+  if (p->frame_id) {
+    set_last_error("sparsepr_probe_fit_noalloc: frame-causal probes need the workspace entry point");
+    return SPARSEPR_EUNSUPPORTED;
+  }
   if (!Q || !K || !V || !label_k || !perm_q || !qoff || !route || !probe_idx || !probe_o_dense || !b_full ||
       !Vr || !W) {
     set_last_error("sparsepr_probe_fit_noalloc: a required pointer is NULL");

@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(NT, 1)
                const __grid_constant__ CUtensorMap tmv, int N, int Gk, int Gq, int P,
                const int* __restrict__ probe_idx, const int* __restrict__ probe_grp, const int* __restrict__ label_k,
                const unsigned char* __restrict__ route, int keys_per_split, float scale_log2,
+               const int* __restrict__ frame_id, const int* __restrict__ fend, int F,
                float* __restrict__ part_o, float* __restrict__ part_ml, int* err) {
   using L = Layout<D>;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -217,6 +218,16 @@ __global__ void __launch_bounds__(NT, 1)
           if (rr[g]) rm[g >> 5] |= 1u << (g & 31);
       }
     }
+    // frame-causal: the row sees the keys before fend[its frame] (frame ids nondecreasing)
+    int kend = k1;
+    if (frame_id && prow < P) {
+      const int row = sQrow[prow];
+      if (row >= 0) {
+        int f = frame_id[row];
+        f = f < 0 ? 0 : (f >= F ? F - 1 : f);
+        kend = min(k1, fend[f]);
+      }
+    }
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nchunks; ++j) {
@@ -225,7 +236,7 @@ __global__ void __launch_bounds__(NT, 1)
       ok = __all_sync(0xffffffffu, wait(bars->s_full[b], (j >> 1) & 1) && wait(bars->full[b], (j >> 1) & 1));
       if (!ok) break;
       tc_fence_after();
-      const int valid = k1 - (k0 + j * BN);
+      const int valid = kend - (k0 + j * BN);
       // keys of this quarter the row may use
       uint32_t km = 0u;
       {
@@ -365,7 +376,8 @@ size_t probe_tc_smem_bytes(int D, int Gk) {
 
 cudaError_t launch_probe_tc(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk, int Gq, int P,
                             const int* probe_idx, const int* probe_grp, const int* label_k, const unsigned char* route,
-                            float scale_log2, int S, float* part_o, float* part_ml, int* err, cudaStream_t st) {
+                            float scale_log2, int S, const Causal& cz, float* part_o, float* part_ml, int* err,
+                            cudaStream_t st) {
   int kps = (N + S - 1) / S;
   kps = (kps + ptc::BN - 1) / ptc::BN * ptc::BN;
   const size_t sm = probe_tc_smem_bytes(D, Gk);
@@ -377,11 +389,13 @@ cudaError_t launch_probe_tc(const void* Q, const void* K, const void* V, int BH,
   if (D == 64) {
     cudaFuncSetAttribute(ptc::k_probe_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     ptc::k_probe_tc<64><<<grid, ptc::NT, sm, st>>>((const __nv_bfloat16*)Q, tmk, tmv, N, Gk, Gq, P, probe_idx,
-                                                   probe_grp, label_k, route, kps, scale_log2, part_o, part_ml, err);
+                                                   probe_grp, label_k, route, kps, scale_log2, cz.frame_id, cz.fend,
+                                                   cz.F, part_o, part_ml, err);
   } else {
     cudaFuncSetAttribute(ptc::k_probe_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     ptc::k_probe_tc<128><<<grid, ptc::NT, sm, st>>>((const __nv_bfloat16*)Q, tmk, tmv, N, Gk, Gq, P, probe_idx,
-                                                    probe_grp, label_k, route, kps, scale_log2, part_o, part_ml, err);
+                                                    probe_grp, label_k, route, kps, scale_log2, cz.frame_id, cz.fend,
+                                                    cz.F, part_o, part_ml, err);
   }
   return cudaGetLastError();
 }

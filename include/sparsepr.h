@@ -32,7 +32,9 @@
  *    the host before anything is enqueued and return SPARSEPR_EINVAL or
  *    SPARSEPR_EUNSUPPORTED; a failed launch returns SPARSEPR_ECUDA.  Device-side
  *    checks (bounded waits, index checks) record an error code in the workspace;
- *    read it with sparsepr_workspace_error() after the stream has drained.
+ *    read it with sparsepr_workspace_error() after the stream has drained.  Codes:
+ *    1 index out of range, 2 bounded wait ran out, 3 random-draw map overflow,
+ *    4 non-finite value, 5 frame ids out of range or decreasing.
  *  - Determinism: for fixed inputs, params and seed every output is bitwise
  *    reproducible (no floating-point atomics on any output path).
  *  - Random draws (query sample, k-means seeds, probe rows) use SplitMix64
@@ -84,7 +86,14 @@ typedef struct {
   float ridge_lambda;      /* ridge penalty, absolute (> 0; default 1e-2)                           */
   float scale;             /* softmax scale; 0 means 1/sqrt(d)                                      */
   unsigned long long seed; /* seed of the SplitMix64 streams                                        */
-  const int* frame_id;     /* must be NULL (frame-causal masking is not built)                      */
+  const int* frame_id;     /* NULL, or device int32 [N]: frame of each token (shared by all b, h);
+                              then query q sees key k only if frame_id[k] <= frame_id[q]
+                              (frame-causal, intersected with the route; the cell mass, cell cost
+                              and budget count visible pairs only).  Ids must be nondecreasing in
+                              token order (frame-major flattening of a video latent) and lie in
+                              [0, n_frames); a violation is recorded as device error 5 and leaves
+                              the outputs unspecified.  Needs N <= 65535 (32-bit cell costs).     */
+  int n_frames;            /* with frame_id: number of frames, 1..64; ignored without frame_id     */
 } sparsepr_params;
 
 /* Optional debug copies of partition intermediates (any pointer may be NULL). */
@@ -128,7 +137,8 @@ SPARSEPR_API sparsepr_status sparsepr_validate(const sparsepr_params* p);
  *   qoff/koff  int32 [BH, G+1]   first permuted position of each group
  *   route      uint8 [BH, G_q, G_k]  1 = cell executed
  *   block_mask uint8 [BH, T, T]  T = ceil(N/block); tile (i, j) of the permuted layout holds a routed pair
- *   rho_exec   float [BH]        realized (routed pairs + P*N) / N^2
+ *   rho_exec   float [BH]        realized (routed pairs + P*N) / N^2; frame-causal: (routed visible
+ *                                pairs + P*V/N) / V with V the visible pairs of the causal mask
  *   trace      optional, may be NULL                                                   */
 SPARSEPR_API sparsepr_status sparsepr_partition(const sparsepr_params* p, const void* Q, const void* K,
                                    int* perm_q, int* perm_k, int* label_q, int* label_k,
@@ -214,8 +224,10 @@ SPARSEPR_API sparsepr_status sparsepr_forward_host(const sparsepr_params* p, con
                                       void* workspace, size_t ws_bytes, void* stream);
 
 /* Dense softmax attention on the same machinery (the comparator for the sparse call):
- * O = softmax(s Q K^T) V (bf16 [B,H,N,d]), lse float [BH, N] (may be NULL).  Uses only
- * the workspace's error word (any workspace of sparsepr_workspace_bytes(p) bytes).    */
+ * O = softmax(s Q K^T) V (bf16 [B,H,N,d]), lse float [BH, N] (may be NULL); with frame ids,
+ * each query attends to the keys of its own and earlier frames.  Uses only the first bytes
+ * of the workspace: the error word (256 bytes; the workspace may then be NULL) and, with
+ * frame ids, the frame ends (512 bytes in all, required).                              */
 SPARSEPR_API sparsepr_status sparsepr_dense_attention(const sparsepr_params* p, const void* Q,
                                          const void* K, const void* V, void* O, float* lse,
                                          void* workspace, size_t ws_bytes, void* stream);

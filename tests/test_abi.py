@@ -50,6 +50,7 @@ int main(void) {
   printf("size %zu\n", sizeof(sparsepr_params));
   F(sparsepr_params, density) F(sparsepr_params, n_kgroups) F(sparsepr_params, kmeans_iters)
   F(sparsepr_params, ridge_lambda) F(sparsepr_params, scale) F(sparsepr_params, seed) F(sparsepr_params, frame_id)
+  F(sparsepr_params, n_frames)
   printf("ptrace %zu\n", sizeof(sparsepr_partition_trace));
   printf("prtrace %zu\n", sizeof(sparsepr_probe_trace));
   return 0;
@@ -63,7 +64,7 @@ int main(void) {
         out = dict(line.split() for line in subprocess.check_output([exe], text=True).splitlines())
     P = spr.Params
     assert int(out["size"]) == ctypes.sizeof(P)
-    for f in ("density", "n_kgroups", "kmeans_iters", "ridge_lambda", "scale", "seed", "frame_id"):
+    for f in ("density", "n_kgroups", "kmeans_iters", "ridge_lambda", "scale", "seed", "frame_id", "n_frames"):
         assert int(out[f]) == getattr(P, f).offset, f
     assert int(out["ptrace"]) == ctypes.sizeof(spr.PartitionTrace)
     assert int(out["prtrace"]) == ctypes.sizeof(spr.ProbeTrace)
@@ -94,6 +95,20 @@ def test_validation(spr, kw, status):
     p = _params(spr, **kw)
     assert spr.sparsepr_validate(p) == status
     assert (spr.sparsepr_workspace_bytes(p) > 0) == (status == 0)
+
+
+@pytest.mark.parametrize("n_frames,N,status", [(4, 1024, 0), (64, 1024, 0), (0, 1024, 1), (65, 1024, 1),
+                                               (4, 70000, 2)])
+def test_validation_frames(spr, n_frames, N, status):
+    """Frame-causal params: 1..64 frames, N <= 65535 (the pointer is never dereferenced)."""
+    p = _params(spr, N=N)
+    p.frame_id = 1 << 20
+    p.n_frames = n_frames
+    assert spr.sparsepr_validate(p) == status
+    if status == 0:
+        plain = _params(spr, N=N)
+        # the causal key streams (one per query group) make the workspace larger
+        assert spr.sparsepr_workspace_bytes(p) > spr.sparsepr_workspace_bytes(plain)
 
 
 def test_calls_reject_before_cuda(spr):

@@ -41,9 +41,21 @@ def _np(t):
         else t.detach().cpu().numpy()
 
 
-def stage_checks(pd, qb, kb, vb, out, heads, rows=None, check_kmeans=True):
+def _lse_close(got, ref, tol):
+    """LSE parity; a row with no usable key (frame-causal) must be -inf on both sides."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    np.testing.assert_array_equal(np.isneginf(got), np.isneginf(ref))
+    fin = np.isfinite(ref)
+    assert np.isfinite(got[fin]).all()
+    if fin.any():
+        assert np.abs(got[fin] - ref[fin]).max() <= tol * max(1.0, np.abs(ref[fin]).max())
+
+
+def stage_checks(pd, qb, kb, vb, out, heads, rows=None, check_kmeans=True, frames=None):
     """Per-stage parity of heads `heads` (flattened b*H + h).  rows: number of sampled
-    query rows for the attention / reconstruction checks (None = all)."""
+    query rows for the attention / reconstruction checks (None = all).  frames: frame of
+    each token for a frame-causal call (None = no mask)."""
     op = oracle_params(pd)
     B, H, N, d = pd["B"], pd["H"], pd["N"], pd["d"]
     s = op.eff_scale(d)
@@ -108,9 +120,18 @@ def stage_checks(pd, qb, kb, vb, out, heads, rows=None, check_kmeans=True):
         n_q = np.diff(qo)
         # --- a9: cell mass and route (route bit-exact given the device's fp32 masses)
         m_gpu = _np(tr["cell_mass"][bh]).astype(np.float64)
-        m_ref = O.cell_mass(z_gpu, lq, n_k, pd["n_qgroups"])
+        if frames is None:
+            m_ref = O.cell_mass(z_gpu, lq, n_k, pd["n_qgroups"])
+            cost = visible = None
+        else:
+            nf = int(frames.max()) + 1
+            vis_k = O.visible_counts(lk, frames, pd["n_kgroups"], nf)
+            hist_q = O.frame_histogram(lq, frames, pd["n_qgroups"], nf)
+            m_ref = O.cell_mass(z_gpu, lq, n_k, pd["n_qgroups"], frames, vis_k)
+            cost = O.cell_cost(n_q, n_k, hist_q, vis_k)
+            visible = float(hist_q.sum(axis=0) @ vis_k.sum(axis=0))
         assert np.abs(m_gpu - m_ref).max() <= 2e-5
-        rr = O.route_select(m_gpu, n_q, n_k, op.density, pd["n_probes"], N)
+        rr = O.route_select(m_gpu, n_q, n_k, op.density, pd["n_probes"], N, cost=cost, visible=visible)
         route = _np(out["route"][bh])
         np.testing.assert_array_equal(route, rr.route)
         assert _np(tr["alpha"])[bh] == rr.alpha
@@ -119,21 +140,23 @@ def stage_checks(pd, qb, kb, vb, out, heads, rows=None, check_kmeans=True):
         np.testing.assert_array_equal(_np(out["block_mask"][bh]), bm)
         # --- a11: routed attention (sampled rows, original order)
         sel = np.arange(N) if rows is None or rows >= N else np.sort(rng.choice(N, rows, replace=False))
-        o_ref, l_ref = O.sparse_attention(q, k, v, s, rr.route, lq, lk, rows=sel)
+        o_ref, l_ref = O.sparse_attention(q, k, v, s, rr.route, lq, lk, rows=sel, frames=frames)
         o_gpu = _np(out["o_sparse"][b, h])[sel].astype(np.float64)
         l_gpu = _np(out["lse"][bh])[sel].astype(np.float64)
         assert rel_l2(o_gpu, o_ref) <= OS_REL_L2, rel_l2(o_gpu, o_ref)
         assert np.abs(o_gpu - o_ref).max() <= OS_MAX_ABS
-        assert np.abs(l_gpu - l_ref).max() <= 2e-3 * max(1.0, np.abs(l_ref).max())
+        _lse_close(l_gpu, l_ref, 2e-3)
         # --- a12/a13: probes
         pidx = O.pick_probes(pq, qo, pd["n_probes"], pd["seed"], bh)
         np.testing.assert_array_equal(_np(out["probe_idx"][bh]), pidx)
-        od_ref, ld_ref = O.attention(q[pidx], k, v, s)
-        os_ref, ls_ref = O.sparse_attention(q, k, v, s, rr.route, lq, lk, rows=pidx)
+        od_ref, ld_ref = O.attention(q[pidx], k, v, s,
+                                     mask=None if frames is None else O.causal_mask(frames, pidx))
+        os_ref, ls_ref = O.sparse_attention(q, k, v, s, rr.route, lq, lk, rows=pidx, frames=frames)
         od_gpu = _np(out["probe_o_dense"][bh]).astype(np.float64)
         os_gpu = _np(ptr["probe_o_sparse"][bh]).astype(np.float64)
         assert rel_l2(od_gpu, od_ref) <= 1e-5 and rel_l2(os_gpu, os_ref) <= 1e-5
-        assert np.abs(_np(ptr["probe_lse_dense"][bh]) - ld_ref).max() <= 1e-4 * max(1, np.abs(ld_ref).max())
+        _lse_close(_np(ptr["probe_lse_dense"][bh]), ld_ref, 1e-4)
+        _lse_close(_np(ptr["probe_lse_sparse"][bh]), ls_ref, 1e-4)
         # --- a14/a15: subspace + ridge (basis-free quantities: B = W V_r^T, b V_r^T)
         fit = O.fit_from_probes(pidx, od_ref, os_ref, ld_ref, ls_ref, pd["sub_rank"], op.ridge_lambda)
         b_gpu = _np(out["b_full"][bh]).astype(np.float64)
