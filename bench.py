@@ -5,6 +5,12 @@ reconstruct) over the 32,760-token, 40-head, d=128 video-shaped workload at 25%
 executed-pair density, inputs resident in HBM.  Prints one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload wan|world]
+
+--workload world times the world-model rollout instead: B=4, H=16, 16 frames of
+32x32 tokens, d=128, a frame-causal mask intersected with the route, and one step
+= 8 consecutive calls on inputs perturbed by N(0, 0.05^2) per call (a random walk),
+each call re-partitioned and re-fitted; the value is ms per call.
 
 --gpus N > 1 runs under torchrun, one rank per GPU, each rank an independent call
 on its own inputs (the heads shard with no data-path collective: weak scaling).
@@ -26,6 +32,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD = "wan"
+ROLLOUT_CALLS = 8        # calls per step of the world-model rollout
+ROLLOUT_SIGMA = 0.05     # per-call perturbation of Q, K, V
 METRIC = "ms/attention call & executed TFLOP/s (frac of BF16 peak) at 25% density; rel-L2"
 UNIT = "ms/call"
 
@@ -41,12 +49,19 @@ def _peaks():
 
 
 def _config(w, extra=None):
-    c = {"workload": f"{w.name}-shaped video tokens {w.grid[0]}x{w.grid[1]}x{w.grid[2]}",
+    name = (f"world-model rollout, {w.grid[0]}x{w.grid[1]}x{w.grid[2]} video tokens, frame-causal, "
+            f"{ROLLOUT_CALLS} perturbed calls per step" if w.frame_causal else
+            f"{w.name}-shaped video tokens {w.grid[0]}x{w.grid[1]}x{w.grid[2]}")
+    c = {"workload": name,
          "global_batch": w.B, "seq_len": w.N, "heads": w.H, "head_dim": w.d, "density": w.density,
          "k_groups": w.n_kgroups, "q_groups": w.n_qgroups, "probes_per_head": w.n_probes,
          "subspace_rank": w.sub_rank, "kmeans_iters": w.kmeans_iters,
          "parallelism": "independent calls per rank (heads shard, no collective)",
-         "l2": "inputs larger than L2 (Q,K,V = 1.0 GB per call), no flush"}
+         "l2": f"inputs larger than L2 (Q,K,V = {3 * w.B * w.H * w.N * w.d * 2 / 1e9:.2f} GB per call), no flush"}
+    if w.frame_causal:
+        c.update({"frames": w.grid[0], "mask": "frame-causal (key frame <= query frame) intersected with the route",
+                  "rollout_calls_per_step": ROLLOUT_CALLS,
+                  "perturbation": f"N(0, {ROLLOUT_SIGMA}^2) added to Q, K, V before each call (random walk)"})
     if extra:
         c.update(extra)
     return c
@@ -153,14 +168,24 @@ def run_cuda(args):
     import free_block_sparse_rcp_b200 as spr
     from synth import generate, workload
 
-    w = workload(WORKLOAD, H=args.heads) if args.heads else workload(WORKLOAD)
+    w = workload(args.workload, H=args.heads) if args.heads else workload(args.workload)
     pd = dict(B=w.B, H=w.H, N=w.N, d=w.d, block=w.block, density=w.density, n_kgroups=w.n_kgroups,
               n_qgroups=w.n_qgroups, n_samples=w.n_samples, n_probes=w.n_probes, eig_rank=w.eig_rank,
               sub_rank=w.sub_rank, kmeans_iters=w.kmeans_iters, ridge_lambda=w.ridge_lambda, seed=0)
-    p = spr.Params.make(**pd)
+    from synth import frame_index, perturb, to_torch
+    frames = frame_index(w.grid) if w.frame_causal else None
+    fid = torch.from_numpy(frames).to(dev) if w.frame_causal else None
+    p = spr.Params.make(**pd, frame_id=fid, n_frames=w.grid[0] if w.frame_causal else 0)
     qb, kb, vb = generate(w, seed=rank)
-    from synth import to_torch
-    Q, K, V = (to_torch(x, dev) for x in (qb, kb, vb))
+    # one input triple per call of a step (the rollout perturbs Q, K, V before every call)
+    calls = ROLLOUT_CALLS if w.frame_causal else 1
+    inputs = []
+    for c in range(calls):
+        if c > 0:
+            qb, kb, vb = (perturb(x, ROLLOUT_SIGMA, 1000 * rank + j, c) for j, x in enumerate((qb, kb, vb)))
+        inputs.append(tuple(to_torch(x, dev) for x in (qb, kb, vb)))
+    del qb, kb, vb
+    Q, K, V = inputs[-1]
     BH, N, d = p.BH, p.N, p.d
     wsb = spr.workspace(p, dev)
     part = spr.alloc_partition(p, dev)
@@ -172,7 +197,11 @@ def run_cuda(args):
 
     launches = [0]
 
-    def step(ev=None):
+    def step(evs_step=None):
+        for c, (Qc, Kc, Vc) in enumerate(inputs):
+            call(Qc, Kc, Vc, None if evs_step is None else evs_step[c])
+
+    def call(Q, K, V, ev=None):
         n = 0
         if ev is not None:
             ev[0].record(stream)
@@ -203,7 +232,8 @@ def run_cuda(args):
     torch.cuda.synchronize()
     assert spr.sparsepr_workspace_error(p, wsb) == 0
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(calls)]
+           for _ in range(args.steps)]
     launches[0] = 0
     if ws > 1:
         torch.distributed.barrier()
@@ -214,26 +244,28 @@ def run_cuda(args):
         torch.cuda.synchronize()
     if ws > 1:
         torch.distributed.barrier()
-    stage = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(args.steps)]
-    total_ms = sum(evs[i][0].elapsed_time(evs[i][4]) for i in range(args.steps))
+    stage = [[evs[i][c][j].elapsed_time(evs[i][c][j + 1]) for j in range(4)]
+             for i in range(args.steps) for c in range(calls)]
+    total_ms = sum(evs[i][0][0].elapsed_time(evs[i][calls - 1][4]) for i in range(args.steps))
     total_ms = max_over_ranks(total_ms, ws, dev)
     ms_per_step = total_ms / args.steps
-    value = job_ms_per_call(total_ms, args.steps, ws)
+    value = job_ms_per_call(total_ms, args.steps * calls, ws)
+    ms_per_call = ms_per_step / calls
     stage_ms = [statistics.mean(s[j] for s in stage) for j in range(4)]
 
-    # --- algorithmic work of the attention kernel (useful routed pairs)
-    nq = torch.diff(part["qoff"].long(), dim=1)
-    nk = torch.diff(part["koff"].long(), dim=1)
-    routed_pairs = int((nq[:, :, None] * nk[:, None, :] * part["route"].long()).sum().item())
-    # MMA-issued pairs: q-tiles of 128 rows x routed key rows padded to 128-key chunks
-    ntile = (nq + 127) // 128
-    rk = (nk[:, None, :] * part["route"].long()).sum(-1)
-    issued_pairs = int((ntile * 128 * ((rk + 127) // 128) * 128).sum().item())
+    # --- algorithmic work of the attention kernel of the last call (useful routed pairs)
+    routed_pairs, issued_pairs = attention_pairs(part, frames)
     attn_flops = 4.0 * d * routed_pairs
     attn_ms = stage_ms[1]
     pk = _peaks()
     achieved = attn_flops / (attn_ms * 1e-3) / 1e12
-    dense_flops = 4.0 * d * N * N * BH
+    # dense comparator work: every (frame-causal: every visible) pair
+    if frames is None:
+        dense_pairs = N * N
+    else:
+        per_frame = np.bincount(frames, minlength=w.grid[0]).astype(np.int64)
+        dense_pairs = int((per_frame * np.cumsum(per_frame)).sum())
+    dense_flops = 4.0 * d * dense_pairs * BH
 
     # --- dense comparator on the same machinery
     o_dense = torch.empty_like(Q)
@@ -279,7 +311,7 @@ def run_cuda(args):
     e2e_value = e2e_total / (e2e_steps * ws)
     bytes_in = 3 * BH * N * d * 2
 
-    traffic = _traffic_record("attend")
+    traffic = _traffic_record("attend_causal" if w.frame_causal else "attend")
     rho = part["rho_exec"].float()
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
@@ -289,13 +321,13 @@ def run_cuda(args):
         "stage_ms": {"partition": round(stage_ms[0], 4), "attend": round(stage_ms[1], 4),
                      "probe_fit": round(stage_ms[2], 4), "reconstruct": round(stage_ms[3], 4)},
         "dense_attention_ms": round(dense_ms, 4),
-        "speedup_vs_dense": round(dense_ms / ms_per_step, 3),
+        "speedup_vs_dense": round(dense_ms / ms_per_call, 3),
         "rho_exec": {"mean": round(float(rho.mean()), 5), "min": round(float(rho.min()), 5),
                      "max": round(float(rho.max()), 5)},
         "attend_tflops_useful": round(achieved, 2),
         "attend_tflops_issued": round(4.0 * d * issued_pairs / (attn_ms * 1e-3) / 1e12, 2),
         "tile_fill": round(routed_pairs / max(1, issued_pairs), 4),
-        "dense_equiv_tflops": round(dense_flops / (ms_per_step * 1e-3) / 1e12, 2),
+        "dense_equiv_tflops": round(dense_flops / (ms_per_call * 1e-3) / 1e12, 2),
         "dense_kernel_tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 2),
         "rel_l2_vs_dense": {"o_sparse": round(err_sparse, 5), "o_reconstructed": round(err_recon, 5)},
         "roofline": {"kernel": "attend (routed flash attention)", "bound": "tensor", "achieved": round(achieved, 2),
@@ -308,14 +340,56 @@ def run_cuda(args):
         "gpu_launches": launches[0],
         "clocks": clk.summary(),
     }
+    if calls > 1:
+        line["ms_per_call"] = round(ms_per_call, 4)
     if rank == 0 and ws == 1 and not args.heads:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_budget)
+        line["cpu_baseline"] = cpu_baseline(w)
     if ws > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def attention_pairs(part, frames=None):
+    """(useful, MMA-issued) query-key pairs of the routed attention of the last call.
+
+    useful: routed pairs (frame-causal: routed pairs whose key frame <= query frame).
+    issued: per 256-row unit of a query group, its 128-row q-tiles times the 128-key
+    chunks of the key stream it walks: all routed keys of the group, or (frame-causal)
+    the routed keys of frames <= the unit's last row frame."""
+    import numpy as np
+    qoff = part["qoff"].long().cpu().numpy()
+    koff = part["koff"].long().cpu().numpy()
+    route = part["route"].long().cpu().numpy()
+    nq, nk = np.diff(qoff, axis=1), np.diff(koff, axis=1)
+    if frames is None:
+        useful = int((nq[:, :, None] * nk[:, None, :] * route).sum())
+        ntile = (nq + 127) // 128
+        rk = (nk[:, None, :] * route).sum(-1)
+        return useful, int((ntile * 128 * ((rk + 127) // 128) * 128).sum())
+    label_q = part["label_q"].long().cpu().numpy()
+    label_k = part["label_k"].long().cpu().numpy()
+    perm_q = part["perm_q"].long().cpu().numpy()
+    fr = np.asarray(frames, np.int64)
+    F = int(fr.max()) + 1
+    Gq, Gk = route.shape[1], route.shape[2]
+    useful = issued = 0
+    for bh in range(route.shape[0]):
+        hist_q = np.zeros((Gq, F), np.int64)
+        np.add.at(hist_q, (label_q[bh], fr), 1)
+        vis_k = np.zeros((Gk, F), np.int64)
+        np.add.at(vis_k, (label_k[bh], fr), 1)
+        vis_k = np.cumsum(vis_k, axis=1)
+        useful += int(((hist_q @ vis_k.T) * route[bh]).sum())
+        tl = route[bh] @ vis_k                      # [Gq, F] stream prefix per frame
+        for a in range(Gq):
+            for u0 in range(qoff[bh, a], qoff[bh, a + 1], 256):
+                rows = min(256, qoff[bh, a + 1] - u0)
+                f_last = fr[perm_q[bh, u0 + rows - 1]]
+                issued += ((rows + 127) // 128) * 128 * ((int(tl[a, f_last]) + 127) // 128) * 128
+    return useful, issued
 
 
 def _traffic_record(kernel: str):
@@ -346,14 +420,17 @@ def oracle_sample(w, rows_frac=1 / 32, seed=0):
                  eig_rank=w.eig_rank, sub_rank=w.sub_rank, kmeans_iters=w.kmeans_iters, density=w.density,
                  ridge_lambda=w.ridge_lambda, seed=0, block=w.block)
     s = p.eff_scale(w.d)
+    from synth import frame_index
+    fr = frame_index(w.grid).astype(np.int64) if w.frame_causal else None
     t0 = time.perf_counter()
-    part = O.partition_head(q, k, p, 0)
+    part = O.partition_head(q, k, p, 0, frames=fr)
     t1 = time.perf_counter()
     n_rows = max(1, int(w.N * rows_frac))
     rows = np.arange(0, w.N, w.N // n_rows)[:n_rows]
-    o_s, _ = O.sparse_attention(q, k, v, s, part.route.route, part.label_q, part.label_k, rows=rows)
+    o_s, _ = O.sparse_attention(q, k, v, s, part.route.route, part.label_q, part.label_k, rows=rows, frames=fr)
     t2 = time.perf_counter()
-    fit = O.probe_fit_head(q, k, v, part.label_q, part.label_k, part.route.route, part.perm_q, part.q_offsets, p, 0)
+    fit = O.probe_fit_head(q, k, v, part.label_q, part.label_k, part.route.route, part.perm_q, part.q_offsets, p, 0,
+                           frames=fr)
     t3 = time.perf_counter()
     _ = o_s + fit.b_full + (o_s @ fit.w) @ fit.vr.T
     t4 = time.perf_counter()
@@ -370,9 +447,7 @@ def _cores():
         return os.cpu_count()
 
 
-def cpu_baseline(budget_s=30.0):
-    from synth import workload
-    w = workload(WORKLOAD)
+def cpu_baseline(w):
     sec, spent, nrows = oracle_sample(w)
     return {"value": round(sec * 1e3, 1), "unit": UNIT, "cores": _cores(), "kind": "oracle",
             "sample": f"head (0,0) of {w.B * w.H}: full partition, probes and fit; routed attention and "
@@ -385,7 +460,7 @@ def run_reference(args):
     if rank != 0:
         return
     from synth import workload
-    w = workload(WORKLOAD)
+    w = workload(args.workload)
     for _ in range(args.warmup):
         oracle_sample(workload("tiny"), rows_frac=1.0)   # warms numpy / BLAS; not timed
     vals, spent = [], 0.0
@@ -413,7 +488,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--cpu-budget", type=float, default=30.0)
+    ap.add_argument("--workload", default=WORKLOAD, choices=["wan", "world"],
+                    help="wan: the 32,760-token call (default); world: the frame-causal rollout")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (small cases for ncu captures; default: the workload's 40)")
     args = ap.parse_args()

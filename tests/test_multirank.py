@@ -73,3 +73,32 @@ def test_reference_arm_other_ranks_do_no_work(monkeypatch, capsys):
         steps, warmup = 2, 3
     bench.run_reference(A())
     assert called == [] and capsys.readouterr().out == ""
+
+
+def test_attention_pairs_counts_visible_routed_pairs():
+    """bench.attention_pairs: the useful pairs are the routed (and, frame-causal,
+    visible) token pairs counted one by one; the issued pairs cover them."""
+    import numpy as np
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench
+    rng = np.random.default_rng(0)
+    BH, N, Gq, Gk, F = 2, 300, 5, 7, 4
+    frames = np.repeat(np.arange(F), N // F)
+    lq = rng.integers(0, Gq, (BH, N))
+    lk = rng.integers(0, Gk, (BH, N))
+    route = (rng.random((BH, Gq, Gk)) < 0.4).astype(np.uint8)
+    part = {"label_q": torch.from_numpy(lq), "label_k": torch.from_numpy(lk), "route": torch.from_numpy(route),
+            "perm_q": torch.from_numpy(np.argsort(lq, axis=1, kind="stable")),
+            "qoff": torch.from_numpy(np.stack([np.r_[0, np.cumsum(np.bincount(x, minlength=Gq))] for x in lq])),
+            "koff": torch.from_numpy(np.stack([np.r_[0, np.cumsum(np.bincount(x, minlength=Gk))] for x in lk]))}
+    for fr in (None, frames):
+        useful, issued = bench.attention_pairs(part, fr)
+        want = 0
+        for bh in range(BH):
+            m = route[bh][lq[bh]][:, lk[bh]].astype(bool)
+            if fr is not None:
+                m &= fr[None, :] <= fr[:, None]
+            want += int(m.sum())
+        assert useful == want
+        assert issued >= useful and issued % (128 * 128) == 0
