@@ -27,8 +27,9 @@
 // columns of P_t,j only after PV_t,j (tcgen05 MMAs of one thread execute in issue order),
 // and when S_t,j+1 is complete so is PV_t,j, so the softmax may rescale O_t in place.
 // The softmax makes one speculative pass per chunk against the running max (exponentials
-// and the chunk max together, packed fp32x2 arithmetic) and keeps it unless some row's max
-// grew by more than 2^8; then the chunk is redone against the new max and O is rescaled.
+// and their row sum, packed fp32x2 arithmetic) and keeps it while the chunk's row sum stays
+// within 2^8 (so no probability exceeds 2^8); otherwise the chunk is redone against its
+// own max and O is rescaled.
 // Frame-causal variant (CAUSAL): a query of frame f sees only keys of frames <= f.  The
 // key stream is then ordered so that the keys a frame-f row may use are a prefix of it:
 // dense, the token order itself (frame ids are nondecreasing), prefix fend[f]; routed, the
@@ -64,7 +65,7 @@ struct Roles {
   static constexpr uint32_t kLoadArrivals = DENSE ? 1 : NPROD_G;   // arrivals per q / K / V stage
 };
 constexpr uint32_t TMEM_COLS = 512;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kSpecSumBound = 256.0f;    // 2^8: largest row sum a speculative chunk may reach
 
 struct Bars {
   uint64_t q, kfull[KST], kempty[KST], vfull[VST], vempty[VST], s_full[TPC], p_full[TPC], o_done[TPC], mma_done;
@@ -113,7 +114,8 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
   Bars* bars = reinterpret_cast<Bars*>(smem + L::oBar);
   int* ints = reinterpret_cast<int*>(smem + L::oInt);
   int* sQrow = ints;                  // [TPC * BM]
-  int* sMisc = sQrow + TPC * BM;      // [0] tmem base, [1] abort, [2] total, [3] cnt, [4] slot ok
+  // [0] tmem base, [1] abort, [2] total, [3] cnt, [4] slot ok, [5] chunks of tile 0 (causal)
+  int* sMisc = sQrow + TPC * BM;
   int* sList = sMisc + 8;             // [Gk]
   int* sKoffL = sList + Gk;           // [Gk]
   int* sCum = sKoffL + Gk;            // [Gk + 1]
@@ -152,11 +154,16 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
     return f < 0 ? 0 : (f >= F ? F - 1 : f);
   };
   if (CAUSAL && tid == 0) {
-    // the unit streams the prefix of its last (latest-frame) row
-    int tot = 0;
-    if (qn > 0) tot = frame_lim[frame_of(DENSE ? q0 + qn - 1 : perm_q[head + q0 + qn - 1])];
-    sMisc[2] = tot < 0 ? 0 : (tot > N ? N : tot);
+    // the unit streams the prefix of its last (latest-frame) row; tile 0 stops at the
+    // prefix of its own last row
+    auto prefix_of = [&](int i) -> int {   // stream prefix of the frame of unit row i
+      const int t = frame_lim[frame_of(DENSE ? q0 + i : perm_q[head + q0 + i])];
+      return t < 0 ? 0 : (t > N ? N : t);
+    };
+    const int tot = qn > 0 ? prefix_of(qn - 1) : 0;
+    sMisc[2] = tot;
     sMisc[3] = 0;
+    sMisc[5] = qn > BM ? min((prefix_of(BM - 1) + BN - 1) / BN, (tot + BN - 1) / BN) : (tot + BN - 1) / BN;
   }
   if (DENSE && !CAUSAL && tid == 0) { sMisc[2] = N; sMisc[3] = 0; }
   if (tid < TPC * BM) {
@@ -198,6 +205,10 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
   const int total = sMisc[2];
   const int cnt = sMisc[3];
   const int nchunks = (total + BN - 1) / BN;
+  // chunks tile t walks: all (the last tile always walks every chunk), or fewer for tile 0
+  // of a frame-causal unit, whose rows end in an earlier frame
+  const int nch0 = CAUSAL ? sMisc[5] : nchunks;
+  auto nch = [&](int t) -> int { return (CAUSAL && t == 0) ? nch0 : nchunks; };
   const uint32_t sQ = base + L::oQ, sK = base + L::oK, sV = base + L::oV;
 
   auto wait = [&](uint64_t& bar, uint32_t parity) -> bool {
@@ -311,10 +322,12 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
       constexpr uint32_t IDS = idesc_bf16(128, BN, false);
       constexpr uint32_t IDO = idesc_bf16(128, D, true);
       bool ok = nchunks == 0 || wait(bars->q, 0);
+      // the first tile that uses chunk j waits for its K / V stage
+      auto first_user = [&](int j) -> int { return j < nch(0) ? 0 : 1; };
       // S_t,j = Q_t K_j^T into the S columns of tile t; the last tile releases K_j
       auto issue_s = [&](int t, int j) -> bool {
         const int ks = j % KST;
-        if (t == 0) {
+        if (t == first_user(j)) {
           if (!wait(bars->kfull[ks], (j / KST) & 1)) return false;
           tc_fence_after();
         }
@@ -332,7 +345,7 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
       auto issue_pv = [&](int t, int j) -> bool {
         const int vs = j % VST;
         if (!wait(bars->p_full[t], j & 1)) return false;
-        if (t == 0 && !wait(bars->vfull[vs], (j / VST) & 1)) return false;
+        if (t == first_user(j) && !wait(bars->vfull[vs], (j / VST) & 1)) return false;
         tc_fence_after();
         const uint32_t vb = sV + vs * L::kTile;
 #pragma unroll
@@ -342,14 +355,23 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
         if (t == ntile - 1) tc_commit(su32(&bars->vempty[vs]));
         return true;
       };
-      for (int t = 0; ok && t < ntile && nchunks > 0; ++t) ok = issue_s(t, 0);
+      for (int t = 0; ok && t < ntile; ++t)
+        if (nch(t) > 0) ok = issue_s(t, 0);
+      bool early0 = false;
       for (int j = 0; ok && j < nchunks; ++j) {
         for (int t = 0; ok && t < ntile; ++t) {
+          if (j >= nch(t)) continue;
           ok = issue_pv(t, j);
-          if (ok && j + 1 < nchunks) ok = issue_s(t, j + 1);
+          if (ok && j + 1 < nch(t)) ok = issue_s(t, j + 1);
+          // a tile whose walk ends before the unit's releases its epilogue early
+          if (ok && CAUSAL && t == 0 && ntile > 1 && j + 1 == nch(0)) {
+            tc_commit(su32(&bars->o_done[0]));
+            early0 = true;
+          }
         }
       }
-      for (int t = 0; t < ntile; ++t) tc_commit(su32(&bars->o_done[t]));
+      for (int t = 0; t < ntile; ++t)
+        if (!(t == 0 && early0)) tc_commit(su32(&bars->o_done[t]));
       // drain: every MMA issued above completes before the TMEM is released
       tc_commit(su32(&bars->mma_done));
       wait(bars->mma_done, 0);
@@ -368,25 +390,25 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
       const int row = sQrow[t * BM + r];
       if (row >= 0) lim = min(total, frame_lim[frame_of(row)]);
     }
+    const int nct = t < ntile ? nch(t) : 0;   // chunks this tile walks
     if (t < ntile) {
       uint32_t sreg[64];
       uint32_t pk[64];
       const uint64_t sc2 = f2pack(scale_log2, scale_log2);
-      for (int j = 0; j < nchunks; ++j) {
+      for (int j = 0; j < nct; ++j) {
         ok = __all_sync(0xffffffffu, wait(bars->s_full[t], j & 1));
         if (!ok) break;
         tc_fence_after();
         const int valid = lim - j * BN;
         const bool full = CAUSAL ? __all_sync(0xffffffffu, valid >= BN) : valid >= BN;
-        // Speculative single pass against the running max: P = exp2(S s log2e - m) and the
-        // chunk's max together; kept only if no row's max grew by more than the threshold.
+        // Speculative single pass against the running max: P = exp2(S s log2e - m) and its
+        // row sum; kept only if that sum stays within kSpecSumBound.
         bool need = true;
         float mx = -INFINITY;
         uint64_t rs2 = 0ull;
         const bool spec = __all_sync(0xffffffffu, m_used != -INFINITY);
         if (spec) {
           const uint64_t nmu2 = f2pack(-m_used, -m_used);
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             tc_ld32(tS + 32 * q, sreg);
@@ -397,7 +419,6 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
                 if (32 * q + c >= valid) s0 = -INFINITY;
                 if (32 * q + c + 1 >= valid) s1 = -INFINITY;
               }
-              m4[(c >> 1) & 3] = fmaxf(m4[(c >> 1) & 3], fmaxf(s0, s1));
               float x0, x1;
               f2unpack(ffma2(f2pack(s0, s1), sc2, nmu2), x0, x1);
               const float p0 = ex2(x0), p1 = ex2(x1);
@@ -405,8 +426,11 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
               pk[16 * q + (c >> 1)] = pack_bf16(p0, p1);
             }
           }
-          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-          need = mx * scale_log2 > m_used + kRescaleThreshold;
+          // kept iff the chunk's row sum stays <= 2^8, which bounds every element by 2^8
+          // (no per-element max is kept)
+          float r0, r1;
+          f2unpack(rs2, r0, r1);
+          need = !(r0 + r1 <= kSpecSumBound);
         }
         const bool warp_need = __any_sync(0xffffffffu, need);
         float alpha = 1.f;
@@ -418,8 +442,8 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
           f2unpack(rs2, r0, r1);
           l += r0 + r1;
         } else {
-          // slow path: the chunk's max (if not known yet), rescale O, then P against it
-          if (!spec) {
+          // slow path: the chunk's max, rescale O, then P against it
+          {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               tc_ld64(tS + 64 * h, sreg);
@@ -467,7 +491,7 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
       }
       // epilogue
       const int row = sQrow[t * BM + r];
-      if (ok && nchunks > 0) ok = __all_sync(0xffffffffu, wait(bars->o_done[t], 0));
+      if (ok && nct > 0) ok = __all_sync(0xffffffffu, wait(bars->o_done[t], 0));
       if (ok) {
         tc_fence_after();
         const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -475,7 +499,7 @@ __global__ void __launch_bounds__(Roles<DENSE>::NT, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          if (nchunks > 0) {
+          if (nct > 0) {
             tc_ld32(tO + c * 32, o);
           } else {
 #pragma unroll
