@@ -63,8 +63,8 @@ __global__ void __launch_bounds__(256) k_seed_rows(const __nv_bfloat16* __restri
 //         group keeps its centroid.  m is updated in place.
 // mode 2: as mode 1 but an empty group gets 0, the means are written to m and no weights
 //         are formed (the K/V group centroids after the last pass).
-// Weights, one warp per centroid: nu = A m (fp32, sequential over c), bias = ||nu||^2,
-//   w = A^T nu -> w_hi = bf16(w), w_lo = bf16(w - w_hi); wnorm = ||w||.
+// Weights, two centroids per warp: nu = A m (fp32, sequential over c), bias = ||nu||^2,
+//   w = A^T nu (sequential over j) -> w_hi = bf16(w), w_lo = bf16(w - w_hi); wnorm = ||w||.
 // Rows g in [G, GP) are padding: w = 0, bias = +inf.
 // grid = (ceil(GP / WG_PER_CTA), BH), block = 256.
 // ---------------------------------------------------------------------------
@@ -91,8 +91,8 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
   double* acc = reinterpret_cast<double*>(sw);               // [WG_PER_CTA][d]
   int* cnt = reinterpret_cast<int*>(acc + WG_PER_CTA * d);   // [WG_PER_CTA]
   float* sA = reinterpret_cast<float*>(cnt + WG_PER_CTA);    // [D][d + 1]
-  float* sm_m = sA + D * (d + 1);                            // [8][d]
-  float* sm_nu = sm_m + 8 * d;                               // [8][128]
+  float* sMg = sA + D * (d + 1);                             // [WG_PER_CTA][d] this CTA's centroids
+  float* sNu = sMg + WG_PER_CTA * d;                         // [WG_PER_CTA][128] their nu
   const int bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g0 = blockIdx.x * WG_PER_CTA, g1 = min(GP, g0 + WG_PER_CTA);
   if (mode != 0) {
@@ -165,11 +165,23 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
     sA[j * (d + 1) + c] = Ah[(size_t)j * sj + (size_t)c * sc];
   }
   __syncthreads();
-  float* wm = sm_m + warp * d;
-  float* wnu = sm_nu + warp * 128;
-  for (int g = g0 + warp; g < g1; g += CW_THREADS / 32) {
-    const size_t wrow = ((size_t)bh * GP + g) * d;
-    if (g >= G) {
+  for (int e = tid; e < WG_PER_CTA * d; e += CW_THREADS) {
+    const int gi = e / d, c = e - gi * d, g = g0 + gi;
+    sMg[e] = (g < g1 && g < G) ? m[((size_t)bh * G + g) * d + c] : 0.f;
+  }
+  __syncthreads();
+  // warp w forms the weights of groups g0 + w and g0 + w + 8 together; lanes split j for
+  // nu = A m and c for w = A^T nu, each sum in ascending order of its index
+  static_assert(WG_PER_CTA == 2 * (CW_THREADS / 32), "two groups per warp");
+  const int gl[2] = {warp, warp + 8};
+  bool live[2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int g = g0 + gl[u];
+    live[u] = g < g1 && g < G;
+    if (g < g1 && g >= G) {
+      // padding group: never the argmin
+      const size_t wrow = ((size_t)bh * GP + g) * d;
       for (int c = lane; c < d; c += 32) {
         w_hi[wrow + c] = __float2bfloat16(0.f);
         w_lo[wrow + c] = __float2bfloat16(0.f);
@@ -178,37 +190,86 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
         bias[(size_t)bh * GP + g] = __int_as_float(0x7f800000);
         wnorm[(size_t)bh * GP + g] = 0.f;
       }
-      continue;
     }
-    for (int c = lane; c < d; c += 32) wm[c] = m[((size_t)bh * G + g) * d + c];
-    __syncwarp();
+  }
+  if (!live[0] && !live[1]) return;
+  float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  {
+    const float* m0 = sMg + gl[0] * d;
+    const float* m1 = sMg + gl[1] * d;
+    for (int c = 0; c < d; ++c) {
+      const float x0 = m0[c], x1 = m1[c];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int j = lane + 32 * k;
+        if (j < D) {
+          const float a = sA[j * (d + 1) + c];
+          acc2[0][k] = fmaf(a, x0, acc2[0][k]);
+          acc2[1][k] = fmaf(a, x1, acc2[1][k]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int g = g0 + gl[u];
     float b2 = 0.f;
-    for (int j = lane; j < D; j += 32) {
-      float a = 0.f;
-      for (int c = 0; c < d; ++c) a = fmaf(sA[j * (d + 1) + c], wm[c], a);
-      a *= a_scale;
-      wnu[j] = a;
-      b2 = fmaf(a, a, b2);
-    }
-    __syncwarp();
-    for (int j = lane; j < DT; j += 32) nu[((size_t)bh * G + g) * DT + j] = j < D ? wnu[j] : 0.f;
-    float n2 = 0.f;
-    for (int c = lane; c < d; c += 32) {
-      float a = 0.f;
-      for (int j = 0; j < D; ++j) a = fmaf(sA[j * (d + 1) + c], wnu[j], a);
-      const float w = a_scale * a;
-      n2 = fmaf(w, w, n2);
-      const __nv_bfloat16 hi = __float2bfloat16(w);
-      w_hi[wrow + c] = hi;
-      w_lo[wrow + c] = __float2bfloat16(w - __bfloat162float(hi));
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int j = lane + 32 * k;
+      if (j < D) {
+        const float a = acc2[u][k] * a_scale;
+        sNu[gl[u] * 128 + j] = a;
+        b2 = fmaf(a, a, b2);
+      }
     }
     b2 = warp_sum(b2);
-    n2 = warp_sum(n2);
-    if (lane == 0) {
-      bias[(size_t)bh * GP + g] = b2;
-      wnorm[(size_t)bh * GP + g] = sqrtf(n2);
+    if (live[u]) {
+      for (int j = lane; j < DT; j += 32) nu[((size_t)bh * G + g) * DT + j] = j < D ? sNu[gl[u] * 128 + j] : 0.f;
+      if (lane == 0) bias[(size_t)bh * GP + g] = b2;
     }
-    __syncwarp();
+  }
+  __syncwarp();
+#pragma unroll
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc2[u][k] = 0.f;
+  {
+    const float* n0 = sNu + gl[0] * 128;
+    const float* n1 = sNu + gl[1] * 128;
+    for (int j = 0; j < D; ++j) {
+      const float y0 = n0[j], y1 = n1[j];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = lane + 32 * k;
+        if (c < d) {
+          const float a = sA[j * (d + 1) + c];
+          acc2[0][k] = fmaf(a, y0, acc2[0][k]);
+          acc2[1][k] = fmaf(a, y1, acc2[1][k]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int g = g0 + gl[u];
+    const size_t wrow = ((size_t)bh * GP + g) * d;
+    float n2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = lane + 32 * k;
+      if (c < d) {
+        const float w = a_scale * acc2[u][k];
+        n2 = fmaf(w, w, n2);
+        if (live[u]) {
+          const __nv_bfloat16 hi = __float2bfloat16(w);
+          w_hi[wrow + c] = hi;
+          w_lo[wrow + c] = __float2bfloat16(w - __bfloat162float(hi));
+        }
+      }
+    }
+    n2 = warp_sum(n2);
+    if (live[u] && lane == 0) wnorm[(size_t)bh * GP + g] = sqrtf(n2);
   }
 }
 
@@ -216,30 +277,34 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
 // Tensor-core assignment fused with the centroid sums of the next update.
 // Persistent: CTA b takes the global 128-row tiles [b per, (b+1) per) (tile i = row tile
 // i mod T of head i / T) and runs them through a pipeline:
-//   warp 17     (lane 0) loads the X tile (contiguous rows, two TMA boxes of 128 rows x 64
+//   warp 19     (lane 0) loads the X tile (contiguous rows, two TMA boxes of 128 rows x 64
 //               columns, 128B-swizzled) into a three-deep ring
-//   warp 16     (lane 0) scores S = X [w_hi w_lo]^T into a double-buffered TMEM tile, then,
+//   warp 18     (lane 0) scores S = X [w_hi w_lo]^T into a double-buffered TMEM tile, then,
 //               once the labels are known, adds onehot(labels)^T X into a TMEM sum
 //               (M = 128 groups x N = d; A and B both MN-major, read straight from the
 //               one-hot tile and the X tile)
 //   warps 0-15  row r = TMEM lane r, columns split in four quarters (warps w, w + 4, w + 8,
-//               w + 12): argmin of bias_g - 2 s_g per quarter, merged through shared memory; the
-//               label goes into the sums through a one-hot row; a row whose runner-up is
-//               within twice the error bound also goes on the list of the exact re-check,
-//               which corrects its label (and, through the correction list, the sums) if
-//               the exact argmin differs.
+//               w + 12): argmin and runner-up of bias_g - 2 s_g per quarter and the
+//               quarter's ||x||^2, handed over through shared memory (double-buffered)
+//   warps 16-17 the finisher, two rows per thread: merges the quarters, writes the label
+//               and the count, puts a row whose runner-up is within twice the error bound
+//               on the list of the exact re-check (which corrects its label and, through
+//               the correction list, the sums), and writes the tile's one-hot rows.  The
+//               argmin warps go on to the next tile meanwhile.
 // When the CTA leaves a head (or ends) the sums and the per-group counts go to the
 // partial slot (CTA, head - first head of the CTA).
 // ---------------------------------------------------------------------------
 namespace kma {
-constexpr int NT = 576;
-constexpr int NEPI = 512;
+constexpr int NT = 640;
+constexpr int NEPI = 512;   // argmin threads (warps 0-15)
+constexpr int NFIN = 64;    // finisher threads (warps 16-17), two rows each
 constexpr int NQ = 4;   // column quarters
-constexpr int MMA_WARP = 16;
-constexpr int LOAD_WARP = 17;
+constexpr int FIN_WARP = 16;
+constexpr int MMA_WARP = 18;
+constexpr int LOAD_WARP = 19;
 constexpr int XS = 3;   // X ring depth
 struct Bars {
-  uint64_t xfull[XS], xempty[XS], tfull[2], tempty[2], ohfull, ohempty, sumdone, xready[2], epidone;
+  uint64_t xfull[XS], xempty[XS], tfull[2], tempty[2], ohfull, ohempty, sumdone, xready[2], xfree[2], epidone;
 };
 struct Half {
   float best, second, xx;
@@ -286,12 +351,14 @@ __global__ void __launch_bounds__(kma::NT, 1)
       mbar_init(su32(&bars->tfull[b]), 1);
       mbar_init(su32(&bars->tempty[b]), kma::NEPI);
     }
-    mbar_init(su32(&bars->ohfull), kma::NEPI);
+    mbar_init(su32(&bars->ohfull), kma::NFIN);
     mbar_init(su32(&bars->ohempty), 1);
     mbar_init(su32(&bars->sumdone), 1);
-    mbar_init(su32(&bars->xready[0]), kma::NEPI);
-    mbar_init(su32(&bars->xready[1]), kma::NEPI);
-    mbar_init(su32(&bars->epidone), kma::NEPI);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(su32(&bars->xready[b]), kma::NEPI);
+      mbar_init(su32(&bars->xfree[b]), kma::NFIN);
+    }
+    mbar_init(su32(&bars->epidone), kma::NFIN);
     fence_barrier_init();
   }
   if (warp == kma::MMA_WARP) {
@@ -313,6 +380,11 @@ __global__ void __launch_bounds__(kma::NT, 1)
 
   int it = 0, sg = 0;   // running tile / segment counters (identical across roles)
   bool ok = true;
+  int prev_c[2] = {-1, -1};   // finisher: chunk of each of its rows' one in the one-hot tile
+  // the one-hot tile starts all zero (the finisher then only moves each row's one)
+  for (int e = tid; e < (int)(kOH / 16); e += kma::NT)
+    *reinterpret_cast<uint4*>(smem + XS * kX + 16 * e) = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async();
   for (int s0 = t0; s0 < t1 && ok;) {
     const int bh = s0 / T;
     const int s1 = min(t1, (bh + 1) * T);
@@ -359,52 +431,146 @@ __global__ void __launch_bounds__(kma::NT, 1)
       it = __shfl_sync(0xffffffffu, it, 0);
     } else if (warp == kma::MMA_WARP) {
       // ---------------- MMA ----------------
+      // Scores and sums are issued as their inputs become ready, not in a fixed order: the
+      // scores of a later tile (needing its X tile and a free score buffer) do not wait
+      // behind the sums of an earlier tile (needing that tile's one-hot rows).
       if (lane == 0) {
-        const int first = it;
-        auto sums = [&](int j) -> bool {
-          const int xj = j % XS;
-          if (!wait(bars->ohfull, j & 1)) return false;
-          tc_fence_after();
+        const int first = it, last = it + (s1 - s0);
+        int ns = first, nm = first;   // next tile to score / to sum
+        const uint64_t t_start = gtimer();
+        while (ok && nm < last) {
+          bool moved = false;
+          if (ns < last) {
+            const int b = ns & 1, xb = ns % XS;
+            if (mbar_test(su32(&bars->xfull[xb]), (ns / XS) & 1) &&
+                (ns < 2 || mbar_test(su32(&bars->tempty[b]), ((ns >> 1) - 1) & 1))) {
+              tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            tc_mma(tSum, sdesc(sOH + k * 2048, 16384, 1024), sdesc(sX + xj * kX + k * 2048, 16384, 1024), IDA,
-                   (j > first || k > 0) ? 1u : 0u);
-          tc_commit(su32(&bars->xempty[xj]));
-          tc_commit(su32(&bars->ohempty));
-          return true;
-        };
-        for (int i = s0; i < s1 && ok; ++i, ++it) {
-          const int b = it & 1, xb = it % XS;
-          ok = wait(bars->xfull[xb], (it / XS) & 1) && (it < 2 || wait(bars->tempty[b], ((it >> 1) - 1) & 1));
-          if (!ok) break;
-          tc_fence_after();
+              for (int k = 0; k < D / 16; ++k) {
+                const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
+                const uint32_t ow = (k >> 2) * (GP * 128) + (k & 3) * 32;
+                tc_mma(tmem + 128 * b, sdesc(sX + xb * kX + ox, 16, 1024), sdesc(sWh + ow, 16, 1024), IDS,
+                       k > 0 ? 1u : 0u);
+              }
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
-            const uint32_t ow = (k >> 2) * (GP * 128) + (k & 3) * 32;
-            tc_mma(tmem + 128 * b, sdesc(sX + xb * kX + ox, 16, 1024), sdesc(sWh + ow, 16, 1024), IDS, k > 0 ? 1u : 0u);
+              for (int k = 0; k < D / 16; ++k) {
+                const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
+                const uint32_t ow = (k >> 2) * (GP * 128) + (k & 3) * 32;
+                tc_mma(tmem + 128 * b, sdesc(sX + xb * kX + ox, 16, 1024), sdesc(sWl + ow, 16, 1024), IDS, 1u);
+              }
+              tc_commit(su32(&bars->tfull[b]));
+              ++ns;
+              moved = true;
+            }
           }
+          if (nm < ns && mbar_test(su32(&bars->ohfull), nm & 1)) {
+            const int xj = nm % XS;
+            tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint32_t ox = (k >> 2) * (128 * 128) + (k & 3) * 32;
-            const uint32_t ow = (k >> 2) * (GP * 128) + (k & 3) * 32;
-            tc_mma(tmem + 128 * b, sdesc(sX + xb * kX + ox, 16, 1024), sdesc(sWl + ow, 16, 1024), IDS, 1u);
+            for (int k = 0; k < 8; ++k)
+              tc_mma(tSum, sdesc(sOH + k * 2048, 16384, 1024), sdesc(sX + xj * kX + k * 2048, 16384, 1024), IDA,
+                     (nm > first || k > 0) ? 1u : 0u);
+            tc_commit(su32(&bars->xempty[xj]));
+            tc_commit(su32(&bars->ohempty));
+            ++nm;
+            moved = true;
           }
-          tc_commit(su32(&bars->tfull[b]));
-          if (it > first) ok = sums(it - 1);
+          if (!moved) {
+            if (*abort_flag) ok = false;
+            else if (gtimer() - t_start > kTimeoutNs) {
+              *abort_flag = 1;
+              set_error(err, DERR_WAIT_TIMEOUT);
+              ok = false;
+            }
+          }
         }
-        if (ok && it > first) ok = sums(it - 1);
+        it = nm;
         tc_commit(su32(&bars->sumdone));
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       it = __shfl_sync(0xffffffffu, it, 0);
+    } else if (warp >= kma::FIN_WARP) {
+      // ---------------- finisher (warps 16-17): merge the quarters of rows f and f + 64,
+      // labels, counts, flags, one-hot rows ----------------
+      const int f = tid - kma::FIN_WARP * 32;
+      for (int i = s0; i < s1 && ok; ++i, ++it) {
+        const int b = it & 1;
+        ok = __all_sync(0xffffffffu, wait(bars->xready[b], (it >> 1) & 1));
+        if (!ok) break;
+        int bi2[2];
+        float best2[2], second2[2], xsum2[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int r = f + 64 * u;
+          // merge in column order, so a lower quarter wins ties
+          kma::Half m = xchg[(b * kma::NQ + 0) * 128 + r];
+          float xsum = m.xx;
+#pragma unroll
+          for (int q = 1; q < kma::NQ; ++q) {
+            const kma::Half o = xchg[(b * kma::NQ + q) * 128 + r];
+            xsum += o.xx;
+            const bool take = o.best < m.best;
+            m.second = take ? fminf(m.best, o.second) : fminf(m.second, o.best);
+            if (take) { m.best = o.best; m.bi = o.bi; }
+          }
+          bi2[u] = m.bi;
+          best2[u] = m.best;
+          second2[u] = m.second;
+          xsum2[u] = xsum;
+        }
+        // xchg[b] may take tile it + 2
+        mbar_arrive(su32(&bars->xfree[b]));
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int r = f + 64 * u, row = (i - bh * T) * 128 + r;
+          if (row < N) {
+            const float best = best2[u], second = second2[u];
+            const int bi = bi2[u];
+            const float bound = kc * sqrtf(xsum2[u]) * wmax + 1e-6f * (fabsf(best) + fabsf(second));
+            labels[head + row] = bi;
+            atomicAdd(&sCnt[bi], 1);
+            if (second - best > 2.f * bound) {
+              if (trace) trace[head + row] = bi;
+            } else {
+              const int fs = atomicAdd(&flag_count[bh], 1);
+              flag_rows[head + fs] = row;
+            }
+          }
+        }
+        // one-hot rows of this tile, once the previous sums read theirs: the tile holds the
+        // previous tile's ones (all zero at the start), so a row clears the 16-byte chunk of
+        // its previous one and sets the chunk of its new one (rows past N stay zero)
+        if (it >= 1) ok = __all_sync(0xffffffffu, wait(bars->ohempty, (it - 1) & 1));
+        if (!ok) break;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int r = f + 64 * u;
+          const bool in = (i - bh * T) * 128 + r < N;
+          const int bi = bi2[u];
+          const int c_new = in ? (bi >> 3) : -1;
+          if (prev_c[u] >= 0 && prev_c[u] != c_new)
+            *reinterpret_cast<uint4*>(smem + XS * kX + tile_off(r, prev_c[u], 128)) = make_uint4(0u, 0u, 0u, 0u);
+          if (c_new >= 0) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t one = 0x3F80u << (16 * (bi & 1));   // bf16 1.0 in the low or high half
+            const int wd = (bi & 7) >> 1;
+            if (wd == 0) v.x = one; else if (wd == 1) v.y = one; else if (wd == 2) v.z = one; else v.w = one;
+            *reinterpret_cast<uint4*>(smem + XS * kX + tile_off(r, c_new, 128)) = v;
+          }
+          prev_c[u] = c_new;
+        }
+        fence_proxy_async();
+        mbar_arrive(su32(&bars->ohfull));
+      }
+      // every row's count of this head is in sCnt
+      mbar_arrive(su32(&bars->epidone));
     } else {
-      // ---------------- labels, one-hot rows, flags (warps 0-15) ----------------
+      // ---------------- argmin per column quarter (warps 0-15) ----------------
       const int hf = warp >> 2;                 // column quarter
       const int r = (warp & 3) * 32 + lane;     // row = TMEM lane
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       for (int i = s0; i < s1 && ok; ++i, ++it) {
-        const int b = it & 1, xb = it % XS, row = (i - bh * T) * 128 + r;
+        const int b = it & 1, xb = it % XS;
         // scores ready; the X tile (read below for ||x||) completed before them
         ok = __all_sync(0xffffffffu, wait(bars->tfull[b], (it >> 1) & 1) && wait(bars->xfull[xb], (it / XS) & 1));
         if (!ok) break;
@@ -419,13 +585,20 @@ __global__ void __launch_bounds__(kma::NT, 1)
           if (cb < GP) {
             uint32_t v[32];
             tc_ld32(tmem + 128 * b + lane_off + cb, v);
+            const uint64_t m2 = f2pack(-2.f, -2.f);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int q = e & 3;
-              const float sc = fmaf(-2.f, __uint_as_float(v[e]), sBias[cb + e]);
-              snd[q] = fminf(snd[q], fmaxf(bst[q], sc));
-              bix[q] = sc < bst[q] ? cb + e : bix[q];
-              bst[q] = fminf(bst[q], sc);
+            for (int e = 0; e < 32; e += 2) {
+              float sc2[2];
+              f2unpack(ffma2(m2, f2pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
+                             f2pack(sBias[cb + e], sBias[cb + e + 1])), sc2[0], sc2[1]);
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const int q = (e + u) & 3;
+                const float sc = sc2[u];
+                snd[q] = fminf(snd[q], fmaxf(bst[q], sc));
+                bix[q] = sc < bst[q] ? cb + e + u : bix[q];
+                bst[q] = fminf(bst[q], sc);
+              }
             }
           }
         }
@@ -447,62 +620,19 @@ __global__ void __launch_bounds__(kma::NT, 1)
           const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(h2[e]);
-            xx = fmaf(f.x, f.x, fmaf(f.y, f.y, xx));
+            const float2 fl = __bfloat1622float2(h2[e]);
+            xx = fmaf(fl.x, fl.x, fmaf(fl.y, fl.y, xx));
           }
         }
         h.xx = xx;
+        // the finisher has read xchg[b] of tile it - 2
+        if (it >= 2) ok = __all_sync(0xffffffffu, wait(bars->xfree[b], ((it >> 1) - 1) & 1));
+        if (!ok) break;
         xchg[(b * kma::NQ + hf) * 128 + r] = h;
-        // every quarter of every row is in (an mbarrier, so an abort cannot strand a warp)
         mbar_arrive(su32(&bars->xready[b]));
-        ok = __all_sync(0xffffffffu, wait(bars->xready[b], (it >> 1) & 1));
-        if (!ok) break;
-        // merge in column order, so a lower quarter wins ties
-        kma::Half m = xchg[(b * kma::NQ + 0) * 128 + r];
-        float xsum = m.xx;
-#pragma unroll
-        for (int q = 1; q < kma::NQ; ++q) {
-          const kma::Half o = xchg[(b * kma::NQ + q) * 128 + r];
-          xsum += o.xx;
-          const bool take = o.best < m.best;
-          m.second = take ? fminf(m.best, o.second) : fminf(m.second, o.best);
-          if (take) { m.best = o.best; m.bi = o.bi; }
-        }
-        const float best = m.best, second = m.second;
-        const int bi = m.bi;
-        const bool in = row < N;
-        if (in && hf == 0) {
-          const float bound = kc * sqrtf(xsum) * wmax + 1e-6f * (fabsf(best) + fabsf(second));
-          labels[head + row] = bi;
-          atomicAdd(&sCnt[bi], 1);
-          if (second - best > 2.f * bound) {
-            if (trace) trace[head + row] = bi;
-          } else {
-            const int fs = atomicAdd(&flag_count[bh], 1);
-            flag_rows[head + fs] = row;
-          }
-        }
-        // one-hot row r of this tile, this quarter's 4 chunks (zero for rows past N)
-        if (it >= 1) ok = __all_sync(0xffffffffu, wait(bars->ohempty, (it - 1) & 1));
-        if (!ok) break;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int c = hf * 4 + cc;
-          uint4 u = make_uint4(0u, 0u, 0u, 0u);
-          if (in && (bi >> 3) == c) {
-            const uint32_t one = 0x3F80u << (16 * (bi & 1));   // bf16 1.0 in the low or high half
-            const int wd = (bi & 7) >> 1;
-            if (wd == 0) u.x = one; else if (wd == 1) u.y = one; else if (wd == 2) u.z = one; else u.w = one;
-          }
-          *reinterpret_cast<uint4*>(smem + XS * kX + tile_off(r, c, 128)) = u;
-        }
-        fence_proxy_async();
-        mbar_arrive(su32(&bars->ohfull));
       }
       // ---- sums and counts of this head -> partial slot (each quarter writes 32 columns)
       if (ok) ok = __all_sync(0xffffffffu, wait(bars->sumdone, sg & 1));
-      // every row's count is in sCnt
-      mbar_arrive(su32(&bars->epidone));
       if (ok) ok = __all_sync(0xffffffffu, wait(bars->epidone, sg & 1));
       if (ok) {
         tc_fence_after();
@@ -946,7 +1076,8 @@ cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_
 }
 
 size_t centroid_weights_smem(int d, int D) {
-  return (size_t)km::WG_PER_CTA * d * 8 + km::WG_PER_CTA * 4 + ((size_t)D * (d + 1) + 8 * d + 8 * 128) * 4;
+  return (size_t)km::WG_PER_CTA * d * 8 + km::WG_PER_CTA * 4 +
+         ((size_t)D * (d + 1) + (size_t)km::WG_PER_CTA * d + (size_t)km::WG_PER_CTA * 128) * 4;
 }
 
 cudaError_t launch_centroid_weights(float* m, int BH, int G, int d, const float* A, size_t a_head, int sj, int sc,
