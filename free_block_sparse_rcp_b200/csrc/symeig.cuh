@@ -4,7 +4,8 @@
 //   1. Householder reduction to tridiagonal form, A = Q T Q^T (Golub & Van Loan, "Matrix
 //      Computations", Householder tridiagonalization): step k reflects column k below the
 //      diagonal onto its first entry; the trailing block is updated as A -= v w^T + w v^T
-//      with p = beta A v, w = p - (beta/2)(v^T p) v.  The reflector v_k is kept in column k
+//      with p = beta A v, w = p - (beta/2)(v^T p) v (a few threads per row for A v and the
+//      update, v^T p reduced in the same pass).  The reflector v_k is kept in column k
 //      below the diagonal.
 //   2. Eigenvalues of T bracketed by multisection on the Sturm count (the number of negative
 //      pivots of the LDL^T factorisation of T - x I), evaluated in fp32: each warp brackets one
@@ -102,6 +103,10 @@ __device__ inline void sym_top_eigen(double* A, int R, double* Z, int ldz, doubl
   constexpr int LD = N + 1;
   constexpr int NC = (N + 31) / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  // threads per row of the trailing-block passes (a power of two <= 32) and rows per pass
+  int TPR = 1;
+  while (TPR < 32 && TPR * 2 * N <= (int)blockDim.x) TPR *= 2;
+  const int RPP = blockDim.x / TPR;
   double* d = sc;            // [N]
   double* e = d + N;         // [N]  e[i] = T[i+1][i]
   double* e2 = e + N;        // [N]
@@ -113,6 +118,7 @@ __device__ inline void sym_top_eigen(double* A, int R, double* Z, int ldz, doubl
   double* shift = p + 2 * N; // [64]
   int* cstart = reinterpret_cast<int*>(shift + 64);  // [64]
   double* misc = shift + 64 + 64;                    // [64 + 8]: gl, gu, tnorm, pivmin
+  double* red = misc + 8;                            // [32] per-warp partial sums (misc has 72)
 
   // ---- 1. tridiagonalisation
   for (int k = 0; k + 2 < N; ++k) {
@@ -144,31 +150,37 @@ __device__ inline void sym_top_eigen(double* A, int R, double* Z, int ldz, doubl
     __syncthreads();
     const double b = beta[k];
     if (b != 0.0) {
-      double vj[NC];
-#pragma unroll
-      for (int c = 0; c < NC; ++c) vj[c] = (lane + 32 * c < m) ? v[lane + 32 * c] : 0.0;
-      for (int i = warp; i < m; i += nw) {
-        const double* row = A + (k + 1 + i) * LD + (k + 1);
+      // p = b A v: TPR threads per row, each a strided part of the dot product, combined
+      // with shuffles; the same pass sums v.p for kk (per warp, then over the warps)
+      double vp = 0.0;
+      for (int i0 = 0; i0 < m; i0 += RPP) {
+        const int i = i0 + tid / TPR, sub = tid % TPR;
         double acc = 0.0;
+        if (i < m) {
+          const double* row = A + (k + 1 + i) * LD + (k + 1);
+          for (int j = sub; j < m; j += TPR) acc += row[j] * v[j];
+        }
 #pragma unroll
-        for (int c = 0; c < NC; ++c)
-          if (lane + 32 * c < m) acc += row[lane + 32 * c] * vj[c];
-        acc = warp_sum_f64(acc);
-        if (lane == 0) p[i] = b * acc;
+        for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (i < m && sub == 0) {
+          const double pi = b * acc;
+          p[i] = pi;
+          vp += v[i] * pi;
+        }
       }
+      vp = warp_sum_f64(vp);
+      if (lane == 0) red[warp] = vp;
       __syncthreads();
-      double kk = 0.0;
-      for (int i = lane; i < m; i += 32) kk += v[i] * p[i];
+      double kk = lane < nw ? red[lane] : 0.0;
       kk = 0.5 * b * warp_sum_f64(kk);
-      double wj[NC];
-#pragma unroll
-      for (int c = 0; c < NC; ++c) wj[c] = (lane + 32 * c < m) ? p[lane + 32 * c] - kk * vj[c] : 0.0;
-      for (int i = warp; i < m; i += nw) {
-        const double vi = v[i], wi = p[i] - kk * vi;
-        double* row = A + (k + 1 + i) * LD + (k + 1);
-#pragma unroll
-        for (int c = 0; c < NC; ++c)
-          if (lane + 32 * c < m) row[lane + 32 * c] -= vi * wj[c] + wi * vj[c];
+      // A -= v w^T + w v^T on the trailing block, w = p - kk v
+      for (int i0 = 0; i0 < m; i0 += RPP) {
+        const int i = i0 + tid / TPR, sub = tid % TPR;
+        if (i < m) {
+          const double vi = v[i], wi = p[i] - kk * vi;
+          double* row = A + (k + 1 + i) * LD + (k + 1);
+          for (int j = sub; j < m; j += TPR) row[j] -= vi * (p[j] - kk * v[j]) + wi * v[j];
+        }
       }
     }
     __syncthreads();
