@@ -168,10 +168,16 @@ def run_cuda(args):
     import free_block_sparse_rcp_b200 as spr
     from synth import generate, workload
 
-    w = workload(args.workload, H=args.heads) if args.heads else workload(args.workload)
+    over = {}
+    if args.heads:
+        over["H"] = args.heads
+    if args.density:
+        over["density"] = args.density
+    w = workload(args.workload, **over)
     pd = dict(B=w.B, H=w.H, N=w.N, d=w.d, block=w.block, density=w.density, n_kgroups=w.n_kgroups,
               n_qgroups=w.n_qgroups, n_samples=w.n_samples, n_probes=w.n_probes, eig_rank=w.eig_rank,
-              sub_rank=w.sub_rank, kmeans_iters=w.kmeans_iters, ridge_lambda=w.ridge_lambda, seed=0)
+              sub_rank=w.sub_rank, kmeans_iters=w.kmeans_iters, ridge_lambda=w.ridge_lambda, seed=0,
+              partition_mode=1 if args.partition == "semantic" else 0)
     from synth import frame_index, perturb, to_torch
     frames = frame_index(w.grid) if w.frame_causal else None
     fid = torch.from_numpy(frames).to(dev) if w.frame_causal else None
@@ -371,6 +377,10 @@ def run_cuda(args):
     }
     if calls > 1:
         line["ms_per_call"] = round(ms_per_call, 4)
+    if args.partition != "coupled":
+        line["config"]["partition"] = "semantic-grouping baseline (keys and queries clustered on raw rows)"
+    if args.diagnostics:
+        line["diagnostics"] = partition_diagnostics(part, Ql, Kl, o_sparse, o_dense, p, frames)
     if rank == 0 and ws == 1 and not args.heads:
         line["cpu_baseline"] = cpu_baseline(w)
     if ws > 1:
@@ -379,6 +389,55 @@ def run_cuda(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def partition_diagnostics(part, Q, K, o_sparse, o_dense, p, frames=None, heads=(0, 1), groups=16, mass=0.9):
+    """Measurements of the partition on a few heads (torch on the device; reporting only).
+
+    support: the fraction of keys that holds `mass` of a query's softmax, per query and
+    for the pooled distribution (mean of the member rows) of each of `groups` query
+    groups (the groups' queries would share one key set).  affine: the share of the
+    residual O_dense - O_sparse that a least-squares affine map of O_sparse explains over
+    all rows, and the unexplained energy relative to the residual energy."""
+    import torch
+    H, N = p.H, p.N
+    s = p.eff_scale()
+    out = {"heads": list(heads), "mass": mass, "groups_per_head": groups}
+    perq, pooled, expl, unexpl = [], [], [], []
+    fr = None if frames is None else torch.as_tensor(frames, device=Q.device).long()
+    for bh in heads:
+        b, h = divmod(bh, H)
+        lq = part["label_q"][bh].long()
+        sizes = torch.bincount(lq, minlength=p.n_qgroups)
+        cand = torch.nonzero(sizes > 0).flatten()
+        pick = cand[torch.linspace(0, cand.numel() - 1, min(groups, cand.numel())).round().long()]
+        k = K[b, h].float()
+        for a in pick.tolist():
+            rows = torch.nonzero(lq == a).flatten()
+            logits = s * (Q[b, h, rows].float() @ k.T)
+            if fr is not None:
+                logits = logits.masked_fill(fr[None, :] > fr[rows][:, None], float("-inf"))
+            pr = torch.softmax(logits.double(), dim=1)
+
+            def frac(x):
+                srt = torch.sort(x, dim=-1, descending=True).values
+                need = (torch.cumsum(srt, dim=-1) < mass * srt.sum(-1, keepdim=True) * (1 - 1e-12)).sum(-1) + 1
+                return need.clamp(max=x.shape[-1]).double() / x.shape[-1]
+            perq.extend(frac(pr).tolist())
+            pooled.append(float(frac(pr.mean(0))))
+        x = o_sparse[b, h].double()
+        r = o_dense[b, h].double() - x
+        xa = torch.cat([torch.ones(N, 1, dtype=x.dtype, device=x.device), x], dim=1)
+        coef = torch.linalg.lstsq(xa, r).solution
+        un = float(((r - xa @ coef) ** 2).sum())
+        tot = float((r ** 2).sum())
+        expl.append(1.0 - un / tot)
+        unexpl.append(un / tot)
+    out["per_query_support"] = round(sum(perq) / len(perq), 5)
+    out["grouped_support"] = round(sum(pooled) / len(pooled), 5)
+    out["affine_explainable"] = round(sum(expl) / len(expl), 5)
+    out["unexplained_energy_rel"] = round(sum(unexpl) / len(unexpl), 5)
+    return out
 
 
 def attention_pairs(part, frames=None):
@@ -519,6 +578,11 @@ def main():
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=["wan", "world"],
                     help="wan: the 32,760-token call (default); world: the frame-causal rollout")
+    ap.add_argument("--partition", default="coupled", choices=["coupled", "semantic"],
+                    help="coupled: the method; semantic: the semantic-grouping baseline of the pages")
+    ap.add_argument("--density", type=float, default=0.0, help="override the workload's target density")
+    ap.add_argument("--diagnostics", action="store_true",
+                    help="add support and affine-explainability measurements of two heads to the line")
     ap.add_argument("--streams", type=int, default=2, choices=[1, 2],
                     help="2: probe_fit beside the routed attention on a second stream (default); 1: in sequence")
     ap.add_argument("--heads", type=int, default=0,

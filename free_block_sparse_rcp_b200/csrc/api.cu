@@ -50,7 +50,7 @@ struct Layout {
   // header
   size_t err;
   // partition
-  size_t sample_idx, metric, eigval, eigvec, proj, eig_lu, m_k, nu_k, key_init, C, m_q, nu_q, query_init, bias, wnorm,
+  size_t ident, sample_idx, metric, eigval, eigvec, proj, eig_lu, m_k, nu_k, key_init, C, m_q, nu_q, query_init, bias, wnorm,
       w_hi, w_lo, flag_count, flag_rows, corr_count, corr, psum, pcnt, mass, order, alpha;
   // attend
   size_t rlist, rcum, rcnt, tiles, tile_count;
@@ -74,11 +74,14 @@ Layout make_layout(const sparsepr_params& p) {
   L.max_tiles = ceil_div(p.N, kAttnTileRows) + p.n_qgroups;
   L.T = ceil_div(p.N, p.block);
   L.S = probe_splits(p.N);
-  L.DTk = kmeans_dt(p.eig_rank);
-  L.DTq = kmeans_dt(p.n_kgroups);
+  // coordinate widths of the two k-means: response coordinates (r_e for keys, G_k for
+  // queries), or the raw d-dimensional rows for the semantic-grouping baseline
+  L.DTk = kmeans_dt(p.partition_mode == 1 ? p.d : p.eig_rank);
+  L.DTq = kmeans_dt(p.partition_mode == 1 ? p.d : p.n_kgroups);
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = al256(o + bytes); return at; };
   L.err = take(256);
+  L.ident = take(p.partition_mode == 1 ? d * d * 4 : 0);
   L.sample_idx = take(BH * p.n_samples * 4);
   L.metric = take(BH * d * d * 4);
   L.eigval = take(BH * re * 4);
@@ -172,6 +175,8 @@ sparsepr_status check_params(const sparsepr_params* p) {
   if (p->kmeans_iters < 1 || p->kmeans_iters > 64) return failv(SPARSEPR_EINVAL, "kmeans_iters must be in [1, 64]", p->kmeans_iters);
   if (!(p->ridge_lambda > 0.f) || !isfinite(p->ridge_lambda)) return fail(SPARSEPR_EINVAL, "ridge_lambda must be > 0");
   if (!(p->scale >= 0.f) || !isfinite(p->scale)) return fail(SPARSEPR_EINVAL, "scale must be >= 0");
+  if (p->partition_mode != 0 && p->partition_mode != 1)
+    return failv(SPARSEPR_EINVAL, "partition_mode must be 0 (response-coupled) or 1 (semantic)", p->partition_mode);
   if (p->frame_id) {
     if (p->n_frames < 1 || p->n_frames > kMaxFrames)
       return failv(SPARSEPR_EINVAL, "n_frames must be in [1, 64] with frame_id", p->n_frames);
@@ -185,9 +190,10 @@ sparsepr_status check_params(const sparsepr_params* p) {
   // kernel limits
   if (p->n_kgroups > 128) return fail(SPARSEPR_EUNSUPPORTED, "n_kgroups > 128 (query coordinates wider than 128) not built");
   if (p->n_qgroups > 128) return fail(SPARSEPR_EUNSUPPORTED, "n_qgroups > 128 not built");
-  if (recheck_smem(p->d, p->n_kgroups, kmeans_dt(p->n_kgroups), p->n_qgroups) > kSmemLimit ||
-      recheck_smem(p->d, p->eig_rank, kmeans_dt(p->eig_rank), p->n_kgroups) > kSmemLimit ||
-      centroid_weights_smem(p->d, p->n_kgroups) > kSmemLimit ||
+  const int Dk = p->partition_mode == 1 ? p->d : p->eig_rank, Dq = p->partition_mode == 1 ? p->d : p->n_kgroups;
+  if (recheck_smem(p->d, Dq, kmeans_dt(Dq), p->n_qgroups) > kSmemLimit ||
+      recheck_smem(p->d, Dk, kmeans_dt(Dk), p->n_kgroups) > kSmemLimit ||
+      centroid_weights_smem(p->d, Dq > Dk ? Dq : Dk) > kSmemLimit ||
       assign_acc_smem(p->d, kmeans_gp(p->n_kgroups > p->n_qgroups ? p->n_kgroups : p->n_qgroups)) > kSmemLimit)
     return fail(SPARSEPR_EUNSUPPORTED, "too many groups for the k-means kernels");
   if (route_select_smem(p->n_qgroups, p->n_kgroups) > kSmemLimit)
@@ -237,10 +243,15 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
   SPR_CUDA(cudaMemsetAsync(err, 0, 4, st));
   float* metric = at<float>(ws, L.metric);
   float* proj = at<float>(ws, L.proj);
-  SPR_LAUNCH(launch_sample_metric(Q, BH, N, d, p.n_samples, p.seed, metric, at<int>(ws, L.sample_idx), err, st));
-  SPR_LAUNCH(launch_metric_eigen(metric, BH, d, re, at<float>(ws, L.eigval), at<float>(ws, L.eigvec), proj,
-                                 at<double>(ws, L.eig_lu), st));
-  if (tr && tr->key_coords) SPR_LAUNCH(launch_key_coords(K, BH, N, d, re, proj, tr->key_coords, st));
+  const bool semantic = p.partition_mode == 1;
+  if (!semantic) {
+    SPR_LAUNCH(launch_sample_metric(Q, BH, N, d, p.n_samples, p.seed, metric, at<int>(ws, L.sample_idx), err, st));
+    SPR_LAUNCH(launch_metric_eigen(metric, BH, d, re, at<float>(ws, L.eigval), at<float>(ws, L.eigvec), proj,
+                                   at<double>(ws, L.eig_lu), st));
+    if (tr && tr->key_coords) SPR_LAUNCH(launch_key_coords(K, BH, N, d, re, proj, tr->key_coords, st));
+  } else {
+    SPR_LAUNCH(launch_identity(at<float>(ws, L.ident), d, st));
+  }
   float* bias = at<float>(ws, L.bias);
   float* wnorm = at<float>(ws, L.wnorm);
   void* w_hi = at<char>(ws, L.w_hi);
@@ -278,14 +289,27 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
   // keys on y = Lambda^{1/2} U^T k: A(j, c) = proj[c][j]; K/V group centroids = mean raw key
   // of the final groups (empty group -> 0)
   float* C = at<float>(ws, L.C);
-  SPR_CHECK(kmeans(K, Gk, PURPOSE_KEY_KMEANS, proj, (size_t)d * re, 1, re, 1.0f, re, L.DTk, at<float>(ws, L.m_k),
-                   at<float>(ws, L.nu_k), at<int>(ws, L.key_init), label_k, perm_k, koff,
-                   tr ? tr->key_label_iters : nullptr, C));
+  const float* ident = at<float>(ws, L.ident);
+  if (!semantic) {
+    SPR_CHECK(kmeans(K, Gk, PURPOSE_KEY_KMEANS, proj, (size_t)d * re, 1, re, 1.0f, re, L.DTk, at<float>(ws, L.m_k),
+                     at<float>(ws, L.nu_k), at<int>(ws, L.key_init), label_k, perm_k, koff,
+                     tr ? tr->key_label_iters : nullptr, C));
+  } else {
+    // semantic-grouping baseline: keys clustered on their raw rows (A = identity)
+    SPR_CHECK(kmeans(K, Gk, PURPOSE_KEY_KMEANS, ident, 0, d, 1, 1.0f, d, L.DTk, at<float>(ws, L.m_k),
+                     at<float>(ws, L.nu_k), at<int>(ws, L.key_init), label_k, perm_k, koff,
+                     tr ? tr->key_label_iters : nullptr, C));
+  }
   if (tr && tr->query_coords) SPR_LAUNCH(launch_query_coords(Q, BH, N, d, C, Gk, scale, tr->query_coords, st));
-  // queries on z = s C q: A(j, c) = s * C[j][c]
-  SPR_CHECK(kmeans(Q, Gq, PURPOSE_QUERY_KMEANS, C, (size_t)Gk * d, d, 1, scale, Gk, L.DTq, at<float>(ws, L.m_q),
-                   at<float>(ws, L.nu_q), at<int>(ws, L.query_init), label_q, perm_q, qoff,
-                   tr ? tr->query_label_iters : nullptr, nullptr));
+  // queries on z = s C q: A(j, c) = s * C[j][c]  (semantic baseline: on the raw rows)
+  if (!semantic)
+    SPR_CHECK(kmeans(Q, Gq, PURPOSE_QUERY_KMEANS, C, (size_t)Gk * d, d, 1, scale, Gk, L.DTq, at<float>(ws, L.m_q),
+                     at<float>(ws, L.nu_q), at<int>(ws, L.query_init), label_q, perm_q, qoff,
+                     tr ? tr->query_label_iters : nullptr, nullptr));
+  else
+    SPR_CHECK(kmeans(Q, Gq, PURPOSE_QUERY_KMEANS, ident, 0, d, 1, 1.0f, d, L.DTq, at<float>(ws, L.m_q),
+                     at<float>(ws, L.nu_q), at<int>(ws, L.query_init), label_q, perm_q, qoff,
+                     tr ? tr->query_label_iters : nullptr, nullptr));
   float* mass = at<float>(ws, L.mass);
   // frame-causal: visible keys per (K/V group, frame), query frame histograms, frame ends
   Causal cz{};
@@ -312,10 +336,12 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
       return dst ? cudaMemcpyAsync(dst, at<char>(ws, off), bytes, cudaMemcpyDeviceToDevice, st) : cudaSuccess;
     };
     const size_t bh = BH;
-    SPR_CUDA(cp(tr->sample_idx, L.sample_idx, bh * p.n_samples * 4));
-    SPR_CUDA(cp(tr->metric, L.metric, bh * d * d * 4));
-    SPR_CUDA(cp(tr->eigval, L.eigval, bh * re * 4));
-    SPR_CUDA(cp(tr->eigvec, L.eigvec, bh * d * re * 4));
+    if (!semantic) {
+      SPR_CUDA(cp(tr->sample_idx, L.sample_idx, bh * p.n_samples * 4));
+      SPR_CUDA(cp(tr->metric, L.metric, bh * d * d * 4));
+      SPR_CUDA(cp(tr->eigval, L.eigval, bh * re * 4));
+      SPR_CUDA(cp(tr->eigvec, L.eigvec, bh * d * re * 4));
+    }
     SPR_CUDA(cp(tr->key_init, L.key_init, bh * Gk * 4));
     SPR_CUDA(cp(tr->key_centroids, L.C, bh * Gk * d * 4));
     SPR_CUDA(cp(tr->query_init, L.query_init, bh * Gq * 4));

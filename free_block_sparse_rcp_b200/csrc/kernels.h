@@ -35,6 +35,7 @@ size_t route_select_smem(int Gq, int Gk);
 cudaError_t launch_route_select(const float* mass, int BH, int N, int Gq, int Gk, const int* qoff,
                                 const int* koff, float density, int P, const Causal& cz, int* order,
                                 unsigned char* route, float* rho_exec, double* alpha, cudaStream_t st);
+cudaError_t launch_identity(float* A, int d, cudaStream_t st);
 cudaError_t launch_block_mask(const unsigned char* route, int BH, int N, int Gq, int Gk, int blk,
                               const int* perm_q, const int* label_q, const int* perm_k, const int* label_k,
                               unsigned char* bmask, cudaStream_t st);

@@ -585,6 +585,17 @@ cudaError_t launch_route_select(const float* mass, int BH, int N, int Gq, int Gk
   return cudaGetLastError();
 }
 
+// Identity matrix (d x d, fp32): the coordinate map of the semantic-grouping baseline.
+__global__ void k_identity(float* __restrict__ A, int d) {
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < d * d; e += gridDim.x * blockDim.x)
+    A[e] = (e / d == e % d) ? 1.f : 0.f;
+}
+
+cudaError_t launch_identity(float* A, int d, cudaStream_t st) {
+  k_identity<<<ceil_div(d * d, 256), 256, 0, st>>>(A, d);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_block_mask(const unsigned char* route, int BH, int N, int Gq, int Gk, int blk,
                               const int* perm_q, const int* label_q, const int* perm_k, const int* label_k,
                               unsigned char* bmask, cudaStream_t st) {

@@ -94,6 +94,12 @@ typedef struct {
                               [0, n_frames); a violation is recorded as device error 5 and leaves
                               the outputs unspecified.  Needs N <= 65535 (32-bit cell costs).     */
   int n_frames;            /* with frame_id: number of frames, 1..64; ignored without frame_id     */
+  int partition_mode;      /* 0: response-coupled partition (the method);
+                              1: the semantic-grouping baseline of the pages' comparison (keys and
+                              queries clustered separately on their raw vectors, same k-means
+                              rules, seed streams, centroids, route and layout).  In mode 1 the
+                              trace's sample_idx, metric, eigval, eigvec and key_coords are not
+                              written.                                                            */
 } sparsepr_params;
 
 /* Optional debug copies of partition intermediates (any pointer may be NULL). */

@@ -55,7 +55,9 @@ def _lse_close(got, ref, tol):
 def stage_checks(pd, qb, kb, vb, out, heads, rows=None, check_kmeans=True, frames=None):
     """Per-stage parity of heads `heads` (flattened b*H + h).  rows: number of sampled
     query rows for the attention / reconstruction checks (None = all).  frames: frame of
-    each token for a frame-causal call (None = no mask)."""
+    each token for a frame-causal call (None = no mask).  pd["partition_mode"] == 1: the
+    semantic-grouping baseline (both k-means on the raw rows; no metric or eigen stage)."""
+    semantic = pd.get("partition_mode", 0) == 1
     op = oracle_params(pd)
     B, H, N, d = pd["B"], pd["H"], pd["N"], pd["d"]
     s = op.eff_scale(d)
@@ -66,6 +68,16 @@ def stage_checks(pd, qb, kb, vb, out, heads, rows=None, check_kmeans=True, frame
     for bh in heads:
         b, h = divmod(bh, H)
         q, k, v = to_f64(qb[b, h]), to_f64(kb[b, h]), to_f64(vb[b, h])
+        if semantic:
+            y_gpu = k   # the key k-means runs on the raw rows
+        else:
+            y_gpu = _metric_eigen_checks(pd, q, k, tr, bh, N)
+        _rest_checks(pd, op, q, k, v, s, tr, ptr, out, bh, b, h, y_gpu, N, T, rng, rows, check_kmeans, frames,
+                     semantic)
+
+
+def _metric_eigen_checks(pd, q, k, tr, bh, N):
+    if True:
         # --- a1/a2: sample and metric
         idx = O.sample_queries(N, pd["n_samples"], pd["seed"], bh)
         np.testing.assert_array_equal(_np(tr["sample_idx"][bh]), idx)
@@ -86,6 +98,12 @@ def stage_checks(pd, qb, kb, vb, out, heads, rows=None, check_kmeans=True, frame
         y_gpu = _np(tr["key_coords"][bh]).astype(np.float64)
         y_ref = O.key_coords(k, lam_gpu, u_gpu)
         assert np.abs(y_gpu - y_ref).max() <= 1e-5 * np.abs(y_ref).max()
+    return y_gpu
+
+
+def _rest_checks(pd, op, q, k, v, s, tr, ptr, out, bh, b, h, y_gpu, N, T, rng, rows, check_kmeans, frames,
+                 semantic):
+    if True:
         # --- a5: key k-means on the device coordinates
         kinit = O.kmeans_init(N, pd["n_kgroups"], pd["seed"], bh, O.STREAM_KEY_KMEANS)
         np.testing.assert_array_equal(_np(tr["key_init"][bh]), kinit)
@@ -106,6 +124,7 @@ def stage_checks(pd, qb, kb, vb, out, heads, rows=None, check_kmeans=True, frame
         z_gpu = _np(tr["query_coords"][bh]).astype(np.float64)
         z_ref = O.query_coords(q, c_gpu, s)
         assert np.abs(z_gpu - z_ref).max() <= 2e-5 * max(1.0, np.abs(z_ref).max())
+        zk = q if semantic else z_gpu   # the query k-means runs on the raw rows in the baseline
         # --- a8: query k-means on the device coordinates
         qinit = O.kmeans_init(N, pd["n_qgroups"], pd["seed"], bh, O.STREAM_QUERY_KMEANS)
         np.testing.assert_array_equal(_np(tr["query_init"][bh]), qinit)
@@ -113,7 +132,7 @@ def stage_checks(pd, qb, kb, vb, out, heads, rows=None, check_kmeans=True, frame
         if check_kmeans:
             iters = [_np(tr["query_label_iters"][t, bh]).astype(np.int64) for t in range(T)]
             np.testing.assert_array_equal(iters[-1], lq)
-            teacher_forced_kmeans(z_gpu, qinit, iters, f"queries head {bh}")
+            teacher_forced_kmeans(zk, qinit, iters, f"queries head {bh}")
         pq, qo = O.group_permutation(lq, pd["n_qgroups"])
         np.testing.assert_array_equal(_np(out["perm_q"][bh]), pq)
         np.testing.assert_array_equal(_np(out["qoff"][bh]), qo)
