@@ -168,12 +168,7 @@ def run_cuda(args):
     import free_block_sparse_rcp_b200 as spr
     from synth import generate, workload
 
-    over = {}
-    if args.heads:
-        over["H"] = args.heads
-    if args.density:
-        over["density"] = args.density
-    w = workload(args.workload, **over)
+    w = bench_workload(args)
     pd = dict(B=w.B, H=w.H, N=w.N, d=w.d, block=w.block, density=w.density, n_kgroups=w.n_kgroups,
               n_qgroups=w.n_qgroups, n_samples=w.n_samples, n_probes=w.n_probes, eig_rank=w.eig_rank,
               sub_rank=w.sub_rank, kmeans_iters=w.kmeans_iters, ridge_lambda=w.ridge_lambda, seed=0,
@@ -391,6 +386,22 @@ def run_cuda(args):
         print(json.dumps(line), flush=True)
 
 
+def bench_workload(args, heads=True):
+    """The workload of this run with the command line's overrides."""
+    from synth import workload
+    over = {}
+    if heads and getattr(args, "heads", 0):
+        over["H"] = args.heads
+    if getattr(args, "density", 0.0):
+        over["density"] = args.density
+    if getattr(args, "groups", 0):
+        over.update(n_kgroups=args.groups, n_qgroups=args.groups)
+    elif getattr(args, "workload", WORKLOAD) == "long":
+        # the kernels take at most 128 groups; the 108,000-token workload runs at that limit
+        over.update(n_kgroups=128, n_qgroups=128)
+    return workload(getattr(args, "workload", WORKLOAD), **over)
+
+
 def partition_diagnostics(part, Q, K, o_sparse, o_dense, p, frames=None, heads=(0, 1), groups=16, mass=0.9):
     """Measurements of the partition on a few heads (torch on the device; reporting only).
 
@@ -548,7 +559,7 @@ def run_reference(args):
     if rank != 0:
         return
     from synth import workload
-    w = workload(args.workload)
+    w = bench_workload(args, heads=False)
     for _ in range(args.warmup):
         oracle_sample(workload("tiny"), rows_frac=1.0)   # warms numpy / BLAS; not timed
     vals, spent = [], 0.0
@@ -576,8 +587,10 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--workload", default=WORKLOAD, choices=["wan", "world"],
-                    help="wan: the 32,760-token call (default); world: the frame-causal rollout")
+    ap.add_argument("--workload", default=WORKLOAD, choices=["wan", "world", "long"],
+                    help="wan: the 32,760-token call (default); world: the frame-causal rollout; "
+                         "long: 108,000 tokens x 24 heads with a per-frame drift (128 groups)")
+    ap.add_argument("--groups", type=int, default=0, help="override the K/V and query group counts")
     ap.add_argument("--partition", default="coupled", choices=["coupled", "semantic"],
                     help="coupled: the method; semantic: the semantic-grouping baseline of the pages")
     ap.add_argument("--density", type=float, default=0.0, help="override the workload's target density")

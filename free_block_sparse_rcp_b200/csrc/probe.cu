@@ -123,20 +123,25 @@ __global__ void __launch_bounds__(128) k_probe_combine(const float* __restrict__
 // Residual subspace + ridge fit, one CTA per head (fp64 arithmetic).
 //   R = O_dense - O_sparse (P x D); top eigenpairs u_i, sigma_i^2 of the Gram R R^T
 //   (Householder + multisection + inverse iteration); v_i = R^T u_i normalised (zero when
-//   sigma_i <= 1e-6 sigma_0); Y = R V_r; centred dual ridge
-//   W = Xc^T (Xc Xc^T + lam I)^-1 Yc, b = ybar - xbar W.
+//   sigma_i <= 1e-6 sigma_0); Y = R V_r; the affine map works inside the subspace: with
+//   X = O_sparse V_r (the probes' sparse outputs in the subspace), centred dual ridge
+//   W_sub = Xc^T (Xc Xc^T + lam I)^-1 Yc, b = ybar - xbar W_sub; exported as W = V_r W_sub
+//   (so a row's residual coordinates are x W = (x V_r) W_sub).
 // grid = BH, block = FIT_THREADS.
 // ---------------------------------------------------------------------------
 constexpr int FIT_THREADS = 1024;
 
 template <int D>
 struct FitLayout {
-  // doubles: G [PR][PR+1] (Gram -> Cholesky -> W), Z [PR][Rk+1], lam [64], eigen scratch,
-  // X = max(3 PR Rk (solver scratch), D Rk + PR Rk (V_r, Y)), xbar [D], ybar, bsub, cs [64 each];
-  // then floats Rm, Xm [PR][D]
+  // doubles: G [PR][PR+1] (Gram -> Cholesky -> W_sub), Z [PR][Rk+1], lam [64], eigen scratch,
+  // X = max(3 PR Rk (solver scratch), (2 D + 2 PR) Rk (V_r, Y, X V_r, W)), xbar [D], ybar,
+  // bsub, cs [64 each]; then floats Rm, Xm [PR][D]
+  __host__ __device__ static size_t xsize(int Rk) {
+    const size_t a = (size_t)3 * PR * Rk, b = (size_t)(2 * D + 2 * PR) * Rk;
+    return a > b ? a : b;
+  }
   static size_t doubles(int Rk) {
-    const size_t x = (size_t)3 * PR * Rk > (size_t)(D + PR) * Rk ? (size_t)3 * PR * Rk : (size_t)(D + PR) * Rk;
-    return (size_t)PR * (PR + 1) + (size_t)PR * (Rk + 1) + 64 + SymEigScratch<PR>::kDoubles + x + D + 3 * 64;
+    return (size_t)PR * (PR + 1) + (size_t)PR * (Rk + 1) + 64 + SymEigScratch<PR>::kDoubles + xsize(Rk) + D + 3 * 64;
   }
   static size_t bytes(int Rk) { return doubles(Rk) * 8 + (size_t)2 * PR * D * 4; }
 };
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
   extern __shared__ __align__(16) unsigned char smem[];
   constexpr int LDP = PR + 1;
   const int ldz = Rk + 1;
-  const size_t xsz = (size_t)3 * PR * Rk > (size_t)(D + PR) * Rk ? (size_t)3 * PR * Rk : (size_t)(D + PR) * Rk;
+  const size_t xsz = FitLayout<D>::xsize(Rk);
   double* G = reinterpret_cast<double*>(smem);    // [PR][LDP]  Gram, later Cholesky, later W
   double* Z = G + PR * LDP;                        // [PR][Rk+1] eigenvectors of R R^T
   double* ev = Z + PR * ldz;                       // [64] eigenvalues, descending
@@ -159,7 +164,9 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
   double* X = esc + SymEigScratch<PR>::kDoubles;   // solver scratch, then V_r and Y
   double* Vr = X;                                  // [D][Rk]
   double* Y = Vr + D * Rk;                         // [PR][Rk] -> solution
-  double* xbar = X + xsz;                          // [D]
+  double* Xs = Y + PR * Rk;                        // [PR][Rk] probe sparse outputs in the subspace
+  double* Wd = Xs + PR * Rk;                       // [D][Rk] W = V_r W_sub
+  double* xbar = X + xsz;                          // [D] (the first Rk: mean of Xs)
   double* ybar = xbar + D;                         // [64]
   double* bsub = ybar + 64;                        // [64]
   double* cs = bsub + 64;                          // [64]
@@ -212,34 +219,39 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
   __syncthreads();
   for (int e = tid; e < D * Rk; e += nt) Vr[e] *= cs[e % Rk];
   __syncthreads();
-  // Y = R Vr, means
+  // Y = R Vr and Xs = X Vr (the probes' residuals and sparse outputs in the subspace), means
   for (int e = tid; e < P * Rk; e += nt) {
     const int p = e / Rk, j = e - p * Rk;
-    double s = 0.0;
-    for (int c = 0; c < D; ++c) s += (double)Rm[p * D + c] * Vr[c * Rk + j];
+    double s = 0.0, t = 0.0;
+    for (int c = 0; c < D; ++c) {
+      s += (double)Rm[p * D + c] * Vr[c * Rk + j];
+      t += (double)Xm[p * D + c] * Vr[c * Rk + j];
+    }
     Y[p * Rk + j] = s;
-  }
-  for (int c = tid; c < D; c += nt) {
-    double s = 0.0;
-    for (int p = 0; p < P; ++p) s += (double)Xm[p * D + c];
-    xbar[c] = s / P;
+    Xs[p * Rk + j] = t;
   }
   __syncthreads();
   for (int j = tid; j < Rk; j += nt) {
-    double s = 0.0;
-    for (int p = 0; p < P; ++p) s += Y[p * Rk + j];
+    double s = 0.0, t = 0.0;
+    for (int p = 0; p < P; ++p) {
+      s += Y[p * Rk + j];
+      t += Xs[p * Rk + j];
+    }
     ybar[j] = s / P;
+    xbar[j] = t / P;
   }
   __syncthreads();
   for (int e = tid; e < P * Rk; e += nt) {
     const int p = e / Rk, j = e - p * Rk;
     Y[p * Rk + j] -= ybar[j];
+    Xs[p * Rk + j] -= xbar[j];
   }
-  // A = Xc Xc^T + lam I  (into G)
+  __syncthreads();
+  // A = Xc Xc^T + lam I  (into G), Xc = centred Xs
   for (int e = tid; e < P * P; e += nt) {
     const int i = e / P, j = e - i * P;
     double s = 0.0;
-    for (int c = 0; c < D; ++c) s += ((double)Xm[i * D + c] - xbar[c]) * ((double)Xm[j * D + c] - xbar[c]);
+    for (int c = 0; c < Rk; ++c) s += Xs[i * Rk + c] * Xs[j * Rk + c];
     G[i * LDP + j] = s + (i == j ? lam : 0.0);
   }
   __syncthreads();
@@ -270,22 +282,29 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
     }
   }
   __syncthreads();
-  // W = Xc^T Z (D x Rk, D * Rk <= PR * (PR + 1)) kept in the Cholesky region, b = ybar - xbar W
-  double* Wd = G;
-  for (int e = tid; e < D * Rk; e += nt) {
-    const int c = e / Rk, j = e - c * Rk;
+  // W_sub = Xc^T Z (Rk x Rk, in the Cholesky region), b = ybar - xbar W_sub
+  double* Ws = G;
+  for (int e = tid; e < Rk * Rk; e += nt) {
+    const int i = e / Rk, j = e - i * Rk;
     double s = 0.0;
-    for (int p = 0; p < P; ++p) s += ((double)Xm[p * D + c] - xbar[c]) * Y[p * Rk + j];
-    Wd[e] = s;
-    W_out[(size_t)bh * D * Rk + e] = (float)s;
-    Vr_out[(size_t)bh * D * Rk + e] = (float)Vr[c * Rk + j];
+    for (int p = 0; p < P; ++p) s += Xs[p * Rk + i] * Y[p * Rk + j];
+    Ws[e] = s;
   }
   __syncthreads();
   for (int j = tid; j < Rk; j += nt) {
     double s = 0.0;
-    for (int c = 0; c < D; ++c) s += xbar[c] * Wd[c * Rk + j];
+    for (int i = 0; i < Rk; ++i) s += xbar[i] * Ws[i * Rk + j];
     bsub[j] = ybar[j] - s;
     if (bsub_out) bsub_out[(size_t)bh * Rk + j] = (float)bsub[j];
+  }
+  // W = V_r W_sub (D x Rk): residual coordinates of a row are x W = (x V_r) W_sub
+  for (int e = tid; e < D * Rk; e += nt) {
+    const int c = e / Rk, j = e - c * Rk;
+    double s = 0.0;
+    for (int i = 0; i < Rk; ++i) s += Vr[c * Rk + i] * Ws[i * Rk + j];
+    Wd[e] = s;
+    W_out[(size_t)bh * D * Rk + e] = (float)s;
+    Vr_out[(size_t)bh * D * Rk + e] = (float)Vr[c * Rk + j];
   }
   __syncthreads();
   for (int c = tid; c < D; c += nt) {

@@ -47,6 +47,19 @@ __device__ __forceinline__ int sturm_count_f32(const float* d, const float* e2, 
   return c;
 }
 
+// the same count in fp64 (for the last steps of the brackets)
+__device__ __forceinline__ int sturm_count_f64(const double* d, const double* e2, int n, double x, double pivmin) {
+  double q = d[0] - x;
+  if (fabs(q) < pivmin) q = -pivmin;
+  int c = q <= 0.0;
+  for (int i = 1; i < n; ++i) {
+    q = (d[i] - x) - e2[i - 1] / q;
+    if (fabs(q) < pivmin) q = -pivmin;
+    c += q <= 0.0;
+  }
+  return c;
+}
+
 // Solve (T - mu I) x = y in place (y[i * ys]), T = tridiag(e, d, e); u: 3n doubles of scratch.
 // Single thread.  Pivots smaller than tol are replaced by +-tol.
 __device__ inline void tri_shifted_solve(const double* d, const double* e, int n, double mu, double tol, double* y,
@@ -225,11 +238,13 @@ __device__ inline void sym_top_eigen(double* A, int R, double* Z, int ldz, doubl
       misc[1] = hi + pad;
       misc[2] = tn;
       misc[3] = fmax((double)FLT_MIN * fmax(1.0, me2), 1e-30 * tn);
+      misc[4] = me2;
     }
   }
   __syncthreads();
   const double tnorm = misc[2];
   const float pivmin32 = (float)misc[3];
+  const double pivmin64 = fmax(DBL_MIN * fmax(1.0, misc[4]), 1e-300);
   // ---- 2. eigenvalues (j-th largest = ascending index N-1-j)
   for (int j = warp; j < R; j += nw) {
     const int t = N - 1 - j;
@@ -243,6 +258,24 @@ __device__ inline void sym_top_eigen(double* A, int R, double* Z, int ldz, doubl
       const double xhi = __shfl_sync(0xffffffffu, x, lo < 31 ? lo + 1 : 31);
       if (lo >= 0) a = xlo;
       if (lo < 31) b = xhi;
+    }
+    // fp64 steps: an eigenvalue far below ||T|| (a weak direction) needs a bracket well
+    // inside its gaps to its neighbours, which the fp32 count cannot resolve; widen the fp32
+    // bracket by its own rounding first
+    {
+      const double pad = 4e-6 * tnorm + 1e-30;
+      a -= pad;
+      b += pad;
+      for (int it = 0; it < 4; ++it) {
+        if (b - a <= 4.0 * DBL_EPSILON * fmax(fabs(a), fabs(b)) + pivmin64 + 1e-300) break;
+        const double x = a + (b - a) * (double)(lane + 1) * (1.0 / 33.0);
+        const unsigned below = __ballot_sync(0xffffffffu, sturm_count_f64(d, e2, N, x, pivmin64) <= t);
+        const int lo = below ? 31 - __clz(below) : -1;
+        const double xlo = __shfl_sync(0xffffffffu, x, lo < 0 ? 0 : lo);
+        const double xhi = __shfl_sync(0xffffffffu, x, lo < 31 ? lo + 1 : 31);
+        if (lo >= 0) a = xlo;
+        if (lo < 31) b = xhi;
+      }
     }
     if (lane == 0) lam[j] = 0.5 * (a + b);
   }

@@ -575,14 +575,19 @@ class ProbeFit:
 def fit_from_probes(probe_idx, o_dense, o_sparse, lse_dense, lse_sparse, rank: int,
                     lam: float) -> ProbeFit:
     """R_P = O_dense - O_sparse on the probes; V_r = top singular subspace of R_P;
-    Y = R_P V_r; ridge fit Y ~ b + x W with x = the probe rows' full sparse output
-    (the correction maps the sparse output into the residual subspace, abstract:
-    "affine correction from the sparse output within the output subspace observed
-    in the probe residuals")."""
+    Y = R_P V_r; ridge fit Y ~ b + (x V_r) W_sub with x = the probe rows' sparse output.
+
+    READING: the affine map works inside the subspace on both sides (abstract: "affine
+    correction from the sparse output within the output subspace observed in the probe
+    residuals"; gist 2.B: the subspace keeps the correction away from directions the
+    probes did not observe): its input is the sparse output projected on V_r, so the fit
+    has r + 1 parameters per direction for the P probes instead of d + 1.  Returned as
+    w = V_r W_sub (d x r), so a row's residual coordinates are x w."""
     r_p = np.asarray(o_dense, np.float64) - np.asarray(o_sparse, np.float64)
     vr, sig = probe_subspace(r_p, rank)
     y = r_p @ vr
-    w, b = ridge_fit(o_sparse, y, lam)
+    w_sub, b = ridge_fit(np.asarray(o_sparse, np.float64) @ vr, y, lam)
+    w = vr @ w_sub
     return ProbeFit(probe_idx=np.asarray(probe_idx), o_dense=np.asarray(o_dense, np.float64),
                     o_sparse=np.asarray(o_sparse, np.float64), lse_dense=np.asarray(lse_dense),
                     lse_sparse=np.asarray(lse_sparse), residual=r_p, vr=vr, sigma=sig, w=w, b=b,

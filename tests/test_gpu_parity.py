@@ -176,21 +176,42 @@ def _rest_checks(pd, op, q, k, v, s, tr, ptr, out, bh, b, h, y_gpu, N, T, rng, r
         assert rel_l2(od_gpu, od_ref) <= 1e-5 and rel_l2(os_gpu, os_ref) <= 1e-5
         _lse_close(_np(ptr["probe_lse_dense"][bh]), ld_ref, 1e-4)
         _lse_close(_np(ptr["probe_lse_sparse"][bh]), ls_ref, 1e-4)
-        # --- a14/a15: subspace + ridge (basis-free quantities: B = W V_r^T, b V_r^T)
-        fit = O.fit_from_probes(pidx, od_ref, os_ref, ld_ref, ls_ref, pd["sub_rank"], op.ridge_lambda)
+        # --- a14: the device's residual subspace (from its own probe outputs): singular values
+        # against the oracle's, an orthonormal basis of an invariant subspace of R^T R.  The
+        # basis itself is not compared: its trailing directions are weak (down to ~3e-4 of
+        # the largest at rank 32) and can rotate with the last bits of the inputs.
+        r_gpu = od_gpu - os_gpu
+        fit_dev = O.fit_from_probes(pidx, od_gpu, os_gpu, ld_ref, ls_ref, pd["sub_rank"], op.ridge_lambda)
+        sig_gpu = _np(ptr["sigma"][bh]).astype(np.float64)
+        s0 = max(fit_dev.sigma[0], 1e-30)
+        assert np.abs(sig_gpu - fit_dev.sigma).max() <= 1e-5 * s0 + 1e-9
         b_gpu = _np(out["b_full"][bh]).astype(np.float64)
         vr_gpu = _np(out["Vr"][bh]).astype(np.float64)
         w_gpu = _np(out["W"][bh]).astype(np.float64)
         bm_gpu = _np(out["Bmat"][bh]).astype(np.float64)
+        assert np.all(vr_gpu[:, sig_gpu == 0] == 0)
+        # v_j = R^T u_j / sigma_j magnifies the error of u_j by sigma_0 / sigma_j, so the basis
+        # is checked on the directions above 1e-3 sigma_0 (the weaker ones carry targets below
+        # 1e-3 of the largest and barely move the correction)
+        # (and above 1e-6 absolute: below that R is the fp32 rounding of the probe outputs)
+        keep = sig_gpu > max(1e-3 * s0, 1e-6)
+        if keep.any():
+            vk = vr_gpu[:, keep]
+            assert np.abs(vk.T @ vk - np.eye(vk.shape[1])).max() <= 1e-4
+            inv = r_gpu.T @ (r_gpu @ vk) - vk * sig_gpu[keep] ** 2
+            assert np.abs(inv).max() <= 1e-5 * s0 ** 2
+        # --- a15: the ridge given the device's subspace (exact up to fp32 rounding)
+        w_sub, b_sub = O.ridge_fit(os_gpu @ vr_gpu, r_gpu @ vr_gpu, op.ridge_lambda)
+        bfull_ref = vr_gpu @ b_sub
+        bmat_ref = vr_gpu @ w_sub @ vr_gpu.T
         np.testing.assert_allclose(bm_gpu, w_gpu @ vr_gpu.T, atol=1e-5 * max(1, np.abs(bm_gpu).max()))
-        # the fit's effect on the output rows: corrections b + x B of the two fits
-        # differ by at most a fifth of the reconstructed-output budget (2e-3 of ||O||)
         corr_gpu = b_gpu + o_ref @ bm_gpu
-        corr_ref = fit.b_full + o_ref @ fit.bmat
+        corr_ref = bfull_ref + o_ref @ bmat_ref
         dc = np.linalg.norm(corr_gpu - corr_ref)
-        assert dc <= 2e-3 * np.linalg.norm(o_ref), (dc, np.linalg.norm(corr_ref), np.linalg.norm(o_ref))
-        # --- a16: reconstruction against the oracle's reconstruction from its own fit
-        o_rows_ref = o_ref + fit.b_full + (o_ref @ fit.w) @ fit.vr.T
+        assert dc <= 1e-4 * np.linalg.norm(o_ref) + 1e-3 * np.linalg.norm(corr_ref), \
+            (dc, np.linalg.norm(corr_ref), np.linalg.norm(o_ref))
+        # --- a16: reconstruction against the oracle's correction with the device's fit
+        o_rows_ref = o_ref + bfull_ref + o_ref @ bmat_ref
         slot = {int(i): j for j, i in enumerate(pidx)}
         for r_, i in enumerate(sel):
             if int(i) in slot:

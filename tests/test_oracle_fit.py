@@ -68,15 +68,16 @@ def test_subspace_rank_deficient_is_zero_columns():
 
 
 def test_correction_exact_for_planted_affine_residual():
-    # if the residual is exactly b + x B with B of rank r inside the probes'
-    # residual span, the corrected output equals the dense one on every row
+    # if the residual is exactly an affine map inside the probes' residual span,
+    # R = (b + (x V) W) V^T with V the span's basis, the corrected output equals the
+    # dense one on every row
     rng = np.random.default_rng(5)
     n, d, r, p = 400, 12, 3, 64
     basis = np.linalg.qr(rng.standard_normal((d, r)))[0]
     b_sub = rng.standard_normal(r)
-    w_sub = rng.standard_normal((d, r))
+    w_sub = rng.standard_normal((r, r))
     o_sparse = rng.standard_normal((n, d))
-    o_dense = o_sparse + (b_sub + o_sparse @ w_sub) @ basis.T
+    o_dense = o_sparse + (b_sub + (o_sparse @ basis) @ w_sub) @ basis.T
     pidx = rng.choice(n, p, replace=False)
     fit = O.fit_from_probes(pidx, o_dense[pidx], o_sparse[pidx], np.zeros(p), np.zeros(p), r, 1e-12)
     np.testing.assert_allclose(fit.vr @ fit.vr.T, basis @ basis.T, atol=1e-9)
@@ -84,6 +85,27 @@ def test_correction_exact_for_planted_affine_residual():
     np.testing.assert_allclose(out, o_dense, atol=1e-7)
     np.testing.assert_allclose(fit.bmat, fit.w @ fit.vr.T)
     np.testing.assert_allclose(out[pidx], o_dense[pidx], atol=0)
+
+
+def test_fit_ignores_sparse_output_outside_the_subspace():
+    # the map's input is the sparse output projected on the residual subspace: adding
+    # to x any component orthogonal to V_r changes neither the fit nor the correction
+    rng = np.random.default_rng(6)
+    n, d, r, p = 300, 10, 3, 48
+    basis = np.linalg.qr(rng.standard_normal((d, d)))[0]
+    v, perp = basis[:, :r], basis[:, r:]
+    o_sparse = rng.standard_normal((n, d))
+    o_dense = o_sparse + (rng.standard_normal(r) + (o_sparse @ v) @ rng.standard_normal((r, r))) @ v.T
+    o_dense += 1e-3 * rng.standard_normal((n, d)) @ v @ v.T
+    pidx = rng.choice(n, p, replace=False)
+    fit = O.fit_from_probes(pidx, o_dense[pidx], o_sparse[pidx], np.zeros(p), np.zeros(p), r, 1e-2)
+    shift = rng.standard_normal((n, d - r)) @ perp.T
+    fit2 = O.fit_from_probes(pidx, o_dense[pidx] + shift[pidx], o_sparse[pidx] + shift[pidx], np.zeros(p),
+                             np.zeros(p), r, 1e-2)
+    np.testing.assert_allclose(fit2.vr @ fit2.vr.T, fit.vr @ fit.vr.T, atol=1e-9)
+    np.testing.assert_allclose(fit2.b_full, fit.b_full, atol=1e-9)
+    np.testing.assert_allclose(fit2.bmat, fit.bmat, atol=1e-9)
+    np.testing.assert_allclose(shift @ fit.bmat, 0, atol=1e-9)
 
 
 def test_probe_rows_take_exact_dense_output():
