@@ -516,6 +516,18 @@ def pick_probes(perm_q, q_offsets, n_probes: int, seed: int, bh: int) -> np.ndar
     return np.array(out, np.int64)
 
 
+def probe_weights(q_offsets, n_probes: int) -> np.ndarray:
+    """Weights of the probe rows for the weighted fit (ai-feeds: a "weighted" affine fit).
+
+    READING: inverse inclusion probability: a probe of query group a stands for the
+    n_a / alloc_a tokens of its group (alloc_a = its group's probe count), in the probe
+    order of pick_probes (group order); normalised to mean 1 so lam keeps its scale."""
+    sizes = np.diff(np.asarray(q_offsets))
+    alloc = probe_allocation(sizes, n_probes)
+    w = np.concatenate([np.full(int(alloc[a]), sizes[a] / alloc[a]) for a in range(len(sizes)) if alloc[a] > 0])
+    return w * (w.size / w.sum())
+
+
 def omitted_mass(lse_sparse, lse_dense) -> np.ndarray:
     """Share of the dense softmax mass that falls on skipped keys: 1 - Z_ret/Z."""
     return 1.0 - np.exp(np.asarray(lse_sparse) - np.asarray(lse_dense))
@@ -538,19 +550,23 @@ def probe_subspace(r_p, rank: int, rel_tol: float = 1e-6):
     return v, sig
 
 
-def ridge_fit(x, y, lam: float):
+def ridge_fit(x, y, lam: float, weights=None):
     """Ridge-regularised affine fit y ~ b + x W (gist 2.B: R ~ b + xB, ridge).
 
     READINGS: the intercept is not penalised (solve on probe-centred x and y,
-    b = mean(y) - mean(x) W); lam is absolute; uniform probe weights.  Dual form
+    b = mean(y) - mean(x) W); lam is absolute; uniform probe weights unless
+    ``weights`` are given (then weighted means and rows scaled by sqrt(weight): the
+    minimiser of sum_i w_i ||y_i - b - x_i W||^2 + lam ||W||^2).  Dual form
     W = Xc^T (Xc Xc^T + lam I)^-1 Yc, identical to the primal
     (Xc^T Xc + lam I)^-1 Xc^T Yc."""
     x = np.asarray(x, np.float64)
     y = np.asarray(y, np.float64)
-    xm = x.mean(axis=0)
-    ym = y.mean(axis=0)
-    xc = x - xm
-    yc = y - ym
+    wt = np.ones(x.shape[0]) if weights is None else np.asarray(weights, np.float64)
+    xm = (wt[:, None] * x).sum(axis=0) / wt.sum()
+    ym = (wt[:, None] * y).sum(axis=0) / wt.sum()
+    sq = np.sqrt(wt)[:, None]
+    xc = (x - xm) * sq
+    yc = (y - ym) * sq
     w = xc.T @ np.linalg.solve(xc @ xc.T + lam * np.eye(x.shape[0]), yc)
     b = ym - xm @ w
     return w, b
@@ -573,7 +589,7 @@ class ProbeFit:
 
 
 def fit_from_probes(probe_idx, o_dense, o_sparse, lse_dense, lse_sparse, rank: int,
-                    lam: float) -> ProbeFit:
+                    lam: float, weights=None) -> ProbeFit:
     """R_P = O_dense - O_sparse on the probes; V_r = top singular subspace of R_P;
     Y = R_P V_r; ridge fit Y ~ b + (x V_r) W_sub with x = the probe rows' sparse output.
 
@@ -586,7 +602,7 @@ def fit_from_probes(probe_idx, o_dense, o_sparse, lse_dense, lse_sparse, rank: i
     r_p = np.asarray(o_dense, np.float64) - np.asarray(o_sparse, np.float64)
     vr, sig = probe_subspace(r_p, rank)
     y = r_p @ vr
-    w_sub, b = ridge_fit(np.asarray(o_sparse, np.float64) @ vr, y, lam)
+    w_sub, b = ridge_fit(np.asarray(o_sparse, np.float64) @ vr, y, lam, weights)
     w = vr @ w_sub
     return ProbeFit(probe_idx=np.asarray(probe_idx), o_dense=np.asarray(o_dense, np.float64),
                     o_sparse=np.asarray(o_sparse, np.float64), lse_dense=np.asarray(lse_dense),
@@ -621,6 +637,7 @@ class Params:
     scale: float = 0.0          # 0 -> 1/sqrt(d)
     seed: int = 0
     block: int = 64
+    fit_weighted: bool = False   # probe weights n_a / alloc_a in the ridge (probe_weights)
 
     def eff_scale(self, d: int) -> float:
         return self.scale if self.scale > 0 else 1.0 / math.sqrt(d)
@@ -792,7 +809,8 @@ def probe_fit_head(q, k, v, part_label_q, part_label_k, route, perm_q, q_offsets
     pidx = pick_probes(perm_q, q_offsets, p.n_probes, p.seed, bh)
     o_d, l_d = attention(q[pidx], k, v, s, mask=None if frames is None else causal_mask(frames, pidx))
     o_s, l_s = sparse_attention(q, k, v, s, route, part_label_q, part_label_k, rows=pidx, frames=frames)
-    return fit_from_probes(pidx, o_d, o_s, l_d, l_s, p.sub_rank, p.ridge_lambda)
+    wts = probe_weights(q_offsets, p.n_probes) if p.fit_weighted else None
+    return fit_from_probes(pidx, o_d, o_s, l_d, l_s, p.sub_rank, p.ridge_lambda, wts)
 
 
 @dataclass

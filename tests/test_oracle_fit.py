@@ -167,3 +167,34 @@ def test_pick_probes_stratified_and_reproducible():
         mem = perm[off[a]:off[a + 1]]
         want += [int(mem[i]) for i in O.draw_without_replacement(g, len(mem), int(alloc[a]))]
     assert list(pidx) == want
+
+
+def test_weighted_ridge_equals_replicated_rows():
+    # integer weights act as replicated probe rows: with weights normalised to mean 1,
+    # the weighted fit equals the plain fit on the replicated rows with lam * sum(w) / P
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((12, 4))
+    y = rng.standard_normal((12, 2))
+    rep = rng.integers(1, 4, 12)
+    wn = rep * (12 / rep.sum())
+    w1, b1 = O.ridge_fit(x, y, 0.3, wn)
+    w2, b2 = O.ridge_fit(np.repeat(x, rep, axis=0), np.repeat(y, rep, axis=0), 0.3 * rep.sum() / 12)
+    np.testing.assert_allclose(w1, w2, atol=1e-10)
+    np.testing.assert_allclose(b1, b2, atol=1e-10)
+    # equal weights are the plain fit
+    w3, b3 = O.ridge_fit(x, y, 0.3, np.ones(12))
+    w4, b4 = O.ridge_fit(x, y, 0.3)
+    np.testing.assert_allclose(w3, w4, atol=1e-12)
+    np.testing.assert_allclose(b3, b4, atol=1e-12)
+
+
+def test_probe_weights_are_inverse_inclusion():
+    # groups of 10, 3 and 50 tokens with 4 probes: allocation 1, 1, 2 (water-filling)
+    qoff = np.array([0, 10, 13, 63])
+    alloc = O.probe_allocation(np.diff(qoff), 4)
+    w = O.probe_weights(qoff, 4)
+    raw = np.concatenate([np.full(a, n / a) for n, a in zip(np.diff(qoff), alloc) if a > 0])
+    np.testing.assert_allclose(w, raw * (raw.size / raw.sum()))
+    assert abs(w.mean() - 1.0) < 1e-12
+    # a probe of the big group stands for more tokens than one of the small group
+    assert w[-1] > w[1]
