@@ -30,7 +30,8 @@ class Params(ctypes.Structure):
                 ("n_qgroups", ctypes.c_int), ("n_samples", ctypes.c_int), ("n_probes", ctypes.c_int),
                 ("eig_rank", ctypes.c_int), ("sub_rank", ctypes.c_int), ("kmeans_iters", ctypes.c_int),
                 ("ridge_lambda", ctypes.c_float), ("scale", ctypes.c_float), ("seed", ctypes.c_ulonglong),
-                ("frame_id", _vp), ("n_frames", ctypes.c_int), ("partition_mode", ctypes.c_int)]
+                ("frame_id", _vp), ("n_frames", ctypes.c_int), ("partition_mode", ctypes.c_int),
+                ("fit_weighted", ctypes.c_int)]
 
     @property
     def BH(self) -> int:
@@ -49,14 +50,15 @@ class Params(ctypes.Structure):
     @classmethod
     def make(cls, B, H, N, d, *, block, density, n_kgroups, n_qgroups, n_samples, n_probes, eig_rank,
              sub_rank, kmeans_iters, ridge_lambda=1e-2, scale=0.0, seed=0, frame_id=None, n_frames=0,
-             partition_mode=0):
+             partition_mode=0, fit_weighted=0):
         """frame_id: optional int32 device tensor [N] (frame-causal masking, kept alive by the
         caller for as long as the params are used)."""
         fid = None if frame_id is None else frame_id.data_ptr()
         return cls(B=B, H=H, N=N, d=d, block=block, density=density, n_kgroups=n_kgroups,
                    n_qgroups=n_qgroups, n_samples=n_samples, n_probes=n_probes, eig_rank=eig_rank,
                    sub_rank=sub_rank, kmeans_iters=kmeans_iters, ridge_lambda=ridge_lambda, scale=scale,
-                   seed=seed, frame_id=fid, n_frames=n_frames, partition_mode=partition_mode)
+                   seed=seed, frame_id=fid, n_frames=n_frames, partition_mode=partition_mode,
+                   fit_weighted=fit_weighted)
 
 
 class PartitionTrace(ctypes.Structure):

@@ -175,6 +175,8 @@ sparsepr_status check_params(const sparsepr_params* p) {
   if (p->kmeans_iters < 1 || p->kmeans_iters > 64) return failv(SPARSEPR_EINVAL, "kmeans_iters must be in [1, 64]", p->kmeans_iters);
   if (!(p->ridge_lambda > 0.f) || !isfinite(p->ridge_lambda)) return fail(SPARSEPR_EINVAL, "ridge_lambda must be > 0");
   if (!(p->scale >= 0.f) || !isfinite(p->scale)) return fail(SPARSEPR_EINVAL, "scale must be >= 0");
+  if (p->fit_weighted != 0 && p->fit_weighted != 1)
+    return failv(SPARSEPR_EINVAL, "fit_weighted must be 0 or 1", p->fit_weighted);
   if (p->partition_mode != 0 && p->partition_mode != 1)
     return failv(SPARSEPR_EINVAL, "partition_mode must be 0 (response-coupled) or 1 (semantic)", p->partition_mode);
   if (p->frame_id) {
@@ -408,7 +410,8 @@ sparsepr_status run_probe_fit(const sparsepr_params& p, const Layout& L, const v
   float* lss = at<float>(ws, L.lse_s);
   SPR_LAUNCH(launch_probe_combine(part_o, part_ml, BH, N, P, d, probe_od, osp, lsd, lss, st));
   SPR_LAUNCH(launch_probe_fit(probe_od, osp, BH, d, P, p.sub_rank, (double)p.ridge_lambda, Vr, W, bfull, Bmat,
-                              tr ? tr->sigma : nullptr, tr ? tr->b_sub : nullptr, st));
+                              tr ? tr->sigma : nullptr, tr ? tr->b_sub : nullptr, p.fit_weighted ? pgrp : nullptr,
+                              qoff, p.n_qgroups, st));
   if (tr) {
     if (tr->probe_o_sparse)
       SPR_CUDA(cudaMemcpyAsync(tr->probe_o_sparse, osp, (size_t)BH * P * d * 4, cudaMemcpyDeviceToDevice, st));

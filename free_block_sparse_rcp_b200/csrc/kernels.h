@@ -112,9 +112,10 @@ cudaError_t launch_probe_combine_splits(const float* part_o, const float* part_m
                                         cudaStream_t st);
 cudaError_t launch_probe_combine(const float* part_o, const float* part_ml, int BH, int N, int P, int D,
                                  float* o_dense, float* o_sparse, float* lse_d, float* lse_s, cudaStream_t st);
+// probe_grp / qoff: the weighted fit's probe groups and query group offsets (NULL: uniform)
 cudaError_t launch_probe_fit(const float* o_dense, const float* o_sparse, int BH, int D, int P, int Rk,
                              double lam, float* Vr, float* W, float* bfull, float* Bmat, float* sigma,
-                             float* bsub, cudaStream_t st);
+                             float* bsub, const int* probe_grp, const int* qoff, int Gq, cudaStream_t st);
 cudaError_t launch_reconstruct(const void* Os, int BH, int N, int D, int Rk, const float* W, const float* Vr,
                                const float* bfull, void* O, cudaStream_t st);
 cudaError_t launch_probe_scatter(const int* probe_idx, const float* o_dense, int BH, int N, int P, int D, void* O,

@@ -152,7 +152,8 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
                                                   double lam, float* __restrict__ Vr_out,
                                                   float* __restrict__ W_out, float* __restrict__ bfull_out,
                                                   float* __restrict__ Bmat, float* __restrict__ sigma_out,
-                                                  float* __restrict__ bsub_out) {
+                                                  float* __restrict__ bsub_out, const int* __restrict__ probe_grp,
+                                                  const int* __restrict__ qoff, int Gq) {
   extern __shared__ __align__(16) unsigned char smem[];
   constexpr int LDP = PR + 1;
   const int ldz = Rk + 1;
@@ -219,6 +220,28 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
   __syncthreads();
   for (int e = tid; e < D * Rk; e += nt) Vr[e] *= cs[e % Rk];
   __syncthreads();
+  // probe weights (cs is free again): 1, or n_a / (probes of group a) normalised to mean 1
+  double* wt = cs;
+  for (int i = tid; i < P; i += nt) {
+    double w = 1.0;
+    if (probe_grp) {
+      const int* pg = probe_grp + (size_t)bh * P;
+      const int a = pg[i];
+      int cnt = 0;
+      for (int k = 0; k < P; ++k) cnt += pg[k] == a;
+      const int* qo = qoff + (size_t)bh * (Gq + 1);
+      w = (a >= 0 && a < Gq && cnt > 0) ? (double)(qo[a + 1] - qo[a]) / cnt : 1.0;
+    }
+    wt[i] = w;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double sw = 0.0;
+    for (int i = 0; i < P; ++i) sw += wt[i];
+    const double f = sw > 0.0 ? (double)P / sw : 1.0;
+    for (int i = 0; i < P; ++i) wt[i] *= f;
+  }
+  __syncthreads();
   // Y = R Vr and Xs = X Vr (the probes' residuals and sparse outputs in the subspace), means
   for (int e = tid; e < P * Rk; e += nt) {
     const int p = e / Rk, j = e - p * Rk;
@@ -231,11 +254,12 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
     Xs[p * Rk + j] = t;
   }
   __syncthreads();
+  // weighted means (the weights average to 1), centred rows scaled by sqrt(weight)
   for (int j = tid; j < Rk; j += nt) {
     double s = 0.0, t = 0.0;
     for (int p = 0; p < P; ++p) {
-      s += Y[p * Rk + j];
-      t += Xs[p * Rk + j];
+      s += wt[p] * Y[p * Rk + j];
+      t += wt[p] * Xs[p * Rk + j];
     }
     ybar[j] = s / P;
     xbar[j] = t / P;
@@ -243,8 +267,9 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
   __syncthreads();
   for (int e = tid; e < P * Rk; e += nt) {
     const int p = e / Rk, j = e - p * Rk;
-    Y[p * Rk + j] -= ybar[j];
-    Xs[p * Rk + j] -= xbar[j];
+    const double sq = sqrt(wt[p]);
+    Y[p * Rk + j] = (Y[p * Rk + j] - ybar[j]) * sq;
+    Xs[p * Rk + j] = (Xs[p * Rk + j] - xbar[j]) * sq;
   }
   __syncthreads();
   // A = Xc Xc^T + lam I  (into G), Xc = centred Xs
@@ -647,14 +672,16 @@ size_t probe_fit_smem(int D, int Rk) { return D == 64 ? FitLayout<64>::bytes(Rk)
 
 cudaError_t launch_probe_fit(const float* o_dense, const float* o_sparse, int BH, int D, int P, int Rk,
                              double lam, float* Vr, float* W, float* bfull, float* Bmat, float* sigma,
-                             float* bsub, cudaStream_t st) {
+                             float* bsub, const int* probe_grp, const int* qoff, int Gq, cudaStream_t st) {
   const size_t sm = probe_fit_smem(D, Rk);
   if (D == 64) {
     cudaFuncSetAttribute(k_probe_fit<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_probe_fit<64><<<BH, FIT_THREADS, sm, st>>>(o_dense, o_sparse, P, Rk, lam, Vr, W, bfull, Bmat, sigma, bsub);
+    k_probe_fit<64><<<BH, FIT_THREADS, sm, st>>>(o_dense, o_sparse, P, Rk, lam, Vr, W, bfull, Bmat, sigma, bsub,
+                                                  probe_grp, qoff, Gq);
   } else {
     cudaFuncSetAttribute(k_probe_fit<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_probe_fit<128><<<BH, FIT_THREADS, sm, st>>>(o_dense, o_sparse, P, Rk, lam, Vr, W, bfull, Bmat, sigma, bsub);
+    k_probe_fit<128><<<BH, FIT_THREADS, sm, st>>>(o_dense, o_sparse, P, Rk, lam, Vr, W, bfull, Bmat, sigma, bsub,
+                                                  probe_grp, qoff, Gq);
   }
   return cudaGetLastError();
 }

@@ -124,7 +124,7 @@ extern "C" sparsepr_status sparsepr_probe_fit_noalloc(const sparsepr_params* p, 
       !step(launch_probe_combine_splits(part_o, part_ml, BH, S, P, d, probe_o_dense, osp, lsd, lss, st),
             "sparsepr_probe_fit_noalloc: probe combine launch failed") ||
       !step(launch_probe_fit(probe_o_dense, osp, BH, d, P, p->sub_rank, (double)p->ridge_lambda, Vr, W, b_full,
-                             Bmat, nullptr, nullptr, st),
+                             Bmat, nullptr, nullptr, p->fit_weighted ? grp : nullptr, qoff, p->n_qgroups, st),
             "sparsepr_probe_fit_noalloc: fit launch failed")) {
     set_launch_count(launches);
     return SPARSEPR_ECUDA;

@@ -100,6 +100,9 @@ typedef struct {
                               rules, seed streams, centroids, route and layout).  In mode 1 the
                               trace's sample_idx, metric, eigval, eigvec and key_coords are not
                               written.                                                            */
+  int fit_weighted;        /* 0: uniform probe weights in the ridge fit; 1: each probe weighted by
+                              n_a / (probes of its group a), normalised to mean 1 (the weighted
+                              affine fit one page mentions)                                       */
 } sparsepr_params;
 
 /* Optional debug copies of partition intermediates (any pointer may be NULL). */

@@ -50,7 +50,7 @@ int main(void) {
   printf("size %zu\n", sizeof(sparsepr_params));
   F(sparsepr_params, density) F(sparsepr_params, n_kgroups) F(sparsepr_params, kmeans_iters)
   F(sparsepr_params, ridge_lambda) F(sparsepr_params, scale) F(sparsepr_params, seed) F(sparsepr_params, frame_id)
-  F(sparsepr_params, n_frames) F(sparsepr_params, partition_mode)
+  F(sparsepr_params, n_frames) F(sparsepr_params, partition_mode) F(sparsepr_params, fit_weighted)
   printf("ptrace %zu\n", sizeof(sparsepr_partition_trace));
   printf("prtrace %zu\n", sizeof(sparsepr_probe_trace));
   return 0;
@@ -64,7 +64,7 @@ int main(void) {
         out = dict(line.split() for line in subprocess.check_output([exe], text=True).splitlines())
     P = spr.Params
     assert int(out["size"]) == ctypes.sizeof(P)
-    for f in ("density", "n_kgroups", "kmeans_iters", "ridge_lambda", "scale", "seed", "frame_id", "n_frames", "partition_mode"):
+    for f in ("density", "n_kgroups", "kmeans_iters", "ridge_lambda", "scale", "seed", "frame_id", "n_frames", "partition_mode", "fit_weighted"):
         assert int(out[f]) == getattr(P, f).offset, f
     assert int(out["ptrace"]) == ctypes.sizeof(spr.PartitionTrace)
     assert int(out["prtrace"]) == ctypes.sizeof(spr.ProbeTrace)
@@ -91,6 +91,7 @@ def _params(spr, **kw):
     (dict(N=37, n_kgroups=37, n_qgroups=4, n_samples=37, n_probes=37, sub_rank=16, density=1.0), 0),
     (dict(d=128, eig_rank=32, sub_rank=33), 2),
     (dict(partition_mode=1), 0), (dict(partition_mode=2), 1), (dict(partition_mode=-1), 1),
+    (dict(fit_weighted=1), 0), (dict(fit_weighted=2), 1),
 ])
 def test_validation(spr, kw, status):
     p = _params(spr, **kw)

@@ -182,6 +182,7 @@ def _rest_checks(pd, op, q, k, v, s, tr, ptr, out, bh, b, h, y_gpu, N, T, rng, r
         # the largest at rank 32) and can rotate with the last bits of the inputs.
         r_gpu = od_gpu - os_gpu
         fit_dev = O.fit_from_probes(pidx, od_gpu, os_gpu, ld_ref, ls_ref, pd["sub_rank"], op.ridge_lambda)
+        # (the singular values do not depend on the fit's weights)
         sig_gpu = _np(ptr["sigma"][bh]).astype(np.float64)
         s0 = max(fit_dev.sigma[0], 1e-30)
         assert np.abs(sig_gpu - fit_dev.sigma).max() <= 1e-5 * s0 + 1e-9
@@ -201,7 +202,8 @@ def _rest_checks(pd, op, q, k, v, s, tr, ptr, out, bh, b, h, y_gpu, N, T, rng, r
             inv = r_gpu.T @ (r_gpu @ vk) - vk * sig_gpu[keep] ** 2
             assert np.abs(inv).max() <= 1e-5 * s0 ** 2
         # --- a15: the ridge given the device's subspace (exact up to fp32 rounding)
-        w_sub, b_sub = O.ridge_fit(os_gpu @ vr_gpu, r_gpu @ vr_gpu, op.ridge_lambda)
+        wts = O.probe_weights(qo, pd["n_probes"]) if op.fit_weighted else None
+        w_sub, b_sub = O.ridge_fit(os_gpu @ vr_gpu, r_gpu @ vr_gpu, op.ridge_lambda, wts)
         bfull_ref = vr_gpu @ b_sub
         bmat_ref = vr_gpu @ w_sub @ vr_gpu.T
         np.testing.assert_allclose(bm_gpu, w_gpu @ vr_gpu.T, atol=1e-5 * max(1, np.abs(bm_gpu).max()))
@@ -225,6 +227,8 @@ def _rest_checks(pd, op, q, k, v, s, tr, ptr, out, bh, b, h, y_gpu, N, T, rng, r
 
 CASES = {
     "tiny": dict(name="tiny"),
+    "tiny_weighted": dict(name="tiny", fit_weighted=1),
+    "mid25_weighted": dict(name="mid", density=0.25, fit_weighted=1),
     "mid15": dict(name="mid", density=0.15),
     "mid25": dict(name="mid", density=0.25),
     "mid40": dict(name="mid", density=0.40),
@@ -251,9 +255,10 @@ def test_stage_parity(gpu, case):
     stage_checks(pd, qb, kb, vb, out, heads, rows=None if w.name == "tiny" else 1024)
 
 
-def test_stage_parity_ragged_d128(gpu):
+@pytest.mark.parametrize("weighted", [0, 1])
+def test_stage_parity_ragged_d128(gpu, weighted):
     w = _ragged_workload()
-    pd = params_dict(w)
+    pd = params_dict(w, fit_weighted=weighted)
     qb, kb, vb = generate(w, seed=3)
     _, out = _run(pd, qb, kb, vb, gpu)
     stage_checks(pd, qb, kb, vb, out, range(w.B * w.H), rows=None)
