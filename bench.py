@@ -172,7 +172,7 @@ def run_cuda(args):
     pd = dict(B=w.B, H=w.H, N=w.N, d=w.d, block=w.block, density=w.density, n_kgroups=w.n_kgroups,
               n_qgroups=w.n_qgroups, n_samples=w.n_samples, n_probes=w.n_probes, eig_rank=w.eig_rank,
               sub_rank=w.sub_rank, kmeans_iters=w.kmeans_iters, ridge_lambda=w.ridge_lambda, seed=0,
-              partition_mode=1 if args.partition == "semantic" else 0)
+              partition_mode=1 if args.partition == "semantic" else 0, fit_weighted=1 if args.weighted_fit else 0)
     from synth import frame_index, perturb, to_torch
     frames = frame_index(w.grid) if w.frame_causal else None
     fid = torch.from_numpy(frames).to(dev) if w.frame_causal else None
@@ -372,6 +372,8 @@ def run_cuda(args):
     }
     if calls > 1:
         line["ms_per_call"] = round(ms_per_call, 4)
+    if args.weighted_fit:
+        line["config"]["fit"] = "weighted ridge (probe weights n_a / probes of group a)"
     if args.partition != "coupled":
         line["config"]["partition"] = "semantic-grouping baseline (keys and queries clustered on raw rows)"
     if args.diagnostics:
@@ -594,6 +596,7 @@ def main():
     ap.add_argument("--partition", default="coupled", choices=["coupled", "semantic"],
                     help="coupled: the method; semantic: the semantic-grouping baseline of the pages")
     ap.add_argument("--density", type=float, default=0.0, help="override the workload's target density")
+    ap.add_argument("--weighted-fit", action="store_true", help="weight the probes of the ridge fit")
     ap.add_argument("--diagnostics", action="store_true",
                     help="add support and affine-explainability measurements of two heads to the line")
     ap.add_argument("--streams", type=int, default=2, choices=[1, 2],
