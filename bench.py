@@ -397,7 +397,7 @@ def run_cuda(args):
         print(json.dumps(line), flush=True)
 
 
-def e2e_pipeline(spr, pd, p, fid, Qh, Kh, Vh, Oh, dev, steps, chunks=8):
+def e2e_pipeline(spr, pd, p, fid, Qh, Kh, Vh, Oh, dev, steps, chunks=4):
     """ms per call from pinned host buffers to pinned host buffers, the heads split into
     `chunks` calls of sparsepr_forward: chunk i's host-to-device copies run on one copy
     stream, its compute on another, its output's copy back on a third, two chunk slots."""
