@@ -329,6 +329,7 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
   const size_t cpart = (size_t)BH * kmeans_gp(Gk) * d * 2;
   SPR_LAUNCH(launch_cell_mass_tc(Q, BH, N, d, Gq, Gk, perm_q, qoff, koff, C, scale, w_hi, w_lo,
                                  at<char>(ws, L.w_lo) + cpart, cz, mass, err, st));
+  ++g_launches;   // the cell-mass launcher also splits C into its bf16 parts (a second kernel)
   SPR_LAUNCH(launch_route_select(mass, BH, N, Gq, Gk, qoff, koff, p.density, p.n_probes, cz, at<int>(ws, L.order),
                                  route, rho, at<double>(ws, L.alpha), st));
   if (bmask)
