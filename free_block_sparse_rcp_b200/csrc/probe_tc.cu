@@ -16,8 +16,12 @@
 // (row group * 32 + lane = TMEM lane) x 32-key quarter of the chunk; the four quarters of a
 // row exchange their maxima once per chunk (mbarrier) and keep separate partial sums,
 // added at the end.  Warp 16: TMEM allocation + MMA issue (lane 0).  Warp 17: loads -- the
-// probe rows (cp.async, gathered through probe_idx), the K and V chunks (TMA, two-deep
-// ring) and the chunk's key labels.
+// probe rows (cp.async, gathered through probe_idx), the K chunks with their key labels and
+// the V chunks (TMA, two-deep rings of their own: a K stage is refilled as soon as its S
+// MMAs completed and every softmax warp built its key mask from the labels, a V stage once
+// its PV MMAs completed, so the next chunk's keys arrive while this one is in the softmax).
+// The softmax warps arrive on the barriers once per warp.  A sparse row's key mask is built
+// from the labels read 16 bytes at a time against the routed-group bits of its query group.
 // TMEM: S at columns 0 / 128 (two buffers), P hi at 256, P lo at 320, O at 384.
 // All waits bounded.
 #include <cuda.h>
@@ -41,7 +45,7 @@ constexpr int NT = 576;
 constexpr float kRescaleThreshold = 8.0f;
 
 struct Bars {
-  uint64_t q, full[2], empty[2], s_full[2], s_free[2], p_full, p_empty, o_done, mma_done, mready[2], ldone;
+  uint64_t q, full[2], empty[2], vfull[2], vempty[2], s_full[2], s_free[2], p_full, p_empty, o_done, mma_done, mready[2], ldone;
 };
 
 template <int D>
@@ -99,17 +103,19 @@ __global__ void __launch_bounds__(NT, 1)
     mbar_init(su32(&bars->q), 32);
     for (int s = 0; s < 2; ++s) {
       mbar_init(su32(&bars->full[s]), 33);   // 32 label arrivals + the TMA transaction arrival
-      mbar_init(su32(&bars->empty[s]), 1);
+      mbar_init(su32(&bars->empty[s]), 1 + NSOFT / 32);   // S MMAs done + every softmax warp read the labels
+      mbar_init(su32(&bars->vfull[s]), 1);
+      mbar_init(su32(&bars->vempty[s]), 1);
       mbar_init(su32(&bars->s_full[s]), 1);
-      mbar_init(su32(&bars->s_free[s]), NSOFT);
+      mbar_init(su32(&bars->s_free[s]), NSOFT / 32);
     }
-    mbar_init(su32(&bars->p_full), NSOFT);
+    mbar_init(su32(&bars->p_full), NSOFT / 32);
     mbar_init(su32(&bars->p_empty), 1);
     mbar_init(su32(&bars->o_done), 1);
     mbar_init(su32(&bars->mma_done), 1);
-    mbar_init(su32(&bars->mready[0]), NSOFT);
-    mbar_init(su32(&bars->mready[1]), NSOFT);
-    mbar_init(su32(&bars->ldone), NSOFT);
+    mbar_init(su32(&bars->mready[0]), NSOFT / 32);
+    mbar_init(su32(&bars->mready[1]), NSOFT / 32);
+    mbar_init(su32(&bars->ldone), NSOFT / 32);
     fence_barrier_init();
   }
   if (warp == MMA_WARP) {
@@ -143,13 +149,11 @@ __global__ void __launch_bounds__(NT, 1)
       if (!ok) break;
       const int c0 = k0 + j * BN;
       if (lane == 0) {
-        // K and V rows c0 .. c0+127 of this head (rows past k1 are masked in the softmax)
-        mbar_arrive_expect_tx(su32(&bars->full[s]), 2 * L::kKV);
+        // K rows c0 .. c0+127 of this head (rows past k1 are masked in the softmax)
+        mbar_arrive_expect_tx(su32(&bars->full[s]), L::kKV);
 #pragma unroll
-        for (int h = 0; h < D / 64; ++h) {
+        for (int h = 0; h < D / 64; ++h)
           tma_load_2d(sK + s * L::kKV + h * BN * 128, &tmk, 64 * h, (int)(head + c0), su32(&bars->full[s]));
-          tma_load_2d(sV + s * L::kKV + h * BN * 128, &tmv, 64 * h, (int)(head + c0), su32(&bars->full[s]));
-        }
       }
       for (int r = lane; r < BN; r += 32) {  // 4-byte labels (label rows are only 4-byte aligned)
         const bool v = c0 + r < k1;
@@ -158,6 +162,15 @@ __global__ void __launch_bounds__(NT, 1)
                      : "memory");
       }
       cp_async_arrive_noinc(su32(&bars->full[s]));
+      // V rows of the chunk: their stage is free once the PV MMAs two chunks back completed
+      if (j >= 2) ok = __all_sync(0xffffffffu, wait(bars->vempty[s], ((j >> 1) - 1) & 1));
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(su32(&bars->vfull[s]), L::kKV);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tma_load_2d(sV + s * L::kKV + h * BN * 128, &tmv, 64 * h, (int)(head + c0), su32(&bars->vfull[s]));
+      }
     }
     cp_async_wait_all();
   } else if (warp == MMA_WARP) {
@@ -167,7 +180,7 @@ __global__ void __launch_bounds__(NT, 1)
       constexpr uint32_t IDO = idesc_bf16(BM, D, true);
       bool ok = nchunks == 0 || wait(bars->q, 0);
       auto issue_pv = [&](int i) -> bool {
-        if (!wait(bars->p_full, i & 1)) return false;
+        if (!wait(bars->p_full, i & 1) || !wait(bars->vfull[i & 1], (i >> 1) & 1)) return false;
         tc_fence_after();
         const uint32_t vb = sV + (i & 1) * L::kKV;
 #pragma unroll
@@ -176,7 +189,7 @@ __global__ void __launch_bounds__(NT, 1)
           tc_mma_ts(tO, tP + k * 8, bd, IDO, (i > 0 || k > 0) ? 1u : 0u);
           tc_mma_ts(tO, tP + 64 + k * 8, bd, IDO, 1u);
         }
-        tc_commit(su32(&bars->empty[i & 1]));
+        tc_commit(su32(&bars->vempty[i & 1]));
         tc_commit(su32(&bars->p_empty));
         return true;
       };
@@ -193,6 +206,7 @@ __global__ void __launch_bounds__(NT, 1)
           tc_mma(tmem + s * BN, sdesc(sQ + oq, 16, 1024), sdesc(kb + ok2, 16, 1024), IDS, k > 0 ? 1u : 0u);
         }
         tc_commit(su32(&bars->s_full[s]));
+        tc_commit(su32(&bars->empty[s]));
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok && nchunks > 0) issue_pv(nchunks - 1);
@@ -214,8 +228,25 @@ __global__ void __launch_bounds__(NT, 1)
       const int a = probe_grp[(size_t)bh * P + prow];
       if (a >= 0 && a < Gq) {
         const unsigned char* rr = route + ((size_t)bh * Gq + a) * Gk;
-        for (int g = 0; g < Gk; ++g)
-          if (rr[g]) rm[g >> 5] |= 1u << (g & 31);
+        if ((Gk & 15) == 0 && (reinterpret_cast<uintptr_t>(rr) & 15) == 0) {
+          uint4 v[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            if (c * 16 < Gk) v[c] = __ldg(reinterpret_cast<const uint4*>(rr) + c);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            if (c * 16 >= Gk) break;
+            const uint32_t w4[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if ((w4[q] >> (8 * e)) & 0xffu) rm[c >> 1] |= 1u << ((c & 1) * 16 + q * 4 + e);
+          }
+        } else {
+          for (int g = 0; g < Gk; ++g)
+            if (rr[g]) rm[g >> 5] |= 1u << (g & 31);
+        }
       }
     }
     // frame-causal: the row sees the keys before fend[its frame] (frame ids nondecreasing)
@@ -238,30 +269,45 @@ __global__ void __launch_bounds__(NT, 1)
       tc_fence_after();
       const int valid = kend - (k0 + j * BN);
       // keys of this quarter the row may use
-      uint32_t km = 0u;
+      uint32_t km;
       {
-        const int* lab = sLab + b * BN + qt * 32;
+        // keys of this quarter before the row's end, then (sparse rows) the routed ones
+        const int nv = valid - qt * 32;
+        const uint32_t vmask = nv >= 32 ? 0xffffffffu : (nv <= 0 ? 0u : ((1u << nv) - 1u));
+        km = vmask;
+        if (sparse) {
+          const int4* lab4 = reinterpret_cast<const int4*>(sLab + b * BN + qt * 32);
+          uint32_t bits = 0u;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          bool use = qt * 32 + e < valid;
-          if (sparse) {
-            const int g = lab[e];
-            const uint32_t word = g < 32 ? rm[0] : g < 64 ? rm[1] : g < 96 ? rm[2] : rm[3];
-            use = use && g >= 0 && g < Gk && ((word >> (g & 31)) & 1u);
+          for (int c = 0; c < 8; ++c) {
+            const int4 g4 = lab4[c];
+            const uint32_t gg[4] = {(uint32_t)g4.x, (uint32_t)g4.y, (uint32_t)g4.z, (uint32_t)g4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t g = gg[e];   // a negative label compares as >= Gk
+              const uint32_t w01 = (g & 32u) ? rm[1] : rm[0];
+              const uint32_t w23 = (g & 32u) ? rm[3] : rm[2];
+              const uint32_t w = (g & 64u) ? w23 : w01;
+              bits |= ((w >> (g & 31u)) & (g < (uint32_t)Gk ? 1u : 0u)) << (c * 4 + e);
+            }
           }
-          km |= (use ? 1u : 0u) << e;
+          km &= bits;
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(su32(&bars->empty[b]));
       uint32_t sreg[32];
       tc_ld32(tmem + b * BN + lane_off + qt * 32, sreg);
       tc_fence_before();
-      mbar_arrive(su32(&bars->s_free[b]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(su32(&bars->s_free[b]));
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int e = 0; e < 32; ++e)
         if ((km >> e) & 1u) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(sreg[e]));
       xm[(b * 4 + qt) * BM + r] = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      mbar_arrive(su32(&bars->mready[b]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(su32(&bars->mready[b]));
       ok = __all_sync(0xffffffffu, wait(bars->mready[b], (j >> 1) & 1));
       if (!ok) break;
       float mx = xm[(b * 4 + 0) * BM + r];
@@ -318,13 +364,15 @@ __global__ void __launch_bounds__(NT, 1)
       tc_st16(tP + lane_off + 64 + 16 * qt, plo);
       tc_fence_before();
       l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
-      mbar_arrive(su32(&bars->p_full));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(su32(&bars->p_full));
     }
     // ---- this split's outputs: O quarter columns, and (quarter 0) max and the row sum
     float* xl = xm + 2 * 4 * BM;   // [4][BM] partial sums (the maxima buffers may still be read)
     xl[qt * BM + r] = l;
     if (ok && nchunks > 0) ok = __all_sync(0xffffffffu, wait(bars->o_done, 0));
-    mbar_arrive(su32(&bars->ldone));
+    __syncwarp();
+    if (lane == 0) mbar_arrive(su32(&bars->ldone));
     if (ok) ok = __all_sync(0xffffffffu, wait(bars->ldone, 0));
     if (ok) {
       tc_fence_after();
