@@ -233,6 +233,12 @@ float eff_scale(const sparsepr_params& p) { return p.scale > 0.f ? p.scale : 1.0
   do {                                                                                    \
     if (!(ptr)) return fail(SPARSEPR_EINVAL, "required pointer " #ptr " is NULL");        \
   } while (0)
+// bf16 token tensors are read and written by TMA: non-NULL and 16-byte aligned
+#define SPR_TILED(ptr)                                                                    \
+  do {                                                                                    \
+    SPR_NONNULL(ptr);                                                                     \
+    if ((uintptr_t)(ptr) & 15u) return fail(SPARSEPR_EINVAL, "tensor " #ptr " is not 16-byte aligned"); \
+  } while (0)
 
 // ---------------------------------------------------------------------------
 sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const void* Q, const void* K, int* perm_q,
@@ -460,7 +466,7 @@ sparsepr_status sparsepr_partition(const sparsepr_params* p, const void* Q, cons
                                    void* workspace, size_t ws_bytes, void* stream) {
   g_launches = 0;
   SPR_CHECK(check_params(p));
-  SPR_NONNULL(Q); SPR_NONNULL(K); SPR_NONNULL(perm_q); SPR_NONNULL(perm_k); SPR_NONNULL(label_q);
+  SPR_TILED(Q); SPR_TILED(K); SPR_NONNULL(perm_q); SPR_NONNULL(perm_k); SPR_NONNULL(label_q);
   SPR_NONNULL(label_k); SPR_NONNULL(qoff); SPR_NONNULL(koff); SPR_NONNULL(route); SPR_NONNULL(rho_exec);
   const Layout L = make_layout(*p);
   SPR_CHECK(check_ws(p, workspace, ws_bytes, L.total));
@@ -474,8 +480,8 @@ sparsepr_status sparsepr_attend(const sparsepr_params* p, const void* Q, const v
                                 size_t ws_bytes, void* stream) {
   g_launches = 0;
   SPR_CHECK(check_params(p));
-  SPR_NONNULL(Q); SPR_NONNULL(K); SPR_NONNULL(V); SPR_NONNULL(perm_q); SPR_NONNULL(perm_k); SPR_NONNULL(qoff);
-  SPR_NONNULL(koff); SPR_NONNULL(route); SPR_NONNULL(O_sparse);
+  SPR_TILED(Q); SPR_TILED(K); SPR_TILED(V); SPR_NONNULL(perm_q); SPR_NONNULL(perm_k); SPR_NONNULL(qoff);
+  SPR_NONNULL(koff); SPR_NONNULL(route); SPR_TILED(O_sparse);
   const Layout L = make_layout(*p);
   SPR_CHECK(check_ws(p, workspace, ws_bytes, L.total));
   return run_attend(*p, L, Q, K, V, perm_q, perm_k, qoff, koff, route, O_sparse, lse, workspace,
@@ -489,7 +495,7 @@ sparsepr_status sparsepr_probe_fit(const sparsepr_params* p, const void* Q, cons
                                    void* stream) {
   g_launches = 0;
   SPR_CHECK(check_params(p));
-  SPR_NONNULL(Q); SPR_NONNULL(K); SPR_NONNULL(V); SPR_NONNULL(label_k); SPR_NONNULL(perm_q); SPR_NONNULL(qoff);
+  SPR_TILED(Q); SPR_TILED(K); SPR_TILED(V); SPR_NONNULL(label_k); SPR_NONNULL(perm_q); SPR_NONNULL(qoff);
   SPR_NONNULL(route); SPR_NONNULL(probe_idx); SPR_NONNULL(probe_o_dense); SPR_NONNULL(b_full); SPR_NONNULL(Vr);
   SPR_NONNULL(W);
   const Layout L = make_layout(*p);
@@ -503,8 +509,8 @@ sparsepr_status sparsepr_reconstruct(const sparsepr_params* p, const void* O_spa
                                      const float* W, void* O, void* stream) {
   g_launches = 0;
   SPR_CHECK(check_params(p));
-  SPR_NONNULL(O_sparse); SPR_NONNULL(probe_idx); SPR_NONNULL(probe_o_dense); SPR_NONNULL(b_full); SPR_NONNULL(Vr);
-  SPR_NONNULL(W); SPR_NONNULL(O);
+  SPR_TILED(O_sparse); SPR_NONNULL(probe_idx); SPR_NONNULL(probe_o_dense); SPR_NONNULL(b_full); SPR_NONNULL(Vr);
+  SPR_NONNULL(W); SPR_TILED(O);
   return run_reconstruct(*p, p->B * p->H, O_sparse, probe_idx, probe_o_dense, b_full, Vr, W, O,
                          (cudaStream_t)stream);
 }
@@ -513,7 +519,7 @@ sparsepr_status sparsepr_forward(const sparsepr_params* p, const void* Q, const 
                                  float* rho_exec, void* workspace, size_t ws_bytes, void* stream) {
   g_launches = 0;
   SPR_CHECK(check_params(p));
-  SPR_NONNULL(Q); SPR_NONNULL(K); SPR_NONNULL(V); SPR_NONNULL(O);
+  SPR_TILED(Q); SPR_TILED(K); SPR_TILED(V); SPR_TILED(O);
   const Layout L = make_layout(*p);
   SPR_CHECK(check_ws(p, workspace, ws_bytes, L.forward_total));
   cudaStream_t st = (cudaStream_t)stream;
@@ -545,8 +551,8 @@ sparsepr_status sparsepr_forward_host(const sparsepr_params* p, const void* Q_ho
                                       size_t ws_bytes, void* stream) {
   g_launches = 0;
   SPR_CHECK(check_params(p));
-  SPR_NONNULL(Q_host); SPR_NONNULL(K_host); SPR_NONNULL(V_host); SPR_NONNULL(O_host); SPR_NONNULL(qkv_dev);
-  SPR_NONNULL(o_dev);
+  SPR_NONNULL(Q_host); SPR_NONNULL(K_host); SPR_NONNULL(V_host); SPR_NONNULL(O_host); SPR_TILED(qkv_dev);
+  SPR_TILED(o_dev);
   cudaStream_t st = (cudaStream_t)stream;
   const size_t bytes = (size_t)p->B * p->H * p->N * p->d * 2;
   char* q = static_cast<char*>(qkv_dev);
@@ -562,7 +568,7 @@ sparsepr_status sparsepr_dense_attention(const sparsepr_params* p, const void* Q
                                          void* O, float* lse, void* workspace, size_t ws_bytes, void* stream) {
   g_launches = 0;
   SPR_CHECK(check_params(p));
-  SPR_NONNULL(Q); SPR_NONNULL(K); SPR_NONNULL(V); SPR_NONNULL(O);
+  SPR_TILED(Q); SPR_TILED(K); SPR_TILED(V); SPR_TILED(O);
   int* err = nullptr;
   const size_t need = p->frame_id ? 512 : 256;   // error word, then the frame ends
   if (workspace || p->frame_id) {

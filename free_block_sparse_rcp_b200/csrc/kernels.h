@@ -52,6 +52,8 @@ cudaError_t launch_causal_stream(const int* rlist, const int* rcnt, const int* k
 // tma_host.cu: 128-byte tensor map (CUtensorMap) of a row-major bf16 matrix for boxes of
 // box_rows x 64 columns with 128B swizzle; rows past the end read as zeros.
 cudaError_t make_tmap_bf16_rows(void* tmap, const void* base, unsigned long long rows, int cols, int box_rows);
+cudaError_t make_tmap_bf16_3d(void* tmap, const void* base, unsigned long long outer, unsigned long long rows,
+                              int cols, int box_rows);
 struct alignas(64) TmapBlob {
   unsigned long long w[16];
 };

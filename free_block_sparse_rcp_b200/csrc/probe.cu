@@ -356,7 +356,10 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
 //               into a three-deep ring
 //   warp 16     (lane 0) issues x B_hi + x B_lo (exact bf16 products, fp32 accumulation)
 //               into a double-buffered TMEM tile
-//   warps 0-15  row r = TMEM lane r, column quarter q: x + b + xB -> bf16 -> O
+//   warps 0-15  row r = TMEM lane r, column quarter q: x + b + xB -> bf16, written in place
+//               over x in the tile's ring slot; then thread 0 stores the slot to O with
+//               TMA (3D map [BH][N][d], so a head's ragged last tile is clipped at row N) and
+//               frees the slot once the store has read it
 // Every row of a tile is loaded before the tile's outputs are written, so O may alias
 // O_sparse.
 // ---------------------------------------------------------------------------
@@ -374,7 +377,8 @@ struct Bars {
 
 template <int D>
 __global__ void __launch_bounds__(rct::NT, 1)
-    k_reconstruct_tc(const __grid_constant__ CUtensorMap tmx, int N, int T, int total, int per, int Rk,
+    k_reconstruct_tc(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmo, int N, int T,
+                     int total, int per, int Rk,
                      const float* __restrict__ W, const float* __restrict__ Vr, const float* __restrict__ bfull,
                      __nv_bfloat16* __restrict__ O, int* err) {
   using namespace spr::tc;
@@ -399,7 +403,7 @@ __global__ void __launch_bounds__(rct::NT, 1)
     sMisc[1] = 0;
     for (int b = 0; b < XS; ++b) {
       mbar_init(su32(&bars->xfull[b]), 1);
-      mbar_init(su32(&bars->xempty[b]), rct::NEPI);
+      mbar_init(su32(&bars->xempty[b]), 1);   // thread 0, once the tile's store has read the slot
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(su32(&bars->tfull[b]), 1);
@@ -497,46 +501,57 @@ __global__ void __launch_bounds__(rct::NT, 1)
       const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
       constexpr int CQ = D / 4;   // columns of this quarter
       for (int i = s0; i < s1 && ok; ++i, ++it) {
-        const int b = it & 1, xb = it % XS, row = (i - bh * T) * 128 + r;
+        const int b = it & 1, xb = it % XS, n0 = (i - bh * T) * 128;
         // xB ready; the X tile (read below) completed before it
-        ok = __all_sync(0xffffffffu, wait(bars->tfull[b], (it >> 1) & 1) && wait(bars->xfull[xb], (it / XS) & 1));
-        if (!ok) break;
-        tc_fence_after();
+        const bool good =
+            __all_sync(0xffffffffu, wait(bars->tfull[b], (it >> 1) & 1) && wait(bars->xfull[xb], (it / XS) & 1));
+        if (good) {
+          tc_fence_after();
 #pragma unroll
-        for (int c0 = 0; c0 < CQ; c0 += 16) {
-          const int cb = qt * CQ + c0;
-          uint32_t acc[16];
-          asm volatile(
-              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-              "tcgen05.wait::ld.sync.aligned;\n"
-              : "=r"(acc[0]), "=r"(acc[1]), "=r"(acc[2]), "=r"(acc[3]), "=r"(acc[4]), "=r"(acc[5]), "=r"(acc[6]),
-                "=r"(acc[7]), "=r"(acc[8]), "=r"(acc[9]), "=r"(acc[10]), "=r"(acc[11]), "=r"(acc[12]),
-                "=r"(acc[13]), "=r"(acc[14]), "=r"(acc[15])
-              : "r"(tmem + 128 * b + lane_off + cb)
-              : "memory");
-          uint32_t w[8];
+          for (int c0 = 0; c0 < CQ; c0 += 16) {
+            const int cb = qt * CQ + c0;
+            uint32_t acc[16];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+                "tcgen05.wait::ld.sync.aligned;\n"
+                : "=r"(acc[0]), "=r"(acc[1]), "=r"(acc[2]), "=r"(acc[3]), "=r"(acc[4]), "=r"(acc[5]), "=r"(acc[6]),
+                  "=r"(acc[7]), "=r"(acc[8]), "=r"(acc[9]), "=r"(acc[10]), "=r"(acc[11]), "=r"(acc[12]),
+                  "=r"(acc[13]), "=r"(acc[14]), "=r"(acc[15])
+                : "r"(tmem + 128 * b + lane_off + cb)
+                : "memory");
+            uint32_t w[8];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const uint4 xv = *reinterpret_cast<const uint4*>(smem_rc + xb * kT + tile_off(r, (cb >> 3) + q, 128));
-            const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
+            for (int q = 0; q < 2; ++q) {
+              const uint4 xv = *reinterpret_cast<const uint4*>(smem_rc + xb * kT + tile_off(r, (cb >> 3) + q, 128));
+              const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&xv);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 x = __bfloat1622float2(x2[e]);
-              const int c = cb + q * 8 + 2 * e;
-              w[q * 4 + e] = pack_bf16(x.x + sb[c] + __uint_as_float(acc[q * 8 + 2 * e]),
-                                       x.y + sb[c + 1] + __uint_as_float(acc[q * 8 + 2 * e + 1]));
+              for (int e = 0; e < 4; ++e) {
+                const float2 x = __bfloat1622float2(x2[e]);
+                const int c = cb + q * 8 + 2 * e;
+                w[q * 4 + e] = pack_bf16(x.x + sb[c] + __uint_as_float(acc[q * 8 + 2 * e]),
+                                         x.y + sb[c + 1] + __uint_as_float(acc[q * 8 + 2 * e + 1]));
+              }
             }
+            // in place: this thread read exactly these 32 bytes of the slot above
+            *reinterpret_cast<uint4*>(smem_rc + xb * kT + tile_off(r, cb >> 3, 128)) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(smem_rc + xb * kT + tile_off(r, (cb >> 3) + 1, 128)) =
+                make_uint4(w[4], w[5], w[6], w[7]);
           }
-          if (row < N) {
-            uint4* dst = reinterpret_cast<uint4*>(O + (head + row) * D + cb);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          }
+          tc_fence_before();
+          mbar_arrive(su32(&bars->tempty[b]));
+          fence_proxy_async();   // the slot's new contents, to the TMA store
         }
-        tc_fence_before();
-        mbar_arrive(su32(&bars->tempty[b]));
-        mbar_arrive(su32(&bars->xempty[xb]));
+        // every epilogue thread passes this barrier once per tile, whatever its waits gave
+        if (!bar_and(1, rct::NEPI, good)) { ok = false; break; }
+        if (tid == 0) {
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h) tma_store_3d(&tmo, sX + xb * kT + h * 16384, 64 * h, n0, bh);
+          bulk_commit();
+          bulk_wait_read_all();
+          mbar_arrive(su32(&bars->xempty[xb]));
+        }
       }
+      if (tid == 0) bulk_wait_all();
     }
     ok = __syncthreads_and(ok ? 1 : 0) != 0;
     s0 = s1;
@@ -692,16 +707,17 @@ cudaError_t launch_reconstruct(const void* Os, int BH, int N, int D, int Rk, con
   const int T = ceil_div(N, 128), total = BH * T;
   const int grid = total < rct::kCtas ? total : rct::kCtas;
   const int per = ceil_div(total, grid);
-  CUtensorMap tmx;
+  CUtensorMap tmx, tmo;
   cudaError_t e = make_tmap_bf16_rows(&tmx, Os, (unsigned long long)BH * N, D, 128);
+  if (e == cudaSuccess) e = make_tmap_bf16_3d(&tmo, O, (unsigned long long)BH, (unsigned long long)N, D, 128);
   if (e != cudaSuccess) return e;
   if (D == 64) {
     cudaFuncSetAttribute(k_reconstruct_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_reconstruct_tc<64><<<grid, rct::NT, sm, st>>>(tmx, N, T, total, per, Rk, W, Vr, bfull, (__nv_bfloat16*)O,
+    k_reconstruct_tc<64><<<grid, rct::NT, sm, st>>>(tmx, tmo, N, T, total, per, Rk, W, Vr, bfull, (__nv_bfloat16*)O,
                                                     nullptr);
   } else {
     cudaFuncSetAttribute(k_reconstruct_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_reconstruct_tc<128><<<grid, rct::NT, sm, st>>>(tmx, N, T, total, per, Rk, W, Vr, bfull, (__nv_bfloat16*)O,
+    k_reconstruct_tc<128><<<grid, rct::NT, sm, st>>>(tmx, tmo, N, T, total, per, Rk, W, Vr, bfull, (__nv_bfloat16*)O,
                                                      nullptr);
   }
   return cudaGetLastError();

@@ -44,4 +44,24 @@ cudaError_t make_tmap_bf16_rows(void* tmap, const void* base, unsigned long long
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Row-major bf16 tensor [outer][rows][cols] seen as 3D, boxes of one outer index x box_rows x
+// 64 columns (128B swizzle, the tensor-core tile layout).  A box reaching past `rows` is
+// clipped at the end of its own outer slice (stores) or reads zeros there (loads).
+cudaError_t make_tmap_bf16_3d(void* tmap, const void* base, unsigned long long outer, unsigned long long rows,
+                              int cols, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  if (((uintptr_t)base & 15u) != 0 || (cols * 2) % 16 != 0 || cols < 64 || box_rows < 1 || box_rows > 256)
+    return cudaErrorInvalidValue;
+  const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)outer};
+  const cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * 2 * rows};
+  const cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = fn(reinterpret_cast<CUtensorMap*>(tmap), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace spr

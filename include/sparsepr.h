@@ -19,8 +19,10 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Tensors are device pointers unless stated.  Q, K, V and outputs named O* are
- *    bf16, contiguous [B, H, N, d] (row stride d elements).  "BH" below is B*H and
- *    every per-head array is laid out head-major ([B, H, ...] flattened).
+ *    bf16, contiguous [B, H, N, d] (row stride d elements), and start on a 16-byte
+ *    boundary (the kernels move them with TMA; a misaligned one is SPARSEPR_EINVAL).
+ *    "BH" below is B*H and every per-head array is laid out head-major ([B, H, ...]
+ *    flattened).
  *  - Token indices are int32 positions in [0, N) of the original sequence.
  *  - Ownership: the caller owns every buffer.  The library allocates nothing and
  *    keeps no state between calls.  Scratch memory is the caller's `workspace`

@@ -131,6 +131,14 @@ def test_calls_reject_before_cuda(spr):
     bad = _params(spr, d=96)
     assert lib.sparsepr_forward(ctypes.byref(bad), fake, fake, fake, fake, None, fake, 1 << 40, None) == 2
     assert lib.sparsepr_reconstruct(ctypes.byref(p), None, fake, fake, fake, fake, fake, fake, None) == 1
+    # bf16 token tensors move by TMA: a pointer off a 16-byte boundary is an argument error
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    st = lib.sparsepr_reconstruct(ctypes.byref(p), fake, fake, fake, fake, fake, fake, odd, None)
+    assert st == 1 and b"O" in lib.sparsepr_last_error()
+    st = lib.sparsepr_forward(ctypes.byref(p), fake, odd, fake, fake, None, fake, 1 << 40, None)
+    assert st == 1 and b"K" in lib.sparsepr_last_error()
+    st = lib.sparsepr_dense_attention(ctypes.byref(p), fake, fake, odd, fake, None, None, 0, None)
+    assert st == 1 and b"V" in lib.sparsepr_last_error()
     assert lib.sparsepr_status_string(0) == b"ok"
 
 
