@@ -282,10 +282,13 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
                                                       float* __restrict__ rho_exec, double* __restrict__ alpha_out) {
   extern __shared__ __align__(16) unsigned char smem[];
   const bool causal = qcum != nullptr;
-  double* cmh = reinterpret_cast<double*>(smem);               // [Gq][Gk] cumulative mass in rank order
-  // [Gq][Gk] cumulative K/V sizes (causal: cumulative cell costs)
-  unsigned* pnk = reinterpret_cast<unsigned*>(cmh + (size_t)Gq * Gk);
-  int* nk = reinterpret_cast<int*>(pnk + (size_t)Gq * Gk);      // [Gk]
+  // rows padded to Gk + 1 entries: the lanes of a warp read different rows at once (the
+  // per-lane prefix searches), and an unpadded 128-entry row stride puts them all in one bank
+  const int GkP = Gk + 1;
+  double* cmh = reinterpret_cast<double*>(smem);               // [Gq][GkP] cumulative mass in rank order
+  // [Gq][GkP] cumulative K/V sizes (causal: cumulative cell costs)
+  unsigned* pnk = reinterpret_cast<unsigned*>(cmh + (size_t)Gq * GkP);
+  int* nk = reinterpret_cast<int*>(pnk + (size_t)Gq * GkP);     // [Gk]
   int* nq = nk + Gk;                                            // [Gq]
   int* misc = nq + Gq;                                          // [0] L, [1..32] round flags
   long long* red = reinterpret_cast<long long*>(                // [32], 8-byte aligned
@@ -313,31 +316,31 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
   const int* vk_h = causal ? visk + (size_t)blockIdx.x * Gk * F : nullptr;
   __syncthreads();
   const int L = misc[0];
-  int GS = 32;
-  while (GS < Gk) GS <<= 1;                   // sort width (power of two, <= 128 * 4 / 4)
-  const int per_lane = GS / 32;               // 1, 2 or 4 elements per lane
+  // The sort always spans 128 elements, four per lane (element e = 4 lane + q), so every
+  // stage and exchange distance is a compile-time constant and the elements stay in
+  // registers; positions g >= Gk carry (-inf, INT_MAX) and sort after every real group.
   for (int a = warp; a < Gq; a += blockDim.x / 32) {
     if (nq[a] == 0) continue;
     float km[4];
     int ki[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int g = lane * per_lane + q;
-      const bool on = q < per_lane && g < Gk && nk[g] > 0;
+      const int g = lane * 4 + q;
+      const bool on = g < Gk && nk[g] > 0;
       km[q] = on ? mh[a * Gk + g] : -INFINITY;
-      ki[q] = q < per_lane ? g : 0x7fffffff;
+      ki[q] = g < Gk ? g : 0x7fffffff;
     }
-    // element e = per_lane * lane + q; "x before y" <=> x.m > y.m || (x.m == y.m && x.i < y.i)
-    for (int k = 2; k <= GS; k <<= 1) {
+    // "x before y" <=> x.m > y.m || (x.m == y.m && x.i < y.i)
+#pragma unroll
+    for (int k = 2; k <= 128; k <<= 1) {
+#pragma unroll
       for (int j = k >> 1; j > 0; j >>= 1) {
-        if (j >= per_lane) {
-          const int lx = j / per_lane;
+        if (j >= 4) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            if (q >= per_lane) continue;
-            const float om = __shfl_xor_sync(0xffffffffu, km[q], lx);
-            const int oi = __shfl_xor_sync(0xffffffffu, ki[q], lx);
-            const int e = lane * per_lane + q;
+            const float om = __shfl_xor_sync(0xffffffffu, km[q], j >> 2);
+            const int oi = __shfl_xor_sync(0xffffffffu, ki[q], j >> 2);
+            const int e = lane * 4 + q;
             const bool first = ((e & k) == 0) == ((e & j) == 0);   // keep the earlier of the pair
             const bool mine_before = km[q] > om || (km[q] == om && ki[q] < oi);
             if (first != mine_before) { km[q] = om; ki[q] = oi; }
@@ -346,8 +349,8 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int q2 = q ^ j;
-            if (q >= per_lane || q2 < q) continue;
-            const int e = lane * per_lane + q;
+            if (q2 < q) continue;
+            const int e = lane * 4 + q;
             const bool asc = (e & k) == 0;
             const bool q_before = km[q] > km[q2] || (km[q] == km[q2] && ki[q] < ki[q2]);
             if (asc != q_before) {
@@ -360,8 +363,8 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int r = lane * per_lane + q;
-      if (q < per_lane && r < L) {
+      const int r = lane * 4 + q;
+      if (r < L) {
         oh[a * Gk + r] = ki[q];
         wm[r] = km[q];
         if (causal) {
@@ -378,13 +381,26 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
     }
     __syncwarp();
     if (lane == 0) {
+      // sequential in rank order; four ranks' inputs are fetched ahead of their sums
       double sm = 0.0;
       unsigned c = 0u;
-      for (int r = 0; r < L; ++r) {
-        sm += (double)wm[r];
-        c += wn[r];
-        cmh[(size_t)a * Gk + r] = sm;
-        pnk[(size_t)a * Gk + r] = c;
+      for (int r0 = 0; r0 < L; r0 += 4) {
+        float m4[4];
+        unsigned n4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          m4[u] = r0 + u < L ? wm[r0 + u] : 0.f;
+          n4[u] = r0 + u < L ? wn[r0 + u] : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (r0 + u < L) {
+            sm += (double)m4[u];
+            c += n4[u];
+            cmh[(size_t)a * GkP + r0 + u] = sm;
+            pnk[(size_t)a * GkP + r0 + u] = c;
+          }
+        }
       }
     }
     __syncwarp();
@@ -400,14 +416,14 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
   const double budget = (double)density * visible - probe_pairs;
   // routed pairs of row a when its prefix holds len cells
   auto row_cost = [&](int a, int len) -> long long {
-    const long long c = (long long)pnk[(size_t)a * Gk + len - 1];
+    const long long c = (long long)pnk[(size_t)a * GkP + len - 1];
     return causal ? c : (long long)nq[a] * c;
   };
   // cost of alpha over the rows a = lane, lane + 32, ... (warp-wide sum)
   auto warp_cost = [&](double al) -> long long {
     long long t = 0;
     for (int a = lane; a < Gq; a += 32)
-      if (nq[a] > 0) t += row_cost(a, prefix_len(cmh + (size_t)a * Gk, L, al));
+      if (nq[a] > 0) t += row_cost(a, prefix_len(cmh + (size_t)a * GkP, L, al));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
     return t;
@@ -457,7 +473,7 @@ __global__ void __launch_bounds__(1024) k_route_select(const float* __restrict__
   long long routed = 0;
   for (int a = tid; a < Gq; a += blockDim.x) {
     if (nq[a] == 0) continue;
-    const int len = all ? L : prefix_len(cmh + (size_t)a * Gk, L, alpha);
+    const int len = all ? L : prefix_len(cmh + (size_t)a * GkP, L, alpha);
     for (int r = 0; r < len; ++r) rh[a * Gk + oh[a * Gk + r]] = 1;
     routed += row_cost(a, len);
   }
@@ -571,7 +587,7 @@ cudaError_t launch_query_coords(const void* Q, int BH, int N, int D, const float
 }
 
 size_t route_select_smem(int Gq, int Gk) {
-  return (size_t)Gq * Gk * 8 + (size_t)Gq * Gk * 4 + (size_t)(Gk + Gq + 40) * 4 + 8 + 32 * 8 +
+  return (size_t)Gq * (Gk + 1) * 8 + (size_t)Gq * (Gk + 1) * 4 + (size_t)(Gk + Gq + 40) * 4 + 8 + 32 * 8 +
          (size_t)32 * 2 * Gk * 4;
 }
 
