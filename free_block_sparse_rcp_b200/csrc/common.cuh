@@ -93,6 +93,33 @@ __device__ inline bool draw_without_replacement(SplitMix64& g, int n, int m, Slo
   return true;
 }
 
+// Block-cooperative form of the same draw (every thread of the block calls it; the map is
+// cleared and the block synchronised beforehand).  The k-th number of a SplitMix64 stream is
+// mix(state + k * gamma), so the offsets j_i = i + (k = i + 1 number) mod (n - i) of all m
+// draws are computed in parallel into jbuf[m]; thread 0 then applies the swaps in draw order.
+// Same out[] as the single-thread form; returns false (on every thread) on overflow.
+__device__ inline bool draw_without_replacement_block(uint64_t state, int n, int m, SlotMap& map, int* out,
+                                                      int* jbuf) {
+  if (2 * m > map.cap) return false;
+  for (int i = threadIdx.x; i < m; i += blockDim.x) {
+    const uint64_t r = sm64_mix(state + 0x9E3779B97F4A7C15ull * (uint64_t)(i + 1));
+    jbuf[i] = i + (int)(r % (uint64_t)(n - i));
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < m; ++i) {
+      const int j = jbuf[i];
+      const int vi = map.get(i);
+      const int vj = map.get(j);
+      map.put(i, vj);
+      map.put(j, vi);
+      out[i] = vj;
+    }
+  }
+  __syncthreads();
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

@@ -34,11 +34,12 @@ __global__ void __launch_bounds__(256) k_sample_metric(const __nv_bfloat16* __re
   SlotMap map{mkey, mval, kMapCap};
   map.clear_all(tid, blockDim.x);
   __syncthreads();
-  if (tid == 0) {
-    SplitMix64 g(stream_state(seed, bh, PURPOSE_QUERY_SAMPLE));
-    if (!draw_without_replacement(g, N, Ms, map, sidx)) set_error(err, DERR_DRAW);
+  // the draw's offsets go to the (not yet used) row buffer: Ms <= kMapCap / 2 <= 64 D
+  if (!draw_without_replacement_block(stream_state(seed, bh, PURPOSE_QUERY_SAMPLE), N, Ms, map, sidx,
+                                      reinterpret_cast<int*>(qs))) {
+    if (tid == 0) set_error(err, DERR_DRAW);
+    return;
   }
-  __syncthreads();
   for (int i = tid; i < Ms; i += blockDim.x) sample_idx[(size_t)bh * Ms + i] = sidx[i];
   constexpr int PER = D * D / 256;
   float acc[PER];
