@@ -17,14 +17,14 @@
 namespace spr {
 
 // ---------------------------------------------------------------------------
-// Sampled queries and M_K.  grid = BH, block = 256.
+// Sampled queries and M_K.  grid = BH, block = D * D / 16 (a 4 x 4 block of M_K per thread).
 // ---------------------------------------------------------------------------
 constexpr int kMapCap = 4096;
 
 template <int D>
-__global__ void __launch_bounds__(256) k_sample_metric(const __nv_bfloat16* __restrict__ Q, int N,
-                                                      int Ms, uint64_t seed, float* __restrict__ metric,
-                                                      int* __restrict__ sample_idx, int* err) {
+__global__ void __launch_bounds__(D * D / 16) k_sample_metric(const __nv_bfloat16* __restrict__ Q, int N,
+                                                             int Ms, uint64_t seed, float* __restrict__ metric,
+                                                             int* __restrict__ sample_idx, int* err) {
   extern __shared__ __align__(16) unsigned char smem[];
   int* mkey = reinterpret_cast<int*>(smem);
   int* mval = mkey + kMapCap;
@@ -41,10 +41,13 @@ __global__ void __launch_bounds__(256) k_sample_metric(const __nv_bfloat16* __re
     return;
   }
   for (int i = tid; i < Ms; i += blockDim.x) sample_idx[(size_t)bh * Ms + i] = sidx[i];
-  constexpr int PER = D * D / 256;
-  float acc[PER];
+  // thread = a 4 x 4 block of M_K: rows 4 rb .. 4 rb + 3, columns 4 cb .. 4 cb + 3; every
+  // entry is a sequential fp32 sum over the samples in draw order
+  constexpr int CB = D / 4;
+  const int rb = tid / CB, cb = tid - rb * CB;
+  float acc[16];
 #pragma unroll
-  for (int j = 0; j < PER; ++j) acc[j] = 0.f;
+  for (int j = 0; j < 16; ++j) acc[j] = 0.f;
   const __nv_bfloat16* Qh = Q + (size_t)bh * N * D;
   for (int s0 = 0; s0 < Ms; s0 += 64) {
     const int ns = min(64, Ms - s0);
@@ -54,18 +57,22 @@ __global__ void __launch_bounds__(256) k_sample_metric(const __nv_bfloat16* __re
     }
     __syncthreads();
     for (int s = 0; s < ns; ++s) {
+      const float4 qr = *reinterpret_cast<const float4*>(qs + s * D + 4 * rb);
+      const float4 qc = *reinterpret_cast<const float4*>(qs + s * D + 4 * cb);
+      const float vr[4] = {qr.x, qr.y, qr.z, qr.w}, vc[4] = {qc.x, qc.y, qc.z, qc.w};
 #pragma unroll
-      for (int j = 0; j < PER; ++j) {
-        int e = tid + 256 * j;
-        int r = e / D, c = e - r * D;
-        acc[j] = fmaf(qs[s * D + r], qs[s * D + c], acc[j]);
-      }
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a * 4 + b] = fmaf(vr[a], vc[b], acc[a * 4 + b]);
     }
     __syncthreads();
   }
   const float inv = 1.0f / (float)Ms;
 #pragma unroll
-  for (int j = 0; j < PER; ++j) metric[(size_t)bh * D * D + tid + 256 * j] = acc[j] * inv;
+  for (int a = 0; a < 4; ++a) {
+    const float4 v = make_float4(acc[a * 4] * inv, acc[a * 4 + 1] * inv, acc[a * 4 + 2] * inv, acc[a * 4 + 3] * inv);
+    *reinterpret_cast<float4*>(metric + (size_t)bh * D * D + (size_t)(4 * rb + a) * D + 4 * cb) = v;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -523,10 +530,11 @@ cudaError_t launch_sample_metric(const void* Q, int BH, int N, int D, int Ms, ui
   size_t sm = sample_smem(Ms, D);
   if (D == 64) {
     cudaFuncSetAttribute(k_sample_metric<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_sample_metric<64><<<BH, 256, sm, st>>>((const __nv_bfloat16*)Q, N, Ms, seed, metric, sample_idx, err);
+    k_sample_metric<64><<<BH, 64 * 64 / 16, sm, st>>>((const __nv_bfloat16*)Q, N, Ms, seed, metric, sample_idx, err);
   } else {
     cudaFuncSetAttribute(k_sample_metric<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_sample_metric<128><<<BH, 256, sm, st>>>((const __nv_bfloat16*)Q, N, Ms, seed, metric, sample_idx, err);
+    k_sample_metric<128><<<BH, 128 * 128 / 16, sm, st>>>((const __nv_bfloat16*)Q, N, Ms, seed, metric,
+                                                         sample_idx, err);
   }
   return cudaGetLastError();
 }
