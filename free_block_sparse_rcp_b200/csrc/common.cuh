@@ -93,28 +93,35 @@ __device__ inline bool draw_without_replacement(SplitMix64& g, int n, int m, Slo
   return true;
 }
 
-// Block-cooperative form of the same draw (every thread of the block calls it; the map is
-// cleared and the block synchronised beforehand).  The k-th number of a SplitMix64 stream is
-// mix(state + k * gamma), so the offsets j_i = i + (k = i + 1 number) mod (n - i) of all m
-// draws are computed in parallel into jbuf[m]; thread 0 then applies the swaps in draw order.
-// Same out[] as the single-thread form; returns false (on every thread) on overflow.
-__device__ inline bool draw_without_replacement_block(uint64_t state, int n, int m, SlotMap& map, int* out,
+// Block-cooperative form of the same draw (every thread of the block calls it).  The k-th
+// number of a SplitMix64 stream is mix(state + k * gamma), so the offsets
+// j_i = i + (number i + 1) mod (n - i) of all m draws are computed in parallel into jbuf[m].
+// The swaps are then replayed per draw instead of in order: before draw t a position p >= t
+// holds p unless an earlier draw t' < t swapped with it (j_t' = p), and then, for the last
+// such t', the value position t' held before draw t' -- the same question one level down.
+// So out[i] (the value at position j_i before draw i) follows that chain backwards; draws
+// rarely collide (m << n), so the chain is short.  Same out[] as the sequential form
+// (cap: the map capacity the sequential form allows, m <= cap / 2); returns false on every
+// thread when m exceeds it.
+__device__ inline bool draw_without_replacement_block(uint64_t state, int n, int m, int cap, int* out,
                                                       int* jbuf) {
-  if (2 * m > map.cap) return false;
+  if (2 * m > cap) return false;
   for (int i = threadIdx.x; i < m; i += blockDim.x) {
     const uint64_t r = sm64_mix(state + 0x9E3779B97F4A7C15ull * (uint64_t)(i + 1));
     jbuf[i] = i + (int)(r % (uint64_t)(n - i));
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < m; ++i) {
-      const int j = jbuf[i];
-      const int vi = map.get(i);
-      const int vj = map.get(j);
-      map.put(i, vj);
-      map.put(j, vi);
-      out[i] = vj;
+  for (int i = threadIdx.x; i < m; i += blockDim.x) {
+    int p = jbuf[i], t = i;
+    while (true) {
+      int tp = -1;
+      for (int k = t - 1; k >= 0; --k)
+        if (jbuf[k] == p) { tp = k; break; }
+      if (tp < 0) break;
+      p = tp;
+      t = tp;
     }
+    out[i] = p;
   }
   __syncthreads();
   return true;

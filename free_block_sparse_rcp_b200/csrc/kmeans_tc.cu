@@ -32,15 +32,10 @@ __global__ void __launch_bounds__(256) k_seed_rows(const __nv_bfloat16* __restri
                                                   uint64_t seed, int purpose, float* __restrict__ m,
                                                   int* __restrict__ init_out, int* err) {
   extern __shared__ __align__(16) unsigned char smem_seed[];
-  int* mkey = reinterpret_cast<int*>(smem_seed);
-  int* mval = mkey + kMapCap;
-  int* sidx = mval + kMapCap;
-  int* jbuf = sidx + G;
+  int* sidx = reinterpret_cast<int*>(smem_seed);   // [G] drawn rows
+  int* jbuf = sidx + G;                             // [G] the draws' offsets
   const int bh = blockIdx.x, tid = threadIdx.x;
-  SlotMap map{mkey, mval, kMapCap};
-  map.clear_all(tid, blockDim.x);
-  __syncthreads();
-  if (!draw_without_replacement_block(stream_state(seed, bh, purpose), N, G, map, sidx, jbuf)) {
+  if (!draw_without_replacement_block(stream_state(seed, bh, purpose), N, G, kMapCap, sidx, jbuf)) {
     if (tid == 0) set_error(err, DERR_DRAW);
     return;
   }
@@ -1069,7 +1064,7 @@ KmPlan kmeans_plan(int BH, int N) {
 
 cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_t seed, int purpose, float* m,
                              int* init_out, int* err, cudaStream_t st) {
-  const size_t sm = (size_t)(2 * km::kMapCap + 2 * G) * 4;
+  const size_t sm = (size_t)2 * G * 4;
   cudaFuncSetAttribute(km::k_seed_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   km::k_seed_rows<<<BH, 256, sm, st>>>((const __nv_bfloat16*)X, N, d, G, seed, purpose, m, init_out, err);
   return cudaGetLastError();

@@ -26,16 +26,11 @@ __global__ void __launch_bounds__(D * D / 16) k_sample_metric(const __nv_bfloat1
                                                              int Ms, uint64_t seed, float* __restrict__ metric,
                                                              int* __restrict__ sample_idx, int* err) {
   extern __shared__ __align__(16) unsigned char smem[];
-  int* mkey = reinterpret_cast<int*>(smem);
-  int* mval = mkey + kMapCap;
-  int* sidx = mval + kMapCap;                                   // [Ms]
+  int* sidx = reinterpret_cast<int*>(smem);                     // [Ms]
   float* qs = reinterpret_cast<float*>(sidx + ((Ms + 3) & ~3)); // [64][D]
   const int bh = blockIdx.x, tid = threadIdx.x;
-  SlotMap map{mkey, mval, kMapCap};
-  map.clear_all(tid, blockDim.x);
-  __syncthreads();
   // the draw's offsets go to the (not yet used) row buffer: Ms <= kMapCap / 2 <= 64 D
-  if (!draw_without_replacement_block(stream_state(seed, bh, PURPOSE_QUERY_SAMPLE), N, Ms, map, sidx,
+  if (!draw_without_replacement_block(stream_state(seed, bh, PURPOSE_QUERY_SAMPLE), N, Ms, kMapCap, sidx,
                                       reinterpret_cast<int*>(qs))) {
     if (tid == 0) set_error(err, DERR_DRAW);
     return;
@@ -522,7 +517,7 @@ __global__ void __launch_bounds__(256) k_block_mask(const unsigned char* __restr
 // Host-side launchers
 // ---------------------------------------------------------------------------
 static size_t sample_smem(int Ms, int D) {
-  return (size_t)(2 * kMapCap + ((Ms + 3) & ~3)) * 4 + (size_t)64 * D * 4;
+  return (size_t)((Ms + 3) & ~3) * 4 + (size_t)64 * D * 4;
 }
 
 cudaError_t launch_sample_metric(const void* Q, int BH, int N, int D, int Ms, uint64_t seed, float* metric,
