@@ -39,9 +39,19 @@ __global__ void __launch_bounds__(256) k_seed_rows(const __nv_bfloat16* __restri
     if (tid == 0) set_error(err, DERR_DRAW);
     return;
   }
-  for (int e = tid; e < G * d; e += blockDim.x) {
-    const int g = e / d, c = e - g * d;
-    m[(size_t)bh * G * d + e] = bf2f(X[((size_t)bh * N + sidx[g]) * d + c]);
+  // 16-byte pieces of the drawn rows (rows are 16-byte aligned: d is a multiple of 8), four
+  // loads in flight per thread
+  const int VPR = d / 8;
+#pragma unroll 4
+  for (int e = tid; e < G * VPR; e += blockDim.x) {
+    const int g = e / VPR, v = e - g * VPR;
+    const uint4 x = *reinterpret_cast<const uint4*>(X + ((size_t)bh * N + sidx[g]) * d + v * 8);
+    const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+    const float2 f0 = __bfloat1622float2(x2[0]), f1 = __bfloat1622float2(x2[1]);
+    const float2 f2 = __bfloat1622float2(x2[2]), f3 = __bfloat1622float2(x2[3]);
+    float4* dst = reinterpret_cast<float4*>(m + ((size_t)bh * G + g) * d + v * 8);
+    dst[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
+    dst[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
   }
   if (init_out)
     for (int g = tid; g < G; g += blockDim.x) init_out[(size_t)bh * G + g] = sidx[g];

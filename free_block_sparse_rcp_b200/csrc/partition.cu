@@ -46,9 +46,15 @@ __global__ void __launch_bounds__(D * D / 16) k_sample_metric(const __nv_bfloat1
   const __nv_bfloat16* Qh = Q + (size_t)bh * N * D;
   for (int s0 = 0; s0 < Ms; s0 += 64) {
     const int ns = min(64, Ms - s0);
-    for (int e = tid; e < ns * D; e += blockDim.x) {
-      int s = e / D, c = e - s * D;
-      qs[s * D + c] = bf2f(Qh[(size_t)sidx[s0 + s] * D + c]);
+    for (int e = tid; e < ns * (D / 8); e += blockDim.x) {   // 16-byte pieces of the rows
+      const int s = e / (D / 8), v = e - s * (D / 8);
+      const uint4 x = *reinterpret_cast<const uint4*>(Qh + (size_t)sidx[s0 + s] * D + v * 8);
+      const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&x);
+      const float2 f0 = __bfloat1622float2(x2[0]), f1 = __bfloat1622float2(x2[1]);
+      const float2 f2 = __bfloat1622float2(x2[2]), f3 = __bfloat1622float2(x2[3]);
+      float4* dst = reinterpret_cast<float4*>(qs + s * D + v * 8);
+      dst[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
+      dst[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
     }
     __syncthreads();
     for (int s = 0; s < ns; ++s) {
