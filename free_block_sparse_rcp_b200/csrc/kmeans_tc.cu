@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
     const int b_lo = h0 / pp.per, b_hi = min(pp.grid - 1, (h1 - 1) / pp.per);
     for (int b = b_lo; b <= b_hi; ++b) {
       const int slot = b * pp.maxh + (bh - (b * pp.per) / pp.T);
+#pragma unroll 8
       for (int e = tid; e < (g1 - g0) * d; e += CW_THREADS) {
         const int gi = e / d, c = e - gi * d;
         acc[gi * d + c] += (double)pp.psum[((size_t)slot * GP + g0 + gi) * d + c];
@@ -165,11 +166,14 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
     if (mode == 2) return;
   }
   const float* Ah = A + a_head * bh;
+  // staging loops unrolled so that each thread keeps several loads in flight
+#pragma unroll 8
   for (int e = tid; e < D * d; e += CW_THREADS) {
     const int j = e / d, c = e - j * d;
     sA[j * (d + 1) + c] = Ah[(size_t)j * sj + (size_t)c * sc];
   }
   __syncthreads();
+#pragma unroll 8
   for (int e = tid; e < WG_PER_CTA * d; e += CW_THREADS) {
     const int gi = e / d, c = e - gi * d, g = g0 + gi;
     sMg[e] = (g < g1 && g < G) ? m[((size_t)bh * G + g) * d + c] : 0.f;
@@ -694,10 +698,13 @@ __global__ void __launch_bounds__(512) k_assign_recheck(const __nv_bfloat16* __r
   const size_t head = (size_t)bh * N;
   const float* Ah = A + a_head * bh;
   const float* nuh = nu + (size_t)bh * G * DT;
+  // staging loops unrolled so that each thread keeps several loads in flight
+#pragma unroll 8
   for (int e = threadIdx.x; e < D * d; e += 512) {
     const int j = e / d, c = e - j * d;
     sA[j * (d + 1) + c] = Ah[(size_t)j * sj + (size_t)c * sc];
   }
+#pragma unroll 8
   for (int e = threadIdx.x; e < G * DT; e += 512) {
     const int g = e / DT, c = e - g * DT;
     sNu[g * (DT + 1) + c] = nuh[e];

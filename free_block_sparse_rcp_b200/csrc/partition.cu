@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(1024) k_metric_eigen(const float* __restrict__
   double* lam = Z + D * ldz;                    // [64]
   double* sc = lam + 64;                        // SymEigScratch<D>
   const int bh = blockIdx.x;
+#pragma unroll 8
   for (int i = threadIdx.x; i < D * D; i += blockDim.x) {
     const int r = i / D, c = i - r * D;
     A[r * LD + c] = (double)metric[(size_t)bh * D * D + i];

@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
   float* Xm = Rm + PR * D;                         // [PR][D]
   const int bh = blockIdx.x, tid = threadIdx.x, nt = blockDim.x;
   // the Gram is padded to PR x PR with zero rows (P <= PR): padding adds zero eigenvalues only
+#pragma unroll 4
   for (int e = tid; e < PR * D; e += nt) {
     const int r = e / D;
     float od = 0.f, os = 0.f;
