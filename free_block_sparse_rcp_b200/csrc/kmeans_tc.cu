@@ -102,19 +102,28 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
   const int g0 = blockIdx.x * WG_PER_CTA, g1 = min(GP, g0 + WG_PER_CTA);
   if (mode != 0) {
     // ---- means from the partial sums of the previous pass
-    for (int e = tid; e < WG_PER_CTA * d; e += CW_THREADS) acc[e] = 0.0;
-    if (tid < WG_PER_CTA) cnt[tid] = 0;
-    __syncthreads();
     const int h0 = bh * pp.T, h1 = h0 + pp.T;
     const int b_lo = h0 / pp.per, b_hi = min(pp.grid - 1, (h1 - 1) / pp.per);
-    for (int b = b_lo; b <= b_hi; ++b) {
-      const int slot = b * pp.maxh + (bh - (b * pp.per) / pp.T);
-#pragma unroll 8
-      for (int e = tid; e < (g1 - g0) * d; e += CW_THREADS) {
-        const int gi = e / d, c = e - gi * d;
-        acc[gi * d + c] += (double)pp.psum[((size_t)slot * GP + g0 + gi) * d + c];
+    // per element, the slots in ascending CTA order (0 + s_lo + ... + s_hi, as the definition
+    // of the mean reads); the loads of all slots of an element are independent and go out
+    // together
+    for (int e = tid; e < WG_PER_CTA * d; e += CW_THREADS) {
+      const int gi = e / d, c = e - gi * d;
+      double a = 0.0;
+      if (gi < g1 - g0) {
+#pragma unroll 4
+        for (int b = b_lo; b <= b_hi; ++b) {
+          const int slot = b * pp.maxh + (bh - (b * pp.per) / pp.T);
+          a += (double)pp.psum[((size_t)slot * GP + g0 + gi) * d + c];
+        }
       }
-      if (tid < g1 - g0) cnt[tid] += pp.pcnt[(size_t)slot * GP + g0 + tid];
+      acc[e] = a;
+    }
+    if (tid < WG_PER_CTA) {
+      int n = 0;
+      if (tid < g1 - g0)
+        for (int b = b_lo; b <= b_hi; ++b) n += pp.pcnt[(size_t)(b * pp.maxh + (bh - (b * pp.per) / pp.T)) * GP + g0 + tid];
+      cnt[tid] = n;
     }
     __syncthreads();
     if (warp == 0) {
