@@ -588,24 +588,39 @@ class ProbeFit:
     bmat: np.ndarray           # [d, d] = w @ vr^T  (the pages' B)
 
 
-def fit_from_probes(probe_idx, o_dense, o_sparse, lse_dense, lse_sparse, rank: int,
-                    lam: float, weights=None) -> ProbeFit:
-    """R_P = O_dense - O_sparse on the probes; V_r = top singular subspace of R_P;
-    Y = R_P V_r; ridge fit Y ~ b + (x V_r) W_sub with x = the probe rows' sparse output.
+FIT_INPUTS = ("full", "subspace")
 
-    READING: the affine map works inside the subspace on both sides (abstract: "affine
-    correction from the sparse output within the output subspace observed in the probe
-    residuals"; gist 2.B: the subspace keeps the correction away from directions the
-    probes did not observe): its input is the sparse output projected on V_r, so the fit
-    has r + 1 parameters per direction for the P probes instead of d + 1.  Returned as
-    w = V_r W_sub (d x r), so a row's residual coordinates are x w."""
+
+def fit_from_probes(probe_idx, o_dense, o_sparse, lse_dense, lse_sparse, rank: int,
+                    lam: float, weights=None, fit_input: str = "full") -> ProbeFit:
+    """R_P = O_dense - O_sparse on the probes; V_r = top singular subspace of R_P;
+    Y = R_P V_r; ridge fit of Y ~ b + (input) W with x = the probe rows' sparse output.
+
+    The pages write the residual as an affine function of the sparse output, R ~ b + xB,
+    fitted by ridge, with the *correction* projected onto the subspace of the probe
+    residuals' leading singular vectors (gist 2.B, subspace restriction; hs method: the
+    corrected result may only fall in the residual directions the probes observed).
+    READINGS of the map's input:
+      fit_input="full" (default): x is the whole d-dimensional sparse output row, the
+        pages' R ~ b + xB taken literally; only the output side is restricted, so
+        B = W V_r^T with W (d x r) the ridge slope onto the residual coordinates Y.
+      fit_input="subspace": x projected on V_r as well (the abstract's "affine correction
+        from the sparse output within the output subspace" read as applying to both
+        sides): Y ~ b + (x V_r) W_sub, r + 1 parameters per direction, returned as
+        w = V_r W_sub so that a row's residual coordinates are x w in both readings."""
+    if fit_input not in FIT_INPUTS:
+        raise ValueError(f"fit_input must be one of {FIT_INPUTS}")
     r_p = np.asarray(o_dense, np.float64) - np.asarray(o_sparse, np.float64)
     vr, sig = probe_subspace(r_p, rank)
     y = r_p @ vr
-    w_sub, b = ridge_fit(np.asarray(o_sparse, np.float64) @ vr, y, lam, weights)
-    w = vr @ w_sub
+    xs = np.asarray(o_sparse, np.float64)
+    if fit_input == "full":
+        w, b = ridge_fit(xs, y, lam, weights)
+    else:
+        w_sub, b = ridge_fit(xs @ vr, y, lam, weights)
+        w = vr @ w_sub
     return ProbeFit(probe_idx=np.asarray(probe_idx), o_dense=np.asarray(o_dense, np.float64),
-                    o_sparse=np.asarray(o_sparse, np.float64), lse_dense=np.asarray(lse_dense),
+                    o_sparse=xs, lse_dense=np.asarray(lse_dense),
                     lse_sparse=np.asarray(lse_sparse), residual=r_p, vr=vr, sigma=sig, w=w, b=b,
                     b_full=vr @ b, bmat=w @ vr.T)
 
@@ -638,6 +653,7 @@ class Params:
     seed: int = 0
     block: int = 64
     fit_weighted: bool = False   # probe weights n_a / alloc_a in the ridge (probe_weights)
+    fit_input: str = "full"      # input of the affine map: "full" sparse output or "subspace" (fit_from_probes)
 
     def eff_scale(self, d: int) -> float:
         return self.scale if self.scale > 0 else 1.0 / math.sqrt(d)
@@ -810,7 +826,7 @@ def probe_fit_head(q, k, v, part_label_q, part_label_k, route, perm_q, q_offsets
     o_d, l_d = attention(q[pidx], k, v, s, mask=None if frames is None else causal_mask(frames, pidx))
     o_s, l_s = sparse_attention(q, k, v, s, route, part_label_q, part_label_k, rows=pidx, frames=frames)
     wts = probe_weights(q_offsets, p.n_probes) if p.fit_weighted else None
-    return fit_from_probes(pidx, o_d, o_s, l_d, l_s, p.sub_rank, p.ridge_lambda, wts)
+    return fit_from_probes(pidx, o_d, o_s, l_d, l_s, p.sub_rank, p.ridge_lambda, wts, p.fit_input)
 
 
 @dataclass

@@ -67,10 +67,11 @@ def test_subspace_rank_deficient_is_zero_columns():
     assert np.all(v0 == 0) and np.all(s0 == 0)
 
 
-def test_correction_exact_for_planted_affine_residual():
+@pytest.mark.parametrize("fit_input", O.FIT_INPUTS)
+def test_correction_exact_for_planted_affine_residual(fit_input):
     # if the residual is exactly an affine map inside the probes' residual span,
     # R = (b + (x V) W) V^T with V the span's basis, the corrected output equals the
-    # dense one on every row
+    # dense one on every row, whichever input the map takes (P = 64 > d + 1 probes)
     rng = np.random.default_rng(5)
     n, d, r, p = 400, 12, 3, 64
     basis = np.linalg.qr(rng.standard_normal((d, r)))[0]
@@ -79,7 +80,8 @@ def test_correction_exact_for_planted_affine_residual():
     o_sparse = rng.standard_normal((n, d))
     o_dense = o_sparse + (b_sub + (o_sparse @ basis) @ w_sub) @ basis.T
     pidx = rng.choice(n, p, replace=False)
-    fit = O.fit_from_probes(pidx, o_dense[pidx], o_sparse[pidx], np.zeros(p), np.zeros(p), r, 1e-12)
+    fit = O.fit_from_probes(pidx, o_dense[pidx], o_sparse[pidx], np.zeros(p), np.zeros(p), r, 1e-12,
+                            fit_input=fit_input)
     np.testing.assert_allclose(fit.vr @ fit.vr.T, basis @ basis.T, atol=1e-9)
     out = O.correct(o_sparse, fit)
     np.testing.assert_allclose(out, o_dense, atol=1e-7)
@@ -87,9 +89,73 @@ def test_correction_exact_for_planted_affine_residual():
     np.testing.assert_allclose(out[pidx], o_dense[pidx], atol=0)
 
 
-def test_fit_ignores_sparse_output_outside_the_subspace():
-    # the map's input is the sparse output projected on the residual subspace: adding
-    # to x any component orthogonal to V_r changes neither the fit nor the correction
+def test_full_input_recovers_residual_driven_from_outside_the_subspace():
+    # R = (b + x M) V^T with M acting on every component of x (gist 2.B: R ~ b + xB,
+    # the correction projected on the subspace): the full-input map recovers it exactly
+    # on every row; the subspace-input map only sees x V and cannot
+    rng = np.random.default_rng(11)
+    n, d, r, p = 500, 10, 3, 64
+    basis = np.linalg.qr(rng.standard_normal((d, d)))[0]
+    v, perp = basis[:, :r], basis[:, r:]
+    m = perp @ rng.standard_normal((d - r, r))       # driven only by x's components outside V
+    b0 = rng.standard_normal(r)
+    o_sparse = rng.standard_normal((n, d))
+    o_dense = o_sparse + (b0 + o_sparse @ m) @ v.T
+    pidx = rng.choice(n, p, replace=False)
+    full = O.fit_from_probes(pidx, o_dense[pidx], o_sparse[pidx], np.zeros(p), np.zeros(p), r, 1e-12,
+                             fit_input="full")
+    np.testing.assert_allclose(O.correct(o_sparse, full), o_dense, atol=1e-7)
+    np.testing.assert_allclose(full.bmat, m @ v.T, atol=1e-8)
+    sub = O.fit_from_probes(pidx, o_dense[pidx], o_sparse[pidx], np.zeros(p), np.zeros(p), r, 1e-12,
+                            fit_input="subspace")
+    rest = np.setdiff1d(np.arange(n), pidx)
+    miss = np.linalg.norm(O.correct(o_sparse, sub)[rest] - o_dense[rest])
+    assert miss > 0.5 * np.linalg.norm((o_sparse[rest] @ m) @ v.T)
+
+
+@pytest.mark.parametrize("fit_input", O.FIT_INPUTS)
+def test_fit_slope_is_the_primal_ridge_of_its_input(fit_input):
+    # the fitted slope equals the primal ridge solution (Xc^T Xc + lam I)^-1 Xc^T Yc of
+    # its reading's input (full x, or x V_r mapped back by V_r), Yc = centred R V_r, and
+    # the intercept b = ybar - xbar W; this checks the dual solve the oracle uses
+    rng = np.random.default_rng(12)
+    p, d, r, lam = 64, 24, 6, 0.05
+    o_s = rng.standard_normal((p, d))
+    o_d = o_s + rng.standard_normal((p, d)) @ np.diag(np.linspace(2, 0.1, d))
+    fit = O.fit_from_probes(np.arange(p), o_d, o_s, np.zeros(p), np.zeros(p), r, lam, fit_input=fit_input)
+    y = (o_d - o_s) @ fit.vr
+    x = o_s if fit_input == "full" else o_s @ fit.vr
+    xc, yc = x - x.mean(0), y - y.mean(0)
+    wp = np.linalg.solve(xc.T @ xc + lam * np.eye(x.shape[1]), xc.T @ yc)
+    w_want = wp if fit_input == "full" else fit.vr @ wp
+    np.testing.assert_allclose(fit.w, w_want, rtol=1e-8, atol=1e-10)
+    np.testing.assert_allclose(fit.b, y.mean(0) - x.mean(0) @ wp, rtol=1e-8, atol=1e-10)
+
+
+@pytest.mark.parametrize("fit_input", O.FIT_INPUTS)
+def test_correction_lies_in_the_probe_residual_subspace(fit_input):
+    # gist 2.B / hs method: whatever the input, the correction of any row falls in the
+    # span of the retained singular directions of the probe residuals
+    rng = np.random.default_rng(13)
+    p, d, r = 64, 16, 4
+    o_s = rng.standard_normal((p, d))
+    o_d = o_s + rng.standard_normal((p, d))
+    fit = O.fit_from_probes(np.arange(p), o_d, o_s, np.zeros(p), np.zeros(p), r, 1e-2, fit_input=fit_input)
+    x = rng.standard_normal((50, d))
+    corr = fit.b_full + x @ fit.bmat
+    np.testing.assert_allclose(corr - corr @ fit.vr @ fit.vr.T, 0, atol=1e-10)
+
+
+def test_fit_rejects_unknown_input():
+    with pytest.raises(ValueError):
+        O.fit_from_probes(np.arange(4), np.ones((4, 3)), np.zeros((4, 3)), np.zeros(4), np.zeros(4), 2, 1e-2,
+                          fit_input="both")
+
+
+def test_subspace_input_ignores_sparse_output_outside_the_subspace():
+    # fit_input="subspace": the map's input is the sparse output projected on the residual
+    # subspace, so adding to x any component orthogonal to V_r changes neither the fit nor
+    # the correction
     rng = np.random.default_rng(6)
     n, d, r, p = 300, 10, 3, 48
     basis = np.linalg.qr(rng.standard_normal((d, d)))[0]
@@ -98,10 +164,11 @@ def test_fit_ignores_sparse_output_outside_the_subspace():
     o_dense = o_sparse + (rng.standard_normal(r) + (o_sparse @ v) @ rng.standard_normal((r, r))) @ v.T
     o_dense += 1e-3 * rng.standard_normal((n, d)) @ v @ v.T
     pidx = rng.choice(n, p, replace=False)
-    fit = O.fit_from_probes(pidx, o_dense[pidx], o_sparse[pidx], np.zeros(p), np.zeros(p), r, 1e-2)
+    fit = O.fit_from_probes(pidx, o_dense[pidx], o_sparse[pidx], np.zeros(p), np.zeros(p), r, 1e-2,
+                            fit_input="subspace")
     shift = rng.standard_normal((n, d - r)) @ perp.T
     fit2 = O.fit_from_probes(pidx, o_dense[pidx] + shift[pidx], o_sparse[pidx] + shift[pidx], np.zeros(p),
-                             np.zeros(p), r, 1e-2)
+                             np.zeros(p), r, 1e-2, fit_input="subspace")
     np.testing.assert_allclose(fit2.vr @ fit2.vr.T, fit.vr @ fit.vr.T, atol=1e-9)
     np.testing.assert_allclose(fit2.b_full, fit.b_full, atol=1e-9)
     np.testing.assert_allclose(fit2.bmat, fit.bmat, atol=1e-9)
