@@ -286,6 +286,7 @@ def run_cuda(args):
     attn_ms = ta[0].elapsed_time(ta[1]) / n_iso
     pk = _peaks()
     achieved = attn_flops / (attn_ms * 1e-3) / 1e12
+    issued_tflops = 4.0 * d * issued_pairs / (attn_ms * 1e-3) / 1e12
     # dense comparator work: every (frame-causal: every visible) pair
     if frames is None:
         dense_pairs = N * N
@@ -314,6 +315,22 @@ def run_cuda(args):
 
     err_sparse = rel(o_sparse, o_dense)
     err_recon = rel(o, o_dense)
+    # the other reading of the affine map's input, on the same partition and sparse output
+    p_alt = spr.Params.make(**dict(pd, fit_input=1 - pd.get("fit_input", 0)), frame_id=fid,
+                            n_frames=w.grid[0] if w.frame_causal else 0)
+    pr_alt = spr.alloc_probe(p_alt, dev)
+    spr.sparsepr_probe_fit(p_alt, Ql, Kl, Vl, part["label_k"], part["perm_q"], part["qoff"], part["route"],
+                           pr_alt["probe_idx"], pr_alt["probe_o_dense"], pr_alt["b_full"], pr_alt["Vr"], pr_alt["W"],
+                           None, wsb)
+    o_alt = torch.empty_like(Q)
+    spr.sparsepr_reconstruct(p_alt, o_sparse, pr_alt["probe_idx"], pr_alt["probe_o_dense"], pr_alt["b_full"],
+                             pr_alt["Vr"], pr_alt["W"], o_alt)
+    torch.cuda.synchronize()
+    err_alt = rel(o_alt, o_dense)
+    del o_alt, pr_alt
+    readings = {0: "whole sparse output", 1: "sparse output projected on the subspace"}
+    fit_errors = {readings[pd.get("fit_input", 0)] + " (this run's)": round(err_recon, 5),
+                  readings[1 - pd.get("fit_input", 0)]: round(err_alt, 5)}
 
     # --- end to end through the C ABI from pinned host buffers
     Qh, Kh, Vh = (torch.empty(Q.shape, dtype=torch.bfloat16, pin_memory=True) for _ in range(3))
@@ -323,6 +340,7 @@ def run_cuda(args):
     o_dev = torch.empty_like(Q)
     fws = spr.workspace(p, dev, forward=True)
     e2e_steps = max(2, min(args.steps, 5))
+    timed_launches = launches[0]
     for _ in range(2):
         spr.sparsepr_forward_host(p, Qh, Kh, Vh, Oh, qkv_dev, o_dev, fws)
     torch.cuda.synchronize()
@@ -337,11 +355,51 @@ def run_cuda(args):
     e2e_total = max_over_ranks(a0.elapsed_time(a1), ws, dev)
     e2e_single = e2e_total / (e2e_steps * ws)
     bytes_in = 3 * BH * N * d * 2
-    # the same call as a pipeline over head chunks: the host-to-device copies of chunk i + 1
-    # and the device-to-host copy of chunk i - 1 run beside the compute of chunk i
-    del qkv_dev, o_dev, fws
-    pipe_ms, n_chunks = e2e_pipeline(spr, pd, p, fid, Qh, Kh, Vh, Oh, dev, e2e_steps)
+    # the same call through the library's pipeline over head chunks: the host-to-device
+    # copies of chunk i + 1 and the device-to-host copy of chunk i - 1 run beside the
+    # compute of chunk i (one C-ABI call per step; same outputs as the unsplit call)
+    del fws
+    oh_single = Oh.clone()
+    n_chunks = next(c for c in (4, 2, 1) if BH >= c)
+    cws = spr.workspace(spr.chunk_params(p, n_chunks), dev, forward=True)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    for _ in range(2):
+        spr.sparsepr_forward_host_chunked(p, Qh, Kh, Vh, Oh, qkv_dev, o_dev, n_chunks, cws, s_in, s_out)
+    torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for _ in range(e2e_steps):
+        spr.sparsepr_forward_host_chunked(p, Qh, Kh, Vh, Oh, qkv_dev, o_dev, n_chunks, cws, s_in, s_out)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    pipe_ms = c0.elapsed_time(c1) / e2e_steps
     e2e_value = max_over_ranks(pipe_ms, ws, dev) / ws
+    e2e_same = bool(torch.equal(Oh, oh_single))
+    del qkv_dev, o_dev, cws
+
+    # --- a second seed of the generator (rank r draws seed 2 r + s): one call, its own dense
+    seeds = {"0": {"ms_per_call": round(ms_per_call, 4), "o_sparse": round(err_sparse, 5),
+                   "o_reconstructed": round(err_recon, 5)}}
+    if args.seed1:
+        q1, k1, v1 = (to_torch(x, dev) for x in generate(w, seed=2 * rank + 1))
+        for _ in range(2):
+            call(q1, k1, v1)
+        torch.cuda.synchronize()
+        ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        n1 = max(3, min(args.steps, 10))
+        s0 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(n1):
+            call(q1, k1, v1, ev1)
+        torch.cuda.synchronize()
+        ms1 = s0.elapsed_time(ev1[4]) / n1
+        spr.sparsepr_dense_attention(p, q1, k1, v1, o_dense, None, wsb)
+        torch.cuda.synchronize()
+        seeds["1"] = {"ms_per_call": round(ms1, 4), "o_sparse": round(rel(o_sparse, o_dense), 5),
+                      "o_reconstructed": round(rel(o, o_dense), 5)}
+        del q1, k1, v1
 
     traffic = _traffic_record("attend_causal" if w.frame_causal else "attend")
     rho = part["rho_exec"].float()
@@ -360,23 +418,30 @@ def run_cuda(args):
                      "max": round(float(rho.max()), 5)},
         "attend_ms_alone": round(attn_ms, 4),
         "attend_tflops_useful": round(achieved, 2),
-        "attend_tflops_issued": round(4.0 * d * issued_pairs / (attn_ms * 1e-3) / 1e12, 2),
+        "attend_tflops_issued": round(issued_tflops, 2),
         "tile_fill": round(routed_pairs / max(1, issued_pairs), 4),
         "dense_equiv_tflops": round(dense_flops / (ms_per_call * 1e-3) / 1e12, 2),
         "dense_kernel_tflops": round(dense_flops / (dense_ms * 1e-3) / 1e12, 2),
-        "rel_l2_vs_dense": {"o_sparse": round(err_sparse, 5), "o_reconstructed": round(err_recon, 5)},
+        "rel_l2_vs_dense": {"o_sparse": round(err_sparse, 5), "o_reconstructed": round(err_recon, 5),
+                            "o_reconstructed_by_fit_input": fit_errors},
         "roofline": {"kernel": "attend (routed flash attention)", "bound": "tensor", "achieved": round(achieved, 2),
-                     "peak": pk["bf16_sus"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_sus"], 4),
-                     "peak_kind": f"bf16 sustained, {pk['src']}",
-                     "frac_of_burst": round(achieved / pk["bf16"], 4),
-                     "traffic": traffic, "algorithmic_flops_per_launch": attn_flops},
+                     "peak": pk["bf16"], "unit": "TFLOP/s", "frac": round(achieved / pk["bf16"], 4),
+                     "peak_kind": f"bf16 burst, {pk['src']} (the attend stage is timed alone, {n_iso} launches "
+                                  f"back to back, {attn_ms * n_iso:.1f} ms)",
+                     "frac_issued": round(issued_tflops / pk["bf16"], 4),
+                     "frac_of_sustained": round(achieved / pk["bf16_sus"], 4),
+                     "traffic": traffic, "algorithmic_flops_per_launch": attn_flops,
+                     "algorithmic_unit": "4 d flops per routed (query, key) pair of the call's route"},
         "e2e": {"value": round(e2e_value, 4), "unit": UNIT, "h2d_bytes_per_step": bytes_in,
                 "d2h_bytes_per_step": BH * N * d * 2,
-                "how": f"pinned host Q, K, V -> device -> O back to pinned host, through sparsepr_forward on "
-                       f"{n_chunks} head chunks (each an independent call; its heads draw the random "
-                       f"streams of heads 0..) with the copies of neighbouring chunks on two copy streams",
-                "single_call_ms": round(e2e_single, 4)},
-        "gpu_launches": launches[0],
+                "how": f"pinned host Q, K, V -> device -> O back to pinned host in one C-ABI call, "
+                       f"sparsepr_forward_host_chunked: {n_chunks} head chunks (head_offset numbering, so the "
+                       f"output is the unsplit call's), copies in / compute / copies out on three streams",
+                "single_call_ms": round(e2e_single, 4),
+                "single_call_how": "sparsepr_forward_host: copies, call and copy back in sequence on one stream",
+                "same_output_as_single_call": e2e_same},
+        "seeds": seeds,
+        "gpu_launches": timed_launches,
         "clocks": clk.summary(),
     }
     if calls > 1:
@@ -395,59 +460,6 @@ def run_cuda(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
-
-
-def e2e_pipeline(spr, pd, p, fid, Qh, Kh, Vh, Oh, dev, steps, chunks=4):
-    """ms per call from pinned host buffers to pinned host buffers, the heads split into
-    `chunks` calls of sparsepr_forward: chunk i's host-to-device copies run on one copy
-    stream, its compute on another, its output's copy back on a third, two chunk slots."""
-    import torch
-    BH, N, d = p.BH, p.N, p.d
-    C = next(c for c in (chunks, 4, 2, 1) if BH % c == 0 and BH >= c)
-    hs = BH // C
-    pc = spr.Params.make(**dict(pd, B=1, H=hs), frame_id=fid, n_frames=p.n_frames)
-    qh, kh, vh, oh = (t.view(BH, N, d) for t in (Qh, Kh, Vh, Oh))
-    slots = [dict(q=torch.empty(1, hs, N, d, dtype=torch.bfloat16, device=dev),
-                  k=torch.empty(1, hs, N, d, dtype=torch.bfloat16, device=dev),
-                  v=torch.empty(1, hs, N, d, dtype=torch.bfloat16, device=dev),
-                  o=torch.empty(1, hs, N, d, dtype=torch.bfloat16, device=dev),
-                  ws=spr.workspace(pc, dev, forward=True),
-                  free=torch.cuda.Event(), done=torch.cuda.Event(), out=torch.cuda.Event())
-             for _ in range(2)]
-    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
-    for sl in slots:
-        sl["out"].record(s_out)
-
-    def one_call():
-        for i in range(C):
-            sl = slots[i % 2]
-            h0, h1 = i * hs, (i + 1) * hs
-            s_in.wait_event(sl["done"] if i >= 2 else sl["out"])
-            with torch.cuda.stream(s_in):
-                sl["q"][0].copy_(qh[h0:h1], non_blocking=True)
-                sl["k"][0].copy_(kh[h0:h1], non_blocking=True)
-                sl["v"][0].copy_(vh[h0:h1], non_blocking=True)
-                sl["free"].record(s_in)
-            s_comp.wait_event(sl["free"])
-            s_comp.wait_event(sl["out"])      # the slot's previous output has left the device
-            with torch.cuda.stream(s_comp):
-                spr.sparsepr_forward(pc, sl["q"], sl["k"], sl["v"], sl["o"], None, sl["ws"])
-                sl["done"].record(s_comp)
-            s_out.wait_event(sl["done"])
-            with torch.cuda.stream(s_out):
-                oh[h0:h1].copy_(sl["o"][0], non_blocking=True)
-                sl["out"].record(s_out)
-
-    for _ in range(2):
-        one_call()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    for _ in range(steps):
-        one_call()
-    e1.record(s_out)
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / steps, C
 
 
 def bench_workload(args, heads=True):
@@ -610,12 +622,39 @@ def _cores():
         return os.cpu_count()
 
 
+def oracle_whole(name: str, threads=None, seed=0):
+    """Seconds of the oracle's whole call (every head, every row) on a small workload;
+    threads: cap on the BLAS threads (None: as configured)."""
+    import contextlib
+    import oracle as O
+    from synth import generate, to_f64, workload
+    w = workload(name)
+    qb, kb, vb = generate(w, seed=seed)
+    p = O.Params(n_kgroups=w.n_kgroups, n_qgroups=w.n_qgroups, n_samples=w.n_samples, n_probes=w.n_probes,
+                 eig_rank=w.eig_rank, sub_rank=w.sub_rank, kmeans_iters=w.kmeans_iters, density=w.density,
+                 ridge_lambda=w.ridge_lambda, seed=seed, block=w.block)
+    ctx = contextlib.nullcontext()
+    if threads is not None:
+        from threadpoolctl import threadpool_limits
+        ctx = threadpool_limits(threads)
+    with ctx:
+        t0 = time.perf_counter()
+        for b in range(w.B):
+            for h in range(w.H):
+                O.sparsepr_head(to_f64(qb[b, h]), to_f64(kb[b, h]), to_f64(vb[b, h]), p, b * w.H + h)
+        return time.perf_counter() - t0
+
+
 def cpu_baseline(w):
     sec, spent, nrows = oracle_sample(w)
+    whole = {"tiny (1024 tokens x 2 heads)": round(oracle_whole("tiny"), 3),
+             "tiny, 1 thread": round(oracle_whole("tiny", threads=1), 3),
+             "mid (8192 tokens x 12 heads)": round(oracle_whole("mid"), 2)}
     return {"value": round(sec * 1e3, 1), "unit": UNIT, "cores": _cores(), "kind": "oracle",
             "sample": f"head (0,0) of {w.B * w.H}: full partition, probes and fit; routed attention and "
                       f"correction on {nrows} of {w.N} rows; extrapolated x{w.B * w.H} heads "
-                      f"(took {spent:.1f} s)"}
+                      f"(took {spent:.1f} s)",
+            "whole_call_s": whole}
 
 
 def run_reference(args):
@@ -663,6 +702,8 @@ def main():
                     help="add support and affine-explainability measurements of two heads to the line")
     ap.add_argument("--streams", type=int, default=2, choices=[1, 2],
                     help="2: probe_fit beside the routed attention on a second stream (default); 1: in sequence")
+    ap.add_argument("--no-seed1", dest="seed1", action="store_false",
+                    help="skip the one-call measurement on the generator's second seed")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (small cases for ncu captures; default: the workload's 40)")
     args = ap.parse_args()

@@ -31,7 +31,8 @@ class Params(ctypes.Structure):
                 ("eig_rank", ctypes.c_int), ("sub_rank", ctypes.c_int), ("kmeans_iters", ctypes.c_int),
                 ("ridge_lambda", ctypes.c_float), ("scale", ctypes.c_float), ("seed", ctypes.c_ulonglong),
                 ("frame_id", _vp), ("n_frames", ctypes.c_int), ("partition_mode", ctypes.c_int),
-                ("fit_weighted", ctypes.c_int)]
+                ("fit_weighted", ctypes.c_int), ("fit_input", ctypes.c_int), ("head_offset", ctypes.c_int),
+                ("heads_total", ctypes.c_int)]
 
     @property
     def BH(self) -> int:
@@ -50,15 +51,18 @@ class Params(ctypes.Structure):
     @classmethod
     def make(cls, B, H, N, d, *, block, density, n_kgroups, n_qgroups, n_samples, n_probes, eig_rank,
              sub_rank, kmeans_iters, ridge_lambda=1e-2, scale=0.0, seed=0, frame_id=None, n_frames=0,
-             partition_mode=0, fit_weighted=0):
+             partition_mode=0, fit_weighted=0, fit_input=0, head_offset=0, heads_total=0):
         """frame_id: optional int32 device tensor [N] (frame-causal masking, kept alive by the
-        caller for as long as the params are used)."""
+        caller for as long as the params are used).  fit_input: 0 = the affine map takes the
+        whole sparse output row, 1 = its projection on the residual subspace.  head_offset /
+        heads_total: this call's heads within the layer (random streams only)."""
         fid = None if frame_id is None else frame_id.data_ptr()
         return cls(B=B, H=H, N=N, d=d, block=block, density=density, n_kgroups=n_kgroups,
                    n_qgroups=n_qgroups, n_samples=n_samples, n_probes=n_probes, eig_rank=eig_rank,
                    sub_rank=sub_rank, kmeans_iters=kmeans_iters, ridge_lambda=ridge_lambda, scale=scale,
                    seed=seed, frame_id=fid, n_frames=n_frames, partition_mode=partition_mode,
-                   fit_weighted=fit_weighted)
+                   fit_weighted=fit_weighted, fit_input=fit_input, head_offset=head_offset,
+                   heads_total=heads_total)
 
 
 class PartitionTrace(ctypes.Structure):
@@ -89,6 +93,8 @@ _sig = {
     "sparsepr_reconstruct": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "sparsepr_forward": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "sparsepr_forward_host": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "sparsepr_forward_host_chunked": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int, _vp,
+                                                     ctypes.c_size_t, _vp, _vp, _vp]),
     "sparsepr_dense_attention": (ctypes.c_int, [_P, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "sparsepr_workspace_error": (ctypes.c_int, [_P, _vp, _vp]),
     "sparsepr_workspace_clear_error": (ctypes.c_int, [_P, _vp, _vp]),
@@ -209,6 +215,26 @@ def sparsepr_forward_host(p, Q_host, K_host, V_host, O_host, qkv_dev, o_dev, ws)
     _check(_lib.sparsepr_forward_host(ctypes.byref(p), _ptr(Q_host), _ptr(K_host), _ptr(V_host),
                                       _ptr(O_host), _ptr(qkv_dev), _ptr(o_dev), _ptr(ws), ws.numel(),
                                       _stream(qkv_dev)), "sparsepr_forward_host")
+
+
+def sparsepr_forward_host_chunked(p, Q_host, K_host, V_host, O_host, qkv_dev, o_dev, n_chunks, ws,
+                                  copy_in_stream=None, copy_out_stream=None):
+    """The chunked host pipeline on the current stream of qkv_dev's device; the copy streams
+    are torch.cuda.Stream objects (None: the current stream)."""
+    def sp(s):
+        return None if s is None else ctypes.c_void_p(s.cuda_stream)
+    _check(_lib.sparsepr_forward_host_chunked(ctypes.byref(p), _ptr(Q_host), _ptr(K_host), _ptr(V_host),
+                                              _ptr(O_host), _ptr(qkv_dev), _ptr(o_dev), int(n_chunks), _ptr(ws),
+                                              ws.numel(), _stream(qkv_dev), sp(copy_in_stream),
+                                              sp(copy_out_stream)), "sparsepr_forward_host_chunked")
+
+
+def chunk_params(p: Params, n_chunks: int) -> Params:
+    """Params of the largest chunk of sparsepr_forward_host_chunked (for its workspace size)."""
+    q = Params.from_buffer_copy(p)
+    q.B, q.H = 1, -(-p.BH // n_chunks)
+    q.head_offset, q.heads_total = 0, 0
+    return q
 
 
 def sparsepr_dense_attention(p, Q, K, V, O, lse, ws=None):

@@ -177,6 +177,14 @@ sparsepr_status check_params(const sparsepr_params* p) {
   if (!(p->scale >= 0.f) || !isfinite(p->scale)) return fail(SPARSEPR_EINVAL, "scale must be >= 0");
   if (p->fit_weighted != 0 && p->fit_weighted != 1)
     return failv(SPARSEPR_EINVAL, "fit_weighted must be 0 or 1", p->fit_weighted);
+  if (p->fit_input != 0 && p->fit_input != 1)
+    return failv(SPARSEPR_EINVAL, "fit_input must be 0 (whole sparse output) or 1 (projected on the subspace)",
+                 p->fit_input);
+  if (p->head_offset < 0) return failv(SPARSEPR_EINVAL, "head_offset must be >= 0", p->head_offset);
+  if (p->heads_total != 0 && (p->heads_total < 0 || (long long)p->heads_total < (long long)p->head_offset + p->H))
+    return failv(SPARSEPR_EINVAL, "heads_total must be 0 or >= head_offset + H", p->heads_total);
+  if ((long long)(p->B - 1) * (p->heads_total ? p->heads_total : p->H) + p->head_offset + p->H > (1ll << 28))
+    return fail(SPARSEPR_EINVAL, "layer head index out of range");
   if (p->partition_mode != 0 && p->partition_mode != 1)
     return failv(SPARSEPR_EINVAL, "partition_mode must be 0 (response-coupled) or 1 (semantic)", p->partition_mode);
   if (p->frame_id) {
@@ -224,6 +232,15 @@ T* at(void* ws, size_t off) {
 
 float eff_scale(const sparsepr_params& p) { return p.scale > 0.f ? p.scale : 1.0f / sqrtf((float)p.d); }
 
+// layer-wide head index of the random streams (head_offset / heads_total)
+HeadMap head_map(const sparsepr_params& p) {
+  HeadMap hm;
+  hm.H = p.H;
+  hm.total = p.heads_total ? p.heads_total : p.H;
+  hm.offset = p.head_offset;
+  return hm;
+}
+
 #define SPR_CHECK(expr)                          \
   do {                                           \
     sparsepr_status s_ = (expr);                 \
@@ -244,16 +261,17 @@ float eff_scale(const sparsepr_params& p) { return p.scale > 0.f ? p.scale : 1.0
 sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const void* Q, const void* K, int* perm_q,
                               int* perm_k, int* label_q, int* label_k, int* qoff, int* koff, unsigned char* route,
                               unsigned char* bmask, float* rho, const sparsepr_partition_trace* tr, void* ws,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool clear_err = true) {
   const int BH = L.BH, N = p.N, d = p.d, Gk = p.n_kgroups, Gq = p.n_qgroups, re = p.eig_rank;
   const float scale = eff_scale(p);
   int* err = at<int>(ws, L.err);
-  SPR_CUDA(cudaMemsetAsync(err, 0, 4, st));
+  if (clear_err) SPR_CUDA(cudaMemsetAsync(err, 0, 4, st));
   float* metric = at<float>(ws, L.metric);
   float* proj = at<float>(ws, L.proj);
   const bool semantic = p.partition_mode == 1;
   if (!semantic) {
-    SPR_LAUNCH(launch_sample_metric(Q, BH, N, d, p.n_samples, p.seed, metric, at<int>(ws, L.sample_idx), err, st));
+    SPR_LAUNCH(launch_sample_metric(Q, BH, N, d, p.n_samples, p.seed, head_map(p), metric, at<int>(ws, L.sample_idx),
+                                    err, st));
     SPR_LAUNCH(launch_metric_eigen(metric, BH, d, re, at<float>(ws, L.eigval), at<float>(ws, L.eigvec), proj,
                                    at<double>(ws, L.eig_lu), st));
     if (tr && tr->key_coords) SPR_LAUNCH(launch_key_coords(K, BH, N, d, re, proj, tr->key_coords, st));
@@ -276,7 +294,7 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
   auto kmeans = [&](const void* X, int G, int purpose, const float* A, size_t a_head, int sj, int sc, float a_scale,
                     int D, int DT, float* m, float* nu, int* init, int* labels, int* perm, int* off,
                     int* trace_iters, float* means_out) -> sparsepr_status {
-    SPR_LAUNCH(launch_seed_rows(X, BH, N, d, G, p.seed, purpose, m, init, err, st));
+    SPR_LAUNCH(launch_seed_rows(X, BH, N, d, G, p.seed, head_map(p), purpose, m, init, err, st));
     for (int t = 0; t < p.kmeans_iters; ++t) {
       int* trc = trace_iters ? trace_iters + (size_t)t * BH * N : nullptr;
       SPR_LAUNCH(launch_centroid_weights(m, BH, G, d, A, a_head, sj, sc, a_scale, D, DT, t == 0 ? 0 : 1, psum, pcnt,
@@ -400,7 +418,8 @@ sparsepr_status run_probe_fit(const sparsepr_params& p, const Layout& L, const v
                               cudaStream_t st) {
   const int BH = L.BH, N = p.N, d = p.d, P = p.n_probes;
   int* pgrp = at<int>(ws, L.probe_grp);
-  SPR_LAUNCH(launch_probe_pick(perm_q, qoff, BH, N, p.n_qgroups, P, p.seed, probe_idx, pgrp, at<int>(ws, L.err), st));
+  SPR_LAUNCH(launch_probe_pick(perm_q, qoff, BH, N, p.n_qgroups, P, p.seed, head_map(p), probe_idx, pgrp,
+                               at<int>(ws, L.err), st));
   float* part_o = at<float>(ws, L.part_o);
   float* part_ml = at<float>(ws, L.part_ml);
   Causal cz{};
@@ -418,7 +437,7 @@ sparsepr_status run_probe_fit(const sparsepr_params& p, const Layout& L, const v
   SPR_LAUNCH(launch_probe_combine(part_o, part_ml, BH, N, P, d, probe_od, osp, lsd, lss, st));
   SPR_LAUNCH(launch_probe_fit(probe_od, osp, BH, d, P, p.sub_rank, (double)p.ridge_lambda, Vr, W, bfull, Bmat,
                               tr ? tr->sigma : nullptr, tr ? tr->b_sub : nullptr, p.fit_weighted ? pgrp : nullptr,
-                              qoff, p.n_qgroups, st));
+                              qoff, p.n_qgroups, p.fit_input == 0, st));
   if (tr) {
     if (tr->probe_o_sparse)
       SPR_CUDA(cudaMemcpyAsync(tr->probe_o_sparse, osp, (size_t)BH * P * d * 4, cudaMemcpyDeviceToDevice, st));
@@ -515,9 +534,9 @@ sparsepr_status sparsepr_reconstruct(const sparsepr_params* p, const void* O_spa
                          (cudaStream_t)stream);
 }
 
-sparsepr_status sparsepr_forward(const sparsepr_params* p, const void* Q, const void* K, const void* V, void* O,
-                                 float* rho_exec, void* workspace, size_t ws_bytes, void* stream) {
-  g_launches = 0;
+// The whole call on device buffers; clear_err: reset the workspace error word first.
+static sparsepr_status forward_impl(const sparsepr_params* p, const void* Q, const void* K, const void* V, void* O,
+                             float* rho_exec, void* workspace, size_t ws_bytes, void* stream, bool clear_err) {
   SPR_CHECK(check_params(p));
   SPR_TILED(Q); SPR_TILED(K); SPR_TILED(V); SPR_TILED(O);
   const Layout L = make_layout(*p);
@@ -533,7 +552,7 @@ sparsepr_status sparsepr_forward(const sparsepr_params* p, const void* Q, const 
   unsigned char* route = at<unsigned char>(ws, L.f_route);
   float* rho = rho_exec ? rho_exec : at<float>(ws, L.f_rho);
   SPR_CHECK(run_partition(*p, L, Q, K, perm_q, perm_k, label_q, label_k, qoff, koff, route, nullptr, rho, nullptr,
-                          ws, st));
+                          ws, st, clear_err));
   SPR_CHECK(run_attend(*p, L, Q, K, V, perm_q, perm_k, qoff, koff, route, O, at<float>(ws, L.f_lse), ws, st));
   int* pidx = at<int>(ws, L.f_probe_idx);
   float* pod = at<float>(ws, L.f_probe_od);
@@ -544,6 +563,12 @@ sparsepr_status sparsepr_forward(const sparsepr_params* p, const void* Q, const 
                           ws, st));
   SPR_CHECK(run_reconstruct(*p, L.BH, O, pidx, pod, bfull, vr, w, O, st));
   return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_forward(const sparsepr_params* p, const void* Q, const void* K, const void* V, void* O,
+                                 float* rho_exec, void* workspace, size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  return forward_impl(p, Q, K, V, O, rho_exec, workspace, ws_bytes, stream, true);
 }
 
 sparsepr_status sparsepr_forward_host(const sparsepr_params* p, const void* Q_host, const void* K_host,
@@ -562,6 +587,102 @@ sparsepr_status sparsepr_forward_host(const sparsepr_params* p, const void* Q_ho
   SPR_CHECK(sparsepr_forward(p, q, q + bytes, q + 2 * bytes, o_dev, nullptr, workspace, ws_bytes, stream));
   SPR_CUDA(cudaMemcpyAsync(O_host, o_dev, bytes, cudaMemcpyDeviceToHost, st));
   return SPARSEPR_OK;
+}
+
+sparsepr_status sparsepr_forward_host_chunked(const sparsepr_params* p, const void* Q_host, const void* K_host,
+                                              const void* V_host, void* O_host, void* qkv_dev, void* o_dev,
+                                              int n_chunks, void* workspace, size_t ws_bytes, void* stream,
+                                              void* copy_in_stream, void* copy_out_stream) {
+  g_launches = 0;
+  SPR_CHECK(check_params(p));
+  SPR_NONNULL(Q_host); SPR_NONNULL(K_host); SPR_NONNULL(V_host); SPR_NONNULL(O_host); SPR_TILED(qkv_dev);
+  SPR_TILED(o_dev);
+  const int BH = p->B * p->H;
+  if (n_chunks < 1 || n_chunks > BH) return failv(SPARSEPR_EINVAL, "n_chunks must be in [1, B*H]", n_chunks);
+  // chunk ranges over the flattened heads; when the layer numbering is not the identity a
+  // chunk may not cross a batch element (each chunk is a B = 1 call over consecutive layer heads)
+  const HeadMap hm = head_map(*p);
+  const bool ident = hm.total == p->H && hm.offset == 0;
+  const int per = ceil_div(BH, n_chunks);
+  constexpr int kMaxChunks = 512;
+  int starts[kMaxChunks + 1];
+  int nc = 0;
+  for (int h0 = 0; h0 < BH;) {
+    int h1 = h0 + per < BH ? h0 + per : BH;
+    if (!ident && (h0 / p->H) != ((h1 - 1) / p->H)) h1 = (h0 / p->H + 1) * p->H;
+    if (nc >= kMaxChunks) return fail(SPARSEPR_EUNSUPPORTED, "more than 512 chunks");
+    starts[nc++] = h0;
+    h0 = h1;
+  }
+  starts[nc] = BH;
+  int hmax = 0;
+  for (int c = 0; c < nc; ++c) hmax = starts[c + 1] - starts[c] > hmax ? starts[c + 1] - starts[c] : hmax;
+  sparsepr_params pc = *p;
+  pc.B = 1;
+  pc.H = hmax;
+  pc.head_offset = 0;
+  pc.heads_total = 0;
+  SPR_CHECK(check_params(&pc));
+  SPR_CHECK(check_ws(&pc, workspace, ws_bytes, make_layout(pc).forward_total));
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaStream_t sin = copy_in_stream ? (cudaStream_t)copy_in_stream : st;
+  cudaStream_t sout = copy_out_stream ? (cudaStream_t)copy_out_stream : st;
+  const size_t head_bytes = (size_t)p->N * p->d * 2, bytes = (size_t)BH * head_bytes;
+  // events are created here and released once enqueued (a pending event is freed when it
+  // completes); none outlives the call
+  cudaEvent_t ev[2 * kMaxChunks + 2];
+  const int nev = 2 * nc + 2;
+  int made = 0;
+  sparsepr_status status = SPARSEPR_OK;
+  auto cuda = [&](cudaError_t e, const char* where) -> bool {
+    if (e != cudaSuccess && status == SPARSEPR_OK) status = fail_cuda(e, where);
+    return e == cudaSuccess;
+  };
+  for (; made < nev; ++made)
+    if (!cuda(cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming), "cudaEventCreateWithFlags")) break;
+  if (status == SPARSEPR_OK) {
+    cudaEvent_t e_start = ev[0], e_end = ev[1];
+    char* q = static_cast<char*>(qkv_dev);
+    char* o = static_cast<char*>(o_dev);
+    // the copies in wait for earlier work on `stream` (which may still read the staging buffers)
+    // the copies in wait for earlier work on `stream` (which may still read the staging
+    // buffers); the error word is cleared once, so a device error of any chunk stays visible
+    bool ok = cuda(cudaMemsetAsync(workspace, 0, 4, st), "cudaMemsetAsync") &&
+              cuda(cudaEventRecord(e_start, st), "cudaEventRecord") &&
+              cuda(cudaStreamWaitEvent(sin, e_start, 0), "cudaStreamWaitEvent");
+    int launches = 0;
+    for (int c = 0; ok && c < nc; ++c) {
+      const int h0 = starts[c], h1 = starts[c + 1];
+      const size_t off = (size_t)h0 * head_bytes, len = (size_t)(h1 - h0) * head_bytes;
+      cudaEvent_t e_in = ev[2 + 2 * c], e_done = ev[3 + 2 * c];
+      ok = cuda(cudaMemcpyAsync(q + off, static_cast<const char*>(Q_host) + off, len, cudaMemcpyHostToDevice, sin),
+                "cudaMemcpyAsync Q") &&
+           cuda(cudaMemcpyAsync(q + bytes + off, static_cast<const char*>(K_host) + off, len,
+                                cudaMemcpyHostToDevice, sin), "cudaMemcpyAsync K") &&
+           cuda(cudaMemcpyAsync(q + 2 * bytes + off, static_cast<const char*>(V_host) + off, len,
+                                cudaMemcpyHostToDevice, sin), "cudaMemcpyAsync V") &&
+           cuda(cudaEventRecord(e_in, sin), "cudaEventRecord") && cuda(cudaStreamWaitEvent(st, e_in, 0),
+                                                                      "cudaStreamWaitEvent");
+      if (!ok) break;
+      pc.H = h1 - h0;
+      pc.head_offset = hm.global(h0);
+      g_launches = 0;
+      const sparsepr_status s = forward_impl(&pc, q + off, q + bytes + off, q + 2 * bytes + off, o + off, nullptr,
+                                             workspace, ws_bytes, stream, false);
+      launches += g_launches;
+      if (s != SPARSEPR_OK) { status = s; ok = false; break; }
+      ok = cuda(cudaEventRecord(e_done, st), "cudaEventRecord") && cuda(cudaStreamWaitEvent(sout, e_done, 0),
+                                                                        "cudaStreamWaitEvent") &&
+           cuda(cudaMemcpyAsync(static_cast<char*>(O_host) + off, o + off, len, cudaMemcpyDeviceToHost, sout),
+                "cudaMemcpyAsync O");
+    }
+    // `stream` completes only after the last copy out
+    if (ok) ok = cuda(cudaEventRecord(e_end, sout), "cudaEventRecord") &&
+                 cuda(cudaStreamWaitEvent(st, e_end, 0), "cudaStreamWaitEvent");
+    g_launches = launches;
+  }
+  for (int i = 0; i < made; ++i) cudaEventDestroy(ev[i]);
+  return status;
 }
 
 sparsepr_status sparsepr_dense_attention(const sparsepr_params* p, const void* Q, const void* K, const void* V,

@@ -52,6 +52,14 @@ __device__ __forceinline__ uint64_t stream_state(uint64_t seed, int bh, int purp
   return sm64_mix(seed + 0xD1B54A32D192ED03ull * (uint64_t)(8ll * bh + purpose + 1));
 }
 
+// Head index of the random streams: a call over heads [offset, offset + H) of a layer with
+// `total` heads per batch element numbers local head bh = b * H + h as b * total + offset + h,
+// so a head-split call draws exactly the streams the unsplit call draws for those heads.
+struct HeadMap {
+  int H = 1, total = 1, offset = 0;
+  __host__ __device__ int global(int bh) const { return (bh / H) * total + offset + bh % H; }
+};
+
 // Partial Fisher-Yates over the virtual array [0, n) with the swapped slots kept in
 // a small open-addressing map (slot -> value) in shared memory.  One thread runs it.
 struct SlotMap {

@@ -4,6 +4,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "common.cuh"
+
 namespace spr {
 
 // Frame-causal inputs of the kernels below (all NULL / 0 without frame ids).
@@ -19,8 +21,8 @@ struct Causal {
 };
 
 // partition.cu
-cudaError_t launch_sample_metric(const void* Q, int BH, int N, int D, int Ms, uint64_t seed, float* metric,
-                                 int* sample_idx, int* err, cudaStream_t st);
+cudaError_t launch_sample_metric(const void* Q, int BH, int N, int D, int Ms, uint64_t seed, HeadMap hm,
+                                 float* metric, int* sample_idx, int* err, cudaStream_t st);
 size_t metric_eigen_smem(int D, int R);
 cudaError_t launch_metric_eigen(const float* metric, int BH, int D, int R, float* eigval, float* eigvec,
                                 float* proj, double* lu, cudaStream_t st);
@@ -62,8 +64,8 @@ struct alignas(64) TmapBlob {
 int kmeans_gp(int G);
 size_t centroid_weights_smem(int d, int D);
 size_t recheck_smem(int d, int D, int DT, int G);
-cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_t seed, int purpose, float* m,
-                             int* init_out, int* err, cudaStream_t st);
+cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_t seed, HeadMap hm, int purpose,
+                             float* m, int* init_out, int* err, cudaStream_t st);
 // Persistent k-means assignment: CTA b takes the global 128-row tiles [b per, (b+1) per)
 // and leaves one partial-sum slot per head it touches (maxh slots per CTA).
 constexpr int kKmeansCtas = 148;
@@ -93,7 +95,7 @@ cudaError_t launch_worklist(const unsigned char* route, const int* qoff, const i
                            int tile_rows, int max_tiles, int* rlist, int* rcum, int* rcnt, int2* tiles,
                            int* tile_count, cudaStream_t st);
 cudaError_t launch_probe_pick(const int* perm_q, const int* qoff, int BH, int N, int Gq, int P, uint64_t seed,
-                              int* probe_idx, int* probe_grp, int* err, cudaStream_t st);
+                              HeadMap hm, int* probe_idx, int* probe_grp, int* err, cudaStream_t st);
 int probe_splits(int N);
 size_t probe_tc_smem_bytes(int D, int Gk);
 cudaError_t launch_probe_tc(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk, int Gq, int P,
@@ -108,16 +110,18 @@ cudaError_t launch_probe_attn(const void* Q, const void* K, const void* V, int B
 cudaError_t launch_probe_attn_splits(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk,
                                      int Gq, int P, const int* probe_idx, const int* probe_grp, const int* label_k,
                                      const unsigned char* route, float scale_log2, int S, float* part_o,
-                                     float* part_ml, cudaStream_t st);
+                                     float* part_ml, int* err, cudaStream_t st);
 cudaError_t launch_probe_combine_splits(const float* part_o, const float* part_ml, int BH, int S, int P, int D,
                                         float* o_dense, float* o_sparse, float* lse_d, float* lse_s,
                                         cudaStream_t st);
 cudaError_t launch_probe_combine(const float* part_o, const float* part_ml, int BH, int N, int P, int D,
                                  float* o_dense, float* o_sparse, float* lse_d, float* lse_s, cudaStream_t st);
-// probe_grp / qoff: the weighted fit's probe groups and query group offsets (NULL: uniform)
+// probe_grp / qoff: the weighted fit's probe groups and query group offsets (NULL: uniform);
+// full_input: 1 = the map takes the whole sparse output row, 0 = its projection on V_r
 cudaError_t launch_probe_fit(const float* o_dense, const float* o_sparse, int BH, int D, int P, int Rk,
                              double lam, float* Vr, float* W, float* bfull, float* Bmat, float* sigma,
-                             float* bsub, const int* probe_grp, const int* qoff, int Gq, cudaStream_t st);
+                             float* bsub, const int* probe_grp, const int* qoff, int Gq, int full_input,
+                             cudaStream_t st);
 cudaError_t launch_reconstruct(const void* Os, int BH, int N, int D, int Rk, const float* W, const float* Vr,
                                const float* bfull, void* O, cudaStream_t st);
 cudaError_t launch_probe_scatter(const int* probe_idx, const float* o_dense, int BH, int N, int P, int D, void* O,

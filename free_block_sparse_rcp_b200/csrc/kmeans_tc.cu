@@ -29,13 +29,13 @@ using namespace spr::tc;
 constexpr int kMapCap = 4096;
 
 __global__ void __launch_bounds__(256) k_seed_rows(const __nv_bfloat16* __restrict__ X, int N, int d, int G,
-                                                  uint64_t seed, int purpose, float* __restrict__ m,
+                                                  uint64_t seed, HeadMap hm, int purpose, float* __restrict__ m,
                                                   int* __restrict__ init_out, int* err) {
   extern __shared__ __align__(16) unsigned char smem_seed[];
   int* sidx = reinterpret_cast<int*>(smem_seed);   // [G] drawn rows
   int* jbuf = sidx + G;                             // [G] the draws' offsets
   const int bh = blockIdx.x, tid = threadIdx.x;
-  if (!draw_without_replacement_block(stream_state(seed, bh, purpose), N, G, kMapCap, sidx, jbuf)) {
+  if (!draw_without_replacement_block(stream_state(seed, hm.global(bh), purpose), N, G, kMapCap, sidx, jbuf)) {
     if (tid == 0) set_error(err, DERR_DRAW);
     return;
   }
@@ -1088,11 +1088,11 @@ KmPlan kmeans_plan(int BH, int N) {
   return pl;
 }
 
-cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_t seed, int purpose, float* m,
-                             int* init_out, int* err, cudaStream_t st) {
+cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_t seed, HeadMap hm, int purpose,
+                             float* m, int* init_out, int* err, cudaStream_t st) {
   const size_t sm = (size_t)2 * G * 4;
   cudaFuncSetAttribute(km::k_seed_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  km::k_seed_rows<<<BH, 256, sm, st>>>((const __nv_bfloat16*)X, N, d, G, seed, purpose, m, init_out, err);
+  km::k_seed_rows<<<BH, 256, sm, st>>>((const __nv_bfloat16*)X, N, d, G, seed, hm, purpose, m, init_out, err);
   return cudaGetLastError();
 }
 

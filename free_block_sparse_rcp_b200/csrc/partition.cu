@@ -23,14 +23,15 @@ constexpr int kMapCap = 4096;
 
 template <int D>
 __global__ void __launch_bounds__(D * D / 16) k_sample_metric(const __nv_bfloat16* __restrict__ Q, int N,
-                                                             int Ms, uint64_t seed, float* __restrict__ metric,
+                                                             int Ms, uint64_t seed, HeadMap hm,
+                                                             float* __restrict__ metric,
                                                              int* __restrict__ sample_idx, int* err) {
   extern __shared__ __align__(16) unsigned char smem[];
   int* sidx = reinterpret_cast<int*>(smem);                     // [Ms]
   float* qs = reinterpret_cast<float*>(sidx + ((Ms + 3) & ~3)); // [64][D]
   const int bh = blockIdx.x, tid = threadIdx.x;
   // the draw's offsets go to the (not yet used) row buffer: Ms <= kMapCap / 2 <= 64 D
-  if (!draw_without_replacement_block(stream_state(seed, bh, PURPOSE_QUERY_SAMPLE), N, Ms, kMapCap, sidx,
+  if (!draw_without_replacement_block(stream_state(seed, hm.global(bh), PURPOSE_QUERY_SAMPLE), N, Ms, kMapCap, sidx,
                                       reinterpret_cast<int*>(qs))) {
     if (tid == 0) set_error(err, DERR_DRAW);
     return;
@@ -527,15 +528,16 @@ static size_t sample_smem(int Ms, int D) {
   return (size_t)((Ms + 3) & ~3) * 4 + (size_t)64 * D * 4;
 }
 
-cudaError_t launch_sample_metric(const void* Q, int BH, int N, int D, int Ms, uint64_t seed, float* metric,
-                                 int* sample_idx, int* err, cudaStream_t st) {
+cudaError_t launch_sample_metric(const void* Q, int BH, int N, int D, int Ms, uint64_t seed, HeadMap hm,
+                                 float* metric, int* sample_idx, int* err, cudaStream_t st) {
   size_t sm = sample_smem(Ms, D);
   if (D == 64) {
     cudaFuncSetAttribute(k_sample_metric<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_sample_metric<64><<<BH, 64 * 64 / 16, sm, st>>>((const __nv_bfloat16*)Q, N, Ms, seed, metric, sample_idx, err);
+    k_sample_metric<64><<<BH, 64 * 64 / 16, sm, st>>>((const __nv_bfloat16*)Q, N, Ms, seed, hm, metric, sample_idx,
+                                                      err);
   } else {
     cudaFuncSetAttribute(k_sample_metric<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    k_sample_metric<128><<<BH, 128 * 128 / 16, sm, st>>>((const __nv_bfloat16*)Q, N, Ms, seed, metric,
+    k_sample_metric<128><<<BH, 128 * 128 / 16, sm, st>>>((const __nv_bfloat16*)Q, N, Ms, seed, hm, metric,
                                                          sample_idx, err);
   }
   return cudaGetLastError();

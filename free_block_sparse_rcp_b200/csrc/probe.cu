@@ -19,7 +19,7 @@ namespace spr {
 // groups in ascending order.  grid = BH, block = 256.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_probe_pick(const int* __restrict__ perm_q, const int* __restrict__ qoff,
-                                                   int N, int Gq, int P, uint64_t seed,
+                                                   int N, int Gq, int P, uint64_t seed, HeadMap hm,
                                                    int* __restrict__ probe_idx, int* __restrict__ probe_grp,
                                                    int* err) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(256) k_probe_pick(const int* __restrict__ perm
         remaining -= add;
       }
     }
-    SplitMix64 g(stream_state(seed, bh, PURPOSE_PROBES));
+    SplitMix64 g(stream_state(seed, hm.global(bh), PURPOSE_PROBES));
     SlotMap map{mkey, mval, 256};
     int outp = 0;
     for (int a = 0; a < Gq; ++a) {
@@ -123,10 +123,12 @@ __global__ void __launch_bounds__(128) k_probe_combine(const float* __restrict__
 // Residual subspace + ridge fit, one CTA per head (fp64 arithmetic).
 //   R = O_dense - O_sparse (P x D); top eigenpairs u_i, sigma_i^2 of the Gram R R^T
 //   (Householder + multisection + inverse iteration); v_i = R^T u_i normalised (zero when
-//   sigma_i <= 1e-6 sigma_0); Y = R V_r; the affine map works inside the subspace: with
-//   X = O_sparse V_r (the probes' sparse outputs in the subspace), centred dual ridge
-//   W_sub = Xc^T (Xc Xc^T + lam I)^-1 Yc, b = ybar - xbar W_sub; exported as W = V_r W_sub
-//   (so a row's residual coordinates are x W = (x V_r) W_sub).
+//   sigma_i <= 1e-6 sigma_0); Y = R V_r (the probes' residual coordinates).  The map's
+//   input X is either the probes' whole sparse output (full_input: the pages' R ~ b + xB
+//   with only the correction restricted to the subspace) or that output projected on V_r.
+//   Centred dual ridge W = Xc^T (Xc Xc^T + lam I)^-1 Yc, b = ybar - xbar W; in the
+//   projected reading W_sub (r x r) is exported as W = V_r W_sub, so in both readings a
+//   row's residual coordinates are x W (x the row's full sparse output).
 // grid = BH, block = FIT_THREADS.
 // ---------------------------------------------------------------------------
 constexpr int FIT_THREADS = 1024;
@@ -153,7 +155,7 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
                                                   float* __restrict__ W_out, float* __restrict__ bfull_out,
                                                   float* __restrict__ Bmat, float* __restrict__ sigma_out,
                                                   float* __restrict__ bsub_out, const int* __restrict__ probe_grp,
-                                                  const int* __restrict__ qoff, int Gq) {
+                                                  const int* __restrict__ qoff, int Gq, int full_input) {
   extern __shared__ __align__(16) unsigned char smem[];
   constexpr int LDP = PR + 1;
   const int ldz = Rk + 1;
@@ -167,7 +169,7 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
   double* Y = Vr + D * Rk;                         // [PR][Rk] -> solution
   double* Xs = Y + PR * Rk;                        // [PR][Rk] probe sparse outputs in the subspace
   double* Wd = Xs + PR * Rk;                       // [D][Rk] W = V_r W_sub
-  double* xbar = X + xsz;                          // [D] (the first Rk: mean of Xs)
+  double* xbar = X + xsz;                          // [D] mean of X (projected reading: the first Rk)
   double* ybar = xbar + D;                         // [64]
   double* bsub = ybar + 64;                        // [64]
   double* cs = bsub + 64;                          // [64]
@@ -249,35 +251,41 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
     double s = 0.0, t = 0.0;
     for (int c = 0; c < D; ++c) {
       s += (double)Rm[p * D + c] * Vr[c * Rk + j];
-      t += (double)Xm[p * D + c] * Vr[c * Rk + j];
+      if (!full_input) t += (double)Xm[p * D + c] * Vr[c * Rk + j];
     }
     Y[p * Rk + j] = s;
     Xs[p * Rk + j] = t;
   }
   __syncthreads();
   // weighted means (the weights average to 1), centred rows scaled by sqrt(weight)
-  for (int j = tid; j < Rk; j += nt) {
+  const int XD = full_input ? D : Rk;   // width of the map's input
+  for (int j = tid; j < (XD > Rk ? XD : Rk); j += nt) {
     double s = 0.0, t = 0.0;
     for (int p = 0; p < P; ++p) {
-      s += wt[p] * Y[p * Rk + j];
-      t += wt[p] * Xs[p * Rk + j];
+      if (j < Rk) s += wt[p] * Y[p * Rk + j];
+      if (j < XD) t += wt[p] * (full_input ? (double)Xm[p * D + j] : Xs[p * Rk + j]);
     }
-    ybar[j] = s / P;
-    xbar[j] = t / P;
+    if (j < Rk) ybar[j] = s / P;
+    if (j < XD) xbar[j] = t / P;
   }
   __syncthreads();
   for (int e = tid; e < P * Rk; e += nt) {
     const int p = e / Rk, j = e - p * Rk;
     const double sq = sqrt(wt[p]);
     Y[p * Rk + j] = (Y[p * Rk + j] - ybar[j]) * sq;
-    Xs[p * Rk + j] = (Xs[p * Rk + j] - xbar[j]) * sq;
+    if (!full_input) Xs[p * Rk + j] = (Xs[p * Rk + j] - xbar[j]) * sq;
   }
   __syncthreads();
-  // A = Xc Xc^T + lam I  (into G), Xc = centred Xs
+  // A = Xc Xc^T + lam I  (into G), Xc = the centred input rows scaled by sqrt(weight)
   for (int e = tid; e < P * P; e += nt) {
     const int i = e / P, j = e - i * P;
     double s = 0.0;
-    for (int c = 0; c < Rk; ++c) s += Xs[i * Rk + c] * Xs[j * Rk + c];
+    if (full_input) {
+      for (int c = 0; c < D; ++c) s += ((double)Xm[i * D + c] - xbar[c]) * ((double)Xm[j * D + c] - xbar[c]);
+      s *= sqrt(wt[i]) * sqrt(wt[j]);
+    } else {
+      for (int c = 0; c < Rk; ++c) s += Xs[i * Rk + c] * Xs[j * Rk + c];
+    }
     G[i * LDP + j] = s + (i == j ? lam : 0.0);
   }
   __syncthreads();
@@ -308,29 +316,48 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
     }
   }
   __syncthreads();
-  // W_sub = Xc^T Z (Rk x Rk, in the Cholesky region), b = ybar - xbar W_sub
-  double* Ws = G;
-  for (int e = tid; e < Rk * Rk; e += nt) {
-    const int i = e / Rk, j = e - i * Rk;
-    double s = 0.0;
-    for (int p = 0; p < P; ++p) s += Xs[p * Rk + i] * Y[p * Rk + j];
-    Ws[e] = s;
-  }
-  __syncthreads();
-  for (int j = tid; j < Rk; j += nt) {
-    double s = 0.0;
-    for (int i = 0; i < Rk; ++i) s += xbar[i] * Ws[i * Rk + j];
-    bsub[j] = ybar[j] - s;
-    if (bsub_out) bsub_out[(size_t)bh * Rk + j] = (float)bsub[j];
-  }
-  // W = V_r W_sub (D x Rk): residual coordinates of a row are x W = (x V_r) W_sub
-  for (int e = tid; e < D * Rk; e += nt) {
-    const int c = e / Rk, j = e - c * Rk;
-    double s = 0.0;
-    for (int i = 0; i < Rk; ++i) s += Vr[c * Rk + i] * Ws[i * Rk + j];
-    Wd[e] = s;
-    W_out[(size_t)bh * D * Rk + e] = (float)s;
-    Vr_out[(size_t)bh * D * Rk + e] = (float)Vr[c * Rk + j];
+  if (full_input) {
+    // W = Xc^T Z (D x Rk), b = ybar - xbar W
+    for (int e = tid; e < D * Rk; e += nt) {
+      const int c = e / Rk, j = e - c * Rk;
+      double s = 0.0;
+      for (int p = 0; p < P; ++p) s += sqrt(wt[p]) * ((double)Xm[p * D + c] - xbar[c]) * Y[p * Rk + j];
+      Wd[e] = s;
+      W_out[(size_t)bh * D * Rk + e] = (float)s;
+      Vr_out[(size_t)bh * D * Rk + e] = (float)Vr[c * Rk + j];
+    }
+    __syncthreads();
+    for (int j = tid; j < Rk; j += nt) {
+      double s = 0.0;
+      for (int c = 0; c < D; ++c) s += xbar[c] * Wd[c * Rk + j];
+      bsub[j] = ybar[j] - s;
+      if (bsub_out) bsub_out[(size_t)bh * Rk + j] = (float)bsub[j];
+    }
+  } else {
+    // W_sub = Xc^T Z (Rk x Rk, in the Cholesky region), b = ybar - xbar W_sub
+    double* Ws = G;
+    for (int e = tid; e < Rk * Rk; e += nt) {
+      const int i = e / Rk, j = e - i * Rk;
+      double s = 0.0;
+      for (int p = 0; p < P; ++p) s += Xs[p * Rk + i] * Y[p * Rk + j];
+      Ws[e] = s;
+    }
+    __syncthreads();
+    for (int j = tid; j < Rk; j += nt) {
+      double s = 0.0;
+      for (int i = 0; i < Rk; ++i) s += xbar[i] * Ws[i * Rk + j];
+      bsub[j] = ybar[j] - s;
+      if (bsub_out) bsub_out[(size_t)bh * Rk + j] = (float)bsub[j];
+    }
+    // W = V_r W_sub (D x Rk): residual coordinates of a row are x W = (x V_r) W_sub
+    for (int e = tid; e < D * Rk; e += nt) {
+      const int c = e / Rk, j = e - c * Rk;
+      double s = 0.0;
+      for (int i = 0; i < Rk; ++i) s += Vr[c * Rk + i] * Ws[i * Rk + j];
+      Wd[e] = s;
+      W_out[(size_t)bh * D * Rk + e] = (float)s;
+      Vr_out[(size_t)bh * D * Rk + e] = (float)Vr[c * Rk + j];
+    }
   }
   __syncthreads();
   for (int c = tid; c < D; c += nt) {
@@ -639,10 +666,10 @@ cudaError_t launch_worklist(const unsigned char* route, const int* qoff, const i
 }
 
 cudaError_t launch_probe_pick(const int* perm_q, const int* qoff, int BH, int N, int Gq, int P, uint64_t seed,
-                              int* probe_idx, int* probe_grp, int* err, cudaStream_t st) {
+                              HeadMap hm, int* probe_idx, int* probe_grp, int* err, cudaStream_t st) {
   size_t sm = (size_t)(3 * Gq + 64 + 512 + 8) * 4;
   cudaFuncSetAttribute(k_probe_pick, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  k_probe_pick<<<BH, 256, sm, st>>>(perm_q, qoff, N, Gq, P, seed, probe_idx, probe_grp, err);
+  k_probe_pick<<<BH, 256, sm, st>>>(perm_q, qoff, N, Gq, P, seed, hm, probe_idx, probe_grp, err);
   return cudaGetLastError();
 }
 
@@ -664,9 +691,9 @@ cudaError_t launch_probe_attn(const void* Q, const void* K, const void* V, int B
 cudaError_t launch_probe_attn_splits(const void* Q, const void* K, const void* V, int BH, int N, int D, int Gk,
                                      int Gq, int P, const int* probe_idx, const int* probe_grp, const int* label_k,
                                      const unsigned char* route, float scale_log2, int S, float* part_o,
-                                     float* part_ml, cudaStream_t st) {
+                                     float* part_ml, int* err, cudaStream_t st) {
   return launch_probe_tc(Q, K, V, BH, N, D, Gk, Gq, P, probe_idx, probe_grp, label_k, route, scale_log2, S, Causal{},
-                         part_o, part_ml, nullptr, st);
+                         part_o, part_ml, err, st);
 }
 
 cudaError_t launch_probe_combine_splits(const float* part_o, const float* part_ml, int BH, int S, int P, int D,
@@ -688,16 +715,17 @@ size_t probe_fit_smem(int D, int Rk) { return D == 64 ? FitLayout<64>::bytes(Rk)
 
 cudaError_t launch_probe_fit(const float* o_dense, const float* o_sparse, int BH, int D, int P, int Rk,
                              double lam, float* Vr, float* W, float* bfull, float* Bmat, float* sigma,
-                             float* bsub, const int* probe_grp, const int* qoff, int Gq, cudaStream_t st) {
+                             float* bsub, const int* probe_grp, const int* qoff, int Gq, int full_input,
+                             cudaStream_t st) {
   const size_t sm = probe_fit_smem(D, Rk);
   if (D == 64) {
     cudaFuncSetAttribute(k_probe_fit<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     k_probe_fit<64><<<BH, FIT_THREADS, sm, st>>>(o_dense, o_sparse, P, Rk, lam, Vr, W, bfull, Bmat, sigma, bsub,
-                                                  probe_grp, qoff, Gq);
+                                                  probe_grp, qoff, Gq, full_input);
   } else {
     cudaFuncSetAttribute(k_probe_fit<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     k_probe_fit<128><<<BH, FIT_THREADS, sm, st>>>(o_dense, o_sparse, P, Rk, lam, Vr, W, bfull, Bmat, sigma, bsub,
-                                                  probe_grp, qoff, Gq);
+                                                  probe_grp, qoff, Gq, full_input);
   }
   return cudaGetLastError();
 }

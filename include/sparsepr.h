@@ -24,11 +24,15 @@
  *    "BH" below is B*H and every per-head array is laid out head-major ([B, H, ...]
  *    flattened).
  *  - Token indices are int32 positions in [0, N) of the original sequence.
- *  - Ownership: the caller owns every buffer.  The library allocates nothing and
- *    keeps no state between calls.  Scratch memory is the caller's `workspace`
- *    (device, 256-byte aligned, at least sparsepr_workspace_bytes(p) bytes);
- *    partition, attend and probe_fit use disjoint regions of it, so attend and
- *    probe_fit may run concurrently on two streams sharing one workspace.
+ *  - Ownership: the caller owns every buffer.  Every entry point except
+ *    sparsepr_probe_fit_noalloc allocates nothing and keeps no state between calls:
+ *    their scratch memory is the caller's `workspace` (device, 256-byte aligned, at
+ *    least sparsepr_workspace_bytes(p) bytes); partition, attend and probe_fit use
+ *    disjoint regions of it, so attend and probe_fit may run concurrently on two
+ *    streams sharing one workspace.  sparsepr_probe_fit_noalloc instead uses a fixed
+ *    16 MiB device array that the library holds on every GPU that loads it (see its
+ *    declaration).  sparsepr_forward_host_chunked creates and releases CUDA events
+ *    inside the call (no device memory).
  *  - Asynchrony: every call only enqueues work on `stream` (a cudaStream_t; NULL
  *    is the legacy default stream) and returns.  Argument errors are detected on
  *    the host before anything is enqueued and return SPARSEPR_EINVAL or
@@ -41,10 +45,13 @@
  *    reproducible (no floating-point atomics on any output path).
  *  - Random draws (query sample, k-means seeds, probe rows) use SplitMix64
  *    (Steele, Lea & Flood 2014) with one stream per (head, purpose):
- *    state0 = mix(seed + 0xD1B54A32D192ED03 * (8*bh + purpose + 1)),
+ *    state0 = mix(seed + 0xD1B54A32D192ED03 * (8*g + purpose + 1)),
  *    purpose 0 = query sample, 1 = key k-means seeds, 2 = query k-means seeds,
  *    3 = probe rows; a draw of m of n items is a partial Fisher-Yates shuffle
- *    (j = i + next() mod (n - i)).
+ *    (j = i + next() mod (n - i)).  g is the head's index in the whole layer:
+ *    g = b * heads_total + head_offset + h for head h of batch element b of the
+ *    call (g = b * H + h by default), so a call split by heads or batch elements
+ *    (over GPUs, or in chunks) reproduces the unsplit call bit for bit.
  */
 #ifndef SPARSEPR_H
 #define SPARSEPR_H
@@ -105,6 +112,15 @@ typedef struct {
   int fit_weighted;        /* 0: uniform probe weights in the ridge fit; 1: each probe weighted by
                               n_a / (probes of its group a), normalised to mean 1 (the weighted
                               affine fit one page mentions)                                       */
+  int fit_input;           /* input x of the affine map R ~ b + xB:
+                              0 (default): the row's whole d-dimensional sparse output, with only
+                              the correction projected onto the residual subspace (gist.science
+                              2.B; huashangw.com method section: the corrected result is limited
+                              to the residual directions the probes observed);
+                              1: the sparse output projected on that subspace as well (x V_r)    */
+  int head_offset;         /* index of this call's first head in the layer (>= 0; default 0)      */
+  int heads_total;         /* heads per batch element of the layer (0: H; else >= head_offset + H);
+                              with head_offset only the random streams depend on them              */
 } sparsepr_params;
 
 /* Optional debug copies of partition intermediates (any pointer may be NULL). */
@@ -191,15 +207,22 @@ SPARSEPR_API sparsepr_status sparsepr_probe_fit(const sparsepr_params* p, const 
  * allocation, or host code where an allocation, which can synchronize the device, is not
  * allowed).  Arguments and outputs are those of sparsepr_probe_fit minus the trace and the
  * workspace; results agree with it up to floating-point summation order.
+ * Frame-causal params (frame_id != NULL) are refused with SPARSEPR_EUNSUPPORTED, and Q, K,
+ * V must be 16-byte aligned (else SPARSEPR_EINVAL), both before any work is enqueued.
  * Scratch: a 16 MiB device array owned by the library, present on every GPU that loads
- * it until the process exits.  The key-split count shrinks to fit it; a problem whose
- * per-call buffers (about B*H*n_probes*(8*d + 16) bytes plus one split) exceed it returns
- * SPARSEPR_EUNSUPPORTED before any work is enqueued.  The first call on a device looks up
- * the array's device address (cudaGetSymbolAddress, with that device current); make that
+ * it until the process exits.  With S key splits it holds
+ *   B*H*(n_probes*(4*d + 12) + S*64*(8*d + 16)) bytes (each region rounded up to 256)
+ * plus a 256-byte error word; S starts at the workspace entry point's split count for N
+ * and shrinks until the problem fits, and a problem that does not fit even with S = 1
+ * returns SPARSEPR_EUNSUPPORTED before any work is enqueued.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress, with that device current)
+ * and keeps it for the life of the process (a cudaDeviceReset invalidates it); make that
  * first call before any stream capture.  All calls share the one array and it keeps the
- * previous call's contents (every byte is rewritten before it is read): calls that overlap
- * on the GPU, on other streams or from other host threads, race and must be serialized by
- * the caller.  Device-side index checks of this variant are not reported.               */
+ * previous call's contents: the call clears its error word and rewrites every other byte
+ * before reading it; calls that overlap on the GPU, on other streams or from other host
+ * threads, race and must be serialized by the caller.  A device-side failure (a bounded
+ * wait that ran out, an index out of range, a failed random draw) sets b_full, Vr, W and
+ * Bmat of every head to NaN instead of leaving stale values.                           */
 SPARSEPR_API sparsepr_status sparsepr_probe_fit_noalloc(const sparsepr_params* p, const void* Q,
                                                         const void* K, const void* V,
                                                         const int* label_k, const int* perm_q,
@@ -233,6 +256,30 @@ SPARSEPR_API sparsepr_status sparsepr_forward_host(const sparsepr_params* p, con
                                       const void* K_host, const void* V_host, void* O_host,
                                       void* qkv_dev, void* o_dev,
                                       void* workspace, size_t ws_bytes, void* stream);
+
+/* sparsepr_forward_host as a pipeline over head chunks, so that the host<->device copies
+ * of one chunk run beside the compute of another.  The B*H heads (flattened b*H + h) are
+ * split into n_chunks (1..min(B*H, 512)) consecutive ranges of ceil(B*H / n_chunks) heads
+ * (with head_offset / heads_total set, also at every batch element).  Chunk c's three
+ * host-to-device copies (one cudaMemcpyAsync per tensor) go on copy_in_stream, its call
+ * (sparsepr_forward with B = 1 over the chunk's heads, head_offset = their layer index, so
+ * every output equals the unsplit call's bit for bit) on `stream`, and the copy of its O
+ * back to O_host on copy_out_stream.  The copies in start after the work already enqueued
+ * on `stream`; `stream` completes after the last copy out, so synchronizing `stream` is
+ * enough.  A NULL copy stream means `stream` (no overlap).
+ *   qkv_dev   device bf16 [3][B, H, N, d] staging of Q, K, V; o_dev device bf16 [B, H, N, d]
+ *   workspace sparsepr_forward_workspace_bytes of the params of one chunk (B = 1,
+ *             H = ceil(B*H / n_chunks)), shared by the chunks (their compute is serialized
+ *             on `stream`); its error word is cleared once and collects every chunk's
+ *             device errors
+ * Host buffers should be pinned for the copies to be asynchronous.  The call creates its
+ * CUDA events and releases them before returning (they are freed once they complete).  */
+SPARSEPR_API sparsepr_status sparsepr_forward_host_chunked(const sparsepr_params* p, const void* Q_host,
+                                                           const void* K_host, const void* V_host,
+                                                           void* O_host, void* qkv_dev, void* o_dev,
+                                                           int n_chunks, void* workspace, size_t ws_bytes,
+                                                           void* stream, void* copy_in_stream,
+                                                           void* copy_out_stream);
 
 /* Dense softmax attention on the same machinery (the comparator for the sparse call):
  * O = softmax(s Q K^T) V (bf16 [B,H,N,d]), lse float [BH, N] (may be NULL); with frame ids,

@@ -28,7 +28,8 @@ def oracle_params(pd: dict) -> O.Params:
                     n_probes=pd["n_probes"], eig_rank=pd["eig_rank"], sub_rank=pd["sub_rank"],
                     kmeans_iters=pd["kmeans_iters"], density=float(np.float32(pd["density"])),
                     ridge_lambda=float(np.float32(pd["ridge_lambda"])), scale=float(np.float32(pd["scale"])),
-                    seed=pd["seed"], block=pd["block"], fit_weighted=bool(pd.get("fit_weighted", 0)))
+                    seed=pd["seed"], block=pd["block"], fit_weighted=bool(pd.get("fit_weighted", 0)),
+                    fit_input="subspace" if pd.get("fit_input", 0) == 1 else "full")
 
 
 def check_labels_near_ties(x, mu, got, want, what=""):

@@ -51,6 +51,7 @@ int main(void) {
   F(sparsepr_params, density) F(sparsepr_params, n_kgroups) F(sparsepr_params, kmeans_iters)
   F(sparsepr_params, ridge_lambda) F(sparsepr_params, scale) F(sparsepr_params, seed) F(sparsepr_params, frame_id)
   F(sparsepr_params, n_frames) F(sparsepr_params, partition_mode) F(sparsepr_params, fit_weighted)
+  F(sparsepr_params, fit_input) F(sparsepr_params, head_offset) F(sparsepr_params, heads_total)
   printf("ptrace %zu\n", sizeof(sparsepr_partition_trace));
   printf("prtrace %zu\n", sizeof(sparsepr_probe_trace));
   return 0;
@@ -64,7 +65,8 @@ int main(void) {
         out = dict(line.split() for line in subprocess.check_output([exe], text=True).splitlines())
     P = spr.Params
     assert int(out["size"]) == ctypes.sizeof(P)
-    for f in ("density", "n_kgroups", "kmeans_iters", "ridge_lambda", "scale", "seed", "frame_id", "n_frames", "partition_mode", "fit_weighted"):
+    for f in ("density", "n_kgroups", "kmeans_iters", "ridge_lambda", "scale", "seed", "frame_id", "n_frames",
+              "partition_mode", "fit_weighted", "fit_input", "head_offset", "heads_total"):
         assert int(out[f]) == getattr(P, f).offset, f
     assert int(out["ptrace"]) == ctypes.sizeof(spr.PartitionTrace)
     assert int(out["prtrace"]) == ctypes.sizeof(spr.ProbeTrace)
@@ -92,6 +94,9 @@ def _params(spr, **kw):
     (dict(d=128, eig_rank=32, sub_rank=33), 2),
     (dict(partition_mode=1), 0), (dict(partition_mode=2), 1), (dict(partition_mode=-1), 1),
     (dict(fit_weighted=1), 0), (dict(fit_weighted=2), 1),
+    (dict(fit_input=1), 0), (dict(fit_input=2), 1), (dict(fit_input=-1), 1),
+    (dict(head_offset=6, heads_total=8), 0), (dict(head_offset=6), 0), (dict(head_offset=-1), 1),
+    (dict(head_offset=7, heads_total=8), 1), (dict(heads_total=1), 1), (dict(heads_total=-2), 1),
 ])
 def test_validation(spr, kw, status):
     p = _params(spr, **kw)
@@ -140,6 +145,31 @@ def test_calls_reject_before_cuda(spr):
     st = lib.sparsepr_dense_attention(ctypes.byref(p), fake, fake, odd, fake, None, None, 0, None)
     assert st == 1 and b"V" in lib.sparsepr_last_error()
     assert lib.sparsepr_status_string(0) == b"ok"
+
+
+def test_chunked_host_call_rejects_before_cuda(spr):
+    lib = spr._lib
+    p = _params(spr)
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the checks fail first
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    args = [fake] * 4
+    # chunk count out of range, misaligned device staging, workspace too small
+    assert lib.sparsepr_forward_host_chunked(ctypes.byref(p), *args, fake, fake, 0, fake, 1 << 40, None, None,
+                                             None) == 1
+    assert lib.sparsepr_forward_host_chunked(ctypes.byref(p), *args, fake, fake, 3, fake, 1 << 40, None, None,
+                                             None) == 1
+    assert lib.sparsepr_forward_host_chunked(ctypes.byref(p), *args, odd, fake, 2, fake, 1 << 40, None, None,
+                                             None) == 1
+    assert lib.sparsepr_forward_host_chunked(ctypes.byref(p), *args, fake, fake, 2, fake, 1024, None, None,
+                                             None) == 3
+    nul = list(args)
+    nul[2] = None
+    assert lib.sparsepr_forward_host_chunked(ctypes.byref(p), *nul, fake, fake, 2, fake, 1 << 40, None, None,
+                                             None) == 1
+    # the workspace of one chunk is enough
+    one = spr.chunk_params(p, 2)
+    assert one.B == 1 and one.H == 1
+    assert spr.sparsepr_forward_workspace_bytes(one) < spr.sparsepr_forward_workspace_bytes(p)
 
 
 def test_workspace_grows_with_problem(spr):

@@ -201,11 +201,16 @@ def _rest_checks(pd, op, q, k, v, s, tr, ptr, out, bh, b, h, y_gpu, N, T, rng, r
             assert np.abs(vk.T @ vk - np.eye(vk.shape[1])).max() <= 1e-4
             inv = r_gpu.T @ (r_gpu @ vk) - vk * sig_gpu[keep] ** 2
             assert np.abs(inv).max() <= 1e-5 * s0 ** 2
-        # --- a15: the ridge given the device's subspace (exact up to fp32 rounding)
+        # --- a15: the ridge given the device's subspace (exact up to fp32 rounding); its input
+        # is the whole sparse output row (fit_input 0) or its projection on V_r (fit_input 1)
         wts = O.probe_weights(qo, pd["n_probes"]) if op.fit_weighted else None
-        w_sub, b_sub = O.ridge_fit(os_gpu @ vr_gpu, r_gpu @ vr_gpu, op.ridge_lambda, wts)
+        if op.fit_input == "full":
+            w_fit, b_sub = O.ridge_fit(os_gpu, r_gpu @ vr_gpu, op.ridge_lambda, wts)
+        else:
+            w_sub, b_sub = O.ridge_fit(os_gpu @ vr_gpu, r_gpu @ vr_gpu, op.ridge_lambda, wts)
+            w_fit = vr_gpu @ w_sub
         bfull_ref = vr_gpu @ b_sub
-        bmat_ref = vr_gpu @ w_sub @ vr_gpu.T
+        bmat_ref = w_fit @ vr_gpu.T
         np.testing.assert_allclose(bm_gpu, w_gpu @ vr_gpu.T, atol=1e-5 * max(1, np.abs(bm_gpu).max()))
         corr_gpu = b_gpu + o_ref @ bm_gpu
         corr_ref = bfull_ref + o_ref @ bmat_ref
