@@ -87,7 +87,7 @@ Layout make_layout(const sparsepr_params& p) {
   L.eigval = take(BH * re * 4);
   L.eigvec = take(BH * d * re * 4);
   L.proj = take(BH * d * re * 4);
-  L.eig_lu = take(BH * 3 * d * re * 8);
+  L.eig_lu = take(BH * 3 * d * re * 4);
   const size_t GPmax = (size_t)kmeans_gp(p.n_kgroups > p.n_qgroups ? p.n_kgroups : p.n_qgroups);
   L.m_k = take(BH * Gk * d * 4);
   L.nu_k = take(BH * Gk * L.DTk * 4);
@@ -273,7 +273,7 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
     SPR_LAUNCH(launch_sample_metric(Q, BH, N, d, p.n_samples, p.seed, head_map(p), metric, at<int>(ws, L.sample_idx),
                                     err, st));
     SPR_LAUNCH(launch_metric_eigen(metric, BH, d, re, at<float>(ws, L.eigval), at<float>(ws, L.eigvec), proj,
-                                   at<double>(ws, L.eig_lu), st));
+                                   at<float>(ws, L.eig_lu), st));
     if (tr && tr->key_coords) SPR_LAUNCH(launch_key_coords(K, BH, N, d, re, proj, tr->key_coords, st));
   } else {
     SPR_LAUNCH(launch_identity(at<float>(ws, L.ident), d, st));

@@ -25,7 +25,7 @@ cudaError_t launch_sample_metric(const void* Q, int BH, int N, int D, int Ms, ui
                                  float* metric, int* sample_idx, int* err, cudaStream_t st);
 size_t metric_eigen_smem(int D, int R);
 cudaError_t launch_metric_eigen(const float* metric, int BH, int D, int R, float* eigval, float* eigvec,
-                                float* proj, double* lu, cudaStream_t st);
+                                float* proj, float* lu, cudaStream_t st);
 cudaError_t launch_key_coords(const void* K, int BH, int N, int D, int R, const float* proj, float* Y,
                               cudaStream_t st);
 int kmeans_dt(int Dc);

@@ -78,36 +78,36 @@ __global__ void __launch_bounds__(D * D / 16) k_sample_metric(const __nv_bfloat1
 }
 
 // ---------------------------------------------------------------------------
-// Leading eigenpairs of M_K (fp64, Householder + multisection + inverse iteration).
+// Leading eigenpairs of M_K (fp32 Householder + multisection + inverse iteration).
 // grid = BH, block = 1024.  Writes eigval [BH, R] (clamped >= 0), eigvec [BH, D, R] and
-// the projector P = U_R Lambda_R^{1/2} [BH, D, R].  lu: BH * 3 * D * R doubles of scratch.
+// the projector P = U_R Lambda_R^{1/2} [BH, D, R].  lu: BH * 3 * D * R floats of scratch.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(1024) k_metric_eigen(const float* __restrict__ metric, int R,
                                                      float* __restrict__ eigval, float* __restrict__ eigvec,
-                                                     float* __restrict__ proj, double* __restrict__ lu) {
+                                                     float* __restrict__ proj, float* __restrict__ lu) {
   extern __shared__ __align__(16) unsigned char smem[];
   constexpr int LD = D + 1;
   const int ldz = R + 1;
-  double* A = reinterpret_cast<double*>(smem);  // [D][D+1]
-  double* Z = A + D * LD;                       // [D][R+1]
-  double* lam = Z + D * ldz;                    // [64]
-  double* sc = lam + 64;                        // SymEigScratch<D>
+  float* A = reinterpret_cast<float*>(smem);   // [D][D+1]
+  float* Z = A + D * LD;                       // [D][R+1]
+  float* lam = Z + D * ldz;                    // [64]
+  float* sc = lam + 64;                        // SymEigScratch<float, D>
   const int bh = blockIdx.x;
 #pragma unroll 8
   for (int i = threadIdx.x; i < D * D; i += blockDim.x) {
     const int r = i / D, c = i - r * D;
-    A[r * LD + c] = (double)metric[(size_t)bh * D * D + i];
+    A[r * LD + c] = metric[(size_t)bh * D * D + i];
   }
   __syncthreads();
-  sym_top_eigen<D>(A, R, Z, ldz, lam, sc, lu + (size_t)bh * 3 * D * R);
+  sym_top_eigen<float, D>(A, R, Z, ldz, lam, sc, lu + (size_t)bh * 3 * D * R);
   for (int e = threadIdx.x; e < D * R; e += blockDim.x) {
     const int c = e / R, k = e - c * R;
-    const double l = fmax(lam[k], 0.0);
-    const double u = Z[c * ldz + k];
-    if (c == 0) eigval[(size_t)bh * R + k] = (float)l;
-    eigvec[(size_t)bh * D * R + e] = (float)u;
-    proj[(size_t)bh * D * R + e] = (float)(u * sqrt(l));
+    const float l = fmaxf(lam[k], 0.f);
+    const float u = Z[c * ldz + k];
+    if (c == 0) eigval[(size_t)bh * R + k] = l;
+    eigvec[(size_t)bh * D * R + e] = u;
+    proj[(size_t)bh * D * R + e] = u * sqrtf(l);
   }
 }
 
@@ -544,12 +544,12 @@ cudaError_t launch_sample_metric(const void* Q, int BH, int N, int D, int Ms, ui
 }
 
 size_t metric_eigen_smem(int D, int R) {
-  const size_t sc = D == 64 ? SymEigScratch<64>::kDoubles : SymEigScratch<128>::kDoubles;
-  return ((size_t)D * (D + 1) + (size_t)D * (R + 1) + 64 + sc) * 8;
+  const size_t sc = D == 64 ? SymEigScratch<float, 64>::kCount : SymEigScratch<float, 128>::kCount;
+  return ((size_t)D * (D + 1) + (size_t)D * (R + 1) + 64 + sc) * 4;
 }
 
 cudaError_t launch_metric_eigen(const float* metric, int BH, int D, int R, float* eigval, float* eigvec,
-                                float* proj, double* lu, cudaStream_t st) {
+                                float* proj, float* lu, cudaStream_t st) {
   const size_t sm = metric_eigen_smem(D, R);
   if (D == 64) {
     cudaFuncSetAttribute(k_metric_eigen<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);

@@ -143,7 +143,7 @@ struct FitLayout {
     return a > b ? a : b;
   }
   static size_t doubles(int Rk) {
-    return (size_t)PR * (PR + 1) + (size_t)PR * (Rk + 1) + 64 + SymEigScratch<PR>::kDoubles + xsize(Rk) + D + 3 * 64;
+    return (size_t)PR * (PR + 1) + (size_t)PR * (Rk + 1) + 64 + SymEigScratch<double, PR>::kCount + xsize(Rk) + D + 3 * 64;
   }
   static size_t bytes(int Rk) { return doubles(Rk) * 8 + (size_t)2 * PR * D * 4; }
 };
@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
   double* Z = G + PR * LDP;                        // [PR][Rk+1] eigenvectors of R R^T
   double* ev = Z + PR * ldz;                       // [64] eigenvalues, descending
   double* esc = ev + 64;                           // eigen scratch
-  double* X = esc + SymEigScratch<PR>::kDoubles;   // solver scratch, then V_r and Y
+  double* X = esc + SymEigScratch<double, PR>::kCount;   // solver scratch, then V_r and Y
   double* Vr = X;                                  // [D][Rk]
   double* Y = Vr + D * Rk;                         // [PR][Rk] -> solution
   double* Xs = Y + PR * Rk;                        // [PR][Rk] probe sparse outputs in the subspace
@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(FIT_THREADS) k_probe_fit(const float* __restri
     G[j * LDP + i] = s;
   }
   __syncthreads();
-  sym_top_eigen<PR>(G, Rk, Z, ldz, ev, esc, X);
+  sym_top_eigen<double, PR>(G, Rk, Z, ldz, ev, esc, X);
   // subspace basis: v_j = R^T u_j / ||R^T u_j|| for the j-th largest eigenvalue of R R^T
   // (in fp64 these are orthogonal to ~1e-10 whenever sigma_j > 1e-6 sigma_max; smaller
   // singular values give zero columns)
