@@ -51,7 +51,7 @@ struct Layout {
   size_t err;
   // partition
   size_t ident, sample_idx, metric, eigval, eigvec, proj, eig_lu, m_k, nu_k, key_init, C, m_q, nu_q, query_init, bias, wnorm,
-      w_hi, w_lo, flag_count, flag_rows, corr_count, corr, psum, pcnt, mass, order, alpha;
+      w_hi, w_lo, flag_count, flag_rows, corr_count, corr, slots, xnorm, mass, order, alpha;
   // attend
   size_t rlist, rcum, rcnt, tiles, tile_count;
   // frame-causal tables (zero-sized without frame ids): partition / attend / probe regions
@@ -100,15 +100,12 @@ Layout make_layout(const sparsepr_params& p) {
   L.wnorm = take(BH * GPmax * 4);
   L.w_hi = take(BH * GPmax * d * 2);
   L.w_lo = take(BH * GPmax * d * 2 * 2);   // also holds the third part of C for the cell mass
-  L.flag_count = take(BH * 4);
+  L.flag_count = take(BH * (size_t)kmeans_plan(1, p.N).SPH * 4);   // uncertified rows per k-means segment
   L.flag_rows = take(BH * N * 4);
   L.corr_count = take(BH * 4);
   L.corr = take(BH * N * 16);
-  {
-    const KmPlan kp = kmeans_plan((int)BH, p.N);
-    L.psum = take((size_t)kp.grid * kp.maxh * GPmax * d * 4);
-    L.pcnt = take((size_t)kp.grid * kp.maxh * GPmax * 4);
-  }
+  L.slots = take(kmeans_slots_bytes((int)BH, p.N, (int)GPmax, (int)d));
+  L.xnorm = take(BH * N * 4);   // ||x||^2 of the rows of the running k-means
   L.mass = take(BH * Gq * Gk * 4);
   L.order = take(BH * Gq * Gk * 4);
   L.alpha = take(BH * 8);
@@ -201,9 +198,9 @@ sparsepr_status check_params(const sparsepr_params* p) {
   if (p->n_kgroups > 128) return fail(SPARSEPR_EUNSUPPORTED, "n_kgroups > 128 (query coordinates wider than 128) not built");
   if (p->n_qgroups > 128) return fail(SPARSEPR_EUNSUPPORTED, "n_qgroups > 128 not built");
   const int Dk = p->partition_mode == 1 ? p->d : p->eig_rank, Dq = p->partition_mode == 1 ? p->d : p->n_kgroups;
-  if (recheck_smem(p->d, Dq, kmeans_dt(Dq), p->n_qgroups) > kSmemLimit ||
-      recheck_smem(p->d, Dk, kmeans_dt(Dk), p->n_kgroups) > kSmemLimit ||
-      centroid_weights_smem(p->d, Dq > Dk ? Dq : Dk) > kSmemLimit ||
+  if (recheck_smem(p->d, Dq, kmeans_dt(Dq), p->n_qgroups, p->N) > kSmemLimit ||
+      recheck_smem(p->d, Dk, kmeans_dt(Dk), p->n_kgroups, p->N) > kSmemLimit ||
+      centroid_weights_smem(p->d, Dq > Dk ? Dq : Dk, p->N) > kSmemLimit ||
       assign_acc_smem(p->d, kmeans_gp(p->n_kgroups > p->n_qgroups ? p->n_kgroups : p->n_qgroups)) > kSmemLimit)
     return fail(SPARSEPR_EUNSUPPORTED, "too many groups for the k-means kernels");
   if (route_select_smem(p->n_qgroups, p->n_kgroups) > kSmemLimit)
@@ -286,8 +283,7 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
   int* frows = at<int>(ws, L.flag_rows);
   int* ccount = at<int>(ws, L.corr_count);
   void* corr = at<char>(ws, L.corr);
-  float* psum = at<float>(ws, L.psum);
-  int* pcnt = at<int>(ws, L.pcnt);
+  void* slots = at<char>(ws, L.slots);
   // One Lloyd k-means of the rows X (bf16, d) on coordinates A x; A(j, c) = a_scale * A[j*sj + c*sc].
   // Each pass assigns every row and leaves the per-group sums of its rows for the next
   // centroid update; means_out (if set) receives the means of the final groups.
@@ -297,18 +293,17 @@ sparsepr_status run_partition(const sparsepr_params& p, const Layout& L, const v
     SPR_LAUNCH(launch_seed_rows(X, BH, N, d, G, p.seed, head_map(p), purpose, m, init, err, st));
     for (int t = 0; t < p.kmeans_iters; ++t) {
       int* trc = trace_iters ? trace_iters + (size_t)t * BH * N : nullptr;
-      SPR_LAUNCH(launch_centroid_weights(m, BH, G, d, A, a_head, sj, sc, a_scale, D, DT, t == 0 ? 0 : 1, psum, pcnt,
+      SPR_LAUNCH(launch_centroid_weights(m, BH, G, d, A, a_head, sj, sc, a_scale, D, DT, t == 0 ? 0 : 1, slots,
                                          ccount, corr, X, N, nu, bias, wnorm, w_hi, w_lo, err, st));
-      SPR_CUDA(cudaMemsetAsync(fcount, 0, (size_t)BH * 4, st));
       SPR_CUDA(cudaMemsetAsync(ccount, 0, (size_t)BH * 4, st));
-      SPR_LAUNCH(launch_assign_acc(X, BH, N, d, G, w_hi, w_lo, bias, wnorm, labels, trc, fcount, frows, psum, pcnt,
-                                   err, st));
+      SPR_LAUNCH(launch_assign_acc(X, BH, N, d, G, w_hi, w_lo, bias, wnorm, labels, trc, fcount, frows, slots,
+                                   at<float>(ws, L.xnorm), t == 0 ? 1 : 0, err, st));
       SPR_LAUNCH(launch_assign_recheck(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, fcount, frows, labels,
                                        trc, ccount, corr, st));
     }
     SPR_LAUNCH(launch_group_sort(labels, BH, N, G, perm, off, err, st));
     if (means_out)
-      SPR_LAUNCH(launch_centroid_weights(means_out, BH, G, d, A, a_head, sj, sc, a_scale, D, DT, 2, psum, pcnt, ccount,
+      SPR_LAUNCH(launch_centroid_weights(means_out, BH, G, d, A, a_head, sj, sc, a_scale, D, DT, 2, slots, ccount,
                                          corr, X, N, nullptr, nullptr, nullptr, nullptr, nullptr, err, st));
     return SPARSEPR_OK;
   };

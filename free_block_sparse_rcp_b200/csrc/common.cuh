@@ -18,7 +18,8 @@ enum DeviceError : int {
   DERR_WAIT_TIMEOUT = 2, // a bounded wait on an mbarrier ran out
   DERR_DRAW = 3,         // random draw map overflow
   DERR_NONFINITE = 4,    // non-finite value where the algorithm forbids one
-  DERR_FRAMES = 5        // frame ids out of [0, n_frames) or decreasing in token order
+  DERR_FRAMES = 5,       // frame ids out of [0, n_frames) or decreasing in token order
+  DERR_CAPACITY = 6      // more k-means label corrections for 16 groups in one pass than the 2048 kept
 };
 
 __device__ __forceinline__ void set_error(int* err, int code) {

@@ -62,27 +62,32 @@ struct alignas(64) TmapBlob {
 
 // kmeans_tc.cu
 int kmeans_gp(int G);
-size_t centroid_weights_smem(int d, int D);
-size_t recheck_smem(int d, int D, int DT, int G);
+size_t centroid_weights_smem(int d, int D, int N);
+size_t recheck_smem(int d, int D, int DT, int G, int N);
 cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_t seed, HeadMap hm, int purpose,
                              float* m, int* init_out, int* err, cudaStream_t st);
-// Persistent k-means assignment: CTA b takes the global 128-row tiles [b per, (b+1) per)
-// and leaves one partial-sum slot per head it touches (maxh slots per CTA).
+// Persistent k-means assignment over segments of kKmeansSeg 128-row tiles of one head (head-
+// major); CTA c takes a contiguous, balanced run of segments and leaves one partial-sum slot
+// per segment, so the sums do not depend on the grid or on the number of heads.
 constexpr int kKmeansCtas = 148;
+constexpr int kKmeansSeg = 8;
 struct KmPlan {
-  int grid, per, T, maxh, total;
+  int grid, T, SPH, nseg;
 };
 KmPlan kmeans_plan(int BH, int N);
+// bytes of the segment slots of one k-means pass with GP (padded) groups and row width d
+size_t kmeans_slots_bytes(int BH, int N, int GP, int d);
 size_t assign_acc_smem(int D, int GP);
 cudaError_t launch_centroid_weights(float* m, int BH, int G, int d, const float* A, size_t a_head, int sj, int sc,
-                                    float a_scale, int D, int DT, int mode, const float* psum, const int* pcnt,
+                                    float a_scale, int D, int DT, int mode, const void* slots,
                                     const int* corr_count, const void* corr, const void* X, int N, float* nu,
                                     float* bias, float* wnorm, void* w_hi, void* w_lo, int* err, cudaStream_t st);
 cudaError_t launch_assign_acc(const void* X, int BH, int N, int d, int G, const void* w_hi, const void* w_lo,
-                              const float* bias, const float* wnorm, int* labels, int* trace, int* flag_count,
-                              int* flag_rows, float* psum, int* pcnt, int* err, cudaStream_t st);
+                              const float* bias, const float* wnorm, int* labels, int* trace, int* flag_seg,
+                              int* flag_rows, void* slots, float* xnorm, int xnorm_store, int* err,
+                              cudaStream_t st);
 cudaError_t launch_assign_recheck(const void* X, int BH, int N, int d, const float* A, size_t a_head, int sj, int sc,
-                                  float a_scale, int D, const float* nu, int G, const int* flag_count,
+                                  float a_scale, int D, const float* nu, int G, const int* flag_seg,
                                   const int* flag_rows, int* labels, int* trace, int* corr_count, void* corr,
                                   cudaStream_t st);
 size_t cell_mass_tc_smem(int D, int GP, int F);

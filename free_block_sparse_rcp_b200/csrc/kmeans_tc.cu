@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(256) k_seed_rows(const __nv_bfloat16* __restri
 // CTA in shared memory as sA[j][c] with row stride d + 1 (conflict-free both ways).
 // mode 0: m holds the centroids (the seeds).
 // mode 1: m_g = (sum of the rows assigned to g) / (their count): the partial sums the
-//         previous assignment pass left per (CTA, head) slot, added in ascending CTA order
+//         previous assignment pass left per segment of the head, added in segment order
 //         in fp64, then the label corrections of the exact re-check applied in ascending
 //         row order (a row moves from its provisional group to its final one); an empty
 //         group keeps its centroid.  m is updated in place.
@@ -75,14 +75,21 @@ __global__ void __launch_bounds__(256) k_seed_rows(const __nv_bfloat16* __restri
 // ---------------------------------------------------------------------------
 constexpr int WG_PER_CTA = 16;
 constexpr int CW_THREADS = 256;
+constexpr int kCorrCap = 2048;   // corrections of one CTA's groups per pass
+
+// floats of the region that holds A for the weights and, before that, the segment-slot rows
+// of the CTA's groups and its sorted corrections
+__host__ __device__ inline int cw_scratch_floats(int d, int D, int SPH) {
+  const int a = D * (d + 1), b = SPH * WG_PER_CTA + 2 * kCorrCap;
+  return ((a > b ? a : b) + 3) & ~3;
+}
 
 struct KmPartials {
-  const float* psum;          // [grid][maxh][GP][d]
-  const int* pcnt;            // [grid][maxh][GP]
+  const unsigned char* slots; // [BH][SPH] segment slots of the assignment pass (kmeans_slot_bytes each)
   const int* corr_count;      // [BH]
   const int4* corr;           // [BH][N] (row, provisional label, final label, -)
   const __nv_bfloat16* X;     // rows
-  int N, T, per, maxh, grid;
+  int N, SPH;
 };
 
 __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restrict__ m, int G, int GP, int d,
@@ -95,72 +102,118 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
   extern __shared__ __align__(16) float sw[];
   double* acc = reinterpret_cast<double*>(sw);               // [WG_PER_CTA][d]
   int* cnt = reinterpret_cast<int*>(acc + WG_PER_CTA * d);   // [WG_PER_CTA]
-  float* sA = reinterpret_cast<float*>(cnt + WG_PER_CTA);    // [D][d + 1]
-  float* sMg = sA + D * (d + 1);                             // [WG_PER_CTA][d] this CTA's centroids
+  float* sA = reinterpret_cast<float*>(cnt + WG_PER_CTA);    // [D][d + 1]  (the means phase uses it as scratch)
+  float* sMg = sA + cw_scratch_floats(d, D, pp.SPH);         // [WG_PER_CTA][d] this CTA's centroids
   float* sNu = sMg + WG_PER_CTA * d;                         // [WG_PER_CTA][128] their nu
   const int bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g0 = blockIdx.x * WG_PER_CTA, g1 = min(GP, g0 + WG_PER_CTA);
   if (mode != 0) {
-    // ---- means from the partial sums of the previous pass
-    const int h0 = bh * pp.T, h1 = h0 + pp.T;
-    const int b_lo = h0 / pp.per, b_hi = min(pp.grid - 1, (h1 - 1) / pp.per);
-    // per element, the slots in ascending CTA order (0 + s_lo + ... + s_hi, as the definition
-    // of the mean reads); the loads of all slots of an element are independent and go out
-    // together
-    for (int e = tid; e < WG_PER_CTA * d; e += CW_THREADS) {
-      const int gi = e / d, c = e - gi * d;
-      double a = 0.0;
-      if (gi < g1 - g0) {
-#pragma unroll 4
-        for (int b = b_lo; b <= b_hi; ++b) {
-          const int slot = b * pp.maxh + (bh - (b * pp.per) / pp.T);
-          a += (double)pp.psum[((size_t)slot * GP + g0 + gi) * d + c];
+    // ---- means from the partial sums of the previous pass: per element, the head's
+    // segment slots in segment order (the mean's definition, summed in fp64); the slot of a
+    // segment holds only the groups that occur in it
+    const size_t sbytes = (size_t)GP * 8 + (size_t)GP * d * 4;
+    const unsigned char* hs = pp.slots + (size_t)bh * pp.SPH * sbytes;
+    int* spos = reinterpret_cast<int*>(sA);                   // [SPH][WG_PER_CTA] slot rows
+    int2* sel = reinterpret_cast<int2*>(spos + pp.SPH * WG_PER_CTA);   // [kCorrCap] corrections
+    __shared__ int s_nsel, s_over;
+    for (int e = tid; e < pp.SPH * WG_PER_CTA; e += CW_THREADS) {
+      const int sgm = e / WG_PER_CTA, gi = e - sgm * WG_PER_CTA;
+      spos[e] = gi < g1 - g0 ? reinterpret_cast<const int*>(hs + (size_t)sgm * sbytes)[g0 + gi] : -1;
+    }
+    if (tid == 0) { s_nsel = 0; s_over = 0; }
+    __syncthreads();
+    // element e = (group gi, column c), E elements per thread (d is 64 or 128: shifts); the
+    // loads of SB segments go out together before they are added in segment order
+    constexpr int E = WG_PER_CTA * 128 / CW_THREADS, SB = 4;
+    const int dl = d == 64 ? 6 : 7;
+    int gis[E], cs[E];
+    double a[E];
+#pragma unroll
+    for (int u = 0; u < E; ++u) {
+      const int e = tid + u * CW_THREADS;
+      gis[u] = e < WG_PER_CTA * d ? e >> dl : -1;
+      cs[u] = e & (d - 1);
+      a[u] = 0.0;
+    }
+    for (int sgm0 = 0; sgm0 < pp.SPH; sgm0 += SB) {
+      float v[SB][E];
+      unsigned occ = 0u;
+#pragma unroll
+      for (int q = 0; q < SB; ++q) {
+        const int sgm = sgm0 + q;
+        const float* rows = reinterpret_cast<const float*>(hs + (size_t)sgm * sbytes + (size_t)GP * 8);
+#pragma unroll
+        for (int u = 0; u < E; ++u) {
+          const int pos = (sgm < pp.SPH && gis[u] >= 0) ? spos[sgm * WG_PER_CTA + gis[u]] : -1;
+          v[q][u] = 0.f;
+          if (pos >= 0) {
+            v[q][u] = rows[(size_t)pos * d + cs[u]];
+            occ |= 1u << (q * E + u);
+          }
         }
       }
-      acc[e] = a;
+#pragma unroll
+      for (int q = 0; q < SB; ++q)
+#pragma unroll
+        for (int u = 0; u < E; ++u)
+          if (occ & (1u << (q * E + u))) a[u] += (double)v[q][u];
     }
+#pragma unroll
+    for (int u = 0; u < E; ++u)
+      if (gis[u] >= 0) acc[tid + u * CW_THREADS] = a[u];
     if (tid < WG_PER_CTA) {
       int n = 0;
       if (tid < g1 - g0)
-        for (int b = b_lo; b <= b_hi; ++b) n += pp.pcnt[(size_t)(b * pp.maxh + (bh - (b * pp.per) / pp.T)) * GP + g0 + tid];
+        for (int sgm = 0; sgm < pp.SPH; ++sgm)
+          n += reinterpret_cast<const int*>(hs + (size_t)sgm * sbytes)[GP + g0 + tid];
       cnt[tid] = n;
     }
+    // the re-check's corrections that move a row out of or into this CTA's groups
+    const int nc = min(pp.corr_count[bh], pp.N);
+    const int4* cl = pp.corr + (size_t)bh * pp.N;
+    for (int i = tid; i < nc; i += CW_THREADS) {
+      const int4 cr = cl[i];
+      const bool from = cr.y >= g0 && cr.y < g1, to = cr.z >= g0 && cr.z < g1;
+      if (from || to) {
+        if (cr.x < 0 || cr.x >= pp.N) { set_error(err, DERR_INDEX); continue; }
+        const int k = atomicAdd(&s_nsel, 1);
+        if (k < kCorrCap) sel[k] = make_int2(cr.x, ((from ? cr.y - g0 : 0xFF) << 8) | (to ? cr.z - g0 : 0xFF));
+        else s_over = 1;
+      }
+    }
     __syncthreads();
-    if (warp == 0) {
-      // corrections in ascending row order (the list itself is in arbitrary order)
-      const int nc = min(pp.corr_count[bh], pp.N);
-      const int4* cl = pp.corr + (size_t)bh * pp.N;
-      int last = -1;
-      while (true) {
-        int best = 0x7fffffff, bi = -1;
-        for (int i = lane; i < nc; i += 32) {
-          const int r = cl[i].x;
-          if (r > last && r < best) { best = r; bi = i; }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const int ob = __shfl_xor_sync(0xffffffffu, best, o);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-          if (ob < best) { best = ob; bi = oi; }
-        }
-        if (bi < 0) break;
-        last = best;
-        const int4 cr = cl[bi];
-        if (cr.x < 0 || cr.x >= pp.N) { if (lane == 0) set_error(err, DERR_INDEX); break; }
-        const bool from = cr.y >= g0 && cr.y < g1, to = cr.z >= g0 && cr.z < g1;
-        if (from || to) {
-          const __nv_bfloat16* xr = pp.X + ((size_t)bh * pp.N + cr.x) * d;
-          for (int c = lane; c < d; c += 32) {
-            const double x = (double)bf2f(xr[c]);
-            if (from) acc[(cr.y - g0) * d + c] -= x;
-            if (to) acc[(cr.z - g0) * d + c] += x;
-          }
-          if (lane == 0) {
-            if (from) cnt[cr.y - g0] -= 1;
-            if (to) cnt[cr.z - g0] += 1;
+    const int ns = min(s_nsel, kCorrCap);
+    if (s_over) { if (tid == 0) set_error(err, DERR_CAPACITY); }
+    // ascending row order (bitonic sort of the selected list, padded with rows past N)
+    int p2 = 1;
+    while (p2 < ns) p2 <<= 1;
+    for (int i = ns + tid; i < p2; i += CW_THREADS) sel[i] = make_int2(0x7fffffff, 0xFFFF);
+    __syncthreads();
+    for (int kk = 2; kk <= p2; kk <<= 1) {
+      for (int j = kk >> 1; j > 0; j >>= 1) {
+        for (int i = tid; i < p2; i += CW_THREADS) {
+          const int l = i ^ j;
+          if (l > i) {
+            const int2 a = sel[i], b = sel[l];
+            const bool up = (i & kk) == 0;
+            if ((a.x > b.x) == up) { sel[i] = b; sel[l] = a; }
           }
         }
-        __syncwarp();
+        __syncthreads();
+      }
+    }
+    // apply them in that order: thread c owns column c of the CTA's groups
+    for (int c = tid; c < d; c += CW_THREADS) {
+      for (int k = 0; k < ns; ++k) {
+        const int2 e = sel[k];
+        const int fi = (e.y >> 8) & 0xFF, ti = e.y & 0xFF;
+        const double x = (double)bf2f(pp.X[((size_t)bh * pp.N + e.x) * d + c]);
+        if (fi != 0xFF) acc[fi * d + c] -= x;
+        if (ti != 0xFF) acc[ti * d + c] += x;
+        if (c == 0) {
+          if (fi != 0xFF) cnt[fi] -= 1;
+          if (ti != 0xFF) cnt[ti] += 1;
+        }
       }
     }
     __syncthreads();
@@ -292,72 +345,81 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
 }
 
 // ---------------------------------------------------------------------------
-// Tensor-core assignment fused with the centroid sums of the next update.
-// Persistent: CTA b takes the global 128-row tiles [b per, (b+1) per) (tile i = row tile
-// i mod T of head i / T) and runs them through a pipeline:
-//   warp 19     (lane 0) loads the X tile (contiguous rows, two TMA boxes of 128 rows x 64
-//               columns, 128B-swizzled) into a three-deep ring
-//   warp 18     (lane 0) scores S = X [w_hi w_lo]^T into a double-buffered TMEM tile, then,
-//               once the labels are known, adds onehot(labels)^T X into a TMEM sum
-//               (M = 128 groups x N = d; A and B both MN-major, read straight from the
-//               one-hot tile and the X tile)
-//   warps 0-15  row r = TMEM lane r, columns split in four quarters (warps w, w + 4, w + 8,
-//               w + 12): argmin and runner-up of bias_g - 2 s_g per quarter and the
-//               quarter's ||x||^2, handed over through shared memory (double-buffered)
-//   warps 16-17 the finisher, two rows per thread: merges the quarters, writes the label
-//               and the count, puts a row whose runner-up is within twice the error bound
-//               on the list of the exact re-check (which corrects its label and, through
-//               the correction list, the sums), and writes the tile's one-hot rows.  The
-//               argmin warps go on to the next tile meanwhile.
-// When the CTA leaves a head (or ends) the sums and the per-group counts go to the
-// partial slot (CTA, head - first head of the CTA).
+// Tensor-core assignment fused with the per-segment centroid sums of the next update.
+// Work: segments of kSeg 128-row tiles of one head (the last segment of a head may be
+// shorter), numbered head-major; CTA c takes a contiguous, balanced run of segments, so
+// every segment is processed whole by one CTA and its sums do not depend on the grid or
+// on how many heads the call holds.  Roles (448 threads):
+//   warps 0-3 / 4-7  argmin groups A / B: the tiles of even / odd running index, one row
+//               per thread (TMEM lane): argmin and runner-up of bias_g - 2 s_g over all
+//               groups, ||x||^2 from the X tile, the label, the certification (a row whose
+//               runner-up is within twice the error bound goes to the exact re-check), the
+//               group count and the row's one in the group's one-hot tile
+//   warp 8      lane 0 issues the MMAs: scores S = X [w_hi w_lo]^T into the group's TMEM
+//               buffer, and, once a tile's one-hot rows are written, onehot^T X into the
+//               TMEM sum buffer of the tile's segment (two buffers, by segment parity)
+//   warp 9      lane 0 loads the X tiles (two TMA boxes of 128 rows x 64 columns per 128
+//               columns, 128B-swizzled) into an XS-deep ring
+//   warps 10-13 flush a finished segment: its sums (TMEM lane = group) and counts go to the
+//               segment's slot, compacted to the groups that occur in it, and the number of
+//               its uncertified rows (listed from the segment's first row on in flag_rows)
+//               to flag_seg
+// A CTA whose run crosses a head drains the pipeline there and loads the next head's
+// weights.  Slot layout: int map[GP] (row of group g in the slot, -1 if absent), int
+// cnt[GP], float rows[...][D].
 // ---------------------------------------------------------------------------
 namespace kma {
-constexpr int NT = 640;
-constexpr int NEPI = 512;   // argmin threads (warps 0-15)
-constexpr int NFIN = 64;    // finisher threads (warps 16-17), two rows each
-constexpr int NQ = 4;   // column quarters
-constexpr int FIN_WARP = 16;
-constexpr int MMA_WARP = 18;
-constexpr int LOAD_WARP = 19;
-constexpr int XS = 3;   // X ring depth
-struct Bars {
-  uint64_t xfull[XS], xempty[XS], tfull[2], tempty[2], ohfull, ohempty, sumdone, xready[2], xfree[2], epidone;
+constexpr int NT = 448;
+constexpr int NARG = 256;    // argmin threads (two groups of 128)
+constexpr int MMA_WARP = 8;
+constexpr int LOAD_WARP = 9;
+constexpr int FL_WARP0 = 10; // flusher warps 10-13
+constexpr int kXSMax = 6;
+template <int D>
+struct Cfg {
+  static constexpr int XS = D == 64 ? 6 : 3;   // X ring depth
 };
-struct Half {
-  float best, second, xx;
-  int bi;
+struct Bars {
+  uint64_t xfull[kXSMax], xempty[kXSMax], tfull[2], tempty[2], ohfull[2], ohempty[2], sumfull[2], sumfree[2],
+      cntready[2], cntfree[4];
 };
 }  // namespace kma
 
+__host__ __device__ inline size_t kmeans_slot_bytes(int GP, int D) { return (size_t)GP * 8 + (size_t)GP * D * 4; }
+
 template <int D>
 __global__ void __launch_bounds__(kma::NT, 1)
-    k_assign_acc(const __grid_constant__ CUtensorMap tmx, int N, int GP, int T, int total, int per, int maxh,
+    k_assign_seg(const __grid_constant__ CUtensorMap tmx, int N, int GP, int T, int SPH, int nseg,
                  const __nv_bfloat16* __restrict__ w_hi, const __nv_bfloat16* __restrict__ w_lo,
                  const float* __restrict__ bias, const float* __restrict__ wnorm, int* __restrict__ labels,
-                 int* __restrict__ trace, int* __restrict__ flag_count, int* __restrict__ flag_rows,
-                 float* __restrict__ psum, int* __restrict__ pcnt, int* err) {
+                 int* __restrict__ trace, int* __restrict__ flag_seg, int* __restrict__ flag_rows,
+                 unsigned char* __restrict__ slots, float* __restrict__ xnorm, int xnorm_store, int* err) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t base = su32(smem);
   if (base & 1023u) {
     if (threadIdx.x == 0) set_error(err, DERR_INDEX);
     return;
   }
-  const int t0 = blockIdx.x * per, t1 = min(total, t0 + per);
-  if (t0 >= t1) return;
+  // this CTA's run of segments
+  const int q = nseg / (int)gridDim.x, rem = nseg % (int)gridDim.x, c = blockIdx.x;
+  const int s_begin = c * q + min(c, rem), s_end = s_begin + q + (c < rem ? 1 : 0);
+  if (s_begin >= s_end) return;
+  constexpr int XS = kma::Cfg<D>::XS;
   constexpr int CPR = D / 8;
   constexpr uint32_t kX = 128u * D * 2u;      // X tile
   constexpr uint32_t kOH = 128u * 128u * 2u;  // one-hot tile [2 halves][128 rows][64 groups]
   const uint32_t kW = (uint32_t)GP * D * 2u;
-  constexpr int XS = kma::XS;
-  const uint32_t sX = base, sOH = base + XS * kX, sWh = sOH + kOH, sWl = sWh + kW;
-  kma::Half* xchg = reinterpret_cast<kma::Half*>(smem + XS * kX + kOH + 2 * kW);   // [2 tiles][NQ][128]
-  float* sBias = reinterpret_cast<float*>(xchg + 2 * kma::NQ * 128);                // [GP]
-  int* sCnt = reinterpret_cast<int*>(sBias + GP);                                    // [GP]
-  kma::Bars* bars = reinterpret_cast<kma::Bars*>(sCnt + GP);
+  const uint32_t sX = base, sOH = base + XS * kX, sWh = sOH + 2 * kOH, sWl = sWh + kW;
+  float* sBias = reinterpret_cast<float*>(smem + XS * kX + 2 * kOH + 2 * kW);   // [GP]
+  int* sCnt = reinterpret_cast<int*>(sBias + GP);                                // [4][GP]
+  int* flw = sCnt + 4 * GP;                                                       // [2][4]
+  int* sFlag = flw + 8;                                                           // [4] flagged rows per segment
+  static_assert(sizeof(kma::Bars) % 8 == 0, "barrier alignment");
+  kma::Bars* bars = reinterpret_cast<kma::Bars*>(sFlag + 4);
   int* sMisc = reinterpret_cast<int*>(bars + 1);   // [0] tmem, [1] abort, [2] max ||w|| bits
   volatile int* abort_flag = sMisc + 1;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t slot_bytes = kmeans_slot_bytes(GP, D);
 
   if (tid == 0) {
     sMisc[1] = 0;
@@ -367,27 +429,30 @@ __global__ void __launch_bounds__(kma::NT, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(su32(&bars->tfull[b]), 1);
-      mbar_init(su32(&bars->tempty[b]), kma::NEPI);
+      mbar_init(su32(&bars->tempty[b]), 128);
+      mbar_init(su32(&bars->ohfull[b]), 128);
+      mbar_init(su32(&bars->ohempty[b]), 1);
+      mbar_init(su32(&bars->sumfull[b]), 1);
+      mbar_init(su32(&bars->sumfree[b]), 128);
+      mbar_init(su32(&bars->cntready[b]), 1);
     }
-    mbar_init(su32(&bars->ohfull), kma::NFIN);
-    mbar_init(su32(&bars->ohempty), 1);
-    mbar_init(su32(&bars->sumdone), 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(su32(&bars->xready[b]), kma::NEPI);
-      mbar_init(su32(&bars->xfree[b]), kma::NFIN);
-    }
-    mbar_init(su32(&bars->epidone), kma::NFIN);
+    for (int b = 0; b < 4; ++b) mbar_init(su32(&bars->cntfree[b]), 128);
     fence_barrier_init();
   }
   if (warp == kma::MMA_WARP) {
     tc_alloc(su32(&sMisc[0]), 512);
     tc_relinquish();
   }
+  // both one-hot tiles start all zero (each row then only moves its one); counts zero
+  for (int e = tid; e < (int)(2 * kOH / 16); e += kma::NT)
+    *reinterpret_cast<uint4*>(smem + XS * kX + 16 * e) = make_uint4(0u, 0u, 0u, 0u);
+  for (int e = tid; e < 4 * GP; e += kma::NT) sCnt[e] = 0;
+  if (tid < 4) sFlag[tid] = 0;
+  fence_proxy_async();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = (uint32_t)sMisc[0];
-  const uint32_t tSum = tmem + 256;
+  const uint32_t tmem = (uint32_t)sMisc[0];   // scores: columns [0, 256); sums: [256, 512)
   const uint32_t IDS = idesc_bf16(128, GP, false);
   constexpr uint32_t IDA = idesc_bf16_mn(128, D, true, true);
   // error bound of one score: 2 |x.w_hi + x.w_lo - x.w| <= 2 (2^-18 + 2 D 2^-24) ||x|| ||w||
@@ -396,30 +461,25 @@ __global__ void __launch_bounds__(kma::NT, 1)
     return bounded_wait(su32(&bar), parity, abort_flag, err);
   };
 
-  int it = 0, sg = 0;   // running tile / segment counters (identical across roles)
+  int it = 0, sgi = 0;          // running tile / segment counters of this CTA (same in every role)
   bool ok = true;
-  int prev_c[2] = {-1, -1};   // finisher: chunk of each of its rows' one in the one-hot tile
-  // the one-hot tile starts all zero (the finisher then only moves each row's one)
-  for (int e = tid; e < (int)(kOH / 16); e += kma::NT)
-    *reinterpret_cast<uint4*>(smem + XS * kX + 16 * e) = make_uint4(0u, 0u, 0u, 0u);
-  fence_proxy_async();
-  for (int s0 = t0; s0 < t1 && ok;) {
-    const int bh = s0 / T;
-    const int s1 = min(t1, (bh + 1) * T);
-    const int slot = blockIdx.x * maxh + (bh - t0 / T);
+  int prev_c = -1;              // argmin thread: chunk of its row's one in its group's one-hot tile
+  for (int gs = s_begin; gs < s_end && ok;) {
+    const int bh = gs / SPH;
+    const int ge = min(s_end, (bh + 1) * SPH);            // segments [gs, ge) of head bh
+    const int t_lo = (gs - bh * SPH) * kKmeansSeg, t_hi = min(T, (ge - bh * SPH) * kKmeansSeg);
+    const int ntile = t_hi - t_lo;
     const size_t head = (size_t)bh * N;
     // ---- this head's weights (every role is idle here)
-    __syncthreads();
     for (int e = tid; e < GP * CPR; e += kma::NT) {
-      const int r = e / CPR, c = e - r * CPR;
-      const size_t off = ((size_t)bh * GP + r) * D + c * 8;
-      cp_async16(sWh + tile_off(r, c, GP), w_hi + off, true);
-      cp_async16(sWl + tile_off(r, c, GP), w_lo + off, true);
+      const int r = e / CPR, cc = e - r * CPR;
+      const size_t off = ((size_t)bh * GP + r) * D + cc * 8;
+      cp_async16(sWh + tile_off(r, cc, GP), w_hi + off, true);
+      cp_async16(sWl + tile_off(r, cc, GP), w_lo + off, true);
     }
     float wm = 0.f;
     for (int g = tid; g < GP; g += kma::NT) {
       sBias[g] = bias[(size_t)bh * GP + g];
-      sCnt[g] = 0;
       wm = fmaxf(wm, wnorm[(size_t)bh * GP + g]);
     }
     wm = warp_max(wm);
@@ -430,14 +490,17 @@ __global__ void __launch_bounds__(kma::NT, 1)
     if (lane == 0) atomicMax(&sMisc[2], __float_as_int(wm));   // non-negative floats order as ints
     __syncthreads();
     const float wmax = __int_as_float(sMisc[2]);
+    const int first = it, sg0 = sgi;   // running indices of this run's first tile / segment
+    // running segment index of the run's tile n (n - first = tile offset in the run)
+    auto seg_of = [&](int n) -> int { return sg0 + (t_lo + (n - first)) / kKmeansSeg - t_lo / kKmeansSeg; };
 
     if (warp == kma::LOAD_WARP) {
       // ---------------- loads (rows past this head's N belong to the next head or read as
       // zeros; their labels and one-hot rows are never used) ----------------
       if (lane == 0) {
-        for (int i = s0; i < s1 && ok; ++i, ++it) {
-          const int xb = it % XS, n0 = (i - bh * T) * 128;
-          if (it >= XS) ok = wait(bars->xempty[xb], ((it / XS) - 1) & 1);
+        for (int n = first; n < first + ntile && ok; ++n) {
+          const int xb = n % XS, n0 = (t_lo + n - first) * 128;
+          if (n >= XS) ok = wait(bars->xempty[xb], ((n / XS) - 1) & 1);
           if (!ok) break;
           mbar_arrive_expect_tx(su32(&bars->xfull[xb]), kX);
 #pragma unroll
@@ -446,14 +509,10 @@ __global__ void __launch_bounds__(kma::NT, 1)
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      it = __shfl_sync(0xffffffffu, it, 0);
     } else if (warp == kma::MMA_WARP) {
-      // ---------------- MMA ----------------
-      // Scores and sums are issued as their inputs become ready, not in a fixed order: the
-      // scores of a later tile (needing its X tile and a free score buffer) do not wait
-      // behind the sums of an earlier tile (needing that tile's one-hot rows).
+      // ---------------- MMA: scores and sums issued as their inputs become ready ----------
       if (lane == 0) {
-        const int first = it, last = it + (s1 - s0);
+        const int last = first + ntile;
         int ns = first, nm = first;   // next tile to score / to sum
         const uint64_t t_start = gtimer();
         while (ok && nm < last) {
@@ -481,17 +540,30 @@ __global__ void __launch_bounds__(kma::NT, 1)
               moved = true;
             }
           }
-          if (nm < ns && mbar_test(su32(&bars->ohfull), nm & 1)) {
-            const int xj = nm % XS;
-            tc_fence_after();
+          if (nm < ns) {
+            const int b = nm & 1, xj = nm % XS;
+            const int tl = t_lo + nm - first;                 // tile index in the head
+            const bool seg_first = (tl % kKmeansSeg) == 0, seg_last = (tl % kKmeansSeg) == kKmeansSeg - 1 || tl == T - 1;
+            const int si = seg_of(nm), sb = si & 1;
+            if (mbar_test(su32(&bars->ohfull[b]), (nm >> 1) & 1) &&
+                (!seg_first || si < 2 || mbar_test(su32(&bars->sumfree[sb]), ((si >> 1) - 1) & 1))) {
+              tc_fence_after();
+              const uint32_t tSum = tmem + 256 + 128 * sb;
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-              tc_mma(tSum, sdesc(sOH + k * 2048, 16384, 1024), sdesc(sX + xj * kX + k * 2048, 16384, 1024), IDA,
-                     (nm > first || k > 0) ? 1u : 0u);
-            tc_commit(su32(&bars->xempty[xj]));
-            tc_commit(su32(&bars->ohempty));
-            ++nm;
-            moved = true;
+              for (int k = 0; k < 8; ++k)
+                tc_mma(tSum, sdesc(sOH + b * kOH + k * 2048, 16384, 1024), sdesc(sX + xj * kX + k * 2048, 16384, 1024),
+                       IDA, (!seg_first || k > 0) ? 1u : 0u);
+              tc_commit(su32(&bars->xempty[xj]));
+              tc_commit(su32(&bars->ohempty[b]));
+              if (seg_last) {
+                tc_commit(su32(&bars->sumfull[sb]));
+                // every count of the segment was made before its tiles' one-hot arrivals,
+                // which this thread has waited for: hand them to the flusher
+                mbar_arrive(su32(&bars->cntready[sb]));
+              }
+              ++nm;
+              moved = true;
+            }
           }
           if (!moved) {
             if (*abort_flag) ok = false;
@@ -502,176 +574,169 @@ __global__ void __launch_bounds__(kma::NT, 1)
             }
           }
         }
-        it = nm;
-        tc_commit(su32(&bars->sumdone));
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      it = __shfl_sync(0xffffffffu, it, 0);
-    } else if (warp >= kma::FIN_WARP) {
-      // ---------------- finisher (warps 16-17): merge the quarters of rows f and f + 64,
-      // labels, counts, flags, one-hot rows ----------------
-      const int f = tid - kma::FIN_WARP * 32;
-      for (int i = s0; i < s1 && ok; ++i, ++it) {
-        const int b = it & 1;
-        ok = __all_sync(0xffffffffu, wait(bars->xready[b], (it >> 1) & 1));
-        if (!ok) break;
-        int bi2[2];
-        float best2[2], second2[2], xsum2[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int r = f + 64 * u;
-          // merge in column order, so a lower quarter wins ties
-          kma::Half m = xchg[(b * kma::NQ + 0) * 128 + r];
-          float xsum = m.xx;
-#pragma unroll
-          for (int q = 1; q < kma::NQ; ++q) {
-            const kma::Half o = xchg[(b * kma::NQ + q) * 128 + r];
-            xsum += o.xx;
-            const bool take = o.best < m.best;
-            m.second = take ? fminf(m.best, o.second) : fminf(m.second, o.best);
-            if (take) { m.best = o.best; m.bi = o.bi; }
-          }
-          bi2[u] = m.bi;
-          best2[u] = m.best;
-          second2[u] = m.second;
-          xsum2[u] = xsum;
-        }
-        // xchg[b] may take tile it + 2
-        mbar_arrive(su32(&bars->xfree[b]));
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int r = f + 64 * u, row = (i - bh * T) * 128 + r;
-          if (row < N) {
-            const float best = best2[u], second = second2[u];
-            const int bi = bi2[u];
-            const float bound = kc * sqrtf(xsum2[u]) * wmax + 1e-6f * (fabsf(best) + fabsf(second));
-            labels[head + row] = bi;
-            atomicAdd(&sCnt[bi], 1);
-            if (second - best > 2.f * bound) {
-              if (trace) trace[head + row] = bi;
-            } else {
-              const int fs = atomicAdd(&flag_count[bh], 1);
-              flag_rows[head + fs] = row;
-            }
-          }
-        }
-        // one-hot rows of this tile, once the previous sums read theirs: the tile holds the
-        // previous tile's ones (all zero at the start), so a row clears the 16-byte chunk of
-        // its previous one and sets the chunk of its new one (rows past N stay zero)
-        if (it >= 1) ok = __all_sync(0xffffffffu, wait(bars->ohempty, (it - 1) & 1));
-        if (!ok) break;
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int r = f + 64 * u;
-          const bool in = (i - bh * T) * 128 + r < N;
-          const int bi = bi2[u];
-          const int c_new = in ? (bi >> 3) : -1;
-          if (prev_c[u] >= 0 && prev_c[u] != c_new)
-            *reinterpret_cast<uint4*>(smem + XS * kX + tile_off(r, prev_c[u], 128)) = make_uint4(0u, 0u, 0u, 0u);
-          if (c_new >= 0) {
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t one = 0x3F80u << (16 * (bi & 1));   // bf16 1.0 in the low or high half
-            const int wd = (bi & 7) >> 1;
-            if (wd == 0) v.x = one; else if (wd == 1) v.y = one; else if (wd == 2) v.z = one; else v.w = one;
-            *reinterpret_cast<uint4*>(smem + XS * kX + tile_off(r, c_new, 128)) = v;
-          }
-          prev_c[u] = c_new;
-        }
-        fence_proxy_async();
-        mbar_arrive(su32(&bars->ohfull));
-      }
-      // every row's count of this head is in sCnt
-      mbar_arrive(su32(&bars->epidone));
-    } else {
-      // ---------------- argmin per column quarter (warps 0-15) ----------------
-      const int hf = warp >> 2;                 // column quarter
-      const int r = (warp & 3) * 32 + lane;     // row = TMEM lane
-      const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-      for (int i = s0; i < s1 && ok; ++i, ++it) {
-        const int b = it & 1, xb = it % XS;
-        // scores ready; the X tile (read below for ||x||) completed before them
-        ok = __all_sync(0xffffffffu, wait(bars->tfull[b], (it >> 1) & 1) && wait(bars->xfull[xb], (it / XS) & 1));
+    } else if (warp >= kma::FL_WARP0) {
+      // ---------------- flusher: one thread per group (TMEM lane) ----------------
+      const int r = 32 * (warp & 3) + lane;
+      const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+      for (int si = sg0; si < sg0 + (ge - gs) && ok; ++si) {
+        const int sb = si & 1;
+        // all four flusher warps agree before their prefix barrier below
+        ok = bar_and(2, 128, wait(bars->sumfull[sb], (si >> 1) & 1) && wait(bars->cntready[sb], (si >> 1) & 1));
         if (!ok) break;
         tc_fence_after();
-        // argmin and runner-up of bias_g - 2 s_g over this quarter, in four interleaved sets
-        float bst[4], snd[4];
-        int bix[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) { bst[q] = __int_as_float(0x7f800000); snd[q] = bst[q]; bix[q] = 0; }
-        {
-          const int cb = hf * 32;
-          if (cb < GP) {
-            uint32_t v[32];
-            tc_ld32(tmem + 128 * b + lane_off + cb, v);
-            const uint64_t m2 = f2pack(-2.f, -2.f);
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              float sc2[2];
-              f2unpack(ffma2(m2, f2pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
-                             f2pack(sBias[cb + e], sBias[cb + e + 1])), sc2[0], sc2[1]);
-#pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                const int q = (e + u) & 3;
-                const float sc = sc2[u];
-                snd[q] = fminf(snd[q], fmaxf(bst[q], sc));
-                bix[q] = sc < bst[q] ? cb + e + u : bix[q];
-                bst[q] = fminf(bst[q], sc);
-              }
-            }
-          }
+        int* cnt4 = sCnt + (si & 3) * GP;
+        const int cnt = r < GP ? cnt4[r] : 0;
+        const bool occ = cnt > 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, occ);
+        int* fl = flw + (si & 1) * 4;
+        // warps in TMEM-lane order: the compacted rows follow the group order
+        if (lane == 0) fl[warp & 3] = __popc(bal);
+        named_sync(2, 128);
+        int idx = __popc(bal & ((1u << lane) - 1u));
+        for (int w = 0; w < (warp & 3); ++w) idx += fl[w];
+        unsigned char* slot = slots + (size_t)(gs + si - sg0) * slot_bytes;
+        int* smap = reinterpret_cast<int*>(slot);
+        int* scnt = smap + GP;
+        float* srow = reinterpret_cast<float*>(scnt + GP);
+        if (r < GP) {
+          smap[r] = occ ? idx : -1;
+          scnt[r] = cnt;
         }
-        tc_fence_before();
-        mbar_arrive(su32(&bars->tempty[b]));
-        kma::Half h;
-        h.best = bst[0]; h.second = snd[0]; h.bi = bix[0];
+        const uint32_t tSum = tmem + 256 + 128 * sb;
 #pragma unroll
-        for (int q = 1; q < 4; ++q) {
-          const bool take = bst[q] < h.best || (bst[q] == h.best && bix[q] < h.bi);
-          h.second = take ? fminf(h.best, snd[q]) : fminf(h.second, bst[q]);
-          if (take) { h.best = bst[q]; h.bi = bix[q]; }
-        }
-        // ||x||^2 of this quarter of the row, from the swizzled tile
-        float xx = 0.f;
-#pragma unroll
-        for (int c = 0; c < CPR / kma::NQ; ++c) {
-          const uint4 u = *reinterpret_cast<const uint4*>(smem + xb * kX + tile_off(r, hf * (CPR / kma::NQ) + c, 128));
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 fl = __bfloat1622float2(h2[e]);
-            xx = fmaf(fl.x, fl.x, fmaf(fl.y, fl.y, xx));
-          }
-        }
-        h.xx = xx;
-        // the finisher has read xchg[b] of tile it - 2
-        if (it >= 2) ok = __all_sync(0xffffffffu, wait(bars->xfree[b], ((it >> 1) - 1) & 1));
-        if (!ok) break;
-        xchg[(b * kma::NQ + hf) * 128 + r] = h;
-        mbar_arrive(su32(&bars->xready[b]));
-      }
-      // ---- sums and counts of this head -> partial slot (each quarter writes 32 columns)
-      if (ok) ok = __all_sync(0xffffffffu, wait(bars->sumdone, sg & 1));
-      if (ok) ok = __all_sync(0xffffffffu, wait(bars->epidone, sg & 1));
-      if (ok) {
-        tc_fence_after();
-        for (int cb = hf * 32; cb < D; cb += 32 * kma::NQ) {
+        for (int cb = 0; cb < D; cb += 32) {
           uint32_t v[32];
           tc_ld32(tSum + lane_off + cb, v);
-          if (r < GP) {
-            float* dst = psum + ((size_t)slot * GP + r) * D + cb;
+          if (occ) {
+            float* dst = srow + (size_t)idx * D + cb;
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
               *reinterpret_cast<float4*>(dst + e) = make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]),
                                                                 __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
           }
         }
-        if (r < GP && hf == 0) pcnt[(size_t)slot * GP + r] = sCnt[r];
+        if (r < GP) cnt4[r] = 0;
+        if (r == 0) {
+          flag_seg[gs + si - sg0] = sFlag[si & 3];
+          sFlag[si & 3] = 0;
+        }
+        mbar_arrive(su32(&bars->cntfree[si & 3]));   // the count buffers may take segment si + 4
         tc_fence_before();
+        mbar_arrive(su32(&bars->sumfree[sb]));
+      }
+    } else {
+      // ---------------- argmin groups (warps 0-3: even tiles, 4-7: odd tiles) ----------
+      const int grp = warp >> 2;
+      const int r = 32 * (warp & 3) + lane;   // row = TMEM lane
+      int cnt_seg = sg0 - 1;                  // last segment whose count buffer this thread checked
+      const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+      for (int n = first + ((first & 1) != grp ? 1 : 0); n < first + ntile && ok; n += 2) {
+        const int b = grp, xb = n % XS;
+        // scores ready; the X tile (read below for ||x||) completed before them
+        ok = __all_sync(0xffffffffu, wait(bars->tfull[b], (n >> 1) & 1) && wait(bars->xfull[xb], (n / XS) & 1));
+        if (!ok) break;
+        const int tl = t_lo + n - first, row = tl * 128 + r;
+        const bool in = row < N;
+        // ||x||^2: computed from the tile by the first pass of a k-means and kept; later passes
+        // read it (the load goes out before the scores are read)
+        float xx = 0.f;
+        if (!xnorm_store && in) xx = xnorm[head + row];
+        tc_fence_after();
+        // argmin and runner-up of bias_g - 2 s_g, in four interleaved sets (columns in order,
+        // so the lower group wins a tie inside a set; sets merged in group order below)
+        float bst[4], snd[4];
+        int bix[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) { bst[u] = __int_as_float(0x7f800000); snd[u] = bst[u]; bix[u] = 0; }
+        const uint64_t m2 = f2pack(-2.f, -2.f);
+        for (int cb = 0; cb < GP; cb += 32) {
+          uint32_t v[32];
+          tc_ld32(tmem + 128 * b + lane_off + cb, v);
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float sc2[2];
+            f2unpack(ffma2(m2, f2pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
+                           f2pack(sBias[cb + e], sBias[cb + e + 1])), sc2[0], sc2[1]);
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int qq = (e + u) & 3;
+              const float sc = sc2[u];
+              snd[qq] = fminf(snd[qq], fmaxf(bst[qq], sc));
+              bix[qq] = sc < bst[qq] ? cb + e + u : bix[qq];
+              bst[qq] = fminf(bst[qq], sc);
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(su32(&bars->tempty[b]));
+        float best = bst[0], second = snd[0];
+        int bi = bix[0];
+#pragma unroll
+        for (int u = 1; u < 4; ++u) {
+          const bool take = bst[u] < best || (bst[u] == best && bix[u] < bi);
+          second = take ? fminf(best, snd[u]) : fminf(second, bst[u]);
+          if (take) { best = bst[u]; bi = bix[u]; }
+        }
+        if (xnorm_store) {
+#pragma unroll
+          for (int cc = 0; cc < CPR; ++cc) {
+            const uint4 u4 = *reinterpret_cast<const uint4*>(smem + xb * kX + tile_off(r, cc, 128));
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 fl = __bfloat1622float2(h2[e]);
+              xx = fmaf(fl.x, fl.x, fmaf(fl.y, fl.y, xx));
+            }
+          }
+          if (in) xnorm[head + row] = xx;
+        }
+        bool certified = true;
+        if (in) {
+          const float bound = kc * sqrtf(xx) * wmax + 1e-6f * (fabsf(best) + fabsf(second));
+          labels[head + row] = bi;
+          certified = second - best > 2.f * bound;
+          if (certified && trace) trace[head + row] = bi;
+        }
+        // the one-hot tile of this group is free once the sums of its tile n - 2 are done
+        if (n >= 2) ok = __all_sync(0xffffffffu, wait(bars->ohempty[b], ((n >> 1) - 1) & 1));
+        if (!ok) break;
+        // the count buffers of segment si were last used by segment si - 4: wait for its flush
+        const int si = seg_of(n);
+        if (si != cnt_seg) {
+          if (si >= 4) ok = __all_sync(0xffffffffu, wait(bars->cntfree[si & 3], ((si >> 2) - 1) & 1));
+          if (!ok) break;
+          cnt_seg = si;
+        }
+        {
+          // one count update per distinct label of the warp
+          const unsigned peers = __match_any_sync(0xffffffffu, in ? bi : -1);
+          if (in && lane == __ffs(peers) - 1) atomicAdd(&sCnt[(si & 3) * GP + bi], __popc(peers));
+        }
+        // uncertified: onto the segment's list for the exact re-check
+        if (in && !certified)
+          flag_rows[head + (size_t)(tl / kKmeansSeg) * (kKmeansSeg * 128) + atomicAdd(&sFlag[si & 3], 1)] = row;
+        const int c_new = in ? (bi >> 3) : -1;
+        const uint32_t oh = XS * kX + b * kOH;
+        if (prev_c >= 0 && prev_c != c_new)
+          *reinterpret_cast<uint4*>(smem + oh + tile_off(r, prev_c, 128)) = make_uint4(0u, 0u, 0u, 0u);
+        if (c_new >= 0) {
+          uint4 v4 = make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t one = 0x3F80u << (16 * (bi & 1));   // bf16 1.0 in the low or high half
+          const int wd = (bi & 7) >> 1;
+          if (wd == 0) v4.x = one; else if (wd == 1) v4.y = one; else if (wd == 2) v4.z = one; else v4.w = one;
+          *reinterpret_cast<uint4*>(smem + oh + tile_off(r, c_new, 128)) = v4;
+        }
+        prev_c = c_new;
+        fence_proxy_async();
+        mbar_arrive(su32(&bars->ohfull[b]));
       }
     }
-    ++sg;
+    it = first + ntile;
+    sgi = sg0 + (ge - gs);
     ok = __syncthreads_and(ok ? 1 : 0) != 0;
-    s0 = s1;
+    gs = ge;
   }
   tc_fence_before();
   __syncthreads();
@@ -692,18 +757,29 @@ template <int DT>
 __global__ void __launch_bounds__(512) k_assign_recheck(const __nv_bfloat16* __restrict__ X, int N, int d,
                                                        const float* __restrict__ A, size_t a_head, int sj, int sc,
                                                        float a_scale, int D, const float* __restrict__ nu, int G,
-                                                       const int* __restrict__ flag_count,
+                                                       const int* __restrict__ flag_seg, int SPH,
                                                        const int* __restrict__ flag_rows, int* __restrict__ labels,
                                                        int* __restrict__ trace, int* __restrict__ corr_count,
                                                        int4* __restrict__ corr) {
   extern __shared__ __align__(16) float sr[];
   const int bh = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int cnt = flag_count[bh];
-  if ((int)blockIdx.x * 16 >= cnt) return;
   float* sA = sr;                       // [D][d + 1]
   float* sNu = sA + D * (d + 1);        // [G][DT + 1]
   float* sx = sNu + G * (DT + 1);       // [16][d]
   float* sy = sx + 16 * d;              // [16][DT]
+  int* pre = reinterpret_cast<int*>(sy + 16 * DT);   // [SPH + 1] first flagged item of each segment
+  // the head's uncertified rows: segment s lists flag_seg[s] of them from row s * kSeg * 128 on
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int sgm = 0; sgm < SPH; ++sgm) {
+      pre[sgm] = acc;
+      acc += flag_seg[(size_t)bh * SPH + sgm];
+    }
+    pre[SPH] = acc;
+  }
+  __syncthreads();
+  const int cnt = pre[SPH];
+  if ((int)blockIdx.x * 16 >= cnt) return;
   const size_t head = (size_t)bh * N;
   const float* Ah = A + a_head * bh;
   const float* nuh = nu + (size_t)bh * G * DT;
@@ -722,7 +798,13 @@ __global__ void __launch_bounds__(512) k_assign_recheck(const __nv_bfloat16* __r
   float* wx = sx + warp * d;
   float* wy = sy + warp * DT;
   for (int i = blockIdx.x * 16 + warp; i < cnt; i += gridDim.x * 16) {
-    const int row = flag_rows[head + i];
+    int lo = 0, hi = SPH - 1;   // segment of item i: the last with pre[s] <= i
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    const int row = flag_rows[head + (size_t)lo * (kKmeansSeg * 128) + (i - pre[lo])];
+    if (row < 0 || row >= N) continue;
     for (int c = lane; c < d; c += 32) wx[c] = bf2f(X[(head + row) * d + c]);
     __syncwarp();
     for (int j = lane; j < DT; j += 32) {
@@ -1074,18 +1156,22 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
 int kmeans_gp(int G) { return (G + 31) / 32 * 32; }
 
 size_t assign_acc_smem(int D, int GP) {
-  return (size_t)km::kma::XS * 128 * D * 2 + (size_t)128 * 128 * 2 + 2 * (size_t)GP * D * 2 +
-         2 * km::kma::NQ * 128 * sizeof(km::kma::Half) + (size_t)GP * 8 + sizeof(km::kma::Bars) + 16;
+  const int XS = D == 64 ? km::kma::Cfg<64>::XS : km::kma::Cfg<128>::XS;
+  return (size_t)XS * 128 * D * 2 + 2 * (size_t)128 * 128 * 2 + 2 * (size_t)GP * D * 2 + (size_t)GP * 4 +
+         (size_t)4 * GP * 4 + 12 * 4 + sizeof(km::kma::Bars) + 16;
 }
 
 KmPlan kmeans_plan(int BH, int N) {
   KmPlan pl{};
   pl.T = ceil_div(N, 128);
-  pl.total = BH * pl.T;
-  pl.grid = pl.total < kKmeansCtas ? pl.total : kKmeansCtas;
-  pl.per = ceil_div(pl.total, pl.grid);
-  pl.maxh = pl.per / pl.T + 2;
+  pl.SPH = ceil_div(pl.T, kKmeansSeg);
+  pl.nseg = BH * pl.SPH;
+  pl.grid = pl.nseg < kKmeansCtas ? pl.nseg : kKmeansCtas;
   return pl;
+}
+
+size_t kmeans_slots_bytes(int BH, int N, int GP, int d) {
+  return (size_t)BH * kmeans_plan(BH, N).SPH * km::kmeans_slot_bytes(GP, d);
 }
 
 cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_t seed, HeadMap hm, int purpose,
@@ -1096,20 +1182,20 @@ cudaError_t launch_seed_rows(const void* X, int BH, int N, int d, int G, uint64_
   return cudaGetLastError();
 }
 
-size_t centroid_weights_smem(int d, int D) {
+size_t centroid_weights_smem(int d, int D, int N) {
+  const int SPH = kmeans_plan(1, N).SPH;
   return (size_t)km::WG_PER_CTA * d * 8 + km::WG_PER_CTA * 4 +
-         ((size_t)D * (d + 1) + (size_t)km::WG_PER_CTA * d + (size_t)km::WG_PER_CTA * 128) * 4;
+         ((size_t)km::cw_scratch_floats(d, D, SPH) + (size_t)km::WG_PER_CTA * d + (size_t)km::WG_PER_CTA * 128) * 4;
 }
 
 cudaError_t launch_centroid_weights(float* m, int BH, int G, int d, const float* A, size_t a_head, int sj, int sc,
-                                    float a_scale, int D, int DT, int mode, const float* psum, const int* pcnt,
+                                    float a_scale, int D, int DT, int mode, const void* slots,
                                     const int* corr_count, const void* corr, const void* X, int N, float* nu,
                                     float* bias, float* wnorm, void* w_hi, void* w_lo, int* err, cudaStream_t st) {
   const int GP = kmeans_gp(G);
-  const size_t sm = centroid_weights_smem(d, D);
+  const size_t sm = centroid_weights_smem(d, D, N);
   const KmPlan pl = kmeans_plan(BH, N);
-  km::KmPartials pp{psum, pcnt, corr_count, (const int4*)corr, (const __nv_bfloat16*)X, N, pl.T, pl.per, pl.maxh,
-                    pl.grid};
+  km::KmPartials pp{(const unsigned char*)slots, corr_count, (const int4*)corr, (const __nv_bfloat16*)X, N, pl.SPH};
   cudaFuncSetAttribute(km::k_centroid_weights, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   km::k_centroid_weights<<<dim3(ceil_div(GP, km::WG_PER_CTA), BH), km::CW_THREADS, sm, st>>>(
       m, G, GP, d, A, a_head, sj, sc, a_scale, D, DT, mode, pp, nu, bias, wnorm, (__nv_bfloat16*)w_hi,
@@ -1118,8 +1204,9 @@ cudaError_t launch_centroid_weights(float* m, int BH, int G, int d, const float*
 }
 
 cudaError_t launch_assign_acc(const void* X, int BH, int N, int d, int G, const void* w_hi, const void* w_lo,
-                              const float* bias, const float* wnorm, int* labels, int* trace, int* flag_count,
-                              int* flag_rows, float* psum, int* pcnt, int* err, cudaStream_t st) {
+                              const float* bias, const float* wnorm, int* labels, int* trace, int* flag_seg,
+                              int* flag_rows, void* slots, float* xnorm, int xnorm_store, int* err,
+                              cudaStream_t st) {
   const int GP = kmeans_gp(G);
   const size_t sm = assign_acc_smem(d, GP);
   const KmPlan pl = kmeans_plan(BH, N);
@@ -1127,46 +1214,48 @@ cudaError_t launch_assign_acc(const void* X, int BH, int N, int d, int G, const 
   cudaError_t e = make_tmap_bf16_rows(&tmx, X, (unsigned long long)BH * N, d, 128);
   if (e != cudaSuccess) return e;
   if (d == 64) {
-    cudaFuncSetAttribute(km::k_assign_acc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    km::k_assign_acc<64><<<pl.grid, km::kma::NT, sm, st>>>(
-        tmx, N, GP, pl.T, pl.total, pl.per, pl.maxh, (const __nv_bfloat16*)w_hi, (const __nv_bfloat16*)w_lo, bias,
-        wnorm, labels, trace, flag_count, flag_rows, psum, pcnt, err);
+    cudaFuncSetAttribute(km::k_assign_seg<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    km::k_assign_seg<64><<<pl.grid, km::kma::NT, sm, st>>>(
+        tmx, N, GP, pl.T, pl.SPH, pl.nseg, (const __nv_bfloat16*)w_hi, (const __nv_bfloat16*)w_lo, bias, wnorm,
+        labels, trace, flag_seg, flag_rows, (unsigned char*)slots, xnorm, xnorm_store, err);
   } else {
-    cudaFuncSetAttribute(km::k_assign_acc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-    km::k_assign_acc<128><<<pl.grid, km::kma::NT, sm, st>>>(
-        tmx, N, GP, pl.T, pl.total, pl.per, pl.maxh, (const __nv_bfloat16*)w_hi, (const __nv_bfloat16*)w_lo, bias,
-        wnorm, labels, trace, flag_count, flag_rows, psum, pcnt, err);
+    cudaFuncSetAttribute(km::k_assign_seg<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    km::k_assign_seg<128><<<pl.grid, km::kma::NT, sm, st>>>(
+        tmx, N, GP, pl.T, pl.SPH, pl.nseg, (const __nv_bfloat16*)w_hi, (const __nv_bfloat16*)w_lo, bias, wnorm,
+        labels, trace, flag_seg, flag_rows, (unsigned char*)slots, xnorm, xnorm_store, err);
   }
   return cudaGetLastError();
 }
 
-size_t recheck_smem(int d, int D, int DT, int G) {
-  return ((size_t)D * (d + 1) + (size_t)G * (DT + 1) + 16 * (size_t)d + 16 * (size_t)DT) * 4;
+size_t recheck_smem(int d, int D, int DT, int G, int N) {
+  return ((size_t)D * (d + 1) + (size_t)G * (DT + 1) + 16 * (size_t)d + 16 * (size_t)DT) * 4 +
+         ((size_t)kmeans_plan(1, N).SPH + 1) * 4;
 }
 
 template <int DT>
 static cudaError_t recheck_dt(const void* X, int BH, int N, int d, const float* A, size_t a_head, int sj, int sc,
-                              float a_scale, int D, const float* nu, int G, const int* flag_count,
+                              float a_scale, int D, const float* nu, int G, const int* flag_seg,
                               const int* flag_rows, int* labels, int* trace, int* corr_count, void* corr,
                               cudaStream_t st) {
-  const size_t sm = recheck_smem(d, D, DT, G);
+  const size_t sm = recheck_smem(d, D, DT, G, N);
+  const int SPH = kmeans_plan(1, N).SPH;
   cudaFuncSetAttribute(km::k_assign_recheck<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   km::k_assign_recheck<DT><<<dim3(km::RC_PER_HEAD, BH), 512, sm, st>>>((const __nv_bfloat16*)X, N, d, A, a_head, sj,
-                                                                      sc, a_scale, D, nu, G, flag_count, flag_rows,
+                                                                      sc, a_scale, D, nu, G, flag_seg, SPH, flag_rows,
                                                                       labels, trace, corr_count, (int4*)corr);
   return cudaGetLastError();
 }
 
 cudaError_t launch_assign_recheck(const void* X, int BH, int N, int d, const float* A, size_t a_head, int sj, int sc,
-                                  float a_scale, int D, const float* nu, int G, const int* flag_count,
+                                  float a_scale, int D, const float* nu, int G, const int* flag_seg,
                                   const int* flag_rows, int* labels, int* trace, int* corr_count, void* corr,
                                   cudaStream_t st) {
   switch (kmeans_dt(D)) {
-    case 8: return recheck_dt<8>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, corr_count, corr, st);
-    case 16: return recheck_dt<16>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, corr_count, corr, st);
-    case 32: return recheck_dt<32>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, corr_count, corr, st);
-    case 64: return recheck_dt<64>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, corr_count, corr, st);
-    case 128: return recheck_dt<128>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_count, flag_rows, labels, trace, corr_count, corr, st);
+    case 8: return recheck_dt<8>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_seg, flag_rows, labels, trace, corr_count, corr, st);
+    case 16: return recheck_dt<16>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_seg, flag_rows, labels, trace, corr_count, corr, st);
+    case 32: return recheck_dt<32>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_seg, flag_rows, labels, trace, corr_count, corr, st);
+    case 64: return recheck_dt<64>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_seg, flag_rows, labels, trace, corr_count, corr, st);
+    case 128: return recheck_dt<128>(X, BH, N, d, A, a_head, sj, sc, a_scale, D, nu, G, flag_seg, flag_rows, labels, trace, corr_count, corr, st);
     default: return cudaErrorInvalidValue;
   }
 }

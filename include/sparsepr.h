@@ -40,7 +40,9 @@
  *    checks (bounded waits, index checks) record an error code in the workspace;
  *    read it with sparsepr_workspace_error() after the stream has drained.  Codes:
  *    1 index out of range, 2 bounded wait ran out, 3 random-draw map overflow,
- *    4 non-finite value, 5 frame ids out of range or decreasing.
+ *    4 non-finite value, 5 frame ids out of range or decreasing, 6 more than 2048
+ *    k-means label corrections for one block of 16 groups in one Lloyd step (the
+ *    exact re-check of near-tie rows; the call's outputs are then unspecified).
  *  - Determinism: for fixed inputs, params and seed every output is bitwise
  *    reproducible (no floating-point atomics on any output path).
  *  - Random draws (query sample, k-means seeds, probe rows) use SplitMix64

@@ -163,6 +163,12 @@ def test_head_chunks_equal_one_call_ragged_batches(gpu):
     _head_chunk_case(gpu, _ragged_workload(), 2, seed=7)
 
 
+def test_head_chunks_equal_one_call_mid(gpu):
+    # 12 heads of 8192 tokens: the k-means runs over many segments per CTA in the unsplit
+    # call and over a different CTA layout in each chunk; its sums are per fixed segment
+    _head_chunk_case(gpu, workload("mid"), 4, seed=8)
+
+
 def test_head_offset_draws_the_layer_streams(gpu):
     """A call on one head with head_offset = h draws head h's random streams: its query
     sample, k-means seeds and probe rows are the oracle's for layer head h."""
