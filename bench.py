@@ -498,13 +498,13 @@ def partition_diagnostics(part, Q, K, o_sparse, o_dense, p, frames=None, heads=(
         sizes = torch.bincount(lq, minlength=p.n_qgroups)
         cand = torch.nonzero(sizes > 0).flatten()
         pick = cand[torch.linspace(0, cand.numel() - 1, min(groups, cand.numel())).round().long()]
-        k = K[b, h].float()
+        k = K[b, h].double()
         for a in pick.tolist():
             rows = torch.nonzero(lq == a).flatten()
-            logits = s * (Q[b, h, rows].float() @ k.T)
+            logits = s * (Q[b, h, rows].double() @ k.T)
             if fr is not None:
                 logits = logits.masked_fill(fr[None, :] > fr[rows][:, None], float("-inf"))
-            pr = torch.softmax(logits.double(), dim=1)
+            pr = torch.softmax(logits, dim=1)
 
             def frac(x):
                 srt = torch.sort(x, dim=-1, descending=True).values

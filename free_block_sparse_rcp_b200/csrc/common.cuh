@@ -61,57 +61,17 @@ struct HeadMap {
   __host__ __device__ int global(int bh) const { return (bh / H) * total + offset + bh % H; }
 };
 
-// Partial Fisher-Yates over the virtual array [0, n) with the swapped slots kept in
-// a small open-addressing map (slot -> value) in shared memory.  One thread runs it.
-struct SlotMap {
-  int* key;
-  int* val;
-  int cap;  // power of two
-  __device__ void clear_all(int tid, int nthreads) {
-    for (int i = tid; i < cap; i += nthreads) key[i] = -1;
-  }
-  __device__ __forceinline__ int find(int pos) const {
-    uint32_t h = ((uint32_t)pos * 2654435761u) & (cap - 1);
-    while (key[h] != -1 && key[h] != pos) h = (h + 1) & (cap - 1);
-    return (int)h;
-  }
-  __device__ __forceinline__ int get(int pos) const {
-    int h = find(pos);
-    return key[h] == pos ? val[h] : pos;
-  }
-  __device__ __forceinline__ void put(int pos, int v) {
-    int h = find(pos);
-    key[h] = pos;
-    val[h] = v;
-  }
-};
-
-// Draw m distinct values of [0, n) (m <= cap/2); out[i] = i-th drawn value.
-// The map must be cleared.  Returns false on overflow.
-__device__ inline bool draw_without_replacement(SplitMix64& g, int n, int m, SlotMap& map,
-                                                int* out) {
-  if (2 * m > map.cap) return false;
-  for (int i = 0; i < m; ++i) {
-    int j = i + (int)(g.next() % (uint64_t)(n - i));
-    int vi = map.get(i);
-    int vj = map.get(j);
-    map.put(i, vj);
-    map.put(j, vi);
-    out[i] = vj;
-  }
-  return true;
-}
-
-// Block-cooperative form of the same draw (every thread of the block calls it).  The k-th
-// number of a SplitMix64 stream is mix(state + k * gamma), so the offsets
-// j_i = i + (number i + 1) mod (n - i) of all m draws are computed in parallel into jbuf[m].
-// The swaps are then replayed per draw instead of in order: before draw t a position p >= t
-// holds p unless an earlier draw t' < t swapped with it (j_t' = p), and then, for the last
-// such t', the value position t' held before draw t' -- the same question one level down.
-// So out[i] (the value at position j_i before draw i) follows that chain backwards; draws
-// rarely collide (m << n), so the chain is short.  Same out[] as the sequential form
-// (cap: the map capacity the sequential form allows, m <= cap / 2); returns false on every
-// thread when m exceeds it.
+// Draw m distinct values of [0, n) by a partial Fisher-Yates shuffle (j_i = i + next() mod
+// (n - i), swap positions i and j_i, out[i] = position i after the swap), block-cooperatively
+// (every thread of the block calls it).  The k-th number of a SplitMix64 stream is
+// mix(state + k * gamma), so the offsets j_i = i + (number i + 1) mod (n - i) of all m draws
+// are computed in parallel into jbuf[m].  The swaps are then replayed per draw instead of in
+// order: before draw t a position p >= t holds p unless an earlier draw t' < t swapped with
+// it (j_t' = p), and then, for the last such t', the value position t' held before draw t'
+// -- the same question one level down.  So out[i] (the value at position j_i before draw i)
+// follows that chain backwards; draws rarely collide (m << n), so the chain is short.  The
+// same out[] as the sequential swaps.  Returns false on every thread when 2 m exceeds cap
+// (the callers' scratch bound).
 __device__ inline bool draw_without_replacement_block(uint64_t state, int n, int m, int cap, int* out,
                                                       int* jbuf) {
   if (2 * m > cap) return false;

@@ -80,7 +80,7 @@ constexpr int kCorrCap = 2048;   // corrections of one CTA's groups per pass
 // floats of the region that holds A for the weights and, before that, the segment-slot rows
 // of the CTA's groups and its sorted corrections
 __host__ __device__ inline int cw_scratch_floats(int d, int D, int SPH) {
-  const int a = D * (d + 1), b = SPH * WG_PER_CTA + 2 * kCorrCap;
+  const int a = D * (d + 1), b = 2 * SPH * WG_PER_CTA + 2 * kCorrCap;
   return ((a > b ? a : b) + 3) & ~3;
 }
 
@@ -114,11 +114,15 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
     const size_t sbytes = (size_t)GP * 8 + (size_t)GP * d * 4;
     const unsigned char* hs = pp.slots + (size_t)bh * pp.SPH * sbytes;
     int* spos = reinterpret_cast<int*>(sA);                   // [SPH][WG_PER_CTA] slot rows
-    int2* sel = reinterpret_cast<int2*>(spos + pp.SPH * WG_PER_CTA);   // [kCorrCap] corrections
+    int* scnt = spos + pp.SPH * WG_PER_CTA;                   // [SPH][WG_PER_CTA] slot counts
+    int2* sel = reinterpret_cast<int2*>(scnt + pp.SPH * WG_PER_CTA);   // [kCorrCap] corrections
     __shared__ int s_nsel, s_over;
     for (int e = tid; e < pp.SPH * WG_PER_CTA; e += CW_THREADS) {
       const int sgm = e / WG_PER_CTA, gi = e - sgm * WG_PER_CTA;
-      spos[e] = gi < g1 - g0 ? reinterpret_cast<const int*>(hs + (size_t)sgm * sbytes)[g0 + gi] : -1;
+      const int* smap = reinterpret_cast<const int*>(hs + (size_t)sgm * sbytes);
+      const bool in = gi < g1 - g0;
+      spos[e] = in ? smap[g0 + gi] : -1;
+      scnt[e] = in ? smap[GP + g0 + gi] : 0;
     }
     if (tid == 0) { s_nsel = 0; s_over = 0; }
     __syncthreads();
@@ -163,9 +167,7 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
       if (gis[u] >= 0) acc[tid + u * CW_THREADS] = a[u];
     if (tid < WG_PER_CTA) {
       int n = 0;
-      if (tid < g1 - g0)
-        for (int sgm = 0; sgm < pp.SPH; ++sgm)
-          n += reinterpret_cast<const int*>(hs + (size_t)sgm * sbytes)[GP + g0 + tid];
+      for (int sgm = 0; sgm < pp.SPH; ++sgm) n += scnt[sgm * WG_PER_CTA + tid];
       cnt[tid] = n;
     }
     // the re-check's corrections that move a row out of or into this CTA's groups
@@ -228,11 +230,20 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
     if (mode == 2) return;
   }
   const float* Ah = A + a_head * bh;
-  // staging loops unrolled so that each thread keeps several loads in flight
+  // staging loops unrolled so that each thread keeps several loads in flight; consecutive
+  // threads read consecutive addresses of A (its unit-stride index runs fastest)
+  if (sj == 1) {
 #pragma unroll 8
-  for (int e = tid; e < D * d; e += CW_THREADS) {
-    const int j = e / d, c = e - j * d;
-    sA[j * (d + 1) + c] = Ah[(size_t)j * sj + (size_t)c * sc];
+    for (int e = tid; e < D * d; e += CW_THREADS) {
+      const int c = e / D, j = e - c * D;
+      sA[j * (d + 1) + c] = Ah[(size_t)j + (size_t)c * sc];
+    }
+  } else {
+#pragma unroll 8
+    for (int e = tid; e < D * d; e += CW_THREADS) {
+      const int j = e / d, c = e - j * d;
+      sA[j * (d + 1) + c] = Ah[(size_t)j * sj + (size_t)c * sc];
+    }
   }
   __syncthreads();
 #pragma unroll 8
@@ -783,11 +794,20 @@ __global__ void __launch_bounds__(512) k_assign_recheck(const __nv_bfloat16* __r
   const size_t head = (size_t)bh * N;
   const float* Ah = A + a_head * bh;
   const float* nuh = nu + (size_t)bh * G * DT;
-  // staging loops unrolled so that each thread keeps several loads in flight
+  // staging loops unrolled so that each thread keeps several loads in flight (A's
+  // unit-stride index fastest)
+  if (sj == 1) {
 #pragma unroll 8
-  for (int e = threadIdx.x; e < D * d; e += 512) {
-    const int j = e / d, c = e - j * d;
-    sA[j * (d + 1) + c] = Ah[(size_t)j * sj + (size_t)c * sc];
+    for (int e = threadIdx.x; e < D * d; e += 512) {
+      const int c = e / D, j = e - c * D;
+      sA[j * (d + 1) + c] = Ah[(size_t)j + (size_t)c * sc];
+    }
+  } else {
+#pragma unroll 8
+    for (int e = threadIdx.x; e < D * d; e += 512) {
+      const int j = e / d, c = e - j * d;
+      sA[j * (d + 1) + c] = Ah[(size_t)j * sj + (size_t)c * sc];
+    }
   }
 #pragma unroll 8
   for (int e = threadIdx.x; e < G * DT; e += 512) {
@@ -1008,6 +1028,10 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
       for (int a = a0; a < a1 && ok; ++a) {
         for (int t0 = qo[a]; t0 < qo[a + 1]; t0 += 128, ++tile) {
           const int b = tile & 1, nr = min(128, qo[a + 1] - t0);
+          // the tile's row indices: all four loads go out together, before the slot wait
+          int rows4[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) rows4[k] = 32 * k + lane < nr ? perm_q[head + t0 + 32 * k + lane] : -1;
           if (tile >= 2) ok = __all_sync(0xffffffffu, wait(bars->xempty[b], ((tile >> 1) - 1) & 1));
           if (!ok) break;
 #pragma unroll
@@ -1015,7 +1039,7 @@ __global__ void __launch_bounds__(cmk::NT, 1) k_cell_mass_tc(const __nv_bfloat16
             const int r = 32 * k + lane;
             int myrow = -1;
             if (r < nr) {
-              myrow = perm_q[head + t0 + r];
+              myrow = rows4[k];
               if (myrow < 0 || myrow >= N) { set_error(err, DERR_INDEX); myrow = -1; }
             }
 #pragma unroll

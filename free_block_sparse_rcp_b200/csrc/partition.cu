@@ -139,58 +139,70 @@ __global__ void __launch_bounds__(256) k_key_coords(const __nv_bfloat16* __restr
 }
 
 // ---------------------------------------------------------------------------
-// Stable counting sort by label.  grid = BH, block = 1024, dynamic smem =
-// (33 * G) ints.  perm[pos] = original index; offsets[g] = first position.
+// Stable counting sort by label.  grid = BH, block = 1024, dynamic smem = (33 * G) ints.
+// perm[pos] = original index; offsets[g] = first position.  Warp w owns the contiguous
+// rows [w R, (w + 1) R) (R = ceil(N / 32)): it counts its labels, the counts are turned
+// into each (warp, label)'s first position (label-major, then warp order, so equal labels
+// keep their row order), and the warp places its rows walking them in order, 32 at a
+// time (a label's rank among the 32 by __match_any_sync).  Three block barriers in all.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) k_group_sort(const int* __restrict__ labels, int N, int G,
                                                     int* __restrict__ perm, int* __restrict__ offsets,
                                                     int* err) {
   extern __shared__ __align__(16) unsigned char smem[];
-  int* base = reinterpret_cast<int*>(smem);  // [G]
-  int* wcnt = base + G;                       // [32][G]
+  int* total = reinterpret_cast<int*>(smem);  // [G]
+  int* wcnt = total + G;                       // [32][G]: counts, then first positions
   const int bh = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int* lab = labels + (size_t)bh * N;
-  for (int g = tid; g < G; g += blockDim.x) base[g] = 0;
+  const int R = (N + 31) / 32, r0 = warp * R, r1 = min(N, r0 + R);
+  for (int e = tid; e < 33 * G; e += blockDim.x) total[e] = 0;
   __syncthreads();
-  for (int i = tid; i < N; i += blockDim.x) {
-    int l = lab[i];
-    if (l < 0 || l >= G) { set_error(err, DERR_INDEX); continue; }
-    atomicAdd(&base[l], 1);
+  int* mine = wcnt + warp * G;
+  for (int i0 = r0; i0 < r1; i0 += 32) {
+    const int i = i0 + lane;
+    int l = -1;
+    if (i < r1) {
+      l = lab[i];
+      if (l < 0 || l >= G) { set_error(err, DERR_INDEX); l = -1; }
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, l);
+    if (l >= 0 && lane == __ffs(peers) - 1) mine[l] += __popc(peers);
+  }
+  __syncthreads();
+  // first position of each (warp, label): offset of the label, then the earlier warps'
+  if (tid < G) {
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int c = wcnt[w * G + tid];
+      wcnt[w * G + tid] = run;
+      run += c;
+    }
+    total[tid] = run;
   }
   __syncthreads();
   if (tid == 0) {
     int run = 0;
     for (int g = 0; g < G; ++g) {
-      int c = base[g];
-      base[g] = run;
+      const int c = total[g];
+      total[g] = run;
       offsets[(size_t)bh * (G + 1) + g] = run;
       run += c;
     }
     offsets[(size_t)bh * (G + 1) + G] = run;
   }
   __syncthreads();
-  for (int t0 = 0; t0 < N; t0 += blockDim.x) {
-    for (int e = tid; e < 32 * G; e += blockDim.x) wcnt[e] = 0;
-    __syncthreads();
-    const int i = t0 + tid;
-    int l = (i < N) ? lab[i] : -1;
-    if (l >= G) l = -1;
+  for (int i0 = r0; i0 < r1; i0 += 32) {
+    const int i = i0 + lane;
+    int l = i < r1 ? lab[i] : -1;
+    if (l >= G || l < 0) l = -1;
     const unsigned peers = __match_any_sync(0xffffffffu, l);
-    const int rank = __popc(peers & ((1u << lane) - 1));
-    if (l >= 0 && lane == __ffs(peers) - 1) wcnt[warp * G + l] = __popc(peers);
-    __syncthreads();
     if (l >= 0) {
-      int pre = 0;
-      for (int w = 0; w < warp; ++w) pre += wcnt[w * G + l];
-      perm[(size_t)bh * N + base[l] + pre + rank] = i;
+      const int rank = __popc(peers & ((1u << lane) - 1));
+      perm[(size_t)bh * N + total[l] + mine[l] + rank] = i;
     }
-    __syncthreads();
-    for (int g = tid; g < G; g += blockDim.x) {
-      int s = 0;
-      for (int w = 0; w < 32; ++w) s += wcnt[w * G + g];
-      base[g] += s;
-    }
-    __syncthreads();
+    __syncwarp();
+    if (l >= 0 && lane == __ffs(peers) - 1) mine[l] += __popc(peers);
+    __syncwarp();
   }
 }
 

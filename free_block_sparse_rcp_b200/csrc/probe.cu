@@ -27,8 +27,6 @@ __global__ void __launch_bounds__(256) k_probe_pick(const int* __restrict__ perm
   int* alloc = size + Gq;                     // [Gq]
   int* order = alloc + Gq;                    // [Gq] open groups by decreasing size
   int* draw = order + Gq;                     // [P]
-  int* mkey = draw + 64;                      // [256]
-  int* mval = mkey + 256;                     // [256]
   const int bh = blockIdx.x, tid = threadIdx.x;
   const int* qo = qoff + (size_t)bh * (Gq + 1);
   for (int a = tid; a < Gq; a += blockDim.x) { size[a] = qo[a + 1] - qo[a]; alloc[a] = 0; }
@@ -61,15 +59,27 @@ __global__ void __launch_bounds__(256) k_probe_pick(const int* __restrict__ perm
       }
     }
     SplitMix64 g(stream_state(seed, hm.global(bh), PURPOSE_PROBES));
-    SlotMap map{mkey, mval, 256};
     int outp = 0;
     for (int a = 0; a < Gq; ++a) {
       const int m = alloc[a];
       if (m == 0) continue;
-      for (int i = 0; i < 256; ++i) mkey[i] = -1;
-      if (!draw_without_replacement(g, size[a], m, map, draw)) { set_error(err, DERR_DRAW); break; }
+      // partial Fisher-Yates of m of the group's n members: offsets j_i = i + next() mod (n - i);
+      // draw i takes what position j_i holds before it, replayed through the earlier swaps
+      // (a position p >= t holds p before draw t unless an earlier draw t' swapped with it,
+      // and then what position t' held before draw t'), so no swap map is kept
+      const int n = size[a];
+      for (int i = 0; i < m; ++i) draw[i] = i + (int)(g.next() % (uint64_t)(n - i));
       for (int i = 0; i < m; ++i) {
-        probe_idx[(size_t)bh * P + outp] = perm_q[(size_t)bh * N + qo[a] + draw[i]];
+        int pos = draw[i], t = i;
+        while (true) {
+          int tp = -1;
+          for (int k = t - 1; k >= 0; --k)
+            if (draw[k] == pos) { tp = k; break; }
+          if (tp < 0) break;
+          pos = tp;
+          t = tp;
+        }
+        probe_idx[(size_t)bh * P + outp] = perm_q[(size_t)bh * N + qo[a] + pos];
         probe_grp[(size_t)bh * P + outp] = a;
         ++outp;
       }
@@ -667,7 +677,7 @@ cudaError_t launch_worklist(const unsigned char* route, const int* qoff, const i
 
 cudaError_t launch_probe_pick(const int* perm_q, const int* qoff, int BH, int N, int Gq, int P, uint64_t seed,
                               HeadMap hm, int* probe_idx, int* probe_grp, int* err, cudaStream_t st) {
-  size_t sm = (size_t)(3 * Gq + 64 + 512 + 8) * 4;
+  size_t sm = (size_t)(3 * Gq + 64 + 8) * 4;
   cudaFuncSetAttribute(k_probe_pick, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   k_probe_pick<<<BH, 256, sm, st>>>(perm_q, qoff, N, Gq, P, seed, hm, probe_idx, probe_grp, err);
   return cudaGetLastError();
