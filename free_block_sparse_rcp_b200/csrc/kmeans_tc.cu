@@ -60,25 +60,27 @@ __global__ void __launch_bounds__(256) k_seed_rows(const __nv_bfloat16* __restri
 // ---------------------------------------------------------------------------
 // Centroid weights.  A(j, c) = a_scale * A[j * sj + c * sc] (D x d) is staged once per
 // CTA in shared memory as sA[j][c] with row stride d + 1 (conflict-free both ways).
+// One warp per group (16 groups per CTA).
 // mode 0: m holds the centroids (the seeds).
 // mode 1: m_g = (sum of the rows assigned to g) / (their count): the partial sums the
 //         previous assignment pass left per segment of the head, added in segment order
-//         in fp64, then the label corrections of the exact re-check applied in ascending
+//         in fp64 (the group's warp, four columns per lane, the loads of eight segments in
+//         flight), then the label corrections of the exact re-check applied in ascending
 //         row order (a row moves from its provisional group to its final one); an empty
 //         group keeps its centroid.  m is updated in place.
 // mode 2: as mode 1 but an empty group gets 0, the means are written to m and no weights
 //         are formed (the K/V group centroids after the last pass).
-// Weights, two centroids per warp: nu = A m (fp32, sequential over c), bias = ||nu||^2,
-//   w = A^T nu (sequential over j) -> w_hi = bf16(w), w_lo = bf16(w - w_hi); wnorm = ||w||.
+// Weights: nu = A m (fp32, sequential over c), bias = ||nu||^2, w = A^T nu (sequential over
+//   j) -> w_hi = bf16(w), w_lo = bf16(w - w_hi); wnorm = ||w||.
 // Rows g in [G, GP) are padding: w = 0, bias = +inf.
-// grid = (ceil(GP / WG_PER_CTA), BH), block = 256.
+// grid = (ceil(GP / WG_PER_CTA), BH), block = 512.
 // ---------------------------------------------------------------------------
 constexpr int WG_PER_CTA = 16;
-constexpr int CW_THREADS = 256;
+constexpr int CW_THREADS = 512;
 constexpr int kCorrCap = 2048;   // corrections of one CTA's groups per pass
 
 // floats of the region that holds A for the weights and, before that, the segment-slot rows
-// of the CTA's groups and its sorted corrections
+// and counts of the CTA's groups and its sorted corrections
 __host__ __device__ inline int cw_scratch_floats(int d, int D, int SPH) {
   const int a = D * (d + 1), b = 2 * SPH * WG_PER_CTA + 2 * kCorrCap;
   return ((a > b ? a : b) + 3) & ~3;
@@ -107,10 +109,11 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
   float* sNu = sMg + WG_PER_CTA * d;                         // [WG_PER_CTA][128] their nu
   const int bh = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g0 = blockIdx.x * WG_PER_CTA, g1 = min(GP, g0 + WG_PER_CTA);
+  static_assert(WG_PER_CTA == CW_THREADS / 32, "one group per warp");
   if (mode != 0) {
-    // ---- means from the partial sums of the previous pass: per element, the head's
-    // segment slots in segment order (the mean's definition, summed in fp64); the slot of a
-    // segment holds only the groups that occur in it
+    // ---- means from the partial sums of the previous pass: the head's segment slots in
+    // segment order (the mean's definition, summed in fp64); the slot of a segment holds
+    // only the groups that occur in it
     const size_t sbytes = (size_t)GP * 8 + (size_t)GP * d * 4;
     const unsigned char* hs = pp.slots + (size_t)bh * pp.SPH * sbytes;
     int* spos = reinterpret_cast<int*>(sA);                   // [SPH][WG_PER_CTA] slot rows
@@ -126,49 +129,44 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
     }
     if (tid == 0) { s_nsel = 0; s_over = 0; }
     __syncthreads();
-    // element e = (group gi, column c), E elements per thread (d is 64 or 128: shifts); the
-    // loads of SB segments go out together before they are added in segment order
-    constexpr int E = WG_PER_CTA * 128 / CW_THREADS, SB = 4;
-    const int dl = d == 64 ? 6 : 7;
-    int gis[E], cs[E];
-    double a[E];
+    {
+      // warp = group; lane = four columns (d = 64: lanes 0-15)
+      const int gi = warp, c4 = lane * 4;
+      const bool act = c4 < d;
+      double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+      constexpr int SB = 8;
+      for (int sgm0 = 0; sgm0 < pp.SPH; sgm0 += SB) {
+        float4 v[SB];
+        int pos[SB];
 #pragma unroll
-    for (int u = 0; u < E; ++u) {
-      const int e = tid + u * CW_THREADS;
-      gis[u] = e < WG_PER_CTA * d ? e >> dl : -1;
-      cs[u] = e & (d - 1);
-      a[u] = 0.0;
-    }
-    for (int sgm0 = 0; sgm0 < pp.SPH; sgm0 += SB) {
-      float v[SB][E];
-      unsigned occ = 0u;
-#pragma unroll
-      for (int q = 0; q < SB; ++q) {
-        const int sgm = sgm0 + q;
-        const float* rows = reinterpret_cast<const float*>(hs + (size_t)sgm * sbytes + (size_t)GP * 8);
-#pragma unroll
-        for (int u = 0; u < E; ++u) {
-          const int pos = (sgm < pp.SPH && gis[u] >= 0) ? spos[sgm * WG_PER_CTA + gis[u]] : -1;
-          v[q][u] = 0.f;
-          if (pos >= 0) {
-            v[q][u] = rows[(size_t)pos * d + cs[u]];
-            occ |= 1u << (q * E + u);
-          }
+        for (int q = 0; q < SB; ++q) {
+          const int sgm = sgm0 + q;
+          pos[q] = sgm < pp.SPH ? spos[sgm * WG_PER_CTA + gi] : -1;
+          v[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (pos[q] >= 0 && act)
+            v[q] = *reinterpret_cast<const float4*>(hs + (size_t)sgm * sbytes + (size_t)GP * 8 +
+                                                    ((size_t)pos[q] * d + c4) * 4);
         }
+#pragma unroll
+        for (int q = 0; q < SB; ++q)
+          if (pos[q] >= 0) {
+            a0 += (double)v[q].x;
+            a1 += (double)v[q].y;
+            a2 += (double)v[q].z;
+            a3 += (double)v[q].w;
+          }
       }
-#pragma unroll
-      for (int q = 0; q < SB; ++q)
-#pragma unroll
-        for (int u = 0; u < E; ++u)
-          if (occ & (1u << (q * E + u))) a[u] += (double)v[q][u];
-    }
-#pragma unroll
-    for (int u = 0; u < E; ++u)
-      if (gis[u] >= 0) acc[tid + u * CW_THREADS] = a[u];
-    if (tid < WG_PER_CTA) {
-      int n = 0;
-      for (int sgm = 0; sgm < pp.SPH; ++sgm) n += scnt[sgm * WG_PER_CTA + tid];
-      cnt[tid] = n;
+      if (act) {
+        acc[gi * d + c4] = a0;
+        acc[gi * d + c4 + 1] = a1;
+        acc[gi * d + c4 + 2] = a2;
+        acc[gi * d + c4 + 3] = a3;
+      }
+      if (lane == 0) {
+        int n = 0;
+        for (int sgm = 0; sgm < pp.SPH; ++sgm) n += scnt[sgm * WG_PER_CTA + gi];
+        cnt[gi] = n;
+      }
     }
     // the re-check's corrections that move a row out of or into this CTA's groups
     const int nc = min(pp.corr_count[bh], pp.N);
@@ -186,35 +184,37 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
     __syncthreads();
     const int ns = min(s_nsel, kCorrCap);
     if (s_over) { if (tid == 0) set_error(err, DERR_CAPACITY); }
-    // ascending row order (bitonic sort of the selected list, padded with rows past N)
-    int p2 = 1;
-    while (p2 < ns) p2 <<= 1;
-    for (int i = ns + tid; i < p2; i += CW_THREADS) sel[i] = make_int2(0x7fffffff, 0xFFFF);
-    __syncthreads();
-    for (int kk = 2; kk <= p2; kk <<= 1) {
-      for (int j = kk >> 1; j > 0; j >>= 1) {
-        for (int i = tid; i < p2; i += CW_THREADS) {
-          const int l = i ^ j;
-          if (l > i) {
-            const int2 a = sel[i], b = sel[l];
-            const bool up = (i & kk) == 0;
-            if ((a.x > b.x) == up) { sel[i] = b; sel[l] = a; }
+    if (ns > 0) {
+      // ascending row order (bitonic sort of the selected list, padded with rows past N)
+      int p2 = 1;
+      while (p2 < ns) p2 <<= 1;
+      for (int i = ns + tid; i < p2; i += CW_THREADS) sel[i] = make_int2(0x7fffffff, 0xFFFF);
+      __syncthreads();
+      for (int kk = 2; kk <= p2; kk <<= 1) {
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+          for (int i = tid; i < p2; i += CW_THREADS) {
+            const int l = i ^ j;
+            if (l > i) {
+              const int2 x = sel[i], y = sel[l];
+              const bool up = (i & kk) == 0;
+              if ((x.x > y.x) == up) { sel[i] = y; sel[l] = x; }
+            }
           }
+          __syncthreads();
         }
-        __syncthreads();
       }
-    }
-    // apply them in that order: thread c owns column c of the CTA's groups
-    for (int c = tid; c < d; c += CW_THREADS) {
-      for (int k = 0; k < ns; ++k) {
-        const int2 e = sel[k];
-        const int fi = (e.y >> 8) & 0xFF, ti = e.y & 0xFF;
-        const double x = (double)bf2f(pp.X[((size_t)bh * pp.N + e.x) * d + c]);
-        if (fi != 0xFF) acc[fi * d + c] -= x;
-        if (ti != 0xFF) acc[ti * d + c] += x;
-        if (c == 0) {
-          if (fi != 0xFF) cnt[fi] -= 1;
-          if (ti != 0xFF) cnt[ti] += 1;
+      // apply them in that order: thread c owns column c of the CTA's groups
+      for (int c = tid; c < d; c += CW_THREADS) {
+        for (int k = 0; k < ns; ++k) {
+          const int2 e = sel[k];
+          const int fi = (e.y >> 8) & 0xFF, ti = e.y & 0xFF;
+          const double x = (double)bf2f(pp.X[((size_t)bh * pp.N + e.x) * d + c]);
+          if (fi != 0xFF) acc[fi * d + c] -= x;
+          if (ti != 0xFF) acc[ti * d + c] += x;
+          if (c == 0) {
+            if (fi != 0xFF) cnt[fi] -= 1;
+            if (ti != 0xFF) cnt[ti] += 1;
+          }
         }
       }
     }
@@ -252,107 +252,79 @@ __global__ void __launch_bounds__(CW_THREADS) k_centroid_weights(float* __restri
     sMg[e] = (g < g1 && g < G) ? m[((size_t)bh * G + g) * d + c] : 0.f;
   }
   __syncthreads();
-  // warp w forms the weights of groups g0 + w and g0 + w + 8 together; lanes split j for
-  // nu = A m and c for w = A^T nu, each sum in ascending order of its index
-  static_assert(WG_PER_CTA == 2 * (CW_THREADS / 32), "two groups per warp");
-  const int gl[2] = {warp, warp + 8};
-  bool live[2];
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int g = g0 + gl[u];
-    live[u] = g < g1 && g < G;
-    if (g < g1 && g >= G) {
-      // padding group: never the argmin
-      const size_t wrow = ((size_t)bh * GP + g) * d;
-      for (int c = lane; c < d; c += 32) {
-        w_hi[wrow + c] = __float2bfloat16(0.f);
-        w_lo[wrow + c] = __float2bfloat16(0.f);
-      }
-      if (lane == 0) {
-        bias[(size_t)bh * GP + g] = __int_as_float(0x7f800000);
-        wnorm[(size_t)bh * GP + g] = 0.f;
-      }
+  // warp w forms the weights of group g0 + w; lanes split j for nu = A m and c for
+  // w = A^T nu, each sum in ascending order of its index
+  const int g = g0 + warp;
+  const bool live = g < g1 && g < G;
+  if (g < g1 && g >= G) {
+    // padding group: never the argmin
+    const size_t wrow = ((size_t)bh * GP + g) * d;
+    for (int c = lane; c < d; c += 32) {
+      w_hi[wrow + c] = __float2bfloat16(0.f);
+      w_lo[wrow + c] = __float2bfloat16(0.f);
+    }
+    if (lane == 0) {
+      bias[(size_t)bh * GP + g] = __int_as_float(0x7f800000);
+      wnorm[(size_t)bh * GP + g] = 0.f;
     }
   }
-  if (!live[0] && !live[1]) return;
-  float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  if (!live) return;
+  float acc4[4] = {0.f, 0.f, 0.f, 0.f};
   {
-    const float* m0 = sMg + gl[0] * d;
-    const float* m1 = sMg + gl[1] * d;
+    const float* m0 = sMg + warp * d;
     for (int c = 0; c < d; ++c) {
-      const float x0 = m0[c], x1 = m1[c];
+      const float x0 = m0[c];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int j = lane + 32 * k;
-        if (j < D) {
-          const float a = sA[j * (d + 1) + c];
-          acc2[0][k] = fmaf(a, x0, acc2[0][k]);
-          acc2[1][k] = fmaf(a, x1, acc2[1][k]);
-        }
+        if (j < D) acc4[k] = fmaf(sA[j * (d + 1) + c], x0, acc4[k]);
       }
     }
   }
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int g = g0 + gl[u];
+  {
     float b2 = 0.f;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int j = lane + 32 * k;
       if (j < D) {
-        const float a = acc2[u][k] * a_scale;
-        sNu[gl[u] * 128 + j] = a;
+        const float a = acc4[k] * a_scale;
+        sNu[warp * 128 + j] = a;
         b2 = fmaf(a, a, b2);
       }
     }
     b2 = warp_sum(b2);
-    if (live[u]) {
-      for (int j = lane; j < DT; j += 32) nu[((size_t)bh * G + g) * DT + j] = j < D ? sNu[gl[u] * 128 + j] : 0.f;
-      if (lane == 0) bias[(size_t)bh * GP + g] = b2;
-    }
+    for (int j = lane; j < DT; j += 32) nu[((size_t)bh * G + g) * DT + j] = j < D ? sNu[warp * 128 + j] : 0.f;
+    if (lane == 0) bias[(size_t)bh * GP + g] = b2;
   }
   __syncwarp();
 #pragma unroll
-  for (int u = 0; u < 2; ++u)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) acc2[u][k] = 0.f;
+  for (int k = 0; k < 4; ++k) acc4[k] = 0.f;
   {
-    const float* n0 = sNu + gl[0] * 128;
-    const float* n1 = sNu + gl[1] * 128;
+    const float* n0 = sNu + warp * 128;
     for (int j = 0; j < D; ++j) {
-      const float y0 = n0[j], y1 = n1[j];
+      const float y0 = n0[j];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int c = lane + 32 * k;
-        if (c < d) {
-          const float a = sA[j * (d + 1) + c];
-          acc2[0][k] = fmaf(a, y0, acc2[0][k]);
-          acc2[1][k] = fmaf(a, y1, acc2[1][k]);
-        }
+        if (c < d) acc4[k] = fmaf(sA[j * (d + 1) + c], y0, acc4[k]);
       }
     }
   }
+  const size_t wrow = ((size_t)bh * GP + g) * d;
+  float n2 = 0.f;
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int g = g0 + gl[u];
-    const size_t wrow = ((size_t)bh * GP + g) * d;
-    float n2 = 0.f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int c = lane + 32 * k;
-      if (c < d) {
-        const float w = a_scale * acc2[u][k];
-        n2 = fmaf(w, w, n2);
-        if (live[u]) {
-          const __nv_bfloat16 hi = __float2bfloat16(w);
-          w_hi[wrow + c] = hi;
-          w_lo[wrow + c] = __float2bfloat16(w - __bfloat162float(hi));
-        }
-      }
+  for (int k = 0; k < 4; ++k) {
+    const int c = lane + 32 * k;
+    if (c < d) {
+      const float w = a_scale * acc4[k];
+      n2 = fmaf(w, w, n2);
+      const __nv_bfloat16 hi = __float2bfloat16(w);
+      w_hi[wrow + c] = hi;
+      w_lo[wrow + c] = __float2bfloat16(w - __bfloat162float(hi));
     }
-    n2 = warp_sum(n2);
-    if (live[u] && lane == 0) wnorm[(size_t)bh * GP + g] = sqrtf(n2);
   }
+  n2 = warp_sum(n2);
+  if (lane == 0) wnorm[(size_t)bh * GP + g] = sqrtf(n2);
 }
 
 // ---------------------------------------------------------------------------
