@@ -454,12 +454,120 @@ def run_cuda(args):
         line["diagnostics"] = partition_diagnostics(part, Ql, Kl, o_sparse, o_dense, p, frames)
     if rank == 0 and ws == 1 and not args.heads:
         line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0 and ws == 1 and not args.heads and args.others and args.workload == WORKLOAD:
+        line["other_workloads"] = {n: other_workload(n, dev, spr, pk) for n in ("world", "long")}
     if ws > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def other_workload(name, dev, spr, pk, steps=2, warmup=2):
+    """A compact measurement of another workload of the pages in the same run: ms per call
+    (partition -> attend beside probe_fit -> reconstruct, on one stream plus a side stream),
+    the attend stage alone with its useful-pair TFLOP/s, this build's dense (frame-causal:
+    causal dense) kernel on the same inputs, and both outputs' rel-L2 against it."""
+    import numpy as np
+    import torch
+    from synth import frame_index, generate, perturb, to_torch
+    w = bench_workload(argparse.Namespace(workload=name), heads=False)
+    pd = dict(B=w.B, H=w.H, N=w.N, d=w.d, block=w.block, density=w.density, n_kgroups=w.n_kgroups,
+              n_qgroups=w.n_qgroups, n_samples=w.n_samples, n_probes=w.n_probes, eig_rank=w.eig_rank,
+              sub_rank=w.sub_rank, kmeans_iters=w.kmeans_iters, ridge_lambda=w.ridge_lambda, seed=0)
+    frames = frame_index(w.grid) if w.frame_causal else None
+    fid = torch.from_numpy(frames).to(dev) if frames is not None else None
+    p = spr.Params.make(**pd, frame_id=fid, n_frames=w.grid[0] if frames is not None else 0)
+    t_gen = time.perf_counter()
+    qb, kb, vb = generate(w, seed=0)
+    calls = ROLLOUT_CALLS if w.frame_causal else 1
+    inputs = []
+    for c in range(calls):
+        if c > 0:
+            qb, kb, vb = (perturb(x, ROLLOUT_SIGMA, j, c) for j, x in enumerate((qb, kb, vb)))
+        inputs.append(tuple(to_torch(x, dev) for x in (qb, kb, vb)))
+    del qb, kb, vb
+    t_gen = time.perf_counter() - t_gen
+    Q, K, V = inputs[-1]
+    wsb = spr.workspace(p, dev)
+    part = spr.alloc_partition(p, dev)
+    pr = spr.alloc_probe(p, dev)
+    o_sparse, o = torch.empty_like(Q), torch.empty_like(Q)
+    lse = torch.empty(p.BH, p.N, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    side = torch.cuda.Stream(dev, priority=-1)
+    fork = [torch.cuda.Event() for _ in range(2)]
+
+    def call(Qc, Kc, Vc):
+        spr.sparsepr_partition(p, Qc, Kc, part["perm_q"], part["perm_k"], part["label_q"], part["label_k"],
+                               part["qoff"], part["koff"], part["route"], part["block_mask"], part["rho_exec"], wsb)
+        fork[0].record(stream)
+        side.wait_event(fork[0])
+        with torch.cuda.stream(side):
+            spr.sparsepr_probe_fit(p, Qc, Kc, Vc, part["label_k"], part["perm_q"], part["qoff"], part["route"],
+                                   pr["probe_idx"], pr["probe_o_dense"], pr["b_full"], pr["Vr"], pr["W"], None, wsb)
+            fork[1].record(side)
+        spr.sparsepr_attend(p, Qc, Kc, Vc, part["perm_q"], part["perm_k"], part["qoff"], part["koff"],
+                            part["route"], o_sparse, lse, wsb)
+        stream.wait_event(fork[1])
+        spr.sparsepr_reconstruct(p, o_sparse, pr["probe_idx"], pr["probe_o_dense"], pr["b_full"], pr["Vr"],
+                                 pr["W"], o)
+
+    for _ in range(warmup):
+        for x in inputs:
+            call(*x)
+    torch.cuda.synchronize()
+    assert spr.sparsepr_workspace_error(p, wsb) == 0
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    e[0].record(stream)
+    for _ in range(steps):
+        for x in inputs:
+            call(*x)
+    e[1].record(stream)
+    for _ in range(3):
+        spr.sparsepr_attend(p, Q, K, V, part["perm_q"], part["perm_k"], part["qoff"], part["koff"], part["route"],
+                            o_sparse, lse, wsb)
+    e[2].record(stream)
+    o_dense = torch.empty_like(Q)
+    spr.sparsepr_dense_attention(p, Q, K, V, o_dense, None, wsb)
+    e[3].record(stream)
+    for _ in range(2):
+        spr.sparsepr_dense_attention(p, Q, K, V, o_dense, None, wsb)
+    e[4].record(stream)
+    call(Q, K, V)   # the last call's outputs, for the errors below
+    # the other reading of the affine map's input on the same partition and sparse output
+    p_alt = spr.Params.make(**dict(pd, fit_input=1), frame_id=fid, n_frames=w.grid[0] if frames is not None else 0)
+    pr_alt = spr.alloc_probe(p_alt, dev)
+    spr.sparsepr_probe_fit(p_alt, Q, K, V, part["label_k"], part["perm_q"], part["qoff"], part["route"],
+                           pr_alt["probe_idx"], pr_alt["probe_o_dense"], pr_alt["b_full"], pr_alt["Vr"], pr_alt["W"],
+                           None, wsb)
+    o_alt = torch.empty_like(Q)
+    spr.sparsepr_reconstruct(p_alt, o_sparse, pr_alt["probe_idx"], pr_alt["probe_o_dense"], pr_alt["b_full"],
+                             pr_alt["Vr"], pr_alt["W"], o_alt)
+    torch.cuda.synchronize()
+    assert spr.sparsepr_workspace_error(p, wsb) == 0
+    ms = e[0].elapsed_time(e[1]) / (steps * calls)
+    attn_ms = e[1].elapsed_time(e[2]) / 3
+    dense_ms = e[3].elapsed_time(e[4]) / 2
+    useful, issued = attention_pairs(part, frames)
+    rel = lambda a, b: float((a.float() - b.float()).norm() / b.float().norm())
+    out = {"config": _config(w), "ms_per_call": round(ms, 4), "calls_timed": steps * calls,
+           "attend_ms_alone": round(attn_ms, 4),
+           "attend_tflops_useful": round(4.0 * w.d * useful / (attn_ms * 1e-3) / 1e12, 2),
+           "attend_frac_useful": round(4.0 * w.d * useful / (attn_ms * 1e-3) / 1e12 / pk["bf16"], 4),
+           "tile_fill": round(useful / max(1, issued), 4),
+           ("causal_dense_attention_ms" if frames is not None else "dense_attention_ms"): round(dense_ms, 4),
+           "speedup_vs_dense": round(dense_ms / ms, 3),
+           "rho_exec_mean": round(float(part["rho_exec"].float().mean()), 5),
+           "rel_l2_vs_dense": {"o_sparse": round(rel(o_sparse, o_dense), 5), "o_reconstructed": round(rel(o, o_dense), 5),
+                               "o_reconstructed, map input projected on the subspace": round(rel(o_alt, o_dense), 5)},
+           "input_generation_s": round(t_gen, 1)}
+    if w.name == "long":
+        out["note"] = "128 K/V and query groups (the kernels' limit), not the ceil(N/256) = 422 of the pages' scale"
+    del inputs, Q, K, V, wsb, part, pr, o_sparse, o, o_dense, lse, pr_alt, o_alt
+    torch.cuda.empty_cache()
+    return out
 
 
 def bench_workload(args, heads=True):
@@ -704,6 +812,8 @@ def main():
                     help="2: probe_fit beside the routed attention on a second stream (default); 1: in sequence")
     ap.add_argument("--no-seed1", dest="seed1", action="store_false",
                     help="skip the one-call measurement on the generator's second seed")
+    ap.add_argument("--no-others", dest="others", action="store_false",
+                    help="skip the compact measurements of the rollout and 108,000-token workloads")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (small cases for ncu captures; default: the workload's 40)")
     args = ap.parse_args()
