@@ -87,8 +87,10 @@ typedef struct {
   int block;               /* tile rows of the permuted layout reported in block_mask (64 or 128)  */
   float density;           /* target executed-pair density rho_exec in (0, 1], probe pairs included;
                               >= 1 routes every non-empty cell                                      */
-  int n_kgroups;           /* K/V groups G_k (1..min(N,1024))                                       */
-  int n_qgroups;           /* query groups G_q (1..min(N,1024))                                     */
+  int n_kgroups;           /* K/V groups G_k: 1..min(N,1024) is valid (else SPARSEPR_EINVAL); the
+                              kernels implement G_k <= 128, more returns SPARSEPR_EUNSUPPORTED     */
+  int n_qgroups;           /* query groups G_q: as G_k (valid up to min(N,1024), implemented up to
+                              128)                                                                 */
   int n_samples;           /* sampled queries M_s for M_K (1..min(N,1024); default max(64, d))      */
   int n_probes;            /* probe rows per head P (1..min(N,64); the article uses 64)             */
   int eig_rank;            /* eigenpairs of M_K kept for key coordinates r_e (16 or 32; default d/4) */
