@@ -332,6 +332,23 @@ def run_cuda(args):
     fit_errors = {readings[pd.get("fit_input", 0)] + " (this run's)": round(err_recon, 5),
                   readings[1 - pd.get("fit_input", 0)]: round(err_alt, 5)}
 
+    # --- the library's single device-buffer entry point (its probe path on a stream of its own)
+    fws0 = spr.workspace(p, dev, forward=True)
+    o_fwd = torch.empty_like(Q)
+    for _ in range(2):
+        spr.sparsepr_forward(p, Ql, Kl, Vl, o_fwd, None, fws0)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nf = max(3, min(args.steps, 10))
+    f0.record(stream)
+    for _ in range(nf):
+        spr.sparsepr_forward(p, Ql, Kl, Vl, o_fwd, None, fws0)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    forward_ms = f0.elapsed_time(f1) / nf
+    assert spr.sparsepr_workspace_error(p, fws0) == 0
+    del fws0, o_fwd
+
     # --- end to end through the C ABI from pinned host buffers
     Qh, Kh, Vh = (torch.empty(Q.shape, dtype=torch.bfloat16, pin_memory=True) for _ in range(3))
     Qh.copy_(Q.cpu()); Kh.copy_(K.cpu()); Vh.copy_(V.cpu())
@@ -412,6 +429,9 @@ def run_cuda(args):
         "stage_ms": {"partition": round(stage_ms[0], 4), "attend": round(stage_ms[1], 4),
                      ("probe_fit" if side is None else "probe_fit_wait"): round(stage_ms[2], 4),
                      "reconstruct": round(stage_ms[3], 4)},
+        "forward_ms": {"value": round(forward_ms, 4),
+                       "how": "sparsepr_forward on device buffers: the whole call in one C-ABI call, its probe "
+                              "path on a second stream of the call's own"},
         "dense_attention_ms": round(dense_ms, 4),
         "speedup_vs_dense": round(dense_ms / ms_per_call, 3),
         "rho_exec": {"mean": round(float(rho.mean()), 5), "min": round(float(rho.min()), 5),

@@ -529,6 +529,55 @@ sparsepr_status sparsepr_reconstruct(const sparsepr_params* p, const void* O_spa
                          (cudaStream_t)stream);
 }
 
+// A second stream forked from `st` for the duration of one call: side() is a fresh
+// non-blocking stream of the highest priority that starts after the work already on `st`
+// (or `st` itself if a stream or event cannot be created); join() makes `st` wait for it.
+// The stream and events are released when the object goes out of scope (the driver frees
+// them once their work completes).
+class ForkJoin {
+ public:
+  explicit ForkJoin(cudaStream_t st) : st_(st) {
+    int lo = 0, hi = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) hi = 0;
+    if (cudaStreamCreateWithPriority(&side_, cudaStreamNonBlocking, hi) != cudaSuccess) { side_ = nullptr; return; }
+    if (cudaEventCreateWithFlags(&fork_, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&done_, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventRecord(fork_, st_) != cudaSuccess || cudaStreamWaitEvent(side_, fork_, 0) != cudaSuccess) {
+      release();
+      cudaGetLastError();
+    }
+  }
+  // on an early return the caller's stream still waits for whatever the side stream took
+  ~ForkJoin() {
+    if (side_ && !joined_ && cudaEventRecord(done_, side_) == cudaSuccess) cudaStreamWaitEvent(st_, done_, 0);
+    release();
+  }
+  cudaStream_t side() const { return side_ ? side_ : st_; }
+  void mark_side_done() {
+    if (side_ && cudaEventRecord(done_, side_) != cudaSuccess) failed_ = true;
+  }
+  sparsepr_status join() {
+    if (!side_) return SPARSEPR_OK;
+    if (failed_) return fail(SPARSEPR_ECUDA, "cudaEventRecord on the probe stream failed");
+    const cudaError_t e = cudaStreamWaitEvent(st_, done_, 0);
+    joined_ = e == cudaSuccess;
+    return joined_ ? SPARSEPR_OK : fail_cuda(e, "cudaStreamWaitEvent(stream, probe path done)");
+  }
+
+ private:
+  void release() {
+    if (fork_) cudaEventDestroy(fork_);
+    if (done_) cudaEventDestroy(done_);
+    if (side_) cudaStreamDestroy(side_);
+    fork_ = done_ = nullptr;
+    side_ = nullptr;
+  }
+  cudaStream_t st_;
+  cudaStream_t side_ = nullptr;
+  cudaEvent_t fork_ = nullptr, done_ = nullptr;
+  bool failed_ = false, joined_ = false;
+};
+
 // The whole call on device buffers; clear_err: reset the workspace error word first.
 static sparsepr_status forward_impl(const sparsepr_params* p, const void* Q, const void* K, const void* V, void* O,
                              float* rho_exec, void* workspace, size_t ws_bytes, void* stream, bool clear_err) {
@@ -548,14 +597,20 @@ static sparsepr_status forward_impl(const sparsepr_params* p, const void* Q, con
   float* rho = rho_exec ? rho_exec : at<float>(ws, L.f_rho);
   SPR_CHECK(run_partition(*p, L, Q, K, perm_q, perm_k, label_q, label_k, qoff, koff, route, nullptr, rho, nullptr,
                           ws, st, clear_err));
-  SPR_CHECK(run_attend(*p, L, Q, K, V, perm_q, perm_k, qoff, koff, route, O, at<float>(ws, L.f_lse), ws, st));
   int* pidx = at<int>(ws, L.f_probe_idx);
   float* pod = at<float>(ws, L.f_probe_od);
   float* bfull = at<float>(ws, L.f_bfull);
   float* vr = at<float>(ws, L.f_vr);
   float* w = at<float>(ws, L.f_w);
+  // attend and probe_fit read only the partition and write disjoint workspace regions: the
+  // probe path runs on a higher-priority stream of this call beside the routed attention and
+  // joins before the correction (one stream for both if the second cannot be created)
+  ForkJoin fj(st);
   SPR_CHECK(run_probe_fit(*p, L, Q, K, V, label_k, perm_q, qoff, route, pidx, pod, bfull, vr, w, nullptr, nullptr,
-                          ws, st));
+                          ws, fj.side()));
+  fj.mark_side_done();
+  SPR_CHECK(run_attend(*p, L, Q, K, V, perm_q, perm_k, qoff, koff, route, O, at<float>(ws, L.f_lse), ws, st));
+  SPR_CHECK(fj.join());
   SPR_CHECK(run_reconstruct(*p, L.BH, O, pidx, pod, bfull, vr, w, O, st));
   return SPARSEPR_OK;
 }

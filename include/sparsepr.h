@@ -31,8 +31,9 @@
  *    disjoint regions of it, so attend and probe_fit may run concurrently on two
  *    streams sharing one workspace.  sparsepr_probe_fit_noalloc instead uses a fixed
  *    16 MiB device array that the library holds on every GPU that loads it (see its
- *    declaration).  sparsepr_forward_host_chunked creates and releases CUDA events
- *    inside the call (no device memory).
+ *    declaration).  sparsepr_forward (and the host entry points built on it) creates
+ *    and releases a second stream and CUDA events inside the call, and
+ *    sparsepr_forward_host_chunked its CUDA events (no device memory).
  *  - Asynchrony: every call only enqueues work on `stream` (a cudaStream_t; NULL
  *    is the legacy default stream) and returns.  Argument errors are detected on
  *    the host before anything is enqueued and return SPARSEPR_EINVAL or
@@ -246,7 +247,12 @@ SPARSEPR_API sparsepr_status sparsepr_reconstruct(const sparsepr_params* p, cons
 
 /* The whole call (partition -> attend -> probe_fit -> reconstruct) on device buffers,
  * with every intermediate kept in the workspace (sparsepr_forward_workspace_bytes).
- * rho_exec (float [BH]) may be NULL.                                                   */
+ * rho_exec (float [BH]) may be NULL.  The probe path (sparsepr_probe_fit's kernels) runs
+ * on a second stream that the call creates, forks from `stream` after the partition and
+ * joins back before the correction, so it overlaps the routed attention; the stream and
+ * its events are released before the call returns (freed once their work completes).
+ * If they cannot be created, everything runs on `stream`.  The results do not depend on
+ * the overlap.                                                                         */
 SPARSEPR_API size_t sparsepr_forward_workspace_bytes(const sparsepr_params* p);
 SPARSEPR_API sparsepr_status sparsepr_forward(const sparsepr_params* p, const void* Q, const void* K,
                                  const void* V, void* O, float* rho_exec,
