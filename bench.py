@@ -377,7 +377,7 @@ def run_cuda(args):
     # compute of chunk i (one C-ABI call per step; same outputs as the unsplit call)
     del fws
     oh_single = Oh.clone()
-    n_chunks = next(c for c in (4, 2, 1) if BH >= c)
+    n_chunks = next(c for c in (5, 4, 2, 1) if BH >= c)
     cws = spr.workspace(spr.chunk_params(p, n_chunks), dev, forward=True)
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     for _ in range(2):
