@@ -531,12 +531,18 @@ sparsepr_status sparsepr_reconstruct(const sparsepr_params* p, const void* O_spa
 
 // A second stream forked from `st` for the duration of one call: side() is a fresh
 // non-blocking stream of the highest priority that starts after the work already on `st`
-// (or `st` itself if a stream or event cannot be created); join() makes `st` wait for it.
-// The stream and events are released when the object goes out of scope (the driver frees
-// them once their work completes).
+// (or `st` itself if a stream or event cannot be created, or if `st` is being captured
+// into a CUDA graph, where a stream created and destroyed inside the capture has no
+// place); join() makes `st` wait for it.  The stream and events are released when the
+// object goes out of scope (the driver frees them once their work completes).
 class ForkJoin {
  public:
   explicit ForkJoin(cudaStream_t st) : st_(st) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st_, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+      cudaGetLastError();
+      return;
+    }
     int lo = 0, hi = 0;
     if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) hi = 0;
     if (cudaStreamCreateWithPriority(&side_, cudaStreamNonBlocking, hi) != cudaSuccess) { side_ = nullptr; return; }

@@ -251,8 +251,8 @@ SPARSEPR_API sparsepr_status sparsepr_reconstruct(const sparsepr_params* p, cons
  * on a second stream that the call creates, forks from `stream` after the partition and
  * joins back before the correction, so it overlaps the routed attention; the stream and
  * its events are released before the call returns (freed once their work completes).
- * If they cannot be created, everything runs on `stream`.  The results do not depend on
- * the overlap.                                                                         */
+ * If they cannot be created, or `stream` is being captured into a CUDA graph, everything
+ * runs on `stream`.  The results do not depend on the overlap.                         */
 SPARSEPR_API size_t sparsepr_forward_workspace_bytes(const sparsepr_params* p);
 SPARSEPR_API sparsepr_status sparsepr_forward(const sparsepr_params* p, const void* Q, const void* K,
                                  const void* V, void* O, float* rho_exec,

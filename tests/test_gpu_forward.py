@@ -225,3 +225,35 @@ def test_fit_readings_end_to_end_tiny(gpu, fit_input):
     for h in range(w.H):
         ref = O.sparsepr_head(to_f64(qb[0, h]), to_f64(kb[0, h]), to_f64(vb[0, h]), op, h)
         assert rel_l2(_np(o[0, h]).astype(np.float64), ref.o) <= O_REL_L2
+
+
+def test_forward_captured_in_cuda_graph(gpu):
+    """The single call captured into a CUDA graph (its probe path then stays on the
+    captured stream) replays to the same bytes as the direct call."""
+    import torch
+    spr = _spr()
+    w = _ragged_workload()
+    pd = params_dict(w)
+    p = spr.Params.make(**pd)
+    qb, kb, vb = generate(w, seed=9)
+    Q, K, V = (to_torch(x, gpu) for x in (qb, kb, vb))
+    o_ref, rho_ref = _forward(p, Q, K, V, gpu)
+    ws = spr.workspace(p, gpu, forward=True)
+    o = torch.empty_like(Q)
+    rho = torch.empty(p.BH, dtype=torch.float32, device=gpu)
+    side = torch.cuda.Stream(gpu)
+    side.wait_stream(torch.cuda.current_stream(gpu))
+    with torch.cuda.stream(side):   # warm-up outside the capture
+        spr.sparsepr_forward(p, Q, K, V, o, rho, ws)
+    torch.cuda.current_stream(gpu).wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        spr.sparsepr_forward(p, Q, K, V, o, rho, ws)
+    o.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert spr.sparsepr_workspace_error(p, ws) == 0
+    assert torch.equal(o, o_ref)
+    assert torch.equal(rho, rho_ref)
+    del g
