@@ -481,7 +481,7 @@ def run_cuda(args):
                 line["other_workloads"][n] = other_workload(n, dev, spr, pk)
             except Exception as e:   # reported in the line; the main measurement above stands
                 line["other_workloads"][n] = {"error": f"{type(e).__name__}: {e}"[:300]}
-                torch.cuda.synchronize()
+                break
     if ws > 1:
         import torch.distributed as dist
         dist.barrier()
