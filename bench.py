@@ -666,8 +666,9 @@ def attention_pairs(part, frames=None):
 
     useful: routed pairs (frame-causal: routed pairs whose key frame <= query frame).
     issued: per 256-row unit of a query group, its 128-row q-tiles times the 128-key
-    chunks of the key stream it walks: all routed keys of the group, or (frame-causal)
-    the routed keys of frames <= the unit's last row frame."""
+    chunks of the key stream each walks: all routed keys of the group, or (frame-causal)
+    the routed keys of frames <= the frame of the tile's last row for the unit's first
+    tile and of the unit's last row for its second."""
     import numpy as np
     qoff = part["qoff"].long().cpu().numpy()
     koff = part["koff"].long().cpu().numpy()
@@ -696,8 +697,11 @@ def attention_pairs(part, frames=None):
         for a in range(Gq):
             for u0 in range(qoff[bh, a], qoff[bh, a + 1], 256):
                 rows = min(256, qoff[bh, a + 1] - u0)
-                f_last = fr[perm_q[bh, u0 + rows - 1]]
-                issued += ((rows + 127) // 128) * 128 * ((int(tl[a, f_last]) + 127) // 128) * 128
+                p_last = int(tl[a, fr[perm_q[bh, u0 + rows - 1]]])
+                chunks = (p_last + 127) // 128
+                if rows > 128:
+                    chunks += (min(int(tl[a, fr[perm_q[bh, u0 + 127]]]), p_last) + 127) // 128
+                issued += chunks * 128 * 128
     return useful, issued
 
 
